@@ -1,0 +1,257 @@
+"""Plain CPU oracle for the FALQON melded FP8 linear step (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It never touches the CUDA library and
+the CUDA library never touches it.
+
+The arithmetic lives in ``falqon_oracle.cpp`` (its header lists every reading
+of the method); this module only marshals numpy arrays through ctypes.  All
+bfloat16 tensors are passed as their uint16 bit patterns.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+
+from .build import build as _build
+
+STATUS_NONFINITE = 1
+STATUS_SCALE_OVERFLOW = 2
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build()
+        L = C.CDLL(path)
+        p = C.c_void_p
+        i64 = C.c_int64
+        L.fo_e4m3_decode.restype = C.c_double
+        L.fo_e4m3_decode.argtypes = [C.c_uint8]
+        L.fo_e4m3_encode.restype = C.c_uint8
+        L.fo_e4m3_encode.argtypes = [C.c_float]
+        L.fo_e4m3_encode_array.argtypes = [p, i64, p]
+        L.fo_bf16_round.restype = C.c_uint16
+        L.fo_bf16_round.argtypes = [C.c_double]
+        L.fo_bf16_round_array.argtypes = [p, i64, p]
+        L.fo_amax.restype = C.c_uint32
+        L.fo_amax.argtypes = [p, C.c_int, i64, p]
+        L.fo_scale.restype = C.c_uint32
+        L.fo_scale.argtypes = [C.c_float, p]
+        L.fo_quantize.argtypes = [p, C.c_int, i64, C.c_float, p]
+        L.fo_residual.argtypes = [p, C.c_int, p, i64, C.c_float, p, p]
+        L.fo_linear_fwd.argtypes = [p, C.c_float, p, C.c_float, i64, i64, i64, i64, i64, p]
+        L.fo_linear_dx.argtypes = [p, C.c_float, p, C.c_float, i64, i64, i64, i64, i64, p]
+        L.fo_adapter_t.argtypes = [p, C.c_float, p, i64, i64, i64, p, p]
+        L.fo_adapter_u.argtypes = [p, C.c_float, p, i64, i64, i64, p, p]
+        L.fo_adapter_db.argtypes = [p, C.c_float, p, p, i64, i64, i64, p]
+        L.fo_adapter_da.argtypes = [p, p, p, C.c_float, i64, i64, i64, p]
+        L.fo_proxy_accumulate.argtypes = [p, p, p, i64, i64, i64]
+        L.fo_proxy_select.argtypes = [p, C.c_float, p, i64, i64, p, p]
+        L.fo_set_threads.argtypes = [C.c_int]
+        L.fo_get_threads.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def set_threads(n: int) -> None:
+    lib().fo_set_threads(int(n))
+
+
+def get_threads() -> int:
+    return int(lib().fo_get_threads())
+
+
+# ------------------------------------------------------------------ codecs
+def e4m3_decode(c: int) -> float:
+    return float(lib().fo_e4m3_decode(int(c)))
+
+
+def e4m3_decode_table() -> np.ndarray:
+    return np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float32)
+    shape = v.shape
+    flat = np.ascontiguousarray(v.reshape(-1))
+    out = np.empty(flat.shape, dtype=np.uint8)
+    lib().fo_e4m3_encode_array(_ptr(flat), flat.size, _ptr(out))
+    return out.reshape(shape)
+
+
+def bf16_round(v) -> np.ndarray:
+    """float64 -> bfloat16 bits, one rounding (nearest, ties to even)."""
+    v = np.asarray(v, dtype=np.float64)
+    shape = v.shape
+    flat = np.ascontiguousarray(v.reshape(-1))
+    out = np.empty(flat.shape, dtype=np.uint16)
+    lib().fo_bf16_round_array(_ptr(flat), flat.size, _ptr(out))
+    return out.reshape(shape)
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+# ------------------------------------------------------------------ C-2, C-3, C-4
+def _xin(x: np.ndarray):
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), 1
+    if x.dtype == np.float32:
+        return np.ascontiguousarray(x), 0
+    raise TypeError("x must be bfloat16 bits (uint16) or float32")
+
+
+def amax(x: np.ndarray):
+    x, is_bf16 = _xin(x)
+    out = np.zeros(1, dtype=np.float32)
+    st = lib().fo_amax(_ptr(x), is_bf16, x.size, _ptr(out))
+    return np.float32(out[0]), int(st)
+
+
+def scale(amax_value) -> tuple:
+    out = np.zeros(1, dtype=np.float32)
+    st = lib().fo_scale(C.c_float(float(amax_value)), _ptr(out))
+    return np.float32(out[0]), int(st)
+
+
+def quantize(x: np.ndarray):
+    """Per-tensor E4M3 quantization: returns (codes, scale, amax, status)."""
+    x, is_bf16 = _xin(x)
+    a, st1 = amax(x)
+    s, st2 = scale(a)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    lib().fo_quantize(_ptr(x), is_bf16, x.size, C.c_float(float(s)), _ptr(codes))
+    return codes, np.float32(s), np.float32(a), st1 | st2
+
+
+def residual(x: np.ndarray, codes: np.ndarray, s) -> tuple:
+    """Eq. 8 quantization error W - DQ(W~): (float64, float32) arrays."""
+    x, is_bf16 = _xin(x)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    r64 = np.empty(x.shape, dtype=np.float64)
+    r32 = np.empty(x.shape, dtype=np.float32)
+    lib().fo_residual(_ptr(x), is_bf16, _ptr(codes), x.size, C.c_float(float(s)),
+                      _ptr(r64), _ptr(r32))
+    return r64, r32
+
+
+# ------------------------------------------------------------------ C-5, C-6
+def linear_fwd(xq, s_x, wq, s_w, rows=None) -> np.ndarray:
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    m0, m1 = (0, M) if rows is None else rows
+    y = np.empty((m1 - m0, N), dtype=np.float64)
+    lib().fo_linear_fwd(_ptr(xq), C.c_float(float(s_x)), _ptr(wq), C.c_float(float(s_w)),
+                        M, N, K, m0, m1, _ptr(y))
+    return y
+
+
+def linear_dx(dyq, s_dy, wq, s_w, rows=None) -> np.ndarray:
+    dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    M, N = dyq.shape
+    K = wq.shape[1]
+    m0, m1 = (0, M) if rows is None else rows
+    dx = np.empty((m1 - m0, K), dtype=np.float64)
+    lib().fo_linear_dx(_ptr(dyq), C.c_float(float(s_dy)), _ptr(wq), C.c_float(float(s_w)),
+                       M, N, K, m0, m1, _ptr(dx))
+    return dx
+
+
+# ------------------------------------------------------------------ C-7, C-8
+def adapter_t(xq, s_x, A):
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    M, K = xq.shape
+    r = A.shape[0]
+    t64 = np.empty((M, r), dtype=np.float64)
+    t16 = np.empty((M, r), dtype=np.uint16)
+    lib().fo_adapter_t(_ptr(xq), C.c_float(float(s_x)), _ptr(A), M, K, r, _ptr(t64), _ptr(t16))
+    return t64, t16
+
+
+def adapter_u(dyq, s_dy, B):
+    dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
+    B = np.ascontiguousarray(B, dtype=np.uint16)
+    M, N = dyq.shape
+    r = B.shape[1]
+    u64 = np.empty((M, r), dtype=np.float64)
+    u16 = np.empty((M, r), dtype=np.uint16)
+    lib().fo_adapter_u(_ptr(dyq), C.c_float(float(s_dy)), _ptr(B), M, N, r, _ptr(u64), _ptr(u16))
+    return u64, u16
+
+
+def adapter_db(dyq, s_dy, t16=None, t64=None):
+    dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
+    M, N = dyq.shape
+    t = t16 if t16 is not None else t64
+    r = t.shape[1]
+    t16c = None if t16 is None else np.ascontiguousarray(t16, dtype=np.uint16)
+    t64c = None if t64 is None or t16 is not None else np.ascontiguousarray(t64, dtype=np.float64)
+    db = np.empty((N, r), dtype=np.float64)
+    lib().fo_adapter_db(_ptr(dyq), C.c_float(float(s_dy)), _ptr(t16c), _ptr(t64c), M, N, r, _ptr(db))
+    return db
+
+
+def adapter_da(xq, s_x, u16=None, u64=None):
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    M, K = xq.shape
+    u = u16 if u16 is not None else u64
+    r = u.shape[1]
+    u16c = None if u16 is None else np.ascontiguousarray(u16, dtype=np.uint16)
+    u64c = None if u64 is None or u16 is not None else np.ascontiguousarray(u64, dtype=np.float64)
+    da = np.empty((r, K), dtype=np.float64)
+    lib().fo_adapter_da(_ptr(u16c), _ptr(u64c), _ptr(xq), C.c_float(float(s_x)), M, K, r, _ptr(da))
+    return da
+
+
+# ------------------------------------------------------------------ C-9, C-10, C-11
+def proxy_accumulate(P: np.ndarray, dB_inc: np.ndarray, A: np.ndarray) -> np.ndarray:
+    """Returns P + (dB_inc . A) with the float32 FMA chain; P is not modified."""
+    P = np.array(P, dtype=np.float32, copy=True, order="C")
+    dB_inc = np.ascontiguousarray(dB_inc, dtype=np.uint16)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    N, K = P.shape
+    r = A.shape[0]
+    lib().fo_proxy_accumulate(_ptr(P), _ptr(dB_inc), _ptr(A), N, K, r)
+    return P
+
+
+def proxy_select(wq: np.ndarray, s_w, P: np.ndarray):
+    """Returns (new wq, new P, mask, n_selected); the inputs are not modified."""
+    wq = np.array(wq, dtype=np.uint8, copy=True, order="C")
+    P = np.array(P, dtype=np.float32, copy=True, order="C")
+    N, K = wq.shape
+    mask = np.zeros(N, dtype=np.uint8)
+    cnt = np.zeros(1, dtype=np.int32)
+    lib().fo_proxy_select(_ptr(wq), C.c_float(float(s_w)), _ptr(P), N, K, _ptr(mask), _ptr(cnt))
+    return wq, P, mask, int(cnt[0])
+
+
+def proxy_update(wq, s_w, P, dB_inc, A, accumulate=True, select=True):
+    """One row-wise proxy update: accumulate, then select/requantize/clear."""
+    Pn = proxy_accumulate(P, dB_inc, A) if accumulate else np.array(P, dtype=np.float32, copy=True)
+    if not select:
+        return np.array(wq, dtype=np.uint8, copy=True), Pn, None, 0
+    return proxy_select(wq, s_w, Pn)
+
+
+from .tolerance import within_tolerance, tolerance_report  # noqa: E402,F401
+from .step import layer_step  # noqa: E402,F401
+

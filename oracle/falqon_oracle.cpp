@@ -1,0 +1,365 @@
+// FALQON melded FP8 linear step: plain CPU oracle.
+//
+// TEST INFRASTRUCTURE.  Only the tests, the package's smoke check and the
+// bench's CPU-baseline leg load this code.  It shares no source, header,
+// table or helper with the CUDA library; the two are written independently
+// from the same reading of the method, and the tests compare them.
+//
+// Source: "FALQON: Accelerating LoRA Fine-tuning with Low-Bit Floating-Point
+// Arithmetic" (Choi, Lee, Park, Kwon, Lee; NeurIPS 2025), as it appears on
+// the abstract/introduction page and in the OpenReview rebuttals.  Sections
+// cited below: [abstract], [intro] (contribution list), [R2-W2] (rebuttal to
+// reviewer 2, rewrite of the scaling sentence), [R2-W7] (high-level method
+// description), [R2-W8] (DQ definition), [R2-W1] (Figure 2 operations),
+// [R2-Q3] (Eq. 8 and Eq. 9), [R2-Q4] (additive quantization error), [R3-Q1]
+// (top-k row selection), [R4-Q1] (gradient of A, freezing A).
+//
+// Every decision the pages leave open is written here.
+//
+//  C-1  E4M3 codec.  [R2-W2] names E4M3 and says the scaled tensor is
+//       "rounded to FP8"; the bit layout is the OCP 8-bit floating point
+//       E4M3 definition: sign, 4 exponent bits (bias 7), 3 mantissa bits,
+//       no infinities, S.1111.111 is NaN, largest finite 448, smallest
+//       subnormal 2^-9.  Encoding rounds to the nearest finite value with
+//       ties to the even code; magnitudes above 448 (including infinity)
+//       saturate to 448 ("satfinite"); NaN encodes as 0x7F; the sign of a
+//       value that rounds to zero is kept.
+//  C-2  Per-tensor scale.  [R2-W2]: a high-precision tensor X is scaled by a
+//       per-tensor factor s_X before rounding; the formula itself is missing
+//       from the pages.  Reading: amax = max |x| over the whole tensor
+//       (current scaling, recomputed each call), s = 448 / amax as one IEEE
+//       float32 division; amax = 0 gives s = 1; a non-finite amax sets the
+//       NONFINITE status bit and gives s = 1; a quotient that overflows to
+//       infinity is clamped to FLT_MAX and sets SCALE_OVERFLOW.
+//  C-3  Quantize.  code = enc( fl32( fl32(x) * s ) ): one float32 multiply
+//       rounded to nearest even, then the C-1 encoding (two roundings, by
+//       definition).
+//  C-4  Initial quantization error.  [R2-Q3]: DQ(W~) + Delta_Q W = W (Eq. 8),
+//       DQ(W~) = W - Delta_Q W (Eq. 9); [R2-Q4]: the error is an additive
+//       tensor; [intro]: the initial error is the implicit LoRA
+//       initialisation.  The residual is R = W - dec(code)/s in float64.
+//       The proxy starts at zero (the pages give no proxy initialisation).
+//  C-5  Forward on the backbone alone ([intro], [R2-W7]: no separate LoRA
+//       path): Y[m,n] = sum_k dec(Xq[m,k]) dec(Wq[n,k]) / (s_X s_W), float64.
+//  C-6  dX on the same quantized backbone:
+//       dX[m,k] = sum_n dec(dYq[m,n]) dec(Wq[n,k]) / (s_dY s_W).
+//  C-7  Gradient of B ([R4-Q1]: it "can be pre-calculated" from A x):
+//       T[m,i] = bf16( sum_k dec(Xq[m,k]) A[i,k] / s_X ),
+//       dB[n,i] = sum_m dec(dYq[m,n]) T[m,i] / s_dY.
+//       Reading: the adapter GEMMs reuse the already-quantized X and dY (no
+//       extra quantize op), A and B are bfloat16, and the intermediates T
+//       and U are materialised in bfloat16.
+//  C-8  Gradient of A ([R4-Q1]: dL/dA = B^T dL/dO x^T; FALQON freezes A, the
+//       output is optional):
+//       U[m,i] = bf16( sum_n dec(dYq[m,n]) B[n,i] / s_dY ),
+//       dA[i,k] = sum_m U[m,i] dec(Xq[m,k]) / s_X.
+//  C-9  Proxy accumulation ([abstract] "row-wise proxy update"; the digest
+//       page's summary: a row-wise proxy matrix accumulates the updates).
+//       D[n,k] is a float32 fused-multiply-add chain over i = 0..r-1 in
+//       index order starting from +0: acc = fma(dB_inc[n,i], A[i,k], acc);
+//       then P[n,k] = fl32(P[n,k] + D[n,k]).  dB_inc is the increment of B
+//       for this step (the caller folds in sign and learning rate).
+//  C-10 Row selection ([intro]: the proxy "selectively applies substantial
+//       weight updates", avoiding updates that vanish under low-bit
+//       quantization).  t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ) (no
+//       fused multiply-add), c' = enc(t); row n is selected iff some k has
+//       dec(c') != dec(Wq[n,k]) as values (so +0 equals -0, and a NaN code
+//       equals nothing).  s_W is the fixed scale of the initial
+//       quantization.  The pages' own rule is a top-k over rows ([R3-Q1],
+//       [R2-W7]) with k not given; the threshold rule here is the contract.
+//  C-11 Requantize and clear.  Selected rows: Wq[n,:] = c'[n,:] for all k
+//       (verbatim, sign of zero included), P[n,:] = +0.  Rows not selected:
+//       Wq untouched (bit-identical), P keeps the accumulated value.
+//
+// Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
+// -ffp-contract=off keeps every float32 multiply and add separately rounded;
+// the only fused multiply-adds are the explicit std::fmaf calls of C-9.
+
+#include <cfloat>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+constexpr uint32_t kNonfinite = 1u;      // C-2: non-finite amax
+constexpr uint32_t kScaleOverflow = 2u;  // C-2: 448/amax overflowed
+
+double dec(uint8_t c) {  // C-1 decoding, straight from the field definition
+  const int sign = c >> 7;
+  const int e = (c >> 3) & 0xF;
+  const int m = c & 0x7;
+  if (e == 15 && m == 7) return std::nan("");
+  const double mag = (e == 0) ? std::ldexp(static_cast<double>(m), -9)
+                              : std::ldexp(8.0 + m, e - 10);  // 2^(e-7) * (1 + m/8)
+  return sign ? -mag : mag;
+}
+
+uint8_t enc(float v) {  // C-1 encoding
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));
+  if (a > 448.0) return sign | 0x7E;  // satfinite
+  if (a < std::ldexp(1.0, -6)) {
+    // Subnormal range: multiples of 2^-9.  nearbyint rounds half to even in
+    // the default rounding mode; 8 * 2^-9 is the smallest normal, code 0x08.
+    const double q = std::nearbyint(std::ldexp(a, 9));
+    return sign | static_cast<uint8_t>(q);
+  }
+  int e2 = 0;
+  std::frexp(a, &e2);
+  int E = e2 - 1;                                   // a in [2^E, 2^(E+1))
+  double q = std::nearbyint(std::ldexp(a, 3 - E));  // significand * 8, in [8, 16]
+  if (q == 16.0) { q = 8.0; E += 1; }
+  return sign | static_cast<uint8_t>(((E + 7) << 3) | (static_cast<int>(q) - 8));
+}
+
+float bf16_to_f32(uint16_t b) {
+  const uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+uint16_t f32_bits_hi(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return static_cast<uint16_t>(u >> 16);
+}
+
+// Rounds a float64 value to bfloat16 once (nearest, ties to even).
+uint16_t bf16_round(double v) {
+  if (std::isnan(v)) return 0x7FC0;
+  const uint16_t sign = std::signbit(v) ? 0x8000 : 0x0000;
+  const double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  if (std::isinf(a)) return sign | 0x7F80;
+  int e2 = 0;
+  std::frexp(a, &e2);
+  const int E = e2 - 1;
+  const int qexp = (E < -126) ? -133 : E - 7;  // spacing of bf16 values near a
+  const double q = std::nearbyint(std::ldexp(a, -qexp));
+  const double val = std::ldexp(q, qexp);  // exactly representable in bf16
+  if (val >= std::ldexp(1.0, 128)) return sign | 0x7F80;
+  return sign | f32_bits_hi(static_cast<float>(val));
+}
+
+int g_threads = 1;
+
+}  // namespace
+
+extern "C" {
+
+// ---------------------------------------------------------------- set-up
+void fo_set_threads(int n) { g_threads = n < 1 ? 1 : n; }
+int fo_get_threads(void) { return g_threads; }
+
+// ---------------------------------------------------------------- C-1
+double fo_e4m3_decode(uint8_t c) { return dec(c); }
+uint8_t fo_e4m3_encode(float v) { return enc(v); }
+void fo_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = enc(v[i]);
+}
+uint16_t fo_bf16_round(double v) { return bf16_round(v); }
+void fo_bf16_round_array(const double* v, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = bf16_round(v[i]);
+}
+
+// ---------------------------------------------------------------- C-2
+// amax over a bfloat16 (is_bf16 = 1, x holds uint16 bits) or float32 tensor.
+uint32_t fo_amax(const void* x, int is_bf16, int64_t n, float* amax) {
+  float m = 0.0f;
+  bool nonfinite = false;
+  for (int64_t i = 0; i < n; ++i) {
+    const float v = is_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(x)[i])
+                            : static_cast<const float*>(x)[i];
+    if (!std::isfinite(v)) {
+      nonfinite = true;
+      continue;
+    }
+    const float a = std::fabs(v);
+    if (a > m) m = a;
+  }
+  *amax = nonfinite ? std::nanf("") : m;
+  return nonfinite ? kNonfinite : 0u;
+}
+
+uint32_t fo_scale(float amax, float* s) {
+  if (!std::isfinite(amax)) { *s = 1.0f; return kNonfinite; }
+  if (amax == 0.0f) { *s = 1.0f; return 0u; }
+  const float q = 448.0f / amax;  // IEEE float32 division
+  if (std::isinf(q)) { *s = FLT_MAX; return kScaleOverflow; }
+  *s = q;
+  return 0u;
+}
+
+// ---------------------------------------------------------------- C-3
+void fo_quantize(const void* x, int is_bf16, int64_t n, float s, uint8_t* codes) {
+  for (int64_t i = 0; i < n; ++i) {
+    const float v = is_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(x)[i])
+                            : static_cast<const float*>(x)[i];
+    const float p = v * s;  // one float32 multiply, round to nearest even
+    codes[i] = enc(p);
+  }
+}
+
+// ---------------------------------------------------------------- C-4
+// r64 = W - dec(code)/s in float64; r32 = that value rounded to float32.
+void fo_residual(const void* x, int is_bf16, const uint8_t* codes, int64_t n, float s,
+                 double* r64, float* r32) {
+  for (int64_t i = 0; i < n; ++i) {
+    const double w = is_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(x)[i])
+                             : static_cast<const float*>(x)[i];
+    const double r = w - dec(codes[i]) / static_cast<double>(s);
+    if (r64) r64[i] = r;
+    if (r32) r32[i] = static_cast<float>(r);
+  }
+}
+
+// ---------------------------------------------------------------- C-5
+// Rows [m0, m1) of Y = Xq Wq^T / (s_X s_W); y holds (m1-m0) x N values.
+void fo_linear_fwd(const uint8_t* xq, float s_x, const uint8_t* wq, float s_w,
+                   int64_t M, int64_t N, int64_t K, int64_t m0, int64_t m1, double* y) {
+  (void)M;
+  const double denom = static_cast<double>(s_x) * static_cast<double>(s_w);
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t m = m0; m < m1; ++m) {
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += dec(xq[m * K + k]) * dec(wq[n * K + k]);
+      y[(m - m0) * N + n] = acc / denom;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- C-6
+// Rows [m0, m1) of dX = dYq Wq / (s_dY s_W); dx holds (m1-m0) x K values.
+void fo_linear_dx(const uint8_t* dyq, float s_dy, const uint8_t* wq, float s_w,
+                  int64_t M, int64_t N, int64_t K, int64_t m0, int64_t m1, double* dx) {
+  (void)M;
+  const double denom = static_cast<double>(s_dy) * static_cast<double>(s_w);
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t m = m0; m < m1; ++m) {
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int64_t n = 0; n < N; ++n) acc += dec(dyq[m * N + n]) * dec(wq[n * K + k]);
+      dx[(m - m0) * K + k] = acc / denom;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- C-7 / C-8
+// Generic skinny product used for T and U:
+//   out[m,i] = sum_j dec(q[m,j]) * bf16(w[i,j] or w[j,i]) / s
+// w_rows_are_i = 1: w is [r, J] (A for T);  0: w is [J, r] (B for U).
+// Writes float64 values and their bfloat16 rounding.
+static void skinny_rows(const uint8_t* q, float s, const uint16_t* w, int w_rows_are_i,
+                        int64_t M, int64_t J, int64_t r, double* out64, uint16_t* out16) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t i = 0; i < r; ++i) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < J; ++j) {
+        const double wv = bf16_to_f32(w_rows_are_i ? w[i * J + j] : w[j * r + i]);
+        acc += dec(q[m * J + j]) * wv;
+      }
+      const double v = acc / static_cast<double>(s);
+      if (out64) out64[m * r + i] = v;
+      if (out16) out16[m * r + i] = bf16_round(v);
+    }
+  }
+}
+
+// T = bf16(Xq A^T / s_X), A is [r, K].
+void fo_adapter_t(const uint8_t* xq, float s_x, const uint16_t* A, int64_t M, int64_t K,
+                  int64_t r, double* t64, uint16_t* t16) {
+  skinny_rows(xq, s_x, A, 1, M, K, r, t64, t16);
+}
+
+// U = bf16(dYq B / s_dY), B is [N, r].
+void fo_adapter_u(const uint8_t* dyq, float s_dy, const uint16_t* B, int64_t M, int64_t N,
+                  int64_t r, double* u64, uint16_t* u16) {
+  skinny_rows(dyq, s_dy, B, 0, M, N, r, u64, u16);
+}
+
+// dB = dYq^T T / s_dY, [N, r].  t is either bfloat16 bits (t16) or float64 (t64);
+// the float64 form exists for the autograd pin that checks the formula itself.
+void fo_adapter_db(const uint8_t* dyq, float s_dy, const uint16_t* t16, const double* t64,
+                   int64_t M, int64_t N, int64_t r, double* db) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t i = 0; i < r; ++i) {
+      double acc = 0.0;
+      for (int64_t m = 0; m < M; ++m) {
+        const double tv = t16 ? static_cast<double>(bf16_to_f32(t16[m * r + i])) : t64[m * r + i];
+        acc += dec(dyq[m * N + n]) * tv;
+      }
+      db[n * r + i] = acc / static_cast<double>(s_dy);
+    }
+  }
+}
+
+// dA = U^T Xq / s_X, [r, K].
+void fo_adapter_da(const uint16_t* u16, const double* u64, const uint8_t* xq, float s_x,
+                   int64_t M, int64_t K, int64_t r, double* da) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t i = 0; i < r; ++i) {
+    for (int64_t k = 0; k < K; ++k) {
+      double acc = 0.0;
+      for (int64_t m = 0; m < M; ++m) {
+        const double uv = u16 ? static_cast<double>(bf16_to_f32(u16[m * r + i])) : u64[m * r + i];
+        acc += uv * dec(xq[m * K + k]);
+      }
+      da[i * K + k] = acc / static_cast<double>(s_x);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- C-9
+// P += D with D the float32 FMA chain of dB_inc[n,:] . A[:,k].
+void fo_proxy_accumulate(float* P, const uint16_t* dB_inc, const uint16_t* A, int64_t N,
+                         int64_t K, int64_t r) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      float acc = 0.0f;
+      for (int64_t i = 0; i < r; ++i)
+        acc = std::fmaf(bf16_to_f32(dB_inc[n * r + i]), bf16_to_f32(A[i * K + k]), acc);
+      P[n * K + k] = P[n * K + k] + acc;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- C-10 / C-11
+void fo_proxy_select(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, uint8_t* mask,
+                     int32_t* n_selected) {
+  int32_t count = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    bool selected = false;
+    for (int64_t k = 0; k < K; ++k) {
+      const float w = static_cast<float>(dec(wq[n * K + k]));  // exact
+      const float upd = s_w * P[n * K + k];
+      const float t = w + upd;
+      const uint8_t c_new = enc(t);
+      if (!(dec(c_new) == dec(wq[n * K + k]))) selected = true;
+    }
+    if (selected) {
+      for (int64_t k = 0; k < K; ++k) {
+        const float w = static_cast<float>(dec(wq[n * K + k]));
+        const float upd = s_w * P[n * K + k];
+        const float t = w + upd;
+        wq[n * K + k] = enc(t);
+        P[n * K + k] = 0.0f;
+      }
+    }
+    if (mask) mask[n] = selected ? 1 : 0;
+    count += selected ? 1 : 0;
+  }
+  if (n_selected) *n_selected = count;
+}
+
+}  // extern "C"

@@ -1,0 +1,232 @@
+"""Pins for the oracle's E4M3 codec, scale and quantize (C-1 .. C-4).
+
+Each check ties the oracle to something other than itself: worked values of
+the E4M3 definition, a brute-force nearest-value search, torch's own e4m3
+cast (a library routine) inside the range where it does not saturate, and
+the closed forms of Eq. 8-9 of the FALQON rebuttal (reviewer 2, Q3).
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synthetic import gen
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "e4m3_worked_values.txt")
+
+
+def _golden():
+    dec, enc = [], []
+    for line in open(GOLDEN):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        kind, a, b = line.split()
+        if kind == "decode":
+            dec.append((int(a, 16), float(b)))
+        else:
+            enc.append((float(a), int(b, 16)))
+    return dec, enc
+
+
+def _finite_table():
+    """All finite E4M3 magnitudes from the definition, indexed by code 0..126."""
+    vals = []
+    for c in range(127):
+        e, m = c >> 3, c & 7
+        vals.append(m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def _brute_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest finite E4M3 value by exhaustive search, ties to the even code."""
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    tab = _finite_table()
+    out = np.zeros(v.shape, dtype=np.uint8)
+    nan = np.isnan(v)
+    a = np.abs(np.where(nan, 0.0, v))
+    a = np.minimum(a, 448.0)  # satfinite
+    d = np.abs(a[:, None] - tab[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    # ties: among equal distances prefer the even code
+    even = (np.arange(127) % 2 == 0)[None, :]
+    pick = np.where(cand & even, 1, 0)
+    has_even = pick.any(axis=1)
+    idx = np.where(has_even, np.argmax(pick, axis=1), np.argmax(cand, axis=1))
+    sign = np.signbit(v) & ~nan
+    out = idx.astype(np.uint8) | np.where(sign, 0x80, 0).astype(np.uint8)
+    out[nan] = 0x7F
+    return out
+
+
+def test_golden_decode():
+    dec, _ = _golden()
+    for code, val in dec:
+        got = O.e4m3_decode(code)
+        if math.isnan(val):
+            assert math.isnan(got), hex(code)
+        else:
+            assert got == val and math.copysign(1, got) == math.copysign(1, val), hex(code)
+
+
+def test_golden_encode():
+    _, enc = _golden()
+    for val, code in enc:
+        assert int(O.e4m3_encode(np.float32(val))) == code, (val, hex(code))
+
+
+def test_roundtrip_all_codes():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        v = O.e4m3_decode(c)
+        assert int(O.e4m3_encode(np.float32(v))) == c, hex(c)
+
+
+def test_decode_matches_table_and_is_monotone():
+    tab = _finite_table()
+    got = np.array([O.e4m3_decode(c) for c in range(127)])
+    assert np.array_equal(got, tab)
+    assert np.all(np.diff(tab) > 0)
+    assert tab[-1] == 448.0 and tab[1] == 2.0 ** -9
+
+
+def test_encode_brute_force_all_bf16_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    v = gen.bf16_bits_to_f32(bits)
+    assert np.array_equal(O.e4m3_encode(v), _brute_encode(v))
+
+
+def test_encode_midpoints_and_neighbours():
+    tab = _finite_table()
+    mids = (tab[:-1] + tab[1:]) / 2  # exact in float32 (at most 5 significant bits)
+    pts = np.concatenate([mids, -mids]).astype(np.float32)
+    near = np.concatenate([np.nextafter(pts, np.float32(np.inf)), np.nextafter(pts, np.float32(-np.inf))])
+    allv = np.concatenate([pts, near, tab.astype(np.float32), np.float32([464, 480, 1e38, 3e-45])])
+    assert np.array_equal(O.e4m3_encode(allv), _brute_encode(allv))
+
+
+def test_encode_random_fp32_vs_brute_force():
+    rng = np.random.default_rng(1)
+    v = (rng.standard_normal(20000) * np.exp2(rng.integers(-14, 10, 20000))).astype(np.float32)
+    assert np.array_equal(O.e4m3_encode(v), _brute_encode(v))
+
+
+def test_encode_matches_torch_cast_in_range():
+    # torch's float8_e4m3fn cast rounds to nearest-even and does not saturate;
+    # inside |v| <= 464 both definitions agree.
+    rng = np.random.default_rng(2)
+    v = (rng.uniform(-464, 464, 50000) * np.exp2(rng.integers(-18, 1, 50000))).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(v), ref)
+
+
+def test_scale_special_cases():
+    s, st = O.scale(np.float32(0.0))
+    assert s == 1.0 and st == 0
+    s, st = O.scale(np.float32(np.inf))
+    assert s == 1.0 and st == O.STATUS_NONFINITE
+    s, st = O.scale(np.float32(np.nan))
+    assert s == 1.0 and st == O.STATUS_NONFINITE
+    s, st = O.scale(np.float32(1e-39))  # 448 / 1e-39 overflows float32
+    assert s == np.finfo(np.float32).max and st == O.STATUS_SCALE_OVERFLOW
+    s, st = O.scale(np.float32(3.5))
+    assert s == np.float32(128.0) and st == 0
+    s, st = O.scale(np.float32(3.0))
+    assert s == np.float32(np.float32(448.0) / np.float32(3.0)) and st == 0
+
+
+def test_quantize_all_zero_tensor():
+    x = np.zeros((7, 16), dtype=np.uint16)
+    codes, s, a, st = O.quantize(x)
+    assert a == 0 and s == 1.0 and st == 0 and np.all(codes == 0)
+
+
+def test_quantize_single_nonzero_is_full_scale():
+    for val in (3.0, -0.001, 1e-20, 65504.0):
+        x = np.zeros((5, 16), dtype=np.float32)
+        x[3, 7] = val
+        codes, s, a, st = O.quantize(x)
+        assert a == abs(np.float32(val))
+        assert codes[3, 7] == (0x7E if val > 0 else 0xFE)
+        assert np.count_nonzero(codes) == 1
+
+
+def test_quantize_amax_element_maps_to_448_and_nonfinite_flag():
+    x = gen.normal_bf16_bits(123, (64, 48), 1.0)
+    codes, s, a, st = O.quantize(x)
+    f = gen.bf16_bits_to_f32(x)
+    i = np.argmax(np.abs(f))
+    assert codes.ravel()[i] & 0x7F == 0x7E
+    x2 = x.copy()
+    x2[5, 5] = 0x7FC0  # a bfloat16 NaN
+    _, _, a2, st2 = O.quantize(x2)
+    assert st2 & O.STATUS_NONFINITE and not np.isfinite(a2)
+
+
+def test_quantize_equals_torch_cast_of_scaled_tensor():
+    x = gen.normal_bf16_bits(7, (96, 80), 1.0)
+    codes, s, a, _ = O.quantize(x)
+    xf = gen.bf16_bits_to_f32(x)
+    assert a == np.max(np.abs(xf))
+    assert s == np.float32(448.0) / a
+    prod = (torch.from_numpy(xf) * torch.tensor(s, dtype=torch.float32))
+    ref = prod.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_eq8_residual_closed_form_and_half_step_bound():
+    w = gen.normal_f32(99, (40, 64), 0.02)
+    codes, s, _, _ = O.quantize(w)
+    r64, r32 = O.residual(w, codes, s)
+    deq = np.array([O.e4m3_decode(c) for c in range(256)])[codes] / np.float64(s)
+    # Eq. 8: DQ(W~) + Delta_Q W = W, exactly in float64
+    assert np.array_equal(deq + r64, w.astype(np.float64))
+    # Eq. 9: DQ(W~) = W - Delta_Q W
+    assert np.array_equal(deq, w.astype(np.float64) - r64)
+    assert np.array_equal(r32, r64.astype(np.float32))
+    # the code is within half an E4M3 step of the float32 product s * w
+    p = (w * s).astype(np.float64)
+    dq = deq * np.float64(s)
+    m = np.minimum(np.abs(p), np.abs(dq))
+    step = np.where(m < 2.0 ** -6, 2.0 ** -9, np.exp2(np.floor(np.log2(np.maximum(m, 2.0 ** -6))) - 3))
+    assert np.all(np.abs(p - dq) <= step / 2)
+
+
+@pytest.mark.parametrize("v,ref", [
+    (0.0, 0x0000), (-0.0, 0x8000), (1.0, 0x3F80), (-3.5, 0xC060),
+    (1.0 + 2.0 ** -8, 0x3F80),        # tie between 1 and 1 + 2^-7: even mantissa wins
+    (-(1.0 + 3 * 2.0 ** -8), 0xBF82),  # tie between 1 + 2^-7 and 1 + 2^-6: even wins
+    (1.0 + 2.0 ** -8 + 2.0 ** -40, 0x3F81),  # just above the tie: rounds up (one rounding)
+    (2.0 ** -133, 0x0001), (2.0 ** -134, 0x0000), (3 * 2.0 ** -134, 0x0002),
+    (1.5 * 2.0 ** 127, 0x7F40), (2.0 ** 128, 0x7F80), (float("inf"), 0x7F80),
+])
+def test_bf16_round_worked_values(v, ref):
+    # bfloat16: 8 significant bits, exponent bias 127, subnormal step 2^-133
+    assert int(O.bf16_round(np.float64(v))) == ref
+
+
+def _bf16_nearest_brute(x):
+    f = x.astype(np.float32)
+    b = (f.view(np.uint32) >> np.uint32(16)).astype(np.int64)
+    best = np.zeros(x.shape, dtype=np.uint16)
+    for i, xv in enumerate(x):
+        cands = [int(b[i]) + d for d in (-1, 0, 1, 2)]
+        vals = [float(gen.bf16_bits_to_f32(np.uint16([c]))[0]) for c in cands]
+        dist = [abs(v - xv) for v in vals]
+        m = min(dist)
+        pick = [c for c, d in zip(cands, dist) if d == m]
+        pick = [c for c in pick if c % 2 == 0] or pick
+        best[i] = pick[0]
+    return best
+
+
+def test_bf16_round_random_vs_brute_force():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(3000) * np.exp2(rng.integers(-20, 20, 3000))
+    assert np.array_equal(O.bf16_round(x), _bf16_nearest_brute(x))
