@@ -1,0 +1,497 @@
+"""Throughput of one melded-FP8 linear training step (FALQON hot path) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl falqon|reference]
+
+A step is the whole hot path for one synthetic token batch of the workload:
+  quantize X -> forward GEMM -> quantize dY -> adapter grads dB, dA -> dX GEMM
+  -> caller's plain SGD on B (two tiny torch ops) -> row-wise proxy update.
+All five library phases run in libfalqon's kernels through the C ABI.
+
+Timing: W untimed warm-up steps, then K timed steps.  The step is captured
+once per input slot in a CUDA graph and replayed; each timed step is bracketed
+by CUDA events on the launching stream and separated from the next by an L2
+flush (a 512 MB write, outside the events).  The timed region is bracketed by
+a barrier and torch.cuda.synchronize() on both sides; with N > 1 every rank
+runs an independent replica on its own batch ("replicas only", weak scaling)
+and the reported time is the max over ranks.
+
+Per-phase CUDA events give each kernel group's duration; the roofline object
+reports the slowest phase against the measured peaks in MEASURED_PEAKS.json.
+`e2e` repeats the step with the inputs in pinned host memory (H2D copies of X
+and dY and D2H copies of Y and dX inside the timed region).  `cpu_baseline`
+times the CPU oracle on a bounded sample (rank 0, N = 1).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from synthetic import WORKLOADS, layer_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama7b_attn_proj_4096x4096x4096_r64"
+METRIC = "melded FP8 linear fwd+bwd+proxy tokens/s; % of FP8 tensor peak / HBM"
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"falqon_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class Step:
+    """Device buffers and the captured step for one workload layer."""
+
+    def __init__(self, wl, layer, torch, F, dev, n_slots=2, seed_offset=0):
+        self.torch, self.F, self.dev = torch, F, dev
+        self.M, self.N, self.K, self.r = wl.M, layer.N, layer.K, wl.r
+        self.lr = wl.lr
+        t = torch
+        d0 = layer_inputs(wl, layer, step=seed_offset, with_b=True)
+
+        def bf16(bits):
+            return t.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(t.bfloat16).to(dev)
+
+        # persistent state of the layer
+        self.W = t.from_numpy(d0["W"]).to(dev)
+        self.wq = t.empty((self.N, self.K), dtype=t.uint8, device=dev)
+        self.s_w = t.empty(1, dtype=t.float32, device=dev)
+        self.A = bf16(d0["A"])
+        self.B = bf16(d0["B"])
+        self.P = t.zeros((self.N, self.K), dtype=t.float32, device=dev)
+        self.status = t.zeros(1, dtype=t.int32, device=dev)
+        # fresh X / dY per step: a few distinct slots, cycled
+        self.X = [bf16(layer_inputs(wl, layer, step=seed_offset + s)["X"]) for s in range(n_slots)]
+        self.dY = [bf16(layer_inputs(wl, layer, step=seed_offset + s)["dY"]) for s in range(n_slots)]
+        # outputs and intermediates
+        self.xq = t.empty((self.M, self.K), dtype=t.uint8, device=dev)
+        self.dyq = t.empty((self.M, self.N), dtype=t.uint8, device=dev)
+        self.s_x = t.empty(1, dtype=t.float32, device=dev)
+        self.s_dy = t.empty(1, dtype=t.float32, device=dev)
+        self.amax = t.empty(1, dtype=t.float32, device=dev)
+        self.y = t.empty((self.M, self.N), dtype=t.bfloat16, device=dev)
+        self.dx = t.empty((self.M, self.K), dtype=t.bfloat16, device=dev)
+        self.dA = t.empty((self.r, self.K), dtype=t.bfloat16, device=dev)
+        self.dB = t.empty((self.N, self.r), dtype=t.bfloat16, device=dev)
+        self.dB_inc = t.empty((self.N, self.r), dtype=t.bfloat16, device=dev)
+        self.mask = t.empty(self.N, dtype=t.uint8, device=dev)
+        self.n_sel = t.zeros(1, dtype=t.int32, device=dev)
+
+        def ws(op, M, N, K, r):
+            n = F.falqon_workspace_size(op, M, N, K, r)
+            return t.empty(max(n, 256), dtype=t.uint8, device=dev)
+
+        self.ws_q = ws(F.OP_QUANTIZE, self.M, max(self.N, self.K), 0, 0)
+        self.ws_q2 = ws(F.OP_QUANTIZE, self.N, self.K, 0, 0)
+        self.ws_bwd = ws(F.OP_LINEAR_BWD, self.M, self.N, self.K, self.r)
+        self.ws_p = ws(F.OP_PROXY_UPDATE, 0, self.N, self.K, self.r)
+        # initial quantization of the backbone (not part of the step)
+        F.falqon_quantize(self.W, codes=self.wq, scale=self.s_w, amax=self.amax,
+                          dev_status=self.status, workspace=self.ws_q2)
+        self.launches_per_step = 2 + 1 + 2 + 8 + 1 + 2  # library kernels per step
+
+    def phases(self, slot, ev=None):
+        """Enqueues one step; `ev` (list of 6 events) brackets the five phases."""
+        F, t = self.F, self.torch
+        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
+        rec(0)
+        F.falqon_quantize(self.X[slot], codes=self.xq, scale=self.s_x, amax=self.amax,
+                          dev_status=self.status, workspace=self.ws_q)
+        F.falqon_linear_fwd(self.xq, self.s_x, self.wq, self.s_w, y=self.y, dev_status=self.status)
+        rec(1)
+        F.falqon_quantize(self.dY[slot], codes=self.dyq, scale=self.s_dy, amax=self.amax,
+                          dev_status=self.status, workspace=self.ws_q)
+        F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, self.xq, self.s_x, self.A,
+                            self.B, dx=None, dA=self.dA, dB=self.dB, dev_status=self.status,
+                            workspace=self.ws_bwd)
+        rec(2)
+        F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, None, None, None, None,
+                            dx=self.dx, dA=None, dB=None, dev_status=self.status)
+        rec(3)
+        # the caller's optimizer: plain SGD on B; the proxy receives the increment
+        t.mul(self.dB, -self.lr, out=self.dB_inc)
+        self.B.add_(self.dB_inc)
+        rec(4)
+        F.falqon_proxy_update(self.wq, self.s_w, self.P, self.dB_inc, self.A,
+                              row_mask=self.mask, n_selected=self.n_sel, dev_status=self.status,
+                              workspace=self.ws_p)
+        rec(5)
+
+
+def _phase_work(st):
+    """Algorithmic flops / bytes of each phase (measurement section)."""
+    M, N, K, r = st.M, st.N, st.K, st.r
+    return {
+        # quantize X (read bf16, read again from L2 or HBM, write codes) + forward GEMM
+        "quantX+fwd": {"flops": 2.0 * M * N * K, "bytes": 3.0 * M * K + M * K + N * K + 2.0 * M * N},
+        # quantize dY + adapter GEMMs (T, dB, U, dA): codes re-read by each product
+        "quantdY+adapters": {"flops": 8.0 * M * r * (N + K) / 2.0,
+                             "bytes": 3.0 * M * N + 2.0 * (M * K + M * N) + 2.0 * r * (N + K)},
+        "dX": {"flops": 2.0 * M * N * K, "bytes": M * N + N * K + 2.0 * M * K},
+        "sgd": {"flops": 0.0, "bytes": 8.0 * N * r},
+        "proxy": {"flops": 2.0 * N * K * r, "bytes": 9.0 * N * K + 2.0 * r * (N + K)},
+    }
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_quantized_lora_b200 as F
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    F.lib()
+    wl = WORKLOADS[args.workload]
+    layer = wl.layers[0]
+    st = Step(wl, layer, torch, F, dev, n_slots=2, seed_offset=rank * 1000)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    # capture the step once per input slot
+    graphs = []
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for slot in range(2):  # warm the library (attributes, tensor-map encoder) first
+            st.phases(slot)
+    torch.cuda.synchronize()
+    if not args.no_graph:
+        for slot in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                st.phases(slot)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def step(i):
+        if graphs:
+            graphs[i % 2].replay()
+        else:
+            st.phases(i % 2)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            flush.fill_(i & 0xFF)
+            step(i)
+    torch.cuda.synchronize()
+    if int(st.status.item()) != 0:
+        raise RuntimeError(f"device status {int(st.status.item())} after warm-up")
+
+    # timed region: per-step events, L2 flush between steps (outside the events)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record()
+            step(i)
+            ends[i].record()
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    if ws > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(np.sum(step_ms))
+    if ws > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    # per-phase timing (eager, same stream, same flush discipline)
+    names = ["quantX+fwd", "quantdY+adapters", "dX", "sgd", "proxy"]
+    acc = {n: 0.0 for n in names}
+    reps = max(5, min(50, args.steps))
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            st.phases(i % 2, ev)
+            torch.cuda.synchronize()
+            for j, n in enumerate(names):
+                acc[n] += ev[j].elapsed_time(ev[j + 1])
+    phase_ms = {n: acc[n] / reps for n in names}
+
+    # e2e through the C ABI with host buffers (pinned), copies inside the timed region
+    hostX = [x.cpu().pin_memory() for x in st.X]
+    hostdY = [x.cpu().pin_memory() for x in st.dY]
+    hostY = torch.empty(st.y.shape, dtype=torch.bfloat16).pin_memory()
+    hostdX = torch.empty(st.dx.shape, dtype=torch.bfloat16).pin_memory()
+    hostSel = torch.empty(1, dtype=torch.int32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e_start.record()
+        for i in range(e2e_steps):
+            st.X[i % 2].copy_(hostX[i % 2], non_blocking=True)
+            st.dY[i % 2].copy_(hostdY[i % 2], non_blocking=True)
+            st.phases(i % 2)
+            hostY.copy_(st.y, non_blocking=True)
+            hostdX.copy_(st.dx, non_blocking=True)
+            hostSel.copy_(st.n_sel, non_blocking=True)
+        e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if ws > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    status = int(st.status.item())
+    n_sel = int(st.n_sel.item())
+
+    tokens_total = wl.M * args.steps * ws
+    value = tokens_total / (total_ms / 1e3)
+    e2e_value = wl.M * e2e_steps * ws / (e2e_ms / 1e3)
+    h2d = 2 * (st.X[0].numel() * 2 + st.dY[0].numel() * 2) // 2
+    d2h = st.y.numel() * 2 + st.dx.numel() * 2 + 4
+
+    peaks = _peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    work = _phase_work(st)
+    phases = {}
+    for n in names:
+        ms = phase_ms[n]
+        w = work[n]
+        tflops = w["flops"] / (ms * 1e-3) / 1e12 if ms > 0 else 0.0
+        gbs = w["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
+        phases[n] = {"ms": round(ms, 5), "tflops": round(tflops, 2), "gbs": round(gbs, 1),
+                     "frac_fp8_peak": round(tflops / fp8_peak, 4),
+                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    # dominant kernel: the forward GEMM phase vs dX: both tensor-bound FP8 GEMMs;
+    # report the dX GEMM (a single kernel per phase) when it is the slowest tensor phase
+    dom = max(names, key=lambda n: phase_ms[n])
+    if dom in ("dX", "quantX+fwd"):
+        roof = {"kernel": "tc_gemm_kernel (FP8 dX GEMM)" if dom == "dX" else "quantize X + FP8 forward GEMM",
+                "bound": "tensor", "achieved": phases[dom]["tflops"], "peak": round(fp8_peak, 1),
+                "unit": "TFLOP/s", "frac": phases[dom]["frac_fp8_peak"],
+                "peak_source": f"{peaks['source']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)"}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": phases[dom]["gbs"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": phases[dom]["frac_hbm"],
+                "peak_source": f"{peaks['source']} copy bandwidth"}
+    roof["traffic"] = None
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "N": layer.N, "K": layer.K, "r": wl.r,
+                   "global_batch_tokens": wl.M * ws, "parallelism": f"replicas{ws}",
+                   "l2": "flushed between timed steps (512 MB write outside the events)",
+                   "cuda_graph": not args.no_graph, "lr": wl.lr},
+        "roofline": roof,
+        "phases": phases,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+        "gpu_launches": st.launches_per_step * args.steps,
+        "clocks": clock_info,
+        "device_status": status,
+        "rows_selected_last_step": n_sel,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, layer, budget_s=args.cpu_budget)
+    if ws > 1:
+        dist.destroy_process_group()
+    return out, rank
+
+
+# ------------------------------------------------------------------ CPU oracle
+class _OracleData:
+    """Inputs of the oracle arm, generated once: two X / dY slots and the backbone."""
+
+    def __init__(self, O, wl, layer):
+        self.slots = [layer_inputs(wl, layer, step=s, with_b=True) for s in range(2)]
+        self.wq, self.s_w, _, _ = O.quantize(self.slots[0]["W"])
+
+
+def _oracle_sample_step(O, wl, layer, data, tokens, proxy_rows, step):
+    """One oracle step on a bounded sample: `tokens` rows of X and dY through
+    quantize / forward / dX / dB / dA, and `proxy_rows` rows of the proxy update."""
+    d = data.slots[step % 2]
+    X, dY = np.ascontiguousarray(d["X"][:tokens]), np.ascontiguousarray(d["dY"][:tokens])
+    wq, s_w = data.wq, data.s_w
+    P = np.zeros((proxy_rows, layer.K), dtype=np.float32)
+    t0 = time.perf_counter()
+    xq, s_x, _, _ = O.quantize(X)
+    O.linear_fwd(xq, s_x, wq, s_w)
+    dyq, s_dy, _, _ = O.quantize(dY)
+    O.linear_dx(dyq, s_dy, wq, s_w)
+    t64, _ = O.adapter_t(xq, s_x, d["A"])
+    db = O.adapter_db(dyq, s_dy, t64=t64)
+    u64, _ = O.adapter_u(dyq, s_dy, d["B"])
+    O.adapter_da(xq, s_x, u64=u64)
+    t1 = time.perf_counter()
+    dB_inc = O.bf16_round(-wl.lr * O.bf16_to_f64(O.bf16_round(db)))
+    O.proxy_update(np.ascontiguousarray(wq[:proxy_rows]), s_w, P,
+                   np.ascontiguousarray(dB_inc[:proxy_rows]), d["A"])
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def cpu_baseline(wl, layer, budget_s=20.0, steps=1):
+    import oracle as O
+
+    cores = os.cpu_count() or 1
+    O.set_threads(cores)
+    tokens, prows = 64, 256
+    data = _OracleData(O, wl, layer)
+    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 0)
+    # per-token and per-proxy-row costs, scaled to the full workload step
+    full_s = tg * (wl.M / tokens) + tp * (layer.N / prows)
+    return {"value": round(wl.M / full_s, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{tokens} of {wl.M} tokens through quantize/fwd/dX/dB/dA and {prows} of "
+                       f"{layer.N} proxy rows (K={layer.K}, r={wl.r}); per-token and per-row "
+                       f"times scaled to one full step"),
+            "sample_seconds": round(tg + tp, 3)}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return None, rank
+    import oracle as O
+
+    wl = WORKLOADS[args.workload]
+    layer = wl.layers[0]
+    cores = os.cpu_count() or 1
+    O.set_threads(cores)
+    tokens, prows = 16, 64
+    data = _OracleData(O, wl, layer)
+    # size the per-step sample so the whole run stays within ~3 minutes
+    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 0)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    scale = max(0.05, min(4.0, budget / max(tg + tp, 1e-6)))
+    tokens = max(1, int(tokens * scale))
+    prows = max(1, int(prows * scale))
+    for i in range(args.warmup):
+        _oracle_sample_step(O, wl, layer, data, tokens, prows, i)
+    tot_g = tot_p = 0.0
+    for i in range(args.steps):
+        g, p = _oracle_sample_step(O, wl, layer, data, tokens, prows, args.warmup + i)
+        tot_g += g
+        tot_p += p
+    per_step = tot_g / args.steps * (wl.M / tokens) + tot_p / args.steps * (layer.N / prows)
+    value = wl.M / per_step
+    sample = (f"{tokens} of {wl.M} tokens and {prows} of {layer.N} proxy rows per step; "
+              f"times scaled to one full step")
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "M": wl.M, "N": layer.N, "K": layer.K, "r": wl.r},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return out, rank
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="falqon", choices=["falqon", "reference"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        out, rank = run_reference(args)
+    else:
+        out, rank = run_gpu(args)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

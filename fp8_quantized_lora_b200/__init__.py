@@ -1,0 +1,198 @@
+"""B200 (sm_100a) hot path of FALQON's melded FP8 linear layer.
+
+A thin ctypes binding over ``libfalqon.so`` (C ABI declared in
+``include/falqon.h``).  Each Python function has the name of the C entry
+point it marshals to and only turns torch tensors into device pointers and
+the current CUDA stream into a ``void*``; all computation runs in the
+library's CUDA kernels.  There is no CPU path: importing this package without
+the built library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+__all__ = [
+    "FalqonError", "lib", "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd",
+    "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
+    "OP_QUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD", "OP_PROXY_UPDATE",
+    "PROXY_ACCUMULATE", "PROXY_SELECT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
+    "LIB_PATH", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfalqon.so")
+
+OP_QUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_PROXY_UPDATE = 0, 1, 2, 3
+DTYPE_BF16, DTYPE_F32 = 0, 1
+PROXY_ACCUMULATE, PROXY_SELECT = 1, 2
+DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
+STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
+
+EXPORTED_SYMBOLS = (
+    "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
+    "falqon_workspace_size", "falqon_status_string", "falqon_version",
+)
+
+
+class FalqonError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({falqon_status_string(self.status)})")
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded C library (ctypes), with argument types declared."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m fp8_quantized_lora_b200.build` "
+            "(there is no CPU fallback)")
+    L = C.CDLL(LIB_PATH)
+    p, i64, u32, sz = C.c_void_p, C.c_int64, C.c_uint32, C.c_size_t
+    L.falqon_quantize.argtypes = [p, C.c_int, i64, i64, p, p, p, p, p, p, sz, p]
+    L.falqon_linear_fwd.argtypes = [p, p, p, p, i64, i64, i64, p, p, p, sz, p]
+    L.falqon_linear_bwd.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p, sz, p]
+    L.falqon_proxy_update.argtypes = [p, p, p, p, p, i64, i64, i64, u32, p, p, p, p, sz, p]
+    for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update"):
+        getattr(L, f).restype = C.c_int
+    L.falqon_workspace_size.argtypes = [C.c_int, i64, i64, i64, i64]
+    L.falqon_workspace_size.restype = sz
+    L.falqon_status_string.argtypes = [C.c_int]
+    L.falqon_status_string.restype = C.c_char_p
+    L.falqon_version.restype = C.c_char_p
+    _LIB = L
+    return L
+
+
+def falqon_status_string(status: int) -> str:
+    return lib().falqon_status_string(int(status)).decode()
+
+
+def falqon_version() -> str:
+    return lib().falqon_version().decode()
+
+
+def falqon_workspace_size(op: int, M: int = 0, N: int = 0, K: int = 0, r: int = 0) -> int:
+    return int(lib().falqon_workspace_size(int(op), int(M), int(N), int(K), int(r)))
+
+
+# ------------------------------------------------------------------ marshalling helpers
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("falqon tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("falqon tensors must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise FalqonError(status, where)
+
+
+def _workspace(op, M, N, K, r, device, workspace):
+    need = falqon_workspace_size(op, M, N, K, r)
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need + 256, dtype=torch.uint8, device=device)
+        off = (-workspace.data_ptr()) % 256
+        workspace = workspace[off:off + need]
+    return workspace, workspace.numel()
+
+
+def _u8(t):
+    return t.view(torch.uint8) if t.dtype != torch.uint8 else t
+
+
+# ------------------------------------------------------------------ entry points
+def falqon_quantize(x, codes=None, scale=None, amax=None, residual=None, dev_status=None,
+                    workspace=None, stream=None):
+    """Per-tensor E4M3 quantization of a 2-D bf16/fp32 tensor; returns (codes, scale, amax)."""
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D")
+    rows, cols = x.shape
+    dt = {torch.bfloat16: DTYPE_BF16, torch.float32: DTYPE_F32}.get(x.dtype)
+    if dt is None:
+        raise ValueError("x must be bfloat16 or float32")
+    dev = x.device
+    codes = torch.empty((rows, cols), dtype=torch.uint8, device=dev) if codes is None else codes
+    scale = torch.empty(1, dtype=torch.float32, device=dev) if scale is None else scale
+    amax = torch.empty(1, dtype=torch.float32, device=dev) if amax is None else amax
+    ws, wsb = _workspace(OP_QUANTIZE, rows, cols, 0, 0, dev, workspace)
+    st = lib().falqon_quantize(_ptr(x), dt, rows, cols, _ptr(_u8(codes)), _ptr(scale), _ptr(amax),
+                               _ptr(residual), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_quantize")
+    return codes, scale, amax
+
+
+def falqon_linear_fwd(xq, s_x, wq, s_w, y=None, dev_status=None, stream=None):
+    """Y = Xq . Wq^T / (s_x s_w) in bf16."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    dev = xq.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    st = lib().falqon_linear_fwd(_ptr(_u8(xq)), _ptr(s_x), _ptr(_u8(wq)), _ptr(s_w), M, N, K,
+                                 _ptr(y), _ptr(dev_status), None, 0, _stream(stream, dev))
+    _check(st, "falqon_linear_fwd")
+    return y
+
+
+def falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=True,
+                      dev_status=None, workspace=None, stream=None):
+    """Backward of the melded layer; each output may be True (allocate), a tensor, or None."""
+    M, N = dyq.shape
+    K = wq.shape[1] if wq is not None else xq.shape[1]
+    r = A.shape[0] if A is not None else 0
+    dev = dyq.device
+
+    def out(v, shape):
+        if v is True:
+            return torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        return v if v is not None and v is not False else None
+
+    dx_t, dA_t, dB_t = out(dx, (M, K)), out(dA, (r, K)), out(dB, (N, r))
+    ws, wsb = (None, 0)
+    if dA_t is not None or dB_t is not None:
+        ws, wsb = _workspace(OP_LINEAR_BWD, M, N, K, r, dev, workspace)
+    st = lib().falqon_linear_bwd(_ptr(_u8(dyq)), _ptr(s_dy), _ptr(None if wq is None else _u8(wq)),
+                                 _ptr(s_w), _ptr(None if xq is None else _u8(xq)), _ptr(s_x),
+                                 _ptr(A), _ptr(B), M, N, K, r, _ptr(dx_t), _ptr(dA_t), _ptr(dB_t),
+                                 _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_linear_bwd")
+    return dx_t, dA_t, dB_t
+
+
+def falqon_proxy_update(wq, s_w, proxy, dB_inc, A, flags=PROXY_ACCUMULATE | PROXY_SELECT,
+                        row_mask=None, n_selected=None, dev_status=None, workspace=None,
+                        stream=None):
+    """Row-wise proxy update in place on (wq, proxy); returns (row_mask, n_selected)."""
+    N, K = proxy.shape
+    r = A.shape[0] if A is not None else 0
+    dev = proxy.device
+    if flags & PROXY_SELECT:
+        row_mask = torch.empty(N, dtype=torch.uint8, device=dev) if row_mask is None else row_mask
+        n_selected = torch.empty(1, dtype=torch.int32, device=dev) if n_selected is None else n_selected
+    ws, wsb = _workspace(OP_PROXY_UPDATE, 0, N, K, r, dev, workspace)
+    st = lib().falqon_proxy_update(_ptr(None if wq is None else _u8(wq)), _ptr(s_w), _ptr(proxy),
+                                   _ptr(dB_inc), _ptr(A), N, K, r, int(flags), _ptr(row_mask),
+                                   _ptr(n_selected), _ptr(dev_status), _ptr(ws), wsb,
+                                   _stream(stream, dev))
+    _check(st, "falqon_proxy_update")
+    return row_mask, n_selected

@@ -1,0 +1,209 @@
+// C ABI of libfalqon: argument validation, workspace layout, dispatch.
+#include <mutex>
+
+#include "../../include/falqon.h"
+#include "internal.h"
+
+namespace falqon {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::once_flag g_info_once[kMaxDevices];
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+falqon_status from_cuda(cudaError_t e) {
+  return e == cudaSuccess ? FALQON_OK
+         : e == cudaErrorInvalidValue ? FALQON_ERR_UNSUPPORTED
+                                      : FALQON_ERR_CUDA;
+}
+
+falqon_status check_ws(size_t need, const void* ws, size_t have) {
+  if (need == 0) return FALQON_OK;
+  if (!ws || have < need || !aligned256(ws)) return FALQON_ERR_WORKSPACE;
+  return FALQON_OK;
+}
+
+}  // namespace
+
+const DeviceInfo* current_device_info() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_info_once[dev], [dev]() {
+    DeviceInfo d;
+    d.device = dev;
+    cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    g_info[dev] = d;
+  });
+  return g_info[dev].sm_count > 0 ? &g_info[dev] : nullptr;
+}
+
+EncodeTiledFn encode_tiled_fn() {
+  std::call_once(g_encode_once, []() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  return g_encode;
+}
+
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes,
+                  const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace falqon
+
+using namespace falqon;
+
+extern "C" {
+
+const char* falqon_version(void) { return "falqon-b200 0.1.0 (sm_100a)"; }
+
+const char* falqon_status_string(falqon_status s) {
+  switch (s) {
+    case FALQON_OK: return "ok";
+    case FALQON_ERR_INVALID_ARG: return "invalid argument";
+    case FALQON_ERR_UNSUPPORTED: return "unsupported shape or alignment";
+    case FALQON_ERR_WORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case FALQON_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r) {
+  switch (op) {
+    case FALQON_OP_QUANTIZE: return quantize_workspace_bytes(M * N);
+    case FALQON_OP_LINEAR_FWD: return 0;
+    case FALQON_OP_LINEAR_BWD:
+      if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+      return adapter_workspace_bytes(M, N, K, r, true);
+    case FALQON_OP_PROXY_UPDATE:
+      if (N <= 0 || K <= 0) return 0;
+      return proxy_workspace_bytes(N, K);
+  }
+  return 0;
+}
+
+falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
+                              uint8_t* codes, float* scale, float* amax, float* residual,
+                              int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (!x || !codes || !scale) return FALQON_ERR_INVALID_ARG;
+  if (rows <= 0 || cols <= 0) return FALQON_ERR_INVALID_ARG;
+  if (dtype != FALQON_DTYPE_BF16 && dtype != FALQON_DTYPE_F32) return FALQON_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes) || (residual && !aligned16(residual)))
+    return FALQON_ERR_UNSUPPORTED;
+  const int64_t n = rows * cols;
+  falqon_status s = check_ws(quantize_workspace_bytes(n), workspace, workspace_bytes);
+  if (s != FALQON_OK) return s;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_quantize(x, dtype == FALQON_DTYPE_BF16, n, codes, scale, amax, residual,
+                                   dev_status, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+falqon_status falqon_linear_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!xq || !s_x || !wq || !s_w || !y) return FALQON_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256)
+    return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(y)) return FALQON_ERR_UNSUPPORTED;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_fp8_gemm_fwd(xq, s_x, wq, s_w, M, N, K, y, dev_status,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                const float* s_w, const uint8_t* xq, const float* s_x,
+                                const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
+  if (!dyq || !s_dy) return FALQON_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256)
+    return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(dyq)) return FALQON_ERR_UNSUPPORTED;
+  if (dx) {
+    if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;
+    if (!aligned16(wq) || !aligned16(dx)) return FALQON_ERR_UNSUPPORTED;
+  }
+  const bool adapters = dA || dB;
+  if (adapters) {
+    if (r <= 0 || !xq || !s_x || !A) return FALQON_ERR_INVALID_ARG;
+    if (dA && !B) return FALQON_ERR_INVALID_ARG;
+    if (r % 16 != 0 || r > 65536) return FALQON_ERR_UNSUPPORTED;
+    if (!aligned16(xq) || !aligned16(A) || (B && !aligned16(B)) || (dA && !aligned16(dA)) ||
+        (dB && !aligned16(dB)))
+      return FALQON_ERR_UNSUPPORTED;
+    falqon_status s =
+        check_ws(adapter_workspace_bytes(M, N, K, r, dA != nullptr), workspace, workspace_bytes);
+    if (s != FALQON_OK) return s;
+  }
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (adapters) {
+    cudaError_t e = launch_adapter_grads(dyq, s_dy, xq, s_x, A, B, M, N, K, r, dA, dB,
+                                         dev_status, workspace, st);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (dx) return from_cuda(launch_fp8_gemm_dx(dyq, s_dy, wq, s_w, M, N, K, dx, dev_status, st));
+  return FALQON_OK;
+}
+
+falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
+                                  const void* dB_inc, const void* A, int64_t N, int64_t K,
+                                  int64_t r, uint32_t flags, uint8_t* row_mask,
+                                  int32_t* n_selected, int32_t* dev_status, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT;
+  if (flags == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
+  if (!proxy || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
+  if (K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(proxy)) return FALQON_ERR_UNSUPPORTED;
+  if (flags & FALQON_PROXY_ACCUMULATE) {
+    if (!dB_inc || !A || r <= 0) return FALQON_ERR_INVALID_ARG;
+  }
+  if (flags & FALQON_PROXY_SELECT) {
+    if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;
+    if (!aligned16(wq)) return FALQON_ERR_UNSUPPORTED;
+    falqon_status s = check_ws(proxy_workspace_bytes(N, K), workspace, workspace_bytes);
+    if (s != FALQON_OK) return s;
+  }
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_proxy_update(wq, s_w, proxy, dB_inc, A, N, K, r, flags, row_mask,
+                                       n_selected, dev_status, workspace,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

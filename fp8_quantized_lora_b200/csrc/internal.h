@@ -1,0 +1,65 @@
+// Host-side declarations shared by the C-ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace falqon {
+
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  int max_smem_optin = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+};
+
+// Cached per device; returns nullptr if the current device cannot be queried.
+const DeviceInfo* current_device_info();
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// 2-D tensor map over a row-major [outer, inner] tensor.
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes,
+                  const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer, bool swizzle128);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- quantize
+size_t quantize_workspace_bytes(int64_t n);
+cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* codes,
+                            float* scale, float* amax, float* residual, int32_t* dev_status,
+                            void* workspace, cudaStream_t stream);
+
+// ---------------------------------------------------------------- GEMMs
+// Y[M,N] = bf16( Xq . Wq^T / (s_x s_w) )
+cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
+                                int32_t* dev_status, cudaStream_t stream);
+// dX[M,K] = bf16( dYq . Wq / (s_dy s_w) )
+cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                               const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
+                               int32_t* dev_status, cudaStream_t stream);
+
+size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da);
+cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const uint8_t* xq,
+                                 const float* s_x, const void* A, const void* B, int64_t M,
+                                 int64_t N, int64_t K, int64_t r, void* dA, void* dB,
+                                 int32_t* dev_status, void* workspace, cudaStream_t stream);
+
+// ---------------------------------------------------------------- proxy
+size_t proxy_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
+                                const void* A, int64_t N, int64_t K, int64_t r, uint32_t flags,
+                                uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
+                                void* workspace, cudaStream_t stream);
+
+}  // namespace falqon

@@ -1,0 +1,190 @@
+/*
+ * falqon.h - C ABI of libfalqon, the B200 (sm_100a) hot path of FALQON's
+ * melded FP8 linear layer: one training step of an FP8-quantized linear layer
+ * whose LoRA adapter is merged into the quantized backbone.
+ *
+ * Method: "FALQON: Accelerating LoRA Fine-tuning with Low-Bit Floating-Point
+ * Arithmetic" (NeurIPS 2025).  The paper's introduction states the problem
+ * this interface follows: quantize activations and gradients per tensor,
+ * run the forward and backward on the FP8 backbone alone (no separate LoRA
+ * path), compute the adapter gradients, and fold the adapter update back
+ * into the backbone with a row-wise proxy.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All matrices are row-major and contiguous.  bfloat16 tensors are passed
+ *    as `void*` holding IEEE bfloat16 values; E4M3 tensors as `uint8_t*`
+ *    holding OCP E4M3 codes; scales as `float*` (one float, on the device).
+ *  - Every tensor pointer is a DEVICE pointer and must be 16-byte aligned.
+ *    The caller owns every buffer; the library allocates no device memory.
+ *  - `stream` is a cudaStream_t passed as `void*` (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream and performs no
+ *    host synchronisation; scales never leave the device.
+ *  - Shape, null-pointer, alignment and workspace errors are reported by the
+ *    return value BEFORE anything is launched.  FALQON_ERR_CUDA reports a
+ *    failed launch.  Data-dependent conditions found while running
+ *    (non-finite input, scale overflow, a bounded wait that ran out) are
+ *    OR-ed into `*dev_status` (an int32 in device memory, nullable) as
+ *    FALQON_DEV_* bits; the caller reads it after its own synchronisation.
+ *  - `workspace` is caller-owned device memory of at least
+ *    falqon_workspace_size(op, ...) bytes, 256-byte aligned; it may be NULL
+ *    when that size is 0.  Calls that overlap on the GPU must not share a
+ *    workspace.  No other aliasing between arguments is allowed except the
+ *    documented in-place operands of falqon_proxy_update.
+ *  - Every function is reentrant; the only global state is a per-device
+ *    cache of device attributes and of the driver's tensor-map encoder.
+ */
+#ifndef FALQON_H_
+#define FALQON_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FALQON_API __attribute__((visibility("default")))
+#else
+#define FALQON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum falqon_status {
+  FALQON_OK = 0,
+  FALQON_ERR_INVALID_ARG = 1, /* null pointer, negative or zero size, bad flag */
+  FALQON_ERR_UNSUPPORTED = 2, /* shape or alignment outside what the kernels take */
+  FALQON_ERR_WORKSPACE = 3,   /* workspace too small or misaligned */
+  FALQON_ERR_CUDA = 4         /* a CUDA runtime or driver call failed */
+} falqon_status;
+
+typedef enum falqon_dtype {
+  FALQON_DTYPE_BF16 = 0,
+  FALQON_DTYPE_F32 = 1
+} falqon_dtype;
+
+typedef enum falqon_op {
+  FALQON_OP_QUANTIZE = 0,
+  FALQON_OP_LINEAR_FWD = 1,
+  FALQON_OP_LINEAR_BWD = 2,
+  FALQON_OP_PROXY_UPDATE = 3
+} falqon_op;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define FALQON_DEV_NONFINITE 1      /* amax of an input was NaN or infinite */
+#define FALQON_DEV_SCALE_OVERFLOW 2 /* 448/amax overflowed; the scale was clamped to FLT_MAX */
+#define FALQON_DEV_TIMEOUT 4        /* a bounded on-chip wait ran out; outputs are invalid */
+
+/* Flags of falqon_proxy_update. */
+#define FALQON_PROXY_ACCUMULATE 1u /* P += dB_inc . A */
+#define FALQON_PROXY_SELECT 2u     /* select rows, requantize them, clear their proxy */
+
+/*
+ * falqon_quantize - per-tensor E4M3 quantization.
+ *
+ * Defined by the OpenReview rebuttal of the paper (reviewer 2, W2, rewrite
+ * of the scaling sentence): a higher-precision tensor X is multiplied by a
+ * per-tensor scaling factor s_X and the product is rounded to FP8 (E4M3).
+ * The scale formula is not printed; this library uses current max-abs
+ * scaling:
+ *     amax = max |x|,  s = 448 / amax (IEEE float32 division; 1 if amax == 0),
+ *     code = E4M3_satfinite_rne( fl32(x * s) ).
+ * The optional residual is the paper's quantization error of Eq. 8
+ * (rebuttal to reviewer 2, Q3): R = x - code/s, computed in float64 and
+ * rounded to float32; it is the implicit initial adapter of melded LoRA.
+ *
+ *  x         [rows, cols] bfloat16 or float32 (dtype), device, read-only.
+ *  codes     [rows, cols] uint8 E4M3 codes, device, written.
+ *  scale     1 float, device, written (s).
+ *  amax      1 float, device, written; nullable.
+ *  residual  [rows, cols] float32, device, written; nullable.
+ *  Requirements: rows >= 1, cols >= 1, cols % 16 == 0.
+ *  Device status: NONFINITE (s is set to 1), SCALE_OVERFLOW.
+ */
+FALQON_API falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
+                              uint8_t* codes, float* scale, float* amax, float* residual,
+                              int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * falqon_linear_fwd - forward GEMM on the FP8 backbone alone.
+ *
+ * The paper's introduction: adapters are merged into the FP8 backbone, so the
+ * forward needs no separate LoRA path and no extra quantization:
+ *     Y[m,n] = sum_k dec(Xq[m,k]) * dec(Wq[n,k]) / (s_X * s_W),
+ * accumulated in float32 on the tensor cores, scaled and rounded to bf16.
+ *
+ *  xq [M, K] E4M3, s_x 1 float; wq [N, K] E4M3 (PyTorch Linear layout:
+ *  out x in), s_w 1 float; y [M, N] bfloat16, written.
+ *  Requirements: M >= 1; N, K >= 16 and multiples of 16.
+ */
+FALQON_API falqon_status falqon_linear_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/*
+ * falqon_linear_bwd - backward of the melded layer.
+ *
+ *   dX = dYq . Wq / (s_dY s_W)                      (backbone only; [M, K])
+ *   T  = bf16( Xq . A^T / s_X )                     ([M, r], kept in workspace)
+ *   dB = dYq^T . T / s_dY                           ([N, r])
+ *   U  = bf16( dYq . B / s_dY ),  dA = U^T . Xq / s_X   ([r, K])
+ * dB follows the rebuttal to reviewer 4 (Q1): B's gradient only needs A x,
+ * known at forward time.  dA is that answer's formula B^T dL/dO x^T; the
+ * paper freezes A, so dA is optional (NULL skips U and dA).
+ *
+ *  dyq [M, N] E4M3, s_dy; wq [N, K] E4M3, s_w; xq [M, K] E4M3, s_x;
+ *  A [r, K] bfloat16; B [N, r] bfloat16 (read only when dA != NULL).
+ *  dx [M, K], dA [r, K], dB [N, r]: bfloat16 outputs, each nullable.
+ *  Requirements: M >= 1; N, K multiples of 16; r >= 16 and a multiple of 16.
+ */
+FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                const float* s_w, const uint8_t* xq, const float* s_x,
+                                const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * falqon_proxy_update - row-wise proxy update of the quantized backbone.
+ *
+ * The abstract and introduction: a row-wise proxy accumulates the adapter
+ * updates and selectively applies substantial ones to the FP8 backbone,
+ * skipping updates that would vanish under quantization.  This library's
+ * rule (the pages' own rule is a top-k over rows with k not given):
+ *   ACCUMULATE: D[n,k] = float32 FMA chain over i = 0..r-1 of
+ *               dB_inc[n,i] * A[i,k], starting at +0; P = fl32(P + D).
+ *   SELECT:     t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ), c' = E4M3(t);
+ *               row n is selected iff some c' differs in value from Wq[n,k]
+ *               (+0 equals -0).  Selected rows: Wq[n,:] = c'[n,:] verbatim
+ *               and P[n,:] = +0.  Other rows: Wq bit-identical, P kept.
+ * The float32 chain is reproduced bit-for-bit (no tensor cores).
+ *
+ *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);
+ *  proxy [N, K] float32, in/out;  dB_inc [N, r] bfloat16 (the increment of
+ *  B this step: the caller folds in sign and learning rate);  A [r, K] bf16.
+ *  row_mask [N] uint8 (0/1) and n_selected (1 int32): written when SELECT is
+ *  set; nullable.
+ *  Requirements: N >= 1; K multiple of 16; r >= 1 (r unused without
+ *  ACCUMULATE); flags a nonzero subset of ACCUMULATE|SELECT.
+ */
+FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
+                                  const void* dB_inc, const void* A, int64_t N, int64_t K,
+                                  int64_t r, uint32_t flags, uint8_t* row_mask,
+                                  int32_t* n_selected, int32_t* dev_status, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Workspace bytes `op` needs for these sizes (arguments an op ignores may be 0). */
+FALQON_API size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r);
+
+/* Static description of a status code. */
+FALQON_API const char* falqon_status_string(falqon_status status);
+
+/* Library version string. */
+FALQON_API const char* falqon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FALQON_H_ */

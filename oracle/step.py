@@ -2,8 +2,8 @@
 
 Order (FALQON, [intro] and [R4-Q1]): quantize X, forward on the backbone,
 quantize dY, dX on the backbone, T = Xq A^T, dB = dYq^T T, optionally
-U = dYq B and dA = U^T Xq, then the row-wise proxy update with the adapter
-increment dB_inc.  Test infrastructure only.
+U = dYq B and dA = U^T Xq (T and U exact, float64), then the row-wise proxy
+update with the adapter increment dB_inc.  Test infrastructure only.
 """
 
 from __future__ import annotations
@@ -28,13 +28,13 @@ def layer_step(X, wq, s_w, A, B, dY, P, dB_inc=None, lr=None, want_da=True, rows
                status=st_x | st_dy)
     out["y"] = linear_fwd(xq, s_x, wq, s_w, rows=rows)
     out["dx"] = linear_dx(dyq, s_dy, wq, s_w, rows=rows)
-    t64, t16 = adapter_t(xq, s_x, A)
-    out["t64"], out["t16"] = t64, t16
-    out["db"] = adapter_db(dyq, s_dy, t16=t16)
+    t64, _ = adapter_t(xq, s_x, A)
+    out["t64"] = t64
+    out["db"] = adapter_db(dyq, s_dy, t64=t64)
     if want_da:
-        u64, u16 = adapter_u(dyq, s_dy, B)
-        out["u64"], out["u16"] = u64, u16
-        out["da"] = adapter_da(xq, s_x, u16=u16)
+        u64, _ = adapter_u(dyq, s_dy, B)
+        out["u64"] = u64
+        out["da"] = adapter_da(xq, s_x, u64=u64)
     if dB_inc is None and lr is not None:
         db16 = bf16_round(out["db"])
         db_f = (db16.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)

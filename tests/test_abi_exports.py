@@ -1,0 +1,108 @@
+"""CPU checks of the C ABI: the library loads, exports what include/falqon.h
+declares, and rejects bad arguments before touching a GPU."""
+
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import fp8_quantized_lora_b200 as F
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "falqon.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FALQON_API\s+[\w\s\*]+?\b(falqon_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls_and_helpers():
+    names = _declared()
+    for n in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
+              "falqon_workspace_size", "falqon_status_string", "falqon_version"):
+        assert n in names
+    assert set(names) == set(F.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = F.lib()
+    for n in _declared():
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", F.LIB_PATH], capture_output=True, text=True)
+    if out.returncode == 0:
+        exported = {line.split()[-1] for line in out.stdout.splitlines() if " T " in line}
+        assert set(_declared()) <= exported
+        assert not [s for s in exported if s.startswith("_ZN6falqon")], "internal symbols leaked"
+
+
+def test_status_strings_and_version():
+    assert F.falqon_status_string(0) == "ok"
+    assert "workspace" in F.falqon_status_string(3)
+    assert "sm_100a" in F.falqon_version()
+
+
+def test_workspace_sizes_are_positive_and_aligned():
+    assert F.falqon_workspace_size(F.OP_LINEAR_FWD, 4096, 4096, 4096, 64) == 0
+    for op in (F.OP_QUANTIZE, F.OP_LINEAR_BWD, F.OP_PROXY_UPDATE):
+        n = F.falqon_workspace_size(op, 4096, 4096, 4096, 64)
+        assert n > 0 and n % 256 == 0
+
+
+# Fake, 256-byte aligned addresses: validation must reject the call before any
+# pointer is dereferenced or any CUDA call is made.
+P = C.c_void_p(1 << 20)
+P8 = C.c_void_p((1 << 20) + 8)
+
+
+def test_quantize_argument_errors():
+    L = F.lib()
+    assert L.falqon_quantize(None, 0, 4, 16, P, P, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_quantize(P, 0, 0, 16, P, P, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_quantize(P, 7, 4, 16, P, P, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_quantize(P, 0, 4, 24, P, P, None, None, None, P, 1 << 20, None) == 2
+    assert L.falqon_quantize(P8, 0, 4, 16, P, P, None, None, None, P, 1 << 20, None) == 2
+    assert L.falqon_quantize(P, 0, 4, 16, P, P, None, None, None, None, 0, None) == 3
+    assert L.falqon_quantize(P, 0, 4, 16, P, P, None, None, None, P, 8, None) == 3
+
+
+def test_linear_argument_errors():
+    L = F.lib()
+    assert L.falqon_linear_fwd(None, P, P, P, 4, 16, 16, P, None, None, 0, None) == 1
+    assert L.falqon_linear_fwd(P, P, P, P, 4, 24, 16, P, None, None, 0, None) == 2
+    assert L.falqon_linear_fwd(P, P, P, P, 4, 16, 40, P, None, None, 0, None) == 2
+    assert L.falqon_linear_fwd(P, P, P, P, -1, 16, 16, P, None, None, 0, None) == 1
+    # no output requested
+    assert L.falqon_linear_bwd(P, P, P, P, P, P, P, P, 4, 16, 16, 16, None, None, None,
+                               None, P, 1 << 20, None) == 1
+    # dA requested without B
+    assert L.falqon_linear_bwd(P, P, P, P, P, P, P, None, 4, 16, 16, 16, None, P, None,
+                               None, P, 1 << 20, None) == 1
+    # r not a multiple of 16
+    assert L.falqon_linear_bwd(P, P, P, P, P, P, P, P, 4, 16, 16, 8, None, None, P,
+                               None, P, 1 << 20, None) == 2
+    # workspace too small
+    assert L.falqon_linear_bwd(P, P, P, P, P, P, P, P, 4, 16, 16, 16, None, None, P,
+                               None, P, 64, None) == 3
+
+
+def test_proxy_argument_errors():
+    L = F.lib()
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 0, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 8, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, None, P, 4, 16, 2, 1, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 20, 2, 3, None, None, None, P, 1 << 20, None) == 2
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3, None, None, None, None, 0, None) == 3
+
+
+@pytest.mark.parametrize("name", ["falqon_quantize", "falqon_linear_fwd"])
+def test_binding_refuses_cpu_tensors(name):
+    import torch
+
+    x = torch.zeros(4, 16)
+    with pytest.raises(ValueError):
+        if name == "falqon_quantize":
+            F.falqon_quantize(x)
+        else:
+            F.falqon_linear_fwd(x.to(torch.uint8), torch.ones(1), x.to(torch.uint8), torch.ones(1))

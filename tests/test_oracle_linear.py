@@ -136,16 +136,23 @@ def test_adapter_t_u_exact_rational_and_bf16_rounding():
     assert np.array_equal(u16, O.bf16_round(u64))
 
 
-def test_db_uses_bf16_t_and_da_uses_bf16_u():
+def test_db_and_da_match_numpy_products_of_exact_intermediates():
     xq, dyq, wq, A, B, s_x, s_dy, _ = _lora_case(40)
-    _, t16 = O.adapter_t(xq, s_x, A)
-    _, u16 = O.adapter_u(dyq, s_dy, B)
-    db = O.adapter_db(dyq, s_dy, t16=t16)
-    da = O.adapter_da(xq, s_x, u16=u16)
-    ref_db = (DEC[dyq].T @ _f(t16)) / np.float64(s_dy)
-    ref_da = (_f(u16).T @ DEC[xq]) / np.float64(s_x)
+    t64, _ = O.adapter_t(xq, s_x, A)
+    u64, _ = O.adapter_u(dyq, s_dy, B)
+    db = O.adapter_db(dyq, s_dy, t64=t64)
+    da = O.adapter_da(xq, s_x, u64=u64)
+    ref_t = (DEC[xq] @ _f(A).T) / np.float64(s_x)
+    ref_u = (DEC[dyq] @ _f(B)) / np.float64(s_dy)
+    assert np.allclose(t64, ref_t, rtol=1e-13, atol=1e-16)
+    assert np.allclose(u64, ref_u, rtol=1e-13, atol=1e-16)
+    ref_db = (DEC[dyq].T @ ref_t) / np.float64(s_dy)
+    ref_da = (ref_u.T @ DEC[xq]) / np.float64(s_x)
     assert np.allclose(db, ref_db, rtol=1e-12, atol=1e-15)
     assert np.allclose(da, ref_da, rtol=1e-12, atol=1e-15)
+    # the bf16-rounded intermediates the oracle also reports are single roundings of T, U
+    _, t16 = O.adapter_t(xq, s_x, A)
+    assert np.array_equal(t16, O.bf16_round(t64))
 
 
 def test_zero_b_gives_exactly_zero_u_and_da():
@@ -153,14 +160,14 @@ def test_zero_b_gives_exactly_zero_u_and_da():
     B0 = np.zeros((24, 8), dtype=np.uint16)
     u64, u16 = O.adapter_u(dyq, s_dy, B0)
     assert np.all(u64 == 0) and np.all(u16 & 0x7FFF == 0)
-    assert np.all(O.adapter_da(xq, s_x, u16=u16) == 0)
+    assert np.all(O.adapter_da(xq, s_x, u64=u64) == 0)
 
 
 def test_zero_dy_gives_exactly_zero_db_and_dx():
     xq, _, wq, A, _, s_x, s_dy, s_w = _lora_case(60)
     dyq0 = np.zeros((13, 24), dtype=np.uint8)
-    _, t16 = O.adapter_t(xq, s_x, A)
-    assert np.all(O.adapter_db(dyq0, s_dy, t16=t16) == 0)
+    t64, _ = O.adapter_t(xq, s_x, A)
+    assert np.all(O.adapter_db(dyq0, s_dy, t64=t64) == 0)
     assert np.all(O.linear_dx(dyq0, s_dy, wq, s_w) == 0)
 
 
