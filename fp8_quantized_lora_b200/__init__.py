@@ -18,7 +18,7 @@ import torch
 __all__ = [
     "FalqonError", "lib", "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd",
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
-    "OP_QUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD", "OP_PROXY_UPDATE",
+    "falqon_linear_bwd_noalloc", "OP_QUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD", "OP_PROXY_UPDATE",
     "PROXY_ACCUMULATE", "PROXY_SELECT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
@@ -34,6 +34,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: 
 EXPORTED_SYMBOLS = (
     "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
+    "falqon_linear_bwd_noalloc",
 )
 
 
@@ -62,7 +63,9 @@ def lib():
     L.falqon_linear_fwd.argtypes = [p, p, p, p, i64, i64, i64, p, p, p, sz, p]
     L.falqon_linear_bwd.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p, sz, p]
     L.falqon_proxy_update.argtypes = [p, p, p, p, p, i64, i64, i64, u32, p, p, p, p, sz, p]
-    for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update"):
+    L.falqon_linear_bwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p]
+    for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
+              "falqon_linear_bwd_noalloc"):
         getattr(L, f).restype = C.c_int
     L.falqon_workspace_size.argtypes = [C.c_int, i64, i64, i64, i64]
     L.falqon_workspace_size.restype = sz
@@ -196,3 +199,28 @@ def falqon_proxy_update(wq, s_w, proxy, dB_inc, A, flags=PROXY_ACCUMULATE | PROX
                                    _stream(stream, dev))
     _check(st, "falqon_proxy_update")
     return row_mask, n_selected
+
+
+def falqon_linear_bwd_noalloc(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=True,
+                              dev_status=None, stream=None):
+    """falqon_linear_bwd without a workspace: the library's built-in scratch
+    array holds the intermediates (for callers that cannot allocate device
+    memory).  Outputs follow falqon_linear_bwd; only the outputs themselves
+    are allocated here when passed as True."""
+    M, N = dyq.shape
+    K = wq.shape[1] if wq is not None else xq.shape[1]
+    r = A.shape[0] if A is not None else 0
+    dev = dyq.device
+
+    def out(v, shape):
+        if v is True:
+            return torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        return v if v is not None and v is not False else None
+
+    dx_t, dA_t, dB_t = out(dx, (M, K)), out(dA, (r, K)), out(dB, (N, r))
+    st = lib().falqon_linear_bwd_noalloc(
+        _ptr(_u8(dyq)), _ptr(s_dy), _ptr(None if wq is None else _u8(wq)), _ptr(s_w),
+        _ptr(None if xq is None else _u8(xq)), _ptr(s_x), _ptr(A), _ptr(B), M, N, K, r,
+        _ptr(dx_t), _ptr(dA_t), _ptr(dB_t), _ptr(dev_status), _stream(stream, dev))
+    _check(st, "falqon_linear_bwd_noalloc")
+    return dx_t, dA_t, dB_t

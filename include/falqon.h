@@ -174,6 +174,38 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/*
+ * falqon_linear_bwd_noalloc - falqon_linear_bwd for callers that cannot
+ * allocate device memory.
+ *
+ * The paper has no counterpart to this call.  It serves callers that cannot
+ * call cudaMalloc on the hot path (a host program that only holds device
+ * pointers to its own tensors under a fixed memory budget, a plugin inside a
+ * runtime that owns every allocation): it takes the same arguments as
+ * falqon_linear_bwd minus the workspace, and keeps the adapter products'
+ * intermediates in one scratch array compiled into the library.
+ *
+ *  - Limit: the scratch array is 16 MiB per device, held by every GPU that
+ *    loads the library until the process exits.  A call whose
+ *    falqon_workspace_size(FALQON_OP_LINEAR_BWD, M, N, K, r) exceeds it (with
+ *    dA requested; slightly less without) returns FALQON_ERR_WORKSPACE before
+ *    launching anything.  A dX-only call needs no scratch.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device); make that first call before
+ *    any stream capture on that device.
+ *  - Sharing: every call uses the same array, which keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls that overlap on
+ *    the GPU race on it; serialise them.
+ *  - Allocation: none (no cudaMalloc, cudaFree or allocating library call).
+ */
+FALQON_API falqon_status falqon_linear_bwd_noalloc(const uint8_t* dyq, const float* s_dy,
+                                                   const uint8_t* wq, const float* s_w,
+                                                   const uint8_t* xq, const float* s_x,
+                                                   const void* A, const void* B, int64_t M,
+                                                   int64_t N, int64_t K, int64_t r, void* dx,
+                                                   void* dA, void* dB, int32_t* dev_status,
+                                                   void* stream);
+
 /* Workspace bytes `op` needs for these sizes (arguments an op ignores may be 0). */
 FALQON_API size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r);
 
