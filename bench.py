@@ -55,6 +55,18 @@ def _peaks():
             "source": "fallback"}
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of `value` over all ranks of the default process group (no-op alone)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -161,32 +173,38 @@ class Step:
                           dev_status=self.status, workspace=self.ws_q2)
         self.launches_per_step = 2 + 1 + 2 + 8 + 1 + 2  # library kernels per step
 
-    def phases(self, slot, ev=None):
-        """Enqueues one step; `ev` (list of 6 events) brackets the five phases."""
+    PHASES = ("quantX+fwd", "quantdY+adapters", "dX", "sgd", "proxy")
+
+    def phase(self, slot, k):
+        """Enqueues phase k of one step on the current stream."""
         F, t = self.F, self.torch
-        rec = (lambda i: ev[i].record()) if ev is not None else (lambda i: None)
-        rec(0)
-        F.falqon_quantize(self.X[slot], codes=self.xq, scale=self.s_x, amax=self.amax,
-                          dev_status=self.status, workspace=self.ws_q)
-        F.falqon_linear_fwd(self.xq, self.s_x, self.wq, self.s_w, y=self.y, dev_status=self.status)
-        rec(1)
-        F.falqon_quantize(self.dY[slot], codes=self.dyq, scale=self.s_dy, amax=self.amax,
-                          dev_status=self.status, workspace=self.ws_q)
-        F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, self.xq, self.s_x, self.A,
-                            self.B, dx=None, dA=self.dA, dB=self.dB, dev_status=self.status,
-                            workspace=self.ws_bwd)
-        rec(2)
-        F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, None, None, None, None,
-                            dx=self.dx, dA=None, dB=None, dev_status=self.status)
-        rec(3)
-        # the caller's optimizer: plain SGD on B; the proxy receives the increment
-        t.mul(self.dB, -self.lr, out=self.dB_inc)
-        self.B.add_(self.dB_inc)
-        rec(4)
-        F.falqon_proxy_update(self.wq, self.s_w, self.P, self.dB_inc, self.A,
-                              row_mask=self.mask, n_selected=self.n_sel, dev_status=self.status,
-                              workspace=self.ws_p)
-        rec(5)
+        if k == 0:
+            F.falqon_quantize(self.X[slot], codes=self.xq, scale=self.s_x, amax=self.amax,
+                              dev_status=self.status, workspace=self.ws_q)
+            F.falqon_linear_fwd(self.xq, self.s_x, self.wq, self.s_w, y=self.y,
+                                dev_status=self.status)
+        elif k == 1:
+            F.falqon_quantize(self.dY[slot], codes=self.dyq, scale=self.s_dy, amax=self.amax,
+                              dev_status=self.status, workspace=self.ws_q)
+            F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, self.xq, self.s_x, self.A,
+                                self.B, dx=None, dA=self.dA, dB=self.dB, dev_status=self.status,
+                                workspace=self.ws_bwd)
+        elif k == 2:
+            F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, None, None, None, None,
+                                dx=self.dx, dA=None, dB=None, dev_status=self.status)
+        elif k == 3:
+            # the caller's optimizer: plain SGD on B; the proxy receives the increment
+            t.mul(self.dB, -self.lr, out=self.dB_inc)
+            self.B.add_(self.dB_inc)
+        else:
+            F.falqon_proxy_update(self.wq, self.s_w, self.P, self.dB_inc, self.A,
+                                  row_mask=self.mask, n_selected=self.n_sel,
+                                  dev_status=self.status, workspace=self.ws_p)
+
+    def phases(self, slot):
+        """Enqueues one whole step."""
+        for k in range(len(self.PHASES)):
+            self.phase(slot, k)
 
 
 def _phase_work(st):
@@ -229,12 +247,20 @@ def run_gpu(args):
         for slot in range(2):  # warm the library (attributes, tensor-map encoder) first
             st.phases(slot)
     torch.cuda.synchronize()
+    phase_graphs = []  # [slot][phase]: each phase alone, for launch-gap-free attribution
     if not args.no_graph:
         for slot in range(2):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 st.phases(slot)
             graphs.append(g)
+            per = []
+            for k in range(len(Step.PHASES)):
+                gk = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gk, stream=stream):
+                    st.phase(slot, k)
+                per.append(gk)
+            phase_graphs.append(per)
     torch.cuda.synchronize()
 
     def step(i):
@@ -271,21 +297,24 @@ def run_gpu(args):
     if ws > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = float(np.sum(step_ms))
-    if ws > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(np.sum(step_ms)), dev)
 
-    # per-phase timing (eager, same stream, same flush discipline)
-    names = ["quantX+fwd", "quantdY+adapters", "dX", "sgd", "proxy"]
+    # per-phase timing: each phase replayed from its own graph, back to back,
+    # events between the replays; same L2 flush discipline as the timed steps
+    names = list(Step.PHASES)
     acc = {n: 0.0 for n in names}
     reps = max(5, min(50, args.steps))
     with torch.cuda.stream(stream):
         for i in range(reps):
             flush.fill_(i & 0xFF)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-            st.phases(i % 2, ev)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            ev[0].record()
+            for k in range(len(names)):
+                if phase_graphs:
+                    phase_graphs[i % 2][k].replay()
+                else:
+                    st.phase(i % 2, k)
+                ev[k + 1].record()
             torch.cuda.synchronize()
             for j, n in enumerate(names):
                 acc[n] += ev[j].elapsed_time(ev[j + 1])
@@ -314,11 +343,7 @@ def run_gpu(args):
             hostSel.copy_(st.n_sel, non_blocking=True)
         e_end.record()
     torch.cuda.synchronize()
-    e2e_ms = e_start.elapsed_time(e_end)
-    if ws > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     status = int(st.status.item())
     n_sel = int(st.n_sel.item())
 

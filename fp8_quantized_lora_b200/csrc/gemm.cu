@@ -43,16 +43,22 @@ constexpr int kRowBytes = 128;  // every smem operand row is one 128-byte swizzl
 struct GemmArgs {
   int32_t m_tiles, n_tiles, splits, kb_total, kb_per_split;
   int64_t M, N;            // output extent (rows = UMMA M side, cols = UMMA N side)
-  void* out;               // bf16 [M, N] (ld = ldo) or fp32 partials [splits][m_pad][n_pad]
+  void* out;               // bf16 output, row-major [M][ldo] (or [N][ldo] when transposed)
+  void* out_lo;            // optional low half: out + out_lo carries ~16 significant bits
   int64_t ldo;
-  int64_t m_pad, n_pad;    // partial-buffer extents
+  int transpose;           // store out[col * ldo + row]
+  // E4M3 codes of an expanded A operand, row-major [a_rows][a_cols], read by the
+  // converter warps straight from global memory (K-major: rows = M side,
+  // cols = contraction; MN-major: rows = contraction, cols = M side)
+  const uint8_t* a_codes;
+  int64_t a_rows, a_cols;
   const float* scale_a;    // alpha = 1 / (scale_a * scale_b); either may be null (= 1)
   const float* scale_b;
   int32_t* dev_status;
 };
 
-template <bool kF8, bool kAMn, bool kBMn, bool kAConv, int kBN, int kStages, bool kPartial,
-          bool kBSplit = false>
+template <bool kF8, bool kAMn, bool kBMn, bool kAConv, int kBN, int kStages, bool kClusterK,
+          bool kBSplit = false, int kRawStages = 0>
 struct Cfg {
   static constexpr bool F8 = kF8;
   static constexpr bool AMn = kAMn;
@@ -60,7 +66,9 @@ struct Cfg {
   static constexpr bool AConv = kAConv;
   static constexpr int BN = kBN;
   static constexpr int Stages = kStages;
-  static constexpr bool Partial = kPartial;
+  // split-K across the CTAs of a cluster: each parks its fp32 tile in shared
+  // memory and the cluster sums the tiles through DSMEM in rank order
+  static constexpr bool ClusterK = kClusterK;
   static constexpr bool BSplit = kBSplit;  // B = B_hi + B_lo: two bf16 tiles, two MMAs per k-step
   static constexpr int ElemBytes = kF8 ? 1 : 2;
   static constexpr int BK = kRowBytes / ElemBytes;       // K per stage (128 fp8 / 64 bf16)
@@ -69,14 +77,20 @@ struct Cfg {
   static constexpr int ABytes = kBM * BK * ElemBytes;     // operand A tile (16 KB)
   static constexpr int BBytes = kBN * BK * ElemBytes;     // operand B tile
   static constexpr int B2Bytes = kBSplit ? BBytes : 0;   // low half of a split B operand
-  static constexpr int RawBytes = kAConv ? kBM * BK : 0;  // fp8 codes of A before expansion
-  static constexpr int StageBytes = ABytes + BBytes + B2Bytes + RawBytes;
-  static constexpr int TmaBytes = (kAConv ? RawBytes : ABytes) + BBytes + B2Bytes;
-  static constexpr int NumConvWarps = kAConv ? 4 : 0;
+  static constexpr int StageBytes = ABytes + BBytes + B2Bytes;
+  static constexpr int TmaBytes = (kAConv ? 0 : ABytes) + BBytes + B2Bytes;
+  static constexpr int NumConvWarps = kAConv ? 8 : 0;
+  // per-converter-thread ring of raw E4M3 codes (32 bytes per thread per k-block),
+  // filled with cp.async kRawStages k-blocks ahead
+  static constexpr int RawStages = kAConv ? kRawStages : 0;
+  static constexpr int RawSlotBytes = 32 * 32 * NumConvWarps;  // 8 KB
+  static_assert(!kAConv || kRawStages >= 2, "raw ring depth");
   static constexpr int Threads = 32 * (6 + NumConvWarps);
   static constexpr uint32_t TmemCols = 2 * kBN < 32 ? 32 : 2 * kBN;
   static constexpr int BarBytes = 8 * (3 * kStages + 5) + 16;
-  static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
+  static constexpr int SmemBytes = kStages * StageBytes + RawStages * RawSlotBytes + BarBytes + 1024;
+  static constexpr int RedStride = kBN + 1;  // fp32 words per row of the reduction tile
+  static_assert(!kClusterK || kBM * RedStride * 4 <= kStages * StageBytes, "reduction tile");
   static constexpr uint32_t IDesc =
       idesc_f32acc(kF8 ? 0u : 1u, kF8 ? 0u : 1u, kAMn ? 1u : 0u, kBMn ? 1u : 0u, kBM, kBN);
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
@@ -97,35 +111,42 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int ks) {
   }
 }
 
-// Expands `kRows x kCols` E4M3 codes (row-major, unswizzled) into bf16 in the
-// SWIZZLE_128B layout: 64-element column blocks of [kRows][128 B], each
-// 16-byte unit of a row XOR-ed with (row % 8).
-template <int kRows, int kCols>
-__device__ __forceinline__ void expand_codes(const uint8_t* raw, uint8_t* dst, int t,
-                                             int nthreads) {
-  constexpr int kGroups = kRows * kCols / 8;
-  for (int g = t; g < kGroups; g += nthreads) {
-    const int row = g / (kCols / 8);
-    const int col = (g % (kCols / 8)) * 8;
-    const uint2 c = *reinterpret_cast<const uint2*>(raw + row * kCols + col);
-    uint32_t out[4];
-    const uint32_t w[2] = {c.x, c.y};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint16_t pair = static_cast<uint16_t>(w[j >> 1] >> (16 * (j & 1)));
-      uint32_t h2;
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-      __half2 h;
-      memcpy(&h, &h2, 4);
-      const float2 f = __half22float2(h);
-      const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
-      memcpy(&out[j], &b, 4);
-    }
-    const int blk = col / 64;
-    const int unit = (col % 64) / 8;
-    uint8_t* p = dst + blk * (kRows * kRowBytes) + row * kRowBytes + ((unit ^ (row & 7)) << 4);
-    *reinterpret_cast<uint4*>(p) = make_uint4(out[0], out[1], out[2], out[3]);
-  }
+// 16-byte global -> shared copy, zero-filled when src_bytes == 0.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+
+// Address of `local` (this CTA's shared memory) in the shared window of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, int rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  return remote;
+}
+
+__device__ __forceinline__ float dsmem_load_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // All lanes wait; the warp agrees on the outcome so it never diverges on a timeout.
@@ -146,7 +167,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::Stages * C::StageBytes);
+  uint8_t* raw_ring = smem + C::Stages * C::StageBytes;  // converters only
+  uint64_t* bars = reinterpret_cast<uint64_t*>(raw_ring + C::RawStages * C::RawSlotBytes);
   uint64_t* full = bars;                      // TMA landed
   uint64_t* conv = bars + C::Stages;          // codes expanded (bf16 kinds)
   uint64_t* empty = bars + 2 * C::Stages;     // MMAs done reading the stage
@@ -210,17 +232,12 @@ __global__ void __launch_bounds__(C::Threads, 1)
           uint8_t* sA = smem + stage * C::StageBytes;
           uint8_t* sB = sA + C::ABytes;
           uint8_t* sB2 = sB + C::BBytes;
-          uint8_t* sRaw = sB2 + C::B2Bytes;
           mbar_arrive_expect_tx(&full[stage], C::TmaBytes);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           // operand A: rows m0.., K block kb
           if constexpr (C::AConv) {
-            if constexpr (C::AMn) {
-              tma_load_2d(sRaw, &tmA, &full[stage], m0, kb * C::BK);  // [BK rows][128 codes]
-            } else {
-              tma_load_2d(sRaw, &tmA, &full[stage], kb * C::BK, m0);  // [128 rows][BK codes]
-            }
+            // A arrives through the converter warps (global loads, expanded in place)
           } else if constexpr (C::AMn) {
 #pragma unroll
             for (int c = 0; c < kBM * C::ElemBytes / kRowBytes; ++c)
@@ -322,20 +339,20 @@ __global__ void __launch_bounds__(C::Threads, 1)
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * kBM + q * 32 + lane;
       const int64_t col_base = static_cast<int64_t>(nt) * C::BN;
+      (void)split;
 #pragma unroll 1
       for (int c = 0; c < C::BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::BN + c * 32, r);
         tmem_ld_wait();
         const int64_t col0 = col_base + c * 32;
-        if constexpr (C::Partial) {
-          float* dst = static_cast<float*>(g.out) +
-                       (static_cast<int64_t>(split) * g.m_pad + row) * g.n_pad + col0;
+        (void)col0;
+        if constexpr (C::ClusterK) {
+          // this CTA's fp32 tile, reusing the (drained) stage buffers; the +1 row
+          // stride keeps the 32 lanes (32 rows) on distinct banks
+          float* red = reinterpret_cast<float*>(smem) + (q * 32 + lane) * C::RedStride + c * 32;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            reinterpret_cast<float4*>(dst)[j] =
-                make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                            __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          for (int j = 0; j < 32; ++j) red[j] = __uint_as_float(r[j]);
         } else {
           if (row < g.M) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
@@ -364,26 +381,132 @@ __global__ void __launch_bounds__(C::Threads, 1)
     }
   } else if constexpr (C::AConv) {
     // ------------------------------------------------------------ converters
+    // 256 threads; each owns 32 codes (two 16-byte chunks) of every A tile:
+    //   K-major  [128 rows][64 codes]: row = t / 2,  columns (t % 2) * 32 ..
+    //   MN-major [64 rows][128 codes]: row = t / 4,  columns (t % 4) * 32 ..
+    // Each thread streams its own chunks with cp.async into a private slot of
+    // the raw ring RawStages k-blocks ahead, so only it reads them back and
+    // no cross-thread synchronisation is needed for the raw codes.
+    constexpr int R = C::RawStages;
+    constexpr int kTileRows = C::AMn ? C::BK : kBM;        // rows of the A tile in smem
+    constexpr int kTileCols = C::AMn ? kBM : C::BK;        // codes per row
+    constexpr int kThrPerRow = kTileCols / 32;
     const int t = threadIdx.x - 6 * 32;
+    const int trow = t / kThrPerRow;
+    const int tcol = (t % kThrPerRow) * 32;
+    uint8_t* my_raw = raw_ring + t * 32;
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int split = w % g.splits;
+      const int mt = w / (g.splits * g.n_tiles);
       const int kb0 = split * g.kb_per_split;
       const int kb1 = min(g.kb_total, kb0 + g.kb_per_split);
+      const int64_t m0 = static_cast<int64_t>(mt) * kBM;
+      auto fetch = [&](int kb, int slot) {
+        const int64_t grow = C::AMn ? static_cast<int64_t>(kb) * C::BK + trow : m0 + trow;
+        const int64_t gcol = C::AMn ? m0 + tcol : static_cast<int64_t>(kb) * C::BK + tcol;
+        const uint8_t* src = g.a_codes + grow * g.a_cols + gcol;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const bool valid = grow < g.a_rows && gcol + 16 * h < g.a_cols;
+          cp_async16(my_raw + slot * C::RawSlotBytes + 16 * h, valid ? src + 16 * h : g.a_codes,
+                     valid ? 16u : 0u);
+        }
+      };
+#pragma unroll 1
+      for (int d = 0; d < R; ++d) {
+        if (kb0 + d < kb1) fetch(kb0 + d, d);
+        cp_async_commit();
+      }
+      int slot = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!warp_wait(&full[stage], phase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+        cp_async_wait<R - 1>();  // this thread's chunks of k-block kb have landed
+        if (!warp_wait(&empty[stage], phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+        const uint4 q0 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes + 16);
         uint8_t* sA = smem + stage * C::StageBytes;
-        const uint8_t* sRaw = sA + C::ABytes + C::BBytes + C::B2Bytes;
-        if constexpr (C::AMn) expand_codes<C::BK, kBM>(sRaw, sA, t, 128);
-        else expand_codes<kBM, C::BK>(sRaw, sA, t, 128);
+        // 32 codes -> 32 bf16 (four 16-byte units of the 128-byte-swizzled layout)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t w0 = (u & 2) ? ((u & 1) ? q1.z : q1.x) : ((u & 1) ? q0.z : q0.x);
+          const uint32_t w1 = (u & 2) ? ((u & 1) ? q1.w : q1.y) : ((u & 1) ? q0.w : q0.y);
+          uint32_t o[4];
+          const uint32_t wv[2] = {w0, w1};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint16_t pair = static_cast<uint16_t>(wv[j >> 1] >> (16 * (j & 1)));
+            uint32_t h2;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+            __half2 hh;
+            memcpy(&hh, &h2, 4);
+            const float2 f = __half22float2(hh);
+            const __nv_bfloat162 bb = __floats2bfloat162_rn(f.x, f.y);
+            memcpy(&o[j], &bb, 4);
+          }
+          const int col = tcol + 8 * u;
+          const int blk = col / 64;
+          const int unit = (col % 64) / 8;
+          uint8_t* dst = sA + blk * (kTileRows * kRowBytes) + trow * kRowBytes +
+                         ((unit ^ (trow & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&conv[stage]);
         if (++stage == C::Stages) { stage = 0; phase ^= 1; }
+        // refill the slot just read (its codes are already in registers)
+        if (kb + R < kb1) fetch(kb + R, slot);
+        cp_async_commit();
+        if (++slot == R) slot = 0;
+      }
+      cp_async_wait<0>();
+    }
+    (void)kTileCols;
+  }
+
+  if constexpr (C::ClusterK) {
+    // One work item per CTA: rank = split.  Sum the cluster's tiles row slice by
+    // row slice (this CTA owns rows [q0, q1) of the tile), in rank order.
+    __syncthreads();
+    cluster_sync_all();
+    const int S = g.splits;
+    const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
+    const int w = blockIdx.x;
+    const int nt = (w / S) % g.n_tiles;
+    const int mt = w / (S * g.n_tiles);
+    const int rows_per = (kBM + S - 1) / S;
+    const int q0 = static_cast<int>(rank) * rows_per;
+    const int q1 = min(kBM, q0 + rows_per);
+    const float* red = reinterpret_cast<const float*>(smem);
+    uint32_t peer[16];
+    for (int sidx = 0; sidx < S && sidx < 16; ++sidx) peer[sidx] = dsmem_addr(red, sidx);
+    double den = 1.0;
+    if (g.scale_a) den *= static_cast<double>(*g.scale_a);
+    if (g.scale_b) den *= static_cast<double>(*g.scale_b);
+    const float alpha = static_cast<float>(1.0 / den);
+    const int nrows = q1 - q0;
+    const int nelem = nrows > 0 ? nrows * C::BN : 0;
+    for (int e = threadIdx.x; e < nelem; e += blockDim.x) {
+      int lr, lc;
+      if (g.transpose) { lr = q0 + e % nrows; lc = e / nrows; }  // walk rows: coalesced out[col][row]
+      else { lr = q0 + e / C::BN; lc = e % C::BN; }
+      const uint32_t off = static_cast<uint32_t>((lr * C::RedStride + lc) * 4);
+      float acc = 0.0f;
+      for (int sidx = 0; sidx < S; ++sidx) acc += dsmem_load_f32(peer[sidx] + off);
+      const int64_t grow = static_cast<int64_t>(mt) * kBM + lr;
+      const int64_t gcol = static_cast<int64_t>(nt) * C::BN + lc;
+      if (grow < g.M && gcol < g.N) {
+        const float v = acc * alpha;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        const int64_t idx = g.transpose ? gcol * g.ldo + grow : grow * g.ldo + gcol;
+        static_cast<__nv_bfloat16*>(g.out)[idx] = hi;
+        if (g.out_lo)
+          static_cast<__nv_bfloat16*>(g.out_lo)[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
       }
     }
+    cluster_sync_all();  // no CTA leaves while a peer still reads its tile
   }
 
   tc_fence_before();
@@ -391,40 +514,6 @@ __global__ void __launch_bounds__(C::Threads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TmemCols);
-  }
-}
-
-// ---------------------------------------------------------------- reduce
-// v = alpha * sum_s part[s] over [rows, cols] (fixed order s = 0..splits-1);
-// out = bf16(v), and when `out_lo` is given out_lo = bf16(v - out), so that
-// out + out_lo carries v to about 16 significant bits.  Transposed store
-// (out[col][row]) when `transpose`.
-__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, int64_t m_pad,
-                                     int64_t n_pad, int64_t rows, int64_t cols,
-                                     const float* scale_a, const float* scale_b, int transpose,
-                                     __nv_bfloat16* __restrict__ out,
-                                     __nv_bfloat16* __restrict__ out_lo) {
-  double den = 1.0;
-  if (scale_a) den *= static_cast<double>(*scale_a);
-  if (scale_b) den *= static_cast<double>(*scale_b);
-  const float alpha = static_cast<float>(1.0 / den);
-  const int64_t n = rows * cols;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    int64_t r, c;
-    if (transpose) {  // consecutive threads walk consecutive output elements out[c][r]
-      c = i / rows;
-      r = i % rows;
-    } else {
-      r = i / cols;
-      c = i % cols;
-    }
-    float acc = 0.0f;
-    for (int s = 0; s < splits; ++s) acc += part[(s * m_pad + r) * n_pad + c];
-    const float v = acc * alpha;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    out[i] = hi;
-    if (out_lo) out_lo[i] = __float2bfloat16_rn(v - __bfloat162float(hi));
   }
 }
 
@@ -443,24 +532,63 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
   const int total = g.m_tiles * g.n_tiles * g.splits;
-  const int grid = total < di->sm_count ? total : di->sm_count;
-  tc_gemm_kernel<C><<<grid, C::Threads, C::SmemBytes, stream>>>(tA, tB, tB2, g);
-  return cudaGetLastError();
+  if constexpr (C::ClusterK) {
+    // one work item per CTA; the `splits` CTAs of an output tile form one cluster
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(g.splits);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(total));
+    cfg.blockDim = dim3(C::Threads);
+    cfg.dynamicSmemBytes = C::SmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<C>, tA, tB, tB2, g);
+  } else {
+    const int grid = total < di->sm_count ? total : di->sm_count;
+    tc_gemm_kernel<C><<<grid, C::Threads, C::SmemBytes, stream>>>(tA, tB, tB2, g);
+    return cudaGetLastError();
+  }
 }
 
 inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 using FwdCfg = Cfg<true, false, false, false, 256, 4, false>;
 using DxCfg = Cfg<true, false, true, false, 256, 4, false>;
+using FwdCfg128 = Cfg<true, false, false, false, 128, 6, false>;
+using DxCfg128 = Cfg<true, false, true, false, 128, 6, false>;
 
-template <int BN> using TCfg = Cfg<false, false, false, true, BN, 4, true>;   // Xq . A^T
-template <int BN> using UCfg = Cfg<false, false, true, true, BN, 4, true>;    // dYq . B
+// Tile width for an FP8 GEMM with an M x Ncols output: 128x256 tiles unless
+// 128x128 tiles fill the last wave of persistent CTAs much better (128-wide
+// tiles move 1/3 more operand bytes per flop, weighed as a 5% cost).
+int fp8_tile_n(int64_t M, int64_t Ncols, int sms) {
+  auto wave_eff = [&](int bn) {
+    const int64_t tiles = ((M + kBM - 1) / kBM) * ((Ncols + bn - 1) / bn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    return static_cast<double>(tiles) / static_cast<double>(waves * sms);
+  };
+  (void)wave_eff;
+  // Measured on B200: 128x128 tiles need 128 B/clk/SM of operand traffic and
+  // run L2-bound (dX 4096^3: 87 us vs 59 us with 128x256), so 256 is kept.
+  return 256;
+}
+
+template <int BN> using TCfg = Cfg<false, false, false, true, BN, (BN >= 256 ? 3 : 4), true, false,
+                                   (BN >= 128 ? 8 : 12)>;  // Xq . A^T
+template <int BN> using UCfg = Cfg<false, false, true, true, BN, (BN >= 256 ? 3 : 4), true, false,
+                                   (BN >= 128 ? 8 : 12)>;  // dYq . B
 // dYq^T . (T_hi + T_lo), Xq^T . (U_hi + U_lo): fewer stages at BN = 256 to fit smem
-template <int BN> using MnCfg = Cfg<false, true, true, true, BN, (BN >= 256 ? 2 : (BN >= 128 ? 3 : 4)), true, true>;
+template <int BN> using MnCfg = Cfg<false, true, true, true, BN, (BN >= 256 ? 2 : (BN >= 128 ? 3 : 4)), true, true,
+                                    (BN >= 256 ? 6 : (BN >= 128 ? 8 : 10))>;
 
-// Split count that fills the SMs with whole K blocks per split.
+// Split count: as many K splits as fit beside the tiles in one wave, at most 8
+// (the portable cluster size), never more than there are K blocks.
 int choose_splits(int tiles, int kb_total, int sm_count) {
-  int s = (sm_count + tiles - 1) / tiles;
+  int s = sm_count / (tiles > 0 ? tiles : 1);
+  if (s > 8) s = 8;
   if (s > kb_total) s = kb_total;
   if (s < 1) s = 1;
   return s;
@@ -483,7 +611,6 @@ int skinny_bn(int64_t r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
 
 struct SkinnyPlan {
   int bn, m_tiles, n_tiles, kb_total, splits, kb_per_split;
-  int64_t m_pad, n_pad;
 };
 
 SkinnyPlan plan_skinny(int64_t rows_out, int64_t r, int64_t kc, int sm_count) {
@@ -495,100 +622,86 @@ SkinnyPlan plan_skinny(int64_t rows_out, int64_t r, int64_t kc, int sm_count) {
   p.splits = choose_splits(p.m_tiles * p.n_tiles, p.kb_total, sm_count);
   p.kb_per_split = ceil_div(p.kb_total, p.splits);
   p.splits = ceil_div(p.kb_total, p.kb_per_split);  // no empty split
-  p.m_pad = static_cast<int64_t>(p.m_tiles) * kBM;
-  p.n_pad = static_cast<int64_t>(p.n_tiles) * p.bn;
   return p;
-}
-
-size_t plan_partial_bytes(const SkinnyPlan& p) {
-  return static_cast<size_t>(p.splits) * p.m_pad * p.n_pad * sizeof(float);
-}
-
-cudaError_t launch_reduce(const float* part, const SkinnyPlan& p, int64_t rows, int64_t cols,
-                          const float* sa, const float* sb, bool transpose, void* out,
-                          void* out_lo, cudaStream_t stream) {
-  const DeviceInfo* di = current_device_info();
-  const int64_t n = rows * cols;
-  int64_t blocks = (n + 255) / 256;
-  if (blocks > di->sm_count * 8) blocks = di->sm_count * 8;
-  splitk_reduce_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(
-      part, p.splits, p.m_pad, p.n_pad, rows, cols, sa, sb, transpose ? 1 : 0,
-      static_cast<__nv_bfloat16*>(out), static_cast<__nv_bfloat16*>(out_lo));
-  return cudaGetLastError();
 }
 
 }  // namespace
 
 // ------------------------------------------------------------------ big GEMMs
+namespace {
+
+template <class C>
+cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
+                     int64_t M, int64_t Ncols, int64_t Kc, bool b_mn, void* out,
+                     int32_t* dev_status, cudaStream_t stream) {
+  CUtensorMap tA, tB;
+  // A [M, Kc] K-major; B K-major [Ncols, Kc] or MN-major [Kc, Ncols]
+  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a, Kc, M, 128, kBM, true))
+    return cudaErrorInvalidValue;
+  const bool okb = b_mn ? make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Ncols, Kc, 128, C::BK, true)
+                        : make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::BN, true);
+  if (!okb) return cudaErrorInvalidValue;
+  GemmArgs g{};
+  g.m_tiles = ceil_div(M, kBM);
+  g.n_tiles = ceil_div(Ncols, C::BN);
+  g.splits = 1;
+  g.kb_total = ceil_div(Kc, C::BK);
+  g.kb_per_split = g.kb_total;
+  g.M = M;
+  g.N = Ncols;
+  g.out = out;
+  g.ldo = Ncols;
+  g.scale_a = sa;
+  g.scale_b = sb;
+  g.dev_status = dev_status;
+  return launch_gemm<C>(tA, tB, tB, g, stream);
+}
+
+}  // namespace
+
 cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
                                 const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
                                 int32_t* dev_status, cudaStream_t stream) {
-  CUtensorMap tA, tB;
-  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, K, M, 128, kBM, true) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, K, N, 128, FwdCfg::BN, true))
-    return cudaErrorInvalidValue;
-  GemmArgs g{};
-  g.m_tiles = ceil_div(M, kBM);
-  g.n_tiles = ceil_div(N, FwdCfg::BN);
-  g.splits = 1;
-  g.kb_total = ceil_div(K, FwdCfg::BK);
-  g.kb_per_split = g.kb_total;
-  g.M = M;
-  g.N = N;
-  g.out = y;
-  g.ldo = N;
-  g.scale_a = s_x;
-  g.scale_b = s_w;
-  g.dev_status = dev_status;
-  return launch_gemm<FwdCfg>(tA, tB, tB, g, stream);
+  const DeviceInfo* di = current_device_info();
+  if (!di) return cudaErrorInvalidDevice;
+  if (fp8_tile_n(M, N, di->sm_count) == 128)
+    return fp8_gemm<FwdCfg128>(xq, s_x, wq, s_w, M, N, K, false, y, dev_status, stream);
+  return fp8_gemm<FwdCfg>(xq, s_x, wq, s_w, M, N, K, false, y, dev_status, stream);
 }
 
 cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
                                int32_t* dev_status, cudaStream_t stream) {
   // contraction over N: A = dYq [M, N] K-major; B = Wq [N, K] read MN-major (K contiguous)
-  CUtensorMap tA, tB;
-  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, dyq, N, M, 128, kBM, true) ||
-      !make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq, K, N, 128, DxCfg::BK, true))
-    return cudaErrorInvalidValue;
-  GemmArgs g{};
-  g.m_tiles = ceil_div(M, kBM);
-  g.n_tiles = ceil_div(K, DxCfg::BN);
-  g.splits = 1;
-  g.kb_total = ceil_div(N, DxCfg::BK);
-  g.kb_per_split = g.kb_total;
-  g.M = M;
-  g.N = K;
-  g.out = dx;
-  g.ldo = K;
-  g.scale_a = s_dy;
-  g.scale_b = s_w;
-  g.dev_status = dev_status;
-  return launch_gemm<DxCfg>(tA, tB, tB, g, stream);
+  const DeviceInfo* di = current_device_info();
+  if (!di) return cudaErrorInvalidDevice;
+  if (fp8_tile_n(M, K, di->sm_count) == 128)
+    return fp8_gemm<DxCfg128>(dyq, s_dy, wq, s_w, M, K, N, true, dx, dev_status, stream);
+  return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, true, dx, dev_status, stream);
 }
 
 // ------------------------------------------------------------------ adapter products
-// Workspace: T_hi, T_lo, U_hi, U_lo bf16 [M, r] | fp32 partials (largest plan).
-// T and U are carried as bf16 hi/lo pairs (about 16 significant bits): a
-// single bf16 rounding of T would move small dB entries by more than one bf16
-// ulp of the tensor's scale.
+// Workspace: T_hi, T_lo, U_hi, U_lo, each bf16 [M, r].  T and U are carried
+// as bf16 hi/lo pairs (about 16 significant bits): a single bf16 rounding of
+// T would move small dB entries by more than one bf16 ulp of the tensor's
+// scale.  The split-K sums never leave the chip (cluster reduction).
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da) {
-  const DeviceInfo* di = current_device_info();
-  const int sms = di ? di->sm_count : 148;
+  (void)N;
+  (void)K;
+  (void)want_da;
   const size_t tu = align_up(static_cast<size_t>(M) * r * 2, 256);
-  size_t part = plan_partial_bytes(plan_skinny(M, r, K, sms));            // T
-  part = std::max(part, plan_partial_bytes(plan_skinny(N, r, M, sms)));   // dB
-  if (want_da) {
-    part = std::max(part, plan_partial_bytes(plan_skinny(M, r, N, sms)));  // U
-    part = std::max(part, plan_partial_bytes(plan_skinny(K, r, M, sms)));  // dA^T
-  }
-  return 4 * tu + align_up(part, 256);
+  return 4 * tu;
 }
 
 namespace {
 
-GemmArgs skinny_args(const SkinnyPlan& p, int64_t rows, int64_t r, float* part, int32_t* st) {
+GemmArgs skinny_args(const SkinnyPlan& p, int64_t rows, int64_t r, void* out, void* out_lo,
+                     int64_t ldo, bool transpose, const float* scale, int32_t* st,
+                     const uint8_t* codes, int64_t code_rows, int64_t code_cols) {
   GemmArgs g{};
+  g.a_codes = codes;
+  g.a_rows = code_rows;
+  g.a_cols = code_cols;
   g.m_tiles = p.m_tiles;
   g.n_tiles = p.n_tiles;
   g.splits = p.splits;
@@ -596,9 +709,12 @@ GemmArgs skinny_args(const SkinnyPlan& p, int64_t rows, int64_t r, float* part, 
   g.kb_per_split = p.kb_per_split;
   g.M = rows;
   g.N = r;
-  g.out = part;
-  g.m_pad = p.m_pad;
-  g.n_pad = p.n_pad;
+  g.out = out;
+  g.out_lo = out_lo;
+  g.ldo = ldo;
+  g.transpose = transpose ? 1 : 0;
+  g.scale_a = scale;
+  g.scale_b = nullptr;
   g.dev_status = st;
   return g;
 }
@@ -617,53 +733,41 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   void* T_lo = ws + tu;
   void* U_hi = ws + 2 * tu;
   void* U_lo = ws + 3 * tu;
-  float* part = reinterpret_cast<float*>(ws + 4 * tu);
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   cudaError_t e;
   CUtensorMap tA, tB, tB2;
 
   if (dB) {
-    // T = Xq . A^T / s_x: A-op Xq [M, K] K-major (expanded), B-op A [r, K] K-major
+    // T = Xq . A^T / s_x -> (T_hi, T_lo): A-op Xq [M, K] K-major (expanded), B-op A [r, K] K-major
     SkinnyPlan p = plan_skinny(M, r, K, di->sm_count);
-    if (!make_tmap_2d(&tA, U8, 1, xq, K, M, 64, kBM, false) ||
-        !make_tmap_2d(&tB, BF, 2, A, K, r, 64, p.bn, true))
-      return cudaErrorInvalidValue;
-    GemmArgs g = skinny_args(p, M, r, part, dev_status);
+    if (!make_tmap_2d(&tB, BF, 2, A, K, r, 64, p.bn, true)) return cudaErrorInvalidValue;
+    tA = tB;  // A is read by the converter warps, not by TMA
+    GemmArgs g = skinny_args(p, M, r, T_hi, T_lo, r, false, s_x, dev_status, xq, M, K);
     if ((e = skinny_dispatch<TCfg>(p.bn, tA, tB, tB, g, stream)) != cudaSuccess) return e;
-    if ((e = launch_reduce(part, p, M, r, s_x, nullptr, false, T_hi, T_lo, stream)) != cudaSuccess)
-      return e;
     // dB = dYq^T . (T_hi + T_lo) / s_dy: A-op dYq^T (MN-major, expanded), B-op T [M, r] MN-major
     SkinnyPlan q = plan_skinny(N, r, M, di->sm_count);
-    if (!make_tmap_2d(&tA, U8, 1, dyq, N, M, 128, 64, false) ||
-        !make_tmap_2d(&tB, BF, 2, T_hi, r, M, 64, 64, true) ||
+    if (!make_tmap_2d(&tB, BF, 2, T_hi, r, M, 64, 64, true) ||
         !make_tmap_2d(&tB2, BF, 2, T_lo, r, M, 64, 64, true))
       return cudaErrorInvalidValue;
-    GemmArgs h = skinny_args(q, N, r, part, dev_status);
+    tA = tB;
+    GemmArgs h = skinny_args(q, N, r, dB, nullptr, r, false, s_dy, dev_status, dyq, M, N);
     if ((e = skinny_dispatch<MnCfg>(q.bn, tA, tB, tB2, h, stream)) != cudaSuccess) return e;
-    if ((e = launch_reduce(part, q, N, r, s_dy, nullptr, false, dB, nullptr, stream)) != cudaSuccess)
-      return e;
   }
   if (dA) {
-    // U = dYq . B / s_dy: A-op dYq [M, N] K-major (expanded), B-op B [N, r] MN-major
+    // U = dYq . B / s_dy -> (U_hi, U_lo): A-op dYq [M, N] K-major (expanded), B-op B [N, r] MN-major
     SkinnyPlan p = plan_skinny(M, r, N, di->sm_count);
-    if (!make_tmap_2d(&tA, U8, 1, dyq, N, M, 64, kBM, false) ||
-        !make_tmap_2d(&tB, BF, 2, B, r, N, 64, 64, true))
-      return cudaErrorInvalidValue;
-    GemmArgs g = skinny_args(p, M, r, part, dev_status);
+    if (!make_tmap_2d(&tB, BF, 2, B, r, N, 64, 64, true)) return cudaErrorInvalidValue;
+    tA = tB;
+    GemmArgs g = skinny_args(p, M, r, U_hi, U_lo, r, false, s_dy, dev_status, dyq, M, N);
     if ((e = skinny_dispatch<UCfg>(p.bn, tA, tB, tB, g, stream)) != cudaSuccess) return e;
-    if ((e = launch_reduce(part, p, M, r, s_dy, nullptr, false, U_hi, U_lo, stream)) != cudaSuccess)
-      return e;
     // dA^T = Xq^T . (U_hi + U_lo) / s_x, stored transposed into dA [r, K]
     SkinnyPlan q = plan_skinny(K, r, M, di->sm_count);
-    if (!make_tmap_2d(&tA, U8, 1, xq, K, M, 128, 64, false) ||
-        !make_tmap_2d(&tB, BF, 2, U_hi, r, M, 64, 64, true) ||
+    if (!make_tmap_2d(&tB, BF, 2, U_hi, r, M, 64, 64, true) ||
         !make_tmap_2d(&tB2, BF, 2, U_lo, r, M, 64, 64, true))
       return cudaErrorInvalidValue;
-    GemmArgs h = skinny_args(q, K, r, part, dev_status);
+    tA = tB;
+    GemmArgs h = skinny_args(q, K, r, dA, nullptr, K, true, s_x, dev_status, xq, M, K);
     if ((e = skinny_dispatch<MnCfg>(q.bn, tA, tB, tB2, h, stream)) != cudaSuccess) return e;
-    if ((e = launch_reduce(part, q, K, r, s_x, nullptr, true, dA, nullptr, stream)) != cudaSuccess)
-      return e;
   }
   return cudaSuccess;
 }

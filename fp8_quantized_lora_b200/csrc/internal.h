@@ -31,7 +31,7 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes
                   const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                   uint32_t box_outer, bool swizzle128);
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // ---------------------------------------------------------------- quantize
 size_t quantize_workspace_bytes(int64_t n);

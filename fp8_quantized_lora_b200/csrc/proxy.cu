@@ -55,6 +55,39 @@ __device__ __forceinline__ bool same_value(uint32_t a, uint32_t b) {
   return !nan && (a == b || ((a & 0x7Fu) == 0u && (b & 0x7Fu) == 0u));
 }
 
+// Values of the two codes in the low 16 bits of `c2` (hardware conversion via f16).
+__device__ __forceinline__ float2 e4m3x2_values(uint32_t c2) {
+  uint32_t h2;
+  const uint16_t c = static_cast<uint16_t>(c2);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+  __half2 h;
+  memcpy(&h, &h2, 4);
+  return __half22float2(h);
+}
+
+// Four codes (bytes of w4) -> four new codes E4M3(dec(c) + s_w * p), no FMA.
+__device__ __forceinline__ uint32_t requantized4(uint32_t w4, float s_w, float4 p) {
+  const float2 d01 = e4m3x2_values(w4);
+  const float2 d23 = e4m3x2_values(w4 >> 16);
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(lo)
+      : "f"(__fadd_rn(d01.y, __fmul_rn(s_w, p.y))), "f"(__fadd_rn(d01.x, __fmul_rn(s_w, p.x))));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+      : "=h"(hi)
+      : "f"(__fadd_rn(d23.y, __fmul_rn(s_w, p.w))), "f"(__fadd_rn(d23.x, __fmul_rn(s_w, p.z))));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Does any of the four byte pairs differ in value (+0 == -0; a NaN code differs)?
+__device__ __forceinline__ bool codes_changed4(uint32_t a, uint32_t b) {
+  bool changed = false;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    changed |= !same_value((a >> (8 * c)) & 0xFFu, (b >> (8 * c)) & 0xFFu);
+  return changed;
+}
+
 // New code for one element: E4M3( dec(c) + s_w * p ), no fused multiply-add.
 __device__ __forceinline__ uint32_t requantized(uint32_t c, float s_w, float p) {
   return e4m3_code(__fadd_rn(e4m3_value(c), __fmul_rn(s_w, p)));
@@ -193,6 +226,357 @@ __global__ void __launch_bounds__(kSelThreads)
   if (threadIdx.x == 0 && my_count && n_selected) atomicAdd(n_selected, my_count);
 }
 
+// ---------------------------------------------------------------- single pass
+// One cluster of `cs` CTAs owns a row group of `rb` rows at a time; CTA q of
+// the cluster owns the column slice [q*wc, (q+1)*wc) for the whole kernel and
+// keeps A[:, slice] resident in shared memory (bf16, converted exactly to
+// float32 at use).  Each thread holds kRT rows x 4 columns of P' = P + D in
+// registers; the per-row "some code changes" bits are OR-ed inside the CTA,
+// published in shared memory and OR-ed across the cluster through DSMEM
+// after one cluster barrier per row group.  Then every element is written
+// once: P' (row kept) or +0 and the new codes (row selected).  Traffic per
+// element: read P and Wq, write P, and write Wq only for selected rows.
+constexpr int kRT = 8;  // rows per thread
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+
+__device__ __forceinline__ uint32_t dsmem_load_u32(const uint32_t* local, uint32_t rank) {
+  uint32_t remote, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// 4-byte store into cluster CTA `rank`'s shared memory at the same offset as
+// `local_dst`, counted as 4 transaction bytes on that CTA's mbarrier at the
+// offset of `local_bar`.
+__device__ __forceinline__ void st_async_u32(uint32_t* local_dst, uint64_t* local_bar,
+                                             uint32_t rank, uint32_t value) {
+  uint32_t rdst, rbar;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rdst) : "r"(smem_u32(local_dst)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(smem_u32(local_bar)), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(rdst),
+               "r"(value), "r"(rbar)
+               : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+struct ProxyGeom {
+  int cs, wc, cg, rs, rb, threads;
+  size_t smem;
+};
+
+template <bool kAcc, bool kSel>
+__global__ void __launch_bounds__(256, 2)
+    proxy_cluster_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
+                         float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
+                         const uint16_t* __restrict__ A, int64_t N, int64_t K, int r,
+                         ProxyGeom geo, int n_groups, uint8_t* row_mask, int32_t* n_selected,
+                         int32_t* dev_status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int wc = geo.wc, cg = geo.cg, rb = geo.rb, cs = geo.cs;
+  uint16_t* As = reinterpret_cast<uint16_t*>(sm);                       // [r][wc] bf16
+  const size_t as_bytes = align_up(static_cast<size_t>(r) * wc * 2, 16);
+  // [2][r][rb] pairs (b, b): the FFMA2 operand comes straight from a broadcast load
+  float2* Bs0 = reinterpret_cast<float2*>(sm + as_bytes);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(Bs0 + 2 * static_cast<size_t>(r) * rb);  // [2]
+  uint32_t* xbuf = reinterpret_cast<uint32_t*>(mbar + 2);  // [2] this CTA's row bits
+  uint32_t* inbox = xbuf + 2;                              // [2][16] row bits from each CTA
+  __shared__ int abort_flag;
+
+  const uint32_t crank = cs > 1 ? cluster_ctarank() : 0u;
+  const int n_clusters = gridDim.x / cs;
+  const int tid = threadIdx.x;
+  const int tcg = tid % cg;
+  const int trs = tid / cg;
+  const bool active = trs < geo.rs;
+  const int64_t c0 = static_cast<int64_t>(crank) * wc;
+  const int64_t col = c0 + 4 * tcg;
+  const bool col_ok = active && (4 * tcg < wc) && col < K;
+
+  // A[:, slice] -> shared memory, once (16-byte chunks; K % 8 == 0 keeps them aligned)
+  if constexpr (kAcc) {
+    const int chunks = wc / 8;
+    for (int e = tid; e < r * chunks; e += blockDim.x) {
+      const int i = e / chunks, c8 = e % chunks;
+      const int64_t gc = c0 + 8 * c8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (gc < K) v = *reinterpret_cast<const uint4*>(A + static_cast<int64_t>(i) * K + gc);
+      *reinterpret_cast<uint4*>(As + static_cast<size_t>(i) * wc + 8 * c8) = v;
+    }
+  }
+  if (tid < 2) xbuf[tid] = 0u;
+  if (tid == 0) {
+    mbar_init(&mbar[0], 1);
+    mbar_init(&mbar[1], 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  const float s_w = kSel ? *s_w_ptr : 1.0f;
+
+  // dB_inc rows of a group -> (registers) -> Bs[buffer] as float32, [i][row]
+  constexpr int kMaxB = 8;  // rb * r <= 32 * 1024 elements over >= 32 threads... bounded below
+  const int per_thread_b = (rb * r + blockDim.x - 1) / blockDim.x;
+  auto load_b = [&](int g, uint16_t (&v)[kMaxB], int k0) {
+#pragma unroll
+    for (int k = 0; k < kMaxB; ++k) {
+      const int e = tid + (k0 + k) * blockDim.x;
+      v[k] = 0;
+      if (k0 + k < per_thread_b && e < rb * r) {
+        const int row = e / r, i = e % r;
+        const int64_t n = static_cast<int64_t>(g) * rb + row;
+        if (n < N) v[k] = dB_inc[n * r + i];
+      }
+    }
+  };
+  auto store_b = [&](const uint16_t (&v)[kMaxB], int k0, float2* dst) {
+#pragma unroll
+    for (int k = 0; k < kMaxB; ++k) {
+      const int e = tid + (k0 + k) * blockDim.x;
+      if (k0 + k < per_thread_b && e < rb * r) {
+        const int row = e / r, i = e % r;
+        const float f = bf16_bits_to_f32(v[k]);
+        dst[static_cast<size_t>(i) * rb + row] = make_float2(f, f);
+      }
+    }
+  };
+  auto stage_b = [&](int g, float2* dst) {
+    for (int k0 = 0; k0 < per_thread_b; k0 += kMaxB) {
+      uint16_t v[kMaxB];
+      load_b(g, v, k0);
+      store_b(v, k0, dst);
+    }
+  };
+  int g = blockIdx.x / cs;
+  if (kAcc && g < n_groups) stage_b(g, Bs0);
+  __syncthreads();
+  int local_count = 0;
+  bool nonfinite = false;
+  for (int it = 0; g < n_groups; g += n_clusters, ++it) {
+    const int64_t n0 = static_cast<int64_t>(g) * rb;
+    const int b = it & 1;
+    float2* Bs = Bs0 + b * static_cast<size_t>(r) * rb;
+
+    // this group's P and Wq: pulled from HBM into L2 now (no registers held),
+    // read from L2 after the FMA chain
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = n0 + trs * kRT + j;
+      if (col_ok && n < N) {
+        prefetch_l2(proxy + n * K + col);
+        if (kSel && (tcg & 3) == 0) prefetch_l2(wq + n * K + col);
+      }
+    }
+    // next group's dB_inc, also in flight during the FMA chain (first kMaxB per thread)
+    const int g_next = g + n_clusters;
+    uint16_t bnext[kMaxB];
+    if (kAcc && g_next < n_groups) load_b(g_next, bnext, 0);
+
+    float2 acc[kRT][2];
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) acc[j][0] = acc[j][1] = make_float2(0.0f, 0.0f);
+    if constexpr (kAcc) {
+      if (active) {
+        const uint16_t* arow = As + 4 * tcg;
+        const float2* brow = Bs + trs * kRT;
+#pragma unroll 4
+        for (int i = 0; i < r; ++i) {
+          const uint2 a2 = *reinterpret_cast<const uint2*>(arow);
+          const float2 a01 = make_float2(__uint_as_float(a2.x << 16), __uint_as_float(a2.x & 0xFFFF0000u));
+          const float2 a23 = make_float2(__uint_as_float(a2.y << 16), __uint_as_float(a2.y & 0xFFFF0000u));
+          float2 bb[kRT];
+#pragma unroll
+          for (int j = 0; j < kRT; j += 2) {
+            const float4 q = *reinterpret_cast<const float4*>(brow + j);
+            bb[j] = make_float2(q.x, q.y);
+            bb[j + 1] = make_float2(q.z, q.w);
+          }
+#pragma unroll
+          for (int j = 0; j < kRT; ++j) {
+            acc[j][0] = __ffma2_rn(bb[j], a01, acc[j][0]);
+            acc[j][1] = __ffma2_rn(bb[j], a23, acc[j][1]);
+          }
+          arow += wc;
+          brow += rb;
+        }
+      }
+    }
+
+    // next group's dB_inc into the other buffer (its readers finished a group ago)
+    if (kAcc && g_next < n_groups) {
+      float2* dst = Bs0 + (b ^ 1) * static_cast<size_t>(r) * rb;
+      store_b(bnext, 0, dst);
+      for (int k0 = kMaxB; k0 < per_thread_b; k0 += kMaxB) {
+        uint16_t v[kMaxB];
+        load_b(g_next, v, k0);
+        store_b(v, k0, dst);
+      }
+    }
+
+    float4 p[kRT];
+    uint32_t w[kRT];
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = n0 + trs * kRT + j;
+      if (col_ok && n < N) {
+        p[j] = *reinterpret_cast<const float4*>(proxy + n * K + col);
+        if (kSel) w[j] = *reinterpret_cast<const uint32_t*>(wq + n * K + col);
+      }
+    }
+
+    // P' = P + D, new codes, per-row change bits
+    uint32_t cnew[kRT];
+    uint32_t mymask = 0;
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = n0 + trs * kRT + j;
+      cnew[j] = 0;
+      if (col_ok && n < N) {
+        if constexpr (kAcc) {
+          p[j].x = __fadd_rn(p[j].x, acc[j][0].x);
+          p[j].y = __fadd_rn(p[j].y, acc[j][0].y);
+          p[j].z = __fadd_rn(p[j].z, acc[j][1].x);
+          p[j].w = __fadd_rn(p[j].w, acc[j][1].y);
+        }
+        nonfinite |= !(isfinite(p[j].x) && isfinite(p[j].y) && isfinite(p[j].z) && isfinite(p[j].w));
+        if constexpr (kSel) {
+          cnew[j] = requantized4(w[j], s_w, p[j]);
+          if (codes_changed4(w[j], cnew[j])) mymask |= 1u << (trs * kRT + j);
+        }
+      }
+    }
+
+    uint32_t rowsel = 0;
+    if constexpr (kSel) {
+      uint32_t* xb = xbuf + b;
+      const uint32_t m = __reduce_or_sync(0xFFFFFFFFu, mymask);
+      if ((tid & 31) == 0 && m) atomicOr(xb, m);
+      __syncthreads();  // this CTA's bits are complete in xb
+      uint32_t* box = inbox + 16 * b;
+      if (cs > 1) {
+        // all-gather of the row bits: push this CTA's word into every CTA's
+        // inbox (slot = own rank), each push counted on that CTA's mbarrier
+        if (tid == 0) {
+          mbar_arrive_expect_tx(&mbar[b], 4u * static_cast<uint32_t>(cs));
+          const uint32_t mine = *xb;
+          for (int q = 0; q < cs; ++q) st_async_u32(box + crank, &mbar[b], static_cast<uint32_t>(q), mine);
+        }
+        // phase of mbar[b] used by group `it` is (it >> 1) & 1; one warp polls,
+        // the others sleep in the barrier below instead of spinning
+        if (tid < 32) {
+          const bool ok = mbar_wait(&mbar[b], static_cast<uint32_t>((it >> 1) & 1), &abort_flag);
+          if (!__all_sync(0xFFFFFFFFu, ok) && tid == 0) {
+            abort_flag = 1;
+            if (dev_status) atomicOr(dev_status, kDevTimeout);
+          }
+        }
+        __syncthreads();
+        for (int q = 0; q < cs; ++q) rowsel |= box[q];
+      } else {
+        rowsel = *xb;
+      }
+    }
+    __syncthreads();  // everyone has rowsel; next Bs staged
+    if (kSel && tid == 0) xbuf[b] = 0u;  // reused two groups from now, after another barrier
+    if (abort_flag) break;
+
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = n0 + trs * kRT + j;
+      if (col_ok && n < N) {
+        const bool sel = kSel && ((rowsel >> (trs * kRT + j)) & 1u);
+        float4* pp = reinterpret_cast<float4*>(proxy + n * K + col);
+        if (sel) {
+          *reinterpret_cast<uint32_t*>(wq + n * K + col) = cnew[j];
+          *pp = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        } else if (kAcc) {
+          *pp = p[j];
+        }
+      }
+    }
+    if (kSel && crank == 0 && tid < rb && n0 + tid < N) {
+      const uint32_t sel = (rowsel >> tid) & 1u;
+      if (row_mask) row_mask[n0 + tid] = static_cast<uint8_t>(sel);
+      local_count += static_cast<int>(sel);
+    }
+  }
+  if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
+    atomicOr(dev_status, kDevNonfinite);
+  if (kSel && n_selected && local_count) atomicAdd(n_selected, local_count);
+  if (cs > 1) cluster_sync_all();  // no CTA leaves while a peer may still push into it
+}
+
+// Picks the cluster split of K; returns false when A's slice does not fit.
+bool plan_proxy(int64_t K, int64_t r, ProxyGeom* geo) {
+  // about 512 columns per CTA; clusters of up to 8 (portable) or 16 CTAs
+  int cs = static_cast<int>((K + 511) / 512);
+  if (cs < 1) cs = 1;
+  if (cs > 8) cs = 16;
+  int wc = static_cast<int>((K + cs - 1) / cs);
+  wc = (wc + 7) / 8 * 8;
+  const int cg = wc / 4;
+  if (cg > 256) return false;
+  int rs = 256 / cg;
+  if (rs > 4) rs = 4;
+  if (rs < 1) rs = 1;
+  const int rb = kRT * rs;  // <= 32 rows: one bit each in a 32-bit mask
+  const int threads = (cg * rs + 31) / 32 * 32;
+  const size_t smem = align_up(static_cast<size_t>(r) * wc * 2, 16) +
+                      2 * static_cast<size_t>(r) * rb * sizeof(float2) + 16 + 8 + 128;
+  if (smem > 200 * 1024) return false;
+  *geo = ProxyGeom{cs, wc, cg, rs, rb, threads, smem};
+  return true;
+}
+
+template <bool kAcc, bool kSel>
+cudaError_t launch_proxy_cluster(const ProxyGeom& geo, uint8_t* wq, const float* s_w, float* proxy,
+                                 const void* dB_inc, const void* A, int64_t N, int64_t K, int r,
+                                 uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
+                                 cudaStream_t stream) {
+  auto kern = proxy_cluster_kernel<kAcc, kSel>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(geo.smem));
+  if (e != cudaSuccess) return e;
+  if (geo.cs > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = geo.cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(geo.threads);
+  cfg.dynamicSmemBytes = geo.smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int max_clusters = 0;
+  cfg.gridDim = dim3(geo.cs);
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+  const int n_groups = static_cast<int>((N + geo.rb - 1) / geo.rb);
+  int clusters = max_clusters < n_groups ? max_clusters : n_groups;
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * geo.cs));
+  return cudaLaunchKernelEx(&cfg, kern, wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc),
+                            static_cast<const uint16_t*>(A), N, K, r, geo, n_groups, row_mask,
+                            n_selected, dev_status);
+}
+
 }  // namespace
 
 size_t proxy_workspace_bytes(int64_t N, int64_t K) {
@@ -204,6 +588,31 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
                                 const void* A, int64_t N, int64_t K, int64_t r, uint32_t flags,
                                 uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
                                 void* workspace, cudaStream_t stream) {
+  const DeviceInfo* di0 = current_device_info();
+  if (!di0) return cudaErrorInvalidDevice;
+  ProxyGeom geo;
+  const bool acc0 = flags & 1u, sel0 = flags & 2u;
+  if (r <= 1024 && plan_proxy(K, acc0 ? r : 0, &geo)) {
+    if (sel0 && n_selected) {
+      cudaError_t e0 = cudaMemsetAsync(n_selected, 0, sizeof(int32_t), stream);
+      if (e0 != cudaSuccess) return e0;
+    }
+    const int rr = acc0 ? static_cast<int>(r) : 0;
+    cudaError_t e1;
+    if (acc0 && sel0)
+      e1 = launch_proxy_cluster<true, true>(geo, wq, s_w, proxy, dB_inc, A, N, K, rr, row_mask,
+                                            n_selected, dev_status, stream);
+    else if (acc0)
+      e1 = launch_proxy_cluster<true, false>(geo, wq, s_w, proxy, dB_inc, A, N, K, rr, row_mask,
+                                             n_selected, dev_status, stream);
+    else
+      e1 = launch_proxy_cluster<false, true>(geo, wq, s_w, proxy, dB_inc, A, N, K, rr, row_mask,
+                                             n_selected, dev_status, stream);
+    if (e1 == cudaSuccess) return cudaSuccess;
+    if (e1 != cudaErrorInvalidConfiguration) return e1;
+    (void)cudaGetLastError();  // no cluster fits: fall through to the two-kernel path
+  }
+
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   const bool acc = flags & 1u, sel = flags & 2u;

@@ -51,34 +51,44 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const void* __re
   __shared__ uint32_t red[32];
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // kUnroll independent 16-byte loads in flight per thread per iteration
+  constexpr int kUnroll = 4;
+  const uint32_t mask = kBF16 ? 0x7FFF7FFFu : 0x7FFFFFFFu;
   uint32_t m = 0;
-  if constexpr (kBF16) {
-    const uint4* v = reinterpret_cast<const uint4*>(x);
-    const int64_t nv = n / 8;
-    for (int64_t i = tid; i < nv; i += stride) {
-      const uint4 q = v[i];
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  const uint4* v = reinterpret_cast<const uint4*>(x);
+  const int64_t nv = n / (kBF16 ? 8 : 4);
+  const int64_t chunk = stride * kUnroll;
+  int64_t i = tid;
+  for (; i + (kUnroll - 1) * stride < nv; i += chunk) {
+    uint4 q[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) q[u] = __ldg(v + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t w[4] = {q[u].x & mask, q[u].y & mask, q[u].z & mask, q[u].w & mask};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        m = max(m, w[j] & 0x7FFFu);
-        m = max(m, (w[j] >> 16) & 0x7FFFu);
+        if constexpr (kBF16) m = max(m, max(w[j] & 0xFFFFu, w[j] >> 16));
+        else m = max(m, w[j]);
       }
     }
-    const uint16_t* s = reinterpret_cast<const uint16_t*>(x);
-    for (int64_t i = nv * 8 + tid; i < n; i += stride) m = max(m, s[i] & 0x7FFFu);
+  }
+  for (; i < nv; i += stride) {
+    const uint4 q = __ldg(v + i);
+    const uint32_t w[4] = {q.x & mask, q.y & mask, q.z & mask, q.w & mask};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if constexpr (kBF16) m = max(m, max(w[j] & 0xFFFFu, w[j] >> 16));
+      else m = max(m, w[j]);
+    }
+  }
+  if constexpr (kBF16) {
+    const uint16_t* s16 = reinterpret_cast<const uint16_t*>(x);
+    for (int64_t e = nv * 8 + tid; e < n; e += stride) m = max(m, s16[e] & 0x7FFFu);
     m <<= 16;  // bfloat16 magnitude bits -> float32 bits
   } else {
-    const uint4* v = reinterpret_cast<const uint4*>(x);
-    const int64_t nv = n / 4;
-    for (int64_t i = tid; i < nv; i += stride) {
-      const uint4 q = v[i];
-      m = max(m, q.x & 0x7FFFFFFFu);
-      m = max(m, q.y & 0x7FFFFFFFu);
-      m = max(m, q.z & 0x7FFFFFFFu);
-      m = max(m, q.w & 0x7FFFFFFFu);
-    }
-    const uint32_t* s = reinterpret_cast<const uint32_t*>(x);
-    for (int64_t i = nv * 4 + tid; i < n; i += stride) m = max(m, s[i] & 0x7FFFFFFFu);
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(x);
+    for (int64_t e = nv * 4 + tid; e < n; e += stride) m = max(m, s32[e] & 0x7FFFFFFFu);
   }
   m = block_max_u32(m, red);
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
@@ -171,14 +181,12 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   const float s = s_shared;
-  const double inv_s_num = static_cast<double>(s);
+  const double s_d = static_cast<double>(s);
 
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t ng = n / 16;
-  for (int64_t g = tid; g < ng; g += stride) {
-    float v[16];
-    load16<kBF16>(x, g, v);
+  auto convert = [&](int64_t g, const float (&v)[16]) {
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -193,14 +201,27 @@ __global__ void __launch_bounds__(kThreads)
       for (int j = 0; j < 8; ++j) {
         const float2 d = e4m3x2_value(w[j >> 1] >> (16 * (j & 1)));
         r[2 * j] = static_cast<float>(static_cast<double>(v[2 * j]) -
-                                      static_cast<double>(d.x) / inv_s_num);
+                                      static_cast<double>(d.x) / s_d);
         r[2 * j + 1] = static_cast<float>(static_cast<double>(v[2 * j + 1]) -
-                                          static_cast<double>(d.y) / inv_s_num);
+                                          static_cast<double>(d.y) / s_d);
       }
       float4* rp = reinterpret_cast<float4*>(residual) + 4 * g;
 #pragma unroll
       for (int j = 0; j < 4; ++j) rp[j] = make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
     }
+  };
+  int64_t g = tid;
+  for (; g + stride < ng; g += 2 * stride) {  // two groups in flight per thread
+    float va[16], vb[16];
+    load16<kBF16>(x, g, va);
+    load16<kBF16>(x, g + stride, vb);
+    convert(g, va);
+    convert(g + stride, vb);
+  }
+  for (; g < ng; g += stride) {
+    float va[16];
+    load16<kBF16>(x, g, va);
+    convert(g, va);
   }
   for (int64_t i = ng * 16 + tid; i < n; i += stride) {  // tail (n % 16 != 0)
     const float v = load1<kBF16>(x, i);
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(kThreads)
     codes[i] = static_cast<uint8_t>(c);
     if (residual) {
       const float2 d = e4m3x2_value(c);
-      residual[i] = static_cast<float>(static_cast<double>(v) - static_cast<double>(d.x) / inv_s_num);
+      residual[i] = static_cast<float>(static_cast<double>(v) - static_cast<double>(d.x) / s_d);
     }
   }
 }

@@ -48,6 +48,8 @@ CASES = [
     (512, 256, 384, 80),    # r not a power of two (128-wide tile, 48 padded columns)
     (256, 384, 256, 256),
     (128, 256, 512, 320),   # two r tiles
+    (2048, 256, 4096, 16),  # 16 row tiles: split-K clusters of 8
+    (1000, 4096, 1024, 64), # many dB/dA^T tiles, few splits
 ]
 
 

@@ -47,8 +47,16 @@ def _compare(gpu, ref):
     assert st == 0
 
 
-@pytest.mark.parametrize("N,K,r", [(512, 512, 16), (37, 48, 5), (64, 272, 33), (130, 512, 64),
-                                   (96, 1024, 100), (40, 11008, 16)])
+@pytest.mark.parametrize("N,K,r", [
+    (512, 512, 16),     # one-CTA clusters
+    (37, 48, 5),        # tiny, ragged rows
+    (64, 272, 33),      # r across the 32-wide staging chunk of the two-kernel path
+    (130, 512, 64),
+    (96, 1024, 100),    # clusters of 2
+    (70, 2048, 64),     # clusters of 4, rows not a multiple of the row group
+    (40, 11008, 16),    # clusters of 16 (the down projection's K)
+    (64, 512, 1100),    # rank beyond the single-pass kernel: two-kernel path
+])
 def test_accumulate_and_select(cuda_device, N, K, r):
     O.set_threads(os.cpu_count() or 8)
     case = _state(N + K + r, N, K, r)
