@@ -171,7 +171,9 @@ class Step:
         # initial quantization of the backbone (not part of the step)
         F.falqon_quantize(self.W, codes=self.wq, scale=self.s_w, amax=self.amax,
                           dev_status=self.status, workspace=self.ws_q2)
-        self.launches_per_step = 2 + 1 + 2 + 8 + 1 + 2  # library kernels per step
+        # library kernels per step: quantize X (2) + forward (1) + quantize dY (2)
+        # + adapter products T, dB, U, dA (4) + dX (1) + proxy stream and clear (2)
+        self.launches_per_step = 2 + 1 + 2 + 4 + 1 + 2
 
     PHASES = ("quantX+fwd", "quantdY+adapters", "dX", "sgd", "proxy")
 

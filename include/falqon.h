@@ -156,8 +156,11 @@ FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy
  *               dB_inc[n,i] * A[i,k], starting at +0; P = fl32(P + D).
  *   SELECT:     t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ), c' = E4M3(t);
  *               row n is selected iff some c' differs in value from Wq[n,k]
- *               (+0 equals -0).  Selected rows: Wq[n,:] = c'[n,:] verbatim
- *               and P[n,:] = +0.  Other rows: Wq bit-identical, P kept.
+ *               (+0 equals -0).  Selected rows: every code whose value
+ *               changes becomes c'[n,k], codes of unchanged value keep their
+ *               bits (so a zero keeps its sign), and P[n,:] = +0.  Other
+ *               rows: Wq bit-identical, P kept.  The decoded backbone is the
+ *               same as with a verbatim rewrite of the row.
  * The float32 chain is reproduced bit-for-bit (no tensor cores).
  *
  *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);

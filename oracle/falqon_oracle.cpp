@@ -73,9 +73,15 @@
 //       equals nothing).  s_W is the fixed scale of the initial
 //       quantization.  The pages' own rule is a top-k over rows ([R3-Q1],
 //       [R2-W7]) with k not given; the threshold rule here is the contract.
-//  C-11 Requantize and clear.  Selected rows: Wq[n,:] = c'[n,:] for all k
-//       (verbatim, sign of zero included), P[n,:] = +0.  Rows not selected:
-//       Wq untouched (bit-identical), P keeps the accumulated value.
+//  C-11 Requantize and clear.  For mask[n] = 1: every code of the row whose
+//       value changes is replaced, Wq[n,k] = c'[n,k] where dec(c') != dec(Wq);
+//       codes whose value is unchanged keep their bit pattern (the only such
+//       case with different bits is a zero whose sign would flip); and
+//       P[n,:] = +0 ("clears their share of the proxy").  For mask[n] = 0: Wq
+//       untouched (bit-identical; no code of the row changes value by
+//       definition), P keeps the accumulated value.  The pages say nothing
+//       about the sign of zero; keeping equal-valued codes as they are makes
+//       the decoded backbone identical to a verbatim rewrite.
 //
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
@@ -369,7 +375,8 @@ void fo_proxy_select(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, uin
         const float w = static_cast<float>(dec(wq[n * K + k]));
         const float upd = s_w * P[n * K + k];
         const float t = w + upd;
-        wq[n * K + k] = enc(t);
+        const uint8_t c_new = enc(t);
+        if (!(dec(c_new) == dec(wq[n * K + k]))) wq[n * K + k] = c_new;
         P[n * K + k] = 0.0f;
       }
     }

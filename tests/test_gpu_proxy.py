@@ -48,14 +48,14 @@ def _compare(gpu, ref):
 
 
 @pytest.mark.parametrize("N,K,r", [
-    (512, 512, 16),     # one-CTA clusters
+    (512, 512, 16),     # one 256-column block per row group
     (37, 48, 5),        # tiny, ragged rows
-    (64, 272, 33),      # r across the 32-wide staging chunk of the two-kernel path
+    (64, 272, 33),      # odd r; K ends in a partial 256-column block
     (130, 512, 64),
-    (96, 1024, 100),    # clusters of 2
-    (70, 2048, 64),     # clusters of 4, rows not a multiple of the row group
-    (40, 11008, 16),    # clusters of 16 (the down projection's K)
-    (64, 512, 1100),    # rank beyond the single-pass kernel: two-kernel path
+    (96, 1024, 100),    # r beyond one 64-wide staging chunk
+    (70, 2048, 64),     # rows not a multiple of the 32-row group
+    (40, 11008, 16),    # the down projection's K (43 column blocks)
+    (64, 512, 1100),    # large rank: many staging chunks
 ])
 def test_accumulate_and_select(cuda_device, N, K, r):
     O.set_threads(os.cpu_count() or 8)

@@ -111,10 +111,27 @@ def test_select_matches_brute_force_restatement():
     sel = changed.any(axis=1)
     assert 0 < sel.sum() < len(sel), "data should select some rows but not all"
     assert np.array_equal(mask.astype(bool), sel) and cnt == sel.sum()
-    assert np.array_equal(wq2[sel], cn[sel])
+    # selected rows: value-changing codes replaced, equal-valued codes kept as they were
+    expect = np.where(changed, cn, wq)
+    assert np.array_equal(wq2[sel], expect[sel])
     assert np.array_equal(wq2[~sel], wq[~sel])
     assert np.all(P2[sel].view(np.uint32) == 0)
     assert np.array_equal(P2[~sel].view(np.uint32), P[~sel].view(np.uint32))
+
+
+def test_selected_row_keeps_zero_sign_of_unchanged_codes():
+    wq, s_w, P, _, _ = _state(9)
+    P[:] = 0
+    wq[3, :] = 0x80                       # -0 codes ...
+    wq[3, 5] = 0x30                       # ... and one 0.5 that an update moves
+    P[3, :] = np.float32(1e-30)           # -0 + tiny -> +0: same value, other bits
+    step = (DEC[0x31] - DEC[0x30]) / np.float64(s_w)
+    P[3, 5] = np.float32(step)
+    wq2, P2, mask, cnt = O.proxy_select(wq, s_w, P)
+    assert cnt == 1 and mask[3] == 1
+    assert wq2[3, 5] == 0x31
+    assert np.all(np.delete(wq2[3], 5) == 0x80)  # -0 kept although t rounds to +0
+    assert np.all(P2[3] == 0)
 
 
 def test_unselected_rows_bit_identical_and_negative_zero_not_a_change():
