@@ -58,7 +58,7 @@ struct GemmArgs {
 };
 
 template <bool kF8, bool kAMn, bool kBMn, bool kAConv, int kBN, int kStages, bool kClusterK,
-          bool kBSplit = false, int kRawStages = 0>
+          bool kBSplit = false, int kRawStages = 0, int kBStages = kStages>
 struct Cfg {
   static constexpr bool F8 = kF8;
   static constexpr bool AMn = kAMn;
@@ -77,8 +77,13 @@ struct Cfg {
   static constexpr int ABytes = kBM * BK * ElemBytes;     // operand A tile (16 KB)
   static constexpr int BBytes = kBN * BK * ElemBytes;     // operand B tile
   static constexpr int B2Bytes = kBSplit ? BBytes : 0;   // low half of a split B operand
-  static constexpr int StageBytes = ABytes + BBytes + B2Bytes;
-  static constexpr int TmaBytes = (kAConv ? 0 : ABytes) + BBytes + B2Bytes;
+  // TMA ring (B, plus A when A comes by TMA) and, with expansion, a separate
+  // ring of expanded A tiles so that B loads run ahead independently
+  static constexpr int BStages = kAConv ? kBStages : kStages;
+  static constexpr int BSlotBytes = (kAConv ? 0 : ABytes) + BBytes + B2Bytes;
+  static constexpr int ARingBytes = kAConv ? kStages * ABytes : 0;
+  static constexpr int BRingBytes = BStages * BSlotBytes;
+  static constexpr int TmaBytes = BSlotBytes;
   static constexpr int NumConvWarps = kAConv ? 8 : 0;
   // per-converter-thread ring of raw E4M3 codes (32 bytes per thread per k-block),
   // filled with cp.async kRawStages k-blocks ahead
@@ -87,10 +92,10 @@ struct Cfg {
   static_assert(!kAConv || kRawStages >= 2, "raw ring depth");
   static constexpr int Threads = 32 * (6 + NumConvWarps);
   static constexpr uint32_t TmemCols = 2 * kBN < 32 ? 32 : 2 * kBN;
-  static constexpr int BarBytes = 8 * (3 * kStages + 5) + 16;
-  static constexpr int SmemBytes = kStages * StageBytes + RawStages * RawSlotBytes + BarBytes + 1024;
-  static constexpr int RedStride = kBN + 1;  // fp32 words per row of the reduction tile
-  static_assert(!kClusterK || kBM * RedStride * 4 <= kStages * StageBytes, "reduction tile");
+  static constexpr int BarBytes = 8 * (2 * kStages + 2 * BStages + 5) + 16;
+  static constexpr int SmemBytes = ARingBytes + BRingBytes + RawStages * RawSlotBytes + BarBytes + 1024;
+  static constexpr int RedStride = kBN + 4;  // fp32 words per row of the reduction tile (16-byte rows)
+  static_assert(!kClusterK || kBM * RedStride * 4 <= ARingBytes + BRingBytes, "reduction tile");
   static constexpr uint32_t IDesc =
       idesc_f32acc(kF8 ? 0u : 1u, kF8 ? 0u : 1u, kAMn ? 1u : 0u, kBMn ? 1u : 0u, kBM, kBN);
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
@@ -109,6 +114,48 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int ks) {
     // k-step = 32 bytes along the swizzled 128-byte row
     return sdesc_sw128(base + ks * 32, 16, 1024);
   }
+}
+
+// Two E4M3 codes, in bytes 0 and 2 of x (bytes 1 and 3 zero), to a bf16x2
+// word, exactly.  Shifted left by 4, a code's exponent and mantissa fields
+// land on the bf16 exponent and the top of the bf16 mantissa, so the word
+// reads as the code's value times 2^-120 (E4M3 bias 7 against bf16 bias 127;
+// E4M3 subnormals land on bf16 subnormals, which scale the same way).  The
+// sign, left at bit 11, moves to bit 15 by adding 15 * 2^11 (= 2^15 - 2^11),
+// and one bf16 multiply by 2^120 (plus -0) restores the value with no
+// rounding.  NaN codes (0x7F, 0xFF) are not handled here.
+__device__ __forceinline__ uint32_t e4m3_pair_to_bf16x2(uint32_t x) {
+  uint32_t h = x << 4;
+  h += 15u * (h & 0x08000800u);
+  uint32_t out;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out) : "r"(h), "r"(0x7B807B80u), "r"(0x80008000u));
+  return out;
+}
+
+// Nonzero iff one of the 16 codes is a NaN code (magnitude bits all ones).
+__device__ __forceinline__ uint32_t has_nan_code(uint4 q) {
+  const uint32_t m = 0x7F7F7F7Fu, one = 0x01010101u;
+  return (((q.x & m) + one) | ((q.y & m) + one) | ((q.z & m) + one) | ((q.w & m) + one)) &
+         0x80808080u;
+}
+
+// Four codes -> four bf16 (two words) through the hardware conversion; exact
+// for every code, NaN included.
+__device__ __forceinline__ void e4m3x4_to_bf16_hw(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t o[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint16_t pair = static_cast<uint16_t>(w >> (16 * j));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    __half2 hh;
+    memcpy(&hh, &h2, 4);
+    const float2 f = __half22float2(hh);
+    const __nv_bfloat162 bb = __floats2bfloat162_rn(f.x, f.y);
+    memcpy(&o[j], &bb, 4);
+  }
+  lo = o[0];
+  hi = o[1];
 }
 
 // 16-byte global -> shared copy, zero-filled when src_bytes == 0.
@@ -143,9 +190,12 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* local, int rank) {
   return remote;
 }
 
-__device__ __forceinline__ float dsmem_load_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 dsmem_load_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
   return v;
 }
 
@@ -167,12 +217,15 @@ __global__ void __launch_bounds__(C::Threads, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* raw_ring = smem + C::Stages * C::StageBytes;  // converters only
+  uint8_t* a_ring = smem;                                // expanded A tiles (expansion only)
+  uint8_t* b_ring = smem + C::ARingBytes;                // TMA-fed tiles
+  uint8_t* raw_ring = b_ring + C::BRingBytes;            // converters' raw codes
   uint64_t* bars = reinterpret_cast<uint64_t*>(raw_ring + C::RawStages * C::RawSlotBytes);
-  uint64_t* full = bars;                      // TMA landed
-  uint64_t* conv = bars + C::Stages;          // codes expanded (bf16 kinds)
-  uint64_t* empty = bars + 2 * C::Stages;     // MMAs done reading the stage
-  uint64_t* acc_full = bars + 3 * C::Stages;  // [2] accumulator ready
+  uint64_t* full = bars;                                 // [BStages] TMA landed
+  uint64_t* empty = full + C::BStages;                   // [BStages] MMAs done with the TMA slot
+  uint64_t* conv = empty + C::BStages;                   // [Stages] codes expanded
+  uint64_t* aempty = conv + C::Stages;                   // [Stages] MMAs done with the A slot
+  uint64_t* acc_full = aempty + C::Stages;               // [2] accumulator ready
   uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained
   uint64_t* drain = acc_empty + 2;            // all issued MMAs retired (teardown)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -183,10 +236,13 @@ __global__ void __launch_bounds__(C::Threads, 1)
   const int total = g.m_tiles * g.n_tiles * g.splits;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::Stages; ++s) {
+    for (int s = 0; s < C::BStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], C::NumConvWarps > 0 ? C::NumConvWarps : 1);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::Stages; ++s) {
+      mbar_init(&conv[s], C::NumConvWarps > 0 ? C::NumConvWarps : 1);
+      mbar_init(&aempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -229,8 +285,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
         const int m0 = mt * kBM, n0 = nt * C::BN;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { fail(); ok = false; break; }
-          uint8_t* sA = smem + stage * C::StageBytes;
-          uint8_t* sB = sA + C::ABytes;
+          uint8_t* sA = b_ring + stage * C::BSlotBytes;  // A by TMA only when not expanded
+          uint8_t* sB = sA + (C::AConv ? 0 : C::ABytes);
           uint8_t* sB2 = sB + C::BBytes;
           mbar_arrive_expect_tx(&full[stage], C::TmaBytes);
           issued |= 1u << stage;
@@ -260,18 +316,18 @@ __global__ void __launch_bounds__(C::Threads, 1)
             tma_load_2d(sB, &tmB, &full[stage], kb * C::BK, n0);
             if constexpr (C::BSplit) tma_load_2d(sB2, &tmB2, &full[stage], kb * C::BK, n0);
           }
-          if (++stage == C::Stages) { stage = 0; phase ^= 1; }
+          if (++stage == C::BStages) { stage = 0; phase ^= 1; }
         }
       }
       // every load this lane issued must land before the CTA exits (matters
       // only after an abort; otherwise the MMA warp already consumed them)
-      for (int s = 0; s < C::Stages; ++s)
+      for (int s = 0; s < C::BStages; ++s)
         if (issued & (1u << s)) mbar_wait_budget(&full[s], (issued_parity >> s) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, astage = 0;
+    uint32_t phase = 0, aphase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -283,14 +339,15 @@ __global__ void __launch_bounds__(C::Threads, 1)
       tc_fence_after();
       const uint32_t tmem_d = tmem_base + acc * C::BN;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!warp_wait(&full[stage], phase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
         if constexpr (C::AConv) {
-          if (!warp_wait(&conv[stage], phase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+          if (!warp_wait(&conv[astage], aphase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
         }
+        if (!warp_wait(&full[stage], phase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a_base = smem_u32(smem + stage * C::StageBytes);
-          const uint32_t b_base = a_base + C::ABytes;
+          const uint32_t slot = smem_u32(b_ring + stage * C::BSlotBytes);
+          const uint32_t a_base = C::AConv ? smem_u32(a_ring + astage * C::ABytes) : slot;
+          const uint32_t b_base = slot + (C::AConv ? 0 : C::ABytes);
 #pragma unroll
           for (int ks = 0; ks < C::KSteps; ++ks) {
             const uint64_t ad = operand_desc<C::AMn, C::ElemBytes, C::BK>(a_base, ks);
@@ -304,9 +361,13 @@ __global__ void __launch_bounds__(C::Threads, 1)
             }
           }
           umma_commit(&empty[stage]);
+          if constexpr (C::AConv) umma_commit(&aempty[astage]);
         }
         __syncwarp();
-        if (++stage == C::Stages) { stage = 0; phase ^= 1; }
+        if (++stage == C::BStages) { stage = 0; phase ^= 1; }
+        if constexpr (C::AConv) {
+          if (++astage == C::Stages) { astage = 0; aphase ^= 1; }
+        }
       }
       if (!ok) break;
       if (lane == 0) umma_commit(&acc_full[acc]);
@@ -348,11 +409,13 @@ __global__ void __launch_bounds__(C::Threads, 1)
         const int64_t col0 = col_base + c * 32;
         (void)col0;
         if constexpr (C::ClusterK) {
-          // this CTA's fp32 tile, reusing the (drained) stage buffers; the +1 row
-          // stride keeps the 32 lanes (32 rows) on distinct banks
-          float* red = reinterpret_cast<float*>(smem) + (q * 32 + lane) * C::RedStride + c * 32;
+          // this CTA's fp32 tile, reusing the (drained) stage buffers
+          float4* red = reinterpret_cast<float4*>(reinterpret_cast<float*>(smem) +
+                                                  (q * 32 + lane) * C::RedStride + c * 32);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) red[j] = __uint_as_float(r[j]);
+          for (int j = 0; j < 8; ++j)
+            red[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
         } else {
           if (row < g.M) {
             __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
@@ -423,34 +486,31 @@ __global__ void __launch_bounds__(C::Threads, 1)
       int slot = 0;
       for (int kb = kb0; kb < kb1; ++kb) {
         cp_async_wait<R - 1>();  // this thread's chunks of k-block kb have landed
-        if (!warp_wait(&empty[stage], phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+        if (!warp_wait(&aempty[stage], phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
         const uint4 q0 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes);
         const uint4 q1 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes + 16);
-        uint8_t* sA = smem + stage * C::StageBytes;
+        uint8_t* sA = a_ring + stage * C::ABytes;
         // 32 codes -> 32 bf16 (four 16-byte units of the 128-byte-swizzled layout)
+        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint32_t o[16];
+        if (!(has_nan_code(q0) | has_nan_code(q1))) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            o[2 * j] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4140));
+            o[2 * j + 1] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4342));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) e4m3x4_to_bf16_hw(words[j], o[2 * j], o[2 * j + 1]);
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t w0 = (u & 2) ? ((u & 1) ? q1.z : q1.x) : ((u & 1) ? q0.z : q0.x);
-          const uint32_t w1 = (u & 2) ? ((u & 1) ? q1.w : q1.y) : ((u & 1) ? q0.w : q0.y);
-          uint32_t o[4];
-          const uint32_t wv[2] = {w0, w1};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint16_t pair = static_cast<uint16_t>(wv[j >> 1] >> (16 * (j & 1)));
-            uint32_t h2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
-            __half2 hh;
-            memcpy(&hh, &h2, 4);
-            const float2 f = __half22float2(hh);
-            const __nv_bfloat162 bb = __floats2bfloat162_rn(f.x, f.y);
-            memcpy(&o[j], &bb, 4);
-          }
           const int col = tcol + 8 * u;
           const int blk = col / 64;
           const int unit = (col % 64) / 8;
           uint8_t* dst = sA + blk * (kTileRows * kRowBytes) + trow * kRowBytes +
                          ((unit ^ (trow & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -487,23 +547,45 @@ __global__ void __launch_bounds__(C::Threads, 1)
     if (g.scale_b) den *= static_cast<double>(*g.scale_b);
     const float alpha = static_cast<float>(1.0 / den);
     const int nrows = q1 - q0;
-    const int nelem = nrows > 0 ? nrows * C::BN : 0;
-    for (int e = threadIdx.x; e < nelem; e += blockDim.x) {
-      int lr, lc;
-      if (g.transpose) { lr = q0 + e % nrows; lc = e / nrows; }  // walk rows: coalesced out[col][row]
-      else { lr = q0 + e / C::BN; lc = e % C::BN; }
-      const uint32_t off = static_cast<uint32_t>((lr * C::RedStride + lc) * 4);
-      float acc = 0.0f;
-      for (int sidx = 0; sidx < S; ++sidx) acc += dsmem_load_f32(peer[sidx] + off);
+    constexpr int G = C::BN / 4;  // float4 groups per row
+    const int ngroups = nrows > 0 ? nrows * G : 0;
+    for (int e = threadIdx.x; e < ngroups; e += blockDim.x) {
+      int lr, lg;
+      if (g.transpose) { lr = q0 + e % nrows; lg = e / nrows; }  // walk rows: coalesced out[col][row]
+      else { lr = q0 + e / G; lg = e % G; }
+      const uint32_t off = static_cast<uint32_t>((lr * C::RedStride + 4 * lg) * 4);
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int sidx = 0; sidx < S; ++sidx) {  // fixed order: rank 0, 1, ...
+        const float4 v = dsmem_load_f32x4(peer[sidx] + off);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
       const int64_t grow = static_cast<int64_t>(mt) * kBM + lr;
-      const int64_t gcol = static_cast<int64_t>(nt) * C::BN + lc;
-      if (grow < g.M && gcol < g.N) {
-        const float v = acc * alpha;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        const int64_t idx = g.transpose ? gcol * g.ldo + grow : grow * g.ldo + gcol;
-        static_cast<__nv_bfloat16*>(g.out)[idx] = hi;
-        if (g.out_lo)
-          static_cast<__nv_bfloat16*>(g.out_lo)[idx] = __float2bfloat16_rn(v - __bfloat162float(hi));
+      const int64_t gcol0 = static_cast<int64_t>(nt) * C::BN + 4 * lg;
+      if (grow >= g.M || gcol0 >= g.N) continue;  // N % 16 == 0: groups of 4 in or out
+      const float vals[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
+      __nv_bfloat16 hi[4], lo[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        hi[k] = __float2bfloat16_rn(vals[k]);
+        lo[k] = __float2bfloat16_rn(vals[k] - __bfloat162float(hi[k]));
+      }
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
+      __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(g.out_lo);
+      if (g.transpose) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          out[(gcol0 + k) * g.ldo + grow] = hi[k];
+          if (out_lo) out_lo[(gcol0 + k) * g.ldo + grow] = lo[k];
+        }
+      } else {
+        uint2 ph, pl;
+        memcpy(&ph, hi, 8);
+        memcpy(&pl, lo, 8);
+        *reinterpret_cast<uint2*>(out + grow * g.ldo + gcol0) = ph;
+        if (out_lo) *reinterpret_cast<uint2*>(out_lo + grow * g.ldo + gcol0) = pl;
       }
     }
     cluster_sync_all();  // no CTA leaves while a peer still reads its tile
@@ -558,31 +640,18 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 
 using FwdCfg = Cfg<true, false, false, false, 256, 4, false>;
 using DxCfg = Cfg<true, false, true, false, 256, 4, false>;
-using FwdCfg128 = Cfg<true, false, false, false, 128, 6, false>;
-using DxCfg128 = Cfg<true, false, true, false, 128, 6, false>;
 
-// Tile width for an FP8 GEMM with an M x Ncols output: 128x256 tiles unless
-// 128x128 tiles fill the last wave of persistent CTAs much better (128-wide
-// tiles move 1/3 more operand bytes per flop, weighed as a 5% cost).
-int fp8_tile_n(int64_t M, int64_t Ncols, int sms) {
-  auto wave_eff = [&](int bn) {
-    const int64_t tiles = ((M + kBM - 1) / kBM) * ((Ncols + bn - 1) / bn);
-    const int64_t waves = (tiles + sms - 1) / sms;
-    return static_cast<double>(tiles) / static_cast<double>(waves * sms);
-  };
-  (void)wave_eff;
-  // Measured on B200: 128x128 tiles need 128 B/clk/SM of operand traffic and
-  // run L2-bound (dX 4096^3: 87 us vs 59 us with 128x256), so 256 is kept.
-  return 256;
-}
-
+// <A stages, raw stages, B stages> sized to ~200 KB of shared memory
 template <int BN> using TCfg = Cfg<false, false, false, true, BN, (BN >= 256 ? 3 : 4), true, false,
-                                   (BN >= 128 ? 8 : 12)>;  // Xq . A^T
+                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8)),
+                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8))>;  // Xq . A^T
 template <int BN> using UCfg = Cfg<false, false, true, true, BN, (BN >= 256 ? 3 : 4), true, false,
-                                   (BN >= 128 ? 8 : 12)>;  // dYq . B
+                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8)),
+                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8))>;  // dYq . B
 // dYq^T . (T_hi + T_lo), Xq^T . (U_hi + U_lo): fewer stages at BN = 256 to fit smem
 template <int BN> using MnCfg = Cfg<false, true, true, true, BN, (BN >= 256 ? 2 : (BN >= 128 ? 3 : 4)), true, true,
-                                    (BN >= 256 ? 6 : (BN >= 128 ? 8 : 10))>;
+                                    (BN >= 256 ? 4 : (BN >= 128 ? 4 : 6)),
+                                    (BN >= 256 ? 2 : (BN >= 128 ? 4 : 6))>;
 
 // Split count: as many K splits as fit beside the tiles in one wave, at most 8
 // (the portable cluster size), never more than there are K blocks.
@@ -662,10 +731,6 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
 cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
                                 const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
                                 int32_t* dev_status, cudaStream_t stream) {
-  const DeviceInfo* di = current_device_info();
-  if (!di) return cudaErrorInvalidDevice;
-  if (fp8_tile_n(M, N, di->sm_count) == 128)
-    return fp8_gemm<FwdCfg128>(xq, s_x, wq, s_w, M, N, K, false, y, dev_status, stream);
   return fp8_gemm<FwdCfg>(xq, s_x, wq, s_w, M, N, K, false, y, dev_status, stream);
 }
 
@@ -673,10 +738,6 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
                                int32_t* dev_status, cudaStream_t stream) {
   // contraction over N: A = dYq [M, N] K-major; B = Wq [N, K] read MN-major (K contiguous)
-  const DeviceInfo* di = current_device_info();
-  if (!di) return cudaErrorInvalidDevice;
-  if (fp8_tile_n(M, K, di->sm_count) == 128)
-    return fp8_gemm<DxCfg128>(dyq, s_dy, wq, s_w, M, K, N, true, dx, dev_status, stream);
   return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, true, dx, dev_status, stream);
 }
 

@@ -9,7 +9,15 @@
 // other rows keep their codes bit-for-bit and their accumulated proxy.
 //
 // Two kernels, no cross-CTA synchronisation:
-//   proxy_stream_kernel  (grid over 32 x 256 tiles of P; two CTAs per SM)
+//   proxy_pipe_kernel  (persistent, one CTA per SM; r <= 64 and r % 8 == 0)
+//     Each CTA walks a contiguous range of 32 x 256 tiles of P, column block
+//     by column block, so the block's A columns stay in shared memory.  Every
+//     thread streams its own P and Wq slices, and the tile's dB_inc rows, two
+//     tiles ahead with cp.async (three slots), while it computes the current
+//     tile; A for the next column block is fetched one tile ahead into the
+//     other of two A buffers.  The arithmetic per tile is the one below.
+//   proxy_stream_kernel  (grid over 32 x 256 tiles of P; two CTAs per SM;
+//     any r)
 //     Each thread owns 8 rows x 4 columns.  Its P and Wq slices stream in
 //     with cp.async while the tile's A columns and dB_inc rows are staged
 //     in shared memory (A as bf16, dB_inc as duplicated float pairs so that
@@ -63,6 +71,10 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all_but_newest() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 
 // Values of the two codes in the low 16 bits of `c2` (hardware conversion via f16).
@@ -222,6 +234,177 @@ __global__ void __launch_bounds__(kThreads, 2)
     atomicOr(dev_status, kDevNonfinite);
 }
 
+// ---------------------------------------------------------------- persistent pipeline
+constexpr int kPipeStages = 3;                     // tiles in flight per thread: current + 2
+constexpr int kPipeRMax = 64;                      // ranks held in shared memory
+constexpr int kDbStride = kPipeRMax * 2 + 16;      // bytes per staged dB_inc row (padded)
+constexpr int kDbRawBytes = kTileRows * kDbStride;                 // 4.5 KB
+constexpr int kPipeAsBytes = kPipeRMax * kTileCols * 2;            // 32 KB per A buffer
+constexpr int kPipeBsBytes = kPipeRMax * kTileRows * 8;            // 16 KB
+constexpr int kPipeSmemBytes =
+    kPipeStages * (kPBytes + kWBytes + kDbRawBytes) + 2 * kPipeAsBytes + kPipeBsBytes;  // 213.5 KB
+
+template <bool kAcc, bool kSel>
+__global__ void __launch_bounds__(kThreads, 1)
+    proxy_pipe_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
+                      float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
+                      const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
+                      int units, uint8_t* __restrict__ rowflag, int32_t* __restrict__ dev_status) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  float4* pst = reinterpret_cast<float4*>(sm);                                // [S][kRT][256]
+  uint32_t* wst = reinterpret_cast<uint32_t*>(sm + kPipeStages * kPBytes);    // [S][kRT][256]
+  uint8_t* dbraw = sm + kPipeStages * (kPBytes + kWBytes);                    // [S][32][kDbStride]
+  uint16_t* As = reinterpret_cast<uint16_t*>(dbraw + kPipeStages * kDbRawBytes);  // [2][r][256]
+  float2* Bs = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(As) + 2 * kPipeAsBytes);  // [r][32]
+
+  const int tid = threadIdx.x;
+  const int tc = tid & 63;  // columns c0 + 4*tc .. +3
+  const int tr = tid >> 6;  // rows r0 + 8*tr .. +7
+  const int u_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * units / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * units / gridDim.x);
+  if (u_begin >= u_end) return;
+  const int chunks_per_row = r / 8;  // 16-byte chunks of one dB_inc row
+
+  // this thread's P / Wq slices and (its share of) the dB_inc rows of tile v
+  auto issue_tile = [&](int v, int slot) {
+    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kTileRows;
+    const int64_t col = static_cast<int64_t>(v / row_groups) * kTileCols + 4 * tc;
+    const bool col_ok = col < K;
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = r0 + tr * kRT + j;
+      const bool ok = col_ok && n < N;
+      cp_async16(pst + (slot * kRT + j) * kThreads + tid,
+                 ok ? static_cast<const void*>(proxy + n * K + col) : proxy, ok ? 16u : 0u);
+      if (kSel)
+        cp_async4(wst + (slot * kRT + j) * kThreads + tid,
+                  ok ? static_cast<const void*>(wq + n * K + col) : wq, ok ? 4u : 0u);
+    }
+    if (kAcc && tid < kTileRows * chunks_per_row) {
+      const int row = tid / chunks_per_row, c8 = tid % chunks_per_row;
+      const int64_t n = r0 + row;
+      const bool ok = n < N;
+      cp_async16(dbraw + slot * kDbRawBytes + row * kDbStride + 16 * c8,
+                 ok ? static_cast<const void*>(dB_inc + n * r + 8 * c8) : dB_inc, ok ? 16u : 0u);
+    }
+  };
+  // A[0:r, cb*256 : cb*256+256] -> As[buf] (zero beyond K)
+  auto issue_A = [&](int cb, int buf) {
+    uint16_t* dst = As + buf * (kPipeAsBytes / 2);
+    for (int e = tid; e < r * (kTileCols / 8); e += kThreads) {
+      const int i = e / (kTileCols / 8), c8 = e % (kTileCols / 8);
+      const int64_t gc = static_cast<int64_t>(cb) * kTileCols + 8 * c8;
+      const bool ok = gc < K;
+      cp_async16(dst + i * kTileCols + 8 * c8,
+                 ok ? static_cast<const void*>(A + static_cast<int64_t>(i) * K + gc) : A,
+                 ok ? 16u : 0u);
+    }
+  };
+
+  // prologue: groups A(u_begin), G(u_begin), G(u_begin + 1)
+  if (kAcc) issue_A(u_begin / row_groups, 0);
+  cp_async_commit();
+  issue_tile(u_begin, 0);
+  cp_async_commit();
+  if (u_begin + 1 < u_end) issue_tile(u_begin + 1, 1);
+  cp_async_commit();
+
+  const float s_w = kSel ? *s_w_ptr : 1.0f;
+  bool nonfinite = false;
+  int abuf = 0;
+  int slot = 0;
+  for (int v = u_begin; v < u_end; ++v) {
+    // outstanding: ..., A(v), G(v), [A(v+1)?], G(v+1): all but the newest have landed
+    cp_async_wait_all_but_newest();
+    if (kAcc) {
+      __syncthreads();  // every thread's copies for v visible; unit v-1 finished everywhere
+      // dB_inc rows of tile v -> (b, b) pairs, [i][row]: 8 ranks per thread
+      const uint8_t* raw = dbraw + slot * kDbRawBytes;
+      for (int e = tid; e < kTileRows * chunks_per_row; e += kThreads) {
+        const int row = e % kTileRows, c8 = e / kTileRows;
+        const uint4 q = *reinterpret_cast<const uint4*>(raw + row * kDbStride + 16 * c8);
+        const uint32_t wds[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float f0 = __uint_as_float(wds[h] << 16);
+          const float f1 = __uint_as_float(wds[h] & 0xFFFF0000u);
+          Bs[(8 * c8 + 2 * h) * kTileRows + row] = make_float2(f0, f0);
+          Bs[(8 * c8 + 2 * h + 1) * kTileRows + row] = make_float2(f1, f1);
+        }
+      }
+    }
+    // prefetch: A of the next tile's column block when it changes, then tile v+2
+    int next_abuf = abuf;
+    if (kAcc && v + 1 < u_end && (v + 1) / row_groups != v / row_groups) {
+      next_abuf = abuf ^ 1;
+      issue_A((v + 1) / row_groups, next_abuf);
+    }
+    cp_async_commit();
+    if (v + 2 < u_end) issue_tile(v + 2, slot == 0 ? 2 : slot - 1);
+    cp_async_commit();
+
+    float2 acc[kRT][2];
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) acc[j][0] = acc[j][1] = make_float2(0.0f, 0.0f);
+    if constexpr (kAcc) {
+      __syncthreads();  // Bs complete
+      const uint16_t* arow = As + abuf * (kPipeAsBytes / 2) + 4 * tc;
+      const float2* brow = Bs + tr * kRT;
+#pragma unroll 4
+      for (int i = 0; i < r; ++i) {
+        const uint2 a2 = *reinterpret_cast<const uint2*>(arow + i * kTileCols);
+        const float2 a01 = make_float2(__uint_as_float(a2.x << 16), __uint_as_float(a2.x & 0xFFFF0000u));
+        const float2 a23 = make_float2(__uint_as_float(a2.y << 16), __uint_as_float(a2.y & 0xFFFF0000u));
+        float2 bb[kRT];
+#pragma unroll
+        for (int j = 0; j < kRT; j += 2) {
+          const float4 q = *reinterpret_cast<const float4*>(brow + i * kTileRows + j);
+          bb[j] = make_float2(q.x, q.y);
+          bb[j + 1] = make_float2(q.z, q.w);
+        }
+#pragma unroll
+        for (int j = 0; j < kRT; ++j) {
+          acc[j][0] = __ffma2_rn(bb[j], a01, acc[j][0]);
+          acc[j][1] = __ffma2_rn(bb[j], a23, acc[j][1]);
+        }
+      }
+    }
+
+    // epilogue: P' = P + D; requantize; write P' and the changed codes
+    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kTileRows;
+    const int64_t col = static_cast<int64_t>(v / row_groups) * kTileCols + 4 * tc;
+    const bool col_ok = col < K;
+#pragma unroll
+    for (int j = 0; j < kRT; ++j) {
+      const int64_t n = r0 + tr * kRT + j;
+      if (!(col_ok && n < N)) continue;
+      float4 p = pst[(slot * kRT + j) * kThreads + tid];
+      if constexpr (kAcc) {
+        p.x = __fadd_rn(p.x, acc[j][0].x);
+        p.y = __fadd_rn(p.y, acc[j][0].y);
+        p.z = __fadd_rn(p.z, acc[j][1].x);
+        p.w = __fadd_rn(p.w, acc[j][1].y);
+        *reinterpret_cast<float4*>(proxy + n * K + col) = p;
+      }
+      nonfinite |= !(isfinite(p.x) && isfinite(p.y) && isfinite(p.z) && isfinite(p.w));
+      if constexpr (kSel) {
+        const uint32_t w = wst[(slot * kRT + j) * kThreads + tid];
+        const uint32_t cn = requantized4(w, s_w, p);
+        const uint32_t m = changed_bytes(w, cn);
+        if (m) {
+          *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
+          rowflag[n] = 1;  // every writer stores the same value
+        }
+      }
+    }
+    abuf = next_abuf;
+    slot = slot == kPipeStages - 1 ? 0 : slot + 1;
+  }
+  cp_async_wait_all();
+  if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
+    atomicOr(dev_status, kDevNonfinite);
+}
+
 constexpr int kClearThreads = 256;
 
 __global__ void __launch_bounds__(kClearThreads)
@@ -262,6 +445,26 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
   return cudaGetLastError();
 }
 
+template <bool kAcc, bool kSel>
+cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
+                        const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
+                        uint8_t* rowflag, int32_t* dev_status, cudaStream_t stream) {
+  static int configured_mask = 0;  // one bit per device ordinal < 31
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int bit = dev < 31 ? (1 << dev) : 0;
+  if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(proxy_pipe_kernel<kAcc, kSel>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPipeSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
+  }
+  proxy_pipe_kernel<kAcc, kSel><<<grid, kThreads, kPipeSmemBytes, stream>>>(
+      wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
+      r, row_groups, units, rowflag, dev_status);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t proxy_workspace_bytes(int64_t N, int64_t K) {
@@ -279,7 +482,13 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   if (r > (int64_t(1) << 30)) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
                   static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
-  if (grid.y > 65535u) return cudaErrorInvalidValue;
+  const int rr = acc ? static_cast<int>(r) : 0;
+  const int64_t row_groups = (N + kTileRows - 1) / kTileRows;
+  const int64_t units = row_groups * grid.x;
+  // the persistent kernel holds A and dB_inc slices of up to 64 ranks in 16-byte chunks
+  const bool pipe = rr <= kPipeRMax && rr % 8 == 0 && units <= (int64_t(1) << 30) &&
+                    di->max_smem_optin >= kPipeSmemBytes;
+  if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
   uint8_t* rowflag = static_cast<uint8_t*>(workspace);
   cudaError_t e;
   if (sel) {
@@ -287,8 +496,16 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
     if (n_selected && (e = cudaMemsetAsync(n_selected, 0, sizeof(int32_t), stream)) != cudaSuccess)
       return e;
   }
-  const int rr = acc ? static_cast<int>(r) : 0;
-  if (acc && sel)
+  if (pipe) {
+    const int g = static_cast<int>(units < di->sm_count ? units : di->sm_count);
+    const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
+    if (acc && sel)
+      e = launch_pipe<true, true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+    else if (acc)
+      e = launch_pipe<true, false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+    else
+      e = launch_pipe<false, true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+  } else if (acc && sel)
     e = launch_stream<true, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);
   else if (acc)
     e = launch_stream<true, false>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);

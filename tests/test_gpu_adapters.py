@@ -94,3 +94,44 @@ def test_llama_attention_full_size(cuda_device, name):
     rda, rdb = _oracle(*case)
     assert O.tolerance_report(db, rdb)["ok"]
     assert O.tolerance_report(da, rda)["ok"]
+
+
+def _every_code(shape, offset):
+    """Codes cycling through all 254 non-NaN E4M3 codes."""
+    valid = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    idx = (np.arange(shape[0] * shape[1]) * 7 + offset) % valid.size
+    return valid[idx].reshape(shape)
+
+
+def test_every_code_expands_exactly(cuda_device):
+    """Each operand holds every non-NaN code (subnormals, zeros of both signs,
+    +-448), so each code's expansion to bf16 enters both products."""
+    M, N, K, r = 256, 384, 512, 32
+    xq, dyq = _every_code((M, K), 0), _every_code((M, N), 3)
+    s_x, s_dy = np.float32(3.0), np.float32(0.5)
+    A = gen.normal_bf16_bits(11, (r, K), 0.01)
+    B = gen.normal_bf16_bits(12, (N, r), 0.01)
+    case = (xq, s_x, dyq, s_dy, A, B)
+    da, db = _gpu(*case)
+    rda, rdb = _oracle(*case)
+    assert O.tolerance_report(db, rdb)["ok"]
+    assert O.tolerance_report(da, rda)["ok"]
+
+
+def test_nan_code_propagates(cuda_device):
+    """A NaN code in Xq poisons its row of T (hence all of dB) and its column
+    of dA, on both sides; everything else still matches."""
+    M, N, K, r = 128, 256, 256, 16
+    xq, s_x, dyq, s_dy, A, B = _case(13, M, N, K, r)
+    xq = xq.copy()
+    xq[5, 77] = 0xFF
+    da, db = _gpu(xq, s_x, dyq, s_dy, A, B)
+    rda, rdb = _oracle(xq, s_x, dyq, s_dy, A, B)
+
+    def isnan(bits):
+        return ((bits & 0x7F80) == 0x7F80) & ((bits & 0x007F) != 0)
+
+    assert np.array_equal(isnan(db), np.isnan(rdb)) and np.isnan(rdb).all()
+    assert np.array_equal(isnan(da), np.isnan(rda))
+    assert np.isnan(rda[:, 77]).all() and not np.isnan(np.delete(rda, 77, axis=1)).any()
+    assert O.tolerance_report(np.delete(da, 77, axis=1), np.delete(rda, 77, axis=1))["ok"]
