@@ -10,7 +10,7 @@ All five library phases run in libfalqon's kernels through the C ABI.
 Timing: W untimed warm-up steps, then K timed steps.  The step is captured
 once per input slot in a CUDA graph and replayed; each timed step is bracketed
 by CUDA events on the launching stream and separated from the next by an L2
-flush (a 512 MB write, outside the events).  The timed region is bracketed by
+flush (a 512 MB write and a 192 MB read, outside the events).  The timed region is bracketed by
 a barrier and torch.cuda.synchronize() on both sides; with N > 1 every rank
 runs an independent replica on its own batch ("replicas only", weak scaling)
 and the reported time is the max over ranks.
@@ -241,6 +241,13 @@ def run_gpu(args):
     st = Step(wl, layer, torch, F, dev, n_slots=2, seed_offset=rank * 1000)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_tail = flush[: 192 << 20].view(torch.int32)
+
+    def l2_flush(i):
+        """Evicts L2: a 512 MB write, then a 192 MB read, so that the lines left
+        behind are clean and no write-back of the flush lands in the next step."""
+        flush.fill_(i & 0xFF)
+        flush_tail.sum()
 
     # capture the step once per input slot
     graphs = []
@@ -273,7 +280,7 @@ def run_gpu(args):
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            flush.fill_(i & 0xFF)
+            l2_flush(i)
             step(i)
     torch.cuda.synchronize()
     if int(st.status.item()) != 0:
@@ -290,7 +297,7 @@ def run_gpu(args):
     time.sleep(0.25)
     with torch.cuda.stream(stream):
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            l2_flush(i)
             starts[i].record()
             step(i)
             ends[i].record()
@@ -308,7 +315,7 @@ def run_gpu(args):
     reps = max(5, min(50, args.steps))
     with torch.cuda.stream(stream):
         for i in range(reps):
-            flush.fill_(i & 0xFF)
+            l2_flush(i)
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
             ev[0].record()
             for k in range(len(names)):
@@ -388,7 +395,7 @@ def run_gpu(args):
         "data": "synthetic",
         "config": {"workload": wl.name, "M": wl.M, "N": layer.N, "K": layer.K, "r": wl.r,
                    "global_batch_tokens": wl.M * ws, "parallelism": f"replicas{ws}",
-                   "l2": "flushed between timed steps (512 MB write outside the events)",
+                   "l2": "flushed between timed steps (512 MB write + 192 MB read, outside the events)",
                    "cuda_graph": not args.no_graph, "lr": wl.lr},
         "roofline": roof,
         "phases": phases,

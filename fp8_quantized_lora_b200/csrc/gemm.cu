@@ -47,15 +47,12 @@ struct GemmArgs {
   void* out_lo;            // optional low half: out + out_lo carries ~16 significant bits
   int64_t ldo;
   int transpose;           // store out[col * ldo + row]
-  // E4M3 codes of an expanded A operand, row-major [a_rows][a_cols], read by the
-  // converter warps straight from global memory (K-major: rows = M side,
-  // cols = contraction; MN-major: rows = contraction, cols = M side)
-  const uint8_t* a_codes;
-  int64_t a_rows, a_cols;
   const float* scale_a;    // alpha = 1 / (scale_a * scale_b); either may be null (= 1)
   const float* scale_b;
   int32_t* dev_status;
 };
+
+constexpr int kMaxSplits = 8;  // split-K partners: at most the portable cluster size
 
 template <bool kF8, bool kAMn, bool kBMn, bool kAConv, int kBN, int kStages, bool kClusterK,
           bool kBSplit = false, int kRawStages = 0, int kBStages = kStages>
@@ -84,15 +81,17 @@ struct Cfg {
   static constexpr int ARingBytes = kAConv ? kStages * ABytes : 0;
   static constexpr int BRingBytes = BStages * BSlotBytes;
   static constexpr int TmaBytes = BSlotBytes;
-  static constexpr int NumConvWarps = kAConv ? 8 : 0;
-  // per-converter-thread ring of raw E4M3 codes (32 bytes per thread per k-block),
-  // filled with cp.async kRawStages k-blocks ahead
+  static constexpr int NumConvWarps = kAConv ? 16 : 0;
+  // ring of raw E4M3 A tiles (one k-block each, unswizzled, row-major), filled
+  // by TMA from a warp of its own kRawStages k-blocks ahead of the converters
   static constexpr int RawStages = kAConv ? kRawStages : 0;
-  static constexpr int RawSlotBytes = 32 * 32 * NumConvWarps;  // 8 KB
+  static constexpr int RawSlotBytes = kAConv ? kBM * BK : 0;  // 8 KB of codes
   static_assert(!kAConv || kRawStages >= 2, "raw ring depth");
-  static constexpr int Threads = 32 * (6 + NumConvWarps);
+  static_assert(!kAConv || RawSlotBytes == 16 * 32 * NumConvWarps, "one 16-byte chunk per converter thread");
+  static constexpr int RawWarp = 6 + NumConvWarps;  // raw-code producer (expansion only)
+  static constexpr int Threads = 32 * (6 + NumConvWarps + (kAConv ? 1 : 0));
   static constexpr uint32_t TmemCols = 2 * kBN < 32 ? 32 : 2 * kBN;
-  static constexpr int BarBytes = 8 * (2 * kStages + 2 * BStages + 5) + 16;
+  static constexpr int BarBytes = 8 * (2 * kStages + 2 * BStages + 2 * RawStages + 5) + 16;
   static constexpr int SmemBytes = ARingBytes + BRingBytes + RawStages * RawSlotBytes + BarBytes + 1024;
   static constexpr int RedStride = kBN + 4;  // fp32 words per row of the reduction tile (16-byte rows)
   static_assert(!kClusterK || kBM * RedStride * 4 <= ARingBytes + BRingBytes, "reduction tile");
@@ -158,19 +157,6 @@ __device__ __forceinline__ void e4m3x4_to_bf16_hw(uint32_t w, uint32_t& lo, uint
   hi = o[1];
 }
 
-// 16-byte global -> shared copy, zero-filled when src_bytes == 0.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -190,12 +176,13 @@ __device__ __forceinline__ uint32_t dsmem_addr(const void* local, int rank) {
   return remote;
 }
 
+// Peer tiles are stable between the two cluster barriers around the
+// reduction, so these loads may be reordered and overlapped freely.
 __device__ __forceinline__ float4 dsmem_load_f32x4(uint32_t addr) {
   float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+      : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+      : "r"(addr));
   return v;
 }
 
@@ -225,7 +212,9 @@ __global__ void __launch_bounds__(C::Threads, 1)
   uint64_t* empty = full + C::BStages;                   // [BStages] MMAs done with the TMA slot
   uint64_t* conv = empty + C::BStages;                   // [Stages] codes expanded
   uint64_t* aempty = conv + C::Stages;                   // [Stages] MMAs done with the A slot
-  uint64_t* acc_full = aempty + C::Stages;               // [2] accumulator ready
+  uint64_t* rawfull = aempty + C::Stages;                // [RawStages] raw codes landed
+  uint64_t* rawempty = rawfull + C::RawStages;           // [RawStages] converters done reading
+  uint64_t* acc_full = rawempty + C::RawStages;          // [2] accumulator ready
   uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained
   uint64_t* drain = acc_empty + 2;            // all issued MMAs retired (teardown)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -243,6 +232,10 @@ __global__ void __launch_bounds__(C::Threads, 1)
     for (int s = 0; s < C::Stages; ++s) {
       mbar_init(&conv[s], C::NumConvWarps > 0 ? C::NumConvWarps : 1);
       mbar_init(&aempty[s], 1);
+    }
+    for (int s = 0; s < C::RawStages; ++s) {
+      mbar_init(&rawfull[s], 1);
+      mbar_init(&rawempty[s], C::NumConvWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -324,6 +317,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
       for (int s = 0; s < C::BStages; ++s)
         if (issued & (1u << s)) mbar_wait_budget(&full[s], (issued_parity >> s) & 1u);
     }
+    __syncwarp();  // the warp reaches the CTA barriers below together
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     int stage = 0, astage = 0;
@@ -443,87 +437,115 @@ __global__ void __launch_bounds__(C::Threads, 1)
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
   } else if constexpr (C::AConv) {
-    // ------------------------------------------------------------ converters
-    // 256 threads; each owns 32 codes (two 16-byte chunks) of every A tile:
-    //   K-major  [128 rows][64 codes]: row = t / 2,  columns (t % 2) * 32 ..
-    //   MN-major [64 rows][128 codes]: row = t / 4,  columns (t % 4) * 32 ..
-    // Each thread streams its own chunks with cp.async into a private slot of
-    // the raw ring RawStages k-blocks ahead, so only it reads them back and
-    // no cross-thread synchronisation is needed for the raw codes.
-    constexpr int R = C::RawStages;
-    constexpr int kTileRows = C::AMn ? C::BK : kBM;        // rows of the A tile in smem
+    constexpr int kTileRows = C::AMn ? C::BK : kBM;        // rows of the A tile (and of its raw box)
     constexpr int kTileCols = C::AMn ? kBM : C::BK;        // codes per row
-    constexpr int kThrPerRow = kTileCols / 32;
-    const int t = threadIdx.x - 6 * 32;
-    const int trow = t / kThrPerRow;
-    const int tcol = (t % kThrPerRow) * 32;
-    uint8_t* my_raw = raw_ring + t * 32;
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      const int split = w % g.splits;
-      const int mt = w / (g.splits * g.n_tiles);
-      const int kb0 = split * g.kb_per_split;
-      const int kb1 = min(g.kb_total, kb0 + g.kb_per_split);
-      const int64_t m0 = static_cast<int64_t>(mt) * kBM;
-      auto fetch = [&](int kb, int slot) {
-        const int64_t grow = C::AMn ? static_cast<int64_t>(kb) * C::BK + trow : m0 + trow;
-        const int64_t gcol = C::AMn ? m0 + tcol : static_cast<int64_t>(kb) * C::BK + tcol;
-        const uint8_t* src = g.a_codes + grow * g.a_cols + gcol;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const bool valid = grow < g.a_rows && gcol + 16 * h < g.a_cols;
-          cp_async16(my_raw + slot * C::RawSlotBytes + 16 * h, valid ? src + 16 * h : g.a_codes,
-                     valid ? 16u : 0u);
+    if (warp == C::RawWarp) {
+      // ---------------------------------------------------------- raw-code producer
+      // One TMA box per k-block: K-major A = codes[m0 .. +128, kb*64 .. +64];
+      // MN-major A = codes[kb*64 .. +64, m0 .. +128] (rows of the code matrix are K).
+      if (lane == 0) {
+        int rs = 0;
+        uint32_t rphase = 0;
+        uint32_t issued = 0, issued_parity = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+          const int split = w % g.splits;
+          const int mt = w / (g.splits * g.n_tiles);
+          const int kb0 = split * g.kb_per_split;
+          const int kb1 = min(g.kb_total, kb0 + g.kb_per_split);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&rawempty[rs], rphase ^ 1, abort_flag)) { fail(); ok = false; break; }
+            mbar_arrive_expect_tx(&rawfull[rs], C::RawSlotBytes);
+            issued |= 1u << rs;
+            issued_parity = (issued_parity & ~(1u << rs)) | (rphase << rs);
+            if constexpr (C::AMn)
+              tma_load_2d(raw_ring + rs * C::RawSlotBytes, &tmA, &rawfull[rs], mt * kBM, kb * C::BK);
+            else
+              tma_load_2d(raw_ring + rs * C::RawSlotBytes, &tmA, &rawfull[rs], kb * C::BK, mt * kBM);
+            if (++rs == C::RawStages) { rs = 0; rphase ^= 1; }
+          }
         }
-      };
-#pragma unroll 1
-      for (int d = 0; d < R; ++d) {
-        if (kb0 + d < kb1) fetch(kb0 + d, d);
-        cp_async_commit();
+        for (int s2 = 0; s2 < C::RawStages; ++s2)
+          if (issued & (1u << s2)) mbar_wait_budget(&rawfull[s2], (issued_parity >> s2) & 1u);
       }
-      int slot = 0;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        cp_async_wait<R - 1>();  // this thread's chunks of k-block kb have landed
-        if (!warp_wait(&aempty[stage], phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
-        const uint4 q0 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(my_raw + slot * C::RawSlotBytes + 16);
-        uint8_t* sA = a_ring + stage * C::ABytes;
-        // 32 codes -> 32 bf16 (four 16-byte units of the 128-byte-swizzled layout)
-        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        uint32_t o[16];
-        if (!(has_nan_code(q0) | has_nan_code(q1))) {
+      __syncwarp();
+    } else {
+      // ---------------------------------------------------------- converters
+      // 512 threads; each expands one 16-byte chunk (16 codes) of every A tile:
+      //   K-major  [128 rows][64 codes]: row = t / 4,  columns (t % 4) * 16 ..
+      //   MN-major [64 rows][128 codes]: row = t / 8,  columns (t % 8) * 16 ..
+      constexpr int kThrPerRow = kTileCols / 16;
+      const int t = threadIdx.x - 6 * 32;
+      const int trow = t / kThrPerRow;
+      const int tcol = (t % kThrPerRow) * 16;
+      const uint32_t raw_off = trow * kTileCols + tcol;
+      // destinations of the two 16-byte units (8 bf16 each) in the swizzled tile
+      const int blk = tcol / 64;
+      const int unit0 = (tcol % 64) / 8;
+      const uint32_t dst_off0 = blk * (kTileRows * kRowBytes) + trow * kRowBytes + ((unit0 ^ (trow & 7)) << 4);
+      const uint32_t dst_off1 = blk * (kTileRows * kRowBytes) + trow * kRowBytes + (((unit0 + 1) ^ (trow & 7)) << 4);
+      // Two k-blocks per iteration: their expansions are independent, so the
+      // two dependency chains overlap within the warp.
+      auto expand = [&](const uint4& q, uint8_t* sA) {
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[8];
+        if (!has_nan_code(q)) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             o[2 * j] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4140));
             o[2 * j + 1] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4342));
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) e4m3x4_to_bf16_hw(words[j], o[2 * j], o[2 * j + 1]);
+          for (int j = 0; j < 4; ++j) e4m3x4_to_bf16_hw(words[j], o[2 * j], o[2 * j + 1]);
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int col = tcol + 8 * u;
-          const int blk = col / 64;
-          const int unit = (col % 64) / 8;
-          uint8_t* dst = sA + blk * (kTileRows * kRowBytes) + trow * kRowBytes +
-                         ((unit ^ (trow & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        *reinterpret_cast<uint4*>(sA + dst_off0) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sA + dst_off1) = make_uint4(o[4], o[5], o[6], o[7]);
+      };
+      int stage = 0, rs = 0;
+      uint32_t phase = 0, rphase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+        const int split = w % g.splits;
+        const int kb0 = split * g.kb_per_split;
+        const int kb1 = min(g.kb_total, kb0 + g.kb_per_split);
+        for (int kb = kb0; kb < kb1; kb += 2) {
+          const bool two = kb + 1 < kb1;
+          // raw codes of k-blocks kb (and kb + 1)
+          const int rs1 = rs + 1 == C::RawStages ? 0 : rs + 1;
+          const uint32_t rphase1 = rs + 1 == C::RawStages ? rphase ^ 1 : rphase;
+          if (!warp_wait(&rawfull[rs], rphase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+          const uint4 q0 = *reinterpret_cast<const uint4*>(raw_ring + rs * C::RawSlotBytes + raw_off);
+          uint4 q1 = make_uint4(0u, 0u, 0u, 0u);
+          if (two) {
+            if (!warp_wait(&rawfull[rs1], rphase1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+            q1 = *reinterpret_cast<const uint4*>(raw_ring + rs1 * C::RawSlotBytes + raw_off);
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&rawempty[rs]);
+            if (two) mbar_arrive(&rawempty[rs1]);
+          }
+          rs = two ? (rs1 + 1 == C::RawStages ? 0 : rs1 + 1) : rs1;
+          rphase = two ? (rs1 + 1 == C::RawStages ? rphase1 ^ 1 : rphase1) : rphase1;
+          // expanded-A stages for kb (and kb + 1)
+          const int st1 = stage + 1 == C::Stages ? 0 : stage + 1;
+          const uint32_t phase1 = stage + 1 == C::Stages ? phase ^ 1 : phase;
+          if (!warp_wait(&aempty[stage], phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+          if (two && !warp_wait(&aempty[st1], phase1 ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+          expand(q0, a_ring + stage * C::ABytes);
+          if (two) expand(q1, a_ring + st1 * C::ABytes);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&conv[stage]);
+            if (two) mbar_arrive(&conv[st1]);
+          }
+          stage = two ? (st1 + 1 == C::Stages ? 0 : st1 + 1) : st1;
+          phase = two ? (st1 + 1 == C::Stages ? phase1 ^ 1 : phase1) : phase1;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&conv[stage]);
-        if (++stage == C::Stages) { stage = 0; phase ^= 1; }
-        // refill the slot just read (its codes are already in registers)
-        if (kb + R < kb1) fetch(kb + R, slot);
-        cp_async_commit();
-        if (++slot == R) slot = 0;
       }
-      cp_async_wait<0>();
     }
-    (void)kTileCols;
   }
 
   if constexpr (C::ClusterK) {
@@ -540,8 +562,9 @@ __global__ void __launch_bounds__(C::Threads, 1)
     const int q0 = static_cast<int>(rank) * rows_per;
     const int q1 = min(kBM, q0 + rows_per);
     const float* red = reinterpret_cast<const float*>(smem);
-    uint32_t peer[16];
-    for (int sidx = 0; sidx < S && sidx < 16; ++sidx) peer[sidx] = dsmem_addr(red, sidx);
+    uint32_t peer[kMaxSplits];
+#pragma unroll
+    for (int sidx = 0; sidx < kMaxSplits; ++sidx) peer[sidx] = dsmem_addr(red, sidx < S ? sidx : 0);
     double den = 1.0;
     if (g.scale_a) den *= static_cast<double>(*g.scale_a);
     if (g.scale_b) den *= static_cast<double>(*g.scale_b);
@@ -555,12 +578,21 @@ __global__ void __launch_bounds__(C::Threads, 1)
       else { lr = q0 + e / G; lg = e % G; }
       const uint32_t off = static_cast<uint32_t>((lr * C::RedStride + 4 * lg) * 4);
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int sidx = 0; sidx < S; ++sidx) {  // fixed order: rank 0, 1, ...
-        const float4 v = dsmem_load_f32x4(peer[sidx] + off);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+#pragma unroll
+      for (int s0 = 0; s0 < kMaxSplits; s0 += 4) {  // fixed order: rank 0, 1, ...
+        float4 part[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (s0 + k < S) part[k] = dsmem_load_f32x4(peer[s0 + k] + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (s0 + k < S) {
+            acc.x += part[k].x;
+            acc.y += part[k].y;
+            acc.z += part[k].z;
+            acc.w += part[k].w;
+          }
+        }
       }
       const int64_t grow = static_cast<int64_t>(mt) * kBM + lr;
       const int64_t gcol0 = static_cast<int64_t>(nt) * C::BN + 4 * lg;
@@ -641,23 +673,23 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 using FwdCfg = Cfg<true, false, false, false, 256, 4, false>;
 using DxCfg = Cfg<true, false, true, false, 256, 4, false>;
 
-// <A stages, raw stages, B stages> sized to ~200 KB of shared memory
-template <int BN> using TCfg = Cfg<false, false, false, true, BN, (BN >= 256 ? 3 : 4), true, false,
-                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8)),
-                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8))>;  // Xq . A^T
-template <int BN> using UCfg = Cfg<false, false, true, true, BN, (BN >= 256 ? 3 : 4), true, false,
-                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8)),
-                                   (BN >= 256 ? 4 : (BN >= 128 ? 6 : 8))>;  // dYq . B
-// dYq^T . (T_hi + T_lo), Xq^T . (U_hi + U_lo): fewer stages at BN = 256 to fit smem
-template <int BN> using MnCfg = Cfg<false, true, true, true, BN, (BN >= 256 ? 2 : (BN >= 128 ? 3 : 4)), true, true,
-                                    (BN >= 256 ? 4 : (BN >= 128 ? 4 : 6)),
-                                    (BN >= 256 ? 2 : (BN >= 128 ? 4 : 6))>;
+// Stage counts <A (expanded), raw codes, B> sized to about 224 KB of shared
+// memory.  The expanded-A ring is the deep one: a stage is released only when
+// the MMAs that read it have completed, so its depth has to cover the MMA
+// completion latency; the raw ring needs only to cover HBM latency.
+template <int BN> using TCfg = Cfg<false, false, false, true, BN, (BN >= 256 ? 3 : (BN >= 128 ? 4 : 6)), true, false,
+                                   (BN >= 256 ? 4 : 8), (BN >= 256 ? 3 : (BN >= 128 ? 4 : 8))>;  // Xq . A^T
+template <int BN> using UCfg = Cfg<false, false, true, true, BN, (BN >= 256 ? 3 : (BN >= 128 ? 4 : 6)), true, false,
+                                   (BN >= 256 ? 4 : 8), (BN >= 256 ? 3 : (BN >= 128 ? 4 : 8))>;  // dYq . B
+// dYq^T . (T_hi + T_lo), Xq^T . (U_hi + U_lo): B is split hi/lo, so fewer stages
+template <int BN> using MnCfg = Cfg<false, true, true, true, BN, (BN >= 256 ? 2 : (BN >= 128 ? 3 : 5)), true, true,
+                                    (BN >= 256 ? 4 : 8), (BN >= 256 ? 2 : (BN >= 128 ? 3 : 5))>;
 
 // Split count: as many K splits as fit beside the tiles in one wave, at most 8
 // (the portable cluster size), never more than there are K blocks.
 int choose_splits(int tiles, int kb_total, int sm_count) {
   int s = sm_count / (tiles > 0 ? tiles : 1);
-  if (s > 8) s = 8;
+  if (s > kMaxSplits) s = kMaxSplits;
   if (s > kb_total) s = kb_total;
   if (s < 1) s = 1;
   return s;
@@ -757,12 +789,8 @@ size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool 
 namespace {
 
 GemmArgs skinny_args(const SkinnyPlan& p, int64_t rows, int64_t r, void* out, void* out_lo,
-                     int64_t ldo, bool transpose, const float* scale, int32_t* st,
-                     const uint8_t* codes, int64_t code_rows, int64_t code_cols) {
+                     int64_t ldo, bool transpose, const float* scale, int32_t* st) {
   GemmArgs g{};
-  g.a_codes = codes;
-  g.a_rows = code_rows;
-  g.a_cols = code_cols;
   g.m_tiles = p.m_tiles;
   g.n_tiles = p.n_tiles;
   g.splits = p.splits;
@@ -778,6 +806,14 @@ GemmArgs skinny_args(const SkinnyPlan& p, int64_t rows, int64_t r, void* out, vo
   g.scale_b = nullptr;
   g.dev_status = st;
   return g;
+}
+
+// Tensor map over an E4M3 code matrix [rows, cols] for the raw-code ring of an
+// expanded A operand, unswizzled: K-major (contraction along cols) boxes are
+// 128 rows x 64 codes; MN-major (contraction along rows) boxes are 64 rows x 128 codes.
+bool codes_tmap(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t cols, bool mn_major) {
+  return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, codes, static_cast<uint64_t>(cols),
+                      static_cast<uint64_t>(rows), mn_major ? 128 : 64, mn_major ? 64 : 128, false);
 }
 
 }  // namespace
@@ -801,33 +837,31 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   if (dB) {
     // T = Xq . A^T / s_x -> (T_hi, T_lo): A-op Xq [M, K] K-major (expanded), B-op A [r, K] K-major
     SkinnyPlan p = plan_skinny(M, r, K, di->sm_count);
-    if (!make_tmap_2d(&tB, BF, 2, A, K, r, 64, p.bn, true)) return cudaErrorInvalidValue;
-    tA = tB;  // A is read by the converter warps, not by TMA
-    GemmArgs g = skinny_args(p, M, r, T_hi, T_lo, r, false, s_x, dev_status, xq, M, K);
+    if (!make_tmap_2d(&tB, BF, 2, A, K, r, 64, p.bn, true) || !codes_tmap(&tA, xq, M, K, false))
+      return cudaErrorInvalidValue;
+    GemmArgs g = skinny_args(p, M, r, T_hi, T_lo, r, false, s_x, dev_status);
     if ((e = skinny_dispatch<TCfg>(p.bn, tA, tB, tB, g, stream)) != cudaSuccess) return e;
     // dB = dYq^T . (T_hi + T_lo) / s_dy: A-op dYq^T (MN-major, expanded), B-op T [M, r] MN-major
     SkinnyPlan q = plan_skinny(N, r, M, di->sm_count);
     if (!make_tmap_2d(&tB, BF, 2, T_hi, r, M, 64, 64, true) ||
-        !make_tmap_2d(&tB2, BF, 2, T_lo, r, M, 64, 64, true))
+        !make_tmap_2d(&tB2, BF, 2, T_lo, r, M, 64, 64, true) || !codes_tmap(&tA, dyq, M, N, true))
       return cudaErrorInvalidValue;
-    tA = tB;
-    GemmArgs h = skinny_args(q, N, r, dB, nullptr, r, false, s_dy, dev_status, dyq, M, N);
+    GemmArgs h = skinny_args(q, N, r, dB, nullptr, r, false, s_dy, dev_status);
     if ((e = skinny_dispatch<MnCfg>(q.bn, tA, tB, tB2, h, stream)) != cudaSuccess) return e;
   }
   if (dA) {
     // U = dYq . B / s_dy -> (U_hi, U_lo): A-op dYq [M, N] K-major (expanded), B-op B [N, r] MN-major
     SkinnyPlan p = plan_skinny(M, r, N, di->sm_count);
-    if (!make_tmap_2d(&tB, BF, 2, B, r, N, 64, 64, true)) return cudaErrorInvalidValue;
-    tA = tB;
-    GemmArgs g = skinny_args(p, M, r, U_hi, U_lo, r, false, s_dy, dev_status, dyq, M, N);
+    if (!make_tmap_2d(&tB, BF, 2, B, r, N, 64, 64, true) || !codes_tmap(&tA, dyq, M, N, false))
+      return cudaErrorInvalidValue;
+    GemmArgs g = skinny_args(p, M, r, U_hi, U_lo, r, false, s_dy, dev_status);
     if ((e = skinny_dispatch<UCfg>(p.bn, tA, tB, tB, g, stream)) != cudaSuccess) return e;
     // dA^T = Xq^T . (U_hi + U_lo) / s_x, stored transposed into dA [r, K]
     SkinnyPlan q = plan_skinny(K, r, M, di->sm_count);
     if (!make_tmap_2d(&tB, BF, 2, U_hi, r, M, 64, 64, true) ||
-        !make_tmap_2d(&tB2, BF, 2, U_lo, r, M, 64, 64, true))
+        !make_tmap_2d(&tB2, BF, 2, U_lo, r, M, 64, 64, true) || !codes_tmap(&tA, xq, M, K, true))
       return cudaErrorInvalidValue;
-    tA = tB;
-    GemmArgs h = skinny_args(q, K, r, dA, nullptr, K, true, s_x, dev_status, xq, M, K);
+    GemmArgs h = skinny_args(q, K, r, dA, nullptr, K, true, s_x, dev_status);
     if ((e = skinny_dispatch<MnCfg>(q.bn, tA, tB, tB2, h, stream)) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -14,6 +14,7 @@ struct DeviceInfo {
   int max_smem_optin = 0;
   int cc_major = 0;
   int cc_minor = 0;
+  int coop_launch = 0;  // cooperative launches supported
 };
 
 // Cached per device; returns nullptr if the current device cannot be queried.

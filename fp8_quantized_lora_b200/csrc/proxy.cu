@@ -8,14 +8,15 @@
 // value of every code whose value changes and have their proxy cleared;
 // other rows keep their codes bit-for-bit and their accumulated proxy.
 //
-// Two kernels, no cross-CTA synchronisation:
-//   proxy_pipe_kernel  (persistent, one CTA per SM; r <= 64 and r % 8 == 0)
-//     Each CTA walks a contiguous range of 32 x 256 tiles of P, column block
-//     by column block, so the block's A columns stay in shared memory.  Every
-//     thread streams its own P and Wq slices, and the tile's dB_inc rows, two
-//     tiles ahead with cp.async (three slots), while it computes the current
-//     tile; A for the next column block is fetched one tile ahead into the
-//     other of two A buffers.  The arithmetic per tile is the one below.
+// Two launches per update (one of the first two kernels, then the clear), no
+// cross-CTA synchronisation:
+//   proxy_pipe_kernel  (accumulation with r <= 64, r % 8 == 0; persistent,
+//     two CTAs per SM) walks a contiguous range of 32 x 256 tiles of P,
+//     column block by column block, keeping the block's A columns in shared
+//     memory.  The next tile's dB_inc rows are fetched with cp.async one tile
+//     ahead; each thread's P and Wq slices of the current tile are fetched when
+//     the tile starts and land while its FMA chains run (8 rows x 8 columns per
+//     thread).  The arithmetic is the one below.
 //   proxy_stream_kernel  (grid over 32 x 256 tiles of P; two CTAs per SM;
 //     any r)
 //     Each thread owns 8 rows x 4 columns.  Its P and Wq slices stream in
@@ -73,9 +74,11 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async_wait_all_but_newest() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+
 
 // Values of the two codes in the low 16 bits of `c2` (hardware conversion via f16).
 __device__ __forceinline__ float2 e4m3x2_values(uint32_t c2) {
@@ -101,19 +104,23 @@ __device__ __forceinline__ uint32_t requantized4(uint32_t w4, float s_w, float4 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// Two codes hold the same value: identical non-NaN codes, or both zero.
-__device__ __forceinline__ bool same_value(uint32_t a, uint32_t b) {
-  const bool nan = ((a & 0x7Fu) == 0x7Fu) || ((b & 0x7Fu) == 0x7Fu);
-  return !nan && (a == b || ((a & 0x7Fu) == 0u && (b & 0x7Fu) == 0u));
+// 0x80 in every byte of x that is zero, 0x00 elsewhere (exact per byte: the
+// masked add cannot carry across bytes).
+__device__ __forceinline__ uint32_t zero_bytes(uint32_t x) {
+  const uint32_t t = (x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu;  // bit 7 set iff the low 7 bits are not all 0
+  return ~(t | x) & 0x80808080u;
 }
 
 // Byte mask (0xFF per byte) of the codes whose value changes from `a` to `b`.
+// Two codes hold the same value when they are identical non-NaN codes or
+// both zero (either sign); a NaN code never holds the same value.
 __device__ __forceinline__ uint32_t changed_bytes(uint32_t a, uint32_t b) {
-  uint32_t m = 0;
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    if (!same_value((a >> (8 * c)) & 0xFFu, (b >> (8 * c)) & 0xFFu)) m |= 0xFFu << (8 * c);
-  return m;
+  const uint32_t mag = 0x7F7F7F7Fu;
+  const uint32_t same_bits = zero_bytes(a ^ b);
+  const uint32_t both_zero = zero_bytes((a | b) & mag);
+  const uint32_t nan = zero_bytes((a & mag) ^ mag) | zero_bytes((b & mag) ^ mag);
+  const uint32_t changed = ~((same_bits | both_zero) & ~nan) & 0x80808080u;
+  return (changed >> 7) * 0xFFu;
 }
 
 template <bool kAcc, bool kSel>
@@ -235,173 +242,201 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------- persistent pipeline
-constexpr int kPipeStages = 3;                     // tiles in flight per thread: current + 2
-constexpr int kPipeRMax = 64;                      // ranks held in shared memory
-constexpr int kDbStride = kPipeRMax * 2 + 16;      // bytes per staged dB_inc row (padded)
-constexpr int kDbRawBytes = kTileRows * kDbStride;                 // 4.5 KB
-constexpr int kPipeAsBytes = kPipeRMax * kTileCols * 2;            // 32 KB per A buffer
-constexpr int kPipeBsBytes = kPipeRMax * kTileRows * 8;            // 16 KB
+// Tiles of 32 rows x 256 columns, four warps per CTA, two CTAs per SM: while
+// one CTA runs its epilogue (memory and integer work) the other keeps the FMA
+// pipe busy.  Warp w owns rows 8w .. 8w+7 of the tile and lane l the columns
+// 8l .. 8l+7, so every thread keeps 8 x 8 accumulators (32 packed FMAs per
+// rank against one 16-byte load of A and four broadcast loads of dB_inc pairs).
+constexpr int kPipeThreads = 128;
+constexpr int kPipeRows = 32;
+constexpr int kPipeRT = 8;                          // rows per thread
+constexpr int kPipeCT = 8;                          // columns per thread
+constexpr int kPipeRMax = 64;                       // ranks held in shared memory
+constexpr int kDbStride = kPipeRMax * 2 + 16;       // bytes per staged dB_inc row (padded)
+constexpr int kPipePBytes = kPipeRows * kTileCols * 4;            // P tile          32 KB
+constexpr int kPipeWBytes = kPipeRows * kTileCols;                // Wq tile          8 KB
+constexpr int kPipeDbBytes = kPipeRows * kDbStride;               // dB_inc rows    4.5 KB
+constexpr int kPipeAsBytes = kPipeRMax * kTileCols * 2;           // A columns       32 KB
+constexpr int kPipeBsBytes = kPipeRMax * kPipeRows * 8;           // (b, b) pairs    16 KB
 constexpr int kPipeSmemBytes =
-    kPipeStages * (kPBytes + kWBytes + kDbRawBytes) + 2 * kPipeAsBytes + kPipeBsBytes;  // 213.5 KB
+    kPipePBytes + kPipeWBytes + 2 * kPipeDbBytes + kPipeAsBytes + kPipeBsBytes;  // 97 KB
 
-template <bool kAcc, bool kSel>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kSel>
+__global__ void __launch_bounds__(kPipeThreads, 2)
     proxy_pipe_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                       float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                       const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
                       int units, uint8_t* __restrict__ rowflag, int32_t* __restrict__ dev_status) {
   extern __shared__ __align__(16) uint8_t sm[];
-  float4* pst = reinterpret_cast<float4*>(sm);                                // [S][kRT][256]
-  uint32_t* wst = reinterpret_cast<uint32_t*>(sm + kPipeStages * kPBytes);    // [S][kRT][256]
-  uint8_t* dbraw = sm + kPipeStages * (kPBytes + kWBytes);                    // [S][32][kDbStride]
-  uint16_t* As = reinterpret_cast<uint16_t*>(dbraw + kPipeStages * kDbRawBytes);  // [2][r][256]
-  float2* Bs = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(As) + 2 * kPipeAsBytes);  // [r][32]
+  float4* pst = reinterpret_cast<float4*>(sm);                                 // [8][2][128]
+  uint2* wst = reinterpret_cast<uint2*>(sm + kPipePBytes);                     // [8][128]
+  uint8_t* dbraw = sm + kPipePBytes + kPipeWBytes;                             // [2][32][kDbStride]
+  uint16_t* As = reinterpret_cast<uint16_t*>(dbraw + 2 * kPipeDbBytes);       // [r][256]
+  float2* Bs = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(As) + kPipeAsBytes);  // [r][32]
 
   const int tid = threadIdx.x;
-  const int tc = tid & 63;  // columns c0 + 4*tc .. +3
-  const int tr = tid >> 6;  // rows r0 + 8*tr .. +7
+  const int lane = tid & 31;
+  const int tr = tid >> 5;  // rows r0 + 8*tr .. +7
   const int u_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * units / gridDim.x);
   const int u_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * units / gridDim.x);
   if (u_begin >= u_end) return;
   const int chunks_per_row = r / 8;  // 16-byte chunks of one dB_inc row
 
-  // this thread's P / Wq slices and (its share of) the dB_inc rows of tile v
-  auto issue_tile = [&](int v, int slot) {
-    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kTileRows;
-    const int64_t col = static_cast<int64_t>(v / row_groups) * kTileCols + 4 * tc;
+  auto tile_r0 = [&](int v) { return static_cast<int64_t>(v % row_groups) * kPipeRows; };
+  auto tile_col = [&](int v) {
+    return static_cast<int64_t>(v / row_groups) * kTileCols + kPipeCT * lane;
+  };
+  // this thread's P and Wq slices of tile v (read back only by this thread)
+  auto issue_pw = [&](int v) {
+    const int64_t r0 = tile_r0(v), col = tile_col(v);
     const bool col_ok = col < K;
 #pragma unroll
-    for (int j = 0; j < kRT; ++j) {
-      const int64_t n = r0 + tr * kRT + j;
+    for (int j = 0; j < kPipeRT; ++j) {
+      const int64_t n = r0 + tr * kPipeRT + j;
       const bool ok = col_ok && n < N;
-      cp_async16(pst + (slot * kRT + j) * kThreads + tid,
-                 ok ? static_cast<const void*>(proxy + n * K + col) : proxy, ok ? 16u : 0u);
-      if (kSel)
-        cp_async4(wst + (slot * kRT + j) * kThreads + tid,
-                  ok ? static_cast<const void*>(wq + n * K + col) : wq, ok ? 4u : 0u);
+      const float* src = ok ? proxy + n * K + col : proxy;
+      cp_async16(pst + (2 * j) * kPipeThreads + tid, src, ok ? 16u : 0u);
+      cp_async16(pst + (2 * j + 1) * kPipeThreads + tid, ok ? src + 4 : proxy, ok ? 16u : 0u);
+      if (kSel) {
+        const uint8_t* wsrc = ok ? wq + n * K + col : wq;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(wst + j * kPipeThreads + tid)),
+                     "l"(wsrc), "r"(ok ? 8u : 0u)
+                     : "memory");
+      }
     }
-    if (kAcc && tid < kTileRows * chunks_per_row) {
-      const int row = tid / chunks_per_row, c8 = tid % chunks_per_row;
+  };
+  // dB_inc rows of tile v -> dbraw[buf] (shared by the CTA)
+  auto issue_db = [&](int v, int buf) {
+    const int64_t r0 = tile_r0(v);
+    for (int e = tid; e < kPipeRows * chunks_per_row; e += kPipeThreads) {
+      const int row = e / chunks_per_row, c8 = e % chunks_per_row;
       const int64_t n = r0 + row;
       const bool ok = n < N;
-      cp_async16(dbraw + slot * kDbRawBytes + row * kDbStride + 16 * c8,
+      cp_async16(dbraw + buf * kPipeDbBytes + row * kDbStride + 16 * c8,
                  ok ? static_cast<const void*>(dB_inc + n * r + 8 * c8) : dB_inc, ok ? 16u : 0u);
     }
   };
-  // A[0:r, cb*256 : cb*256+256] -> As[buf] (zero beyond K)
-  auto issue_A = [&](int cb, int buf) {
-    uint16_t* dst = As + buf * (kPipeAsBytes / 2);
-    for (int e = tid; e < r * (kTileCols / 8); e += kThreads) {
+  // A[0:r, cb*256 : cb*256+256] -> As (zero beyond K)
+  auto issue_A = [&](int cb) {
+    for (int e = tid; e < r * (kTileCols / 8); e += kPipeThreads) {
       const int i = e / (kTileCols / 8), c8 = e % (kTileCols / 8);
       const int64_t gc = static_cast<int64_t>(cb) * kTileCols + 8 * c8;
       const bool ok = gc < K;
-      cp_async16(dst + i * kTileCols + 8 * c8,
+      cp_async16(As + i * kTileCols + 8 * c8,
                  ok ? static_cast<const void*>(A + static_cast<int64_t>(i) * K + gc) : A,
                  ok ? 16u : 0u);
     }
   };
 
-  // prologue: groups A(u_begin), G(u_begin), G(u_begin + 1)
-  if (kAcc) issue_A(u_begin / row_groups, 0);
-  cp_async_commit();
-  issue_tile(u_begin, 0);
-  cp_async_commit();
-  if (u_begin + 1 < u_end) issue_tile(u_begin + 1, 1);
+  // prologue: dB_inc rows of the first tile
+  issue_db(u_begin, 0);
   cp_async_commit();
 
   const float s_w = kSel ? *s_w_ptr : 1.0f;
-  bool nonfinite = false;
-  int abuf = 0;
-  int slot = 0;
+  uint32_t maxmag = 0;  // largest |P'| bit pattern: >= 0x7F800000 means inf or NaN
+  int cur_cb = -1, dbuf = 0;
   for (int v = u_begin; v < u_end; ++v) {
-    // outstanding: ..., A(v), G(v), [A(v+1)?], G(v+1): all but the newest have landed
-    cp_async_wait_all_but_newest();
-    if (kAcc) {
-      __syncthreads();  // every thread's copies for v visible; unit v-1 finished everywhere
-      // dB_inc rows of tile v -> (b, b) pairs, [i][row]: 8 ranks per thread
-      const uint8_t* raw = dbraw + slot * kDbRawBytes;
-      for (int e = tid; e < kTileRows * chunks_per_row; e += kThreads) {
-        const int row = e % kTileRows, c8 = e / kTileRows;
+    cp_async_wait_all();  // dB_inc rows of tile v (this thread's copies)
+    __syncthreads();      // everyone's copies visible; tile v-1 finished everywhere
+    // groups, oldest first: A (empty unless the column block changes), P / Wq of
+    // tile v, dB_inc rows of tile v+1
+    const int cb = v / row_groups;
+    const bool new_block = cb != cur_cb;
+    if (new_block) issue_A(cb);
+    cp_async_commit();
+    issue_pw(v);
+    cp_async_commit();
+    if (v + 1 < u_end) issue_db(v + 1, dbuf ^ 1);
+    cp_async_commit();
+    cur_cb = cb;
+    // dB_inc rows of tile v -> (b, b) pairs, [i][row]
+    {
+      const uint8_t* raw = dbraw + dbuf * kPipeDbBytes;
+      for (int e = tid; e < kPipeRows * chunks_per_row; e += kPipeThreads) {
+        const int row = e % kPipeRows, c8 = e / kPipeRows;
         const uint4 q = *reinterpret_cast<const uint4*>(raw + row * kDbStride + 16 * c8);
         const uint32_t wds[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           const float f0 = __uint_as_float(wds[h] << 16);
           const float f1 = __uint_as_float(wds[h] & 0xFFFF0000u);
-          Bs[(8 * c8 + 2 * h) * kTileRows + row] = make_float2(f0, f0);
-          Bs[(8 * c8 + 2 * h + 1) * kTileRows + row] = make_float2(f1, f1);
+          Bs[(8 * c8 + 2 * h) * kPipeRows + row] = make_float2(f0, f0);
+          Bs[(8 * c8 + 2 * h + 1) * kPipeRows + row] = make_float2(f1, f1);
         }
       }
     }
-    // prefetch: A of the next tile's column block when it changes, then tile v+2
-    int next_abuf = abuf;
-    if (kAcc && v + 1 < u_end && (v + 1) / row_groups != v / row_groups) {
-      next_abuf = abuf ^ 1;
-      issue_A((v + 1) / row_groups, next_abuf);
-    }
-    cp_async_commit();
-    if (v + 2 < u_end) issue_tile(v + 2, slot == 0 ? 2 : slot - 1);
-    cp_async_commit();
+    if (new_block) cp_async_wait_group<2>();  // this thread's share of A has landed
+    __syncthreads();                           // Bs and A complete
 
-    float2 acc[kRT][2];
+    float2 acc[kPipeRT][4];
 #pragma unroll
-    for (int j = 0; j < kRT; ++j) acc[j][0] = acc[j][1] = make_float2(0.0f, 0.0f);
-    if constexpr (kAcc) {
-      __syncthreads();  // Bs complete
-      const uint16_t* arow = As + abuf * (kPipeAsBytes / 2) + 4 * tc;
-      const float2* brow = Bs + tr * kRT;
+    for (int j = 0; j < kPipeRT; ++j)
+#pragma unroll
+      for (int h = 0; h < 4; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
+    const uint16_t* arow = As + kPipeCT * lane;
+    const float2* brow = Bs + tr * kPipeRT;
 #pragma unroll 4
-      for (int i = 0; i < r; ++i) {
-        const uint2 a2 = *reinterpret_cast<const uint2*>(arow + i * kTileCols);
-        const float2 a01 = make_float2(__uint_as_float(a2.x << 16), __uint_as_float(a2.x & 0xFFFF0000u));
-        const float2 a23 = make_float2(__uint_as_float(a2.y << 16), __uint_as_float(a2.y & 0xFFFF0000u));
-        float2 bb[kRT];
+    for (int i = 0; i < r; ++i) {
+      const uint4 a4 = *reinterpret_cast<const uint4*>(arow + i * kTileCols);
+      const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
+      float2 av[4];
 #pragma unroll
-        for (int j = 0; j < kRT; j += 2) {
-          const float4 q = *reinterpret_cast<const float4*>(brow + i * kTileRows + j);
-          bb[j] = make_float2(q.x, q.y);
-          bb[j + 1] = make_float2(q.z, q.w);
-        }
+      for (int h = 0; h < 4; ++h)
+        av[h] = make_float2(__uint_as_float(aw[h] << 16), __uint_as_float(aw[h] & 0xFFFF0000u));
 #pragma unroll
-        for (int j = 0; j < kRT; ++j) {
-          acc[j][0] = __ffma2_rn(bb[j], a01, acc[j][0]);
-          acc[j][1] = __ffma2_rn(bb[j], a23, acc[j][1]);
+      for (int j = 0; j < kPipeRT; j += 2) {
+        const float4 q = *reinterpret_cast<const float4*>(brow + i * kPipeRows + j);
+        const float2 b0 = make_float2(q.x, q.y), b1 = make_float2(q.z, q.w);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          acc[j][h] = __ffma2_rn(b0, av[h], acc[j][h]);
+          acc[j + 1][h] = __ffma2_rn(b1, av[h], acc[j + 1][h]);
         }
       }
     }
 
     // epilogue: P' = P + D; requantize; write P' and the changed codes
-    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kTileRows;
-    const int64_t col = static_cast<int64_t>(v / row_groups) * kTileCols + 4 * tc;
+    cp_async_wait_group<1>();  // P / Wq of tile v (not dB_inc of tile v+1)
+    const int64_t r0 = tile_r0(v), col = tile_col(v);
     const bool col_ok = col < K;
 #pragma unroll
-    for (int j = 0; j < kRT; ++j) {
-      const int64_t n = r0 + tr * kRT + j;
+    for (int j = 0; j < kPipeRT; ++j) {
+      const int64_t n = r0 + tr * kPipeRT + j;
       if (!(col_ok && n < N)) continue;
-      float4 p = pst[(slot * kRT + j) * kThreads + tid];
-      if constexpr (kAcc) {
-        p.x = __fadd_rn(p.x, acc[j][0].x);
-        p.y = __fadd_rn(p.y, acc[j][0].y);
-        p.z = __fadd_rn(p.z, acc[j][1].x);
-        p.w = __fadd_rn(p.w, acc[j][1].y);
-        *reinterpret_cast<float4*>(proxy + n * K + col) = p;
-      }
-      nonfinite |= !(isfinite(p.x) && isfinite(p.y) && isfinite(p.z) && isfinite(p.w));
+      float4 p0 = pst[(2 * j) * kPipeThreads + tid];
+      float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
+      p0.x = __fadd_rn(p0.x, acc[j][0].x);
+      p0.y = __fadd_rn(p0.y, acc[j][0].y);
+      p0.z = __fadd_rn(p0.z, acc[j][1].x);
+      p0.w = __fadd_rn(p0.w, acc[j][1].y);
+      p1.x = __fadd_rn(p1.x, acc[j][2].x);
+      p1.y = __fadd_rn(p1.y, acc[j][2].y);
+      p1.z = __fadd_rn(p1.z, acc[j][3].x);
+      p1.w = __fadd_rn(p1.w, acc[j][3].y);
+      float4* dst = reinterpret_cast<float4*>(proxy + n * K + col);
+      dst[0] = p0;
+      dst[1] = p1;
+      const uint32_t mg = 0x7FFFFFFFu;
+      maxmag = max(maxmag, max(max(max(__float_as_uint(p0.x) & mg, __float_as_uint(p0.y) & mg),
+                                   max(__float_as_uint(p0.z) & mg, __float_as_uint(p0.w) & mg)),
+                               max(max(__float_as_uint(p1.x) & mg, __float_as_uint(p1.y) & mg),
+                                   max(__float_as_uint(p1.z) & mg, __float_as_uint(p1.w) & mg))));
       if constexpr (kSel) {
-        const uint32_t w = wst[(slot * kRT + j) * kThreads + tid];
-        const uint32_t cn = requantized4(w, s_w, p);
-        const uint32_t m = changed_bytes(w, cn);
-        if (m) {
-          *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
+        const uint2 w = wst[j * kPipeThreads + tid];
+        const uint32_t c0 = requantized4(w.x, s_w, p0);
+        const uint32_t c1 = requantized4(w.y, s_w, p1);
+        const uint32_t m0 = changed_bytes(w.x, c0), m1 = changed_bytes(w.y, c1);
+        if (m0 | m1) {
+          *reinterpret_cast<uint2*>(wq + n * K + col) =
+              make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
           rowflag[n] = 1;  // every writer stores the same value
         }
       }
     }
-    abuf = next_abuf;
-    slot = slot == kPipeStages - 1 ? 0 : slot + 1;
+    dbuf ^= 1;
   }
   cp_async_wait_all();
-  if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
+  if (__any_sync(0xFFFFFFFFu, maxmag >= 0x7F800000u) && lane == 0 && dev_status)
     atomicOr(dev_status, kDevNonfinite);
 }
 
@@ -445,7 +480,7 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
   return cudaGetLastError();
 }
 
-template <bool kAcc, bool kSel>
+template <bool kSel>
 cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                         const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
                         uint8_t* rowflag, int32_t* dev_status, cudaStream_t stream) {
@@ -454,12 +489,12 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   cudaGetDevice(&dev);
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(proxy_pipe_kernel<kAcc, kSel>,
+    cudaError_t e = cudaFuncSetAttribute(proxy_pipe_kernel<kSel>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kPipeSmemBytes);
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  proxy_pipe_kernel<kAcc, kSel><<<grid, kThreads, kPipeSmemBytes, stream>>>(
+  proxy_pipe_kernel<kSel><<<grid, kPipeThreads, kPipeSmemBytes, stream>>>(
       wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
       r, row_groups, units, rowflag, dev_status);
   return cudaGetLastError();
@@ -483,11 +518,12 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
                   static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
   const int rr = acc ? static_cast<int>(r) : 0;
-  const int64_t row_groups = (N + kTileRows - 1) / kTileRows;
+  const int64_t row_groups = (N + kPipeRows - 1) / kPipeRows;
   const int64_t units = row_groups * grid.x;
-  // the persistent kernel holds A and dB_inc slices of up to 64 ranks in 16-byte chunks
-  const bool pipe = rr <= kPipeRMax && rr % 8 == 0 && units <= (int64_t(1) << 30) &&
-                    di->max_smem_optin >= kPipeSmemBytes;
+  // the persistent kernel accumulates with A and dB_inc slices of up to 64
+  // ranks held in 16-byte chunks; selection alone streams through the grid kernel
+  const bool pipe = acc && rr >= 1 && rr <= kPipeRMax && rr % 8 == 0 &&
+                    units <= (int64_t(1) << 30) && di->max_smem_optin >= kPipeSmemBytes;
   if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
   uint8_t* rowflag = static_cast<uint8_t*>(workspace);
   cudaError_t e;
@@ -497,14 +533,13 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
       return e;
   }
   if (pipe) {
-    const int g = static_cast<int>(units < di->sm_count ? units : di->sm_count);
+    const int64_t resident = 2 * static_cast<int64_t>(di->sm_count);  // two CTAs per SM
+    const int g = static_cast<int>(units < resident ? units : resident);
     const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
-    if (acc && sel)
-      e = launch_pipe<true, true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
-    else if (acc)
-      e = launch_pipe<true, false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+    if (sel)
+      e = launch_pipe<true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
     else
-      e = launch_pipe<false, true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+      e = launch_pipe<false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
   } else if (acc && sel)
     e = launch_stream<true, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);
   else if (acc)

@@ -5,6 +5,8 @@
 // factor is s = 448 / max|x| and the rounding is the hardware's
 // round-to-nearest-even, saturating E4M3 conversion.
 //
+// One cooperative launch (quantize_stream_kernel, below) when the device
+// supports it; otherwise two launches:
 // Pass 1 (amax_partial_kernel): every CTA reduces a grid-stride share of the
 //   tensor with 128-bit loads.  |x| is taken on the bit pattern (sign bit
 //   cleared): for IEEE formats that order matches the order of magnitudes,
@@ -44,13 +46,10 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t v, uint32_t* red) {
   return v;
 }
 
+// This thread's share of max|x| as float32 magnitude bits (bf16 widened).
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) amax_partial_kernel(const void* __restrict__ x,
-                                                                int64_t n,
-                                                                uint32_t* __restrict__ partials) {
-  __shared__ uint32_t red[32];
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+__device__ __forceinline__ uint32_t amax_share(const void* __restrict__ x, int64_t n, int64_t tid,
+                                               int64_t stride) {
   // kUnroll independent 16-byte loads in flight per thread per iteration
   constexpr int kUnroll = 4;
   const uint32_t mask = kBF16 ? 0x7FFF7FFFu : 0x7FFFFFFFu;
@@ -90,6 +89,17 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const void* __re
     const uint32_t* s32 = reinterpret_cast<const uint32_t*>(x);
     for (int64_t e = nv * 4 + tid; e < n; e += stride) m = max(m, s32[e] & 0x7FFFFFFFu);
   }
+  return m;
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads) amax_partial_kernel(const void* __restrict__ x,
+                                                                int64_t n,
+                                                                uint32_t* __restrict__ partials) {
+  __shared__ uint32_t red[32];
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  uint32_t m = amax_share<kBF16>(x, n, tid, stride);
   m = block_max_u32(m, red);
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
 }
@@ -144,15 +154,11 @@ __device__ __forceinline__ float load1(const void* x, int64_t i) {
   }
 }
 
-template <bool kBF16>
-__global__ void __launch_bounds__(kThreads)
-    quantize_cast_kernel(const void* __restrict__ x, int64_t n,
-                         const uint32_t* __restrict__ partials, int nparts,
-                         uint8_t* __restrict__ codes, float* __restrict__ scale_out,
-                         float* __restrict__ amax_out, float* __restrict__ residual,
-                         int32_t* __restrict__ dev_status) {
-  __shared__ uint32_t red[32];
-  __shared__ float s_shared;
+// Folds the partial maxima and derives s = 448 / amax (IEEE division); CTA 0
+// publishes scale, amax and the status.  Returns s to every thread.
+__device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int nparts,
+                                                uint32_t* red, float* s_shared, float* scale_out,
+                                                float* amax_out, int32_t* dev_status) {
   uint32_t m = 0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, partials[i]);
   m = block_max_u32(m, red);
@@ -172,7 +178,7 @@ __global__ void __launch_bounds__(kThreads)
         st = kDevScaleOverflow;
       }
     }
-    s_shared = s;
+    *s_shared = s;
     if (blockIdx.x == 0) {
       *scale_out = s;
       if (amax_out) *amax_out = amax;
@@ -180,11 +186,16 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   __syncthreads();
-  const float s = s_shared;
-  const double s_d = static_cast<double>(s);
+  return *s_shared;
+}
 
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+// Casts this thread's grid-stride share: codes = E4M3(fl32(x * s)), and the
+// optional residual x - dec(code) / s (fp64, rounded once to float32).
+template <bool kBF16>
+__device__ __forceinline__ void cast_share(const void* __restrict__ x, int64_t n, float s,
+                                           uint8_t* __restrict__ codes, float* __restrict__ residual,
+                                           int64_t tid, int64_t stride) {
+  const double s_d = static_cast<double>(s);
   const int64_t ng = n / 16;
   auto convert = [&](int64_t g, const float (&v)[16]) {
     uint32_t w[4];
@@ -234,6 +245,247 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads)
+    quantize_cast_kernel(const void* __restrict__ x, int64_t n,
+                         const uint32_t* __restrict__ partials, int nparts,
+                         uint8_t* __restrict__ codes, float* __restrict__ scale_out,
+                         float* __restrict__ amax_out, float* __restrict__ residual,
+                         int32_t* __restrict__ dev_status) {
+  __shared__ uint32_t red[32];
+  __shared__ float s_shared;
+  const float s = fold_and_scale(partials, nparts, red, &s_shared, scale_out, amax_out, dev_status);
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  cast_share<kBF16>(x, n, s, codes, residual, tid, stride);
+}
+
+// ---------------------------------------------------------------- one launch
+// quantize_stream_kernel: cooperative, one CTA per SM.  Each CTA owns a
+// contiguous run of 16 KB chunks of x.  Warp 0 (one lane) streams the chunks
+// into a ring of shared-memory slots with bulk asynchronous copies; eight
+// consumer warps read each slot, then release it.  Pass 1 reduces max|x|;
+// after a grid barrier on a counter in the workspace (bounded wait) every
+// CTA folds the per-CTA maxima and pass 2 streams the same run again -- it is
+// still in L2 -- and writes the codes.
+constexpr int kChunkBytes = 16384;
+constexpr int kStreamStages = 8;                       // 128 KB in flight per SM
+constexpr int kConsumerWarps = 16;
+constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
+constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
+constexpr int kBarWords = 64;                          // counter at [0], generation at [1]; partials from [64]
+constexpr long long kBarrierBudget = 2000000000LL;    // cycles (about 1 s), then give up
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    quantize_stream_kernel(const void* __restrict__ x, int64_t n, uint32_t* __restrict__ ws,
+                           uint8_t* __restrict__ codes, float* __restrict__ scale_out,
+                           float* __restrict__ amax_out, float* __restrict__ residual,
+                           int32_t* __restrict__ dev_status) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + kStreamStages * kChunkBytes);
+  uint64_t* empty = full + kStreamStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStreamStages);
+  __shared__ uint32_t red[32];
+  __shared__ float s_shared;
+
+  constexpr int kElem = kBF16 ? 2 : 4;
+  constexpr int kPerChunk = kChunkBytes / kElem;  // elements per chunk
+  const int64_t body_bytes = (n * kElem) / 16 * 16;  // bulk-copied part; the rest is the tail
+  const int64_t nchunks = (body_bytes + kChunkBytes - 1) / kChunkBytes;
+  const int64_t c_begin = static_cast<int64_t>(blockIdx.x) * nchunks / gridDim.x;
+  const int64_t c_end = static_cast<int64_t>(blockIdx.x + 1) * nchunks / gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ct = threadIdx.x - 32;  // consumer thread index for warps 1..kConsumerWarps
+  constexpr int kConsumers = 32 * kConsumerWarps;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStreamStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  int stage = 0;
+  uint32_t phase = 0;
+  // one pass over this CTA's chunks; consume(chunk, slot) runs in the consumer threads
+  auto stream = [&](auto consume) {
+    if (warp == 0) {
+      if (lane == 0) {
+        uint32_t issued = 0, parity = 0;
+        for (int64_t c = c_begin; c < c_end; ++c) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) {
+            *abort_flag = 1;
+            if (dev_status) atomicOr(dev_status, kDevTimeout);
+            break;
+          }
+          const int64_t off = c * kChunkBytes;
+          const uint32_t bytes = static_cast<uint32_t>(
+              body_bytes - off < kChunkBytes ? body_bytes - off : kChunkBytes);
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          bulk_load(sm + stage * kChunkBytes, static_cast<const uint8_t*>(x) + off, bytes, &full[stage]);
+          issued |= 1u << stage;
+          parity = (parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStreamStages) { stage = 0; phase ^= 1; }
+        }
+        // nothing may still be landing when the pass (or the CTA) ends
+        for (int st = 0; st < kStreamStages; ++st)
+          if (issued & (1u << st)) mbar_wait_budget(&full[st], (parity >> st) & 1u);
+      }
+      __syncwarp();  // the warp reaches the CTA barrier below together
+    } else {
+      for (int64_t c = c_begin; c < c_end; ++c) {
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[stage], phase, abort_flag));
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            if (dev_status) atomicOr(dev_status, kDevTimeout);
+          }
+          break;
+        }
+        consume(c, sm + stage * kChunkBytes);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == kStreamStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    // both roles leave the pass with the same ring position
+    __syncthreads();
+  };
+
+  // ---- pass 1: max|x| (bit patterns, as in amax_share)
+  const uint32_t mask = kBF16 ? 0x7FFF7FFFu : 0x7FFFFFFFu;
+  uint32_t m = 0;
+  stream([&](int64_t c, const uint8_t* slot) {
+    const int64_t off = c * kChunkBytes;
+    const int64_t valid = body_bytes - off < kChunkBytes ? body_bytes - off : kChunkBytes;
+#pragma unroll
+    for (int k = 0; k < kChunkBytes / 16 / kConsumers; ++k) {
+      const int u = k * kConsumers + ct;  // 16-byte unit of the chunk
+      if (static_cast<int64_t>(u) * 16 < valid) {
+        const uint4 q = reinterpret_cast<const uint4*>(slot)[u];
+        const uint32_t w[4] = {q.x & mask, q.y & mask, q.z & mask, q.w & mask};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if constexpr (kBF16) m = max(m, max(w[j] & 0xFFFFu, w[j] >> 16) << 16);
+          else m = max(m, w[j]);
+        }
+      }
+    }
+  });
+  // tail elements past the last whole 16 bytes (fewer than 8): the last CTA
+  const int64_t tail0 = body_bytes / kElem;
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 32) {
+    for (int64_t e = tail0; e < n; ++e) {
+      if constexpr (kBF16) m = max(m, (reinterpret_cast<const uint16_t*>(x)[e] & 0x7FFFu) << 16);
+      else m = max(m, reinterpret_cast<const uint32_t*>(x)[e] & 0x7FFFFFFFu);
+    }
+  }
+  m = block_max_u32(m, red);
+
+  uint32_t* partials = ws + kBarWords;
+  if (threadIdx.x == 0) {
+    // grid barrier: the launch is cooperative, so every CTA is resident.
+    // Release/acquire at gpu scope orders the partials around it.
+    uint32_t gen0;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen0) : "l"(ws + 1) : "memory");
+    // (read before arriving: the generation cannot move until every CTA has arrived)
+    partials[blockIdx.x] = m;
+    uint32_t prev;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ws) : "memory");
+    if (prev == gridDim.x - 1) {
+      ws[0] = 0u;  // ready for the next launch
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ws + 1), "r"(gen0 + 1u) : "memory");
+    } else {
+      const long long t0 = clock64();
+      while (true) {
+        uint32_t g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(ws + 1) : "memory");
+        if (g != gen0) break;
+        if (clock64() - t0 > kBarrierBudget) {
+          if (dev_status) atomicOr(dev_status, kDevTimeout);
+          break;
+        }
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  const float s = fold_and_scale(partials, gridDim.x, red, &s_shared, scale_out, amax_out, dev_status);
+  const double s_d = static_cast<double>(s);
+
+  // ---- pass 2: codes (and the optional residual)
+  stream([&](int64_t c, const uint8_t* slot) {
+    const int64_t off = c * kChunkBytes;
+    const int64_t valid = body_bytes - off < kChunkBytes ? body_bytes - off : kChunkBytes;
+    const int64_t e0 = c * kPerChunk;  // first element of the chunk
+#pragma unroll
+    for (int k = 0; k < kChunkBytes / 16 / kConsumers; ++k) {
+      const int u = k * kConsumers + ct;
+      if (static_cast<int64_t>(u) * 16 >= valid) continue;
+      const uint4 q = reinterpret_cast<const uint4*>(slot)[u];
+      constexpr int kE = 16 / kElem;  // elements in this unit: 8 (bf16) or 4 (fp32)
+      float v[kE];
+      if constexpr (kBF16) {
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[2 * j] = __uint_as_float(w[j] << 16);
+          v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+      } else {
+        v[0] = __uint_as_float(q.x);
+        v[1] = __uint_as_float(q.y);
+        v[2] = __uint_as_float(q.z);
+        v[3] = __uint_as_float(q.w);
+      }
+      uint32_t cw[kE / 4];
+#pragma unroll
+      for (int j = 0; j < kE / 4; ++j) {
+        const uint32_t c01 = e4m3x2(__fmul_rn(v[4 * j], s), __fmul_rn(v[4 * j + 1], s));
+        const uint32_t c23 = e4m3x2(__fmul_rn(v[4 * j + 2], s), __fmul_rn(v[4 * j + 3], s));
+        cw[j] = c01 | (c23 << 16);
+      }
+      const int64_t e = e0 + static_cast<int64_t>(u) * kE;
+      if constexpr (kBF16) *reinterpret_cast<uint2*>(codes + e) = make_uint2(cw[0], cw[1]);
+      else *reinterpret_cast<uint32_t*>(codes + e) = cw[0];
+      if (residual) {
+#pragma unroll
+        for (int j = 0; j < kE; j += 2) {
+          const float2 d = e4m3x2_value(cw[j >> 2] >> (8 * (j & 3)));
+          residual[e + j] = static_cast<float>(static_cast<double>(v[j]) - static_cast<double>(d.x) / s_d);
+          residual[e + j + 1] =
+              static_cast<float>(static_cast<double>(v[j + 1]) - static_cast<double>(d.y) / s_d);
+        }
+      }
+    }
+  });
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 32) {
+    for (int64_t e = tail0; e < n; ++e) {
+      float v;
+      if constexpr (kBF16) v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(x)[e]) << 16);
+      else v = reinterpret_cast<const float*>(x)[e];
+      const uint32_t c = e4m3x2(__fmul_rn(v, s), 0.0f) & 0xFFu;
+      codes[e] = static_cast<uint8_t>(c);
+      if (residual) {
+        const float2 d = e4m3x2_value(c);
+        residual[e] = static_cast<float>(static_cast<double>(v) - static_cast<double>(d.x) / s_d);
+      }
+    }
+  }
+}
+
 int amax_blocks(int64_t n, int sm_count) {
   const int64_t per_block = static_cast<int64_t>(kThreads) * 64;  // >= 64 elements per thread
   int64_t b = (n + per_block - 1) / per_block;
@@ -247,7 +499,7 @@ int amax_blocks(int64_t n, int sm_count) {
 
 size_t quantize_workspace_bytes(int64_t n) {
   (void)n;
-  return 4096 * sizeof(uint32_t);  // amax partials (at most 4 per SM, up to 1024 SMs)
+  return 4096 * sizeof(uint32_t);  // barrier words + amax partials (at most 4032 CTAs)
 }
 
 cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* codes,
@@ -255,7 +507,46 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
                             void* workspace, cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
-  uint32_t* partials = static_cast<uint32_t*>(workspace);
+  uint32_t* ws = static_cast<uint32_t*>(workspace);
+  if (di->coop_launch && di->max_smem_optin >= kStreamSmemBytes) {
+    static int configured_mask[2] = {0, 0};  // per dtype, one bit per device ordinal < 31
+    const int dev = di->device;
+    const int bit = dev < 31 ? (1 << dev) : 0;
+    int& cm = configured_mask[is_bf16 ? 1 : 0];
+    if (!bit || !(__atomic_load_n(&cm, __ATOMIC_ACQUIRE) & bit)) {
+      cudaError_t e = is_bf16 ? cudaFuncSetAttribute(quantize_stream_kernel<true>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     kStreamSmemBytes)
+                              : cudaFuncSetAttribute(quantize_stream_kernel<false>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     kStreamSmemBytes);
+      if (e != cudaSuccess) return e;
+      if (bit) __atomic_fetch_or(&cm, bit, __ATOMIC_ACQ_REL);
+    }
+    // one CTA per SM, never more CTAs than chunks (at least one)
+    const int64_t body = (n * (is_bf16 ? 2 : 4)) / 16 * 16;
+    int64_t chunks = (body + kChunkBytes - 1) / kChunkBytes;
+    int grid = static_cast<int>(chunks < di->sm_count ? (chunks > 0 ? chunks : 1) : di->sm_count);
+    if (grid > 4096 - kBarWords) grid = 4096 - kBarWords;
+    cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kStreamThreads);
+    cfg.dynamicSmemBytes = kStreamSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (is_bf16)
+      return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<true>, x, n, ws, codes, scale, amax,
+                                residual, dev_status);
+    return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<false>, x, n, ws, codes, scale, amax,
+                              residual, dev_status);
+  }
+  uint32_t* partials = ws;
   const int pb = amax_blocks(n, di->sm_count);
   const int64_t per_cast_block = static_cast<int64_t>(kThreads) * 16 * 4;
   int64_t cb = (n + per_cast_block - 1) / per_cast_block;

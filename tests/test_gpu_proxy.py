@@ -56,7 +56,7 @@ def _compare(gpu, ref):
     (70, 2048, 64),     # rows not a multiple of the 32-row group
     (40, 11008, 16),    # the down projection's K (43 column blocks)
     (64, 512, 1100),    # large rank: many staging chunks
-    (96, 16384, 64),    # persistent CTAs whose tiles span two column blocks
+    (160, 32768, 64),   # persistent CTAs whose tiles span column blocks
     (20, 65536, 8),     # one row group: every tile starts a new column block
 ])
 def test_accumulate_and_select(cuda_device, N, K, r):
