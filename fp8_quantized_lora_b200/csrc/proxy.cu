@@ -111,6 +111,12 @@ __device__ __forceinline__ uint32_t zero_bytes(uint32_t x) {
   return ~(t | x) & 0x80808080u;
 }
 
+// 0xFF in every byte of `a` that holds a NaN code.
+__device__ __forceinline__ uint32_t nan_bytes(uint32_t a) {
+  const uint32_t mag = 0x7F7F7F7Fu;
+  return (zero_bytes((a & mag) ^ mag) >> 7) * 0xFFu;
+}
+
 // Byte mask (0xFF per byte) of the codes whose value changes from `a` to `b`.
 // Two codes hold the same value when they are identical non-NaN codes or
 // both zero (either sign); a NaN code never holds the same value.
@@ -128,8 +134,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     proxy_stream_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                         float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                         const uint16_t* __restrict__ A, int64_t N, int64_t K, int r,
-                        uint8_t* __restrict__ rowflag, int32_t* __restrict__ dev_status) {
+                        uint8_t* __restrict__ rowflag, int32_t* __restrict__ n_selected,
+                        int32_t* __restrict__ dev_status) {
   extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int tile_flag[kTileRows];  // a code of the row changed in this tile
   uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kIChunk][256]
   float2* Bs = reinterpret_cast<float2*>(sm + kAsBytes);                       // [kIChunk][32]
   float4* pbuf = reinterpret_cast<float4*>(sm + kAsBytes + kBsBytes);          // [kRT][256]
@@ -214,6 +222,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const float s_w = kSel ? *s_w_ptr : 1.0f;
   bool nonfinite = false;
+  if (kSel) {
+    if (tid < kTileRows) tile_flag[tid] = 0;
+    if (n_selected && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *n_selected = 0;  // the clear pass counts
+    __syncthreads();
+  }
 #pragma unroll
   for (int j = 0; j < kRT; ++j) {
     const int64_t n = r0 + tr * kRT + j;
@@ -233,9 +246,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t m = changed_bytes(w, cn);
       if (m) {
         *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
-        rowflag[n] = 1;  // every writer stores the same value
+        tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
       }
     }
+  }
+  if (kSel) {
+    // this tile's verdict for each of its rows, written whether or not a code changed
+    __syncthreads();
+    const int64_t ncb = gridDim.x;
+    if (tid < kTileRows && r0 + tid < N) rowflag[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint8_t>(tile_flag[tid]);
   }
   if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
     atomicOr(dev_status, kDevNonfinite);
@@ -266,7 +285,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     proxy_pipe_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                       float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                       const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
-                      int units, uint8_t* __restrict__ rowflag, int32_t* __restrict__ dev_status) {
+                      int units, int ncb, uint8_t* __restrict__ rowflag,
+                      int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status) {
   extern __shared__ __align__(16) uint8_t sm[];
   float4* pst = reinterpret_cast<float4*>(sm);                                 // [8][2][128]
   uint2* wst = reinterpret_cast<uint2*>(sm + kPipePBytes);                     // [8][128]
@@ -333,6 +353,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   cp_async_commit();
 
   const float s_w = kSel ? *s_w_ptr : 1.0f;
+  if (kSel && n_selected && blockIdx.x == 0 && threadIdx.x == 0) *n_selected = 0;  // the clear pass counts
   uint32_t maxmag = 0;  // largest |P'| bit pattern: >= 0x7F800000 means inf or NaN
   int cur_cb = -1, dbuf = 0;
   for (int v = u_begin; v < u_end; ++v) {
@@ -401,36 +422,45 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     const bool col_ok = col < K;
 #pragma unroll
     for (int j = 0; j < kPipeRT; ++j) {
-      const int64_t n = r0 + tr * kPipeRT + j;
-      if (!(col_ok && n < N)) continue;
-      float4 p0 = pst[(2 * j) * kPipeThreads + tid];
-      float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
-      p0.x = __fadd_rn(p0.x, acc[j][0].x);
-      p0.y = __fadd_rn(p0.y, acc[j][0].y);
-      p0.z = __fadd_rn(p0.z, acc[j][1].x);
-      p0.w = __fadd_rn(p0.w, acc[j][1].y);
-      p1.x = __fadd_rn(p1.x, acc[j][2].x);
-      p1.y = __fadd_rn(p1.y, acc[j][2].y);
-      p1.z = __fadd_rn(p1.z, acc[j][3].x);
-      p1.w = __fadd_rn(p1.w, acc[j][3].y);
-      float4* dst = reinterpret_cast<float4*>(proxy + n * K + col);
-      dst[0] = p0;
-      dst[1] = p1;
-      const uint32_t mg = 0x7FFFFFFFu;
-      maxmag = max(maxmag, max(max(max(__float_as_uint(p0.x) & mg, __float_as_uint(p0.y) & mg),
-                                   max(__float_as_uint(p0.z) & mg, __float_as_uint(p0.w) & mg)),
-                               max(max(__float_as_uint(p1.x) & mg, __float_as_uint(p1.y) & mg),
-                                   max(__float_as_uint(p1.z) & mg, __float_as_uint(p1.w) & mg))));
-      if constexpr (kSel) {
-        const uint2 w = wst[j * kPipeThreads + tid];
-        const uint32_t c0 = requantized4(w.x, s_w, p0);
-        const uint32_t c1 = requantized4(w.y, s_w, p1);
-        const uint32_t m0 = changed_bytes(w.x, c0), m1 = changed_bytes(w.y, c1);
-        if (m0 | m1) {
-          *reinterpret_cast<uint2*>(wq + n * K + col) =
-              make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
-          rowflag[n] = 1;  // every writer stores the same value
+      const int64_t n = r0 + tr * kPipeRT + j;  // the warp's row: uniform across the warp
+      bool changed = false;
+      if (col_ok && n < N) {
+        float4 p0 = pst[(2 * j) * kPipeThreads + tid];
+        float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
+        p0.x = __fadd_rn(p0.x, acc[j][0].x);
+        p0.y = __fadd_rn(p0.y, acc[j][0].y);
+        p0.z = __fadd_rn(p0.z, acc[j][1].x);
+        p0.w = __fadd_rn(p0.w, acc[j][1].y);
+        p1.x = __fadd_rn(p1.x, acc[j][2].x);
+        p1.y = __fadd_rn(p1.y, acc[j][2].y);
+        p1.z = __fadd_rn(p1.z, acc[j][3].x);
+        p1.w = __fadd_rn(p1.w, acc[j][3].y);
+        float4* dst = reinterpret_cast<float4*>(proxy + n * K + col);
+        dst[0] = p0;
+        dst[1] = p1;
+        const uint32_t mg = 0x7FFFFFFFu;
+        maxmag = max(maxmag, max(max(max(__float_as_uint(p0.x) & mg, __float_as_uint(p0.y) & mg),
+                                     max(__float_as_uint(p0.z) & mg, __float_as_uint(p0.w) & mg)),
+                                 max(max(__float_as_uint(p1.x) & mg, __float_as_uint(p1.y) & mg),
+                                     max(__float_as_uint(p1.z) & mg, __float_as_uint(p1.w) & mg))));
+        if constexpr (kSel) {
+          const uint2 w = wst[j * kPipeThreads + tid];
+          const uint32_t c0 = requantized4(w.x, s_w, p0);
+          const uint32_t c1 = requantized4(w.y, s_w, p1);
+          // identical words change only where they hold NaN codes (the common case)
+          const uint32_t m0 = c0 == w.x ? nan_bytes(w.x) : changed_bytes(w.x, c0);
+          const uint32_t m1 = c1 == w.y ? nan_bytes(w.y) : changed_bytes(w.y, c1);
+          if (m0 | m1) {
+            *reinterpret_cast<uint2*>(wq + n * K + col) =
+                make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
+            changed = true;
+          }
         }
+      }
+      if constexpr (kSel) {
+        // the tile's verdict for row n, written whether or not a code changed
+        const bool any = __any_sync(0xFFFFFFFFu, changed);
+        if (lane == 0 && n < N) rowflag[n * ncb + v / row_groups] = any ? 1 : 0;
       }
     }
     dbuf ^= 1;
@@ -443,12 +473,14 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 constexpr int kClearThreads = 256;
 
 __global__ void __launch_bounds__(kClearThreads)
-    proxy_clear_kernel(float* __restrict__ proxy, int64_t N, int64_t K,
+    proxy_clear_kernel(float* __restrict__ proxy, int64_t N, int64_t K, int ncb,
                        const uint8_t* __restrict__ rowflag, uint8_t* __restrict__ row_mask,
                        int32_t* __restrict__ n_selected) {
   int count = 0;
   for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
-    const int sel = rowflag[n];
+    // OR of the row's per-column-block verdicts (every CTA thread computes it)
+    int sel = 0;
+    for (int c = 0; c < ncb; ++c) sel |= rowflag[n * ncb + c];
     if (threadIdx.x == 0) {
       if (row_mask) row_mask[n] = static_cast<uint8_t>(sel);
       count += sel;
@@ -463,7 +495,7 @@ __global__ void __launch_bounds__(kClearThreads)
 template <bool kAcc, bool kSel>
 cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                           const void* A, int64_t N, int64_t K, int r, uint8_t* rowflag,
-                          int32_t* dev_status, cudaStream_t stream) {
+                          int32_t* n_selected, int32_t* dev_status, cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -476,14 +508,15 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
   }
   proxy_stream_kernel<kAcc, kSel><<<grid, kThreads, kSmemBytes, stream>>>(
       wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
-      r, rowflag, dev_status);
+      r, rowflag, n_selected, dev_status);
   return cudaGetLastError();
 }
 
 template <bool kSel>
 cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                         const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
-                        uint8_t* rowflag, int32_t* dev_status, cudaStream_t stream) {
+                        int ncb, uint8_t* rowflag, int32_t* n_selected, int32_t* dev_status,
+                        cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -496,15 +529,15 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   }
   proxy_pipe_kernel<kSel><<<grid, kPipeThreads, kPipeSmemBytes, stream>>>(
       wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
-      r, row_groups, units, rowflag, dev_status);
+      r, row_groups, units, ncb, rowflag, n_selected, dev_status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t proxy_workspace_bytes(int64_t N, int64_t K) {
-  (void)K;
-  return align_up(static_cast<size_t>(N), 256);  // one selection flag per row
+  // one verdict byte per (row, 256-column block)
+  return align_up(static_cast<size_t>(N) * static_cast<size_t>((K + kTileCols - 1) / kTileCols), 256);
 }
 
 cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
@@ -525,30 +558,33 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   const bool pipe = acc && rr >= 1 && rr <= kPipeRMax && rr % 8 == 0 &&
                     units <= (int64_t(1) << 30) && di->max_smem_optin >= kPipeSmemBytes;
   if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
+  // per (row, 256-column block) verdicts, each written by the tile that owns it:
+  // nothing to clear beforehand
   uint8_t* rowflag = static_cast<uint8_t*>(workspace);
+  const int ncb = static_cast<int>(grid.x);
   cudaError_t e;
-  if (sel) {
-    if ((e = cudaMemsetAsync(rowflag, 0, static_cast<size_t>(N), stream)) != cudaSuccess) return e;
-    if (n_selected && (e = cudaMemsetAsync(n_selected, 0, sizeof(int32_t), stream)) != cudaSuccess)
-      return e;
-  }
   if (pipe) {
     const int64_t resident = 2 * static_cast<int64_t>(di->sm_count);  // two CTAs per SM
     const int g = static_cast<int>(units < resident ? units : resident);
     const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
     if (sel)
-      e = launch_pipe<true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+      e = launch_pipe<true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
+                            dev_status, stream);
     else
-      e = launch_pipe<false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, rowflag, dev_status, stream);
+      e = launch_pipe<false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
+                             dev_status, stream);
   } else if (acc && sel)
-    e = launch_stream<true, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);
+    e = launch_stream<true, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                  dev_status, stream);
   else if (acc)
-    e = launch_stream<true, false>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);
+    e = launch_stream<true, false>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                   dev_status, stream);
   else
-    e = launch_stream<false, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, dev_status, stream);
+    e = launch_stream<false, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                   dev_status, stream);
   if (e != cudaSuccess || !sel) return e;
   int64_t blocks = N < static_cast<int64_t>(di->sm_count) * 8 ? N : static_cast<int64_t>(di->sm_count) * 8;
-  proxy_clear_kernel<<<static_cast<int>(blocks), kClearThreads, 0, stream>>>(proxy, N, K, rowflag,
+  proxy_clear_kernel<<<static_cast<int>(blocks), kClearThreads, 0, stream>>>(proxy, N, K, ncb, rowflag,
                                                                              row_mask, n_selected);
   return cudaGetLastError();
 }
