@@ -171,30 +171,34 @@ class Step:
         # initial quantization of the backbone (not part of the step)
         F.falqon_quantize(self.W, codes=self.wq, scale=self.s_w, amax=self.amax,
                           dev_status=self.status, workspace=self.ws_q2)
-        # library kernels per step: quantize X (2) + forward (1) + quantize dY (2)
-        # + adapter products T, dB, U, dA (4) + dX (1) + proxy stream and clear (2)
-        self.launches_per_step = 2 + 1 + 2 + 4 + 1 + 2
+        # library kernels per step: quantize X (1) + forward (1) + quantize dY (1)
+        # + adapter products (T with U, dB with dA: 2) + dX (1) + proxy update and clear (2)
+        self.launches_per_step = 1 + 1 + 1 + 2 + 1 + 2
 
-    PHASES = ("quantX+fwd", "quantdY+adapters", "dX", "sgd", "proxy")
+    # one C-ABI call per phase (the caller's SGD: two torch ops)
+    PHASES = ("quantX", "fwd", "quantdY", "adapters", "dX", "sgd", "proxy")
 
     def phase(self, slot, k):
         """Enqueues phase k of one step on the current stream."""
         F, t = self.F, self.torch
-        if k == 0:
+        name = self.PHASES[k]
+        if name == "quantX":
             F.falqon_quantize(self.X[slot], codes=self.xq, scale=self.s_x, amax=self.amax,
                               dev_status=self.status, workspace=self.ws_q)
+        elif name == "fwd":
             F.falqon_linear_fwd(self.xq, self.s_x, self.wq, self.s_w, y=self.y,
                                 dev_status=self.status)
-        elif k == 1:
+        elif name == "quantdY":
             F.falqon_quantize(self.dY[slot], codes=self.dyq, scale=self.s_dy, amax=self.amax,
                               dev_status=self.status, workspace=self.ws_q)
+        elif name == "adapters":
             F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, self.xq, self.s_x, self.A,
                                 self.B, dx=None, dA=self.dA, dB=self.dB, dev_status=self.status,
                                 workspace=self.ws_bwd)
-        elif k == 2:
+        elif name == "dX":
             F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, None, None, None, None,
                                 dx=self.dx, dA=None, dB=None, dev_status=self.status)
-        elif k == 3:
+        elif name == "sgd":
             # the caller's optimizer: plain SGD on B; the proxy receives the increment
             t.mul(self.dB, -self.lr, out=self.dB_inc)
             self.B.add_(self.dB_inc)
@@ -209,18 +213,34 @@ class Step:
             self.phase(slot, k)
 
 
+# FP32 FMA peak of the CUDA cores (the proxy's bound at large r): 148 SMs x 128
+# FP32 lanes x 2 flops x 1.965 GHz (the B200's boost clock)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def _phase_work(st):
-    """Algorithmic flops / bytes of each phase (measurement section)."""
+    """Algorithmic work and bound of each phase: flops, bytes (each tensor
+    once at its storage width), the roofline that bounds it and its kernels."""
     M, N, K, r = st.M, st.N, st.K, st.r
+    proxy_flops, proxy_bytes = 2.0 * N * K * r, 9.0 * N * K + 2.0 * r * (N + K)
+    # the proxy is bound by the FP32 FMA pipe when its FMA time exceeds its HBM time
+    proxy_alu = proxy_flops / (FP32_FMA_TFLOPS * 1e12) > proxy_bytes / (_peaks()["hbm_gbs"] * 1e9)
     return {
-        # quantize X (read bf16, read again from L2 or HBM, write codes) + forward GEMM
-        "quantX+fwd": {"flops": 2.0 * M * N * K, "bytes": 3.0 * M * K + M * K + N * K + 2.0 * M * N},
-        # quantize dY + adapter GEMMs (T, dB, U, dA): codes re-read by each product
-        "quantdY+adapters": {"flops": 8.0 * M * r * (N + K) / 2.0,
-                             "bytes": 3.0 * M * N + 2.0 * (M * K + M * N) + 2.0 * r * (N + K)},
-        "dX": {"flops": 2.0 * M * N * K, "bytes": M * N + N * K + 2.0 * M * K},
-        "sgd": {"flops": 0.0, "bytes": 8.0 * N * r},
-        "proxy": {"flops": 2.0 * N * K * r, "bytes": 9.0 * N * K + 2.0 * r * (N + K)},
+        "quantX": {"flops": 0.0, "bytes": 3.0 * M * K, "bound": "hbm",
+                   "kernels": "quantize_stream_kernel"},
+        "fwd": {"flops": 2.0 * M * N * K, "bytes": M * K + N * K + 2.0 * M * N, "bound": "tensor",
+                "kernels": "tc_gemm_kernel (forward)"},
+        "quantdY": {"flops": 0.0, "bytes": 3.0 * M * N, "bound": "hbm",
+                    "kernels": "quantize_stream_kernel"},
+        # each code matrix is read by two products; A, B, dA, dB and the T / U hi-lo pairs
+        "adapters": {"flops": 4.0 * M * r * (N + K),
+                     "bytes": 2.0 * (M * K + M * N) + 4.0 * r * (N + K) + 16.0 * M * r,
+                     "bound": "hbm", "kernels": "skinny_kernel x2 (T with U, dB with dA^T)"},
+        "dX": {"flops": 2.0 * M * N * K, "bytes": M * N + N * K + 2.0 * M * K, "bound": "tensor",
+               "kernels": "tc_gemm_kernel (dX)"},
+        "sgd": {"flops": 0.0, "bytes": 8.0 * N * r, "bound": None, "kernels": "torch (caller's SGD)"},
+        "proxy": {"flops": proxy_flops, "bytes": proxy_bytes, "bound": "alu" if proxy_alu else "hbm",
+                  "kernels": "proxy_pipe_kernel + proxy_clear_kernel"},
     }
 
 
@@ -371,21 +391,32 @@ def run_gpu(args):
         w = work[n]
         tflops = w["flops"] / (ms * 1e-3) / 1e12 if ms > 0 else 0.0
         gbs = w["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
-        phases[n] = {"ms": round(ms, 5), "tflops": round(tflops, 2), "gbs": round(gbs, 1),
-                     "frac_fp8_peak": round(tflops / fp8_peak, 4),
-                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-    # dominant kernel: the forward GEMM phase vs dX: both tensor-bound FP8 GEMMs;
-    # report the dX GEMM (a single kernel per phase) when it is the slowest tensor phase
-    dom = max(names, key=lambda n: phase_ms[n])
-    if dom in ("dX", "quantX+fwd"):
-        roof = {"kernel": "tc_gemm_kernel (FP8 dX GEMM)" if dom == "dX" else "quantize X + FP8 forward GEMM",
-                "bound": "tensor", "achieved": phases[dom]["tflops"], "peak": round(fp8_peak, 1),
-                "unit": "TFLOP/s", "frac": phases[dom]["frac_fp8_peak"],
+        ph = {"ms": round(ms, 5), "kernels": w["kernels"], "bound": w["bound"],
+              "tflops": round(tflops, 2), "gbs": round(gbs, 1),
+              "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        if w["bound"] == "tensor":
+            ph["frac_fp8_peak"] = round(tflops / fp8_peak, 4)
+        if w["bound"] == "alu":
+            ph["frac_fp32_fma_peak"] = round(tflops / FP32_FMA_TFLOPS, 4)
+        phases[n] = ph
+    # dominant kernel: the library phase with the largest share of the step
+    dom = max((n for n in names if work[n]["bound"]), key=lambda n: phase_ms[n])
+    b = work[dom]["bound"]
+    if b == "tensor":
+        roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "tensor",
+                "achieved": phases[dom]["tflops"], "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": phases[dom]["frac_fp8_peak"],
                 "peak_source": f"{peaks['source']} bf16 burst x {FP8_OVER_BF16} (nominal FP8/BF16)"}
+    elif b == "alu":
+        roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "alu",
+                "achieved": phases[dom]["tflops"], "peak": round(FP32_FMA_TFLOPS, 1), "unit": "TFLOP/s",
+                "frac": phases[dom]["frac_fp32_fma_peak"],
+                "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 flops x 1.965 GHz (nominal units and clock)",
+                "hbm_frac": phases[dom]["frac_hbm"]}
     else:
-        roof = {"kernel": dom, "bound": "hbm", "achieved": phases[dom]["gbs"],
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": phases[dom]["frac_hbm"],
-                "peak_source": f"{peaks['source']} copy bandwidth"}
+        roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "hbm",
+                "achieved": phases[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": phases[dom]["frac_hbm"], "peak_source": f"{peaks['source']} copy bandwidth"}
     roof["traffic"] = None
 
     out = {

@@ -156,12 +156,10 @@ __device__ __forceinline__ float load1(const void* x, int64_t i) {
 
 // Folds the partial maxima and derives s = 448 / amax (IEEE division); CTA 0
 // publishes scale, amax and the status.  Returns s to every thread.
-__device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int nparts,
-                                                uint32_t* red, float* s_shared, float* scale_out,
-                                                float* amax_out, int32_t* dev_status) {
-  uint32_t m = 0;
-  for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, partials[i]);
-  m = block_max_u32(m, red);
+// s = 448 / amax from the amax bit pattern `m` (valid in thread 0); CTA 0
+// publishes scale, amax and the status.  Returns s to every thread.
+__device__ __forceinline__ float scale_from_amax(uint32_t m, float* s_shared, float* scale_out,
+                                                 float* amax_out, int32_t* dev_status) {
   if (threadIdx.x == 0) {
     const float amax = __uint_as_float(m);
     float s;
@@ -187,6 +185,15 @@ __device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int np
   }
   __syncthreads();
   return *s_shared;
+}
+
+__device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int nparts,
+                                                uint32_t* red, float* s_shared, float* scale_out,
+                                                float* amax_out, int32_t* dev_status) {
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, partials[i]);
+  m = block_max_u32(m, red);
+  return scale_from_amax(m, s_shared, scale_out, amax_out, dev_status);
 }
 
 // Casts this thread's grid-stride share: codes = E4M3(fl32(x * s)), and the
@@ -263,17 +270,17 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------- one launch
 // quantize_stream_kernel: cooperative, one CTA per SM.  Each CTA owns a
 // contiguous run of 16 KB chunks of x.  Warp 0 (one lane) streams the chunks
-// into a ring of shared-memory slots with bulk asynchronous copies; eight
+// into a ring of shared-memory slots with bulk asynchronous copies; sixteen
 // consumer warps read each slot, then release it.  Pass 1 reduces max|x|;
-// after a grid barrier on a counter in the workspace (bounded wait) every
-// CTA folds the per-CTA maxima and pass 2 streams the same run again -- it is
-// still in L2 -- and writes the codes.
+// every CTA publishes its maximum in a marked workspace word and waits
+// (bounded) until all words are marked, reduces them, and pass 2 streams the
+// same run again -- it is still in L2 -- and writes the codes.
 constexpr int kChunkBytes = 16384;
 constexpr int kStreamStages = 8;                       // 128 KB in flight per SM
 constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
-constexpr int kBarWords = 64;                          // counter at [0], generation at [1]; partials from [64]
+constexpr int kBarWords = 64;                          // per-CTA words start 256 bytes in
 constexpr long long kBarrierBudget = 2000000000LL;    // cycles (about 1 s), then give up
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -394,35 +401,43 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
   m = block_max_u32(m, red);
 
+  // Grid exchange of the per-CTA maxima (the launch is cooperative, so every
+  // CTA is resident).  A CTA's word is its max with bit 31 set as the arrival
+  // mark (a magnitude pattern never has it); the words were zeroed before the
+  // launch.  Warp 0 of every CTA polls all words (relaxed loads, one acquire
+  // fence once all are marked), bounded, and reduces them.
   uint32_t* partials = ws + kBarWords;
-  if (threadIdx.x == 0) {
-    // grid barrier: the launch is cooperative, so every CTA is resident.
-    // Release/acquire at gpu scope orders the partials around it.
-    uint32_t gen0;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen0) : "l"(ws + 1) : "memory");
-    // (read before arriving: the generation cannot move until every CTA has arrived)
-    partials[blockIdx.x] = m;
-    uint32_t prev;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(prev) : "l"(ws) : "memory");
-    if (prev == gridDim.x - 1) {
-      ws[0] = 0u;  // ready for the next launch
-      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ws + 1), "r"(gen0 + 1u) : "memory");
-    } else {
-      const long long t0 = clock64();
-      while (true) {
-        uint32_t g;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(ws + 1) : "memory");
-        if (g != gen0) break;
-        if (clock64() - t0 > kBarrierBudget) {
-          if (dev_status) atomicOr(dev_status, kDevTimeout);
-          break;
-        }
+  __shared__ uint32_t amax_bits;
+  if (warp == 0) {
+    if (lane == 0)
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(partials + blockIdx.x), "r"(m | 0x80000000u)
+                   : "memory");
+    __syncwarp();
+    const long long t0 = clock64();
+    uint32_t mx = 0;
+    while (true) {
+      bool all = true;
+      mx = 0;
+      for (int i = lane; i < static_cast<int>(gridDim.x); i += 32) {
+        uint32_t w;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w) : "l"(partials + i) : "memory");
+        all = all && (w >> 31) != 0u;
+        mx = max(mx, w & 0x7FFFFFFFu);
+      }
+      if (__all_sync(0xFFFFFFFFu, all)) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the marked words
+        break;
+      }
+      if (clock64() - t0 > kBarrierBudget) {
+        if (lane == 0 && dev_status) atomicOr(dev_status, kDevTimeout);
+        break;
       }
     }
-    __threadfence();
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) amax_bits = mx;
   }
   __syncthreads();
-  const float s = fold_and_scale(partials, gridDim.x, red, &s_shared, scale_out, amax_out, dev_status);
+  const float s = scale_from_amax(amax_bits, &s_shared, scale_out, amax_out, dev_status);
   const double s_d = static_cast<double>(s);
 
   // ---- pass 2: codes (and the optional residual)
@@ -528,7 +543,7 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
     int64_t chunks = (body + kChunkBytes - 1) / kChunkBytes;
     int grid = static_cast<int>(chunks < di->sm_count ? (chunks > 0 ? chunks : 1) : di->sm_count);
     if (grid > 4096 - kBarWords) grid = 4096 - kBarWords;
-    cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(uint32_t), stream);
+    cudaError_t e = cudaMemsetAsync(ws + kBarWords, 0, static_cast<size_t>(grid) * sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
