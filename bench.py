@@ -260,6 +260,16 @@ def run_gpu(args):
     layer = wl.layers[0]
     st = Step(wl, layer, torch, F, dev, n_slots=2, seed_offset=rank * 1000)
     stream = torch.cuda.Stream(device=dev)
+    if args.only:
+        # one phase alone, eagerly, warm-up + steps times (for profiler captures)
+        k = Step.PHASES.index(args.only)
+        with torch.cuda.stream(stream):
+            st.phases(0)  # one whole step first, so every input of the phase is real data
+            for i in range(args.warmup + args.steps):
+                st.phase(i % 2, k)
+        torch.cuda.synchronize()
+        status = int(st.status.item())
+        return {"only": args.only, "launches": args.warmup + args.steps, "device_status": status}, rank
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     flush_tail = flush[: 192 << 20].view(torch.int32)
 
@@ -547,6 +557,9 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--only", default=None, choices=list(Step.PHASES),
+                    help="run one phase alone (warm-up + steps calls) and print no bench line; "
+                         "for profiler captures")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
