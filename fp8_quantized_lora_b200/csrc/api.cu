@@ -61,11 +61,11 @@ EncodeTiledFn encode_tiled_fn() {
 
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes,
                   const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                  uint32_t box_outer, bool swizzle128) {
+                  uint32_t box_outer, bool swizzle128, uint64_t ld) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint64_t strides[1] = {(ld ? ld : inner) * elem_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,

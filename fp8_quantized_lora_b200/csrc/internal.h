@@ -27,10 +27,11 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_tiled_fn();
 
-// 2-D tensor map over a row-major [outer, inner] tensor.
+// 2-D tensor map over a row-major [outer, inner] tensor whose rows are `ld`
+// elements apart (0: ld = inner).
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes,
                   const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                  uint32_t box_outer, bool swizzle128);
+                  uint32_t box_outer, bool swizzle128, uint64_t ld = 0);
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

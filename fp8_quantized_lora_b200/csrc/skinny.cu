@@ -2,42 +2,56 @@
 //
 // FALQON, OpenReview rebuttal (reviewer 4, Q1): B's gradient comes from the
 // precomputable product A x, and A's from B^T dL/dO; both reuse the E4M3
-// codes the quantize step produced.  With T = Xq A^T / s_X and
-// U = dYq B / s_dY (fp32 tiles kept as bf16 hi/lo pairs):
-//   T   = Xq . A^T          [M, r]   A-op Xq   K-major,  B-op A   [r, K]  K-major
-//   U   = dYq . B           [M, r]   A-op dYq  K-major,  B-op B   [N, r]  MN-major
-//   dB  = dYq^T . T / s_dY  [N, r]   A-op dYq^T MN-major, B-op T (hi + lo) MN-major
-//   dA^T= Xq^T . U / s_X    [K, r]   A-op Xq^T  MN-major, B-op U (hi + lo) MN-major
+// codes the quantize step produced.  Every product puts the small rank
+// dimension on the UMMA M side and 256 tokens or features on the N side, so
+// one 128 x 256 x 16 MMA does the most work a single instruction can:
+//   T^T  = A . Xq^T / s_X          [r, M]  A-op A [r, K] K-major,  B-op Xq codes K-major
+//   U^T  = B^T . dYq^T / s_dY      [r, M]  A-op B [N, r] MN-major, B-op dYq codes K-major
+//   dB^T = (T_hi + T_lo)^T . dYq / s_dY   [r, N]  A-op T^T hi over lo, B-op dYq codes MN-major
+//   dA   = (U_hi + U_lo)^T . Xq / s_X     [r, K]  A-op U^T hi over lo, B-op Xq codes MN-major
+// T and U are kept as bf16 hi/lo pairs, stored transposed ([r, M]).  In dB
+// and dA the hi and lo operands fill the upper and lower 64 rows of one
+// M = 128 tile, and the reduction adds the two halves.
 //
-// The E4M3 codes are expanded exactly to bf16 in shared memory and fed to
-// tcgen05 kind::f16 (every E4M3 value is a bf16 value).  One launch runs two
-// independent products (T with U, then dB with dA): the first `ctas0` CTAs
-// work on problem 0, the others on problem 1, two CTAs per SM where the tiles
-// allow, so the start-up and reduction phases of one CTA overlap the main
-// loop of its neighbour.  Each CTA owns one (row tile, K split) work item;
-// the `splits` CTAs of a row tile form one cluster and sum their fp32 tiles
-// through DSMEM in rank order (deterministic).
+// The E4M3 codes are expanded exactly to bf16 in shared memory (every E4M3
+// value is a bf16 value) and fed to tcgen05 kind::f16 as the B operand.  One
+// launch runs two independent products (T with U, then dB with dA): the first
+// `ctas0` CTAs work on problem 0, the rest on problem 1.  Each CTA owns one
+// (rank tile, column tile, K split) work item; the `splits` CTAs of an output
+// tile form one cluster and sum their fp32 tiles through DSMEM in rank order
+// (deterministic).
+//
+// Two warps issue MMAs, on alternate pairs of K blocks, into two TMEM
+// accumulators: a warp that waits on a barrier stalls its own MMA stream, and
+// the other warp's keeps the tensor pipe busy meanwhile.  The epilogue adds
+// the two accumulators in a fixed order.
 //
 // Roles per CTA:
-//   warp 0       TMA producer for the small bf16 operand (one lane)
-//   warp 1       TMEM owner and UMMA issuer (one lane issues)
+//   warp 0       TMA producer for the bf16 A operand (one lane)
+//   warp 1       TMEM owner; MMA issuer for even K-block pairs (one lane)
 //   warps 2-5    epilogue: TMEM -> fp32 reduction tile in shared memory
 //   warps 6-13   converters: raw E4M3 tile -> bf16, 128-byte-swizzled
 //   warp 14      TMA producer for the raw E4M3 tiles (one lane)
+//   warp 15      MMA issuer for odd K-block pairs (one lane)
 #include "internal.h"
 #include "tc_common.cuh"
 
 namespace falqon {
 namespace {
 
+constexpr int kSkN = 256;  // UMMA N: tokens or features per tile
+constexpr int kSkK = 64;   // bf16 K per stage (one 128-byte swizzle row)
+
 struct SkinnyProblem {
   int32_t m_tiles, n_tiles, splits, kb_total, kb_per_split;
-  int64_t M, N;        // output rows (UMMA M side) and columns (r)
-  void* out;           // bf16 [M][ldo] (or [N][ldo] when transposed)
+  int64_t rows;        // r: ranks (output rows before any transpose)
+  int64_t cols;        // tokens or features (output columns before any transpose)
+  void* out;           // bf16 [rows][ldo], or [cols][ldo] when transposed
   void* out_lo;        // optional low half of a hi/lo pair
   int64_t ldo;
   int transpose;       // store out[col * ldo + row]
-  int b_mn;            // the bf16 operand is MN-major (else K-major)
+  int a_mn;            // the A operand is MN-major (B for U^T) instead of K-major
+  int hilo;            // A rows [0, 64) hi and [64, 128) lo of the same ranks: add the halves
   const float* scale;  // alpha = 1 / *scale
 };
 
@@ -47,56 +61,56 @@ struct SkinnyArgs {
   int32_t* dev_status;
 };
 
-template <int kBN, bool kAMn, bool kBSplit, int kSA, int kSB, int kSR, int kMinBlocks>
+template <bool kBMn, int kStages, int kRawStages>
 struct SkCfg {
-  static constexpr int BN = kBN;
-  static constexpr bool AMn = kAMn;
-  static constexpr bool BSplit = kBSplit;  // B = B_hi + B_lo: two tiles, two MMAs per k-step
-  static constexpr int SA = kSA, SB = kSB, SR = kSR;
-  static constexpr int MinBlocks = kMinBlocks;
-  static constexpr int BK = 64;                             // bf16 K per stage
-  static constexpr int KSteps = 4;                          // UMMA K = 16
-  static constexpr int ABytes = kBM * BK * 2;               // expanded A tile, 16 KB
-  static constexpr int BBytes = kBN * BK * 2;
-  static constexpr int BSlotBytes = BBytes * (kBSplit ? 2 : 1);
-  static constexpr int RawSlotBytes = kBM * BK;             // 8 KB of codes
+  static constexpr bool BMn = kBMn;  // codes are the MN-major B operand (dB^T, dA)
+  static constexpr int S = kStages, SR = kRawStages;
+  static constexpr int KSteps = kSkK / 16;                // UMMA K = 16
+  static constexpr int ABytes = kBM * kSkK * 2;           // bf16 A tile, 16 KB
+  static constexpr int BBytes = kSkN * kSkK * 2;          // expanded B tile, 32 KB
+  static constexpr int StageBytes = ABytes + BBytes;
+  static constexpr int RawBytes = kSkN * kSkK;            // raw codes, 16 KB
+  static constexpr int RawRowBytes = kBMn ? kSkN : kSkK;  // row length of the raw box
   static constexpr int ConvWarps = 8;
+  static constexpr int ChunksPerThread = RawBytes / 16 / (32 * ConvWarps);  // 4
   static constexpr int RawWarp = 6 + ConvWarps;
-  static constexpr int Threads = 32 * (RawWarp + 1);        // 480
-  static constexpr uint32_t TmemCols = kBN < 32 ? 32 : kBN;
-  static constexpr int ARing = kSA * ABytes, BRing = kSB * BSlotBytes, RawRing = kSR * RawSlotBytes;
-  static constexpr int BarBytes = 8 * (2 * kSA + 2 * kSB + 2 * kSR + 2) + 16;
-  static constexpr int SmemBytes = ARing + BRing + RawRing + BarBytes + 1024;
-  static constexpr int RedStride = kBN + 4;  // fp32 words per row of the reduction tile
-  static_assert(kBM * RedStride * 4 <= ARing + BRing, "reduction tile");
-  static_assert(kBN % 64 == 0 && kBN <= 256, "UMMA N, 128-byte MN-major blocks");
-  static_assert(RawSlotBytes == 2 * 16 * 32 * ConvWarps, "two 16-byte chunks per converter thread");
-  static_assert(kSA >= 2 && kSB >= 2 && kSR >= 2, "ring depths");
-  static_assert(SmemBytes * kMinBlocks <= 228 * 1024 - 1024 * kMinBlocks, "shared memory per SM");
+  static constexpr int Mma2Warp = RawWarp + 1;
+  static constexpr int Threads = 32 * (Mma2Warp + 1);     // 512
+  static constexpr uint32_t TmemCols = 2 * kSkN;          // two accumulators
+  static constexpr int Ring = kStages * StageBytes, RawRing = kRawStages * RawBytes;
+  static constexpr int BarBytes = 8 * (2 * kStages + 2 * kRawStages + 5) + 16;
+  static constexpr int SmemBytes = Ring + RawRing + BarBytes + 1024;
+  static constexpr int RedStride = kSkN + 4;   // [rank][col] reduction tile, fp32 words per row
+  static constexpr int RedStrideT = kBM + 4;   // [col][rank] reduction tile (transposed outputs)
+  static_assert(kBM * RedStride * 4 <= Ring && kSkN * RedStrideT * 4 <= Ring, "reduction tile");
+  static_assert(ChunksPerThread * 16 * 32 * ConvWarps == RawBytes, "chunks per converter");
+  static_assert(kStages >= 2 && kRawStages >= 2, "ring depths");
+  // pconv[m] may not complete a pair's phase before its issuer saw the previous
+  // one: the converters' last stage of pair p + 2 must reuse a slot of pair p
+  static_assert(kStages <= 4, "pair barriers");
+  static_assert(SmemBytes <= 232448, "shared memory per CTA");
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::Threads, C::MinBlocks)
-    skinny_kernel(const __grid_constant__ CUtensorMap raw0, const __grid_constant__ CUtensorMap b0,
-                  const __grid_constant__ CUtensorMap b20, const __grid_constant__ CUtensorMap raw1,
-                  const __grid_constant__ CUtensorMap b1, const __grid_constant__ CUtensorMap b21,
+__global__ void __launch_bounds__(C::Threads, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap raw0, const __grid_constant__ CUtensorMap a0,
+                  const __grid_constant__ CUtensorMap a20, const __grid_constant__ CUtensorMap raw1,
+                  const __grid_constant__ CUtensorMap a1, const __grid_constant__ CUtensorMap a21,
                   const SkinnyArgs args) {
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* a_ring = smem;                                 // expanded A tiles
-  uint8_t* b_ring = smem + C::ARing;                      // bf16 operand tiles
-  uint8_t* raw_ring = b_ring + C::BRing;                  // raw E4M3 tiles
+  uint8_t* ring = smem;                                   // stages of [A 16 KB][B 32 KB]
+  uint8_t* raw_ring = smem + C::Ring;                     // raw E4M3 tiles (TMA)
   uint64_t* bars = reinterpret_cast<uint64_t*>(raw_ring + C::RawRing);
-  uint64_t* full = bars;                                  // [SB] B landed
-  uint64_t* empty = full + C::SB;                         // [SB] MMAs done with the B slot
-  uint64_t* conv = empty + C::SB;                         // [SA] A expanded
-  uint64_t* aempty = conv + C::SA;                        // [SA] MMAs done with the A slot
-  uint64_t* rawfull = aempty + C::SA;                     // [SR] raw codes landed
+  uint64_t* full = bars;                                  // [S] A landed
+  uint64_t* empty = full + C::S;                          // [S] MMAs done with the stage
+  uint64_t* pconv = empty + C::S;                         // [2] a pair of stages ready, per issuer
+  uint64_t* rawfull = pconv + 2;                          // [SR] raw codes landed
   uint64_t* rawempty = rawfull + C::SR;                   // [SR] converters done reading
-  uint64_t* acc_full = rawempty + C::SR;                  // accumulator complete
-  uint64_t* drain = acc_full + 1;                         // all MMAs retired (teardown)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* acc_full = rawempty + C::SR;                  // both accumulators complete
+  uint64_t* drain = acc_full + 1;                         // [2] each issuer's MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -104,36 +118,40 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
   const bool second = static_cast<int>(blockIdx.x) >= args.ctas0;
   const SkinnyProblem& g = args.p[second ? 1 : 0];
   const CUtensorMap* tmRaw = second ? &raw1 : &raw0;
-  const CUtensorMap* tmB = second ? &b1 : &b0;
-  const CUtensorMap* tmB2 = second ? &b21 : &b20;
+  const CUtensorMap* tmA = second ? &a1 : &a0;
+  const CUtensorMap* tmA2 = second ? &a21 : &a20;
   const int w = static_cast<int>(blockIdx.x) - (second ? args.ctas0 : 0);  // work item
   const int split = w % g.splits;
   const int nt = (w / g.splits) % g.n_tiles;
   const int mt = w / (g.splits * g.n_tiles);
   const int kb0 = split * g.kb_per_split;
-  const int kb1 = min(g.kb_total, kb0 + g.kb_per_split);
-  const bool b_mn = g.b_mn != 0;
+  const int nkb = max(0, min(g.kb_total, kb0 + g.kb_per_split) - kb0);
+  const int npairs = (nkb + 1) / 2;
+  const bool a_mn = g.a_mn != 0;
+  const bool hilo = g.hilo != 0;
+  const int row_span = hilo ? 64 : kBM;  // ranks per tile
+  const int i0 = mt * row_span;
+  const int n0 = nt * kSkN;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::SB; ++s) {
+    for (int s = 0; s < C::S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int s = 0; s < C::SA; ++s) {
-      mbar_init(&conv[s], C::ConvWarps);
-      mbar_init(&aempty[s], 1);
-    }
+    mbar_init(&pconv[0], C::ConvWarps);
+    mbar_init(&pconv[1], C::ConvWarps);
     for (int s = 0; s < C::SR; ++s) {
       mbar_init(&rawfull[s], 1);
       mbar_init(&rawempty[s], C::ConvWarps);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(drain, 1);
+    mbar_init(acc_full, 2);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(tmRaw);
-    tma_prefetch_desc(tmB);
-    if constexpr (C::BSplit) tma_prefetch_desc(tmB2);
+    tma_prefetch_desc(tmA);
+    if (hilo) tma_prefetch_desc(tmA2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TmemCols);
@@ -148,16 +166,16 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     *abort_flag = 1;
     raise_status(args.dev_status, kDevTimeout);
   };
-  // one producer lane: waits `emp`, then fills `ful` with `load(slot, kb)`
+  // one producer lane: waits `emp`, then fills `ful` with `load(slot, k-block)`
   auto produce = [&](uint64_t* ful, uint64_t* emp, int depth, uint32_t bytes, auto load) {
     int s = 0;
     uint32_t ph = 0, issued = 0, issued_parity = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
+    for (int i = 0; i < nkb; ++i) {
       if (!mbar_wait(&emp[s], ph ^ 1, abort_flag)) { fail(); break; }
       mbar_arrive_expect_tx(&ful[s], bytes);
       issued |= 1u << s;
       issued_parity = (issued_parity & ~(1u << s)) | (ph << s);
-      load(s, kb);
+      load(s, kb0 + i);
       if (++s == depth) { s = 0; ph ^= 1; }
     }
     // every load issued must land before shared memory is reused or released
@@ -165,103 +183,116 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       if (issued & (1u << t)) mbar_wait_budget(&ful[t], (issued_parity >> t) & 1u);
   };
 
-  constexpr int kTileRows = C::AMn ? C::BK : kBM;  // rows of the A tile (and of its raw box)
-  constexpr int kTileCols = C::AMn ? kBM : C::BK;  // codes per row
   if (warp == 0) {
-    // ------------------------------------------------------------ bf16 operand producer
+    // ------------------------------------------------------------ A producer
     if (lane == 0) {
-      const int n0 = nt * C::BN;
-      produce(full, empty, C::SB, static_cast<uint32_t>(C::BSlotBytes), [&](int s, int kb) {
-        uint8_t* sB = b_ring + s * C::BSlotBytes;
-        if (b_mn) {
-          // [K rows][N] row-major: 128-byte column blocks of 64 K rows each
-#pragma unroll
-          for (int c = 0; c < C::BN / 64; ++c) {
-            tma_load_2d(sB + c * C::BK * kRowBytes, tmB, &full[s], n0 + c * 64, kb * C::BK);
-            if constexpr (C::BSplit)
-              tma_load_2d(sB + C::BBytes + c * C::BK * kRowBytes, tmB2, &full[s], n0 + c * 64, kb * C::BK);
-          }
+      produce(full, empty, C::S, static_cast<uint32_t>(C::ABytes), [&](int s, int kb) {
+        uint8_t* sA = ring + s * C::StageBytes;
+        const int k0 = kb * kSkK;
+        if (hilo) {
+          // ranks i0 .. +64 of the hi operand in rows 0-63, of the lo operand in rows 64-127
+          tma_load_2d(sA, tmA, &full[s], k0, i0);
+          tma_load_2d(sA + 64 * kRowBytes, tmA2, &full[s], k0, i0);
+        } else if (a_mn) {
+          // [K rows][ranks] row-major: two 128-byte column blocks of 64 ranks
+          tma_load_2d(sA, tmA, &full[s], i0, k0);
+          tma_load_2d(sA + kSkK * kRowBytes, tmA, &full[s], i0 + 64, k0);
         } else {
-          tma_load_2d(sB, tmB, &full[s], kb * C::BK, n0);
-          if constexpr (C::BSplit) tma_load_2d(sB + C::BBytes, tmB2, &full[s], kb * C::BK, n0);
+          tma_load_2d(sA, tmA, &full[s], k0, i0);
         }
       });
     }
     __syncwarp();
   } else if (warp == C::RawWarp) {
     // ------------------------------------------------------------ raw-code producer
-    // K-major A = codes[m0 .. +128, kb*64 .. +64]; MN-major A = codes[kb*64 .. +64, m0 .. +128]
+    // K-major codes[n0 .. +256][kb*64 .. +64]; MN-major codes[kb*64 .. +64][n0 .. +256]
     if (lane == 0) {
-      produce(rawfull, rawempty, C::SR, static_cast<uint32_t>(C::RawSlotBytes), [&](int s, int kb) {
-        if constexpr (C::AMn)
-          tma_load_2d(raw_ring + s * C::RawSlotBytes, tmRaw, &rawfull[s], mt * kBM, kb * C::BK);
+      produce(rawfull, rawempty, C::SR, static_cast<uint32_t>(C::RawBytes), [&](int s, int kb) {
+        if constexpr (C::BMn)
+          tma_load_2d(raw_ring + s * C::RawBytes, tmRaw, &rawfull[s], n0, kb * kSkK);
         else
-          tma_load_2d(raw_ring + s * C::RawSlotBytes, tmRaw, &rawfull[s], kb * C::BK, mt * kBM);
+          tma_load_2d(raw_ring + s * C::RawBytes, tmRaw, &rawfull[s], kb * kSkK, n0);
       });
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    const uint32_t idesc = idesc_f32acc(1u, 1u, C::AMn ? 1u : 0u, b_mn ? 1u : 0u, kBM, C::BN);
-    int sb = 0, sa = 0;
-    uint32_t pb = 0, pa = 0;
+  } else if (warp == 1 || warp == C::Mma2Warp) {
+    // ------------------------------------------------------------ MMA issuers
+    // Issuer m takes K-block pairs m, m + 2, ... into accumulator m, and
+    // waits once per pair on its own barrier pconv[m], whose phases it sees
+    // one by one: the converters arrive there when both stages of the pair
+    // are expanded and both A tiles have landed.  (A wait on a per-stage
+    // barrier could not tell its phases apart here: the issuer that did not
+    // see a stage's previous use may find it two phases behind.)
+    const int m = warp == 1 ? 0 : 1;
+    const uint32_t idesc = idesc_f32acc(1u, 1u, a_mn ? 1u : 0u, C::BMn ? 1u : 0u, kBM, kSkN);
+    const uint32_t acc = tmem_base + static_cast<uint32_t>(m * kSkN);
     bool ok = true;
     tc_fence_after();
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!warp_wait(&conv[sa], pa, abort_flag) || !warp_wait(&full[sb], pb, abort_flag)) {
+    for (int p = m; p < npairs; p += 2) {
+      const int i_first = 2 * p;
+      const int i_last = min(2 * p + 1, nkb - 1);
+      if (!warp_wait(&pconv[m], static_cast<uint32_t>((p >> 1) & 1), abort_flag)) {
         if (lane == 0) fail();
         ok = false;
         break;
       }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a_base = smem_u32(a_ring + sa * C::ABytes);
-        const uint32_t b_base = smem_u32(b_ring + sb * C::BSlotBytes);
+        for (int i = i_first; i <= i_last; ++i) {
+          const int s = i % C::S;
+          const uint32_t a_base = smem_u32(ring + s * C::StageBytes);
+          const uint32_t b_base = a_base + C::ABytes;
 #pragma unroll
-        for (int ks = 0; ks < C::KSteps; ++ks) {
-          const uint64_t ad = operand_desc_rt<2, C::BK>(C::AMn, a_base, ks);
-          const uint64_t bd = operand_desc_rt<2, C::BK>(b_mn, b_base, ks);
-          umma_bf16(tmem_base, ad, bd, idesc, (kb > kb0 || ks > 0) ? 1u : 0u);
-          if constexpr (C::BSplit)
-            umma_bf16(tmem_base, ad, operand_desc_rt<2, C::BK>(b_mn, b_base + C::BBytes, ks), idesc, 1u);
+          for (int ks = 0; ks < C::KSteps; ++ks)
+            umma_bf16(acc, operand_desc_rt<2, kSkK>(a_mn, a_base, ks),
+                      operand_desc_rt<2, kSkK>(C::BMn, b_base, ks), idesc,
+                      (p > m || i > i_first || ks > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[sb]);
-        umma_commit(&aempty[sa]);
       }
       __syncwarp();
-      if (++sb == C::SB) { sb = 0; pb ^= 1; }
-      if (++sa == C::SA) { sa = 0; pa ^= 1; }
     }
     if (lane == 0) {
       if (ok) umma_commit(acc_full);
-      umma_commit(drain);
-      mbar_wait_budget(drain, 0);
+      umma_commit(&drain[m]);
+      mbar_wait_budget(&drain[m], 0);
     }
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
-    // fp32 accumulator rows -> reduction tile in shared memory (the rings are
-    // idle once every MMA has completed)
+    // acc0 + acc1 -> fp32 reduction tile in shared memory (the ring is idle
+    // once every MMA has completed): [rank][col] for row-major outputs,
+    // [col][rank] for transposed ones, so that either reduction reads
+    // float4 along the output's contiguous dimension.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     if (warp_wait(acc_full, 0, abort_flag)) {
       tc_fence_after();
-      float* red_row = reinterpret_cast<float*>(smem) + (q * 32 + lane) * C::RedStride;
-      const bool empty_split = kb1 <= kb0;  // no K blocks: the partial sum is zero
+      const int row = q * 32 + lane;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      float* red = reinterpret_cast<float*>(smem);
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 16; ++c) {
-        uint32_t r[16];
-        if (!empty_split) {
-          tmem_ld_16cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + c * 16, r);
-          tmem_ld_wait();
-        } else {
+      for (int c = 0; c < kSkN / 16; ++c) {
+        float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) r[j] = 0u;
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          if (npairs > a) {
+            uint32_t r[16];
+            tmem_ld_16cols(lane_base + a * kSkN + c * 16, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
+          }
         }
-        float4* red = reinterpret_cast<float4*>(red_row + c * 16);
+        if (g.transpose) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          red[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+          for (int j = 0; j < 16; ++j) red[(c * 16 + j) * C::RedStrideT + row] = v[j];
+        } else {
+          float4* dst = reinterpret_cast<float4*>(red + row * C::RedStride + c * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
       }
     } else if (lane == 0) {
       fail();
@@ -269,95 +300,118 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_fence_before();
   } else {
     // ------------------------------------------------------------ converters
-    // 256 threads; each expands two 16-byte chunks (32 codes) of every A tile:
-    //   K-major  [128 rows][64 codes]:  rows t/4 and t/4 + 64,  columns (t % 4) * 16 ..
-    //   MN-major [64 rows][128 codes]:  rows t/8 and t/8 + 32,  columns (t % 8) * 16 ..
-    constexpr int kThrPerRow = kTileCols / 16;
-    constexpr int kRowStep = 256 / kThrPerRow;  // second chunk: this many rows further down
+    // 256 threads; each expands four 16-byte chunks (64 codes) of every tile:
+    //   K-major  raw [256 rows][64 codes]:  rows t/4 + 64j,  codes (t % 4) * 16 ..
+    //   MN-major raw [64 rows][256 codes]:  rows t/16 + 16j, codes (t % 16) * 16 ..
+    // into the 128-byte-swizzled bf16 tile (MN-major: four 64-column blocks).
+    constexpr int kThrPerRow = C::RawRowBytes / 16;
+    constexpr int kRowStep = 256 / kThrPerRow;
+    constexpr int kBlkBytes = (C::BMn ? kSkK : kSkN) * kRowBytes;  // one 128-byte column block
     const int t = threadIdx.x - 6 * 32;
     const int trow = t / kThrPerRow;
     const int tcol = (t % kThrPerRow) * 16;
-    const uint32_t raw_off0 = trow * kTileCols + tcol;
-    const uint32_t raw_off1 = (trow + kRowStep) * kTileCols + tcol;
     const int blk = tcol / 64;
     const int unit0 = (tcol % 64) / 8;
-    auto dst_off = [&](int row, int unit) {
-      return static_cast<uint32_t>(blk * (kTileRows * kRowBytes) + row * kRowBytes +
-                                   ((unit ^ (row & 7)) << 4));
-    };
-    const uint32_t d00 = dst_off(trow, unit0), d01 = dst_off(trow, unit0 + 1);
-    const uint32_t d10 = dst_off(trow + kRowStep, unit0), d11 = dst_off(trow + kRowStep, unit0 + 1);
-    int sa = 0, sr = 0;
-    uint32_t pa = 0, pr = 0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-      if (!warp_wait(&rawfull[sr], pr, abort_flag)) { if (lane == 0) fail(); break; }
-      const uint4 q0 = *reinterpret_cast<const uint4*>(raw_ring + sr * C::RawSlotBytes + raw_off0);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(raw_ring + sr * C::RawSlotBytes + raw_off1);
+    // MN-major: the two column blocks a quarter-warp writes share banks, so
+    // odd blocks store their two 16-byte units in the opposite order
+    const bool swap = C::BMn && (blk & 1);
+    for (int i = 0; i < nkb; ++i) {
+      const int sr = i % C::SR, s = i % C::S;
+      if (!warp_wait(&rawfull[sr], static_cast<uint32_t>((i / C::SR) & 1), abort_flag)) {
+        if (lane == 0) fail();
+        break;
+      }
+      uint4 q[C::ChunksPerThread];
+#pragma unroll
+      for (int j = 0; j < C::ChunksPerThread; ++j)
+        q[j] = *reinterpret_cast<const uint4*>(raw_ring + sr * C::RawBytes +
+                                               (trow + j * kRowStep) * C::RawRowBytes + tcol);
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[sr]);
-      if (++sr == C::SR) { sr = 0; pr ^= 1; }
-      uint32_t o0[8], o1[8];
-      e4m3x16_to_bf16(q0, o0);
-      e4m3x16_to_bf16(q1, o1);
-      if (!warp_wait(&aempty[sa], pa ^ 1, abort_flag)) { if (lane == 0) fail(); break; }
-      uint8_t* sA = a_ring + sa * C::ABytes;
-      *reinterpret_cast<uint4*>(sA + d00) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-      *reinterpret_cast<uint4*>(sA + d01) = make_uint4(o0[4], o0[5], o0[6], o0[7]);
-      *reinterpret_cast<uint4*>(sA + d10) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-      *reinterpret_cast<uint4*>(sA + d11) = make_uint4(o1[4], o1[5], o1[6], o1[7]);
+      if (!warp_wait(&empty[s], static_cast<uint32_t>(((i / C::S) & 1) ^ 1), abort_flag)) {
+        if (lane == 0) fail();
+        break;
+      }
+      uint8_t* sB = ring + s * C::StageBytes + C::ABytes + blk * kBlkBytes;
+#pragma unroll
+      for (int j = 0; j < C::ChunksPerThread; ++j) {
+        uint32_t o[8];
+        e4m3x16_to_bf16(q[j], o);
+        const int row = trow + j * kRowStep;
+        const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
+        const uint4 hi = make_uint4(o[4], o[5], o[6], o[7]);
+        const uint32_t off_lo = row * kRowBytes + ((unit0 ^ (row & 7)) << 4);
+        const uint32_t off_hi = row * kRowBytes + (((unit0 + 1) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(sB + (swap ? off_hi : off_lo)) = swap ? hi : lo;
+        *reinterpret_cast<uint4*>(sB + (swap ? off_lo : off_hi)) = swap ? lo : hi;
+      }
       fence_proxy_async_smem();
+      // the stage's A tile must have landed too: pconv[] then covers both operands
+      if (!warp_wait(&full[s], static_cast<uint32_t>((i / C::S) & 1), abort_flag)) {
+        if (lane == 0) fail();
+        break;
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&conv[sa]);
-      if (++sa == C::SA) { sa = 0; pa ^= 1; }
+      // K blocks 2p and 2p + 1 form pair p, issued from accumulator p % 2's warp
+      if (lane == 0 && ((i & 1) || i == nkb - 1)) mbar_arrive(&pconv[(i >> 1) & 1]);
     }
   }
 
   // ---------------------------------------------------------------- split-K reduction
-  // Sum the cluster's tiles row slice by row slice (this CTA owns rows
-  // [q0, q1) of the tile), in rank order, and write bf16 (or hi/lo pairs).
+  // The cluster's tiles are summed in rank order over a flat range of float4
+  // groups (this CTA owns one slice), scaled by 1/s and written as bf16 (or
+  // hi/lo pairs).
   __syncthreads();
   cluster_sync_all();
   {
     const int S = g.splits;
     const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
-    const int rows_per = (kBM + S - 1) / S;
-    const int q0 = static_cast<int>(rank) * rows_per;
-    const int q1 = min(kBM, q0 + rows_per);
+    const int nvalid = static_cast<int>(g.rows - i0 < row_span ? g.rows - i0 : row_span);  // ranks, % 4 == 0
+    const bool tr = g.transpose != 0;
+    const int ng = tr ? nvalid / 4 : kSkN / 4;  // float4 groups along the contiguous dimension
+    const int total = tr ? kSkN * ng : nvalid * ng;
+    const int chunk = (total + S - 1) / S;
+    const int e_begin = static_cast<int>(rank) * chunk;
+    const int e_end = min(total, e_begin + chunk);
     const float* red = reinterpret_cast<const float*>(smem);
     uint32_t peer[kMaxSplits];
 #pragma unroll
     for (int sidx = 0; sidx < kMaxSplits; ++sidx) peer[sidx] = dsmem_addr(red, sidx < S ? sidx : 0);
     const float alpha = g.scale ? static_cast<float>(1.0 / static_cast<double>(*g.scale)) : 1.0f;
-    const int nrows = q1 - q0;
-    constexpr int G = C::BN / 4;  // float4 groups per row
-    const int ngroups = nrows > 0 ? nrows * G : 0;
+    // offset of the lo half: 64 ranks further on
+    const uint32_t lo_off = static_cast<uint32_t>((tr ? 64 : 64 * C::RedStride) * 4);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
     __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(g.out_lo);
-    for (int e = threadIdx.x; e < ngroups; e += blockDim.x) {
-      int lr, lg;
-      if (g.transpose) { lr = q0 + e % nrows; lg = e / nrows; }  // walk rows: coalesced out[col][row]
-      else { lr = q0 + e / G; lg = e % G; }
-      const uint32_t off = static_cast<uint32_t>((lr * C::RedStride + 4 * lg) * 4);
+    for (int e = e_begin + static_cast<int>(threadIdx.x); e < e_end; e += blockDim.x) {
+      const int major = e / ng, lg = e % ng;  // tr: (col, rank group); else (rank, col group)
+      const int64_t gcol = n0 + (tr ? major : 4 * lg);
+      if (gcol >= g.cols) continue;  // row-major outputs: ldo covers the whole group
+      const uint32_t off = static_cast<uint32_t>(
+          (tr ? major * C::RedStrideT + 4 * lg : major * C::RedStride + 4 * lg) * 4);
+      float4 part[kMaxSplits], part_lo[kMaxSplits];
+#pragma unroll
+      for (int sidx = 0; sidx < kMaxSplits; ++sidx) {
+        if (sidx < S) {
+          part[sidx] = dsmem_load_f32x4(peer[sidx] + off);
+          if (hilo) part_lo[sidx] = dsmem_load_f32x4(peer[sidx] + off + lo_off);
+        }
+      }
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-      for (int s0 = 0; s0 < kMaxSplits; s0 += 4) {  // fixed order: rank 0, 1, ...
-        float4 part[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (s0 + k < S) part[k] = dsmem_load_f32x4(peer[s0 + k] + off);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (s0 + k < S) {
-            acc.x += part[k].x;
-            acc.y += part[k].y;
-            acc.z += part[k].z;
-            acc.w += part[k].w;
+      for (int sidx = 0; sidx < kMaxSplits; ++sidx) {  // fixed order: rank 0, 1, ...
+        if (sidx < S) {
+          acc.x += part[sidx].x;
+          acc.y += part[sidx].y;
+          acc.z += part[sidx].z;
+          acc.w += part[sidx].w;
+          if (hilo) {
+            acc.x += part_lo[sidx].x;
+            acc.y += part_lo[sidx].y;
+            acc.z += part_lo[sidx].z;
+            acc.w += part_lo[sidx].w;
           }
         }
       }
-      const int64_t grow = static_cast<int64_t>(mt) * kBM + lr;
-      const int64_t gcol0 = static_cast<int64_t>(nt) * C::BN + 4 * lg;
-      if (grow >= g.M || gcol0 >= g.N) continue;  // N % 16 == 0: groups of 4 in or out
       const float vals[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
       __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
@@ -365,19 +419,12 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         hi[k] = __float2bfloat16_rn(vals[k]);
         lo[k] = __float2bfloat16_rn(vals[k] - __bfloat162float(hi[k]));
       }
-      if (g.transpose) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          out[(gcol0 + k) * g.ldo + grow] = hi[k];
-          if (out_lo) out_lo[(gcol0 + k) * g.ldo + grow] = lo[k];
-        }
-      } else {
-        uint2 ph, pl;
-        memcpy(&ph, hi, 8);
-        memcpy(&pl, lo, 8);
-        *reinterpret_cast<uint2*>(out + grow * g.ldo + gcol0) = ph;
-        if (out_lo) *reinterpret_cast<uint2*>(out_lo + grow * g.ldo + gcol0) = pl;
-      }
+      const int64_t o = tr ? gcol * g.ldo + i0 + 4 * lg : static_cast<int64_t>(i0 + major) * g.ldo + gcol;
+      uint2 ph, pl;
+      memcpy(&ph, hi, 8);
+      memcpy(&pl, lo, 8);
+      *reinterpret_cast<uint2*>(out + o) = ph;
+      if (out_lo) *reinterpret_cast<uint2*>(out_lo + o) = pl;
     }
   }
   cluster_sync_all();  // no CTA leaves while a peer still reads its tile
@@ -391,11 +438,10 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 }
 
 // ---------------------------------------------------------------- host side
-// Stage depths <A (expanded), B (bf16 operand), raw codes>: two CTAs per SM
-// where 64-wide (and 128-wide K-major) tiles allow, one otherwise.
-template <int BN> using KCfg = SkCfg<BN, false, false, 3, (BN == 128 ? 2 : 3), (BN == 128 ? 3 : 4), (BN <= 128 ? 2 : 1)>;
-template <int BN> using MCfg = SkCfg<BN, true, true, (BN == 256 ? 2 : 3), (BN == 64 ? 2 : (BN == 128 ? 3 : 2)),
-                                     (BN == 64 ? 3 : 4), (BN == 64 ? 2 : 1)>;
+// Stages of [A 16 KB | expanded codes 32 KB] and a deeper ring of 16 KB raw
+// code tiles, which carries the HBM latency more cheaply.
+using KCfg = SkCfg<false, 3, 4>;  // T^T, U^T: codes are the K-major operand
+using MCfg = SkCfg<true, 3, 4>;   // dB^T, dA: codes are the MN-major operand
 
 template <class C>
 cudaError_t launch_skinny(const CUtensorMap (&maps)[6], const SkinnyArgs& args, int grid,
@@ -426,87 +472,84 @@ cudaError_t launch_skinny(const CUtensorMap (&maps)[6], const SkinnyArgs& args, 
                             maps[5], args);
 }
 
-int skinny_bn(int64_t r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
-
-// One product: rows_out x r output, contraction kc.
+// One product: out (r x cols, or its transpose) = A-op . codes, contraction kc.
 struct Product {
-  int64_t rows_out, kc;
+  int64_t cols, kc;
   void* out;
   void* out_lo;
   int64_t ldo;
-  bool transpose, b_mn;
+  bool transpose, a_mn, hilo;
   const float* scale;
-  CUtensorMap raw, b, b2;
+  CUtensorMap raw, a, a2;
 };
 
 // Launches one or two products (the second may be null) as one grid.
-template <template <int> class CF>
+template <class C>
 cudaError_t run_products(const Product* p0, const Product* p1, int64_t r, const DeviceInfo* di,
                          int32_t* dev_status, cudaStream_t stream) {
-  const int bn = skinny_bn(r);
-  const int n_tiles = ceil_div(r, bn);
-  const int per_sm = bn == 64 || (bn == 128 && !CF<128>::AMn) ? 2 : 1;
   const Product* ps[2] = {p0, p1};
   int tiles[2] = {0, 0}, kbt[2] = {0, 0};
   for (int i = 0; i < 2; ++i) {
     if (!ps[i]) continue;
-    tiles[i] = ceil_div(ps[i]->rows_out, kBM) * n_tiles;
-    kbt[i] = ceil_div(ps[i]->kc, 64);
+    tiles[i] = ceil_div(r, ps[i]->hilo ? 64 : kBM) * ceil_div(ps[i]->cols, kSkN);
+    kbt[i] = ceil_div(ps[i]->kc, kSkK);
   }
   // one split count for the whole grid (the cluster size is per launch)
   const int kb_min = p1 ? std::min(kbt[0], kbt[1]) : kbt[0];
-  const int splits = choose_splits(tiles[0] + tiles[1], kb_min, per_sm * di->sm_count);
+  const int splits = choose_splits(tiles[0] + tiles[1], kb_min, di->sm_count);
   SkinnyArgs args{};
   args.dev_status = dev_status;
   CUtensorMap maps[6];
   for (int i = 0; i < 2; ++i) {
     const Product* p = ps[i] ? ps[i] : ps[0];
     SkinnyProblem& q = args.p[i];
-    q.m_tiles = ceil_div(p->rows_out, kBM);
-    q.n_tiles = n_tiles;
+    q.m_tiles = ceil_div(r, p->hilo ? 64 : kBM);
+    q.n_tiles = ceil_div(p->cols, kSkN);
     q.splits = splits;
-    q.kb_total = ceil_div(p->kc, 64);
+    q.kb_total = ceil_div(p->kc, kSkK);
     q.kb_per_split = ceil_div(q.kb_total, splits);
-    q.M = p->rows_out;
-    q.N = r;
+    q.rows = r;
+    q.cols = p->cols;
     q.out = p->out;
     q.out_lo = p->out_lo;
     q.ldo = p->ldo;
     q.transpose = p->transpose ? 1 : 0;
-    q.b_mn = p->b_mn ? 1 : 0;
+    q.a_mn = p->a_mn ? 1 : 0;
+    q.hilo = p->hilo ? 1 : 0;
     q.scale = p->scale;
     maps[3 * i] = p->raw;
-    maps[3 * i + 1] = p->b;
-    maps[3 * i + 2] = p->b2;
+    maps[3 * i + 1] = p->a;
+    maps[3 * i + 2] = p->a2;
   }
-  args.ctas0 = args.p[0].m_tiles * n_tiles * splits;
-  const int grid = args.ctas0 + (p1 ? args.p[1].m_tiles * n_tiles * splits : 0);
-  switch (bn) {
-    case 64: return launch_skinny<CF<64>>(maps, args, grid, stream);
-    case 128: return launch_skinny<CF<128>>(maps, args, grid, stream);
-    default: return launch_skinny<CF<256>>(maps, args, grid, stream);
-  }
+  args.ctas0 = args.p[0].m_tiles * args.p[0].n_tiles * splits;
+  const int grid = args.ctas0 + (p1 ? args.p[1].m_tiles * args.p[1].n_tiles * splits : 0);
+  return launch_skinny<C>(maps, args, grid, stream);
 }
 
 // Tensor map over an E4M3 code matrix [rows, cols] for the raw-code ring,
-// unswizzled: K-major (contraction along cols) boxes are 128 rows x 64 codes;
-// MN-major (contraction along rows) boxes are 64 rows x 128 codes.
+// unswizzled: K-major (contraction along cols) boxes are 256 rows x 64 codes;
+// MN-major (contraction along rows) boxes are 64 rows x 256 codes.
 bool codes_tmap(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t cols, bool mn_major) {
   return make_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, codes, static_cast<uint64_t>(cols),
-                      static_cast<uint64_t>(rows), mn_major ? 128 : 64, mn_major ? 64 : 128, false);
+                      static_cast<uint64_t>(rows), mn_major ? kSkN : kSkK, mn_major ? kSkK : kSkN, false);
 }
+
+// Row stride (elements) of the transposed T / U workspace: M rounded up so
+// that rows start 16-byte aligned.
+int64_t tu_ld(int64_t M) { return (M + 7) / 8 * 8; }
 
 }  // namespace
 
-// Workspace: T_hi, T_lo, U_hi, U_lo, each bf16 [M, r].  T and U are carried
-// as bf16 hi/lo pairs (about 16 significant bits): a single bf16 rounding of
-// T would move small dB entries by more than one bf16 ulp of the tensor's
-// scale.  The split-K sums never leave the chip (cluster reduction).
+// Workspace: T_hi^T, T_lo^T, U_hi^T, U_lo^T, each bf16 [r, M] (rows padded to
+// a multiple of 8 elements).  T and U are carried as bf16 hi/lo pairs (about
+// 16 significant bits): a single bf16 rounding of T would move small dB
+// entries by more than one bf16 ulp of the tensor's scale.  The split-K sums
+// never leave the chip (cluster reduction).
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da) {
   (void)N;
   (void)K;
   (void)want_da;
-  const size_t tu = align_up(static_cast<size_t>(M) * r * 2, 256);
+  const size_t tu = align_up(static_cast<size_t>(tu_ld(M)) * r * 2, 256);
   return 4 * tu;
 }
 
@@ -517,51 +560,52 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t tu = align_up(static_cast<size_t>(M) * r * 2, 256);
+  const int64_t ld = tu_ld(M);
+  const size_t tu = align_up(static_cast<size_t>(ld) * r * 2, 256);
   void* T_hi = ws;
   void* T_lo = ws + tu;
   void* U_hi = ws + 2 * tu;
   void* U_lo = ws + 3 * tu;
   const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int bn = skinny_bn(r);
-  const uint32_t bn_box = static_cast<uint32_t>(bn);
 
-  // stage 1: T = Xq . A^T / s_x (for dB) and U = dYq . B / s_dy (for dA), one grid
+  // stage 1: T^T = A . Xq^T / s_x (for dB) and U^T = B^T . dYq^T / s_dy (for dA), one grid
   Product t{}, u{};
   if (dB) {
-    t.rows_out = M; t.kc = K; t.out = T_hi; t.out_lo = T_lo; t.ldo = r;
-    t.transpose = false; t.b_mn = false; t.scale = s_x;
-    if (!codes_tmap(&t.raw, xq, M, K, false) || !make_tmap_2d(&t.b, BF, 2, A, K, r, 64, bn_box, true))
+    t.cols = M; t.kc = K; t.out = T_hi; t.out_lo = T_lo; t.ldo = ld;
+    t.transpose = false; t.a_mn = false; t.hilo = false; t.scale = s_x;
+    if (!codes_tmap(&t.raw, xq, M, K, false) || !make_tmap_2d(&t.a, BF, 2, A, K, r, kSkK, kBM, true))
       return cudaErrorInvalidValue;
-    t.b2 = t.b;
+    t.a2 = t.a;
   }
   if (dA) {
-    u.rows_out = M; u.kc = N; u.out = U_hi; u.out_lo = U_lo; u.ldo = r;
-    u.transpose = false; u.b_mn = true; u.scale = s_dy;
-    if (!codes_tmap(&u.raw, dyq, M, N, false) || !make_tmap_2d(&u.b, BF, 2, B, r, N, 64, 64, true))
+    u.cols = M; u.kc = N; u.out = U_hi; u.out_lo = U_lo; u.ldo = ld;
+    u.transpose = false; u.a_mn = true; u.hilo = false; u.scale = s_dy;
+    if (!codes_tmap(&u.raw, dyq, M, N, false) || !make_tmap_2d(&u.a, BF, 2, B, r, N, 64, kSkK, true))
       return cudaErrorInvalidValue;
-    u.b2 = u.b;
+    u.a2 = u.a;
   }
   cudaError_t e;
   if (dB && dA) e = run_products<KCfg>(&t, &u, r, di, dev_status, stream);
   else e = run_products<KCfg>(dB ? &t : &u, nullptr, r, di, dev_status, stream);
   if (e != cudaSuccess) return e;
 
-  // stage 2: dB = dYq^T . (T_hi + T_lo) / s_dy and dA^T = Xq^T . (U_hi + U_lo) / s_x
+  // stage 2: dB^T = (T_hi + T_lo)^T . dYq / s_dy, stored as dB [N, r], and
+  // dA = (U_hi + U_lo)^T . Xq / s_x [r, K]
   Product db{}, da{};
   if (dB) {
-    db.rows_out = N; db.kc = M; db.out = dB; db.out_lo = nullptr; db.ldo = r;
-    db.transpose = false; db.b_mn = true; db.scale = s_dy;
-    if (!codes_tmap(&db.raw, dyq, M, N, true) || !make_tmap_2d(&db.b, BF, 2, T_hi, r, M, 64, 64, true) ||
-        !make_tmap_2d(&db.b2, BF, 2, T_lo, r, M, 64, 64, true))
+    db.cols = N; db.kc = M; db.out = dB; db.out_lo = nullptr; db.ldo = r;
+    db.transpose = true; db.a_mn = false; db.hilo = true; db.scale = s_dy;
+    if (!codes_tmap(&db.raw, dyq, M, N, true) ||
+        !make_tmap_2d(&db.a, BF, 2, T_hi, M, r, kSkK, 64, true, ld) ||
+        !make_tmap_2d(&db.a2, BF, 2, T_lo, M, r, kSkK, 64, true, ld))
       return cudaErrorInvalidValue;
   }
   if (dA) {
-    // stored transposed into dA [r, K]
-    da.rows_out = K; da.kc = M; da.out = dA; da.out_lo = nullptr; da.ldo = K;
-    da.transpose = true; da.b_mn = true; da.scale = s_x;
-    if (!codes_tmap(&da.raw, xq, M, K, true) || !make_tmap_2d(&da.b, BF, 2, U_hi, r, M, 64, 64, true) ||
-        !make_tmap_2d(&da.b2, BF, 2, U_lo, r, M, 64, 64, true))
+    da.cols = K; da.kc = M; da.out = dA; da.out_lo = nullptr; da.ldo = K;
+    da.transpose = false; da.a_mn = false; da.hilo = true; da.scale = s_x;
+    if (!codes_tmap(&da.raw, xq, M, K, true) ||
+        !make_tmap_2d(&da.a, BF, 2, U_hi, M, r, kSkK, 64, true, ld) ||
+        !make_tmap_2d(&da.a2, BF, 2, U_lo, M, r, kSkK, 64, true, ld))
       return cudaErrorInvalidValue;
   }
   if (dB && dA) return run_products<MCfg>(&db, &da, r, di, dev_status, stream);

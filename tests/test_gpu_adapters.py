@@ -50,6 +50,8 @@ CASES = [
     (128, 256, 512, 320),   # two r tiles
     (2048, 256, 4096, 16),  # 16 row tiles: split-K clusters of 8
     (1000, 4096, 1024, 64), # many dB/dA^T tiles, few splits
+    (3, 256, 512, 16),      # fewer tokens than one K block of dB / dA
+    (333, 512, 768, 192),   # odd M (padded T/U rows); r over one rank tile
 ]
 
 
