@@ -312,9 +312,6 @@ __global__ void __launch_bounds__(C::Threads, 1)
     const int tcol = (t % kThrPerRow) * 16;
     const int blk = tcol / 64;
     const int unit0 = (tcol % 64) / 8;
-    // MN-major: the two column blocks a quarter-warp writes share banks, so
-    // odd blocks store their two 16-byte units in the opposite order
-    const bool swap = C::BMn && (blk & 1);
     for (int i = 0; i < nkb; ++i) {
       const int sr = i % C::SR, s = i % C::S;
       if (!warp_wait(&rawfull[sr], static_cast<uint32_t>((i / C::SR) & 1), abort_flag)) {
@@ -328,6 +325,10 @@ __global__ void __launch_bounds__(C::Threads, 1)
                                                (trow + j * kRowStep) * C::RawRowBytes + tcol);
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[sr]);
+      uint32_t nan_acc = 0u;
+#pragma unroll
+      for (int j = 0; j < C::ChunksPerThread; ++j) nan_acc = nan_fold(nan_acc, q[j]);
+      const bool nan = nan_found(nan_acc);
       if (!warp_wait(&empty[s], static_cast<uint32_t>(((i / C::S) & 1) ^ 1), abort_flag)) {
         if (lane == 0) fail();
         break;
@@ -336,14 +337,12 @@ __global__ void __launch_bounds__(C::Threads, 1)
 #pragma unroll
       for (int j = 0; j < C::ChunksPerThread; ++j) {
         uint32_t o[8];
-        e4m3x16_to_bf16(q[j], o);
+        e4m3x16_to_bf16(q[j], nan, o);
         const int row = trow + j * kRowStep;
-        const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]);
-        const uint4 hi = make_uint4(o[4], o[5], o[6], o[7]);
-        const uint32_t off_lo = row * kRowBytes + ((unit0 ^ (row & 7)) << 4);
-        const uint32_t off_hi = row * kRowBytes + (((unit0 + 1) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(sB + (swap ? off_hi : off_lo)) = swap ? hi : lo;
-        *reinterpret_cast<uint4*>(sB + (swap ? off_lo : off_hi)) = swap ? lo : hi;
+        *reinterpret_cast<uint4*>(sB + row * kRowBytes + ((unit0 ^ (row & 7)) << 4)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(sB + row * kRowBytes + (((unit0 + 1) ^ (row & 7)) << 4)) =
+            make_uint4(o[4], o[5], o[6], o[7]);
       }
       fence_proxy_async_smem();
       // the stage's A tile must have landed too: pconv[] then covers both operands

@@ -36,28 +36,32 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int ks) {
   return operand_desc_rt<kElemBytes, kKRows>(kMn, base, ks);
 }
 
-// Two E4M3 codes, in bytes 0 and 2 of x (bytes 1 and 3 zero), to a bf16x2
-// word, exactly.  Shifted left by 4, a code's exponent and mantissa fields
-// land on the bf16 exponent and the top of the bf16 mantissa, so the word
-// reads as the code's value times 2^-120 (E4M3 bias 7 against bf16 bias 127;
-// E4M3 subnormals land on bf16 subnormals, which scale the same way).  The
-// sign, left at bit 11, moves to bit 15 by adding 15 * 2^11 (= 2^15 - 2^11),
-// and one bf16 multiply by 2^120 (plus -0) restores the value with no
+// Two E4M3 codes (bytes `sel` picks from w) to a bf16x2 word, exactly.  The
+// byte permute puts each code in the low byte of its 16-bit lane and its sign
+// bit, replicated, in the high byte.  Shifted left by 4 and masked, the
+// lane holds the sign at bit 15 and the code's exponent and mantissa fields
+// on the low four bits of the bf16 exponent and the top of the bf16
+// mantissa: it reads as the code's value times 2^-120 (E4M3 bias 7 against
+// bf16 bias 127; E4M3 subnormals land on bf16 subnormals, which scale the
+// same way).  One bf16 multiply by 2^120 (plus -0) restores the value with no
 // rounding.  NaN codes (0x7F, 0xFF) are not handled here.
-__device__ __forceinline__ uint32_t e4m3_pair_to_bf16x2(uint32_t x) {
-  uint32_t h = x << 4;
-  h += 15u * (h & 0x08000800u);
-  uint32_t out;
+template <uint32_t kSel>
+__device__ __forceinline__ uint32_t e4m3_pair_to_bf16x2(uint32_t w) {
+  uint32_t y, out;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(w), "n"(kSel));
+  const uint32_t h = (y << 4) & 0x87F087F0u;
   asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out) : "r"(h), "r"(0x7B807B80u), "r"(0x80008000u));
   return out;
 }
 
-// Nonzero iff one of the 16 codes is a NaN code (magnitude bits all ones).
-__device__ __forceinline__ uint32_t has_nan_code(uint4 q) {
+// Accumulates NaN evidence over code words: bit 7 of a byte of the result of
+// nan_fold ends up set iff that byte of some folded word had all seven
+// magnitude bits set (a NaN code); test with nan_found.
+__device__ __forceinline__ uint32_t nan_fold(uint32_t acc, uint4 q) {
   const uint32_t m = 0x7F7F7F7Fu, one = 0x01010101u;
-  return (((q.x & m) + one) | ((q.y & m) + one) | ((q.z & m) + one) | ((q.w & m) + one)) &
-         0x80808080u;
+  return acc | ((q.x & m) + one) | ((q.y & m) + one) | ((q.z & m) + one) | ((q.w & m) + one);
 }
+__device__ __forceinline__ bool nan_found(uint32_t acc) { return (acc & 0x80808080u) != 0u; }
 
 // Four codes -> four bf16 (two words) through the hardware conversion; exact
 // for every code, NaN included.
@@ -78,14 +82,15 @@ __device__ __forceinline__ void e4m3x4_to_bf16_hw(uint32_t w, uint32_t& lo, uint
   hi = o[1];
 }
 
-// Sixteen codes -> sixteen bf16 (eight words, in code order).
-__device__ __forceinline__ void e4m3x16_to_bf16(uint4 q, uint32_t (&o)[8]) {
+// Sixteen codes -> sixteen bf16 (eight words, in code order); `nan` selects
+// the hardware conversion, which also carries NaN codes.
+__device__ __forceinline__ void e4m3x16_to_bf16(uint4 q, bool nan, uint32_t (&o)[8]) {
   const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-  if (!has_nan_code(q)) {
+  if (!nan) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      o[2 * j] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4140));
-      o[2 * j + 1] = e4m3_pair_to_bf16x2(__byte_perm(words[j], 0u, 0x4342));
+      o[2 * j] = e4m3_pair_to_bf16x2<0x9180u>(words[j]);      // codes 0, 1 of the word
+      o[2 * j + 1] = e4m3_pair_to_bf16x2<0xB3A2u>(words[j]);  // codes 2, 3
     }
   } else {
 #pragma unroll
