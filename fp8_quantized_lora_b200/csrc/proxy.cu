@@ -28,7 +28,7 @@
 //     written back, and t = dec(c) + s_W * P' (no FMA) is re-encoded.  Codes
 //     whose value changes are written at once -- such a change already
 //     selects the row -- and the row's flag is set.
-//   proxy_clear_kernel  (grid over rows)
+//   proxy_clear_kernel  (one warp per row)
 //     Selected rows get P = +0; writes the row mask and the selected count.
 // Every step is reproduced bit-for-bit by the float32 arithmetic.
 #include <cuda_fp16.h>
@@ -471,25 +471,39 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 }
 
 constexpr int kClearThreads = 256;
+constexpr int kClearWarps = kClearThreads / 32;
 
+// One warp per row: the lanes read the row's verdict bytes once each and
+// agree on their OR; a selected row is then cleared by the same warp with
+// 16-byte stores.
 __global__ void __launch_bounds__(kClearThreads)
     proxy_clear_kernel(float* __restrict__ proxy, int64_t N, int64_t K, int ncb,
                        const uint8_t* __restrict__ rowflag, uint8_t* __restrict__ row_mask,
                        int32_t* __restrict__ n_selected) {
+  __shared__ int warp_count[kClearWarps];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   int count = 0;
-  for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
-    // OR of the row's per-column-block verdicts (every CTA thread computes it)
-    int sel = 0;
-    for (int c = 0; c < ncb; ++c) sel |= rowflag[n * ncb + c];
-    if (threadIdx.x == 0) {
-      if (row_mask) row_mask[n] = static_cast<uint8_t>(sel);
-      count += sel;
+  for (int64_t n = static_cast<int64_t>(blockIdx.x) * kClearWarps + warp; n < N;
+       n += static_cast<int64_t>(gridDim.x) * kClearWarps) {
+    uint32_t f = 0;
+    for (int c = lane; c < ncb; c += 32) f |= rowflag[n * ncb + c];
+    const bool sel = __any_sync(0xFFFFFFFFu, f != 0u);
+    if (lane == 0) {
+      if (row_mask) row_mask[n] = sel ? 1 : 0;
+      count += sel ? 1 : 0;
     }
     if (!sel) continue;
     float4* row = reinterpret_cast<float4*>(proxy + n * K);
-    for (int64_t c = threadIdx.x; c < K / 4; c += kClearThreads) row[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t c = lane; c < K / 4; c += 32) row[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (threadIdx.x == 0 && count && n_selected) atomicAdd(n_selected, count);
+  if (lane == 0) warp_count[warp] = count;
+  __syncthreads();
+  if (threadIdx.x == 0 && n_selected) {
+    int total = 0;
+    for (int w = 0; w < kClearWarps; ++w) total += warp_count[w];
+    if (total) atomicAdd(n_selected, total);
+  }
 }
 
 template <bool kAcc, bool kSel>
@@ -583,7 +597,9 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
     e = launch_stream<false, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
                                    dev_status, stream);
   if (e != cudaSuccess || !sel) return e;
-  int64_t blocks = N < static_cast<int64_t>(di->sm_count) * 8 ? N : static_cast<int64_t>(di->sm_count) * 8;
+  const int64_t row_blocks = (N + kClearWarps - 1) / kClearWarps;
+  const int64_t blocks = row_blocks < static_cast<int64_t>(di->sm_count) * 8 ? row_blocks
+                                                                              : static_cast<int64_t>(di->sm_count) * 8;
   proxy_clear_kernel<<<static_cast<int>(blocks), kClearThreads, 0, stream>>>(proxy, N, K, ncb, rowflag,
                                                                              row_mask, n_selected);
   return cudaGetLastError();

@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads)
 // (bounded) until all words are marked, reduces them, and pass 2 streams the
 // same run again -- it is still in L2 -- and writes the codes.
 constexpr int kChunkBytes = 16384;
-constexpr int kStreamStages = 8;                       // 128 KB in flight per SM
+constexpr int kStreamStages = 13;                      // 208 KB in flight per SM
 constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
@@ -405,7 +405,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   // CTA is resident).  A CTA's word is its max with bit 31 set as the arrival
   // mark (a magnitude pattern never has it); the words were zeroed before the
   // launch.  Warp 0 of every CTA polls all words (relaxed loads, one acquire
-  // fence once all are marked), bounded, and reduces them.
+  // fence once all are marked), bounded, and reduces them.  A poll round
+  // issues all of a lane's loads before it looks at any: one L2 round trip
+  // per round, not one per word.
   uint32_t* partials = ws + kBarWords;
   __shared__ uint32_t amax_bits;
   if (warp == 0) {
@@ -415,14 +417,24 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     __syncwarp();
     const long long t0 = clock64();
     uint32_t mx = 0;
+    constexpr int kPerLane = 8;  // words per lane per batch of loads (256 CTAs)
     while (true) {
       bool all = true;
       mx = 0;
-      for (int i = lane; i < static_cast<int>(gridDim.x); i += 32) {
-        uint32_t w;
-        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w) : "l"(partials + i) : "memory");
-        all = all && (w >> 31) != 0u;
-        mx = max(mx, w & 0x7FFFFFFFu);
+      for (int b = 0; b < static_cast<int>(gridDim.x); b += 32 * kPerLane) {
+        uint32_t w[kPerLane];
+#pragma unroll
+        for (int k = 0; k < kPerLane; ++k) {
+          const int i = b + lane + 32 * k;
+          w[k] = 0x80000000u;  // absent CTAs count as arrived with max 0
+          if (i < static_cast<int>(gridDim.x))
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w[k]) : "l"(partials + i));
+        }
+#pragma unroll
+        for (int k = 0; k < kPerLane; ++k) {
+          all = all && (w[k] >> 31) != 0u;
+          mx = max(mx, w[k] & 0x7FFFFFFFu);
+        }
       }
       if (__all_sync(0xFFFFFFFFu, all)) {
         asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the marked words
