@@ -217,6 +217,28 @@ class Step:
 # FP32 lanes x 2 flops x 1.965 GHz (the B200's boost clock)
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
+# DRAM traffic per call of a phase (dram__bytes_read.sum + dram__bytes_write.sum
+# of every kernel the call launches, from one ncu capture of the bench's own
+# workload; the command and the figures are in the named profile).  A figure
+# holds only for the kernel sources it was measured on: when a source's hash
+# differs, the roofline's traffic is null.
+TRAFFIC = {}
+
+
+def _traffic(phase):
+    import hashlib
+    t = TRAFFIC.get(phase)
+    if not t:
+        return None
+    for path, digest in t["sources"].items():
+        try:
+            with open(os.path.join(ROOT, path), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return t["bytes"]
+
 
 def _phase_work(st):
     """Algorithmic work and bound of each phase: flops, bytes (each tensor
@@ -427,7 +449,9 @@ def run_gpu(args):
         roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "hbm",
                 "achieved": phases[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": phases[dom]["frac_hbm"], "peak_source": f"{peaks['source']} copy bandwidth"}
-    roof["traffic"] = None
+    roof["traffic"] = _traffic(dom)
+    if roof["traffic"] is not None:
+        roof["traffic_source"] = TRAFFIC[dom]["profile"]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,

@@ -100,6 +100,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -255,8 +257,7 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const Gemm
   }
   const int total = g.m_tiles * g.n_tiles;
   const int grid = total < di->sm_count ? total : di->sm_count;
-  tc_gemm_kernel<C><<<grid, C::Threads, C::SmemBytes, stream>>>(tA, tB, g);
-  return cudaGetLastError();
+  return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, g);
 }
 
 // 128 x 256 tiles for both: narrower tiles fill the last wave better (a

@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const uint16_t* __restrict__ A, int64_t N, int64_t K, int r,
                         uint8_t* __restrict__ rowflag, int32_t* __restrict__ n_selected,
                         int32_t* __restrict__ dev_status) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int tile_flag[kTileRows];  // a code of the row changed in this tile
   uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kIChunk][256]
@@ -287,6 +289,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
                       const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
                       int units, int ncb, uint8_t* __restrict__ rowflag,
                       int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status) {
+  // No early trigger: the clear kernel that follows needs no shared memory, so
+  // its CTAs would sit beside this kernel's on the SMs while they wait.
+  pdl_wait();  // the previous kernel's results are complete and visible
   extern __shared__ __align__(16) uint8_t sm[];
   float4* pst = reinterpret_cast<float4*>(sm);                                 // [8][2][128]
   uint2* wst = reinterpret_cast<uint2*>(sm + kPipePBytes);                     // [8][128]
@@ -480,6 +485,8 @@ __global__ void __launch_bounds__(kClearThreads)
     proxy_clear_kernel(float* __restrict__ proxy, int64_t N, int64_t K, int ncb,
                        const uint8_t* __restrict__ rowflag, uint8_t* __restrict__ row_mask,
                        int32_t* __restrict__ n_selected) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
   __shared__ int warp_count[kClearWarps];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -520,10 +527,9 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  proxy_stream_kernel<kAcc, kSel><<<grid, kThreads, kSmemBytes, stream>>>(
-      wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
-      r, rowflag, n_selected, dev_status);
-  return cudaGetLastError();
+  return launch_pdl(proxy_stream_kernel<kAcc, kSel>, grid, dim3(kThreads), kSmemBytes, stream, 1u, wq, s_w,
+                    proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
+                    rowflag, n_selected, dev_status);
 }
 
 template <bool kSel>
@@ -541,10 +547,9 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  proxy_pipe_kernel<kSel><<<grid, kPipeThreads, kPipeSmemBytes, stream>>>(
-      wq, s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K,
-      r, row_groups, units, ncb, rowflag, n_selected, dev_status);
-  return cudaGetLastError();
+  return launch_pdl(proxy_pipe_kernel<kSel>, dim3(grid), dim3(kPipeThreads), kPipeSmemBytes, stream, 1u, wq,
+                    s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
+                    row_groups, units, ncb, rowflag, n_selected, dev_status);
 }
 
 }  // namespace
@@ -600,9 +605,8 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   const int64_t row_blocks = (N + kClearWarps - 1) / kClearWarps;
   const int64_t blocks = row_blocks < static_cast<int64_t>(di->sm_count) * 8 ? row_blocks
                                                                               : static_cast<int64_t>(di->sm_count) * 8;
-  proxy_clear_kernel<<<static_cast<int>(blocks), kClearThreads, 0, stream>>>(proxy, N, K, ncb, rowflag,
-                                                                             row_mask, n_selected);
-  return cudaGetLastError();
+  return launch_pdl(proxy_clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
+                    proxy, N, K, ncb, rowflag, row_mask, n_selected);
 }
 
 }  // namespace falqon

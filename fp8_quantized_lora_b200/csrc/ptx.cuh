@@ -78,6 +78,14 @@ __device__ __forceinline__ bool mbar_wait_budget(uint64_t* bar, uint32_t parity)
   return true;
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the grids this one
+// depends on have completed and their memory is visible (returns at once
+// when the launch did not enable the overlap).  pdl_trigger: let the next
+// grid in the stream start launching (it still waits for this one before it
+// touches memory).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Generic-proxy writes to shared memory become visible to the async proxy
 // (tensor cores, TMA) after this fence.
 __device__ __forceinline__ void fence_proxy_async_smem() {

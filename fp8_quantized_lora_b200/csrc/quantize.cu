@@ -96,6 +96,8 @@ template <bool kBF16>
 __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const void* __restrict__ x,
                                                                 int64_t n,
                                                                 uint32_t* __restrict__ partials) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
   __shared__ uint32_t red[32];
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -259,6 +261,8 @@ __global__ void __launch_bounds__(kThreads)
                          uint8_t* __restrict__ codes, float* __restrict__ scale_out,
                          float* __restrict__ amax_out, float* __restrict__ residual,
                          int32_t* __restrict__ dev_status) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
   __shared__ uint32_t red[32];
   __shared__ float s_shared;
   const float s = fold_and_scale(partials, nparts, red, &s_shared, scale_out, amax_out, dev_status);
@@ -323,6 +327,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // (no-op: this launch is cooperative and waits in order)
 
   int stage = 0;
   uint32_t phase = 0;
@@ -581,15 +587,15 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
   if (cb > ccap) cb = ccap;
   if (cb < 1) cb = 1;
   if (is_bf16) {
-    amax_partial_kernel<true><<<pb, kThreads, 0, stream>>>(x, n, partials);
-    quantize_cast_kernel<true><<<static_cast<int>(cb), kThreads, 0, stream>>>(
-        x, n, partials, pb, codes, scale, amax, residual, dev_status);
-  } else {
-    amax_partial_kernel<false><<<pb, kThreads, 0, stream>>>(x, n, partials);
-    quantize_cast_kernel<false><<<static_cast<int>(cb), kThreads, 0, stream>>>(
-        x, n, partials, pb, codes, scale, amax, residual, dev_status);
+    cudaError_t e = launch_pdl(amax_partial_kernel<true>, dim3(pb), dim3(kThreads), 0, stream, 1u, x, n, partials);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(quantize_cast_kernel<true>, dim3(static_cast<unsigned>(cb)), dim3(kThreads), 0, stream, 1u, x,
+                      n, static_cast<const uint32_t*>(partials), pb, codes, scale, amax, residual, dev_status);
   }
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(amax_partial_kernel<false>, dim3(pb), dim3(kThreads), 0, stream, 1u, x, n, partials);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(quantize_cast_kernel<false>, dim3(static_cast<unsigned>(cb)), dim3(kThreads), 0, stream, 1u, x,
+                    n, static_cast<const uint32_t*>(partials), pb, codes, scale, amax, residual, dev_status);
 }
 
 }  // namespace falqon

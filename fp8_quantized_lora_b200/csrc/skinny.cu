@@ -161,6 +161,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
 
   auto fail = [&]() {
     *abort_flag = 1;
@@ -455,20 +457,9 @@ cudaError_t launch_skinny(const CUtensorMap (&maps)[6], const SkinnyArgs& args, 
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(args.p[0].splits);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(C::Threads);
-  cfg.dynamicSmemBytes = C::SmemBytes;
-  cfg.stream = stream;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, skinny_kernel<C>, maps[0], maps[1], maps[2], maps[3], maps[4],
-                            maps[5], args);
+  return launch_pdl(skinny_kernel<C>, dim3(static_cast<unsigned>(grid)), dim3(C::Threads), C::SmemBytes,
+                    stream, static_cast<unsigned>(args.p[0].splits), maps[0], maps[1], maps[2], maps[3],
+                    maps[4], maps[5], args);
 }
 
 // One product: out (r x cols, or its transpose) = A-op . codes, contraction kc.
