@@ -7,12 +7,18 @@
 // FALQON's point (paper introduction) is that both run on the FP8 backbone
 // alone: the adapter is merged into Wq, so there is no separate LoRA path.
 //
-// Roles (one CTA per SM, persistent over 128 x 256 output tiles):
+// Roles (persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer (one lane): fills a `kStages`-deep smem ring.
-//   warp 1      TMEM owner and UMMA issuer (one lane issues, the warp waits).
+//   warp 1      TMEM owner and UMMA issuer (one lane issues).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, bf16 store.
-// The accumulator lives in TMEM, double-buffered (2 x BN fp32 columns), so
-// the epilogue of one tile overlaps the MMAs of the next.
+//   warp 6      MMA waiter: waits on the stage and accumulator mbarriers and
+//               releases the issuer through a named barrier.  An mbarrier
+//               wait in the issuing thread holds back its MMA stream until
+//               the MMAs in flight retire (measured: half the tensor rate
+//               with a wait every 4 UMMAs); a named barrier does not.
+// The accumulator lives in TMEM (kAcc buffers of BN fp32 columns); with two
+// buffers the epilogue of one tile overlaps the MMAs of the next.  (Two CTAs
+// per SM with a 2-stage ring and one accumulator each measured slower.)
 //
 // Every operand tile in smem is a stack of 128-byte rows in the SWIZZLE_128B
 // layout TMA writes: K-major tiles are [rows][128 B of K]; MN-major tiles are
@@ -26,6 +32,8 @@
 namespace falqon {
 namespace {
 
+constexpr int kMmaBar = 1;  // named barrier between the MMA issuer and its waiter
+
 struct GemmArgs {
   int32_t m_tiles, n_tiles, kb_total;
   int64_t M, N;            // output extent
@@ -36,29 +44,36 @@ struct GemmArgs {
   int32_t* dev_status;
 };
 
-template <bool kBMn, int kBN, int kStages>
+template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks>
 struct Cfg {
   static constexpr bool BMn = kBMn;
   static constexpr int BN = kBN;
   static constexpr int Stages = kStages;
+  static constexpr int Acc = kAcc;              // accumulator buffers in TMEM
+  static constexpr int MinBlocks = kMinBlocks;  // CTAs per SM
   static constexpr int BK = kRowBytes;                // K per stage (128 E4M3 codes)
   static constexpr int KSteps = BK / 32;              // UMMA K = 32 for 8-bit kinds
   static constexpr int ABytes = kBM * BK;             // 16 KB
   static constexpr int BBytes = kBN * BK;
   static constexpr int StageBytes = ABytes + BBytes;
-  static constexpr int Threads = 32 * 6;
-  // two accumulators of BN columns; allocations are powers of two >= 32
-  static constexpr uint32_t TmemCols = 2 * kBN <= 32 ? 32 : (2 * kBN <= 64 ? 64 : (2 * kBN <= 128 ? 128 : (2 * kBN <= 256 ? 256 : 512)));
-  static constexpr int BarBytes = 8 * (2 * kStages + 5) + 16;
+  static constexpr int WaiterWarp = 6;
+  static constexpr int Threads = 32 * 7;
+  // kAcc accumulators of BN columns; allocations are powers of two >= 32
+  static constexpr int AccCols = kAcc * kBN;
+  static constexpr uint32_t TmemCols = AccCols <= 32 ? 32 : (AccCols <= 64 ? 64 : (AccCols <= 128 ? 128 : (AccCols <= 256 ? 256 : 512)));
+  static constexpr int BarBytes = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
   static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
   static constexpr uint32_t IDesc = idesc_f32acc(0u, 0u, 0u, kBMn ? 1u : 0u, kBM, kBN);
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
   static_assert(!kBMn || kBN % kRowBytes == 0, "MN-major B needs 128-byte blocks");
   static_assert(SmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kMinBlocks * (SmemBytes + 1024) <= 233472, "shared memory per SM");
+  static_assert(kMinBlocks * TmemCols <= 512, "tensor memory per SM");
+  static_assert(kAcc == 1 || kAcc == 2, "accumulator buffers");
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::Threads, 1)
+__global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs g) {
   extern __shared__ uint8_t smem_dyn[];
@@ -67,9 +82,9 @@ __global__ void __launch_bounds__(C::Threads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::Stages * C::StageBytes);
   uint64_t* full = bars;                      // [Stages] TMA landed
   uint64_t* empty = bars + C::Stages;         // [Stages] MMAs done with the slot
-  uint64_t* acc_full = bars + 2 * C::Stages;  // [2] accumulator ready
-  uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained
-  uint64_t* drain = acc_empty + 2;            // all issued MMAs retired (teardown)
+  uint64_t* acc_full = bars + 2 * C::Stages;  // [Acc] accumulator ready
+  uint64_t* acc_empty = acc_full + C::Acc;    // [Acc] accumulator drained
+  uint64_t* drain = acc_empty + C::Acc;       // all issued MMAs retired (teardown)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -82,7 +97,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::Acc; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
@@ -146,17 +161,18 @@ __global__ void __launch_bounds__(C::Threads, 1)
     __syncwarp();  // the warp reaches the CTA barrier below together
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Released by the waiter once per tile (accumulator free) and once per K
+    // block (stage landed); the barrier's OR carries an abort, and both warps
+    // leave their loops at the same point.
     int stage = 0;
-    uint32_t phase = 0;
     int acc = 0;
-    uint32_t acc_phase = 0;
-    bool ok = true;
-    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-      if (!warp_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      if (bar_red_or(kMmaBar, 64, false)) break;
       tc_fence_after();
       const uint32_t tmem_d = tmem_base + acc * C::BN;
+      bool abort = false;
       for (int kb = 0; kb < g.kb_total; ++kb) {
-        if (!warp_wait(&full[stage], phase, abort_flag)) { if (lane == 0) fail(); ok = false; break; }
+        if (bar_red_or(kMmaBar, 64, false)) { abort = true; break; }
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a_base = smem_u32(smem + stage * C::StageBytes);
@@ -170,12 +186,12 @@ __global__ void __launch_bounds__(C::Threads, 1)
           umma_commit(&empty[stage]);
         }
         __syncwarp();
-        if (++stage == C::Stages) { stage = 0; phase ^= 1; }
+        if (++stage == C::Stages) stage = 0;
       }
-      if (!ok) break;
+      if (abort) break;
       if (lane == 0) umma_commit(&acc_full[acc]);
       __syncwarp();
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (++acc == C::Acc) acc = 0;
     }
     // drain the tensor pipe before TMEM is released
     if (lane == 0) {
@@ -183,6 +199,28 @@ __global__ void __launch_bounds__(C::Threads, 1)
       mbar_wait_budget(drain, 0);
     }
     __syncwarp();
+  } else if (warp == C::WaiterWarp) {
+    // ------------------------------------------------------------ MMA waiter
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int w = blockIdx.x; w < total; w += gridDim.x) {
+      const bool ok_acc = warp_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag);
+      if (!ok_acc && lane == 0) fail();
+      __syncwarp();  // converged at the (aligned) named barrier
+      if (bar_red_or(kMmaBar, 64, !ok_acc)) break;
+      bool abort = false;
+      for (int kb = 0; kb < g.kb_total; ++kb) {
+        const bool ok = warp_wait(&full[stage], phase, abort_flag);
+        if (!ok && lane == 0) fail();
+        __syncwarp();
+        if (bar_red_or(kMmaBar, 64, !ok)) { abort = true; break; }
+        if (++stage == C::Stages) { stage = 0; phase ^= 1; }
+      }
+      if (abort) break;
+      if (++acc == C::Acc) { acc = 0; acc_phase ^= 1; }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -229,7 +267,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (++acc == C::Acc) { acc = 0; acc_phase ^= 1; }
     }
   }
 
@@ -256,15 +294,16 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const Gemm
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
   const int total = g.m_tiles * g.n_tiles;
-  const int grid = total < di->sm_count ? total : di->sm_count;
+  const int slots = C::MinBlocks * di->sm_count;
+  const int grid = total < slots ? total : slots;
   return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, g);
 }
 
 // 128 x 256 tiles for both: narrower tiles fill the last wave better (a
 // 4096-square product makes 3.46 waves) but read more L2 bytes per flop, and
 // measured slower (128 x 192 and 128 x 128).
-using FwdCfg = Cfg<false, 256, 4>;
-using DxCfg = Cfg<true, 256, 4>;
+using FwdCfg = Cfg<false, 256, 4, 2, 1>;
+using DxCfg = Cfg<true, 256, 4, 2, 1>;
 
 template <class C>
 cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,

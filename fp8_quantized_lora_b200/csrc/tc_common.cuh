@@ -126,6 +126,24 @@ __device__ __forceinline__ float4 dsmem_load_f32x4(uint32_t addr) {
   return v;
 }
 
+// Named barrier `id` over `nthreads` threads (whole warps) that also ORs a
+// predicate across them: every participant gets true iff one passed true.
+// Unlike an mbarrier wait, it does not hold back the tcgen05.mma stream of an
+// issuing thread that takes part, so an MMA issuer can be released stage by
+// stage through it by a warp that does the mbarrier waits.
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0u;
+}
+
 // All lanes wait; the warp agrees on the outcome so it never diverges on a timeout.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort_flag) {
