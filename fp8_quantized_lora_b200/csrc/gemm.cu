@@ -44,22 +44,26 @@ struct GemmArgs {
   int32_t* dev_status;
 };
 
-template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks>
+template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks, int kHalves>
 struct Cfg {
   static constexpr bool BMn = kBMn;
   static constexpr int BN = kBN;
   static constexpr int Stages = kStages;
   static constexpr int Acc = kAcc;              // accumulator buffers in TMEM
   static constexpr int MinBlocks = kMinBlocks;  // CTAs per SM
+  static constexpr int Halves = kHalves;        // 128-row halves of a tile (one MMA each per K step)
+  static constexpr int TileM = kHalves * kBM;
   static constexpr int BK = kRowBytes;                // K per stage (128 E4M3 codes)
   static constexpr int KSteps = BK / 32;              // UMMA K = 32 for 8-bit kinds
-  static constexpr int ABytes = kBM * BK;             // 16 KB
+  static constexpr int AHalfBytes = kBM * BK;         // 16 KB
+  static constexpr int ABytes = kHalves * AHalfBytes;
   static constexpr int BBytes = kBN * BK;
   static constexpr int StageBytes = ABytes + BBytes;
-  static constexpr int WaiterWarp = 6;
-  static constexpr int Threads = 32 * 7;
-  // kAcc accumulators of BN columns; allocations are powers of two >= 32
-  static constexpr int AccCols = kAcc * kBN;
+  static constexpr int EpiWarps = 4 * kHalves;        // warps 2 .. 2 + EpiWarps - 1
+  static constexpr int WaiterWarp = 2 + EpiWarps;
+  static constexpr int Threads = 32 * (WaiterWarp + 1);
+  // kAcc accumulators of Halves x BN columns; allocations are powers of two >= 32
+  static constexpr int AccCols = kAcc * kHalves * kBN;
   static constexpr uint32_t TmemCols = AccCols <= 32 ? 32 : (AccCols <= 64 ? 64 : (AccCols <= 128 ? 128 : (AccCols <= 256 ? 256 : 512)));
   static constexpr int BarBytes = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
   static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
@@ -70,6 +74,8 @@ struct Cfg {
   static_assert(kMinBlocks * (SmemBytes + 1024) <= 233472, "shared memory per SM");
   static_assert(kMinBlocks * TmemCols <= 512, "tensor memory per SM");
   static_assert(kAcc == 1 || kAcc == 2, "accumulator buffers");
+  static_assert(kHalves == 1 || kHalves == 2, "tile halves");
+  static_assert(AccCols <= 512, "tensor memory");
 };
 
 template <class C>
@@ -99,7 +105,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     }
     for (int b = 0; b < C::Acc; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], C::EpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -133,7 +139,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int nt = w % g.n_tiles;
         const int mt = w / g.n_tiles;
-        const int m0 = mt * kBM, n0 = nt * C::BN;
+        const int m0 = mt * C::TileM, n0 = nt * C::BN;
         for (int kb = 0; kb < g.kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { fail(); ok = false; break; }
           uint8_t* sA = smem + stage * C::StageBytes;
@@ -141,7 +147,9 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
           mbar_arrive_expect_tx(&full[stage], C::StageBytes);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-          tma_load_2d(sA, &tmA, &full[stage], kb * C::BK, m0);  // rows m0.., K block kb
+#pragma unroll
+          for (int h = 0; h < C::Halves; ++h)  // rows m0 + 128 h .., K block kb
+            tma_load_2d(sA + h * C::AHalfBytes, &tmA, &full[stage], kb * C::BK, m0 + h * kBM);
           if constexpr (C::BMn) {
             // B is [K][N] row-major: 128-byte column blocks of BK rows each
 #pragma unroll
@@ -169,7 +177,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
       if (bar_red_or(kMmaBar, 64, false)) break;
       tc_fence_after();
-      const uint32_t tmem_d = tmem_base + acc * C::BN;
+      const uint32_t tmem_d = tmem_base + acc * C::Halves * C::BN;
       bool abort = false;
       for (int kb = 0; kb < g.kb_total; ++kb) {
         if (bar_red_or(kMmaBar, 64, false)) { abort = true; break; }
@@ -179,9 +187,11 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
           const uint32_t b_base = a_base + C::ABytes;
 #pragma unroll
           for (int ks = 0; ks < C::KSteps; ++ks) {
-            const uint64_t ad = operand_desc<false, 1, C::BK>(a_base, ks);
             const uint64_t bd = operand_desc<C::BMn, 1, C::BK>(b_base, ks);
-            umma_f8(tmem_d, ad, bd, C::IDesc, (kb > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < C::Halves; ++h)  // the halves share the B tile
+              umma_f8(tmem_d + h * C::BN, operand_desc<false, 1, C::BK>(a_base + h * C::AHalfBytes, ks), bd,
+                      C::IDesc, (kb > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
         }
@@ -223,7 +233,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // 128-row half this warp drains
     float alpha = 1.0f;
     {
       double den = 1.0;
@@ -238,12 +249,13 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       const int mt = w / g.n_tiles;
       if (!warp_wait(&acc_full[acc], acc_phase, abort_flag)) { if (lane == 0) fail(); break; }
       tc_fence_after();
-      const int64_t row = static_cast<int64_t>(mt) * kBM + q * 32 + lane;
+      const int64_t row = static_cast<int64_t>(mt) * C::TileM + half * kBM + q * 32 + lane;
       const int64_t col_base = static_cast<int64_t>(nt) * C::BN;
 #pragma unroll 1
       for (int c = 0; c < C::BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * C::BN + c * 32, r);
+        tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * C::Halves + half) * C::BN +
+                           c * 32, r);
         tmem_ld_wait();
         if (row < g.M) {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
@@ -299,11 +311,12 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const Gemm
   return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, g);
 }
 
-// 128 x 256 tiles for both: narrower tiles fill the last wave better (a
-// 4096-square product makes 3.46 waves) but read more L2 bytes per flop, and
-// measured slower (128 x 192 and 128 x 128).
-using FwdCfg = Cfg<false, 256, 4, 2, 1>;
-using DxCfg = Cfg<true, 256, 4, 2, 1>;
+// 128 x 256 tiles, 4-stage ring, double-buffered accumulator, one CTA per SM.
+// Measured slower on the 4096-square product: 128 x 192 and 128 x 128 tiles
+// (more L2 bytes per flop), 256 x 256 tiles (two MMAs per K step sharing B;
+// 1.73 waves, no accumulator double buffer) and two CTAs per SM.
+using FwdCfg = Cfg<false, 256, 4, 2, 1, 1>;
+using DxCfg = Cfg<true, 256, 4, 2, 1, 1>;
 
 template <class C>
 cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
@@ -318,7 +331,7 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
                        : make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::BN, true);
   if (!okb) return cudaErrorInvalidValue;
   GemmArgs g{};
-  g.m_tiles = ceil_div(M, kBM);
+  g.m_tiles = ceil_div(M, C::TileM);
   g.n_tiles = ceil_div(Ncols, C::BN);
   g.kb_total = ceil_div(Kc, C::BK);
   g.M = M;
