@@ -511,14 +511,19 @@ def _oracle_sample_step(O, wl, layer, data, tokens, proxy_rows, step):
     return t1 - t0, t2 - t1
 
 
-def cpu_baseline(wl, layer, budget_s=20.0, steps=1):
+def cpu_baseline(wl, layer, budget_s=20.0):
     import oracle as O
 
     cores = os.cpu_count() or 1
     O.set_threads(cores)
-    tokens, prows = 64, 256
     data = _OracleData(O, wl, layer)
+    # a small probe sizes the sample to about budget_s seconds of CPU work
+    tokens, prows = 64, 256
     tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 0)
+    scale = max(1.0, budget_s / max(tg + tp, 1e-6))
+    tokens = int(min(wl.M, tokens * scale))
+    prows = int(min(layer.N, prows * scale))
+    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 1)
     # per-token and per-proxy-row costs, scaled to the full workload step
     full_s = tg * (wl.M / tokens) + tp * (layer.N / prows)
     return {"value": round(wl.M / full_s, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
