@@ -222,7 +222,17 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # workload; the command and the figures are in the named profile).  A figure
 # holds only for the kernel sources it was measured on: when a source's hash
 # differs, the roofline's traffic is null.
-TRAFFIC = {}
+TRAFFIC = {
+    "proxy": {
+        "bytes": 107227392,
+        "profile": "profiles/proxy_update_llama7b_attn_proj_4096_r64.md",
+        "sources": {
+            "fp8_quantized_lora_b200/csrc/proxy.cu": "ef21e5a05cbf0ef861d2413eaae2749d7f506305d21a5a73a4a92587a12b289b",
+            "fp8_quantized_lora_b200/csrc/ptx.cuh": "1ec40a2067b4ae4960ba3532651728a393a070d5a79f0c934e7e37f8439b9c2e",
+            "fp8_quantized_lora_b200/csrc/internal.h": "953e4f0eefaccb9f774eb403aff06f254e1e9b8a18c7a80e01518aca130f3403",
+        },
+    },
+}
 
 
 def _traffic(phase):
@@ -257,7 +267,7 @@ def _phase_work(st):
         # each code matrix is read by two products; A, B, dA, dB and the T / U hi-lo pairs
         "adapters": {"flops": 4.0 * M * r * (N + K),
                      "bytes": 2.0 * (M * K + M * N) + 4.0 * r * (N + K) + 16.0 * M * r,
-                     "bound": "hbm", "kernels": "skinny_kernel x2 (T with U, dB with dA^T)"},
+                     "bound": "hbm", "kernels": "skinny_kernel x2 (T^T with U^T, dB^T with dA)"},
         "dX": {"flops": 2.0 * M * N * K, "bytes": M * N + N * K + 2.0 * M * K, "bound": "tensor",
                "kernels": "tc_gemm_kernel (dX)"},
         "sgd": {"flops": 0.0, "bytes": 8.0 * N * r, "bound": None, "kernels": "torch (caller's SGD)"},
