@@ -82,15 +82,27 @@
 //       definition), P keeps the accumulated value.  The pages say nothing
 //       about the sign of zero; keeping equal-valued codes as they are makes
 //       the decoded backbone identical to a verbatim rewrite.
+//  C-13 Top-k row selection (the pages' own rule: OpenReview rebuttal,
+//       reviewer 2, W7 -- the update is merged into the weight "using top-k
+//       row selection"; reviewer 3, Q1 -- it reduces the update from r to k,
+//       about 0.5% of the step).  The pages give neither the score nor k.
+//       Reading: a row's score is the number of its codes whose value C-10's
+//       c' would change; the selected rows are the k rows of highest
+//       positive score, ties going to the lower row index; a row of score 0
+//       is never selected (selecting it would only clear its proxy).  The
+//       selected rows then follow C-11; every other row keeps Wq bit-identical
+//       and its accumulated proxy, whatever its score.  k is the caller's.
 //
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
 // the only fused multiply-adds are the explicit std::fmaf calls of C-9.
 
+#include <algorithm>
 #include <cfloat>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #ifdef _OPENMP
 #include <omp.h>
@@ -382,6 +394,45 @@ void fo_proxy_select(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, uin
     }
     if (mask) mask[n] = selected ? 1 : 0;
     count += selected ? 1 : 0;
+  }
+  if (n_selected) *n_selected = count;
+}
+
+// ---------------------------------------------------------------- C-13
+void fo_proxy_select_topk(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, int64_t k_rows,
+                          uint8_t* mask, int32_t* n_selected) {
+  // score of every row: how many of its codes C-10 would change in value
+  std::vector<int64_t> score(static_cast<size_t>(N), 0);
+  for (int64_t n = 0; n < N; ++n) {
+    for (int64_t k = 0; k < K; ++k) {
+      const float w = static_cast<float>(dec(wq[n * K + k]));
+      const float upd = s_w * P[n * K + k];
+      const float t = w + upd;
+      if (!(dec(enc(t)) == dec(wq[n * K + k]))) score[n] += 1;
+    }
+  }
+  // rows by decreasing score; a stable sort keeps equal scores in index order
+  std::vector<int64_t> order(static_cast<size_t>(N));
+  for (int64_t n = 0; n < N; ++n) order[n] = n;
+  std::stable_sort(order.begin(), order.end(), [&](int64_t a, int64_t b) { return score[a] > score[b]; });
+  std::vector<uint8_t> chosen(static_cast<size_t>(N), 0);
+  for (int64_t j = 0; j < N && j < k_rows; ++j)
+    if (score[order[j]] > 0) chosen[order[j]] = 1;
+  // C-11 on the chosen rows
+  int32_t count = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    if (chosen[n]) {
+      for (int64_t k = 0; k < K; ++k) {
+        const float w = static_cast<float>(dec(wq[n * K + k]));
+        const float upd = s_w * P[n * K + k];
+        const float t = w + upd;
+        const uint8_t c_new = enc(t);
+        if (!(dec(c_new) == dec(wq[n * K + k]))) wq[n * K + k] = c_new;
+        P[n * K + k] = 0.0f;
+      }
+      count += 1;
+    }
+    if (mask) mask[n] = chosen[n];
   }
   if (n_selected) *n_selected = count;
 }
