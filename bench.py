@@ -417,6 +417,7 @@ def run_gpu(args):
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     status = int(st.status.item())
     n_sel = int(st.n_sel.item())
+    topk = _time_topk(st, F, torch, stream, l2_flush, args, dev) if args.topk > 0 else None
 
     tokens_total = wl.M * args.steps * ws
     value = tokens_total / (total_ms / 1e3)
@@ -480,12 +481,46 @@ def run_gpu(args):
         "clocks": clock_info,
         "device_status": status,
         "rows_selected_last_step": n_sel,
+        "extra": {"proxy_topk": topk},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, layer, budget_s=args.cpu_budget)
     if ws > 1:
         dist.destroy_process_group()
     return out, rank
+
+
+def _time_topk(st, F, torch, stream, l2_flush, args, dev):
+    """The proxy update with top-k row selection (not part of the step): on
+    copies of the step's Wq and P with its last dB_inc, eager calls timed
+    with CUDA events on the launching stream, L2 flushed before each."""
+    N, K = st.P.shape
+    wq, P = st.wq.clone(), st.P.clone()
+    mask = torch.empty(N, dtype=torch.uint8, device=dev)
+    cnt = torch.zeros(1, dtype=torch.int32, device=dev)
+    wsz = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, N, K, st.r)
+    ws = torch.empty(max(wsz, 256), dtype=torch.uint8, device=dev)
+    reps = max(5, min(50, args.steps))
+    total = 0.0
+    with torch.cuda.stream(stream):
+        for i in range(3 + reps):
+            l2_flush(i)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            F.falqon_proxy_update_topk(wq, st.s_w, P, st.dB_inc, st.A, args.topk, row_mask=mask,
+                                       n_selected=cnt, dev_status=st.status, workspace=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                total += e0.elapsed_time(e1)
+    ms = total / reps
+    flops = 2.0 * N * K * st.r
+    return {"k": args.topk, "ms": round(ms, 5), "rows_selected": int(cnt.item()),
+            "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
+            "kernels": "proxy_pipe_kernel (count) + proxy_topk_select_kernel + proxy_topk_apply_kernel",
+            "device_status": int(st.status.item())}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -596,6 +631,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--topk", type=int, default=256,
+                    help="also time the proxy update with top-k row selection at this k (0: skip)")
     ap.add_argument("--only", default=None, choices=list(Step.PHASES),
                     help="run one phase alone (warm-up + steps calls) and print no bench line; "
                          "for profiler captures")

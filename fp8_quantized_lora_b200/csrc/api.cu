@@ -104,6 +104,9 @@ size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int6
     case FALQON_OP_PROXY_UPDATE:
       if (N <= 0 || K <= 0) return 0;
       return proxy_workspace_bytes(N, K);
+    case FALQON_OP_PROXY_UPDATE_TOPK:
+      if (N <= 0 || K <= 0) return 0;
+      return proxy_topk_workspace_bytes(N, K);
   }
   return 0;
 }
@@ -205,6 +208,23 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
   return from_cuda(launch_proxy_update(wq, s_w, proxy, dB_inc, A, N, K, r, flags, row_mask,
                                        n_selected, dev_status, workspace,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
+                                       const void* dB_inc, const void* A, int64_t N, int64_t K,
+                                       int64_t r, int64_t k, uint8_t* row_mask,
+                                       int32_t* n_selected, int32_t* dev_status, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!wq || !s_w || !proxy || !dB_inc || !A) return FALQON_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || r <= 0 || k < 0) return FALQON_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N > INT32_MAX) return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(proxy) || !aligned16(wq)) return FALQON_ERR_UNSUPPORTED;
+  falqon_status s = check_ws(proxy_topk_workspace_bytes(N, K), workspace, workspace_bytes);
+  if (s != FALQON_OK) return s;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_proxy_update_topk(wq, s_w, proxy, dB_inc, A, N, K, r, k, row_mask,
+                                            n_selected, dev_status, workspace,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -30,6 +30,21 @@
 //     selects the row -- and the row's flag is set.
 //   proxy_clear_kernel  (one warp per row)
 //     Selected rows get P = +0; writes the row mask and the selected count.
+//
+// Top-k row selection (the rebuttal's rule, OpenReview reviewer 2 W7 and
+// reviewer 3 Q1; score and k are not given there): a row's score is the
+// number of its codes whose value the requantization would change; the k rows
+// of highest positive score are selected, ties to the lower row index, and
+// get the selected-row treatment above; every other row keeps its codes and
+// its accumulated proxy.  Three launches:
+//   proxy_pipe_kernel / proxy_stream_kernel in count mode: P' written, and
+//     per (row, 256-column block) the number of changing codes; no code is
+//     written (a row with changes may not be among the k).
+//   proxy_topk_select_kernel (one CTA): row scores, the k-th score by
+//     bisection on the integer scores, ties taken in index order by a
+//     block-wide scan; row mask, count and the list of selected rows.
+//   proxy_topk_apply_kernel: requantizes the selected rows from P' (the same
+//     arithmetic as above) and clears their proxy.
 // Every step is reproduced bit-for-bit by the float32 arithmetic.
 #include <cuda_fp16.h>
 
@@ -38,6 +53,11 @@
 
 namespace falqon {
 namespace {
+
+// Selection mode of the accumulation kernels.
+constexpr int kModeNone = 0;    // accumulate only
+constexpr int kModeSelect = 1;  // threshold rule: changed codes written at once, per-block row flags
+constexpr int kModeCount = 2;   // top-k: per-(row, 256-column block) counts of changing codes, no code write
 
 constexpr int kThreads = 256;
 constexpr int kTileRows = 32;   // 4 row groups of kRT rows
@@ -129,7 +149,7 @@ __device__ __forceinline__ uint32_t changed_bytes(uint32_t a, uint32_t b) {
   return (changed >> 7) * 0xFFu;
 }
 
-template <bool kAcc, bool kSel>
+template <bool kAcc, int kSel>
 __global__ void __launch_bounds__(kThreads, 2)
     proxy_stream_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                         float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
@@ -139,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ int tile_flag[kTileRows];  // a code of the row changed in this tile
+  __shared__ int tile_flag[kTileRows];  // select: a code of the row changed; count: how many
   uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kIChunk][256]
   float2* Bs = reinterpret_cast<float2*>(sm + kAsBytes);                       // [kIChunk][32]
   float4* pbuf = reinterpret_cast<float4*>(sm + kAsBytes + kBsBytes);          // [kRT][256]
@@ -160,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool ok = col_ok && n < N;
     cp_async16(pbuf + j * kThreads + tid, ok ? static_cast<const void*>(proxy + n * K + col) : proxy,
                ok ? 16u : 0u);
-    if (kSel)
+    if (kSel != kModeNone)
       cp_async4(wbuf + j * kThreads + tid, ok ? static_cast<const void*>(wq + n * K + col) : wq,
                 ok ? 4u : 0u);
   }
@@ -222,11 +242,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   cp_async_wait_all();
 
-  const float s_w = kSel ? *s_w_ptr : 1.0f;
+  const float s_w = kSel != kModeNone ? *s_w_ptr : 1.0f;
   bool nonfinite = false;
-  if (kSel) {
+  if (kSel != kModeNone) {
     if (tid < kTileRows) tile_flag[tid] = 0;
-    if (n_selected && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *n_selected = 0;  // the clear pass counts
+    if (kSel == kModeSelect && n_selected && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0)
+      *n_selected = 0;  // the clear pass counts
     __syncthreads();
   }
 #pragma unroll
@@ -242,21 +263,30 @@ __global__ void __launch_bounds__(kThreads, 2)
       *reinterpret_cast<float4*>(proxy + n * K + col) = p;
     }
     nonfinite |= !(isfinite(p.x) && isfinite(p.y) && isfinite(p.z) && isfinite(p.w));
-    if constexpr (kSel) {
+    if constexpr (kSel != kModeNone) {
       const uint32_t w = wbuf[j * kThreads + tid];
       const uint32_t cn = requantized4(w, s_w, p);
       const uint32_t m = changed_bytes(w, cn);
       if (m) {
-        *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
-        tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
+        if constexpr (kSel == kModeSelect) {
+          *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
+          tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
+        } else {
+          atomicAdd(&tile_flag[tr * kRT + j], __popc(m) >> 3);
+        }
       }
     }
   }
-  if (kSel) {
-    // this tile's verdict for each of its rows, written whether or not a code changed
+  if (kSel != kModeNone) {
+    // this tile's verdict (or count) for each of its rows, written in every case
     __syncthreads();
     const int64_t ncb = gridDim.x;
-    if (tid < kTileRows && r0 + tid < N) rowflag[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint8_t>(tile_flag[tid]);
+    if (tid < kTileRows && r0 + tid < N) {
+      if (kSel == kModeSelect)
+        rowflag[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint8_t>(tile_flag[tid]);
+      else
+        reinterpret_cast<uint16_t*>(rowflag)[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint16_t>(tile_flag[tid]);
+    }
   }
   if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
     atomicOr(dev_status, kDevNonfinite);
@@ -282,7 +312,7 @@ constexpr int kPipeBsBytes = kPipeRMax * kPipeRows * 8;           // (b, b) pair
 constexpr int kPipeSmemBytes =
     kPipePBytes + kPipeWBytes + 2 * kPipeDbBytes + kPipeAsBytes + kPipeBsBytes;  // 97 KB
 
-template <bool kSel>
+template <int kSel>
 __global__ void __launch_bounds__(kPipeThreads, 2)
     proxy_pipe_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                       float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
@@ -322,7 +352,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       const float* src = ok ? proxy + n * K + col : proxy;
       cp_async16(pst + (2 * j) * kPipeThreads + tid, src, ok ? 16u : 0u);
       cp_async16(pst + (2 * j + 1) * kPipeThreads + tid, ok ? src + 4 : proxy, ok ? 16u : 0u);
-      if (kSel) {
+      if (kSel != kModeNone) {
         const uint8_t* wsrc = ok ? wq + n * K + col : wq;
         asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(wst + j * kPipeThreads + tid)),
                      "l"(wsrc), "r"(ok ? 8u : 0u)
@@ -357,8 +387,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   issue_db(u_begin, 0);
   cp_async_commit();
 
-  const float s_w = kSel ? *s_w_ptr : 1.0f;
-  if (kSel && n_selected && blockIdx.x == 0 && threadIdx.x == 0) *n_selected = 0;  // the clear pass counts
+  const float s_w = kSel != kModeNone ? *s_w_ptr : 1.0f;
+  if (kSel == kModeSelect && n_selected && blockIdx.x == 0 && threadIdx.x == 0)
+    *n_selected = 0;  // the clear pass counts
   uint32_t maxmag = 0;  // largest |P'| bit pattern: >= 0x7F800000 means inf or NaN
   int cur_cb = -1, dbuf = 0;
   for (int v = u_begin; v < u_end; ++v) {
@@ -429,6 +460,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     for (int j = 0; j < kPipeRT; ++j) {
       const int64_t n = r0 + tr * kPipeRT + j;  // the warp's row: uniform across the warp
       bool changed = false;
+      int nchanged = 0;
       if (col_ok && n < N) {
         float4 p0 = pst[(2 * j) * kPipeThreads + tid];
         float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
@@ -448,24 +480,32 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
                                      max(__float_as_uint(p0.z) & mg, __float_as_uint(p0.w) & mg)),
                                  max(max(__float_as_uint(p1.x) & mg, __float_as_uint(p1.y) & mg),
                                      max(__float_as_uint(p1.z) & mg, __float_as_uint(p1.w) & mg))));
-        if constexpr (kSel) {
+        if constexpr (kSel != kModeNone) {
           const uint2 w = wst[j * kPipeThreads + tid];
           const uint32_t c0 = requantized4(w.x, s_w, p0);
           const uint32_t c1 = requantized4(w.y, s_w, p1);
           // identical words change only where they hold NaN codes (the common case)
           const uint32_t m0 = c0 == w.x ? nan_bytes(w.x) : changed_bytes(w.x, c0);
           const uint32_t m1 = c1 == w.y ? nan_bytes(w.y) : changed_bytes(w.y, c1);
-          if (m0 | m1) {
-            *reinterpret_cast<uint2*>(wq + n * K + col) =
-                make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
-            changed = true;
+          if constexpr (kSel == kModeSelect) {
+            if (m0 | m1) {
+              *reinterpret_cast<uint2*>(wq + n * K + col) =
+                  make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
+              changed = true;
+            }
+          } else {
+            nchanged = (__popc(m0) + __popc(m1)) >> 3;
           }
         }
       }
-      if constexpr (kSel) {
+      if constexpr (kSel == kModeSelect) {
         // the tile's verdict for row n, written whether or not a code changed
         const bool any = __any_sync(0xFFFFFFFFu, changed);
         if (lane == 0 && n < N) rowflag[n * ncb + v / row_groups] = any ? 1 : 0;
+      } else if constexpr (kSel == kModeCount) {
+        // the number of the row's codes in this tile whose value would change
+        const int cnt = __reduce_add_sync(0xFFFFFFFFu, nchanged);
+        if (lane == 0 && n < N) reinterpret_cast<uint16_t*>(rowflag)[n * ncb + v / row_groups] = static_cast<uint16_t>(cnt);
       }
     }
     dbuf ^= 1;
@@ -513,7 +553,7 @@ __global__ void __launch_bounds__(kClearThreads)
   }
 }
 
-template <bool kAcc, bool kSel>
+template <bool kAcc, int kSel>
 cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                           const void* A, int64_t N, int64_t K, int r, uint8_t* rowflag,
                           int32_t* n_selected, int32_t* dev_status, cudaStream_t stream) {
@@ -532,7 +572,7 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
                     rowflag, n_selected, dev_status);
 }
 
-template <bool kSel>
+template <int kSel>
 cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                         const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
                         int ncb, uint8_t* rowflag, int32_t* n_selected, int32_t* dev_status,
@@ -550,6 +590,161 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   return launch_pdl(proxy_pipe_kernel<kSel>, dim3(grid), dim3(kPipeThreads), kPipeSmemBytes, stream, 1u, wq,
                     s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
                     row_groups, units, ncb, rowflag, n_selected, dev_status);
+}
+
+constexpr int kTopkThreads = 512;
+
+// Block-wide helpers for the one-CTA selection (all threads call them).
+__device__ __forceinline__ int topk_block_sum(int v, int* red) {
+  v = __reduce_add_sync(0xFFFFFFFFu, v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();  // red is free again
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = 0;
+  for (int w = 0; w < kTopkThreads / 32; ++w) t += red[w];
+  return t;
+}
+
+__device__ __forceinline__ int topk_block_max(int v, int* red) {
+  v = __reduce_max_sync(0xFFFFFFFFu, v);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = 0;
+  for (int w = 0; w < kTopkThreads / 32; ++w) t = max(t, red[w]);
+  return t;
+}
+
+// Exclusive prefix sum of `v` over the CTA in thread order; *total = the sum.
+__device__ __forceinline__ int topk_block_scan(int v, int* red, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, d);
+    if (lane >= d) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  int before = 0, all = 0;
+  for (int w = 0; w < kTopkThreads / 32; ++w) {
+    if (w < warp) before += red[w];
+    all += red[w];
+  }
+  *total = all;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 1)
+    proxy_topk_select_kernel(const uint16_t* __restrict__ rowcount, int64_t N, int ncb, int64_t k,
+                             int32_t* __restrict__ score, int32_t* __restrict__ sel_rows,
+                             int32_t* __restrict__ n_sel, uint8_t* __restrict__ row_mask,
+                             int32_t* __restrict__ n_selected) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
+  __shared__ int red[kTopkThreads / 32];
+  const int tid = threadIdx.x;
+  // scores, the largest score and the number of candidates (score > 0)
+  int local_max = 0, local_cand = 0;
+  for (int64_t n = tid; n < N; n += kTopkThreads) {
+    int sc = 0;
+    for (int c = 0; c < ncb; ++c) sc += rowcount[n * ncb + c];
+    score[n] = sc;
+    local_max = max(local_max, sc);
+    local_cand += sc > 0 ? 1 : 0;
+  }
+  __syncthreads();  // the scores are visible to the whole CTA
+  const int max_score = topk_block_max(local_max, red);
+  const int64_t cand = topk_block_sum(local_cand, red);
+  const int64_t kk = k < cand ? k : cand;  // rows that will be selected
+  // tau: the largest score with at least kk rows scoring tau or more
+  auto count_at_least = [&](int t) {
+    int c = 0;
+    for (int64_t n = tid; n < N; n += kTopkThreads) c += score[n] >= t ? 1 : 0;
+    return topk_block_sum(c, red);
+  };
+  int tau = max_score + 1;  // kk == 0: nothing reaches it
+  if (kk > 0) {
+    int lo = 1, hi = max_score;
+    while (lo < hi) {  // every thread takes the same branches
+      const int mid = lo + (hi - lo + 1) / 2;
+      if (count_at_least(mid) >= kk) lo = mid;
+      else hi = mid - 1;
+    }
+    tau = lo;
+  }
+  const int64_t need = kk > 0 ? kk - count_at_least(tau + 1) : 0;  // ties at tau to take, in index order
+  // walk the rows in index order
+  int64_t ties_before = 0, out = 0;
+  for (int64_t base = 0; base < N; base += kTopkThreads) {
+    const int64_t n = base + tid;
+    const int sc = n < N ? score[n] : -1;
+    const int tie = (kk > 0 && sc == tau) ? 1 : 0;
+    int tie_total = 0;
+    const int64_t tie_rank = ties_before + topk_block_scan(tie, red, &tie_total);
+    const int chosen = (kk > 0 && sc > tau) || (tie && tie_rank < need) ? 1 : 0;
+    int chosen_total = 0;
+    const int64_t pos = out + topk_block_scan(chosen, red, &chosen_total);
+    if (n < N) {
+      if (row_mask) row_mask[n] = static_cast<uint8_t>(chosen);
+      if (chosen) sel_rows[pos] = static_cast<int32_t>(n);
+    }
+    ties_before += tie_total;
+    out += chosen_total;
+  }
+  if (tid == 0) {
+    *n_sel = static_cast<int32_t>(out);
+    if (n_selected) *n_selected = static_cast<int32_t>(out);
+  }
+}
+
+// Selected rows: every code whose value changes takes E4M3(dec(c) + s_w * P'),
+// and P' = +0.  Grid-stride over the list the selection kernel wrote.
+__global__ void __launch_bounds__(kClearThreads)
+    proxy_topk_apply_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
+                            float* __restrict__ proxy, int64_t K, const int32_t* __restrict__ sel_rows,
+                            const int32_t* __restrict__ n_sel) {
+  pdl_trigger();  // the next kernel may start launching; it waits for this one
+  pdl_wait();     // the previous kernel's results are complete and visible
+  const int64_t ns = *n_sel;
+  const float s_w = *s_w_ptr;
+  for (int64_t j = blockIdx.x; j < ns; j += gridDim.x) {
+    const int64_t n = sel_rows[j];
+    for (int64_t c = 4 * static_cast<int64_t>(threadIdx.x); c < K; c += 4 * kClearThreads) {
+      uint32_t* wp = reinterpret_cast<uint32_t*>(wq + n * K + c);
+      float4* pp = reinterpret_cast<float4*>(proxy + n * K + c);
+      const uint32_t w = *wp;
+      const uint32_t cn = requantized4(w, s_w, *pp);
+      const uint32_t m = cn == w ? nan_bytes(w) : changed_bytes(w, cn);
+      if (m) *wp = (cn & m) | (w & ~m);
+      *pp = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+  }
+}
+
+struct TopkWorkspace {
+  uint16_t* rowcount;  // [N][ncb]
+  int32_t* score;      // [N]
+  int32_t* sel_rows;   // [N]
+  int32_t* n_sel;      // [1]
+};
+
+TopkWorkspace topk_layout(void* ws, int64_t N, int64_t ncb, size_t* bytes) {
+  const size_t a = align_up(static_cast<size_t>(N) * static_cast<size_t>(ncb) * 2, 256);
+  const size_t b = align_up(static_cast<size_t>(N) * 4, 256);
+  TopkWorkspace t{};
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  if (p) {
+    t.rowcount = reinterpret_cast<uint16_t*>(p);
+    t.score = reinterpret_cast<int32_t*>(p + a);
+    t.sel_rows = reinterpret_cast<int32_t*>(p + a + b);
+    t.n_sel = reinterpret_cast<int32_t*>(p + a + 2 * b);
+  }
+  if (bytes) *bytes = a + 2 * b + 256;
+  return t;
 }
 
 }  // namespace
@@ -587,26 +782,75 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
     const int g = static_cast<int>(units < resident ? units : resident);
     const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
     if (sel)
-      e = launch_pipe<true>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                            dev_status, stream);
+      e = launch_pipe<kModeSelect>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
+                                   dev_status, stream);
     else
-      e = launch_pipe<false>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                             dev_status, stream);
+      e = launch_pipe<kModeNone>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
+                                 dev_status, stream);
   } else if (acc && sel)
-    e = launch_stream<true, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                  dev_status, stream);
+    e = launch_stream<true, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                         dev_status, stream);
   else if (acc)
-    e = launch_stream<true, false>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                   dev_status, stream);
+    e = launch_stream<true, kModeNone>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                       dev_status, stream);
   else
-    e = launch_stream<false, true>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                   dev_status, stream);
+    e = launch_stream<false, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
+                                          dev_status, stream);
   if (e != cudaSuccess || !sel) return e;
   const int64_t row_blocks = (N + kClearWarps - 1) / kClearWarps;
   const int64_t blocks = row_blocks < static_cast<int64_t>(di->sm_count) * 8 ? row_blocks
                                                                               : static_cast<int64_t>(di->sm_count) * 8;
   return launch_pdl(proxy_clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
                     proxy, N, K, ncb, rowflag, row_mask, n_selected);
+}
+
+size_t proxy_topk_workspace_bytes(int64_t N, int64_t K) {
+  size_t bytes = 0;
+  topk_layout(nullptr, N, (K + kTileCols - 1) / kTileCols, &bytes);
+  return bytes;
+}
+
+cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
+                                     const void* A, int64_t N, int64_t K, int64_t r, int64_t k,
+                                     uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
+                                     void* workspace, cudaStream_t stream) {
+  const DeviceInfo* di = current_device_info();
+  if (!di) return cudaErrorInvalidDevice;
+  if (r < 1 || r > (int64_t(1) << 30) || N > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
+                  static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
+  const int rr = static_cast<int>(r);
+  const int ncb = static_cast<int>(grid.x);
+  const TopkWorkspace t = topk_layout(workspace, N, ncb, nullptr);
+  uint8_t* counts = reinterpret_cast<uint8_t*>(t.rowcount);
+  const int64_t row_groups = (N + kPipeRows - 1) / kPipeRows;
+  const int64_t units = row_groups * grid.x;
+  const bool pipe = rr <= kPipeRMax && rr % 8 == 0 && units <= (int64_t(1) << 30) &&
+                    di->max_smem_optin >= kPipeSmemBytes;
+  if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
+  cudaError_t e;
+  // 1. P' and the per-(row, column block) counts of changing codes
+  if (pipe) {
+    const int64_t resident = 2 * static_cast<int64_t>(di->sm_count);
+    const int g = static_cast<int>(units < resident ? units : resident);
+    e = launch_pipe<kModeCount>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, static_cast<int>(row_groups),
+                                static_cast<int>(units), ncb, counts, nullptr, dev_status, stream);
+  } else {
+    e = launch_stream<true, kModeCount>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, counts, nullptr,
+                                        dev_status, stream);
+  }
+  if (e != cudaSuccess) return e;
+  // 2. the k rows
+  e = launch_pdl(proxy_topk_select_kernel, dim3(1), dim3(kTopkThreads), 0, stream, 1u,
+                 static_cast<const uint16_t*>(t.rowcount), N, ncb, k, t.score, t.sel_rows, t.n_sel, row_mask,
+                 n_selected);
+  if (e != cudaSuccess) return e;
+  // 3. requantize and clear them
+  const int64_t cap = static_cast<int64_t>(di->sm_count) * 8;
+  const int64_t kmax = k < N ? k : N;
+  const int64_t blocks = kmax < 1 ? 1 : (kmax < cap ? kmax : cap);
+  return launch_pdl(proxy_topk_apply_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
+                    wq, s_w, proxy, K, static_cast<const int32_t*>(t.sel_rows), static_cast<const int32_t*>(t.n_sel));
 }
 
 }  // namespace falqon

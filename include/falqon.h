@@ -67,7 +67,8 @@ typedef enum falqon_op {
   FALQON_OP_QUANTIZE = 0,
   FALQON_OP_LINEAR_FWD = 1,
   FALQON_OP_LINEAR_BWD = 2,
-  FALQON_OP_PROXY_UPDATE = 3
+  FALQON_OP_PROXY_UPDATE = 3,
+  FALQON_OP_PROXY_UPDATE_TOPK = 4
 } falqon_op;
 
 /* Bits OR-ed into *dev_status by the kernels. */
@@ -176,6 +177,37 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
                                   int64_t r, uint32_t flags, uint8_t* row_mask,
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+/*
+ * falqon_proxy_update_topk - row-wise proxy update with top-k row selection.
+ *
+ * The rebuttal's own rule (OpenReview reviewer 2, W7: the update is merged
+ * into the weight "using top-k row selection"; reviewer 3, Q1: it costs about
+ * 0.5% of the step and reduces the update from r to k).  The pages give
+ * neither the score nor k; this library's reading:
+ *   ACCUMULATE as in falqon_proxy_update (the same float32 FMA chain).
+ *   score[n] = number of k with dec(c'[n,k]) != dec(Wq[n,k]), c' as in
+ *              falqon_proxy_update's SELECT.
+ *   The selected rows are the k rows of highest positive score; ties go to
+ *   the lower row index; a row of score 0 is never selected.  Selected rows
+ *   are requantized and cleared exactly as in falqon_proxy_update; every
+ *   other row keeps Wq bit-identical and its accumulated proxy (so with
+ *   k >= N the result equals falqon_proxy_update with both flags).
+ *
+ *  wq, s_w, proxy, dB_inc, A: as in falqon_proxy_update (r >= 1).
+ *  k >= 0: the largest number of rows to select (0: accumulate only).
+ *  row_mask [N] uint8 (0/1) and n_selected (1 int32): nullable.
+ *  workspace: falqon_workspace_size(FALQON_OP_PROXY_UPDATE_TOPK, 0, N, K, r)
+ *  bytes (per-(row, 256-column block) counts, row scores, the selected list).
+ *  Requirements: N >= 1 and below 2^31; K multiple of 16; r >= 1; k >= 0.
+ *  Three launches (accumulate and count, select, requantize), all on
+ *  `stream`; nothing is synchronised with the host.
+ */
+FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
+                                       const void* dB_inc, const void* A, int64_t N, int64_t K,
+                                       int64_t r, int64_t k, uint8_t* row_mask,
+                                       int32_t* n_selected, int32_t* dev_status, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * falqon_linear_bwd_noalloc - falqon_linear_bwd for callers that cannot
