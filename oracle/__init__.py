@@ -52,7 +52,8 @@ def lib():
         L.fo_adapter_da.argtypes = [p, p, p, C.c_float, i64, i64, i64, p]
         L.fo_proxy_accumulate.argtypes = [p, p, p, i64, i64, i64]
         L.fo_proxy_select.argtypes = [p, C.c_float, p, i64, i64, p, p]
-        L.fo_proxy_select_topk.argtypes = [p, C.c_float, p, i64, i64, i64, p, p]
+        L.fo_proxy_select_topk.argtypes = [p, C.c_float, p, i64, i64, i64, C.c_int, p, p]
+        L.fo_proxy_select_residual.argtypes = [p, C.c_float, p, i64, i64, p, p]
         L.fo_set_threads.argtypes = [C.c_int]
         L.fo_get_threads.restype = C.c_int
         _lib = L
@@ -245,29 +246,44 @@ def proxy_select(wq: np.ndarray, s_w, P: np.ndarray):
     return wq, P, mask, int(cnt[0])
 
 
-def proxy_select_topk(wq: np.ndarray, s_w, P: np.ndarray, k: int):
-    """C-13: returns (new wq, new P, mask, n_selected) with at most k rows
-    selected (highest number of changing codes, ties to the lower index)."""
+def proxy_select_residual(wq: np.ndarray, s_w, P: np.ndarray):
+    """C-10 with C-14 (residual-keeping clear): returns (new wq, new P, mask,
+    n_selected); the inputs are not modified."""
     wq = np.array(wq, dtype=np.uint8, copy=True, order="C")
     P = np.array(P, dtype=np.float32, copy=True, order="C")
     N, K = wq.shape
     mask = np.zeros(N, dtype=np.uint8)
     cnt = np.zeros(1, dtype=np.int32)
-    lib().fo_proxy_select_topk(_ptr(wq), C.c_float(float(s_w)), _ptr(P), N, K, int(k), _ptr(mask), _ptr(cnt))
+    lib().fo_proxy_select_residual(_ptr(wq), C.c_float(float(s_w)), _ptr(P), N, K, _ptr(mask), _ptr(cnt))
     return wq, P, mask, int(cnt[0])
 
 
-def proxy_update_topk(wq, s_w, P, dB_inc, A, k):
+def proxy_select_topk(wq: np.ndarray, s_w, P: np.ndarray, k: int, keep_residual: bool = False):
+    """C-13: returns (new wq, new P, mask, n_selected) with at most k rows
+    selected (highest number of changing codes, ties to the lower index);
+    keep_residual applies C-14 instead of C-11 to them."""
+    wq = np.array(wq, dtype=np.uint8, copy=True, order="C")
+    P = np.array(P, dtype=np.float32, copy=True, order="C")
+    N, K = wq.shape
+    mask = np.zeros(N, dtype=np.uint8)
+    cnt = np.zeros(1, dtype=np.int32)
+    lib().fo_proxy_select_topk(_ptr(wq), C.c_float(float(s_w)), _ptr(P), N, K, int(k), int(bool(keep_residual)),
+                               _ptr(mask), _ptr(cnt))
+    return wq, P, mask, int(cnt[0])
+
+
+def proxy_update_topk(wq, s_w, P, dB_inc, A, k, keep_residual=False):
     """One proxy update with top-k row selection: accumulate (C-9), then C-13."""
-    return proxy_select_topk(wq, s_w, proxy_accumulate(P, dB_inc, A), k)
+    return proxy_select_topk(wq, s_w, proxy_accumulate(P, dB_inc, A), k, keep_residual)
 
 
-def proxy_update(wq, s_w, P, dB_inc, A, accumulate=True, select=True):
-    """One row-wise proxy update: accumulate, then select/requantize/clear."""
+def proxy_update(wq, s_w, P, dB_inc, A, accumulate=True, select=True, keep_residual=False):
+    """One row-wise proxy update: accumulate, then select/requantize/clear
+    (C-11) or keep the residual (C-14)."""
     Pn = proxy_accumulate(P, dB_inc, A) if accumulate else np.array(P, dtype=np.float32, copy=True)
     if not select:
         return np.array(wq, dtype=np.uint8, copy=True), Pn, None, 0
-    return proxy_select(wq, s_w, Pn)
+    return proxy_select_residual(wq, s_w, Pn) if keep_residual else proxy_select(wq, s_w, Pn)
 
 
 from .tolerance import within_tolerance, tolerance_report  # noqa: E402,F401

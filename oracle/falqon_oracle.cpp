@@ -92,6 +92,15 @@
 //       is never selected (selecting it would only clear its proxy).  The
 //       selected rows then follow C-11; every other row keeps Wq bit-identical
 //       and its accumulated proxy, whatever its score.  k is the caller's.
+//  C-14 Residual-keeping clear (error feedback; the variant of C-11 the
+//       pages leave open: C-11 drops the sub-step residual
+//       dec(old)/s_W + P - dec(c')/s_W).  In a selected row, a code whose
+//       value changes takes c' and keeps the part of its proxy the new code
+//       did not apply: P = fl32( P - fl32( fl32(dec(c') - dec(old)) / s_W ) )
+//       (the difference of two E4M3 values is exact in float32; one IEEE
+//       division, one subtraction); a code whose value does not change keeps
+//       its bits and its proxy.  Under the threshold rule every row then
+//       follows the same formula (an unselected row has no changing code).
 //
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
@@ -398,9 +407,47 @@ void fo_proxy_select(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, uin
   if (n_selected) *n_selected = count;
 }
 
+// C-11 / C-14 on one selected row: codes whose value changes take c'; the
+// proxy is cleared (keep_residual = 0) or keeps what the new codes did not
+// apply (keep_residual = 1).
+static void requantize_row(uint8_t* wq, float s_w, float* P, int64_t K, int keep_residual) {
+  for (int64_t k = 0; k < K; ++k) {
+    const double old_v = dec(wq[k]);
+    const float w = static_cast<float>(old_v);
+    const float upd = s_w * P[k];
+    const float t = w + upd;
+    const uint8_t c_new = enc(t);
+    const bool changes = !(dec(c_new) == old_v);
+    if (changes) wq[k] = c_new;
+    if (!keep_residual) {
+      P[k] = 0.0f;
+    } else if (changes) {
+      const float d = static_cast<float>(dec(c_new)) - static_cast<float>(old_v);  // exact
+      P[k] = P[k] - d / s_w;
+    }
+  }
+}
+
+void fo_proxy_select_residual(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, uint8_t* mask,
+                              int32_t* n_selected) {
+  // threshold rule (C-10) with C-14 in place of C-11
+  int32_t count = 0;
+  for (int64_t n = 0; n < N; ++n) {
+    bool selected = false;
+    for (int64_t k = 0; k < K; ++k) {
+      const float t = static_cast<float>(dec(wq[n * K + k])) + s_w * P[n * K + k];
+      if (!(dec(enc(t)) == dec(wq[n * K + k]))) selected = true;
+    }
+    if (selected) requantize_row(wq + n * K, s_w, P + n * K, K, 1);
+    if (mask) mask[n] = selected ? 1 : 0;
+    count += selected ? 1 : 0;
+  }
+  if (n_selected) *n_selected = count;
+}
+
 // ---------------------------------------------------------------- C-13
 void fo_proxy_select_topk(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, int64_t k_rows,
-                          uint8_t* mask, int32_t* n_selected) {
+                          int keep_residual, uint8_t* mask, int32_t* n_selected) {
   // score of every row: how many of its codes C-10 would change in value
   std::vector<int64_t> score(static_cast<size_t>(N), 0);
   for (int64_t n = 0; n < N; ++n) {
@@ -418,18 +465,11 @@ void fo_proxy_select_topk(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K
   std::vector<uint8_t> chosen(static_cast<size_t>(N), 0);
   for (int64_t j = 0; j < N && j < k_rows; ++j)
     if (score[order[j]] > 0) chosen[order[j]] = 1;
-  // C-11 on the chosen rows
+  // C-11 (or C-14) on the chosen rows
   int32_t count = 0;
   for (int64_t n = 0; n < N; ++n) {
     if (chosen[n]) {
-      for (int64_t k = 0; k < K; ++k) {
-        const float w = static_cast<float>(dec(wq[n * K + k]));
-        const float upd = s_w * P[n * K + k];
-        const float t = w + upd;
-        const uint8_t c_new = enc(t);
-        if (!(dec(c_new) == dec(wq[n * K + k]))) wq[n * K + k] = c_new;
-        P[n * K + k] = 0.0f;
-      }
+      requantize_row(wq + n * K, s_w, P + n * K, K, keep_residual);
       count += 1;
     }
     if (mask) mask[n] = chosen[n];
