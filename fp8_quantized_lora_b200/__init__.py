@@ -20,7 +20,7 @@ __all__ = [
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "OP_QUANTIZE", "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK",
-    "PROXY_ACCUMULATE", "PROXY_SELECT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
+    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfalqon.s
 
 OP_QUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_PROXY_UPDATE, OP_PROXY_UPDATE_TOPK = 0, 1, 2, 3, 4
 DTYPE_BF16, DTYPE_F32 = 0, 1
-PROXY_ACCUMULATE, PROXY_SELECT = 1, 2
+PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL = 1, 2, 4
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
 
@@ -64,7 +64,7 @@ def lib():
     L.falqon_linear_fwd.argtypes = [p, p, p, p, i64, i64, i64, p, p, p, sz, p]
     L.falqon_linear_bwd.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p, sz, p]
     L.falqon_proxy_update.argtypes = [p, p, p, p, p, i64, i64, i64, u32, p, p, p, p, sz, p]
-    L.falqon_proxy_update_topk.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, sz, p]
+    L.falqon_proxy_update_topk.argtypes = [p, p, p, p, p, i64, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_linear_bwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p]
     for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
               "falqon_linear_bwd_noalloc"):
@@ -203,8 +203,8 @@ def falqon_proxy_update(wq, s_w, proxy, dB_inc, A, flags=PROXY_ACCUMULATE | PROX
     return row_mask, n_selected
 
 
-def falqon_proxy_update_topk(wq, s_w, proxy, dB_inc, A, k, row_mask=None, n_selected=None,
-                             dev_status=None, workspace=None, stream=None):
+def falqon_proxy_update_topk(wq, s_w, proxy, dB_inc, A, k, keep_residual=False, row_mask=None,
+                             n_selected=None, dev_status=None, workspace=None, stream=None):
     """Proxy update with top-k row selection, in place on (wq, proxy);
     returns (row_mask, n_selected)."""
     N, K = proxy.shape
@@ -214,7 +214,8 @@ def falqon_proxy_update_topk(wq, s_w, proxy, dB_inc, A, k, row_mask=None, n_sele
     n_selected = torch.empty(1, dtype=torch.int32, device=dev) if n_selected is None else n_selected
     ws, wsb = _workspace(OP_PROXY_UPDATE_TOPK, 0, N, K, r, dev, workspace)
     st = lib().falqon_proxy_update_topk(_ptr(_u8(wq)), _ptr(s_w), _ptr(proxy), _ptr(dB_inc), _ptr(A), N, K, r,
-                                        int(k), _ptr(row_mask), _ptr(n_selected), _ptr(dev_status), _ptr(ws),
+                                        int(k), PROXY_KEEP_RESIDUAL if keep_residual else 0, _ptr(row_mask),
+                                        _ptr(n_selected), _ptr(dev_status), _ptr(ws),
                                         wsb, _stream(stream, dev))
     _check(st, "falqon_proxy_update_topk")
     return row_mask, n_selected

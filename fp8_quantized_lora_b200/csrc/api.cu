@@ -190,8 +190,9 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   int64_t r, uint32_t flags, uint8_t* row_mask,
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream) {
-  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT;
-  if (flags == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
+  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL;
+  if ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
+  if ((flags & FALQON_PROXY_KEEP_RESIDUAL) && !(flags & FALQON_PROXY_SELECT)) return FALQON_ERR_INVALID_ARG;
   if (!proxy || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
   if (K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
   if (!aligned16(proxy)) return FALQON_ERR_UNSUPPORTED;
@@ -212,17 +213,18 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
 
 falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
                                        const void* dB_inc, const void* A, int64_t N, int64_t K,
-                                       int64_t r, int64_t k, uint8_t* row_mask,
+                                       int64_t r, int64_t k, uint32_t flags, uint8_t* row_mask,
                                        int32_t* n_selected, int32_t* dev_status, void* workspace,
                                        size_t workspace_bytes, void* stream) {
   if (!wq || !s_w || !proxy || !dB_inc || !A) return FALQON_ERR_INVALID_ARG;
+  if (flags & ~FALQON_PROXY_KEEP_RESIDUAL) return FALQON_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || r <= 0 || k < 0) return FALQON_ERR_INVALID_ARG;
   if (K % 16 != 0 || N > INT32_MAX) return FALQON_ERR_UNSUPPORTED;
   if (!aligned16(proxy) || !aligned16(wq)) return FALQON_ERR_UNSUPPORTED;
   falqon_status s = check_ws(proxy_topk_workspace_bytes(N, K), workspace, workspace_bytes);
   if (s != FALQON_OK) return s;
   if (!current_device_info()) return FALQON_ERR_CUDA;
-  return from_cuda(launch_proxy_update_topk(wq, s_w, proxy, dB_inc, A, N, K, r, k, row_mask,
+  return from_cuda(launch_proxy_update_topk(wq, s_w, proxy, dB_inc, A, N, K, r, k, flags, row_mask,
                                             n_selected, dev_status, workspace,
                                             static_cast<cudaStream_t>(stream)));
 }

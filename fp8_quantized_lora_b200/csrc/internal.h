@@ -96,7 +96,7 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
 size_t proxy_topk_workspace_bytes(int64_t N, int64_t K);
 cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                                      const void* A, int64_t N, int64_t K, int64_t r, int64_t k,
-                                     uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
-                                     void* workspace, cudaStream_t stream);
+                                     uint32_t flags, uint8_t* row_mask, int32_t* n_selected,
+                                     int32_t* dev_status, void* workspace, cudaStream_t stream);
 
 }  // namespace falqon

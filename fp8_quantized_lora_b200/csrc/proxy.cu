@@ -149,13 +149,27 @@ __device__ __forceinline__ uint32_t changed_bytes(uint32_t a, uint32_t b) {
   return (changed >> 7) * 0xFFu;
 }
 
+// Residual-keeping clear: for the codes in byte mask m (their value changes
+// from w_old to w_new) the proxy keeps what the new code does not apply,
+// P - (dec(new) - dec(old)) / s_w (the difference of two E4M3 values is exact
+// in float32; one IEEE division, one subtraction); other lanes keep P.
+__device__ __forceinline__ float4 residual4(float4 p, uint32_t w_old, uint32_t w_new, uint32_t m, float s_w) {
+  const float2 o01 = e4m3x2_values(w_old), o23 = e4m3x2_values(w_old >> 16);
+  const float2 n01 = e4m3x2_values(w_new), n23 = e4m3x2_values(w_new >> 16);
+  if (m & 0x000000FFu) p.x = __fsub_rn(p.x, __fdiv_rn(__fsub_rn(n01.x, o01.x), s_w));
+  if (m & 0x0000FF00u) p.y = __fsub_rn(p.y, __fdiv_rn(__fsub_rn(n01.y, o01.y), s_w));
+  if (m & 0x00FF0000u) p.z = __fsub_rn(p.z, __fdiv_rn(__fsub_rn(n23.x, o23.x), s_w));
+  if (m & 0xFF000000u) p.w = __fsub_rn(p.w, __fdiv_rn(__fsub_rn(n23.y, o23.y), s_w));
+  return p;
+}
+
 template <bool kAcc, int kSel>
 __global__ void __launch_bounds__(kThreads, 2)
     proxy_stream_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                         float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                         const uint16_t* __restrict__ A, int64_t N, int64_t K, int r,
                         uint8_t* __restrict__ rowflag, int32_t* __restrict__ n_selected,
-                        int32_t* __restrict__ dev_status) {
+                        int32_t* __restrict__ dev_status, int keep_residual) {
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   extern __shared__ __align__(16) uint8_t sm[];
@@ -271,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if constexpr (kSel == kModeSelect) {
           *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
           tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
+          if (keep_residual) *reinterpret_cast<float4*>(proxy + n * K + col) = residual4(p, w, cn, m, s_w);
         } else {
           atomicAdd(&tile_flag[tr * kRT + j], __popc(m) >> 3);
         }
@@ -318,7 +333,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
                       float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                       const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
                       int units, int ncb, uint8_t* __restrict__ rowflag,
-                      int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status) {
+                      int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status,
+                      int keep_residual) {
   // No early trigger: the clear kernel that follows needs no shared memory, so
   // its CTAs would sit beside this kernel's on the SMs while they wait.
   pdl_wait();  // the previous kernel's results are complete and visible
@@ -492,6 +508,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
               *reinterpret_cast<uint2*>(wq + n * K + col) =
                   make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
               changed = true;
+              if (keep_residual) {
+                dst[0] = residual4(p0, w.x, c0, m0, s_w);
+                dst[1] = residual4(p1, w.y, c1, m1, s_w);
+              }
             }
           } else {
             nchanged = (__popc(m0) + __popc(m1)) >> 3;
@@ -524,7 +544,7 @@ constexpr int kClearWarps = kClearThreads / 32;
 __global__ void __launch_bounds__(kClearThreads)
     proxy_clear_kernel(float* __restrict__ proxy, int64_t N, int64_t K, int ncb,
                        const uint8_t* __restrict__ rowflag, uint8_t* __restrict__ row_mask,
-                       int32_t* __restrict__ n_selected) {
+                       int32_t* __restrict__ n_selected, int clear) {
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   __shared__ int warp_count[kClearWarps];
@@ -540,7 +560,7 @@ __global__ void __launch_bounds__(kClearThreads)
       if (row_mask) row_mask[n] = sel ? 1 : 0;
       count += sel ? 1 : 0;
     }
-    if (!sel) continue;
+    if (!sel || !clear) continue;
     float4* row = reinterpret_cast<float4*>(proxy + n * K);
     for (int64_t c = lane; c < K / 4; c += 32) row[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
@@ -556,7 +576,7 @@ __global__ void __launch_bounds__(kClearThreads)
 template <bool kAcc, int kSel>
 cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                           const void* A, int64_t N, int64_t K, int r, uint8_t* rowflag,
-                          int32_t* n_selected, int32_t* dev_status, cudaStream_t stream) {
+                          int32_t* n_selected, int32_t* dev_status, int keep_residual, cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -569,14 +589,14 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
   }
   return launch_pdl(proxy_stream_kernel<kAcc, kSel>, grid, dim3(kThreads), kSmemBytes, stream, 1u, wq, s_w,
                     proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
-                    rowflag, n_selected, dev_status);
+                    rowflag, n_selected, dev_status, keep_residual);
 }
 
 template <int kSel>
 cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                         const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
                         int ncb, uint8_t* rowflag, int32_t* n_selected, int32_t* dev_status,
-                        cudaStream_t stream) {
+                        int keep_residual, cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -589,7 +609,7 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   }
   return launch_pdl(proxy_pipe_kernel<kSel>, dim3(grid), dim3(kPipeThreads), kPipeSmemBytes, stream, 1u, wq,
                     s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
-                    row_groups, units, ncb, rowflag, n_selected, dev_status);
+                    row_groups, units, ncb, rowflag, n_selected, dev_status, keep_residual);
 }
 
 constexpr int kTopkThreads = 512;
@@ -706,7 +726,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
 __global__ void __launch_bounds__(kClearThreads)
     proxy_topk_apply_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
                             float* __restrict__ proxy, int64_t K, const int32_t* __restrict__ sel_rows,
-                            const int32_t* __restrict__ n_sel) {
+                            const int32_t* __restrict__ n_sel, int keep_residual) {
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   const int64_t ns = *n_sel;
@@ -717,10 +737,11 @@ __global__ void __launch_bounds__(kClearThreads)
       uint32_t* wp = reinterpret_cast<uint32_t*>(wq + n * K + c);
       float4* pp = reinterpret_cast<float4*>(proxy + n * K + c);
       const uint32_t w = *wp;
-      const uint32_t cn = requantized4(w, s_w, *pp);
+      const float4 p = *pp;
+      const uint32_t cn = requantized4(w, s_w, p);
       const uint32_t m = cn == w ? nan_bytes(w) : changed_bytes(w, cn);
       if (m) *wp = (cn & m) | (w & ~m);
-      *pp = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      *pp = keep_residual ? residual4(p, w, cn, m, s_w) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
   }
 }
@@ -761,6 +782,7 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   const bool acc = flags & 1u, sel = flags & 2u;
+  const int keep_res = (flags & 4u) ? 1 : 0;  // residual-keeping clear instead of P = +0
   if (r > (int64_t(1) << 30)) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
                   static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
@@ -783,25 +805,25 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
     const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
     if (sel)
       e = launch_pipe<kModeSelect>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                                   dev_status, stream);
+                                   dev_status, keep_res, stream);
     else
       e = launch_pipe<kModeNone>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                                 dev_status, stream);
+                                 dev_status, keep_res, stream);
   } else if (acc && sel)
     e = launch_stream<true, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                         dev_status, stream);
+                                         dev_status, keep_res, stream);
   else if (acc)
     e = launch_stream<true, kModeNone>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                       dev_status, stream);
+                                       dev_status, keep_res, stream);
   else
     e = launch_stream<false, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                          dev_status, stream);
+                                          dev_status, keep_res, stream);
   if (e != cudaSuccess || !sel) return e;
   const int64_t row_blocks = (N + kClearWarps - 1) / kClearWarps;
   const int64_t blocks = row_blocks < static_cast<int64_t>(di->sm_count) * 8 ? row_blocks
                                                                               : static_cast<int64_t>(di->sm_count) * 8;
   return launch_pdl(proxy_clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
-                    proxy, N, K, ncb, rowflag, row_mask, n_selected);
+                    proxy, N, K, ncb, rowflag, row_mask, n_selected, keep_res ? 0 : 1);
 }
 
 size_t proxy_topk_workspace_bytes(int64_t N, int64_t K) {
@@ -812,8 +834,9 @@ size_t proxy_topk_workspace_bytes(int64_t N, int64_t K) {
 
 cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                                      const void* A, int64_t N, int64_t K, int64_t r, int64_t k,
-                                     uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
-                                     void* workspace, cudaStream_t stream) {
+                                     uint32_t flags, uint8_t* row_mask, int32_t* n_selected,
+                                     int32_t* dev_status, void* workspace, cudaStream_t stream) {
+  const int keep_res = (flags & 4u) ? 1 : 0;  // residual-keeping clear instead of P = +0
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   if (r < 1 || r > (int64_t(1) << 30) || N > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
@@ -834,10 +857,10 @@ cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy
     const int64_t resident = 2 * static_cast<int64_t>(di->sm_count);
     const int g = static_cast<int>(units < resident ? units : resident);
     e = launch_pipe<kModeCount>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, static_cast<int>(row_groups),
-                                static_cast<int>(units), ncb, counts, nullptr, dev_status, stream);
+                                static_cast<int>(units), ncb, counts, nullptr, dev_status, 0, stream);
   } else {
     e = launch_stream<true, kModeCount>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, counts, nullptr,
-                                        dev_status, stream);
+                                        dev_status, 0, stream);
   }
   if (e != cudaSuccess) return e;
   // 2. the k rows
@@ -850,7 +873,8 @@ cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy
   const int64_t kmax = k < N ? k : N;
   const int64_t blocks = kmax < 1 ? 1 : (kmax < cap ? kmax : cap);
   return launch_pdl(proxy_topk_apply_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
-                    wq, s_w, proxy, K, static_cast<const int32_t*>(t.sel_rows), static_cast<const int32_t*>(t.n_sel));
+                    wq, s_w, proxy, K, static_cast<const int32_t*>(t.sel_rows), static_cast<const int32_t*>(t.n_sel),
+                    keep_res);
 }
 
 }  // namespace falqon

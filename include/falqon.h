@@ -79,6 +79,7 @@ typedef enum falqon_op {
 /* Flags of falqon_proxy_update. */
 #define FALQON_PROXY_ACCUMULATE 1u /* P += dB_inc . A */
 #define FALQON_PROXY_SELECT 2u     /* select rows, requantize them, clear their proxy */
+#define FALQON_PROXY_KEEP_RESIDUAL 4u /* with SELECT (or top-k): keep the unapplied residual, no clear */
 
 /*
  * falqon_quantize - per-tensor E4M3 quantization.
@@ -162,6 +163,11 @@ FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy
  *               bits (so a zero keeps its sign), and P[n,:] = +0.  Other
  *               rows: Wq bit-identical, P kept.  The decoded backbone is the
  *               same as with a verbatim rewrite of the row.
+ *   KEEP_RESIDUAL (with SELECT): the error-feedback variant of the clear
+ *               (the pages drop nothing explicitly; clearing drops the
+ *               sub-step residual): a code whose value changes keeps
+ *               P = fl32(P - fl32(fl32(dec(c') - dec(old)) / s_W)); every
+ *               other code keeps its proxy.  Row mask and count as SELECT.
  * The float32 chain is reproduced bit-for-bit (no tensor cores).
  *
  *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);
@@ -170,7 +176,8 @@ FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy
  *  row_mask [N] uint8 (0/1) and n_selected (1 int32): written when SELECT is
  *  set; nullable.
  *  Requirements: N >= 1; K multiple of 16; r >= 1 (r unused without
- *  ACCUMULATE); flags a nonzero subset of ACCUMULATE|SELECT.
+ *  ACCUMULATE); flags: ACCUMULATE and/or SELECT, plus KEEP_RESIDUAL only
+ *  with SELECT.
  */
 FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   const void* dB_inc, const void* A, int64_t N, int64_t K,
@@ -196,6 +203,8 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
  *
  *  wq, s_w, proxy, dB_inc, A: as in falqon_proxy_update (r >= 1).
  *  k >= 0: the largest number of rows to select (0: accumulate only).
+ *  flags: 0, or FALQON_PROXY_KEEP_RESIDUAL (selected rows keep the residual
+ *  instead of a cleared proxy; see falqon_proxy_update).
  *  row_mask [N] uint8 (0/1) and n_selected (1 int32): nullable.
  *  workspace: falqon_workspace_size(FALQON_OP_PROXY_UPDATE_TOPK, 0, N, K, r)
  *  bytes (per-(row, 256-column block) counts, row scores, the selected list).
@@ -205,7 +214,7 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
  */
 FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
                                        const void* dB_inc, const void* A, int64_t N, int64_t K,
-                                       int64_t r, int64_t k, uint8_t* row_mask,
+                                       int64_t r, int64_t k, uint32_t flags, uint8_t* row_mask,
                                        int32_t* n_selected, int32_t* dev_status, void* workspace,
                                        size_t workspace_bytes, void* stream);
 

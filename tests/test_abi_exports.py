@@ -94,6 +94,9 @@ def test_proxy_argument_errors():
     assert L.falqon_proxy_update(P, P, P, None, P, 4, 16, 2, 1, None, None, None, P, 1 << 20, None) == 1
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 20, 2, 3, None, None, None, P, 1 << 20, None) == 2
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3, None, None, None, None, 0, None) == 3
+    # KEEP_RESIDUAL only together with SELECT
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 5, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 4, None, None, None, P, 1 << 20, None) == 1
 
 
 def test_proxy_topk_argument_errors():
@@ -101,14 +104,15 @@ def test_proxy_topk_argument_errors():
     ws = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, 4, 16, 2)
     assert ws >= 256 and ws % 256 == 0
     f = L.falqon_proxy_update_topk
-    assert f(None, P, P, P, P, 4, 16, 2, 1, None, None, None, P, ws, None) == 1   # no codes
-    assert f(P, P, P, None, P, 4, 16, 2, 1, None, None, None, P, ws, None) == 1   # no increment
-    assert f(P, P, P, P, P, 4, 16, 0, 1, None, None, None, P, ws, None) == 1      # r = 0
-    assert f(P, P, P, P, P, 4, 16, 2, -1, None, None, None, P, ws, None) == 1     # k < 0
-    assert f(P, P, P, P, P, 0, 16, 2, 1, None, None, None, P, ws, None) == 1      # N = 0
-    assert f(P, P, P, P, P, 4, 20, 2, 1, None, None, None, P, ws, None) == 2      # K % 16
-    assert f(P, P, P8, P, P, 4, 16, 2, 1, None, None, None, P, ws, None) == 2     # unaligned proxy
-    assert f(P, P, P, P, P, 4, 16, 2, 1, None, None, None, P, ws - 256, None) == 3  # workspace
+    assert f(None, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 1   # no codes
+    assert f(P, P, P, None, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 1   # no increment
+    assert f(P, P, P, P, P, 4, 16, 0, 1, 0, None, None, None, P, ws, None) == 1      # r = 0
+    assert f(P, P, P, P, P, 4, 16, 2, -1, 0, None, None, None, P, ws, None) == 1     # k < 0
+    assert f(P, P, P, P, P, 4, 16, 2, 1, 1, None, None, None, P, ws, None) == 1      # unknown flag
+    assert f(P, P, P, P, P, 0, 16, 2, 1, 0, None, None, None, P, ws, None) == 1      # N = 0
+    assert f(P, P, P, P, P, 4, 20, 2, 1, 4, None, None, None, P, ws, None) == 2      # K % 16
+    assert f(P, P, P8, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 2     # unaligned proxy
+    assert f(P, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws - 256, None) == 3  # workspace
 
 
 @pytest.mark.parametrize("name", ["falqon_quantize", "falqon_linear_fwd"])

@@ -125,3 +125,37 @@ def test_twenty_step_trajectory_matches(cuda_device):
         np.testing.assert_array_equal(host(p).view(np.uint32), P.view(np.uint32))
         np.testing.assert_array_equal(host(mask), rmask)
         assert int(host(cnt)[0]) == rcnt
+
+
+@pytest.mark.parametrize("N,K,r", [
+    (256, 256, 16),     # persistent kernel
+    (37, 48, 5),        # grid kernel, ragged
+    (70, 2048, 64),
+    (96, 1024, 100),
+])
+def test_keep_residual_matches_oracle(cuda_device, N, K, r):
+    """Error-feedback clear (C-14): codes as the clearing rule, the proxy keeps
+    what the new codes did not apply."""
+    O.set_threads(os.cpu_count() or 8)
+    case = _state(N + K + r + 7, N, K, r, p_std=1e-6, inc_std=1e-4)
+    ref = O.proxy_update(*case, keep_residual=True)
+    assert 0 < ref[3] <= N
+    flags = F.PROXY_ACCUMULATE | F.PROXY_SELECT | F.PROXY_KEEP_RESIDUAL
+    _compare(_gpu(*case, flags=flags), ref)
+
+
+def test_keep_residual_trajectory_matches(cuda_device):
+    N, K, r = 128, 512, 16
+    wq, s_w, P, _, A = _state(17, N, K, r, p_std=0)
+    w, p = dev_u8(wq), dev_f32(P)
+    s_dev, A_dev = dev_f32([s_w]), dev_bf16(A)
+    flags = F.PROXY_ACCUMULATE | F.PROXY_SELECT | F.PROXY_KEEP_RESIDUAL
+    for step in range(10):
+        dB = gen.normal_bf16_bits(3000 + step, (N, r), 3e-4)
+        mask, cnt = F.falqon_proxy_update(w, s_dev, p, dev_bf16(dB), A_dev, flags=flags)
+        wq, P, rmask, rcnt = O.proxy_update(wq, s_w, P, dB, A, keep_residual=True)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(w), wq)
+        np.testing.assert_array_equal(host(p).view(np.uint32), P.view(np.uint32))
+        np.testing.assert_array_equal(host(mask), rmask)
+        assert int(host(cnt)[0]) == rcnt

@@ -104,3 +104,21 @@ def test_topk_trajectory_matches(cuda_device):
         assert int(host(cnt)[0]) == rcnt
         np.testing.assert_array_equal(host(w), wq)
         np.testing.assert_array_equal(host(p).view(np.uint32), P.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,K,r,k", [
+    (256, 256, 16, 32),
+    (37, 48, 5, 4),
+    (70, 2048, 64, 17),
+])
+def test_topk_keep_residual_matches_oracle(cuda_device, N, K, r, k):
+    O.set_threads(os.cpu_count() or 8)
+    case = _state(N + K + r + k + 3, N, K, r)
+    ref = O.proxy_update_topk(*case, k, keep_residual=True)
+    w = dev_u8(case[0])
+    p = dev_f32(case[2])
+    st = status_word()
+    mask, cnt = F.falqon_proxy_update_topk(w, dev_f32([case[1]]), p, dev_bf16(case[3]), dev_bf16(case[4]), k,
+                                           keep_residual=True, dev_status=st)
+    torch.cuda.synchronize()
+    _compare((host(w), host(p), host(mask), int(host(cnt)[0]), int(host(st)[0])), ref)
