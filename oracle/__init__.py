@@ -41,14 +41,17 @@ def lib():
         L.fo_amax.restype = C.c_uint32
         L.fo_amax.argtypes = [p, C.c_int, i64, p]
         L.fo_scale.restype = C.c_uint32
-        L.fo_scale.argtypes = [C.c_float, p]
-        L.fo_quantize.argtypes = [p, C.c_int, i64, C.c_float, p]
+        L.fo_scale.argtypes = [C.c_float, C.c_int, p]
+        L.fo_quantize.argtypes = [p, C.c_int, i64, C.c_float, C.c_int, p]
+        L.fo_e5m2_decode.restype = C.c_double
+        L.fo_e5m2_decode.argtypes = [C.c_uint8]
+        L.fo_e5m2_encode_array.argtypes = [p, i64, p]
         L.fo_residual.argtypes = [p, C.c_int, p, i64, C.c_float, p, p]
         L.fo_linear_fwd.argtypes = [p, C.c_float, p, C.c_float, i64, i64, i64, i64, i64, p]
-        L.fo_linear_dx.argtypes = [p, C.c_float, p, C.c_float, i64, i64, i64, i64, i64, p]
+        L.fo_linear_dx.argtypes = [p, C.c_float, C.c_int, p, C.c_float, i64, i64, i64, i64, i64, p]
         L.fo_adapter_t.argtypes = [p, C.c_float, p, i64, i64, i64, p, p]
-        L.fo_adapter_u.argtypes = [p, C.c_float, p, i64, i64, i64, p, p]
-        L.fo_adapter_db.argtypes = [p, C.c_float, p, p, i64, i64, i64, p]
+        L.fo_adapter_u.argtypes = [p, C.c_float, C.c_int, p, i64, i64, i64, p, p]
+        L.fo_adapter_db.argtypes = [p, C.c_float, C.c_int, p, p, i64, i64, i64, p]
         L.fo_adapter_da.argtypes = [p, p, p, C.c_float, i64, i64, i64, p]
         L.fo_proxy_accumulate.argtypes = [p, p, p, i64, i64, i64]
         L.fo_proxy_select.argtypes = [p, C.c_float, p, i64, i64, p, p]
@@ -93,6 +96,22 @@ def e4m3_encode(v) -> np.ndarray:
     return out.reshape(shape)
 
 
+FORMATS = {"e4m3": 0, "e5m2": 1}
+
+
+def e5m2_decode(c: int) -> float:
+    return float(lib().fo_e5m2_decode(int(c)))
+
+
+def e5m2_encode(v) -> np.ndarray:
+    v = np.asarray(v, dtype=np.float32)
+    shape = v.shape
+    flat = np.ascontiguousarray(v.reshape(-1))
+    out = np.empty(flat.shape, dtype=np.uint8)
+    lib().fo_e5m2_encode_array(_ptr(flat), flat.size, _ptr(out))
+    return out.reshape(shape)
+
+
 def bf16_round(v) -> np.ndarray:
     """float64 -> bfloat16 bits, one rounding (nearest, ties to even)."""
     v = np.asarray(v, dtype=np.float64)
@@ -124,19 +143,20 @@ def amax(x: np.ndarray):
     return np.float32(out[0]), int(st)
 
 
-def scale(amax_value) -> tuple:
+def scale(amax_value, fmt: str = "e4m3") -> tuple:
     out = np.zeros(1, dtype=np.float32)
-    st = lib().fo_scale(C.c_float(float(amax_value)), _ptr(out))
+    st = lib().fo_scale(C.c_float(float(amax_value)), FORMATS[fmt], _ptr(out))
     return np.float32(out[0]), int(st)
 
 
-def quantize(x: np.ndarray):
-    """Per-tensor E4M3 quantization: returns (codes, scale, amax, status)."""
+def quantize(x: np.ndarray, fmt: str = "e4m3"):
+    """Per-tensor FP8 quantization (E4M3, or E5M2 per C-15): returns (codes,
+    scale, amax, status)."""
     x, is_bf16 = _xin(x)
     a, st1 = amax(x)
-    s, st2 = scale(a)
+    s, st2 = scale(a, fmt)
     codes = np.empty(x.shape, dtype=np.uint8)
-    lib().fo_quantize(_ptr(x), is_bf16, x.size, C.c_float(float(s)), _ptr(codes))
+    lib().fo_quantize(_ptr(x), is_bf16, x.size, C.c_float(float(s)), FORMATS[fmt], _ptr(codes))
     return codes, np.float32(s), np.float32(a), st1 | st2
 
 
@@ -164,14 +184,14 @@ def linear_fwd(xq, s_x, wq, s_w, rows=None) -> np.ndarray:
     return y
 
 
-def linear_dx(dyq, s_dy, wq, s_w, rows=None) -> np.ndarray:
+def linear_dx(dyq, s_dy, wq, s_w, rows=None, dy_fmt: str = "e4m3") -> np.ndarray:
     dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
     wq = np.ascontiguousarray(wq, dtype=np.uint8)
     M, N = dyq.shape
     K = wq.shape[1]
     m0, m1 = (0, M) if rows is None else rows
     dx = np.empty((m1 - m0, K), dtype=np.float64)
-    lib().fo_linear_dx(_ptr(dyq), C.c_float(float(s_dy)), _ptr(wq), C.c_float(float(s_w)),
+    lib().fo_linear_dx(_ptr(dyq), C.c_float(float(s_dy)), FORMATS[dy_fmt], _ptr(wq), C.c_float(float(s_w)),
                        M, N, K, m0, m1, _ptr(dx))
     return dx
 
@@ -188,18 +208,19 @@ def adapter_t(xq, s_x, A):
     return t64, t16
 
 
-def adapter_u(dyq, s_dy, B):
+def adapter_u(dyq, s_dy, B, dy_fmt: str = "e4m3"):
     dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
     B = np.ascontiguousarray(B, dtype=np.uint16)
     M, N = dyq.shape
     r = B.shape[1]
     u64 = np.empty((M, r), dtype=np.float64)
     u16 = np.empty((M, r), dtype=np.uint16)
-    lib().fo_adapter_u(_ptr(dyq), C.c_float(float(s_dy)), _ptr(B), M, N, r, _ptr(u64), _ptr(u16))
+    lib().fo_adapter_u(_ptr(dyq), C.c_float(float(s_dy)), FORMATS[dy_fmt], _ptr(B), M, N, r, _ptr(u64),
+                       _ptr(u16))
     return u64, u16
 
 
-def adapter_db(dyq, s_dy, t16=None, t64=None):
+def adapter_db(dyq, s_dy, t16=None, t64=None, dy_fmt: str = "e4m3"):
     dyq = np.ascontiguousarray(dyq, dtype=np.uint8)
     M, N = dyq.shape
     t = t16 if t16 is not None else t64
@@ -207,7 +228,8 @@ def adapter_db(dyq, s_dy, t16=None, t64=None):
     t16c = None if t16 is None else np.ascontiguousarray(t16, dtype=np.uint16)
     t64c = None if t64 is None or t16 is not None else np.ascontiguousarray(t64, dtype=np.float64)
     db = np.empty((N, r), dtype=np.float64)
-    lib().fo_adapter_db(_ptr(dyq), C.c_float(float(s_dy)), _ptr(t16c), _ptr(t64c), M, N, r, _ptr(db))
+    lib().fo_adapter_db(_ptr(dyq), C.c_float(float(s_dy)), FORMATS[dy_fmt], _ptr(t16c), _ptr(t64c), M, N, r,
+                        _ptr(db))
     return db
 
 

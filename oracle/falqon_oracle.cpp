@@ -101,6 +101,17 @@
 //       division, one subtraction); a code whose value does not change keeps
 //       its bits and its proxy.  Under the threshold rule every row then
 //       follows the same formula (an unselected row has no changing code).
+//  C-15 E5M2 gradients.  The rebuttal (reviewer 2, W2) names E5M2 beside
+//       E4M3 as an FP8 format under the same per-tensor scaling; the step
+//       can carry dY in it.  Format (OCP 8-bit FP): sign, 5 exponent bits
+//       (bias 15), 2 mantissa bits; exponent 31 holds infinity (mantissa 0)
+//       and NaN; subnormals are multiples of 2^-16; the largest finite value
+//       is 57344.  Encoding: nearest, ties to even, saturating (every
+//       magnitude above 57344, infinity included, encodes as +-57344), NaN
+//       as 0x7F, a value that rounds to zero keeps its sign.  Scale:
+//       s = 57344 / amax (C-2 with the format's largest value); codes as C-3.
+//       dX (C-6), U and dB (C-7, C-8) read dYq through this decoding; every
+//       other step is unchanged.
 //
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
@@ -151,6 +162,39 @@ uint8_t enc(float v) {  // C-1 encoding
   return sign | static_cast<uint8_t>(((E + 7) << 3) | (static_cast<int>(q) - 8));
 }
 
+double dec5(uint8_t c) {  // C-15 decoding, from the field definition
+  const int sign = c >> 7;
+  const int e = (c >> 2) & 0x1F;
+  const int m = c & 0x3;
+  double mag;
+  if (e == 31) {
+    if (m != 0) return std::nan("");
+    mag = INFINITY;
+  } else {
+    mag = (e == 0) ? std::ldexp(static_cast<double>(m), -16)
+                   : std::ldexp(4.0 + m, e - 17);  // 2^(e-15) * (1 + m/4)
+  }
+  return sign ? -mag : mag;
+}
+
+uint8_t enc5(float v) {  // C-15 encoding
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));
+  if (a > 57344.0) return sign | 0x7B;  // satfinite
+  if (a < std::ldexp(1.0, -14)) {
+    // subnormal range: multiples of 2^-16; 4 * 2^-16 is the smallest normal, code 0x04
+    const double q = std::nearbyint(std::ldexp(a, 16));
+    return sign | static_cast<uint8_t>(q);
+  }
+  int e2 = 0;
+  std::frexp(a, &e2);
+  int E = e2 - 1;                                   // a in [2^E, 2^(E+1))
+  double q = std::nearbyint(std::ldexp(a, 2 - E));  // significand * 4, in [4, 8]
+  if (q == 8.0) { q = 4.0; E += 1; }
+  return sign | static_cast<uint8_t>(((E + 15) << 2) | (static_cast<int>(q) - 4));
+}
+
 float bf16_to_f32(uint16_t b) {
   const uint32_t u = static_cast<uint32_t>(b) << 16;
   float f;
@@ -183,16 +227,19 @@ uint16_t bf16_round(double v) {
 
 int g_threads = 1;
 
-// dec() of all 256 codes, tabulated once; the GEMM loops read this table.
+// dec() / dec5() of all 256 codes, tabulated once; the GEMM loops read them.
 struct DecodeTable {
   double v[256];
-  DecodeTable() {
-    for (int c = 0; c < 256; ++c) v[c] = dec(static_cast<uint8_t>(c));
+  explicit DecodeTable(double (*f)(uint8_t)) {
+    for (int c = 0; c < 256; ++c) v[c] = f(static_cast<uint8_t>(c));
   }
 };
-const DecodeTable kDec;
+const DecodeTable kDec(dec);
+const DecodeTable kDec5(dec5);
 
 inline double dv(uint8_t c) { return kDec.v[c]; }
+// decoding table of a code matrix: fmt 0 = E4M3, 1 = E5M2
+inline const double* table(int fmt) { return fmt ? kDec5.v : kDec.v; }
 
 }  // namespace
 
@@ -205,6 +252,10 @@ int fo_get_threads(void) { return g_threads; }
 // ---------------------------------------------------------------- C-1
 double fo_e4m3_decode(uint8_t c) { return dec(c); }
 uint8_t fo_e4m3_encode(float v) { return enc(v); }
+double fo_e5m2_decode(uint8_t c) { return dec5(c); }
+void fo_e5m2_encode_array(const float* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = enc5(v[i]);
+}
 void fo_e4m3_encode_array(const float* v, int64_t n, uint8_t* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = enc(v[i]);
 }
@@ -232,22 +283,22 @@ uint32_t fo_amax(const void* x, int is_bf16, int64_t n, float* amax) {
   return nonfinite ? kNonfinite : 0u;
 }
 
-uint32_t fo_scale(float amax, float* s) {
+uint32_t fo_scale(float amax, int fmt, float* s) {
   if (!std::isfinite(amax)) { *s = 1.0f; return kNonfinite; }
   if (amax == 0.0f) { *s = 1.0f; return 0u; }
-  const float q = 448.0f / amax;  // IEEE float32 division
+  const float q = (fmt ? 57344.0f : 448.0f) / amax;  // IEEE float32 division
   if (std::isinf(q)) { *s = FLT_MAX; return kScaleOverflow; }
   *s = q;
   return 0u;
 }
 
 // ---------------------------------------------------------------- C-3
-void fo_quantize(const void* x, int is_bf16, int64_t n, float s, uint8_t* codes) {
+void fo_quantize(const void* x, int is_bf16, int64_t n, float s, int fmt, uint8_t* codes) {
   for (int64_t i = 0; i < n; ++i) {
     const float v = is_bf16 ? bf16_to_f32(static_cast<const uint16_t*>(x)[i])
                             : static_cast<const float*>(x)[i];
     const float p = v * s;  // one float32 multiply, round to nearest even
-    codes[i] = enc(p);
+    codes[i] = fmt ? enc5(p) : enc(p);
   }
 }
 
@@ -282,15 +333,16 @@ void fo_linear_fwd(const uint8_t* xq, float s_x, const uint8_t* wq, float s_w,
 
 // ---------------------------------------------------------------- C-6
 // Rows [m0, m1) of dX = dYq Wq / (s_dY s_W); dx holds (m1-m0) x K values.
-void fo_linear_dx(const uint8_t* dyq, float s_dy, const uint8_t* wq, float s_w,
+void fo_linear_dx(const uint8_t* dyq, float s_dy, int dy_fmt, const uint8_t* wq, float s_w,
                   int64_t M, int64_t N, int64_t K, int64_t m0, int64_t m1, double* dx) {
   (void)M;
   const double denom = static_cast<double>(s_dy) * static_cast<double>(s_w);
+  const double* dyv = table(dy_fmt);
 #pragma omp parallel for num_threads(g_threads) schedule(static)
   for (int64_t m = m0; m < m1; ++m) {
     for (int64_t k = 0; k < K; ++k) {
       double acc = 0.0;
-      for (int64_t n = 0; n < N; ++n) acc += dv(dyq[m * N + n]) * dv(wq[n * K + k]);
+      for (int64_t n = 0; n < N; ++n) acc += dyv[dyq[m * N + n]] * dv(wq[n * K + k]);
       dx[(m - m0) * K + k] = acc / denom;
     }
   }
@@ -301,7 +353,7 @@ void fo_linear_dx(const uint8_t* dyq, float s_dy, const uint8_t* wq, float s_w,
 //   out[m,i] = sum_j dec(q[m,j]) * bf16(w[i,j] or w[j,i]) / s
 // w_rows_are_i = 1: w is [r, J] (A for T);  0: w is [J, r] (B for U).
 // Writes float64 values and their bfloat16 rounding.
-static void skinny_rows(const uint8_t* q, float s, const uint16_t* w, int w_rows_are_i,
+static void skinny_rows(const uint8_t* q, const double* qv, float s, const uint16_t* w, int w_rows_are_i,
                         int64_t M, int64_t J, int64_t r, double* out64, uint16_t* out16) {
 #pragma omp parallel for num_threads(g_threads) schedule(static)
   for (int64_t m = 0; m < M; ++m) {
@@ -309,7 +361,7 @@ static void skinny_rows(const uint8_t* q, float s, const uint16_t* w, int w_rows
       double acc = 0.0;
       for (int64_t j = 0; j < J; ++j) {
         const double wv = bf16_to_f32(w_rows_are_i ? w[i * J + j] : w[j * r + i]);
-        acc += dv(q[m * J + j]) * wv;
+        acc += qv[q[m * J + j]] * wv;
       }
       const double v = acc / static_cast<double>(s);
       if (out64) out64[m * r + i] = v;
@@ -321,26 +373,27 @@ static void skinny_rows(const uint8_t* q, float s, const uint16_t* w, int w_rows
 // T = bf16(Xq A^T / s_X), A is [r, K].
 void fo_adapter_t(const uint8_t* xq, float s_x, const uint16_t* A, int64_t M, int64_t K,
                   int64_t r, double* t64, uint16_t* t16) {
-  skinny_rows(xq, s_x, A, 1, M, K, r, t64, t16);
+  skinny_rows(xq, kDec.v, s_x, A, 1, M, K, r, t64, t16);
 }
 
 // U = bf16(dYq B / s_dY), B is [N, r].
-void fo_adapter_u(const uint8_t* dyq, float s_dy, const uint16_t* B, int64_t M, int64_t N,
+void fo_adapter_u(const uint8_t* dyq, float s_dy, int dy_fmt, const uint16_t* B, int64_t M, int64_t N,
                   int64_t r, double* u64, uint16_t* u16) {
-  skinny_rows(dyq, s_dy, B, 0, M, N, r, u64, u16);
+  skinny_rows(dyq, table(dy_fmt), s_dy, B, 0, M, N, r, u64, u16);
 }
 
 // dB = dYq^T T / s_dY, [N, r].  t is either bfloat16 bits (t16) or float64 (t64);
 // the float64 form exists for the autograd pin that checks the formula itself.
-void fo_adapter_db(const uint8_t* dyq, float s_dy, const uint16_t* t16, const double* t64,
+void fo_adapter_db(const uint8_t* dyq, float s_dy, int dy_fmt, const uint16_t* t16, const double* t64,
                    int64_t M, int64_t N, int64_t r, double* db) {
+  const double* dyv = table(dy_fmt);
 #pragma omp parallel for num_threads(g_threads) schedule(static)
   for (int64_t n = 0; n < N; ++n) {
     for (int64_t i = 0; i < r; ++i) {
       double acc = 0.0;
       for (int64_t m = 0; m < M; ++m) {
         const double tv = t16 ? static_cast<double>(bf16_to_f32(t16[m * r + i])) : t64[m * r + i];
-        acc += dv(dyq[m * N + n]) * tv;
+        acc += dyv[dyq[m * N + n]] * tv;
       }
       db[n * r + i] = acc / static_cast<double>(s_dy);
     }
