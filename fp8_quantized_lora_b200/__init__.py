@@ -35,7 +35,8 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: 
 EXPORTED_SYMBOLS = (
     "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
-    "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk",
+    "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
+    "falqon_linear_bwd_e5m2",
 )
 
 
@@ -61,8 +62,10 @@ def lib():
     L = C.CDLL(LIB_PATH)
     p, i64, u32, sz = C.c_void_p, C.c_int64, C.c_uint32, C.c_size_t
     L.falqon_quantize.argtypes = [p, C.c_int, i64, i64, p, p, p, p, p, p, sz, p]
+    L.falqon_quantize_e5m2.argtypes = [p, C.c_int, i64, i64, p, p, p, p, p, sz, p]
     L.falqon_linear_fwd.argtypes = [p, p, p, p, i64, i64, i64, p, p, p, sz, p]
     L.falqon_linear_bwd.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p, sz, p]
+    L.falqon_linear_bwd_e5m2.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p, sz, p]
     L.falqon_proxy_update.argtypes = [p, p, p, p, p, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_proxy_update_topk.argtypes = [p, p, p, p, p, i64, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_linear_bwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p]
@@ -128,8 +131,9 @@ def _u8(t):
 
 # ------------------------------------------------------------------ entry points
 def falqon_quantize(x, codes=None, scale=None, amax=None, residual=None, dev_status=None,
-                    workspace=None, stream=None):
-    """Per-tensor E4M3 quantization of a 2-D bf16/fp32 tensor; returns (codes, scale, amax)."""
+                    workspace=None, stream=None, fmt="e4m3"):
+    """Per-tensor FP8 quantization of a 2-D bf16/fp32 tensor (E4M3, or E5M2
+    for gradients: fmt="e5m2", no residual); returns (codes, scale, amax)."""
     if x.dim() != 2:
         raise ValueError("x must be 2-D")
     rows, cols = x.shape
@@ -141,6 +145,15 @@ def falqon_quantize(x, codes=None, scale=None, amax=None, residual=None, dev_sta
     scale = torch.empty(1, dtype=torch.float32, device=dev) if scale is None else scale
     amax = torch.empty(1, dtype=torch.float32, device=dev) if amax is None else amax
     ws, wsb = _workspace(OP_QUANTIZE, rows, cols, 0, 0, dev, workspace)
+    if fmt == "e5m2":
+        if residual is not None:
+            raise ValueError("the residual is defined for E4M3 only")
+        st = lib().falqon_quantize_e5m2(_ptr(x), dt, rows, cols, _ptr(_u8(codes)), _ptr(scale), _ptr(amax),
+                                        _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+        _check(st, "falqon_quantize_e5m2")
+        return codes, scale, amax
+    if fmt != "e4m3":
+        raise ValueError("fmt must be 'e4m3' or 'e5m2'")
     st = lib().falqon_quantize(_ptr(x), dt, rows, cols, _ptr(_u8(codes)), _ptr(scale), _ptr(amax),
                                _ptr(residual), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
     _check(st, "falqon_quantize")
@@ -160,8 +173,9 @@ def falqon_linear_fwd(xq, s_x, wq, s_w, y=None, dev_status=None, stream=None):
 
 
 def falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=True,
-                      dev_status=None, workspace=None, stream=None):
-    """Backward of the melded layer; each output may be True (allocate), a tensor, or None."""
+                      dev_status=None, workspace=None, stream=None, dy_fmt="e4m3"):
+    """Backward of the melded layer; each output may be True (allocate), a tensor, or None.
+    dy_fmt="e5m2": dyq holds E5M2 codes (falqon_quantize(..., fmt="e5m2"))."""
     M, N = dyq.shape
     K = wq.shape[1] if wq is not None else xq.shape[1]
     r = A.shape[0] if A is not None else 0
@@ -176,11 +190,14 @@ def falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=Tr
     ws, wsb = (None, 0)
     if dA_t is not None or dB_t is not None:
         ws, wsb = _workspace(OP_LINEAR_BWD, M, N, K, r, dev, workspace)
-    st = lib().falqon_linear_bwd(_ptr(_u8(dyq)), _ptr(s_dy), _ptr(None if wq is None else _u8(wq)),
-                                 _ptr(s_w), _ptr(None if xq is None else _u8(xq)), _ptr(s_x),
-                                 _ptr(A), _ptr(B), M, N, K, r, _ptr(dx_t), _ptr(dA_t), _ptr(dB_t),
-                                 _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
-    _check(st, "falqon_linear_bwd")
+    if dy_fmt not in ("e4m3", "e5m2"):
+        raise ValueError("dy_fmt must be 'e4m3' or 'e5m2'")
+    fn = lib().falqon_linear_bwd_e5m2 if dy_fmt == "e5m2" else lib().falqon_linear_bwd
+    st = fn(_ptr(_u8(dyq)), _ptr(s_dy), _ptr(None if wq is None else _u8(wq)),
+            _ptr(s_w), _ptr(None if xq is None else _u8(xq)), _ptr(s_x),
+            _ptr(A), _ptr(B), M, N, K, r, _ptr(dx_t), _ptr(dA_t), _ptr(dB_t),
+            _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_linear_bwd_e5m2" if dy_fmt == "e5m2" else "falqon_linear_bwd")
     return dx_t, dA_t, dB_t
 
 

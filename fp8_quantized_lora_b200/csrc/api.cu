@@ -111,10 +111,13 @@ size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int6
   return 0;
 }
 
-falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
-                              uint8_t* codes, float* scale, float* amax, float* residual,
-                              int32_t* dev_status, void* workspace, size_t workspace_bytes,
-                              void* stream) {
+}  // extern "C"
+
+namespace {
+
+falqon_status quantize_call(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols, uint8_t* codes,
+                            float* scale, float* amax, float* residual, int32_t* dev_status, void* workspace,
+                            size_t workspace_bytes, void* stream, bool e5m2) {
   if (!x || !codes || !scale) return FALQON_ERR_INVALID_ARG;
   if (rows <= 0 || cols <= 0) return FALQON_ERR_INVALID_ARG;
   if (dtype != FALQON_DTYPE_BF16 && dtype != FALQON_DTYPE_F32) return FALQON_ERR_INVALID_ARG;
@@ -126,7 +129,26 @@ falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int64_t rows, i
   if (s != FALQON_OK) return s;
   if (!current_device_info()) return FALQON_ERR_CUDA;
   return from_cuda(launch_quantize(x, dtype == FALQON_DTYPE_BF16, n, codes, scale, amax, residual,
-                                   dev_status, workspace, static_cast<cudaStream_t>(stream)));
+                                   dev_status, workspace, static_cast<cudaStream_t>(stream), e5m2));
+}
+
+}  // namespace
+
+extern "C" {
+
+falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
+                              uint8_t* codes, float* scale, float* amax, float* residual,
+                              int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  return quantize_call(x, dtype, rows, cols, codes, scale, amax, residual, dev_status, workspace,
+                       workspace_bytes, stream, false);
+}
+
+falqon_status falqon_quantize_e5m2(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
+                                   uint8_t* codes, float* scale, float* amax, int32_t* dev_status,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return quantize_call(x, dtype, rows, cols, codes, scale, amax, nullptr, dev_status, workspace,
+                       workspace_bytes, stream, true);
 }
 
 falqon_status falqon_linear_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
@@ -146,11 +168,14 @@ falqon_status falqon_linear_fwd(const uint8_t* xq, const float* s_x, const uint8
                                        static_cast<cudaStream_t>(stream)));
 }
 
-falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
-                                const float* s_w, const uint8_t* xq, const float* s_x,
-                                const void* A, const void* B, int64_t M, int64_t N, int64_t K,
-                                int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+falqon_status linear_bwd_call(const uint8_t* dyq, const float* s_dy, const uint8_t* wq, const float* s_w,
+                              const uint8_t* xq, const float* s_x, const void* A, const void* B, int64_t M,
+                              int64_t N, int64_t K, int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, void* stream, bool dy_e5m2) {
   if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
   if (!dyq || !s_dy) return FALQON_ERR_INVALID_ARG;
   if (M <= 0 || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
@@ -178,11 +203,33 @@ falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uin
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (adapters) {
     cudaError_t e = launch_adapter_grads(dyq, s_dy, xq, s_x, A, B, M, N, K, r, dA, dB,
-                                         dev_status, workspace, st);
+                                         dev_status, workspace, st, dy_e5m2);
     if (e != cudaSuccess) return from_cuda(e);
   }
-  if (dx) return from_cuda(launch_fp8_gemm_dx(dyq, s_dy, wq, s_w, M, N, K, dx, dev_status, st));
+  if (dx) return from_cuda(launch_fp8_gemm_dx(dyq, s_dy, wq, s_w, M, N, K, dx, dev_status, st, dy_e5m2));
   return FALQON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                const float* s_w, const uint8_t* xq, const float* s_x,
+                                const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_bwd_call(dyq, s_dy, wq, s_w, xq, s_x, A, B, M, N, K, r, dx, dA, dB, dev_status, workspace,
+                         workspace_bytes, stream, false);
+}
+
+falqon_status falqon_linear_bwd_e5m2(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                     const float* s_w, const uint8_t* xq, const float* s_x,
+                                     const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                     int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_bwd_call(dyq, s_dy, wq, s_w, xq, s_x, A, B, M, N, K, r, dx, dA, dB, dev_status, workspace,
+                         workspace_bytes, stream, true);
 }
 
 falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,

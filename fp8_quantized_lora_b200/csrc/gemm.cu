@@ -44,7 +44,7 @@ struct GemmArgs {
   int32_t* dev_status;
 };
 
-template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks, int kHalves>
+template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks, int kHalves, int kAFmt = 0>
 struct Cfg {
   static constexpr bool BMn = kBMn;
   static constexpr int BN = kBN;
@@ -67,7 +67,8 @@ struct Cfg {
   static constexpr uint32_t TmemCols = AccCols <= 32 ? 32 : (AccCols <= 64 ? 64 : (AccCols <= 128 ? 128 : (AccCols <= 256 ? 256 : 512)));
   static constexpr int BarBytes = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
   static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
-  static constexpr uint32_t IDesc = idesc_f32acc(0u, 0u, 0u, kBMn ? 1u : 0u, kBM, kBN);
+  // A in E4M3 (kAFmt 0) or E5M2 (1; the dX GEMM of E5M2 gradients), B in E4M3
+  static constexpr uint32_t IDesc = idesc_f32acc(static_cast<uint32_t>(kAFmt), 0u, 0u, kBMn ? 1u : 0u, kBM, kBN);
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
   static_assert(!kBMn || kBN % kRowBytes == 0, "MN-major B needs 128-byte blocks");
   static_assert(SmemBytes <= 232448, "shared memory per CTA");
@@ -317,6 +318,7 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const Gemm
 // 1.73 waves, no accumulator double buffer) and two CTAs per SM.
 using FwdCfg = Cfg<false, 256, 4, 2, 1, 1>;
 using DxCfg = Cfg<true, 256, 4, 2, 1, 1>;
+using DxE5Cfg = Cfg<true, 256, 4, 2, 1, 1, 1>;  // dYq in E5M2
 
 template <class C>
 cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
@@ -354,8 +356,9 @@ cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8
 
 cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
-                               int32_t* dev_status, cudaStream_t stream) {
+                               int32_t* dev_status, cudaStream_t stream, bool dy_e5m2) {
   // contraction over N: A = dYq [M, N] K-major; B = Wq [N, K] read MN-major (K contiguous)
+  if (dy_e5m2) return fp8_gemm<DxE5Cfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
   return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
 }
 

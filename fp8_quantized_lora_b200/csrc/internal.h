@@ -69,7 +69,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 size_t quantize_workspace_bytes(int64_t n);
 cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* codes,
                             float* scale, float* amax, float* residual, int32_t* dev_status,
-                            void* workspace, cudaStream_t stream);
+                            void* workspace, cudaStream_t stream, bool e5m2 = false);
 
 // ---------------------------------------------------------------- GEMMs
 // Y[M,N] = bf16( Xq . Wq^T / (s_x s_w) )
@@ -79,13 +79,13 @@ cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8
 // dX[M,K] = bf16( dYq . Wq / (s_dy s_w) )
 cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
-                               int32_t* dev_status, cudaStream_t stream);
+                               int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
 
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da);
 cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const uint8_t* xq,
                                  const float* s_x, const void* A, const void* B, int64_t M,
                                  int64_t N, int64_t K, int64_t r, void* dA, void* dB,
-                                 int32_t* dev_status, void* workspace, cudaStream_t stream);
+                                 int32_t* dev_status, void* workspace, cudaStream_t stream, bool dy_e5m2 = false);
 
 // ---------------------------------------------------------------- proxy
 size_t proxy_workspace_bytes(int64_t N, int64_t K);

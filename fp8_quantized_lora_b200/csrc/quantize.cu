@@ -113,6 +113,18 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Two float32 values -> two codes of the tensor's format (E5M2 when kE5).
+template <bool kE5>
+__device__ __forceinline__ uint32_t fp8x2(float lo, float hi) {
+  if constexpr (kE5) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+  } else {
+    return e4m3x2(lo, hi);
+  }
+}
+
 // Two E4M3 codes (lo in the low byte) -> their exact values.
 __device__ __forceinline__ float2 e4m3x2_value(uint32_t codes16) {
   uint32_t h2;
@@ -156,11 +168,10 @@ __device__ __forceinline__ float load1(const void* x, int64_t i) {
   }
 }
 
-// Folds the partial maxima and derives s = 448 / amax (IEEE division); CTA 0
+// s = fmax / amax from the amax bit pattern `m` (valid in thread 0), fmax the
+// format's largest finite value (448 for E4M3, 57344 for E5M2); CTA 0
 // publishes scale, amax and the status.  Returns s to every thread.
-// s = 448 / amax from the amax bit pattern `m` (valid in thread 0); CTA 0
-// publishes scale, amax and the status.  Returns s to every thread.
-__device__ __forceinline__ float scale_from_amax(uint32_t m, float* s_shared, float* scale_out,
+__device__ __forceinline__ float scale_from_amax(uint32_t m, float fmax, float* s_shared, float* scale_out,
                                                  float* amax_out, int32_t* dev_status) {
   if (threadIdx.x == 0) {
     const float amax = __uint_as_float(m);
@@ -172,7 +183,7 @@ __device__ __forceinline__ float scale_from_amax(uint32_t m, float* s_shared, fl
     } else if (m == 0u) {
       s = 1.0f;
     } else {
-      s = __fdiv_rn(448.0f, amax);
+      s = __fdiv_rn(fmax, amax);
       if (isinf(s)) {
         s = FLT_MAX;
         st = kDevScaleOverflow;
@@ -189,18 +200,23 @@ __device__ __forceinline__ float scale_from_amax(uint32_t m, float* s_shared, fl
   return *s_shared;
 }
 
-__device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int nparts,
+// Folds the partial maxima and derives the scale as scale_from_amax.
+__device__ __forceinline__ float fold_and_scale(const uint32_t* partials, int nparts, float fmax,
                                                 uint32_t* red, float* s_shared, float* scale_out,
                                                 float* amax_out, int32_t* dev_status) {
   uint32_t m = 0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, partials[i]);
   m = block_max_u32(m, red);
-  return scale_from_amax(m, s_shared, scale_out, amax_out, dev_status);
+  return scale_from_amax(m, fmax, s_shared, scale_out, amax_out, dev_status);
 }
 
-// Casts this thread's grid-stride share: codes = E4M3(fl32(x * s)), and the
-// optional residual x - dec(code) / s (fp64, rounded once to float32).
-template <bool kBF16>
+template <bool kE5>
+constexpr float kFmtMax = kE5 ? 57344.0f : 448.0f;
+
+// Casts this thread's grid-stride share: codes = FP8(fl32(x * s)) (E5M2
+// when kE5), and, for E4M3, the optional residual x - dec(code) / s (fp64,
+// rounded once to float32).
+template <bool kBF16, bool kE5>
 __device__ __forceinline__ void cast_share(const void* __restrict__ x, int64_t n, float s,
                                            uint8_t* __restrict__ codes, float* __restrict__ residual,
                                            int64_t tid, int64_t stride) {
@@ -210,12 +226,12 @@ __device__ __forceinline__ void cast_share(const void* __restrict__ x, int64_t n
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t c01 = e4m3x2(__fmul_rn(v[4 * j], s), __fmul_rn(v[4 * j + 1], s));
-      const uint32_t c23 = e4m3x2(__fmul_rn(v[4 * j + 2], s), __fmul_rn(v[4 * j + 3], s));
+      const uint32_t c01 = fp8x2<kE5>(__fmul_rn(v[4 * j], s), __fmul_rn(v[4 * j + 1], s));
+      const uint32_t c23 = fp8x2<kE5>(__fmul_rn(v[4 * j + 2], s), __fmul_rn(v[4 * j + 3], s));
       w[j] = c01 | (c23 << 16);
     }
     reinterpret_cast<uint4*>(codes)[g] = make_uint4(w[0], w[1], w[2], w[3]);
-    if (residual) {
+    if (!kE5 && residual) {
       float r[16];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -245,16 +261,16 @@ __device__ __forceinline__ void cast_share(const void* __restrict__ x, int64_t n
   }
   for (int64_t i = ng * 16 + tid; i < n; i += stride) {  // tail (n % 16 != 0)
     const float v = load1<kBF16>(x, i);
-    const uint32_t c = e4m3x2(__fmul_rn(v, s), 0.0f) & 0xFFu;
+    const uint32_t c = fp8x2<kE5>(__fmul_rn(v, s), 0.0f) & 0xFFu;
     codes[i] = static_cast<uint8_t>(c);
-    if (residual) {
+    if (!kE5 && residual) {
       const float2 d = e4m3x2_value(c);
       residual[i] = static_cast<float>(static_cast<double>(v) - static_cast<double>(d.x) / s_d);
     }
   }
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kE5>
 __global__ void __launch_bounds__(kThreads)
     quantize_cast_kernel(const void* __restrict__ x, int64_t n,
                          const uint32_t* __restrict__ partials, int nparts,
@@ -265,10 +281,11 @@ __global__ void __launch_bounds__(kThreads)
   pdl_wait();     // the previous kernel's results are complete and visible
   __shared__ uint32_t red[32];
   __shared__ float s_shared;
-  const float s = fold_and_scale(partials, nparts, red, &s_shared, scale_out, amax_out, dev_status);
+  const float s = fold_and_scale(partials, nparts, kFmtMax<kE5>, red, &s_shared, scale_out, amax_out,
+                                 dev_status);
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  cast_share<kBF16>(x, n, s, codes, residual, tid, stride);
+  cast_share<kBF16, kE5>(x, n, s, codes, residual, tid, stride);
 }
 
 // ---------------------------------------------------------------- one launch
@@ -295,7 +312,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kE5>
 __global__ void __launch_bounds__(kStreamThreads, 1)
     quantize_stream_kernel(const void* __restrict__ x, int64_t n, uint32_t* __restrict__ ws,
                            uint8_t* __restrict__ codes, float* __restrict__ scale_out,
@@ -455,7 +472,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     if (lane == 0) amax_bits = mx;
   }
   __syncthreads();
-  const float s = scale_from_amax(amax_bits, &s_shared, scale_out, amax_out, dev_status);
+  const float s = scale_from_amax(amax_bits, kFmtMax<kE5>, &s_shared, scale_out, amax_out, dev_status);
   const double s_d = static_cast<double>(s);
 
   // ---- pass 2: codes (and the optional residual)
@@ -486,14 +503,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       uint32_t cw[kE / 4];
 #pragma unroll
       for (int j = 0; j < kE / 4; ++j) {
-        const uint32_t c01 = e4m3x2(__fmul_rn(v[4 * j], s), __fmul_rn(v[4 * j + 1], s));
-        const uint32_t c23 = e4m3x2(__fmul_rn(v[4 * j + 2], s), __fmul_rn(v[4 * j + 3], s));
+        const uint32_t c01 = fp8x2<kE5>(__fmul_rn(v[4 * j], s), __fmul_rn(v[4 * j + 1], s));
+        const uint32_t c23 = fp8x2<kE5>(__fmul_rn(v[4 * j + 2], s), __fmul_rn(v[4 * j + 3], s));
         cw[j] = c01 | (c23 << 16);
       }
       const int64_t e = e0 + static_cast<int64_t>(u) * kE;
       if constexpr (kBF16) *reinterpret_cast<uint2*>(codes + e) = make_uint2(cw[0], cw[1]);
       else *reinterpret_cast<uint32_t*>(codes + e) = cw[0];
-      if (residual) {
+      if (!kE5 && residual) {
 #pragma unroll
         for (int j = 0; j < kE; j += 2) {
           const float2 d = e4m3x2_value(cw[j >> 2] >> (8 * (j & 3)));
@@ -509,9 +526,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       float v;
       if constexpr (kBF16) v = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(x)[e]) << 16);
       else v = reinterpret_cast<const float*>(x)[e];
-      const uint32_t c = e4m3x2(__fmul_rn(v, s), 0.0f) & 0xFFu;
+      const uint32_t c = fp8x2<kE5>(__fmul_rn(v, s), 0.0f) & 0xFFu;
       codes[e] = static_cast<uint8_t>(c);
-      if (residual) {
+      if (!kE5 && residual) {
         const float2 d = e4m3x2_value(c);
         residual[e] = static_cast<float>(static_cast<double>(v) - static_cast<double>(d.x) / s_d);
       }
@@ -535,29 +552,24 @@ size_t quantize_workspace_bytes(int64_t n) {
   return 4096 * sizeof(uint32_t);  // barrier words + amax partials (at most 4032 CTAs)
 }
 
-cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* codes,
-                            float* scale, float* amax, float* residual, int32_t* dev_status,
-                            void* workspace, cudaStream_t stream) {
-  const DeviceInfo* di = current_device_info();
-  if (!di) return cudaErrorInvalidDevice;
-  uint32_t* ws = static_cast<uint32_t*>(workspace);
+namespace {
+
+template <bool kBF16, bool kE5>
+cudaError_t launch_quantize_t(const DeviceInfo* di, const void* x, int64_t n, uint8_t* codes, float* scale,
+                              float* amax, float* residual, int32_t* dev_status, uint32_t* ws,
+                              cudaStream_t stream) {
   if (di->coop_launch && di->max_smem_optin >= kStreamSmemBytes) {
-    static int configured_mask[2] = {0, 0};  // per dtype, one bit per device ordinal < 31
+    static int configured_mask = 0;  // one bit per device ordinal < 31
     const int dev = di->device;
     const int bit = dev < 31 ? (1 << dev) : 0;
-    int& cm = configured_mask[is_bf16 ? 1 : 0];
-    if (!bit || !(__atomic_load_n(&cm, __ATOMIC_ACQUIRE) & bit)) {
-      cudaError_t e = is_bf16 ? cudaFuncSetAttribute(quantize_stream_kernel<true>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     kStreamSmemBytes)
-                              : cudaFuncSetAttribute(quantize_stream_kernel<false>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     kStreamSmemBytes);
+    if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
+      cudaError_t e = cudaFuncSetAttribute(quantize_stream_kernel<kBF16, kE5>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBytes);
       if (e != cudaSuccess) return e;
-      if (bit) __atomic_fetch_or(&cm, bit, __ATOMIC_ACQ_REL);
+      if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
     }
     // one CTA per SM, never more CTAs than chunks (at least one)
-    const int64_t body = (n * (is_bf16 ? 2 : 4)) / 16 * 16;
+    const int64_t body = (n * (kBF16 ? 2 : 4)) / 16 * 16;
     int64_t chunks = (body + kChunkBytes - 1) / kChunkBytes;
     int grid = static_cast<int>(chunks < di->sm_count ? (chunks > 0 ? chunks : 1) : di->sm_count);
     if (grid > 4096 - kBarWords) grid = 4096 - kBarWords;
@@ -573,11 +585,8 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (is_bf16)
-      return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<true>, x, n, ws, codes, scale, amax,
-                                residual, dev_status);
-    return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<false>, x, n, ws, codes, scale, amax,
-                              residual, dev_status);
+    return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<kBF16, kE5>, x, n, ws, codes, scale, amax, residual,
+                              dev_status);
   }
   uint32_t* partials = ws;
   const int pb = amax_blocks(n, di->sm_count);
@@ -586,16 +595,27 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
   const int64_t ccap = static_cast<int64_t>(di->sm_count) * 8;
   if (cb > ccap) cb = ccap;
   if (cb < 1) cb = 1;
-  if (is_bf16) {
-    cudaError_t e = launch_pdl(amax_partial_kernel<true>, dim3(pb), dim3(kThreads), 0, stream, 1u, x, n, partials);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_cast_kernel<true>, dim3(static_cast<unsigned>(cb)), dim3(kThreads), 0, stream, 1u, x,
-                      n, static_cast<const uint32_t*>(partials), pb, codes, scale, amax, residual, dev_status);
-  }
-  cudaError_t e = launch_pdl(amax_partial_kernel<false>, dim3(pb), dim3(kThreads), 0, stream, 1u, x, n, partials);
+  cudaError_t e = launch_pdl(amax_partial_kernel<kBF16>, dim3(pb), dim3(kThreads), 0, stream, 1u, x, n, partials);
   if (e != cudaSuccess) return e;
-  return launch_pdl(quantize_cast_kernel<false>, dim3(static_cast<unsigned>(cb)), dim3(kThreads), 0, stream, 1u, x,
-                    n, static_cast<const uint32_t*>(partials), pb, codes, scale, amax, residual, dev_status);
+  return launch_pdl(quantize_cast_kernel<kBF16, kE5>, dim3(static_cast<unsigned>(cb)), dim3(kThreads), 0, stream,
+                    1u, x, n, static_cast<const uint32_t*>(partials), pb, codes, scale, amax, residual, dev_status);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* codes,
+                            float* scale, float* amax, float* residual, int32_t* dev_status,
+                            void* workspace, cudaStream_t stream, bool e5m2) {
+  const DeviceInfo* di = current_device_info();
+  if (!di) return cudaErrorInvalidDevice;
+  uint32_t* ws = static_cast<uint32_t*>(workspace);
+  if (e5m2) {
+    if (residual) return cudaErrorInvalidValue;  // the residual is defined for E4M3 weights only
+    return is_bf16 ? launch_quantize_t<true, true>(di, x, n, codes, scale, amax, nullptr, dev_status, ws, stream)
+                   : launch_quantize_t<false, true>(di, x, n, codes, scale, amax, nullptr, dev_status, ws, stream);
+  }
+  return is_bf16 ? launch_quantize_t<true, false>(di, x, n, codes, scale, amax, residual, dev_status, ws, stream)
+                 : launch_quantize_t<false, false>(di, x, n, codes, scale, amax, residual, dev_status, ws, stream);
 }
 
 }  // namespace falqon

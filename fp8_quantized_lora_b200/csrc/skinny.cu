@@ -52,6 +52,7 @@ struct SkinnyProblem {
   int transpose;       // store out[col * ldo + row]
   int a_mn;            // the A operand is MN-major (B for U^T) instead of K-major
   int hilo;            // A rows [0, 64) hi and [64, 128) lo of the same ranks: add the halves
+  int code_e5;         // the codes are E5M2 (dY of E5M2 gradients) instead of E4M3
   const float* scale;  // alpha = 1 / *scale
 };
 
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
   const int npairs = (nkb + 1) / 2;
   const bool a_mn = g.a_mn != 0;
   const bool hilo = g.hilo != 0;
+  const bool e5 = g.code_e5 != 0;
   const int row_span = hilo ? 64 : kBM;  // ranks per tile
   const int i0 = mt * row_span;
   const int n0 = nt * kSkN;
@@ -327,9 +329,12 @@ __global__ void __launch_bounds__(C::Threads, 1)
                                                (trow + j * kRowStep) * C::RawRowBytes + tcol);
       __syncwarp();
       if (lane == 0) mbar_arrive(&rawempty[sr]);
+      // codes the bit placement cannot take (E4M3 NaN; E5M2 infinity / NaN)
+      // send the batch through the hardware conversion
       uint32_t nan_acc = 0u;
 #pragma unroll
-      for (int j = 0; j < C::ChunksPerThread; ++j) nan_acc = nan_fold(nan_acc, q[j]);
+      for (int j = 0; j < C::ChunksPerThread; ++j)
+        nan_acc = e5 ? special5_fold(nan_acc, q[j]) : nan_fold(nan_acc, q[j]);
       const bool nan = nan_found(nan_acc);
       if (!warp_wait(&empty[s], static_cast<uint32_t>(((i / C::S) & 1) ^ 1), abort_flag)) {
         if (lane == 0) fail();
@@ -339,7 +344,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
 #pragma unroll
       for (int j = 0; j < C::ChunksPerThread; ++j) {
         uint32_t o[8];
-        e4m3x16_to_bf16(q[j], nan, o);
+        if (e5) e5m2x16_to_bf16(q[j], nan, o);
+        else e4m3x16_to_bf16(q[j], nan, o);
         const int row = trow + j * kRowStep;
         *reinterpret_cast<uint4*>(sB + row * kRowBytes + ((unit0 ^ (row & 7)) << 4)) =
             make_uint4(o[0], o[1], o[2], o[3]);
@@ -468,7 +474,7 @@ struct Product {
   void* out;
   void* out_lo;
   int64_t ldo;
-  bool transpose, a_mn, hilo;
+  bool transpose, a_mn, hilo, code_e5;
   const float* scale;
   CUtensorMap raw, a, a2;
 };
@@ -506,6 +512,7 @@ cudaError_t run_products(const Product* p0, const Product* p1, int64_t r, const 
     q.transpose = p->transpose ? 1 : 0;
     q.a_mn = p->a_mn ? 1 : 0;
     q.hilo = p->hilo ? 1 : 0;
+    q.code_e5 = p->code_e5 ? 1 : 0;
     q.scale = p->scale;
     maps[3 * i] = p->raw;
     maps[3 * i + 1] = p->a;
@@ -546,7 +553,7 @@ size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool 
 cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const uint8_t* xq,
                                  const float* s_x, const void* A, const void* B, int64_t M,
                                  int64_t N, int64_t K, int64_t r, void* dA, void* dB,
-                                 int32_t* dev_status, void* workspace, cudaStream_t stream) {
+                                 int32_t* dev_status, void* workspace, cudaStream_t stream, bool dy_e5m2) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -569,7 +576,7 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   }
   if (dA) {
     u.cols = M; u.kc = N; u.out = U_hi; u.out_lo = U_lo; u.ldo = ld;
-    u.transpose = false; u.a_mn = true; u.hilo = false; u.scale = s_dy;
+    u.transpose = false; u.a_mn = true; u.hilo = false; u.code_e5 = dy_e5m2; u.scale = s_dy;
     if (!codes_tmap(&u.raw, dyq, M, N, false) || !make_tmap_2d(&u.a, BF, 2, B, r, N, 64, kSkK, true))
       return cudaErrorInvalidValue;
     u.a2 = u.a;
@@ -584,7 +591,7 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   Product db{}, da{};
   if (dB) {
     db.cols = N; db.kc = M; db.out = dB; db.out_lo = nullptr; db.ldo = r;
-    db.transpose = true; db.a_mn = false; db.hilo = true; db.scale = s_dy;
+    db.transpose = true; db.a_mn = false; db.hilo = true; db.code_e5 = dy_e5m2; db.scale = s_dy;
     if (!codes_tmap(&db.raw, dyq, M, N, true) ||
         !make_tmap_2d(&db.a, BF, 2, T_hi, M, r, kSkK, 64, true, ld) ||
         !make_tmap_2d(&db.a2, BF, 2, T_lo, M, r, kSkK, 64, true, ld))

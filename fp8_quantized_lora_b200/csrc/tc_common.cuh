@@ -98,6 +98,64 @@ __device__ __forceinline__ void e4m3x16_to_bf16(uint4 q, bool nan, uint32_t (&o)
   }
 }
 
+// E5M2 codes (sign, 5 exponent bits of bias 15, 2 mantissa bits) to bf16,
+// the same way: the byte permute replicates each code's sign into the high
+// byte, a shift by 5 and a mask put the exponent on the low five bits of the
+// bf16 exponent and the mantissa on the top of the bf16 mantissa, and one
+// exact bf16 multiply by 2^112 (the bias difference 127 - 15) restores the
+// value; subnormals land on bf16 subnormals and scale the same way.  Codes
+// with an all-ones exponent (infinity, NaN) are not handled here.
+template <uint32_t kSel>
+__device__ __forceinline__ uint32_t e5m2_pair_to_bf16x2(uint32_t w) {
+  uint32_t y, out;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(y) : "r"(w), "n"(kSel));
+  const uint32_t h = (y << 5) & 0x8FE08FE0u;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(out) : "r"(h), "r"(0x77807780u), "r"(0x80008000u));
+  return out;
+}
+
+// Evidence of E5M2 codes with an all-ones exponent (infinity or NaN): bit 7
+// of a byte of the fold ends up set iff that byte of some folded word has it.
+__device__ __forceinline__ uint32_t special5_fold(uint32_t acc, uint4 q) {
+  const uint32_t m = 0x7C7C7C7Cu, one = 0x04040404u;
+  return acc | ((q.x & m) + one) | ((q.y & m) + one) | ((q.z & m) + one) | ((q.w & m) + one);
+}
+
+// Four E5M2 codes -> four bf16 (two words) through the hardware conversion;
+// exact for every code, infinity and NaN included.
+__device__ __forceinline__ void e5m2x4_to_bf16_hw(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  uint32_t o[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint16_t pair = static_cast<uint16_t>(w >> (16 * j));
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(pair));
+    __half2 hh;
+    memcpy(&hh, &h2, 4);
+    const float2 f = __half22float2(hh);
+    const __nv_bfloat162 bb = __floats2bfloat162_rn(f.x, f.y);
+    memcpy(&o[j], &bb, 4);
+  }
+  lo = o[0];
+  hi = o[1];
+}
+
+// Sixteen E5M2 codes -> sixteen bf16 (eight words, in code order); `special`
+// selects the hardware conversion.
+__device__ __forceinline__ void e5m2x16_to_bf16(uint4 q, bool special, uint32_t (&o)[8]) {
+  const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+  if (!special) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      o[2 * j] = e5m2_pair_to_bf16x2<0x9180u>(words[j]);
+      o[2 * j + 1] = e5m2_pair_to_bf16x2<0xB3A2u>(words[j]);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) e5m2x4_to_bf16_hw(words[j], o[2 * j], o[2 * j + 1]);
+  }
+}
+
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));

@@ -109,6 +109,22 @@ FALQON_API falqon_status falqon_quantize(const void* x, falqon_dtype dtype, int6
                               void* stream);
 
 /*
+ * falqon_quantize_e5m2 - per-tensor E5M2 quantization, for gradients.
+ *
+ * The rebuttal (reviewer 2, W2) names E5M2 beside E4M3 as an FP8 format
+ * under the same per-tensor scaling.  As falqon_quantize with the E5M2 format
+ * (sign, 5 exponent bits of bias 15, 2 mantissa bits; largest finite value
+ * 57344): amax = max|x|, s = 57344 / amax (one IEEE float32 division; the
+ * same status bits), codes = E5M2(fl32(x * s)), nearest-even, saturating
+ * (every magnitude above 57344, infinity included, encodes as +-57344), NaN
+ * as 0x7F.  No residual.  Arguments, requirements and workspace as
+ * falqon_quantize (workspace: falqon_workspace_size(FALQON_OP_QUANTIZE, ...)).
+ */
+FALQON_API falqon_status falqon_quantize_e5m2(const void* x, falqon_dtype dtype, int64_t rows, int64_t cols,
+                                   uint8_t* codes, float* scale, float* amax, int32_t* dev_status,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * falqon_linear_fwd - forward GEMM on the FP8 backbone alone.
  *
  * The paper's introduction: adapters are merged into the FP8 backbone, so the
@@ -146,6 +162,20 @@ FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy
                                 const void* A, const void* B, int64_t M, int64_t N, int64_t K,
                                 int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * falqon_linear_bwd_e5m2 - falqon_linear_bwd with the gradient in E5M2.
+ *
+ * Identical to falqon_linear_bwd (same arguments, outputs, requirements and
+ * workspace) except that dyq holds E5M2 codes and s_dy is their scale, as
+ * falqon_quantize_e5m2 writes them: dX is a mixed E5M2 x E4M3 tcgen05 GEMM,
+ * and U and dB read dYq through the E5M2 decoding.
+ */
+FALQON_API falqon_status falqon_linear_bwd_e5m2(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                     const float* s_w, const uint8_t* xq, const float* s_x,
+                                     const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                     int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * falqon_proxy_update - row-wise proxy update of the quantized backbone.
