@@ -418,6 +418,7 @@ def run_gpu(args):
     status = int(st.status.item())
     n_sel = int(st.n_sel.item())
     topk = _time_topk(st, F, torch, stream, l2_flush, args, dev) if args.topk > 0 else None
+    e5 = _time_e5m2(st, F, torch, stream, l2_flush, args, dev) if args.e5m2 else None
 
     tokens_total = wl.M * args.steps * ws
     value = tokens_total / (total_ms / 1e3)
@@ -481,7 +482,7 @@ def run_gpu(args):
         "clocks": clock_info,
         "device_status": status,
         "rows_selected_last_step": n_sel,
-        "extra": {"proxy_topk": topk},
+        "extra": {"proxy_topk": topk, "e5m2_gradients": e5},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, layer, budget_s=args.cpu_budget)
@@ -521,6 +522,42 @@ def _time_topk(st, F, torch, stream, l2_flush, args, dev):
             "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
             "kernels": "proxy_pipe_kernel (count) + proxy_topk_select_kernel + proxy_topk_apply_kernel",
             "device_status": int(st.status.item())}
+
+
+def _time_e5m2(st, F, torch, stream, l2_flush, args, dev):
+    """The backward with E5M2 gradients (not part of the step): quantize dY
+    to E5M2, then the adapter products and dX reading it; eager calls timed
+    with CUDA events on the launching stream, L2 flushed before each rep."""
+    dyq = torch.empty_like(st.dyq)
+    s_dy = torch.empty(1, dtype=torch.float32, device=dev)
+    dA, dB, dx = torch.empty_like(st.dA), torch.empty_like(st.dB), torch.empty_like(st.dx)
+    names = ("quantdY", "adapters", "dX")
+    reps = max(5, min(50, args.steps))
+    acc = dict.fromkeys(names, 0.0)
+    with torch.cuda.stream(stream):
+        for i in range(3 + reps):
+            l2_flush(i)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record()
+            F.falqon_quantize(st.dY[i % 2], codes=dyq, scale=s_dy, amax=st.amax, dev_status=st.status,
+                              workspace=st.ws_q, fmt="e5m2")
+            ev[1].record()
+            F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, st.xq, st.s_x, st.A, st.B, dx=None, dA=dA, dB=dB,
+                                dev_status=st.status, workspace=st.ws_bwd, dy_fmt="e5m2")
+            ev[2].record()
+            F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, None, None, None, None, dx=dx, dA=None, dB=None,
+                                dev_status=st.status, dy_fmt="e5m2")
+            ev[3].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                for j, n in enumerate(names):
+                    acc[n] += ev[j].elapsed_time(ev[j + 1])
+    out = {n: round(acc[n] / reps, 5) for n in names}
+    M, N, K = st.M, st.N, st.K
+    out["dX_tflops"] = round(2.0 * M * N * K / (out["dX"] * 1e-3) / 1e12, 1)
+    out["unit"] = "ms per call"
+    out["device_status"] = int(st.status.item())
+    return out
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -631,6 +668,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--e5m2", type=int, default=1,
+                    help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--topk", type=int, default=256,
                     help="also time the proxy update with top-k row selection at this k (0: skip)")
     ap.add_argument("--only", default=None, choices=list(Step.PHASES),

@@ -42,16 +42,37 @@ def uniform01(seed: int, count: int) -> np.ndarray:
     return ((z >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
 
 
-def normal(seed: int, count: int, std: float = 1.0) -> np.ndarray:
-    """float64 N(0, std^2) draws by Box-Muller on consecutive uniform pairs."""
-    pairs = (count + 1) // 2
-    u = uniform01(seed, 2 * pairs)
+def _box_muller(seed: int, p0: int, p1: int, out: np.ndarray) -> None:
+    """Pairs p0 .. p1-1 of the stream (uniform draws 2p, 2p+1) into out[2p0 : 2p1]."""
+    z = splitmix64(seed, 2 * (p1 - p0), offset=2 * p0)
+    u = ((z >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
     u1, u2 = u[0::2], u[1::2]
     rad = np.sqrt(-2.0 * np.log(u1))
     ang = 2.0 * np.pi * u2
+    seg = out[2 * p0:2 * p1]
+    seg[0::2] = rad * np.cos(ang)
+    seg[1::2] = rad * np.sin(ang)
+
+
+_BLOCK_PAIRS = 1 << 20  # a multiple of the SIMD width, so every draw is computed the same way
+
+
+def normal(seed: int, count: int, std: float = 1.0) -> np.ndarray:
+    """float64 N(0, std^2) draws by Box-Muller on consecutive uniform pairs.
+
+    Large draws are split into blocks of pairs computed on a thread pool (numpy
+    releases the GIL in its loops); each draw depends only on its index, so the
+    result is the same for any split."""
+    pairs = (count + 1) // 2
     out = np.empty(2 * pairs, dtype=np.float64)
-    out[0::2] = rad * np.cos(ang)
-    out[1::2] = rad * np.sin(ang)
+    blocks = [(p, min(pairs, p + _BLOCK_PAIRS)) for p in range(0, pairs, _BLOCK_PAIRS)]
+    if len(blocks) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        import os
+        with ThreadPoolExecutor(max_workers=min(len(blocks), os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda b: _box_muller(seed, b[0], b[1], out), blocks))
+    elif blocks:
+        _box_muller(seed, 0, pairs, out)
     return out[:count] * std
 
 

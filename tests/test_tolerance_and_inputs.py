@@ -30,6 +30,19 @@ def test_normal_draws_are_deterministic_and_standard():
     assert abs(gen.normal(43, 100000, 0.02).std() - 0.02) < 0.0005
 
 
+def test_normal_draws_do_not_depend_on_the_thread_split():
+    count = 2 * gen._BLOCK_PAIRS * 2 + 3  # two full blocks of pairs and a ragged third
+    blocked = gen.normal(44, count, 1.0)
+    whole = np.empty(2 * ((count + 1) // 2))
+    gen._box_muller(44, 0, (count + 1) // 2, whole)
+    assert np.array_equal(blocked.view(np.uint64), whole[:count].view(np.uint64))
+    # each draw depends only on its index: a block starting mid-stream agrees
+    part = np.empty_like(whole)
+    gen._box_muller(44, 12345, 12345 + 64, part)
+    assert np.array_equal(part[2 * 12345:2 * 12345 + 128].view(np.uint64),
+                          whole[2 * 12345:2 * 12345 + 128].view(np.uint64))
+
+
 def test_bf16_rounding_of_inputs():
     f = np.float32([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, np.inf])
     assert gen.f32_to_bf16_bits(f).tolist() == [0x3F80, 0x3F80, 0x3F82, 0xC020, 0x7F80]
