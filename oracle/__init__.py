@@ -245,6 +245,31 @@ def adapter_da(xq, s_x, u16=None, u64=None):
     return da
 
 
+# ------------------------------------------------------------------ C-16
+def folded_t(xq, s_x, aq, s_a) -> np.ndarray:
+    """C-16: the adapter columns of the folded forward product
+    [Y | T] = Xq . [Wq ; A~q]^T, i.e. C-5's sum with the codes of A~ and
+    their scale in place of the backbone's (float64, not rounded)."""
+    return linear_fwd(xq, s_x, aq, s_a)
+
+
+def folded_u(dyq, s_dy, bq, s_b, dy_fmt: str = "e4m3") -> np.ndarray:
+    """C-16: the adapter columns of the folded dX product
+    [dX | U] = dYq . [Wq | B~q], i.e. C-6's sum with B~q [N, r] in place of
+    Wq [N, K] (float64, not rounded)."""
+    return linear_dx(dyq, s_dy, bq, s_b, dy_fmt=dy_fmt)
+
+
+def folded_adapter_grads(xq, s_x, dyq, s_dy, aq, s_a, bq=None, s_b=None, dy_fmt: str = "e4m3"):
+    """C-16: (T, dB, U, dA) of the folded path; U and dA are None without B~q."""
+    t64 = folded_t(xq, s_x, aq, s_a)
+    db = adapter_db(dyq, s_dy, t64=t64, dy_fmt=dy_fmt)
+    if bq is None:
+        return t64, db, None, None
+    u64 = folded_u(dyq, s_dy, bq, s_b, dy_fmt=dy_fmt)
+    return t64, db, u64, adapter_da(xq, s_x, u64=u64)
+
+
 # ------------------------------------------------------------------ C-9, C-10, C-11
 def proxy_accumulate(P: np.ndarray, dB_inc: np.ndarray, A: np.ndarray) -> np.ndarray:
     """Returns P + (dB_inc . A) with the float32 FMA chain; P is not modified."""

@@ -113,6 +113,21 @@
 //       dX (C-6), U and dB (C-7, C-8) read dYq through this decoding; every
 //       other step is unchanged.
 //
+//  C-16 Quantized adapters folded into the backbone products.  In the
+//       paper's Fig. 2, as the rebuttal to reviewer 2 (W1, W9) describes it,
+//       activations are multiplied with the quantized W~, A~ and B~; the
+//       rebuttal to reviewer 3 (W3.1) has both backbone and adapters in FP8;
+//       the rebuttal to reviewer 4 (Q1) has B's gradient needing only A x,
+//       known at forward time.  Reading: A and B are quantized per tensor
+//       like any other operand (C-2, C-3: A~q with s_A, B~q with s_B), and
+//       their products join the backbone products as extra output columns:
+//           [Y | T] = Xq . [Wq ; A~q]^T        T = Xq . A~q^T / (s_X s_A)
+//           [dX | U] = dYq . [Wq | B~q]        U = dYq . B~q / (s_dY s_B)
+//       T is C-5's sum with A~q in place of Wq and U is C-6's with B~q in
+//       place of Wq (exact, float64); dB and dA are C-7 and C-8 on these T
+//       and U.  Y and dX are unchanged.  No new arithmetic lives here: the
+//       Python layer composes C-3, C-5, C-6, C-7 and C-8.
+//
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
 // the only fused multiply-adds are the explicit std::fmaf calls of C-9.
