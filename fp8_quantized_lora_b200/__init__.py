@@ -18,8 +18,9 @@ import torch
 __all__ = [
     "FalqonError", "lib", "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd",
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
-    "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "OP_QUANTIZE", "OP_LINEAR_FWD",
-    "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK",
+    "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
+    "falqon_linear_bwd_folded", "folded_t_planes", "OP_QUANTIZE", "OP_LINEAR_FWD",
+    "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
     "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
@@ -27,6 +28,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfalqon.so")
 
 OP_QUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_PROXY_UPDATE, OP_PROXY_UPDATE_TOPK = 0, 1, 2, 3, 4
+OP_FOLDED_T, OP_LINEAR_BWD_FOLDED = 5, 6
 DTYPE_BF16, DTYPE_F32 = 0, 1
 PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL = 1, 2, 4
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
@@ -36,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
-    "falqon_linear_bwd_e5m2",
+    "falqon_linear_bwd_e5m2", "falqon_linear_fwd_folded", "falqon_linear_bwd_folded",
 )
 
 
@@ -69,6 +71,9 @@ def lib():
     L.falqon_proxy_update.argtypes = [p, p, p, p, p, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_proxy_update_topk.argtypes = [p, p, p, p, p, i64, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_linear_bwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p]
+    L.falqon_linear_fwd_folded.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p, p]
+    L.falqon_linear_bwd_folded.argtypes = [p, p, p, p, p, p, p, p, p, sz, i64, i64, i64, i64, p, p, p, p, p,
+                                           sz, p]
     for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
               "falqon_linear_bwd_noalloc"):
         getattr(L, f).restype = C.c_int
@@ -260,4 +265,62 @@ def falqon_linear_bwd_noalloc(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=Tru
         _ptr(None if xq is None else _u8(xq)), _ptr(s_x), _ptr(A), _ptr(B), M, N, K, r,
         _ptr(dx_t), _ptr(dA_t), _ptr(dB_t), _ptr(dev_status), _stream(stream, dev))
     _check(st, "falqon_linear_bwd_noalloc")
+    return dx_t, dA_t, dB_t
+
+
+def _folded_t_bytes(M, r):
+    return falqon_workspace_size(OP_FOLDED_T, M, 0, 0, r)
+
+
+def falqon_linear_fwd_folded(xq, s_x, wq, s_w, aq, s_a, y=None, t_saved=None, dev_status=None, stream=None):
+    """[Y | T] = Xq . [Wq ; A~q]^T in one GEMM (quantized adapter folded into
+    the backbone); returns (y, t_saved), t_saved being the uint8 buffer that
+    holds T for falqon_linear_bwd_folded (see folded_t_planes)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    r = aq.shape[0]
+    dev = xq.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    if t_saved is None:
+        t_saved, _ = _workspace(OP_FOLDED_T, M, 0, 0, r, dev, None)
+    st = lib().falqon_linear_fwd_folded(_ptr(_u8(xq)), _ptr(s_x), _ptr(_u8(wq)), _ptr(s_w), _ptr(_u8(aq)),
+                                        _ptr(s_a), M, N, K, r, _ptr(y), _ptr(t_saved), t_saved.numel(),
+                                        _ptr(dev_status), _stream(stream, dev))
+    _check(st, "falqon_linear_fwd_folded")
+    return y, t_saved
+
+
+def folded_t_planes(t_saved, M, r):
+    """(hi, lo) bfloat16 views [r, ld] of a folded T (or U) buffer: T[m, i] = hi[i, m] + lo[i, m]."""
+    ld = (M + 7) // 8 * 8
+    plane = (ld * r * 2 + 255) // 256 * 256
+    hi = t_saved[:ld * r * 2].view(torch.bfloat16).view(r, ld)
+    lo = t_saved[plane:plane + ld * r * 2].view(torch.bfloat16).view(r, ld)
+    return hi, lo
+
+
+def falqon_linear_bwd_folded(dyq, s_dy, wq, s_w, bq, s_b, xq, s_x, t_saved, r, dx=True, dA=True, dB=True,
+                             dev_status=None, workspace=None, stream=None):
+    """[dX | U] = dYq . [Wq | B~q] in one GEMM, then dB from the forward's T
+    and dA from U in one launch; each output may be True (allocate), a
+    tensor, or None.  Returns (dx, dA, dB)."""
+    M, N = dyq.shape
+    K = wq.shape[1] if wq is not None else xq.shape[1]
+    dev = dyq.device
+
+    def out(v, shape):
+        if v is True:
+            return torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        return v if v is not None and v is not False else None
+
+    dx_t, dA_t, dB_t = out(dx, (M, K)), out(dA, (r, K)), out(dB, (N, r))
+    ws, wsb = (None, 0)
+    if dA_t is not None:
+        ws, wsb = _workspace(OP_LINEAR_BWD_FOLDED, M, N, K, r, dev, workspace)
+    st = lib().falqon_linear_bwd_folded(
+        _ptr(_u8(dyq)), _ptr(s_dy), _ptr(None if wq is None else _u8(wq)), _ptr(s_w),
+        _ptr(None if bq is None else _u8(bq)), _ptr(s_b), _ptr(None if xq is None else _u8(xq)), _ptr(s_x),
+        _ptr(t_saved), 0 if t_saved is None else t_saved.numel(), M, N, K, r, _ptr(dx_t), _ptr(dA_t),
+        _ptr(dB_t), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_linear_bwd_folded")
     return dx_t, dA_t, dB_t

@@ -107,6 +107,10 @@ size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int6
     case FALQON_OP_PROXY_UPDATE_TOPK:
       if (N <= 0 || K <= 0) return 0;
       return proxy_topk_workspace_bytes(N, K);
+    case FALQON_OP_FOLDED_T:
+    case FALQON_OP_LINEAR_BWD_FOLDED:
+      if (M <= 0 || r <= 0) return 0;
+      return 2 * adapter_plane_bytes(M, r);
   }
   return 0;
 }
@@ -274,6 +278,83 @@ falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* pro
   return from_cuda(launch_proxy_update_topk(wq, s_w, proxy, dB_inc, A, N, K, r, k, flags, row_mask,
                                             n_selected, dev_status, workspace,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shape checks shared by the folded calls: the backbone's, plus r.
+falqon_status folded_shape(int64_t M, int64_t N, int64_t K, int64_t r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return FALQON_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0 || r % 16 != 0 || r > 65536) return FALQON_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256)
+    return FALQON_ERR_UNSUPPORTED;
+  return FALQON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+falqon_status falqon_linear_fwd_folded(const uint8_t* xq, const float* s_x, const uint8_t* wq, const float* s_w,
+                                       const uint8_t* aq, const float* s_a, int64_t M, int64_t N, int64_t K,
+                                       int64_t r, void* y, void* t_saved, size_t t_saved_bytes,
+                                       int32_t* dev_status, void* stream) {
+  if (!xq || !s_x || !wq || !s_w || !aq || !s_a || !y) return FALQON_ERR_INVALID_ARG;
+  falqon_status s = folded_shape(M, N, K, r);
+  if (s != FALQON_OK) return s;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(aq) || !aligned16(y)) return FALQON_ERR_UNSUPPORTED;
+  const size_t plane = adapter_plane_bytes(M, r);
+  s = check_ws(2 * plane, t_saved, t_saved_bytes);
+  if (s != FALQON_OK) return s;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  uint8_t* t = static_cast<uint8_t*>(t_saved);
+  return from_cuda(launch_fp8_gemm_fwd_folded(xq, s_x, wq, s_w, aq, s_a, M, N, K, r, y, t, t + plane,
+                                              adapter_tu_ld(M), dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const float* s_dy, const uint8_t* wq, const float* s_w,
+                                       const uint8_t* bq, const float* s_b, const uint8_t* xq, const float* s_x,
+                                       const void* t_saved, size_t t_saved_bytes, int64_t M, int64_t N, int64_t K,
+                                       int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
+  if (!dyq || !s_dy) return FALQON_ERR_INVALID_ARG;
+  falqon_status s = folded_shape(M, N, K, r);
+  if (s != FALQON_OK) return s;
+  if (!aligned16(dyq)) return FALQON_ERR_UNSUPPORTED;
+  if (dx) {
+    if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;
+    if (!aligned16(wq) || !aligned16(dx)) return FALQON_ERR_UNSUPPORTED;
+  }
+  const size_t plane = adapter_plane_bytes(M, r);
+  if (dB) {
+    if (!aligned16(dB)) return FALQON_ERR_UNSUPPORTED;
+    if (!t_saved) return FALQON_ERR_INVALID_ARG;
+    s = check_ws(2 * plane, t_saved, t_saved_bytes);
+    if (s != FALQON_OK) return s;
+  }
+  if (dA) {
+    if (!bq || !s_b || !xq || !s_x) return FALQON_ERR_INVALID_ARG;
+    if (!aligned16(bq) || !aligned16(xq) || !aligned16(dA)) return FALQON_ERR_UNSUPPORTED;
+    s = check_ws(2 * plane, workspace, workspace_bytes);
+    if (s != FALQON_OK) return s;
+  }
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* u = static_cast<uint8_t*>(workspace);
+  const int64_t ld = adapter_tu_ld(M);
+  if (dx || dA) {
+    cudaError_t e = launch_fp8_gemm_dx_folded(dyq, s_dy, wq, s_w, dA ? bq : nullptr, s_b, M, N, K, r, dx,
+                                              dA ? u : nullptr, dA ? u + plane : nullptr, ld, dev_status, st);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (!dA && !dB) return FALQON_OK;
+  const uint8_t* t = static_cast<const uint8_t*>(t_saved);
+  return from_cuda(launch_adapter_stage2(dyq, s_dy, xq, s_x, dB ? t : nullptr, dB ? t + plane : nullptr,
+                                         dA ? u : nullptr, dA ? u + plane : nullptr, ld, M, N, K, r, dA, dB,
+                                         dev_status, st));
 }
 
 }  // extern "C"

@@ -7,6 +7,15 @@
 // FALQON's point (paper introduction) is that both run on the FP8 backbone
 // alone: the adapter is merged into Wq, so there is no separate LoRA path.
 //
+// Folded quantized adapters (the paper's Fig. 2 with quantized A~ and B~):
+// the same kernel appends the adapter columns to either product,
+//   [Y | T]  = Xq  . [Wq ; A~q]^T     T = Xq . A~q^T / (s_X s_A)
+//   [dX | U] = dYq . [Wq | B~q]       U = dYq . B~q / (s_dY s_B)
+// as a second B segment: output tiles past the backbone's read their B tile
+// from a second tensor map (rows past r are zero-filled by TMA) and write
+// their columns transposed, as a bf16 hi/lo pair [r][ld] (about 16
+// significant bits), the layout the dB / dA products read.
+//
 // Roles (persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer (one lane): fills a `kStages`-deep smem ring.
 //   warp 1      TMEM owner and UMMA issuer (one lane issues).
@@ -36,11 +45,17 @@ constexpr int kMmaBar = 1;  // named barrier between the MMA issuer and its wait
 
 struct GemmArgs {
   int32_t m_tiles, n_tiles, kb_total;
-  int64_t M, N;            // output extent
+  int32_t n_tiles0;        // tiles of the backbone segment; tiles nt >= n_tiles0 are the adapter's
+  int64_t M, N;            // output extent of the backbone segment
   void* out;               // bf16 output, row-major [M][ldo]
   int64_t ldo;
   const float* scale_a;    // alpha = 1 / (scale_a * scale_b); either may be null (= 1)
   const float* scale_b;
+  int64_t N2;              // adapter columns (r); 0 without an adapter segment
+  void* out2_hi;           // adapter columns transposed: bf16 [N2][ld2], hi + lo = value
+  void* out2_lo;
+  int64_t ld2;
+  const float* scale_b2;   // alpha2 = 1 / (scale_a * scale_b2)
   int32_t* dev_status;
 };
 
@@ -82,7 +97,7 @@ struct Cfg {
 template <class C>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmArgs g) {
+                   const __grid_constant__ CUtensorMap tmB2, const GemmArgs g) {
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -113,6 +128,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (g.n_tiles0 < g.n_tiles) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TmemCols);
@@ -140,7 +156,9 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int nt = w % g.n_tiles;
         const int mt = w / g.n_tiles;
-        const int m0 = mt * C::TileM, n0 = nt * C::BN;
+        const bool seg2 = nt >= g.n_tiles0;  // an adapter tile
+        const CUtensorMap* tb = seg2 ? &tmB2 : &tmB;
+        const int m0 = mt * C::TileM, n0 = (seg2 ? nt - g.n_tiles0 : nt) * C::BN;
         for (int kb = 0; kb < g.kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { fail(); ok = false; break; }
           uint8_t* sA = smem + stage * C::StageBytes;
@@ -155,9 +173,9 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
             // B is [K][N] row-major: 128-byte column blocks of BK rows each
 #pragma unroll
             for (int c = 0; c < C::BN / kRowBytes; ++c)
-              tma_load_2d(sB + c * C::BK * kRowBytes, &tmB, &full[stage], n0 + c * kRowBytes, kb * C::BK);
+              tma_load_2d(sB + c * C::BK * kRowBytes, tb, &full[stage], n0 + c * kRowBytes, kb * C::BK);
           } else {
-            tma_load_2d(sB, &tmB, &full[stage], kb * C::BK, n0);
+            tma_load_2d(sB, tb, &full[stage], kb * C::BK, n0);
           }
           if (++stage == C::Stages) { stage = 0; phase ^= 1; }
         }
@@ -236,12 +254,17 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // 128-row half this warp drains
-    float alpha = 1.0f;
+    float alpha = 1.0f, alpha2 = 1.0f;
     {
-      double den = 1.0;
-      if (g.scale_a) den *= static_cast<double>(*g.scale_a);
+      const double sa = g.scale_a ? static_cast<double>(*g.scale_a) : 1.0;
+      double den = sa;
       if (g.scale_b) den *= static_cast<double>(*g.scale_b);
       alpha = static_cast<float>(1.0 / den);
+      if (g.n_tiles0 < g.n_tiles) {
+        double den2 = sa;
+        if (g.scale_b2) den2 *= static_cast<double>(*g.scale_b2);
+        alpha2 = static_cast<float>(1.0 / den2);
+      }
     }
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -251,6 +274,37 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       if (!warp_wait(&acc_full[acc], acc_phase, abort_flag)) { if (lane == 0) fail(); break; }
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * C::TileM + half * kBM + q * 32 + lane;
+      if (nt >= g.n_tiles0) {
+        // adapter columns: rank i of token `row` goes to out2[i][row]; the 32
+        // lanes of a warp hold 32 consecutive tokens, so each store is 64 bytes
+        const int64_t i0 = static_cast<int64_t>(nt - g.n_tiles0) * C::BN;
+        __nv_bfloat16* hi_out = static_cast<__nv_bfloat16*>(g.out2_hi);
+        __nv_bfloat16* lo_out = static_cast<__nv_bfloat16*>(g.out2_lo);
+#pragma unroll 1
+        for (int c = 0; c < C::BN / 32 && i0 + c * 32 < g.N2; ++c) {  // warp-uniform bound
+          uint32_t r[32];
+          tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * C::Halves + half) * C::BN +
+                             c * 32, r);
+          tmem_ld_wait();
+          if (row < g.M) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int64_t i = i0 + c * 32 + j;
+              if (i < g.N2) {
+                const float v = __uint_as_float(r[j]) * alpha2;
+                const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                hi_out[i * g.ld2 + row] = h;
+                lo_out[i * g.ld2 + row] = __float2bfloat16_rn(v - __bfloat162float(h));
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (++acc == C::Acc) { acc = 0; acc_phase ^= 1; }
+        continue;
+      }
       const int64_t col_base = static_cast<int64_t>(nt) * C::BN;
 #pragma unroll 1
       for (int c = 0; c < C::BN / 32; ++c) {
@@ -294,7 +348,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 
 // ---------------------------------------------------------------- host side
 template <class C>
-cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const GemmArgs& g,
+cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const GemmArgs& g,
                         cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
@@ -309,7 +363,7 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const Gemm
   const int total = g.m_tiles * g.n_tiles;
   const int slots = C::MinBlocks * di->sm_count;
   const int grid = total < slots ? total : slots;
-  return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, g);
+  return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2, g);
 }
 
 // 128 x 256 tiles, 4-stage ring, double-buffered accumulator, one CTA per SM.
@@ -320,30 +374,58 @@ using FwdCfg = Cfg<false, 256, 4, 2, 1, 1>;
 using DxCfg = Cfg<true, 256, 4, 2, 1, 1>;
 using DxE5Cfg = Cfg<true, 256, 4, 2, 1, 1, 1>;  // dYq in E5M2
 
+// The adapter segment, when present: B2 (A~q [N2, Kc] K-major, or B~q
+// [Kc, N2] MN-major) with scale sb2, written transposed to the hi/lo planes
+// out2_hi / out2_lo [N2][ld2].  `out` may be null (no backbone segment: the
+// grid then covers the adapter tiles alone).
+struct Segment2 {
+  const uint8_t* b = nullptr;
+  const float* sb = nullptr;
+  int64_t n = 0;
+  void* hi = nullptr;
+  void* lo = nullptr;
+  int64_t ld = 0;
+};
+
+template <class C>
+bool b_tmap(CUtensorMap* t, const uint8_t* b, int64_t Ncols, int64_t Kc) {
+  // B K-major [Ncols, Kc] or MN-major [Kc, Ncols]
+  return C::BMn ? make_tmap_2d(t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Ncols, Kc, 128, C::BK, true)
+                : make_tmap_2d(t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::BN, true);
+}
+
 template <class C>
 cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
                      int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
-                     cudaStream_t stream) {
-  CUtensorMap tA, tB;
-  // A [M, Kc] K-major; B K-major [Ncols, Kc] or MN-major [Kc, Ncols]
+                     cudaStream_t stream, const Segment2& s2 = Segment2{}) {
+  CUtensorMap tA, tB, tB2;
+  // A [M, Kc] K-major
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a, Kc, M, 128, kBM, true))
     return cudaErrorInvalidValue;
-  const bool okb = C::BMn
-                       ? make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Ncols, Kc, 128, C::BK, true)
-                       : make_tmap_2d(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::BN, true);
-  if (!okb) return cudaErrorInvalidValue;
+  const bool seg1 = out != nullptr;
+  if (seg1 && !b_tmap<C>(&tB, b, Ncols, Kc)) return cudaErrorInvalidValue;
+  if (s2.n > 0 && !b_tmap<C>(&tB2, s2.b, s2.n, Kc)) return cudaErrorInvalidValue;
+  if (!seg1) tB = tB2;
+  if (s2.n <= 0) tB2 = tB;
   GemmArgs g{};
   g.m_tiles = ceil_div(M, C::TileM);
-  g.n_tiles = ceil_div(Ncols, C::BN);
+  g.n_tiles0 = seg1 ? ceil_div(Ncols, C::BN) : 0;
+  g.n_tiles = g.n_tiles0 + (s2.n > 0 ? ceil_div(s2.n, C::BN) : 0);
   g.kb_total = ceil_div(Kc, C::BK);
   g.M = M;
-  g.N = Ncols;
+  g.N = seg1 ? Ncols : 0;
   g.out = out;
   g.ldo = Ncols;
   g.scale_a = sa;
   g.scale_b = sb;
+  g.N2 = s2.n > 0 ? s2.n : 0;
+  g.out2_hi = s2.hi;
+  g.out2_lo = s2.lo;
+  g.ld2 = s2.ld;
+  g.scale_b2 = s2.sb;
   g.dev_status = dev_status;
-  return launch_gemm<C>(tA, tB, g, stream);
+  if (g.n_tiles == 0) return cudaSuccess;
+  return launch_gemm<C>(tA, tB, tB2, g, stream);
 }
 
 }  // namespace
@@ -360,6 +442,25 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
   // contraction over N: A = dYq [M, N] K-major; B = Wq [N, K] read MN-major (K contiguous)
   if (dy_e5m2) return fp8_gemm<DxE5Cfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
   return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
+}
+
+cudaError_t launch_fp8_gemm_fwd_folded(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                       const float* s_w, const uint8_t* aq, const float* s_a, int64_t M,
+                                       int64_t N, int64_t K, int64_t r, void* y, void* t_hi, void* t_lo,
+                                       int64_t ld, int32_t* dev_status, cudaStream_t stream) {
+  Segment2 s2;
+  s2.b = aq; s2.sb = s_a; s2.n = r; s2.hi = t_hi; s2.lo = t_lo; s2.ld = ld;
+  return fp8_gemm<FwdCfg>(xq, s_x, wq, s_w, M, N, K, y, dev_status, stream, s2);
+}
+
+cudaError_t launch_fp8_gemm_dx_folded(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                      const float* s_w, const uint8_t* bq, const float* s_b, int64_t M,
+                                      int64_t N, int64_t K, int64_t r, void* dx, void* u_hi, void* u_lo,
+                                      int64_t ld, int32_t* dev_status, cudaStream_t stream) {
+  // contraction over N: B~q [N, r] is the MN-major second segment beside Wq [N, K]
+  Segment2 s2;
+  s2.b = bq; s2.sb = s_b; s2.n = bq ? r : 0; s2.hi = u_hi; s2.lo = u_lo; s2.ld = ld;
+  return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream, s2);
 }
 
 }  // namespace falqon

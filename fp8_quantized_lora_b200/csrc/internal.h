@@ -86,6 +86,30 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
                                  const float* s_x, const void* A, const void* B, int64_t M,
                                  int64_t N, int64_t K, int64_t r, void* dA, void* dB,
                                  int32_t* dev_status, void* workspace, cudaStream_t stream, bool dy_e5m2 = false);
+// dB / dA from T and U held as transposed bf16 hi/lo planes [r][ld]
+cudaError_t launch_adapter_stage2(const uint8_t* dyq, const float* s_dy, const uint8_t* xq, const float* s_x,
+                                  const void* T_hi, const void* T_lo, const void* U_hi, const void* U_lo,
+                                  int64_t ld, int64_t M, int64_t N, int64_t K, int64_t r, void* dA, void* dB,
+                                  int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
+// Row stride (elements) of a transposed T / U plane: M rounded up to 8.
+inline int64_t adapter_tu_ld(int64_t M) { return (M + 7) / 8 * 8; }
+// Bytes of one [r][ld] bf16 plane, padded to 256.
+inline size_t adapter_plane_bytes(int64_t M, int64_t r) {
+  return align_up(static_cast<size_t>(adapter_tu_ld(M)) * static_cast<size_t>(r) * 2, 256);
+}
+
+// Folded quantized adapters: the backbone GEMMs with the adapter columns
+// appended (T = Xq . A~q^T / (s_x s_a), U = dYq . B~q / (s_dy s_b)), written
+// transposed as bf16 hi/lo planes [r][ld].  y / dx may be null (adapter
+// columns only); bq may be null in the dX launch (no U).
+cudaError_t launch_fp8_gemm_fwd_folded(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                       const float* s_w, const uint8_t* aq, const float* s_a, int64_t M,
+                                       int64_t N, int64_t K, int64_t r, void* y, void* t_hi, void* t_lo,
+                                       int64_t ld, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_fp8_gemm_dx_folded(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                      const float* s_w, const uint8_t* bq, const float* s_b, int64_t M,
+                                      int64_t N, int64_t K, int64_t r, void* dx, void* u_hi, void* u_lo,
+                                      int64_t ld, int32_t* dev_status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- proxy
 size_t proxy_workspace_bytes(int64_t N, int64_t K);

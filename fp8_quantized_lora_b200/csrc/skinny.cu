@@ -533,7 +533,7 @@ bool codes_tmap(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t co
 
 // Row stride (elements) of the transposed T / U workspace: M rounded up so
 // that rows start 16-byte aligned.
-int64_t tu_ld(int64_t M) { return (M + 7) / 8 * 8; }
+int64_t tu_ld(int64_t M) { return adapter_tu_ld(M); }
 
 }  // namespace
 
@@ -585,9 +585,22 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
   if (dB && dA) e = run_products<KCfg>(&t, &u, r, di, dev_status, stream);
   else e = run_products<KCfg>(dB ? &t : &u, nullptr, r, di, dev_status, stream);
   if (e != cudaSuccess) return e;
+  return launch_adapter_stage2(dyq, s_dy, xq, s_x, T_hi, T_lo, U_hi, U_lo, ld, M, N, K, r, dA, dB, dev_status,
+                               stream, dy_e5m2);
+}
 
-  // stage 2: dB^T = (T_hi + T_lo)^T . dYq / s_dy, stored as dB [N, r], and
-  // dA = (U_hi + U_lo)^T . Xq / s_x [r, K]
+// Stage 2 on T and U given as transposed bf16 hi/lo planes [r][ld] (from
+// stage 1 above, or from the folded FP8 GEMMs' adapter columns):
+//   dB^T = (T_hi + T_lo)^T . dYq / s_dy, stored as dB [N, r]
+//   dA   = (U_hi + U_lo)^T . Xq / s_x   [r, K]
+cudaError_t launch_adapter_stage2(const uint8_t* dyq, const float* s_dy, const uint8_t* xq, const float* s_x,
+                                  const void* T_hi, const void* T_lo, const void* U_hi, const void* U_lo,
+                                  int64_t ld, int64_t M, int64_t N, int64_t K, int64_t r, void* dA, void* dB,
+                                  int32_t* dev_status, cudaStream_t stream, bool dy_e5m2) {
+  const DeviceInfo* di = current_device_info();
+  if (!di) return cudaErrorInvalidDevice;
+  if (!dA && !dB) return cudaSuccess;
+  const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   Product db{}, da{};
   if (dB) {
     db.cols = N; db.kc = M; db.out = dB; db.out_lo = nullptr; db.ldo = r;

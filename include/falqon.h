@@ -68,7 +68,9 @@ typedef enum falqon_op {
   FALQON_OP_LINEAR_FWD = 1,
   FALQON_OP_LINEAR_BWD = 2,
   FALQON_OP_PROXY_UPDATE = 3,
-  FALQON_OP_PROXY_UPDATE_TOPK = 4
+  FALQON_OP_PROXY_UPDATE_TOPK = 4,
+  FALQON_OP_FOLDED_T = 5,          /* the buffer T of the folded forward keeps for the backward */
+  FALQON_OP_LINEAR_BWD_FOLDED = 6  /* workspace of falqon_linear_bwd_folded (U, when dA is wanted) */
 } falqon_op;
 
 /* Bits OR-ed into *dev_status by the kernels. */
@@ -176,6 +178,59 @@ FALQON_API falqon_status falqon_linear_bwd_e5m2(const uint8_t* dyq, const float*
                                      const void* A, const void* B, int64_t M, int64_t N, int64_t K,
                                      int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * falqon_linear_fwd_folded - forward with quantized adapters folded into the
+ * backbone GEMM.
+ *
+ * The paper's Fig. 2 (as the rebuttal to reviewer 2, W1/W9, describes it)
+ * multiplies the activations with quantized weights W~, A~ and B~, and the
+ * rebuttal to reviewer 3 (W3.1) has backbone and adapters in FP8; B's
+ * gradient needs only A x, known at forward time (rebuttal to reviewer 4,
+ * Q1).  With A~q = E4M3 codes of A and s_a its scale (falqon_quantize of A),
+ * one tcgen05 GEMM computes
+ *     [Y | T] = Xq . [Wq ; A~q]^T,   Y as falqon_linear_fwd (bit-identical),
+ *     T[m,i] = sum_k dec(Xq[m,k]) * dec(A~q[i,k]) / (s_X * s_A),
+ * accumulated in float32 and kept for falqon_linear_bwd_folded.
+ *
+ *  xq [M, K], s_x; wq [N, K], s_w; aq [r, K] E4M3, s_a 1 float; y [M, N]
+ *  bfloat16, written.
+ *  t_saved: caller-owned device buffer of falqon_workspace_size(
+ *    FALQON_OP_FOLDED_T, M, 0, 0, r) bytes (256-byte aligned), written: T
+ *    transposed as two bfloat16 planes, hi then lo, each [r][ld] with
+ *    ld = M rounded up to a multiple of 8 and the plane padded to 256 bytes;
+ *    T[m,i] = hi[i][m] + lo[i][m] (about 16 significant bits).
+ *  Requirements: M >= 1; N, K multiples of 16; r a multiple of 16.
+ */
+FALQON_API falqon_status falqon_linear_fwd_folded(const uint8_t* xq, const float* s_x, const uint8_t* wq,
+                                       const float* s_w, const uint8_t* aq, const float* s_a, int64_t M,
+                                       int64_t N, int64_t K, int64_t r, void* y, void* t_saved,
+                                       size_t t_saved_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * falqon_linear_bwd_folded - backward with quantized adapters folded into
+ * the backbone GEMM (the counterpart of falqon_linear_fwd_folded).
+ *
+ * With B~q the E4M3 codes of B [N, r] and s_b its scale, one tcgen05 GEMM
+ * computes [dX | U] = dYq . [Wq | B~q]: dX as falqon_linear_bwd
+ * (bit-identical), U[m,i] = sum_n dec(dYq[m,n]) * dec(B~q[n,i]) / (s_dY s_B);
+ * then one launch computes
+ *     dB = dYq^T . T / s_dY     (T from the forward's t_saved)   [N, r]
+ *     dA = U^T . Xq / s_X                                        [r, K]
+ *
+ *  dyq [M, N], s_dy; wq [N, K], s_w (read when dx != NULL); bq [N, r],
+ *  s_b, xq [M, K], s_x (read when dA != NULL); t_saved as the forward wrote
+ *  it (read when dB != NULL).  dx, dA, dB: bfloat16 outputs, each nullable.
+ *  workspace: falqon_workspace_size(FALQON_OP_LINEAR_BWD_FOLDED, M, N, K, r)
+ *  bytes when dA != NULL (U), else unused.
+ *  Requirements: as falqon_linear_fwd_folded.
+ */
+FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
+                                       const float* s_w, const uint8_t* bq, const float* s_b,
+                                       const uint8_t* xq, const float* s_x, const void* t_saved,
+                                       size_t t_saved_bytes, int64_t M, int64_t N, int64_t K, int64_t r,
+                                       void* dx, void* dA, void* dB, int32_t* dev_status, void* workspace,
+                                       size_t workspace_bytes, void* stream);
 
 /*
  * falqon_proxy_update - row-wise proxy update of the quantized backbone.

@@ -115,6 +115,35 @@ def test_proxy_topk_argument_errors():
     assert f(P, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws - 256, None) == 3  # workspace
 
 
+def test_folded_argument_errors():
+    L = F.lib()
+    M, N, K, r = 64, 32, 48, 16
+    tb = F.falqon_workspace_size(F.OP_FOLDED_T, M, 0, 0, r)
+    assert tb == F.falqon_workspace_size(F.OP_LINEAR_BWD_FOLDED, M, N, K, r)
+    assert tb >= 2 * 64 * 16 * 2 and tb % 256 == 0  # two bf16 planes [r][M]
+    fwd = L.falqon_linear_fwd_folded
+    assert fwd(P, P, P, P, None, P, M, N, K, r, P, P, tb, None, None) == 1       # no A~q
+    assert fwd(P, P, P, P, P, P, M, N, K, 0, P, P, tb, None, None) == 1          # r = 0
+    assert fwd(P, P, P, P, P, P, M, N, K, 24, P, P, tb, None, None) == 2         # r % 16
+    assert fwd(P, P, P, P, P, P, M, N, 40, r, P, P, tb, None, None) == 2         # K % 16
+    assert fwd(P, P, P, P, P8, P, M, N, K, r, P, P, tb, None, None) == 2         # unaligned A~q
+    assert fwd(P, P, P, P, P, P, M, N, K, r, P, P, tb - 256, None, None) == 3    # T buffer too small
+    assert fwd(P, P, P, P, P, P, M, N, K, r, P, P8, tb, None, None) == 3         # T buffer misaligned
+    bwd = L.falqon_linear_bwd_folded
+    args = dict(dyq=P, s_dy=P, wq=P, s_w=P, bq=P, s_b=P, xq=P, s_x=P, t=P, tb=tb, dx=P, dA=P, dB=P, ws=P, wsb=tb)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return bwd(a["dyq"], a["s_dy"], a["wq"], a["s_w"], a["bq"], a["s_b"], a["xq"], a["s_x"], a["t"], a["tb"],
+                   M, N, K, r, a["dx"], a["dA"], a["dB"], None, a["ws"], a["wsb"], None)
+    assert call(dx=None, dA=None, dB=None) == 1   # nothing to compute
+    assert call(bq=None) == 1                     # dA needs B~q
+    assert call(t=None) == 1                      # dB needs the forward's T
+    assert call(tb=tb - 256) == 3                 # T buffer too small
+    assert call(ws=None, wsb=0) == 3              # dA needs U's workspace
+    assert call(dA=P8) == 2                       # unaligned output
+
+
 @pytest.mark.parametrize("name", ["falqon_quantize", "falqon_linear_fwd"])
 def test_binding_refuses_cpu_tensors(name):
     import torch
