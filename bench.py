@@ -224,12 +224,12 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # differs, the roofline's traffic is null.
 TRAFFIC = {
     "proxy": {
-        "bytes": 107227392,
+        "bytes": 103531008,
         "profile": "profiles/proxy_update_llama7b_attn_proj_4096_r64.md",
         "sources": {
-            "fp8_quantized_lora_b200/csrc/proxy.cu": "ef21e5a05cbf0ef861d2413eaae2749d7f506305d21a5a73a4a92587a12b289b",
+            "fp8_quantized_lora_b200/csrc/proxy.cu": "7f9871f1e86a9f2136e6bfcee8147affd9f32ed4e9e9df9d5da8e9ab7af18366",
             "fp8_quantized_lora_b200/csrc/ptx.cuh": "1ec40a2067b4ae4960ba3532651728a393a070d5a79f0c934e7e37f8439b9c2e",
-            "fp8_quantized_lora_b200/csrc/internal.h": "953e4f0eefaccb9f774eb403aff06f254e1e9b8a18c7a80e01518aca130f3403",
+            "fp8_quantized_lora_b200/csrc/internal.h": "f1af0da524732c61365588d5645c5a3c5bdd585f99131659048ed968374d86e0",
         },
     },
 }
@@ -419,6 +419,7 @@ def run_gpu(args):
     n_sel = int(st.n_sel.item())
     topk = _time_topk(st, F, torch, stream, l2_flush, args, dev) if args.topk > 0 else None
     e5 = _time_e5m2(st, F, torch, stream, l2_flush, args, dev) if args.e5m2 else None
+    folded = _time_folded(st, F, torch, stream, l2_flush, args, dev) if args.folded else None
 
     tokens_total = wl.M * args.steps * ws
     value = tokens_total / (total_ms / 1e3)
@@ -482,7 +483,7 @@ def run_gpu(args):
         "clocks": clock_info,
         "device_status": status,
         "rows_selected_last_step": n_sel,
-        "extra": {"proxy_topk": topk, "e5m2_gradients": e5},
+        "extra": {"proxy_topk": topk, "e5m2_gradients": e5, "folded_adapters": folded},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, layer, budget_s=args.cpu_budget)
@@ -556,6 +557,53 @@ def _time_e5m2(st, F, torch, stream, l2_flush, args, dev):
     M, N, K = st.M, st.N, st.K
     out["dX_tflops"] = round(2.0 * M * N * K / (out["dX"] * 1e-3) / 1e12, 1)
     out["unit"] = "ms per call"
+    out["device_status"] = int(st.status.item())
+    return out
+
+
+def _time_folded(st, F, torch, stream, l2_flush, args, dev):
+    """Quantized adapters folded into the backbone GEMMs (not part of the
+    step): quantize B, the forward with T's columns, the dX GEMM with U's
+    columns and the dB / dA launch; A is frozen and quantized once, outside
+    the timing.  Eager calls timed with CUDA events on the launching stream,
+    L2 flushed before each rep."""
+    aq, s_a, _ = F.falqon_quantize(st.A, dev_status=st.status)
+    bq = torch.empty((st.N, st.r), dtype=torch.uint8, device=dev)
+    s_b = torch.empty(1, dtype=torch.float32, device=dev)
+    amax = torch.empty(1, dtype=torch.float32, device=dev)
+    ws_b = torch.empty(max(F.falqon_workspace_size(F.OP_QUANTIZE, st.N, st.r), 256), dtype=torch.uint8,
+                       device=dev)
+    t_saved = torch.empty(F.falqon_workspace_size(F.OP_FOLDED_T, st.M, 0, 0, st.r), dtype=torch.uint8,
+                          device=dev)
+    ws_u = torch.empty(F.falqon_workspace_size(F.OP_LINEAR_BWD_FOLDED, st.M, st.N, st.K, st.r),
+                       dtype=torch.uint8, device=dev)
+    y, dx = torch.empty_like(st.y), torch.empty_like(st.dx)
+    dA, dB = torch.empty_like(st.dA), torch.empty_like(st.dB)
+    names = ("quantB", "fwd_T", "bwd")
+    reps = max(5, min(50, args.steps))
+    acc = dict.fromkeys(names, 0.0)
+    with torch.cuda.stream(stream):
+        for i in range(3 + reps):
+            l2_flush(i)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            ev[0].record()
+            F.falqon_quantize(st.B, codes=bq, scale=s_b, amax=amax, dev_status=st.status, workspace=ws_b)
+            ev[1].record()
+            F.falqon_linear_fwd_folded(st.xq, st.s_x, st.wq, st.s_w, aq, s_a, y=y, t_saved=t_saved,
+                                       dev_status=st.status)
+            ev[2].record()
+            F.falqon_linear_bwd_folded(st.dyq, st.s_dy, st.wq, st.s_w, bq, s_b, st.xq, st.s_x, t_saved, st.r,
+                                       dx=dx, dA=dA, dB=dB, dev_status=st.status, workspace=ws_u)
+            ev[3].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                for j, n in enumerate(names):
+                    acc[n] += ev[j].elapsed_time(ev[j + 1])
+    out = {n: round(acc[n] / reps, 5) for n in names}
+    out["total"] = round(sum(out[n] for n in names), 5)
+    out["unit"] = "ms per call"
+    out["kernels"] = ("quantize_stream_kernel (B); tc_gemm_kernel with T columns; tc_gemm_kernel (dX) with U "
+                      "columns + skinny_kernel (dB^T with dA)")
     out["device_status"] = int(st.status.item())
     return out
 
@@ -668,6 +716,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--folded", type=int, default=1,
+                    help="also time the folded quantized-adapter path (1) or skip it (0)")
     ap.add_argument("--e5m2", type=int, default=1,
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--topk", type=int, default=256,
