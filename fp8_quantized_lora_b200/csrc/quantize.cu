@@ -536,6 +536,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   }
 }
 
+constexpr int64_t kSmallTensor = int64_t(1) << 20;  // elements
+
 int amax_blocks(int64_t n, int sm_count) {
   const int64_t per_block = static_cast<int64_t>(kThreads) * 64;  // >= 64 elements per thread
   int64_t b = (n + per_block - 1) / per_block;
@@ -558,7 +560,10 @@ template <bool kBF16, bool kE5>
 cudaError_t launch_quantize_t(const DeviceInfo* di, const void* x, int64_t n, uint8_t* codes, float* scale,
                               float* amax, float* residual, int32_t* dev_status, uint32_t* ws,
                               cudaStream_t stream) {
-  if (di->coop_launch && di->max_smem_optin >= kStreamSmemBytes) {
+  // Small tensors (an adapter, a bias) take the two-launch path: its fixed
+  // cost (two short PDL-overlapped launches) is below the cooperative
+  // launch's memset, launch and grid exchange.
+  if (n > kSmallTensor && di->coop_launch && di->max_smem_optin >= kStreamSmemBytes) {
     static int configured_mask = 0;  // one bit per device ordinal < 31
     const int dev = di->device;
     const int bit = dev < 31 ? (1 << dev) : 0;

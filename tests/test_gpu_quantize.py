@@ -35,12 +35,15 @@ def _check(x_np, residual=False):
         np.testing.assert_array_equal(res.view(np.uint32), r32.view(np.uint32))
 
 
-@pytest.mark.parametrize("shape", [(256, 512), (1, 16), (37, 48), (129, 272), (1000, 1008)])
+# up to 2^20 elements the library takes the two-launch path (amax partials,
+# then the cast); above it the cooperative one-launch stream kernel
+@pytest.mark.parametrize("shape", [(256, 512), (1, 16), (37, 48), (129, 272), (1000, 1008), (1024, 1024),
+                                   (1031, 1040), (4097, 272), (2048, 2064)])
 def test_bf16_activations(cuda_device, shape):
     _check(gen.normal_bf16_bits(11 + shape[0], shape, 1.0))
 
 
-@pytest.mark.parametrize("shape", [(512, 512), (37, 48), (300, 4096)])
+@pytest.mark.parametrize("shape", [(512, 512), (37, 48), (300, 4096), (257, 4112)])
 def test_f32_weights_with_eq8_residual(cuda_device, shape):
     _check(gen.normal_f32(21 + shape[0], shape, 0.02), residual=True)
 
