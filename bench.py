@@ -492,10 +492,45 @@ def run_gpu(args):
     return out, rank
 
 
+def _graph_phase_times(torch, stream, l2_flush, fns, reps, use_graph=True):
+    """Device time (ms) of each enqueueing function in ``fns``: each is
+    captured in its own CUDA graph and the graphs are replayed back to back
+    with events between them (no host launch gaps inside a phase), L2 flushed
+    before every rep outside the events; 3 untimed reps first."""
+    with torch.cuda.stream(stream):
+        for f in fns:  # warm the library (attributes, tensor-map encoder)
+            f()
+    torch.cuda.synchronize()
+    graphs = []
+    if use_graph:
+        for f in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                f()
+            graphs.append(g)
+    torch.cuda.synchronize()
+    acc = [0.0] * len(fns)
+    with torch.cuda.stream(stream):
+        for i in range(3 + reps):
+            l2_flush(i)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+            ev[0].record()
+            for k, f in enumerate(fns):
+                if graphs:
+                    graphs[k].replay()
+                else:
+                    f()
+                ev[k + 1].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                for k in range(len(fns)):
+                    acc[k] += ev[k].elapsed_time(ev[k + 1])
+    return [a / reps for a in acc]
+
+
 def _time_topk(st, F, torch, stream, l2_flush, args, dev):
-    """The proxy update with top-k row selection (not part of the step): on
-    copies of the step's Wq and P with its last dB_inc, eager calls timed
-    with CUDA events on the launching stream, L2 flushed before each."""
+    """The proxy update with top-k row selection (not part of the step), on
+    copies of the step's Wq and P with its last dB_inc."""
     N, K = st.P.shape
     wq, P = st.wq.clone(), st.P.clone()
     mask = torch.empty(N, dtype=torch.uint8, device=dev)
@@ -503,70 +538,51 @@ def _time_topk(st, F, torch, stream, l2_flush, args, dev):
     wsz = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, N, K, st.r)
     ws = torch.empty(max(wsz, 256), dtype=torch.uint8, device=dev)
     reps = max(5, min(50, args.steps))
-    total = 0.0
-    with torch.cuda.stream(stream):
-        for i in range(3 + reps):
-            l2_flush(i)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            F.falqon_proxy_update_topk(wq, st.s_w, P, st.dB_inc, st.A, args.topk, row_mask=mask,
-                                       n_selected=cnt, dev_status=st.status, workspace=ws)
-            e1.record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                total += e0.elapsed_time(e1)
-    ms = total / reps
+
+    def call():
+        F.falqon_proxy_update_topk(wq, st.s_w, P, st.dB_inc, st.A, args.topk, row_mask=mask,
+                                   n_selected=cnt, dev_status=st.status, workspace=ws)
+    (ms,) = _graph_phase_times(torch, stream, l2_flush, [call], reps, not args.no_graph)
     flops = 2.0 * N * K * st.r
     return {"k": args.topk, "ms": round(ms, 5), "rows_selected": int(cnt.item()),
             "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
             "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
             "kernels": "proxy_pipe_kernel (count) + proxy_topk_select_kernel + proxy_topk_apply_kernel",
+            "timing": "CUDA graph replay, events on the launching stream",
             "device_status": int(st.status.item())}
 
 
 def _time_e5m2(st, F, torch, stream, l2_flush, args, dev):
     """The backward with E5M2 gradients (not part of the step): quantize dY
-    to E5M2, then the adapter products and dX reading it; eager calls timed
-    with CUDA events on the launching stream, L2 flushed before each rep."""
+    to E5M2, then the adapter products and dX reading it."""
     dyq = torch.empty_like(st.dyq)
     s_dy = torch.empty(1, dtype=torch.float32, device=dev)
     dA, dB, dx = torch.empty_like(st.dA), torch.empty_like(st.dB), torch.empty_like(st.dx)
     names = ("quantdY", "adapters", "dX")
     reps = max(5, min(50, args.steps))
-    acc = dict.fromkeys(names, 0.0)
-    with torch.cuda.stream(stream):
-        for i in range(3 + reps):
-            l2_flush(i)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            ev[0].record()
-            F.falqon_quantize(st.dY[i % 2], codes=dyq, scale=s_dy, amax=st.amax, dev_status=st.status,
-                              workspace=st.ws_q, fmt="e5m2")
-            ev[1].record()
-            F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, st.xq, st.s_x, st.A, st.B, dx=None, dA=dA, dB=dB,
-                                dev_status=st.status, workspace=st.ws_bwd, dy_fmt="e5m2")
-            ev[2].record()
-            F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, None, None, None, None, dx=dx, dA=None, dB=None,
-                                dev_status=st.status, dy_fmt="e5m2")
-            ev[3].record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                for j, n in enumerate(names):
-                    acc[n] += ev[j].elapsed_time(ev[j + 1])
-    out = {n: round(acc[n] / reps, 5) for n in names}
+    fns = [
+        lambda: F.falqon_quantize(st.dY[0], codes=dyq, scale=s_dy, amax=st.amax, dev_status=st.status,
+                                  workspace=st.ws_q, fmt="e5m2"),
+        lambda: F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, st.xq, st.s_x, st.A, st.B, dx=None, dA=dA,
+                                    dB=dB, dev_status=st.status, workspace=st.ws_bwd, dy_fmt="e5m2"),
+        lambda: F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, None, None, None, None, dx=dx, dA=None,
+                                    dB=None, dev_status=st.status, dy_fmt="e5m2"),
+    ]
+    ms = _graph_phase_times(torch, stream, l2_flush, fns, reps, not args.no_graph)
+    out = {n: round(t, 5) for n, t in zip(names, ms)}
     M, N, K = st.M, st.N, st.K
     out["dX_tflops"] = round(2.0 * M * N * K / (out["dX"] * 1e-3) / 1e12, 1)
     out["unit"] = "ms per call"
+    out["timing"] = "CUDA graph replay per call, events on the launching stream"
     out["device_status"] = int(st.status.item())
     return out
 
 
 def _time_folded(st, F, torch, stream, l2_flush, args, dev):
     """Quantized adapters folded into the backbone GEMMs (not part of the
-    step): quantize B, the forward with T's columns, the dX GEMM with U's
-    columns and the dB / dA launch; A is frozen and quantized once, outside
-    the timing.  Eager calls timed with CUDA events on the launching stream,
-    L2 flushed before each rep."""
+    step): quantize B, the forward with T's columns, then the dX GEMM with
+    U's columns and the dB / dA launch; A is frozen and quantized once,
+    outside the timing."""
     aq, s_a, _ = F.falqon_quantize(st.A, dev_status=st.status)
     bq = torch.empty((st.N, st.r), dtype=torch.uint8, device=dev)
     s_b = torch.empty(1, dtype=torch.float32, device=dev)
@@ -581,29 +597,20 @@ def _time_folded(st, F, torch, stream, l2_flush, args, dev):
     dA, dB = torch.empty_like(st.dA), torch.empty_like(st.dB)
     names = ("quantB", "fwd_T", "bwd")
     reps = max(5, min(50, args.steps))
-    acc = dict.fromkeys(names, 0.0)
-    with torch.cuda.stream(stream):
-        for i in range(3 + reps):
-            l2_flush(i)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            ev[0].record()
-            F.falqon_quantize(st.B, codes=bq, scale=s_b, amax=amax, dev_status=st.status, workspace=ws_b)
-            ev[1].record()
-            F.falqon_linear_fwd_folded(st.xq, st.s_x, st.wq, st.s_w, aq, s_a, y=y, t_saved=t_saved,
-                                       dev_status=st.status)
-            ev[2].record()
-            F.falqon_linear_bwd_folded(st.dyq, st.s_dy, st.wq, st.s_w, bq, s_b, st.xq, st.s_x, t_saved, st.r,
-                                       dx=dx, dA=dA, dB=dB, dev_status=st.status, workspace=ws_u)
-            ev[3].record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                for j, n in enumerate(names):
-                    acc[n] += ev[j].elapsed_time(ev[j + 1])
-    out = {n: round(acc[n] / reps, 5) for n in names}
-    out["total"] = round(sum(out[n] for n in names), 5)
+    fns = [
+        lambda: F.falqon_quantize(st.B, codes=bq, scale=s_b, amax=amax, dev_status=st.status, workspace=ws_b),
+        lambda: F.falqon_linear_fwd_folded(st.xq, st.s_x, st.wq, st.s_w, aq, s_a, y=y, t_saved=t_saved,
+                                           dev_status=st.status),
+        lambda: F.falqon_linear_bwd_folded(st.dyq, st.s_dy, st.wq, st.s_w, bq, s_b, st.xq, st.s_x, t_saved,
+                                           st.r, dx=dx, dA=dA, dB=dB, dev_status=st.status, workspace=ws_u),
+    ]
+    ms = _graph_phase_times(torch, stream, l2_flush, fns, reps, not args.no_graph)
+    out = {n: round(t, 5) for n, t in zip(names, ms)}
+    out["total"] = round(sum(ms), 5)
     out["unit"] = "ms per call"
-    out["kernels"] = ("quantize_stream_kernel (B); tc_gemm_kernel with T columns; tc_gemm_kernel (dX) with U "
-                      "columns + skinny_kernel (dB^T with dA)")
+    out["timing"] = "CUDA graph replay per call, events on the launching stream"
+    out["kernels"] = ("amax_partial_kernel + quantize_cast_kernel (B); tc_gemm_kernel with T columns; "
+                      "tc_gemm_kernel (dX) with U columns + skinny_kernel (dB^T with dA)")
     out["device_status"] = int(st.status.item())
     return out
 
