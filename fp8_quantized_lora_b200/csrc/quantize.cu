@@ -294,10 +294,12 @@ __global__ void __launch_bounds__(kThreads)
 // into a ring of shared-memory slots with bulk asynchronous copies; sixteen
 // consumer warps read each slot, then release it.  Pass 1 reduces max|x|;
 // every CTA publishes its maximum in a marked workspace word and waits
-// (bounded) until all words are marked, reduces them, and pass 2 streams the
-// same run again -- it is still in L2 -- and writes the codes.
+// (bounded) until all words are marked, reduces them, and pass 2 writes the
+// codes: from the ring in place when the CTA's run fits it (up to 14 chunks:
+// a 4096 x 4096 bf16 tensor on 148 SMs), else streaming the run again (it is
+// still in L2).
 constexpr int kChunkBytes = 16384;
-constexpr int kStreamStages = 13;                      // 208 KB in flight per SM
+constexpr int kStreamStages = 14;                      // 224 KB in flight per SM
 constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
@@ -476,7 +478,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   const double s_d = static_cast<double>(s);
 
   // ---- pass 2: codes (and the optional residual)
-  stream([&](int64_t c, const uint8_t* slot) {
+  auto cast_chunk = [&](int64_t c, const uint8_t* slot) {
     const int64_t off = c * kChunkBytes;
     const int64_t valid = body_bytes - off < kChunkBytes ? body_bytes - off : kChunkBytes;
     const int64_t e0 = c * kPerChunk;  // first element of the chunk
@@ -520,7 +522,18 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         }
       }
     }
-  });
+  };
+  if (c_end - c_begin <= kStreamStages) {
+    // Resident run: pass 1 put chunk c_begin + i in slot i and nothing
+    // overwrote it, and every consumer thread waited on every slot's landing
+    // in pass 1, so the cast reads the slots in place instead of streaming
+    // the run from L2 again.
+    if (warp != 0 && !*abort_flag)
+      for (int64_t c = c_begin; c < c_end; ++c) cast_chunk(c, sm + (c - c_begin) * kChunkBytes);
+    __syncthreads();
+  } else {
+    stream(cast_chunk);
+  }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 32) {
     for (int64_t e = tail0; e < n; ++e) {
       float v;
