@@ -94,7 +94,9 @@ struct Cfg {
   static_assert(AccCols <= 512, "tensor memory");
 };
 
-template <class C>
+// kSeg2: the grid carries adapter tiles (a second B segment); the plain
+// backbone GEMMs are compiled without that code.
+template <class C, bool kSeg2>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const GemmArgs g) {
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (g.n_tiles0 < g.n_tiles) tma_prefetch_desc(&tmB2);
+    if (kSeg2) tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TmemCols);
@@ -156,7 +158,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
         const int nt = w % g.n_tiles;
         const int mt = w / g.n_tiles;
-        const bool seg2 = nt >= g.n_tiles0;  // an adapter tile
+        const bool seg2 = kSeg2 && nt >= g.n_tiles0;  // an adapter tile
         const CUtensorMap* tb = seg2 ? &tmB2 : &tmB;
         const int m0 = mt * C::TileM, n0 = (seg2 ? nt - g.n_tiles0 : nt) * C::BN;
         for (int kb = 0; kb < g.kb_total; ++kb) {
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       double den = sa;
       if (g.scale_b) den *= static_cast<double>(*g.scale_b);
       alpha = static_cast<float>(1.0 / den);
-      if (g.n_tiles0 < g.n_tiles) {
+      if (kSeg2) {
         double den2 = sa;
         if (g.scale_b2) den2 *= static_cast<double>(*g.scale_b2);
         alpha2 = static_cast<float>(1.0 / den2);
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       if (!warp_wait(&acc_full[acc], acc_phase, abort_flag)) { if (lane == 0) fail(); break; }
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * C::TileM + half * kBM + q * 32 + lane;
-      if (nt >= g.n_tiles0) {
+      if (kSeg2 && nt >= g.n_tiles0) {
         // adapter columns: rank i of token `row` goes to out2[i][row]; the 32
         // lanes of a warp hold 32 consecutive tokens, so each store is 64 bytes
         const int64_t i0 = static_cast<int64_t>(nt - g.n_tiles0) * C::BN;
@@ -347,7 +349,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 }
 
 // ---------------------------------------------------------------- host side
-template <class C>
+template <class C, bool kSeg2>
 cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const GemmArgs& g,
                         cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
@@ -355,7 +357,7 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
   static int configured_mask = 0;  // one bit per device ordinal < 31
   const int bit = di->device < 31 ? (1 << di->device) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C, kSeg2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SmemBytes);
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
@@ -363,7 +365,8 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
   const int total = g.m_tiles * g.n_tiles;
   const int slots = C::MinBlocks * di->sm_count;
   const int grid = total < slots ? total : slots;
-  return launch_pdl(tc_gemm_kernel<C>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2, g);
+  return launch_pdl(tc_gemm_kernel<C, kSeg2>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2,
+                    g);
 }
 
 // 128 x 256 tiles, 4-stage ring, double-buffered accumulator, one CTA per SM.
@@ -425,7 +428,8 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
   g.scale_b2 = s2.sb;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
-  return launch_gemm<C>(tA, tB, tB2, g, stream);
+  if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, g, stream);
+  return launch_gemm<C, false>(tA, tB, tB2, g, stream);
 }
 
 }  // namespace
