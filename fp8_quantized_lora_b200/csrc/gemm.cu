@@ -45,6 +45,11 @@ constexpr int kMmaBar = 1;  // named barrier between the MMA issuer and its wait
 
 struct GemmArgs {
   int32_t m_tiles, n_tiles, kb_total;
+  // Work items: items [0, n_full) are whole tiles (tile = item); the last
+  // n_half items are the 128-column halves of the tiles n_full ..
+  // n_full + n_half/2 - 1 (the partial last wave, split so that it takes
+  // about half as long).  total = n_full + n_half.
+  int32_t n_full, n_half;
   int32_t n_tiles0;        // tiles of the backbone segment; tiles nt >= n_tiles0 are the adapter's
   int64_t M, N;            // output extent of the backbone segment
   void* out;               // bf16 output, row-major [M][ldo]
@@ -84,6 +89,11 @@ struct Cfg {
   static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
   // A in E4M3 (kAFmt 0) or E5M2 (1; the dX GEMM of E5M2 gradients), B in E4M3
   static constexpr uint32_t IDesc = idesc_f32acc(static_cast<uint32_t>(kAFmt), 0u, 0u, kBMn ? 1u : 0u, kBM, kBN);
+  // a half tile: the first 128 columns of the B tile (one 128-byte block when MN-major)
+  static constexpr int HalfN = kRowBytes;
+  static constexpr uint32_t IDescHalf =
+      idesc_f32acc(static_cast<uint32_t>(kAFmt), 0u, 0u, kBMn ? 1u : 0u, kBM, HalfN);
+  static constexpr int HalfStageBytes = ABytes + BBytes / 2;
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
   static_assert(!kBMn || kBN % kRowBytes == 0, "MN-major B needs 128-byte blocks");
   static_assert(SmemBytes <= 232448, "shared memory per CTA");
@@ -99,7 +109,8 @@ struct Cfg {
 template <class C, bool kSeg2>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const GemmArgs g) {
+                   const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmBh,
+                   const GemmArgs g) {
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -114,7 +125,18 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int total = g.m_tiles * g.n_tiles;
+  const int total = g.n_full + g.n_half;
+  // work item -> (tile, column half): nh = -1 for a whole tile, else 0 or 1
+  auto item = [&](int w, int& mt, int& nt, int& nh) {
+    int t = w;
+    nh = -1;
+    if (w >= g.n_full) {
+      t = g.n_full + ((w - g.n_full) >> 1);
+      nh = (w - g.n_full) & 1;
+    }
+    nt = t % g.n_tiles;
+    mt = t / g.n_tiles;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::Stages; ++s) {
@@ -156,28 +178,30 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       uint32_t issued = 0, issued_parity = 0;  // per-stage: ever loaded / parity of last load
       bool ok = true;
       for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
-        const int nt = w % g.n_tiles;
-        const int mt = w / g.n_tiles;
+        int mt, nt, nh;
+        item(w, mt, nt, nh);
         const bool seg2 = kSeg2 && nt >= g.n_tiles0;  // an adapter tile
         const CUtensorMap* tb = seg2 ? &tmB2 : &tmB;
-        const int m0 = mt * C::TileM, n0 = (seg2 ? nt - g.n_tiles0 : nt) * C::BN;
+        const int m0 = mt * C::TileM;
+        const int n0 = (seg2 ? nt - g.n_tiles0 : nt) * C::BN + (nh > 0 ? C::HalfN : 0);
         for (int kb = 0; kb < g.kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { fail(); ok = false; break; }
           uint8_t* sA = smem + stage * C::StageBytes;
           uint8_t* sB = sA + C::ABytes;
-          mbar_arrive_expect_tx(&full[stage], C::StageBytes);
+          mbar_arrive_expect_tx(&full[stage], nh >= 0 ? C::HalfStageBytes : C::StageBytes);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
 #pragma unroll
           for (int h = 0; h < C::Halves; ++h)  // rows m0 + 128 h .., K block kb
             tma_load_2d(sA + h * C::AHalfBytes, &tmA, &full[stage], kb * C::BK, m0 + h * kBM);
           if constexpr (C::BMn) {
-            // B is [K][N] row-major: 128-byte column blocks of BK rows each
-#pragma unroll
-            for (int c = 0; c < C::BN / kRowBytes; ++c)
+            // B is [K][N] row-major: 128-byte column blocks of BK rows each (one for a half tile)
+            const int blocks = nh >= 0 ? 1 : C::BN / kRowBytes;
+            for (int c = 0; c < blocks; ++c)
               tma_load_2d(sB + c * C::BK * kRowBytes, tb, &full[stage], n0 + c * kRowBytes, kb * C::BK);
           } else {
-            tma_load_2d(sB, tb, &full[stage], kb * C::BK, n0);
+            // a half tile loads 128 rows of B through the half-height box
+            tma_load_2d(sB, nh >= 0 ? &tmBh : tb, &full[stage], kb * C::BK, n0);
           }
           if (++stage == C::Stages) { stage = 0; phase ^= 1; }
         }
@@ -199,6 +223,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
       if (bar_red_or(kMmaBar, 64, false)) break;
       tc_fence_after();
       const uint32_t tmem_d = tmem_base + acc * C::Halves * C::BN;
+      const uint32_t idesc = w >= g.n_full ? C::IDescHalf : C::IDesc;
       bool abort = false;
       for (int kb = 0; kb < g.kb_total; ++kb) {
         if (bar_red_or(kMmaBar, 64, false)) { abort = true; break; }
@@ -212,7 +237,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 #pragma unroll
             for (int h = 0; h < C::Halves; ++h)  // the halves share the B tile
               umma_f8(tmem_d + h * C::BN, operand_desc<false, 1, C::BK>(a_base + h * C::AHalfBytes, ks), bd,
-                      C::IDesc, (kb > 0 || ks > 0) ? 1u : 0u);
+                      idesc, (kb > 0 || ks > 0) ? 1u : 0u);
           }
           umma_commit(&empty[stage]);
         }
@@ -271,8 +296,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
-      const int nt = w % g.n_tiles;
-      const int mt = w / g.n_tiles;
+      int mt, nt, nh;
+      item(w, mt, nt, nh);
       if (!warp_wait(&acc_full[acc], acc_phase, abort_flag)) { if (lane == 0) fail(); break; }
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mt) * C::TileM + half * kBM + q * 32 + lane;
@@ -307,9 +332,10 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         if (++acc == C::Acc) { acc = 0; acc_phase ^= 1; }
         continue;
       }
-      const int64_t col_base = static_cast<int64_t>(nt) * C::BN;
+      const int64_t col_base = static_cast<int64_t>(nt) * C::BN + (nh > 0 ? C::HalfN : 0);
+      const int chunks = (nh >= 0 ? C::HalfN : C::BN) / 32;
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c) {
+      for (int c = 0; c < chunks; ++c) {
         uint32_t r[32];
         tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * C::Halves + half) * C::BN +
                            c * 32, r);
@@ -350,8 +376,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 
 // ---------------------------------------------------------------- host side
 template <class C, bool kSeg2>
-cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const GemmArgs& g,
-                        cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const CUtensorMap& tBh,
+                        GemmArgs g, cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
   static int configured_mask = 0;  // one bit per device ordinal < 31
@@ -362,11 +388,21 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  const int total = g.m_tiles * g.n_tiles;
+  const int tiles = g.m_tiles * g.n_tiles;
   const int slots = C::MinBlocks * di->sm_count;
-  const int grid = total < slots ? total : slots;
+  const int grid = tiles < slots ? tiles : slots;
+  // A partial last wave of at most half the grid's width runs as half tiles
+  // (twice as many items, each about half as long).  The adapter-tile
+  // launches keep whole tiles.
+  const int tail = tiles % grid;
+  g.n_full = tiles;
+  g.n_half = 0;
+  if (!kSeg2 && C::BN == 2 * C::HalfN && tiles > grid && tail > 0 && 2 * tail <= grid) {
+    g.n_full = tiles - tail;
+    g.n_half = 2 * tail;
+  }
   return launch_pdl(tc_gemm_kernel<C, kSeg2>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2,
-                    g);
+                    tBh, g);
 }
 
 // 128 x 256 tiles, 4-stage ring, double-buffered accumulator, one CTA per SM.
@@ -401,7 +437,7 @@ template <class C>
 cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
                      int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
                      cudaStream_t stream, const Segment2& s2 = Segment2{}) {
-  CUtensorMap tA, tB, tB2;
+  CUtensorMap tA, tB, tB2, tBh;
   // A [M, Kc] K-major
   if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a, Kc, M, 128, kBM, true))
     return cudaErrorInvalidValue;
@@ -410,6 +446,10 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
   if (s2.n > 0 && !b_tmap<C>(&tB2, s2.b, s2.n, Kc)) return cudaErrorInvalidValue;
   if (!seg1) tB = tB2;
   if (s2.n <= 0) tB2 = tB;
+  // K-major half tiles load 128 rows of B through a half-height box
+  tBh = tB;
+  if (!C::BMn && seg1 && !make_tmap_2d(&tBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::HalfN, true))
+    return cudaErrorInvalidValue;
   GemmArgs g{};
   g.m_tiles = ceil_div(M, C::TileM);
   g.n_tiles0 = seg1 ? ceil_div(Ncols, C::BN) : 0;
@@ -428,8 +468,8 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
   g.scale_b2 = s2.sb;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
-  if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, g, stream);
-  return launch_gemm<C, false>(tA, tB, tB2, g, stream);
+  if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, tBh, g, stream);
+  return launch_gemm<C, false>(tA, tB, tB2, tBh, g, stream);
 }
 
 }  // namespace

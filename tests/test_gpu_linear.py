@@ -66,6 +66,20 @@ def test_dx(cuda_device, M, N, K):
     _assert_close(_dx(dyq, s_dy, wq, s_w), O.linear_dx(dyq, s_dy, wq, s_w), (M, N, K))
 
 
+def test_partial_last_wave_runs_as_half_tiles(cuda_device):
+    """185 output tiles of 128 x 256 on 148 SMs: the 37 tiles of the last
+    wave run as 74 half tiles (128 x 128, N = 128 MMAs, half the B bytes).
+    Every output element is compared, the forward and dX both."""
+    O.set_threads(os.cpu_count() or 8)
+    M, N, K = 37 * 128, 5 * 256, 256
+    xq, s_x = _codes(811, (M, K))
+    wq, s_w = _codes(812, (N, K), 0.02)
+    _assert_close(_fwd(xq, s_x, wq, s_w), O.linear_fwd(xq, s_x, wq, s_w), "fwd")
+    dyq, s_dy = _codes(813, (M, K), 1e-3)  # dX [M, N]: contraction over K here
+    wq2, s_w2 = _codes(814, (K, N), 0.02)
+    _assert_close(_dx(dyq, s_dy, wq2, s_w2), O.linear_dx(dyq, s_dy, wq2, s_w2), "dx")
+
+
 def test_forward_identity_backbone_is_exact(cuda_device):
     M, K = 130, 256
     xq, s_x = _codes(7, (M, K))
