@@ -391,29 +391,59 @@ def run_gpu(args):
                 acc[n] += ev[j].elapsed_time(ev[j + 1])
     phase_ms = {n: acc[n] / reps for n in names}
 
-    # e2e through the C ABI with host buffers (pinned), copies inside the timed region
+    # e2e through the C ABI with host buffers (pinned), copies inside the timed
+    # region.  Inputs are copied in on one stream, the step runs on the compute
+    # stream, outputs are copied out on a third, with two slots of every
+    # buffer: the copies of neighbouring steps overlap the step and each other
+    # (the link is full duplex).  Events order each slot's reuse.
     hostX = [x.cpu().pin_memory() for x in st.X]
     hostdY = [x.cpu().pin_memory() for x in st.dY]
-    hostY = torch.empty(st.y.shape, dtype=torch.bfloat16).pin_memory()
-    hostdX = torch.empty(st.dx.shape, dtype=torch.bfloat16).pin_memory()
-    hostSel = torch.empty(1, dtype=torch.int32).pin_memory()
+    ys = [st.y, torch.empty_like(st.y)]
+    dxs = [st.dx, torch.empty_like(st.dx)]
+    hostY = [torch.empty(st.y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hostdX = [torch.empty(st.dx.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    hostSel = [torch.empty(1, dtype=torch.int32).pin_memory() for _ in range(2)]
+    sel = [torch.empty_like(st.n_sel) for _ in range(2)]  # each step's count, kept per slot
     e2e_steps = max(3, min(args.steps, 50))
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        e_start.record()
-        for i in range(e2e_steps):
-            st.X[i % 2].copy_(hostX[i % 2], non_blocking=True)
-            st.dY[i % 2].copy_(hostdY[i % 2], non_blocking=True)
-            st.phases(i % 2)
-            hostY.copy_(st.y, non_blocking=True)
-            hostdX.copy_(st.dx, non_blocking=True)
-            hostSel.copy_(st.n_sel, non_blocking=True)
-        e_end.record()
+    e_start.record(s_in)
+    stream.wait_event(e_start)
+    s_out.wait_event(e_start)
+    for i in range(e2e_steps):
+        k = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_done[i - 2])  # step i-2 no longer reads slot k's inputs
+            st.X[k].copy_(hostX[k], non_blocking=True)
+            st.dY[k].copy_(hostdY[k], non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])  # slot k's outputs of step i-2 copied out
+            st.y, st.dx = ys[k], dxs[k]
+            st.phases(k)
+            sel[k].copy_(st.n_sel)
+            ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            hostY[k].copy_(ys[k], non_blocking=True)
+            hostdX[k].copy_(dxs[k], non_blocking=True)
+            hostSel[k].copy_(sel[k], non_blocking=True)
+            ev_out[i].record(s_out)
+    s_out.wait_event(ev_done[e2e_steps - 1])
+    e_end.record(s_out)
     torch.cuda.synchronize()
+    st.y, st.dx = ys[0], dxs[0]
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     status = int(st.status.item())
     n_sel = int(st.n_sel.item())
@@ -478,7 +508,8 @@ def run_gpu(args):
         "roofline": roof,
         "phases": phases,
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+                "pipelining": "copy-in, step and copy-out on three streams, two buffer slots"},
         "gpu_launches": st.launches_per_step * args.steps,
         "clocks": clock_info,
         "device_status": status,
