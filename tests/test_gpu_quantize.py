@@ -116,3 +116,39 @@ def test_fp32_patterns_encode_like_the_oracle(cuda_device):
     codes, s, _, _, _ = _run(f)
     assert s == 1.0
     np.testing.assert_array_equal(codes, O.e4m3_encode(f))
+
+
+def test_every_fp32_pattern_up_to_448_encodes_like_the_oracle(cuda_device):
+    """Exhaustive: every float32 bit pattern from +0 to 448 (1.14e9 values),
+    quantized on the GPU in chunks that each hold 448 (so s = 1 exactly),
+    against the oracle's encoder; the negative patterns are checked by the
+    format's sign symmetry (the code of -x is the code of x with bit 7 set)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    top = 0x43E00000  # 448.0
+    chunk = 1 << 27
+    dev = torch.device("cuda:0")
+    st = status_word()
+    ws = torch.empty(F.falqon_workspace_size(F.OP_QUANTIZE, 1, chunk + 16), dtype=torch.uint8, device=dev)
+    pool = ThreadPoolExecutor(max_workers=16)
+
+    def oracle_codes(f):
+        parts = np.array_split(f, 16)
+        return np.concatenate(list(pool.map(O.e4m3_encode, parts)))
+
+    for lo in range(0, top + 1, chunk):
+        hi = min(top + 1, lo + chunk)
+        pats = np.arange(lo, hi, dtype=np.uint32)
+        n = len(pats) + 1
+        pad = (-n) % 16
+        f = np.concatenate([pats.view(np.float32), np.float32([448.0]), np.zeros(pad, np.float32)])
+        x = torch.from_numpy(f).to(dev)
+        codes, s, _ = F.falqon_quantize(x.view(-1, 16), dev_status=st, workspace=ws)
+        neg, s_neg, _ = F.falqon_quantize((-x).view(-1, 16), dev_status=st, workspace=ws)
+        torch.cuda.synchronize()
+        assert float(s.item()) == 1.0 and float(s_neg.item()) == 1.0
+        assert torch.equal(neg.view(-1)[: len(pats)], codes.view(-1)[: len(pats)] | 0x80), hex(lo)
+        np.testing.assert_array_equal(host(codes).reshape(-1)[: len(pats)], oracle_codes(pats.view(np.float32)),
+                                      err_msg=hex(lo))
+    pool.shutdown()
+    assert int(st.item()) == 0
