@@ -21,7 +21,7 @@ __all__ = [
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
     "falqon_linear_bwd_folded", "folded_t_planes", "OP_QUANTIZE", "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
-    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
+    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
@@ -30,7 +30,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfalqon.s
 OP_QUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_PROXY_UPDATE, OP_PROXY_UPDATE_TOPK = 0, 1, 2, 3, 4
 OP_FOLDED_T, OP_LINEAR_BWD_FOLDED = 5, 6
 DTYPE_BF16, DTYPE_F32 = 0, 1
-PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL = 1, 2, 4
+PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL, PROXY_STRICT = 1, 2, 4, 8
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
 

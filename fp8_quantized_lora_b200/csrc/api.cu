@@ -241,7 +241,8 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   int64_t r, uint32_t flags, uint8_t* row_mask,
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream) {
-  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL;
+  const uint32_t known =
+      FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL | FALQON_PROXY_STRICT;
   if ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
   if ((flags & FALQON_PROXY_KEEP_RESIDUAL) && !(flags & FALQON_PROXY_SELECT)) return FALQON_ERR_INVALID_ARG;
   if (!proxy || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
@@ -268,7 +269,7 @@ falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* pro
                                        int32_t* n_selected, int32_t* dev_status, void* workspace,
                                        size_t workspace_bytes, void* stream) {
   if (!wq || !s_w || !proxy || !dB_inc || !A) return FALQON_ERR_INVALID_ARG;
-  if (flags & ~FALQON_PROXY_KEEP_RESIDUAL) return FALQON_ERR_INVALID_ARG;
+  if (flags & ~(FALQON_PROXY_KEEP_RESIDUAL | FALQON_PROXY_STRICT)) return FALQON_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || r <= 0 || k < 0) return FALQON_ERR_INVALID_ARG;
   if (K % 16 != 0 || N > INT32_MAX) return FALQON_ERR_UNSUPPORTED;
   if (!aligned16(proxy) || !aligned16(wq)) return FALQON_ERR_UNSUPPORTED;

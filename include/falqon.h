@@ -82,6 +82,8 @@ typedef enum falqon_op {
 #define FALQON_PROXY_ACCUMULATE 1u /* P += dB_inc . A */
 #define FALQON_PROXY_SELECT 2u     /* select rows, requantize them, clear their proxy */
 #define FALQON_PROXY_KEEP_RESIDUAL 4u /* with SELECT (or top-k): keep the unapplied residual, no clear */
+#define FALQON_PROXY_STRICT 8u        /* accepted, changes nothing: the accumulation is always the
+                                         strict float32 FMA chain in index order, for every r */
 
 /*
  * falqon_quantize - per-tensor E4M3 quantization.
@@ -253,6 +255,8 @@ FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const floa
  *               sub-step residual): a code whose value changes keeps
  *               P = fl32(P - fl32(fl32(dec(c') - dec(old)) / s_W)); every
  *               other code keeps its proxy.  Row mask and count as SELECT.
+ *   STRICT:     accepted with the flags above and changes nothing: the
+ *               accumulation is always the strict float32 chain.
  * The float32 chain is reproduced bit-for-bit (no tensor cores).
  *
  *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);
@@ -289,7 +293,8 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
  *  wq, s_w, proxy, dB_inc, A: as in falqon_proxy_update (r >= 1).
  *  k >= 0: the largest number of rows to select (0: accumulate only).
  *  flags: 0, or FALQON_PROXY_KEEP_RESIDUAL (selected rows keep the residual
- *  instead of a cleared proxy; see falqon_proxy_update).
+ *  instead of a cleared proxy; see falqon_proxy_update), optionally with
+ *  FALQON_PROXY_STRICT.
  *  row_mask [N] uint8 (0/1) and n_selected (1 int32): nullable.
  *  workspace: falqon_workspace_size(FALQON_OP_PROXY_UPDATE_TOPK, 0, N, K, r)
  *  bytes (per-(row, 256-column block) counts, row scores, the selected list).

@@ -97,6 +97,12 @@ def test_proxy_argument_errors():
     # KEEP_RESIDUAL only together with SELECT
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 5, None, None, None, P, 1 << 20, None) == 1
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 4, None, None, None, P, 1 << 20, None) == 1
+    # STRICT is accepted with any valid combination (the K % 16 check fires next) ...
+    for flags in (1 | 8, 3 | 8, 7 | 8):
+        assert L.falqon_proxy_update(P, P, P, P, P, 4, 20, 2, flags, None, None, None, P, 1 << 20, None) == 2
+    # ... but not alone, and unknown bits are still rejected
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 8, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3 | 16, None, None, None, P, 1 << 20, None) == 1
 
 
 def test_proxy_topk_argument_errors():
@@ -111,6 +117,7 @@ def test_proxy_topk_argument_errors():
     assert f(P, P, P, P, P, 4, 16, 2, 1, 1, None, None, None, P, ws, None) == 1      # unknown flag
     assert f(P, P, P, P, P, 0, 16, 2, 1, 0, None, None, None, P, ws, None) == 1      # N = 0
     assert f(P, P, P, P, P, 4, 20, 2, 1, 4, None, None, None, P, ws, None) == 2      # K % 16
+    assert f(P, P, P, P, P, 4, 20, 2, 1, 4 | 8, None, None, None, P, ws, None) == 2  # STRICT accepted
     assert f(P, P, P8, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 2     # unaligned proxy
     assert f(P, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws - 256, None) == 3  # workspace
 
