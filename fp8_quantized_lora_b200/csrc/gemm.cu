@@ -16,7 +16,8 @@
 // their columns transposed, as a bf16 hi/lo pair [r][ld] (about 16
 // significant bits), the layout the dB / dA products read.
 //
-// Roles (persistent over 128 x 256 output tiles):
+// Roles (persistent over 128 x 256 output tiles; when the last wave would
+// leave at least half the SMs idle, its tiles run as 128 x 128 halves):
 //   warp 0      TMA producer (one lane): fills a `kStages`-deep smem ring.
 //   warp 1      TMEM owner and UMMA issuer (one lane issues).
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, bf16 store.
