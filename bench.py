@@ -224,10 +224,10 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # differs, the roofline's traffic is null.
 TRAFFIC = {
     "proxy": {
-        "bytes": 103531008,
+        "bytes": 104477440,
         "profile": "profiles/proxy_update_llama7b_attn_proj_4096_r64.md",
         "sources": {
-            "fp8_quantized_lora_b200/csrc/proxy.cu": "7f9871f1e86a9f2136e6bfcee8147affd9f32ed4e9e9df9d5da8e9ab7af18366",
+            "fp8_quantized_lora_b200/csrc/proxy.cu": "f798eb2ff5985b20869722ff6fd9fcf8cb464a0429bdf076147002a0fc2b8832",
             "fp8_quantized_lora_b200/csrc/ptx.cuh": "1ec40a2067b4ae4960ba3532651728a393a070d5a79f0c934e7e37f8439b9c2e",
             "fp8_quantized_lora_b200/csrc/internal.h": "f1af0da524732c61365588d5645c5a3c5bdd585f99131659048ed968374d86e0",
         },

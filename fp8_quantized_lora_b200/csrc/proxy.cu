@@ -40,9 +40,10 @@
 //   proxy_pipe_kernel / proxy_stream_kernel in count mode: P' written, and
 //     per (row, 256-column block) the number of changing codes; no code is
 //     written (a row with changes may not be among the k).
-//   proxy_topk_select_kernel (one CTA): row scores, the k-th score by
-//     bisection on the integer scores, ties taken in index order by a
-//     block-wide scan; row mask, count and the list of selected rows.
+//   proxy_topk_select_kernel (one CTA): row scores, the k-th score by a
+//     16-way search on the integer scores (15 thresholds per block
+//     reduction), ties taken in index order by a block-wide scan; row mask,
+//     count and the list of selected rows.
 //   proxy_topk_apply_kernel: requantizes the selected rows from P' (the same
 //     arithmetic as above) and clears their proxy.
 // Every step is reproduced bit-for-bit by the float32 arithmetic.
@@ -669,9 +670,19 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   const int tid = threadIdx.x;
   // scores, the largest score and the number of candidates (score > 0)
   int local_max = 0, local_cand = 0;
+  const bool vec = (ncb & 7) == 0;  // rows of 16-byte units (the buffer is 256-byte aligned)
   for (int64_t n = tid; n < N; n += kTopkThreads) {
     int sc = 0;
-    for (int c = 0; c < ncb; ++c) sc += rowcount[n * ncb + c];
+    if (vec) {
+      const uint4* q = reinterpret_cast<const uint4*>(rowcount + n * ncb);
+      for (int c = 0; c < ncb / 8; ++c) {
+        const uint4 u = q[c];
+        sc += static_cast<int>((u.x & 0xFFFFu) + (u.x >> 16) + (u.y & 0xFFFFu) + (u.y >> 16) +
+                               (u.z & 0xFFFFu) + (u.z >> 16) + (u.w & 0xFFFFu) + (u.w >> 16));
+      }
+    } else {
+      for (int c = 0; c < ncb; ++c) sc += rowcount[n * ncb + c];
+    }
     score[n] = sc;
     local_max = max(local_max, sc);
     local_cand += sc > 0 ? 1 : 0;
@@ -688,11 +699,51 @@ __global__ void __launch_bounds__(kTopkThreads, 1)
   };
   int tau = max_score + 1;  // kk == 0: nothing reaches it
   if (kk > 0) {
+    // 16-way search: kProbes thresholds split (lo, hi] per round, one block
+    // reduction of all their counts; count_at_least(lo) >= kk throughout
+    constexpr int kProbes = 15;
+    __shared__ int probe_red[kTopkThreads / 32][kProbes];
+    __shared__ int probe_tot[kProbes];
     int lo = 1, hi = max_score;
     while (lo < hi) {  // every thread takes the same branches
-      const int mid = lo + (hi - lo + 1) / 2;
-      if (count_at_least(mid) >= kk) lo = mid;
-      else hi = mid - 1;
+      const int64_t span = hi - lo;
+      int t[kProbes], c[kProbes];
+#pragma unroll
+      for (int j = 0; j < kProbes; ++j) {
+        t[j] = lo + static_cast<int>((span * (j + 1) + kProbes) / (kProbes + 1));  // in (lo, hi], rising
+        c[j] = 0;
+      }
+      for (int64_t n = tid; n < N; n += kTopkThreads) {
+        const int sc = score[n];
+#pragma unroll
+        for (int j = 0; j < kProbes; ++j) c[j] += sc >= t[j] ? 1 : 0;
+      }
+      const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+      for (int j = 0; j < kProbes; ++j) {
+        const int v = __reduce_add_sync(0xFFFFFFFFu, c[j]);
+        if (lane == 0) probe_red[warp][j] = v;
+      }
+      __syncthreads();
+      if (tid < kProbes) {
+        int tot = 0;
+        for (int w = 0; w < kTopkThreads / 32; ++w) tot += probe_red[w][tid];
+        probe_tot[tid] = tot;
+      }
+      __syncthreads();
+      int J = -1;
+#pragma unroll
+      for (int j = 0; j < kProbes; ++j)
+        if (probe_tot[j] >= kk) J = j;  // counts fall as t rises: the last such j
+      auto probe = [&](int j) { return lo + static_cast<int>((span * (j + 1) + kProbes) / (kProbes + 1)); };
+      if (J < 0) {
+        hi = probe(0) - 1;
+      } else {
+        const int new_lo = probe(J);
+        if (J + 1 < kProbes) hi = probe(J + 1) - 1;
+        lo = new_lo;
+      }
+      __syncthreads();  // probe_red / probe_tot are reused next round
     }
     tau = lo;
   }
