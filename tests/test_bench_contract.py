@@ -33,3 +33,45 @@ def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"],
                          cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_phase_work_matches_the_stated_algorithmic_work():
+    """The roofline numerators bench.py divides by the measured times: the
+    per-step work stated for each kernel, recomputed by hand for the
+    attention projection (M = N = K = 4096, r = 64) and a rank-16 layer."""
+    import types
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    st = types.SimpleNamespace(M=4096, N=4096, K=4096, r=64)
+    w = bench._phase_work(st)
+    M = N = K = 4096
+    assert w["fwd"]["flops"] == 2 * M * N * K == 137438953472
+    assert w["dX"]["flops"] == w["fwd"]["flops"]
+    assert w["fwd"]["bytes"] == M * K + N * K + 2 * M * N  # codes in, bf16 out
+    assert w["quantX"]["bytes"] == 3 * M * K  # bf16 in, codes out
+    assert w["quantdY"]["bytes"] == 3 * M * N
+    assert w["adapters"]["flops"] == 4 * M * 64 * (N + K)  # T, U, dB, dA
+    assert w["proxy"]["flops"] == 2 * N * K * 64  # r FMAs per element
+    assert w["proxy"]["bytes"] == 9 * N * K + 2 * 64 * (N + K)  # read P and Wq, write P; the adapters
+    # at r = 64 the FMA chain outlasts the 9 bytes per element; at r = 16 HBM bounds it
+    assert w["proxy"]["bound"] == "alu"
+    assert bench._phase_work(types.SimpleNamespace(M=4096, N=4096, K=4096, r=16))["proxy"]["bound"] == "hbm"
+    assert w["fwd"]["bound"] == w["dX"]["bound"] == "tensor" and w["quantX"]["bound"] == "hbm"
+
+
+def test_traffic_is_withheld_when_a_source_changes(tmp_path, monkeypatch):
+    """bench.py reports the captured DRAM traffic only while the kernel
+    sources hash as they did at the capture."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench._traffic("proxy") == bench.TRAFFIC["proxy"]["bytes"]  # the committed sources
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    for rel in bench.TRAFFIC["proxy"]["sources"]:
+        p = tmp_path / rel
+        p.parent.mkdir(parents=True, exist_ok=True)
+        p.write_text("changed")
+    assert bench._traffic("proxy") is None
+    assert bench._traffic("fwd") is None  # no capture recorded for it
