@@ -13,8 +13,9 @@
  * Conventions shared by every call
  * --------------------------------
  *  - All matrices are row-major and contiguous.  bfloat16 tensors are passed
- *    as `void*` holding IEEE bfloat16 values; E4M3 tensors as `uint8_t*`
- *    holding OCP E4M3 codes; scales as `float*` (one float, on the device).
+ *    as `void*` holding IEEE bfloat16 values; FP8 tensors as `uint8_t*`
+ *    holding OCP E4M3 codes (E5M2 codes where a call's name ends in _e5m2);
+ *    scales as `float*` (one float, on the device).
  *  - Every tensor pointer is a DEVICE pointer and must be 16-byte aligned.
  *    The caller owns every buffer; the library allocates no device memory.
  *  - `stream` is a cudaStream_t passed as `void*` (NULL = legacy default
@@ -75,7 +76,8 @@ typedef enum falqon_op {
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define FALQON_DEV_NONFINITE 1      /* amax of an input was NaN or infinite */
-#define FALQON_DEV_SCALE_OVERFLOW 2 /* 448/amax overflowed; the scale was clamped to FLT_MAX */
+#define FALQON_DEV_SCALE_OVERFLOW 2 /* fmax/amax overflowed (fmax 448 for E4M3, 57344 for E5M2);
+                                       the scale was clamped to FLT_MAX */
 #define FALQON_DEV_TIMEOUT 4        /* a bounded on-chip wait ran out; outputs are invalid */
 
 /* Flags of falqon_proxy_update. */
