@@ -19,7 +19,8 @@ __all__ = [
     "FalqonError", "lib", "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd",
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
-    "falqon_linear_bwd_folded", "folded_t_planes", "OP_QUANTIZE", "OP_LINEAR_FWD",
+    "falqon_linear_bwd_folded", "folded_t_planes", "falqon_selftest_bounded_waits", "OP_QUANTIZE",
+    "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
     "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = (
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
     "falqon_linear_bwd_e5m2", "falqon_linear_fwd_folded", "falqon_linear_bwd_folded",
+    "falqon_selftest_bounded_waits",
 )
 
 
@@ -72,6 +74,7 @@ def lib():
     L.falqon_proxy_update_topk.argtypes = [p, p, p, p, p, i64, i64, i64, i64, u32, p, p, p, p, sz, p]
     L.falqon_linear_bwd_noalloc.argtypes = [p, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, p, p, p]
     L.falqon_linear_fwd_folded.argtypes = [p, p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p, p]
+    L.falqon_selftest_bounded_waits.argtypes = [p, p, p, p]
     L.falqon_linear_bwd_folded.argtypes = [p, p, p, p, p, p, p, p, p, sz, i64, i64, i64, i64, p, p, p, p, p,
                                            sz, p]
     for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
@@ -324,3 +327,11 @@ def falqon_linear_bwd_folded(dyq, s_dy, wq, s_w, bq, s_b, xq, s_x, t_saved, r, d
         _ptr(dB_t), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
     _check(st, "falqon_linear_bwd_folded")
     return dx_t, dA_t, dB_t
+
+
+def falqon_selftest_bounded_waits(flag, dev_status, which, stream=None):
+    """Launches the library's self-test of its bounded waits (about one
+    second): see include/falqon.h."""
+    st = lib().falqon_selftest_bounded_waits(_ptr(flag), _ptr(dev_status), _ptr(which),
+                                             _stream(stream, flag.device))
+    _check(st, "falqon_selftest_bounded_waits")

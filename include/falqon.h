@@ -342,6 +342,26 @@ FALQON_API falqon_status falqon_linear_bwd_noalloc(const uint8_t* dyq, const flo
                                                    void* dA, void* dB, int32_t* dev_status,
                                                    void* stream);
 
+/*
+ * falqon_selftest_bounded_waits - exercises the failure detection on the GPU
+ * without a fault.
+ *
+ * Every wait inside the library's kernels is bounded (about one second of
+ * clock cycles); when it runs out, the kernel ORs FALQON_DEV_TIMEOUT into
+ * *dev_status and returns, and the context stays usable.  This call launches
+ * one small kernel whose waits cannot complete: an mbarrier wait (the kind
+ * the tcgen05 and quantize kernels use) on a phase nothing arrives on, and a
+ * bounded poll (the kind the quantize kernel's grid exchange uses) of *flag.
+ * Each wait that gives up sets FALQON_DEV_TIMEOUT and a bit in *which: 1 for
+ * the mbarrier wait (always), 2 for the poll (only while *flag stays 0).
+ * Takes about one second.
+ *
+ *  flag: 1 int32, device, read.  dev_status, which: 1 int32 each, device,
+ *  OR-ed into.
+ */
+FALQON_API falqon_status falqon_selftest_bounded_waits(const int32_t* flag, int32_t* dev_status,
+                                                       int32_t* which, void* stream);
+
 /* Workspace bytes `op` needs for these sizes (arguments an op ignores may be 0). */
 FALQON_API size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r);
 
