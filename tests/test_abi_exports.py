@@ -151,6 +151,14 @@ def test_folded_argument_errors():
     assert call(dA=P8) == 2                       # unaligned output
 
 
+def test_selftest_argument_errors():
+    L = F.lib()
+    f = L.falqon_selftest_bounded_waits
+    assert f(None, P, P, None) == 1
+    assert f(P, None, P, None) == 1
+    assert f(P, P, None, None) == 1
+
+
 @pytest.mark.parametrize("name", ["falqon_quantize", "falqon_linear_fwd"])
 def test_binding_refuses_cpu_tensors(name):
     import torch
