@@ -55,7 +55,8 @@ def lib():
         L.fo_adapter_da.argtypes = [p, p, p, C.c_float, i64, i64, i64, p]
         L.fo_proxy_accumulate.argtypes = [p, p, p, i64, i64, i64]
         L.fo_proxy_select.argtypes = [p, C.c_float, p, i64, i64, p, p]
-        L.fo_proxy_select_topk.argtypes = [p, C.c_float, p, i64, i64, i64, C.c_int, p, p]
+        L.fo_proxy_topk.restype = C.c_uint32
+        L.fo_proxy_topk.argtypes = [p, C.c_float, p, p, p, i64, i64, i64, i64, C.c_int, C.c_int, p, p, p]
         L.fo_proxy_select_residual.argtypes = [p, C.c_float, p, i64, i64, p, p]
         L.fo_set_threads.argtypes = [C.c_int]
         L.fo_get_threads.restype = C.c_int
@@ -305,23 +306,41 @@ def proxy_select_residual(wq: np.ndarray, s_w, P: np.ndarray):
     return wq, P, mask, int(cnt[0])
 
 
-def proxy_select_topk(wq: np.ndarray, s_w, P: np.ndarray, k: int, keep_residual: bool = False):
-    """C-13: returns (new wq, new P, mask, n_selected) with at most k rows
-    selected (highest number of changing codes, ties to the lower index);
-    keep_residual applies C-14 instead of C-11 to them."""
+def proxy_update_topk(wq, s_w, Q, dB_inc, A, k, accumulate=True, select=True):
+    """C-13: one update of the top-k proxy over the r rank components.
+
+    Q is float32 [r, N] (row i: the unmerged part of B's column i), dB_inc
+    bfloat16 bits [N, r] (read when accumulate), A bfloat16 bits [r, K].
+    Returns (new wq, new Q, component mask [r], number merged, status); the
+    inputs are not modified."""
     wq = np.array(wq, dtype=np.uint8, copy=True, order="C")
-    P = np.array(P, dtype=np.float32, copy=True, order="C")
+    Q = np.array(Q, dtype=np.float32, copy=True, order="C")
+    A = np.ascontiguousarray(A, dtype=np.uint16)
     N, K = wq.shape
-    mask = np.zeros(N, dtype=np.uint8)
+    r = A.shape[0]
+    assert Q.shape == (r, N), "Q must be [r, N]"
+    dBc = None if dB_inc is None else np.ascontiguousarray(dB_inc, dtype=np.uint16)
+    if accumulate:
+        assert dBc is not None and dBc.shape == (N, r)
+    mask = np.zeros(r, dtype=np.uint8)
     cnt = np.zeros(1, dtype=np.int32)
-    lib().fo_proxy_select_topk(_ptr(wq), C.c_float(float(s_w)), _ptr(P), N, K, int(k), int(bool(keep_residual)),
-                               _ptr(mask), _ptr(cnt))
-    return wq, P, mask, int(cnt[0])
+    st = lib().fo_proxy_topk(_ptr(wq), C.c_float(float(s_w)), _ptr(Q), _ptr(dBc), _ptr(A), N, K, r, int(k),
+                             int(bool(accumulate)), int(bool(select)), None, _ptr(mask), _ptr(cnt))
+    return wq, Q, mask, int(cnt[0]), int(st)
 
 
-def proxy_update_topk(wq, s_w, P, dB_inc, A, k, keep_residual=False):
-    """One proxy update with top-k row selection: accumulate (C-9), then C-13."""
-    return proxy_select_topk(wq, s_w, proxy_accumulate(P, dB_inc, A), k, keep_residual)
+def proxy_topk_scores(Q, A):
+    """C-13 scores of the r components of Q [r, N] with A [r, K] (float64),
+    and the status bits."""
+    Q = np.ascontiguousarray(Q, dtype=np.float32)
+    A = np.ascontiguousarray(A, dtype=np.uint16)
+    r, N = Q.shape
+    K = A.shape[1]
+    wq = np.zeros((N, K), dtype=np.uint8)
+    sc = np.zeros(r, dtype=np.float64)
+    st = lib().fo_proxy_topk(_ptr(wq), C.c_float(1.0), _ptr(Q), None, _ptr(A), N, K, r, 0, 0, 0, _ptr(sc),
+                             None, None)
+    return sc, int(st)
 
 
 def proxy_update(wq, s_w, P, dB_inc, A, accumulate=True, select=True, keep_residual=False):

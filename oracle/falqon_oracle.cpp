@@ -16,8 +16,8 @@
 //
 // Every decision the pages leave open is written here.
 //
-//  C-1  E4M3 codec.  [R2-W2] names E4M3 and says the scaled tensor is
-//       "rounded to FP8"; the bit layout is the OCP 8-bit floating point
+//  C-1  E4M3 codec.  [R2-W2] names E4M3 and has the scaled tensor
+//       rounded into that format; the bit layout is the OCP 8-bit floating point
 //       E4M3 definition: sign, 4 exponent bits (bias 7), 3 mantissa bits,
 //       no infinities, S.1111.111 is NaN, largest finite 448, smallest
 //       subnormal 2^-9.  Encoding rounds to the nearest finite value with
@@ -43,7 +43,7 @@
 //       path): Y[m,n] = sum_k dec(Xq[m,k]) dec(Wq[n,k]) / (s_X s_W), float64.
 //  C-6  dX on the same quantized backbone:
 //       dX[m,k] = sum_n dec(dYq[m,n]) dec(Wq[n,k]) / (s_dY s_W).
-//  C-7  Gradient of B ([R4-Q1]: it "can be pre-calculated" from A x):
+//  C-7  Gradient of B ([R4-Q1]: it can be computed ahead from A x):
 //       T[m,i]  = sum_k dec(Xq[m,k]) A[i,k] / s_X,
 //       dB[n,i] = sum_m dec(dYq[m,n]) T[m,i] / s_dY,
 //       all in float64, T kept exact (no rounding of the intermediate).
@@ -65,14 +65,15 @@
 //       index order starting from +0: acc = fma(dB_inc[n,i], A[i,k], acc);
 //       then P[n,k] = fl32(P[n,k] + D[n,k]).  dB_inc is the increment of B
 //       for this step (the caller folds in sign and learning rate).
-//  C-10 Row selection ([intro]: the proxy "selectively applies substantial
-//       weight updates", avoiding updates that vanish under low-bit
-//       quantization).  t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ) (no
+//  C-10 Row selection ([intro]: the proxy applies only the substantial
+//       weight updates and skips those that low-bit quantization would
+//       erase).  t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ) (no
 //       fused multiply-add), c' = enc(t); row n is selected iff some k has
 //       dec(c') != dec(Wq[n,k]) as values (so +0 equals -0, and a NaN code
 //       equals nothing).  s_W is the fixed scale of the initial
-//       quantization.  The pages' own rule is a top-k over rows ([R3-Q1],
-//       [R2-W7]) with k not given; the threshold rule here is the contract.
+//       quantization.  The pages' own rule is a top-k over the r rank
+//       components ([R3-Q1], [R2-W7]; C-13) with k not given; the threshold
+//       rule here is the contract of the step.
 //  C-11 Requantize and clear.  For mask[n] = 1: every code of the row whose
 //       value changes is replaced, Wq[n,k] = c'[n,k] where dec(c') != dec(Wq);
 //       codes whose value is unchanged keep their bit pattern (the only such
@@ -82,16 +83,34 @@
 //       definition), P keeps the accumulated value.  The pages say nothing
 //       about the sign of zero; keeping equal-valued codes as they are makes
 //       the decoded backbone identical to a verbatim rewrite.
-//  C-13 Top-k row selection (the pages' own rule: OpenReview rebuttal,
-//       reviewer 2, W7 -- the update is merged into the weight "using top-k
-//       row selection"; reviewer 3, Q1 -- it reduces the update from r to k,
-//       about 0.5% of the step).  The pages give neither the score nor k.
-//       Reading: a row's score is the number of its codes whose value C-10's
-//       c' would change; the selected rows are the k rows of highest
-//       positive score, ties going to the lower row index; a row of score 0
-//       is never selected (selecting it would only clear its proxy).  The
-//       selected rows then follow C-11; every other row keeps Wq bit-identical
-//       and its accumulated proxy, whatever its score.  k is the caller's.
+//  C-13 Top-k selection over the r rank components (the pages' own rule).
+//       [R3-Q1]: the top-k step runs over r rows, with r much smaller than
+//       the layer's dimension, and it shrinks the inner dimension of the
+//       weight update from r to k, which is what makes the update cheaper;
+//       [R2-W7]: the update is merged into the original weight by top-k row
+//       selection, which saves memory as well as update cost.  Neither the
+//       score nor k is printed.  Reading: the proxy of this rule is r rows,
+//       Q [r, N] float32, row i holding the part of B's column i (rank
+//       component i, whose update to the weight is the outer product
+//       Q[i,:]^T A[i,:]) not yet merged into the backbone; it starts at 0.
+//         accumulate: Q[i,n] = fl32( Q[i,n] + dB_inc[n,i] ).
+//         score:      score_i = max_n |Q[i,n]| * max_k |A[i,k]|, the largest
+//                     element of component i's update, as a float64 product
+//                     of two float32 magnitudes (exact); a component whose Q
+//                     or A row holds a non-finite value scores +infinity and
+//                     sets NONFINITE.
+//         select:     S = the k components of highest score, ties to the
+//                     lower index; a score of 0 is never selected.
+//         merge:      D[n,k] = float32 FMA chain over i in S in increasing
+//                     index order from +0, acc = fma(Q[i,n], A[i,k], acc);
+//                     t = fl32( dec(Wq[n,k]) + fl32(s_W * D[n,k]) ), c' = enc(t);
+//                     as in C-11, every code whose value changes takes c'
+//                     and every other code keeps its bits (no row is singled
+//                     out: the selection is over components).
+//         clear:      Q[i,:] = +0 for i in S; the part of the merged update
+//                     below a code step is dropped, as C-11 drops it.
+//       With S the whole set, D is C-9's chain of Q^T A, so merging every
+//       component reproduces C-9 .. C-11 applied to a proxy that starts at 0.
 //  C-14 Residual-keeping clear (error feedback; the variant of C-11 the
 //       pages leave open: C-11 drops the sub-step residual
 //       dec(old)/s_W + P - dec(c')/s_W).  In a selected row, a code whose
@@ -101,6 +120,8 @@
 //       division, one subtraction); a code whose value does not change keeps
 //       its bits and its proxy.  Under the threshold rule every row then
 //       follows the same formula (an unselected row has no changing code).
+//       The top-k rule of C-13 keeps no per-weight proxy, so it has no
+//       residual-keeping form.
 //  C-15 E5M2 gradients.  The rebuttal (reviewer 2, W2) names E5M2 beside
 //       E4M3 as an FP8 format under the same per-tensor scaling; the step
 //       can carry dY in it.  Format (OCP 8-bit FP): sign, 5 exponent bits
@@ -514,35 +535,64 @@ void fo_proxy_select_residual(uint8_t* wq, float s_w, float* P, int64_t N, int64
 }
 
 // ---------------------------------------------------------------- C-13
-void fo_proxy_select_topk(uint8_t* wq, float s_w, float* P, int64_t N, int64_t K, int64_t k_rows,
-                          int keep_residual, uint8_t* mask, int32_t* n_selected) {
-  // score of every row: how many of its codes C-10 would change in value
-  std::vector<int64_t> score(static_cast<size_t>(N), 0);
-  for (int64_t n = 0; n < N; ++n) {
-    for (int64_t k = 0; k < K; ++k) {
-      const float w = static_cast<float>(dec(wq[n * K + k]));
-      const float upd = s_w * P[n * K + k];
-      const float t = w + upd;
-      if (!(dec(enc(t)) == dec(wq[n * K + k]))) score[n] += 1;
-    }
+// Q [r, N] float32 in/out; dB_inc [N, r] bf16 (read when accumulate);
+// A [r, K] bf16; wq [N, K] in/out (written when select).  score_out [r],
+// comp_mask [r] and n_selected are optional.  Returns the status bits.
+uint32_t fo_proxy_topk(uint8_t* wq, float s_w, float* Q, const uint16_t* dB_inc, const uint16_t* A,
+                       int64_t N, int64_t K, int64_t r, int64_t k, int accumulate, int select,
+                       double* score_out, uint8_t* comp_mask, int32_t* n_selected) {
+  uint32_t status = 0;
+  if (accumulate) {
+    for (int64_t i = 0; i < r; ++i)
+      for (int64_t n = 0; n < N; ++n) Q[i * N + n] = Q[i * N + n] + bf16_to_f32(dB_inc[n * r + i]);
   }
-  // rows by decreasing score; a stable sort keeps equal scores in index order
-  std::vector<int64_t> order(static_cast<size_t>(N));
-  for (int64_t n = 0; n < N; ++n) order[n] = n;
+  std::vector<double> score(static_cast<size_t>(r), 0.0);
+  for (int64_t i = 0; i < r; ++i) {
+    bool nonfinite = false;
+    double mq = 0.0, ma = 0.0;
+    for (int64_t n = 0; n < N; ++n) {
+      const float v = Q[i * N + n];
+      if (!std::isfinite(v)) nonfinite = true;
+      else mq = std::max(mq, std::fabs(static_cast<double>(v)));
+    }
+    for (int64_t c = 0; c < K; ++c) {
+      const float a = bf16_to_f32(A[i * K + c]);
+      if (!std::isfinite(a)) nonfinite = true;
+      else ma = std::max(ma, std::fabs(static_cast<double>(a)));
+    }
+    if (nonfinite) status |= kNonfinite;
+    score[i] = nonfinite ? INFINITY : mq * ma;  // 24-bit by 8-bit significands: exact in float64
+    if (score_out) score_out[i] = score[i];
+  }
+  if (!select) return status;
+  // components by decreasing score; the stable sort keeps equal scores in index order
+  std::vector<int64_t> order(static_cast<size_t>(r));
+  for (int64_t i = 0; i < r; ++i) order[i] = i;
   std::stable_sort(order.begin(), order.end(), [&](int64_t a, int64_t b) { return score[a] > score[b]; });
-  std::vector<uint8_t> chosen(static_cast<size_t>(N), 0);
-  for (int64_t j = 0; j < N && j < k_rows; ++j)
-    if (score[order[j]] > 0) chosen[order[j]] = 1;
-  // C-11 (or C-14) on the chosen rows
-  int32_t count = 0;
+  std::vector<uint8_t> chosen(static_cast<size_t>(r), 0);
+  for (int64_t j = 0; j < r && j < k; ++j)
+    if (score[order[j]] > 0.0) chosen[order[j]] = 1;
+  std::vector<int64_t> S;
+  for (int64_t i = 0; i < r; ++i)
+    if (chosen[i]) S.push_back(i);
+  // merge the chosen components into the codes
+#pragma omp parallel for num_threads(g_threads) schedule(static)
   for (int64_t n = 0; n < N; ++n) {
-    if (chosen[n]) {
-      requantize_row(wq + n * K, s_w, P + n * K, K, keep_residual);
-      count += 1;
+    for (int64_t c = 0; c < K; ++c) {
+      float acc = 0.0f;
+      for (const int64_t i : S) acc = std::fmaf(Q[i * N + n], bf16_to_f32(A[i * K + c]), acc);
+      const double old_v = dec(wq[n * K + c]);
+      const float t = static_cast<float>(old_v) + s_w * acc;
+      const uint8_t c_new = enc(t);
+      if (!(dec(c_new) == old_v)) wq[n * K + c] = c_new;
     }
-    if (mask) mask[n] = chosen[n];
   }
-  if (n_selected) *n_selected = count;
+  for (const int64_t i : S)
+    for (int64_t n = 0; n < N; ++n) Q[i * N + n] = 0.0f;
+  if (comp_mask)
+    for (int64_t i = 0; i < r; ++i) comp_mask[i] = chosen[i];
+  if (n_selected) *n_selected = static_cast<int32_t>(S.size());
+  return status;
 }
 
 }  // extern "C"

@@ -58,16 +58,3 @@ def test_unchanged_codes_and_unselected_rows_keep_their_proxy():
     assert np.array_equal(P2[same].view(np.uint32), P[same].view(np.uint32))
     sel = mask.astype(bool)
     assert np.array_equal(wq2[~sel], wq[~sel])
-
-
-@pytest.mark.parametrize("k", [1, 9, 1000])
-def test_topk_with_residual(k):
-    wq, s_w, P = _state(33)
-    a = O.proxy_select_topk(wq, s_w, P, k, keep_residual=True)
-    b = O.proxy_select_topk(wq, s_w, P, k)
-    assert np.array_equal(a[0], b[0]) and np.array_equal(a[2], b[2]) and a[3] == b[3] > 0
-    sel = a[2].astype(bool)
-    assert np.array_equal(a[1][~sel].view(np.uint32), P[~sel].view(np.uint32))
-    # selected rows: exactly the residual rule's rows
-    c = O.proxy_select_residual(wq, s_w, P)
-    assert np.array_equal(a[1][sel].view(np.uint32), c[1][sel].view(np.uint32))
