@@ -217,22 +217,12 @@ class Step:
 # FP32 lanes x 2 flops x 1.965 GHz (the B200's boost clock)
 FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
-# DRAM traffic per call of a phase (dram__bytes_read.sum + dram__bytes_write.sum
+# DRAM traffic per call of a phase: dram__bytes_read.sum + dram__bytes_write.sum
 # of every kernel the call launches, from one ncu capture of the bench's own
-# workload; the command and the figures are in the named profile).  A figure
-# holds only for the kernel sources it was measured on: when a source's hash
+# workload (the capture command is stored beside the figure).  A figure holds
+# only for the kernel sources it was measured on: when a source's hash
 # differs, the roofline's traffic is null.
-TRAFFIC = {
-    "proxy": {
-        "bytes": 104477440,
-        "profile": "profiles/proxy_update_llama7b_attn_proj_4096_r64.md",
-        "sources": {
-            "fp8_quantized_lora_b200/csrc/proxy.cu": "f798eb2ff5985b20869722ff6fd9fcf8cb464a0429bdf076147002a0fc2b8832",
-            "fp8_quantized_lora_b200/csrc/ptx.cuh": "1ec40a2067b4ae4960ba3532651728a393a070d5a79f0c934e7e37f8439b9c2e",
-            "fp8_quantized_lora_b200/csrc/internal.h": "f1af0da524732c61365588d5645c5a3c5bdd585f99131659048ed968374d86e0",
-        },
-    },
-}
+TRAFFIC = {}
 
 
 def _traffic(phase):
@@ -494,7 +484,7 @@ def run_gpu(args):
                 "frac": phases[dom]["frac_hbm"], "peak_source": f"{peaks['source']} copy bandwidth"}
     roof["traffic"] = _traffic(dom)
     if roof["traffic"] is not None:
-        roof["traffic_source"] = TRAFFIC[dom]["profile"]
+        roof["traffic_capture"] = TRAFFIC[dom]["capture"]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
@@ -560,25 +550,29 @@ def _graph_phase_times(torch, stream, l2_flush, fns, reps, use_graph=True):
 
 
 def _time_topk(st, F, torch, stream, l2_flush, args, dev):
-    """The proxy update with top-k row selection (not part of the step), on
-    copies of the step's Wq and P with its last dB_inc."""
-    N, K = st.P.shape
-    wq, P = st.wq.clone(), st.P.clone()
-    mask = torch.empty(N, dtype=torch.uint8, device=dev)
+    """The top-k proxy update over the r rank components (not part of the
+    step): a proxy Q [r, N] holding the step's last dB_inc added to a copy of
+    the step's Wq, k components merged per call."""
+    N, K, r = st.N, st.K, st.r
+    k = min(args.topk, r)
+    wq = st.wq.clone()
+    Q = torch.zeros((r, N), dtype=torch.float32, device=dev)
+    mask = torch.empty(r, dtype=torch.uint8, device=dev)
     cnt = torch.zeros(1, dtype=torch.int32, device=dev)
-    wsz = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, N, K, st.r)
+    wsz = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, N, K, r)
     ws = torch.empty(max(wsz, 256), dtype=torch.uint8, device=dev)
     reps = max(5, min(50, args.steps))
 
     def call():
-        F.falqon_proxy_update_topk(wq, st.s_w, P, st.dB_inc, st.A, args.topk, row_mask=mask,
-                                   n_selected=cnt, dev_status=st.status, workspace=ws)
+        F.falqon_proxy_update_topk(wq, st.s_w, Q, st.dB_inc, st.A, k, comp_mask=mask, n_selected=cnt,
+                                   dev_status=st.status, workspace=ws)
     (ms,) = _graph_phase_times(torch, stream, l2_flush, [call], reps, not args.no_graph)
-    flops = 2.0 * N * K * st.r
-    return {"k": args.topk, "ms": round(ms, 5), "rows_selected": int(cnt.item()),
+    flops = 2.0 * N * K * k
+    nbytes = 2.0 * N * K + 8.0 * r * N + 2.0 * r * N + 2.0 * r * K  # Wq read + write, Q, dB_inc, A
+    return {"k": k, "r": r, "ms": round(ms, 5), "components_merged": int(cnt.item()),
             "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
-            "frac_fp32_fma_peak": round(flops / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS, 4),
-            "kernels": "proxy_pipe_kernel (count) + proxy_topk_select_kernel + proxy_topk_apply_kernel",
+            "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "kernels": "topk_accum_kernel + topk_select_kernel + topk_merge_kernel + topk_clear_kernel",
             "timing": "CUDA graph replay, events on the launching stream",
             "device_status": int(st.status.item())}
 
@@ -758,8 +752,8 @@ def main():
                     help="also time the folded quantized-adapter path (1) or skip it (0)")
     ap.add_argument("--e5m2", type=int, default=1,
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
-    ap.add_argument("--topk", type=int, default=256,
-                    help="also time the proxy update with top-k row selection at this k (0: skip)")
+    ap.add_argument("--topk", type=int, default=16,
+                    help="also time the top-k proxy update merging this many of the r components (0: skip)")
     ap.add_argument("--only", default=None, choices=list(Step.PHASES),
                     help="run one phase alone (warm-up + steps calls) and print no bench line; "
                          "for profiler captures")

@@ -228,22 +228,24 @@ def falqon_proxy_update(wq, s_w, proxy, dB_inc, A, flags=PROXY_ACCUMULATE | PROX
     return row_mask, n_selected
 
 
-def falqon_proxy_update_topk(wq, s_w, proxy, dB_inc, A, k, keep_residual=False, row_mask=None,
-                             n_selected=None, dev_status=None, workspace=None, stream=None):
-    """Proxy update with top-k row selection, in place on (wq, proxy);
-    returns (row_mask, n_selected)."""
-    N, K = proxy.shape
-    r = A.shape[0]
-    dev = proxy.device
-    row_mask = torch.empty(N, dtype=torch.uint8, device=dev) if row_mask is None else row_mask
-    n_selected = torch.empty(1, dtype=torch.int32, device=dev) if n_selected is None else n_selected
-    ws, wsb = _workspace(OP_PROXY_UPDATE_TOPK, 0, N, K, r, dev, workspace)
-    st = lib().falqon_proxy_update_topk(_ptr(_u8(wq)), _ptr(s_w), _ptr(proxy), _ptr(dB_inc), _ptr(A), N, K, r,
-                                        int(k), PROXY_KEEP_RESIDUAL if keep_residual else 0, _ptr(row_mask),
-                                        _ptr(n_selected), _ptr(dev_status), _ptr(ws),
-                                        wsb, _stream(stream, dev))
+def falqon_proxy_update_topk(wq, s_w, proxy_q, dB_inc, A, k, flags=PROXY_ACCUMULATE | PROXY_SELECT,
+                             comp_mask=None, n_selected=None, dev_status=None, workspace=None, stream=None):
+    """Top-k proxy update over the r rank components, in place on (wq, proxy_q);
+    proxy_q is float32 [r, N].  Returns (comp_mask, n_selected) (None, None
+    without PROXY_SELECT)."""
+    r, N = proxy_q.shape
+    K = wq.shape[1] if wq is not None else (A.shape[1] if A is not None else 0)
+    dev = proxy_q.device
+    ws, wsb = (None, 0)
+    if flags & PROXY_SELECT:
+        comp_mask = torch.empty(r, dtype=torch.uint8, device=dev) if comp_mask is None else comp_mask
+        n_selected = torch.empty(1, dtype=torch.int32, device=dev) if n_selected is None else n_selected
+        ws, wsb = _workspace(OP_PROXY_UPDATE_TOPK, 0, N, K, r, dev, workspace)
+    st = lib().falqon_proxy_update_topk(_ptr(None if wq is None else _u8(wq)), _ptr(s_w), _ptr(proxy_q),
+                                        _ptr(dB_inc), _ptr(A), N, K, r, int(k), int(flags), _ptr(comp_mask),
+                                        _ptr(n_selected), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
     _check(st, "falqon_proxy_update_topk")
-    return row_mask, n_selected
+    return comp_mask, n_selected
 
 
 def falqon_linear_bwd_noalloc(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=True,

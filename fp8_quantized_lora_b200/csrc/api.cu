@@ -105,8 +105,8 @@ size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int6
       if (N <= 0 || K <= 0) return 0;
       return proxy_workspace_bytes(N, K);
     case FALQON_OP_PROXY_UPDATE_TOPK:
-      if (N <= 0 || K <= 0) return 0;
-      return proxy_topk_workspace_bytes(N, K);
+      if (N <= 0 || K <= 0 || r <= 0) return 0;
+      return proxy_topk_workspace_bytes(N, K, r);
     case FALQON_OP_FOLDED_T:
     case FALQON_OP_LINEAR_BWD_FOLDED:
       if (M <= 0 || r <= 0) return 0;
@@ -263,20 +263,26 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                        static_cast<cudaStream_t>(stream)));
 }
 
-falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
+falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy_q,
                                        const void* dB_inc, const void* A, int64_t N, int64_t K,
-                                       int64_t r, int64_t k, uint32_t flags, uint8_t* row_mask,
+                                       int64_t r, int64_t k, uint32_t flags, uint8_t* comp_mask,
                                        int32_t* n_selected, int32_t* dev_status, void* workspace,
                                        size_t workspace_bytes, void* stream) {
-  if (!wq || !s_w || !proxy || !dB_inc || !A) return FALQON_ERR_INVALID_ARG;
-  if (flags & ~(FALQON_PROXY_KEEP_RESIDUAL | FALQON_PROXY_STRICT)) return FALQON_ERR_INVALID_ARG;
-  if (N <= 0 || K <= 0 || r <= 0 || k < 0) return FALQON_ERR_INVALID_ARG;
-  if (K % 16 != 0 || N > INT32_MAX) return FALQON_ERR_UNSUPPORTED;
-  if (!aligned16(proxy) || !aligned16(wq)) return FALQON_ERR_UNSUPPORTED;
-  falqon_status s = check_ws(proxy_topk_workspace_bytes(N, K), workspace, workspace_bytes);
-  if (s != FALQON_OK) return s;
+  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_STRICT;
+  if ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) == 0 || (flags & ~known))
+    return FALQON_ERR_INVALID_ARG;
+  if (!proxy_q || N <= 0 || K <= 0 || r <= 0 || k < 0) return FALQON_ERR_INVALID_ARG;
+  if ((flags & FALQON_PROXY_ACCUMULATE) && !dB_inc) return FALQON_ERR_INVALID_ARG;
+  const bool select = flags & FALQON_PROXY_SELECT;
+  if (select && (!wq || !s_w || !A)) return FALQON_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N > INT32_MAX || r > kTopkMaxRank) return FALQON_ERR_UNSUPPORTED;
+  if (select && (!aligned16(wq) || !aligned16(A))) return FALQON_ERR_UNSUPPORTED;
+  if (select) {
+    falqon_status s = check_ws(proxy_topk_workspace_bytes(N, K, r), workspace, workspace_bytes);
+    if (s != FALQON_OK) return s;
+  }
   if (!current_device_info()) return FALQON_ERR_CUDA;
-  return from_cuda(launch_proxy_update_topk(wq, s_w, proxy, dB_inc, A, N, K, r, k, flags, row_mask,
+  return from_cuda(launch_proxy_update_topk(wq, s_w, proxy_q, dB_inc, A, N, K, r, k, flags, comp_mask,
                                             n_selected, dev_status, workspace,
                                             static_cast<cudaStream_t>(stream)));
 }

@@ -117,10 +117,13 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
                                 const void* A, int64_t N, int64_t K, int64_t r, uint32_t flags,
                                 uint8_t* row_mask, int32_t* n_selected, int32_t* dev_status,
                                 void* workspace, cudaStream_t stream);
-size_t proxy_topk_workspace_bytes(int64_t N, int64_t K);
-cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
+// Top-k over the r rank components: Q [r, N] float32 (row i: the unmerged
+// part of B's column i).  flags: 1 accumulate, 2 select / merge / clear.
+constexpr int64_t kTopkMaxRank = 16384;  // the select kernel keeps r 8-byte keys in shared memory
+size_t proxy_topk_workspace_bytes(int64_t N, int64_t K, int64_t r);
+cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* Q, const void* dB_inc,
                                      const void* A, int64_t N, int64_t K, int64_t r, int64_t k,
-                                     uint32_t flags, uint8_t* row_mask, int32_t* n_selected,
+                                     uint32_t flags, uint8_t* comp_mask, int32_t* n_selected,
                                      int32_t* dev_status, void* workspace, cudaStream_t stream);
 
 }  // namespace falqon

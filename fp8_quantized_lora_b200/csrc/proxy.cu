@@ -31,34 +31,21 @@
 //   proxy_clear_kernel  (one warp per row)
 //     Selected rows get P = +0; writes the row mask and the selected count.
 //
-// Top-k row selection (the rebuttal's rule, OpenReview reviewer 2 W7 and
-// reviewer 3 Q1; score and k are not given there): a row's score is the
-// number of its codes whose value the requantization would change; the k rows
-// of highest positive score are selected, ties to the lower row index, and
-// get the selected-row treatment above; every other row keeps its codes and
-// its accumulated proxy.  Three launches:
-//   proxy_pipe_kernel / proxy_stream_kernel in count mode: P' written, and
-//     per (row, 256-column block) the number of changing codes; no code is
-//     written (a row with changes may not be among the k).
-//   proxy_topk_select_kernel (one CTA): row scores, the k-th score by a
-//     16-way search on the integer scores (15 thresholds per block
-//     reduction), ties taken in index order by a block-wide scan; row mask,
-//     count and the list of selected rows.
-//   proxy_topk_apply_kernel: requantizes the selected rows from P' (the same
-//     arithmetic as above) and clears their proxy.
 // Every step is reproduced bit-for-bit by the float32 arithmetic.
 #include <cuda_fp16.h>
 
+#include "codes.cuh"
 #include "internal.h"
 #include "ptx.cuh"
 
 namespace falqon {
 namespace {
 
+using namespace codes;
+
 // Selection mode of the accumulation kernels.
 constexpr int kModeNone = 0;    // accumulate only
 constexpr int kModeSelect = 1;  // threshold rule: changed codes written at once, per-block row flags
-constexpr int kModeCount = 2;   // top-k: per-(row, 256-column block) counts of changing codes, no code write
 
 constexpr int kThreads = 256;
 constexpr int kTileRows = 32;   // 4 row groups of kRT rows
@@ -72,83 +59,6 @@ constexpr int kBsBytes = kIChunk * kTileRows * 8;                  // (b, b) pai
 constexpr int kPBytes = kRT * kThreads * 16;                       // P slices       32 KB
 constexpr int kWBytes = kRT * kThreads * 4;                        // Wq slices       8 KB
 constexpr int kSmemBytes = kAsBytes + kBsBytes + kPBytes + kWBytes;  // 88 KB
-
-__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-
-// Values of the two codes in the low 16 bits of `c2` (hardware conversion via f16).
-__device__ __forceinline__ float2 e4m3x2_values(uint32_t c2) {
-  uint32_t h2;
-  const uint16_t c = static_cast<uint16_t>(c2);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
-  __half2 h;
-  memcpy(&h, &h2, 4);
-  return __half22float2(h);
-}
-
-// Four codes (bytes of w4) -> the four codes E4M3(dec(c) + s_w * p), no FMA.
-__device__ __forceinline__ uint32_t requantized4(uint32_t w4, float s_w, float4 p) {
-  const float2 d01 = e4m3x2_values(w4);
-  const float2 d23 = e4m3x2_values(w4 >> 16);
-  uint16_t lo, hi;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-      : "=h"(lo)
-      : "f"(__fadd_rn(d01.y, __fmul_rn(s_w, p.y))), "f"(__fadd_rn(d01.x, __fmul_rn(s_w, p.x))));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-      : "=h"(hi)
-      : "f"(__fadd_rn(d23.y, __fmul_rn(s_w, p.w))), "f"(__fadd_rn(d23.x, __fmul_rn(s_w, p.z))));
-  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-}
-
-// 0x80 in every byte of x that is zero, 0x00 elsewhere (exact per byte: the
-// masked add cannot carry across bytes).
-__device__ __forceinline__ uint32_t zero_bytes(uint32_t x) {
-  const uint32_t t = (x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu;  // bit 7 set iff the low 7 bits are not all 0
-  return ~(t | x) & 0x80808080u;
-}
-
-// 0xFF in every byte of `a` that holds a NaN code.
-__device__ __forceinline__ uint32_t nan_bytes(uint32_t a) {
-  const uint32_t mag = 0x7F7F7F7Fu;
-  return (zero_bytes((a & mag) ^ mag) >> 7) * 0xFFu;
-}
-
-// Byte mask (0xFF per byte) of the codes whose value changes from `a` to `b`.
-// Two codes hold the same value when they are identical non-NaN codes or
-// both zero (either sign); a NaN code never holds the same value.
-__device__ __forceinline__ uint32_t changed_bytes(uint32_t a, uint32_t b) {
-  const uint32_t mag = 0x7F7F7F7Fu;
-  const uint32_t same_bits = zero_bytes(a ^ b);
-  const uint32_t both_zero = zero_bytes((a | b) & mag);
-  const uint32_t nan = zero_bytes((a & mag) ^ mag) | zero_bytes((b & mag) ^ mag);
-  const uint32_t changed = ~((same_bits | both_zero) & ~nan) & 0x80808080u;
-  return (changed >> 7) * 0xFFu;
-}
 
 // Residual-keeping clear: for the codes in byte mask m (their value changes
 // from w_old to w_new) the proxy keeps what the new code does not apply,
@@ -174,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ int tile_flag[kTileRows];  // select: a code of the row changed; count: how many
+  __shared__ int tile_flag[kTileRows];  // a code of the row changed
   uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kIChunk][256]
   float2* Bs = reinterpret_cast<float2*>(sm + kAsBytes);                       // [kIChunk][32]
   float4* pbuf = reinterpret_cast<float4*>(sm + kAsBytes + kBsBytes);          // [kRT][256]
@@ -283,26 +193,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t cn = requantized4(w, s_w, p);
       const uint32_t m = changed_bytes(w, cn);
       if (m) {
-        if constexpr (kSel == kModeSelect) {
-          *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
-          tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
-          if (keep_residual) *reinterpret_cast<float4*>(proxy + n * K + col) = residual4(p, w, cn, m, s_w);
-        } else {
-          atomicAdd(&tile_flag[tr * kRT + j], __popc(m) >> 3);
-        }
+        *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (w & ~m);
+        tile_flag[tr * kRT + j] = 1;  // every writer stores the same value
+        if (keep_residual) *reinterpret_cast<float4*>(proxy + n * K + col) = residual4(p, w, cn, m, s_w);
       }
     }
   }
   if (kSel != kModeNone) {
-    // this tile's verdict (or count) for each of its rows, written in every case
+    // this tile's verdict for each of its rows, written in every case
     __syncthreads();
     const int64_t ncb = gridDim.x;
-    if (tid < kTileRows && r0 + tid < N) {
-      if (kSel == kModeSelect)
-        rowflag[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint8_t>(tile_flag[tid]);
-      else
-        reinterpret_cast<uint16_t*>(rowflag)[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint16_t>(tile_flag[tid]);
-    }
+    if (tid < kTileRows && r0 + tid < N) rowflag[(r0 + tid) * ncb + blockIdx.x] = static_cast<uint8_t>(tile_flag[tid]);
   }
   if (__any_sync(0xFFFFFFFFu, nonfinite) && (tid & 31) == 0 && dev_status)
     atomicOr(dev_status, kDevNonfinite);
@@ -477,7 +378,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     for (int j = 0; j < kPipeRT; ++j) {
       const int64_t n = r0 + tr * kPipeRT + j;  // the warp's row: uniform across the warp
       bool changed = false;
-      int nchanged = 0;
       if (col_ok && n < N) {
         float4 p0 = pst[(2 * j) * kPipeThreads + tid];
         float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
@@ -504,18 +404,14 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           // identical words change only where they hold NaN codes (the common case)
           const uint32_t m0 = c0 == w.x ? nan_bytes(w.x) : changed_bytes(w.x, c0);
           const uint32_t m1 = c1 == w.y ? nan_bytes(w.y) : changed_bytes(w.y, c1);
-          if constexpr (kSel == kModeSelect) {
-            if (m0 | m1) {
-              *reinterpret_cast<uint2*>(wq + n * K + col) =
-                  make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
-              changed = true;
-              if (keep_residual) {
-                dst[0] = residual4(p0, w.x, c0, m0, s_w);
-                dst[1] = residual4(p1, w.y, c1, m1, s_w);
-              }
+          if (m0 | m1) {
+            *reinterpret_cast<uint2*>(wq + n * K + col) =
+                make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
+            changed = true;
+            if (keep_residual) {
+              dst[0] = residual4(p0, w.x, c0, m0, s_w);
+              dst[1] = residual4(p1, w.y, c1, m1, s_w);
             }
-          } else {
-            nchanged = (__popc(m0) + __popc(m1)) >> 3;
           }
         }
       }
@@ -523,10 +419,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         // the tile's verdict for row n, written whether or not a code changed
         const bool any = __any_sync(0xFFFFFFFFu, changed);
         if (lane == 0 && n < N) rowflag[n * ncb + v / row_groups] = any ? 1 : 0;
-      } else if constexpr (kSel == kModeCount) {
-        // the number of the row's codes in this tile whose value would change
-        const int cnt = __reduce_add_sync(0xFFFFFFFFu, nchanged);
-        if (lane == 0 && n < N) reinterpret_cast<uint16_t*>(rowflag)[n * ncb + v / row_groups] = static_cast<uint16_t>(cnt);
       }
     }
     dbuf ^= 1;
@@ -613,212 +505,6 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
                     row_groups, units, ncb, rowflag, n_selected, dev_status, keep_residual);
 }
 
-constexpr int kTopkThreads = 512;
-
-// Block-wide helpers for the one-CTA selection (all threads call them).
-__device__ __forceinline__ int topk_block_sum(int v, int* red) {
-  v = __reduce_add_sync(0xFFFFFFFFu, v);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();  // red is free again
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int t = 0;
-  for (int w = 0; w < kTopkThreads / 32; ++w) t += red[w];
-  return t;
-}
-
-__device__ __forceinline__ int topk_block_max(int v, int* red) {
-  v = __reduce_max_sync(0xFFFFFFFFu, v);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int t = 0;
-  for (int w = 0; w < kTopkThreads / 32; ++w) t = max(t, red[w]);
-  return t;
-}
-
-// Exclusive prefix sum of `v` over the CTA in thread order; *total = the sum.
-__device__ __forceinline__ int topk_block_scan(int v, int* red, int* total) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int x = v;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int y = __shfl_up_sync(0xFFFFFFFFu, x, d);
-    if (lane >= d) x += y;
-  }
-  __syncthreads();
-  if (lane == 31) red[warp] = x;
-  __syncthreads();
-  int before = 0, all = 0;
-  for (int w = 0; w < kTopkThreads / 32; ++w) {
-    if (w < warp) before += red[w];
-    all += red[w];
-  }
-  *total = all;
-  return before + x - v;
-}
-
-__global__ void __launch_bounds__(kTopkThreads, 1)
-    proxy_topk_select_kernel(const uint16_t* __restrict__ rowcount, int64_t N, int ncb, int64_t k,
-                             int32_t* __restrict__ score, int32_t* __restrict__ sel_rows,
-                             int32_t* __restrict__ n_sel, uint8_t* __restrict__ row_mask,
-                             int32_t* __restrict__ n_selected) {
-  pdl_trigger();  // the next kernel may start launching; it waits for this one
-  pdl_wait();     // the previous kernel's results are complete and visible
-  __shared__ int red[kTopkThreads / 32];
-  const int tid = threadIdx.x;
-  // scores, the largest score and the number of candidates (score > 0)
-  int local_max = 0, local_cand = 0;
-  const bool vec = (ncb & 7) == 0;  // rows of 16-byte units (the buffer is 256-byte aligned)
-  for (int64_t n = tid; n < N; n += kTopkThreads) {
-    int sc = 0;
-    if (vec) {
-      const uint4* q = reinterpret_cast<const uint4*>(rowcount + n * ncb);
-      for (int c = 0; c < ncb / 8; ++c) {
-        const uint4 u = q[c];
-        sc += static_cast<int>((u.x & 0xFFFFu) + (u.x >> 16) + (u.y & 0xFFFFu) + (u.y >> 16) +
-                               (u.z & 0xFFFFu) + (u.z >> 16) + (u.w & 0xFFFFu) + (u.w >> 16));
-      }
-    } else {
-      for (int c = 0; c < ncb; ++c) sc += rowcount[n * ncb + c];
-    }
-    score[n] = sc;
-    local_max = max(local_max, sc);
-    local_cand += sc > 0 ? 1 : 0;
-  }
-  __syncthreads();  // the scores are visible to the whole CTA
-  const int max_score = topk_block_max(local_max, red);
-  const int64_t cand = topk_block_sum(local_cand, red);
-  const int64_t kk = k < cand ? k : cand;  // rows that will be selected
-  // tau: the largest score with at least kk rows scoring tau or more
-  auto count_at_least = [&](int t) {
-    int c = 0;
-    for (int64_t n = tid; n < N; n += kTopkThreads) c += score[n] >= t ? 1 : 0;
-    return topk_block_sum(c, red);
-  };
-  int tau = max_score + 1;  // kk == 0: nothing reaches it
-  if (kk > 0) {
-    // 16-way search: kProbes thresholds split (lo, hi] per round, one block
-    // reduction of all their counts; count_at_least(lo) >= kk throughout
-    constexpr int kProbes = 15;
-    __shared__ int probe_red[kTopkThreads / 32][kProbes];
-    __shared__ int probe_tot[kProbes];
-    int lo = 1, hi = max_score;
-    while (lo < hi) {  // every thread takes the same branches
-      const int64_t span = hi - lo;
-      int t[kProbes], c[kProbes];
-#pragma unroll
-      for (int j = 0; j < kProbes; ++j) {
-        t[j] = lo + static_cast<int>((span * (j + 1) + kProbes) / (kProbes + 1));  // in (lo, hi], rising
-        c[j] = 0;
-      }
-      for (int64_t n = tid; n < N; n += kTopkThreads) {
-        const int sc = score[n];
-#pragma unroll
-        for (int j = 0; j < kProbes; ++j) c[j] += sc >= t[j] ? 1 : 0;
-      }
-      const int warp = tid >> 5, lane = tid & 31;
-#pragma unroll
-      for (int j = 0; j < kProbes; ++j) {
-        const int v = __reduce_add_sync(0xFFFFFFFFu, c[j]);
-        if (lane == 0) probe_red[warp][j] = v;
-      }
-      __syncthreads();
-      if (tid < kProbes) {
-        int tot = 0;
-        for (int w = 0; w < kTopkThreads / 32; ++w) tot += probe_red[w][tid];
-        probe_tot[tid] = tot;
-      }
-      __syncthreads();
-      int J = -1;
-#pragma unroll
-      for (int j = 0; j < kProbes; ++j)
-        if (probe_tot[j] >= kk) J = j;  // counts fall as t rises: the last such j
-      auto probe = [&](int j) { return lo + static_cast<int>((span * (j + 1) + kProbes) / (kProbes + 1)); };
-      if (J < 0) {
-        hi = probe(0) - 1;
-      } else {
-        const int new_lo = probe(J);
-        if (J + 1 < kProbes) hi = probe(J + 1) - 1;
-        lo = new_lo;
-      }
-      __syncthreads();  // probe_red / probe_tot are reused next round
-    }
-    tau = lo;
-  }
-  const int64_t need = kk > 0 ? kk - count_at_least(tau + 1) : 0;  // ties at tau to take, in index order
-  // walk the rows in index order
-  int64_t ties_before = 0, out = 0;
-  for (int64_t base = 0; base < N; base += kTopkThreads) {
-    const int64_t n = base + tid;
-    const int sc = n < N ? score[n] : -1;
-    const int tie = (kk > 0 && sc == tau) ? 1 : 0;
-    int tie_total = 0;
-    const int64_t tie_rank = ties_before + topk_block_scan(tie, red, &tie_total);
-    const int chosen = (kk > 0 && sc > tau) || (tie && tie_rank < need) ? 1 : 0;
-    int chosen_total = 0;
-    const int64_t pos = out + topk_block_scan(chosen, red, &chosen_total);
-    if (n < N) {
-      if (row_mask) row_mask[n] = static_cast<uint8_t>(chosen);
-      if (chosen) sel_rows[pos] = static_cast<int32_t>(n);
-    }
-    ties_before += tie_total;
-    out += chosen_total;
-  }
-  if (tid == 0) {
-    *n_sel = static_cast<int32_t>(out);
-    if (n_selected) *n_selected = static_cast<int32_t>(out);
-  }
-}
-
-// Selected rows: every code whose value changes takes E4M3(dec(c) + s_w * P'),
-// and P' = +0.  Grid-stride over the list the selection kernel wrote.
-__global__ void __launch_bounds__(kClearThreads)
-    proxy_topk_apply_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
-                            float* __restrict__ proxy, int64_t K, const int32_t* __restrict__ sel_rows,
-                            const int32_t* __restrict__ n_sel, int keep_residual) {
-  pdl_trigger();  // the next kernel may start launching; it waits for this one
-  pdl_wait();     // the previous kernel's results are complete and visible
-  const int64_t ns = *n_sel;
-  const float s_w = *s_w_ptr;
-  for (int64_t j = blockIdx.x; j < ns; j += gridDim.x) {
-    const int64_t n = sel_rows[j];
-    for (int64_t c = 4 * static_cast<int64_t>(threadIdx.x); c < K; c += 4 * kClearThreads) {
-      uint32_t* wp = reinterpret_cast<uint32_t*>(wq + n * K + c);
-      float4* pp = reinterpret_cast<float4*>(proxy + n * K + c);
-      const uint32_t w = *wp;
-      const float4 p = *pp;
-      const uint32_t cn = requantized4(w, s_w, p);
-      const uint32_t m = cn == w ? nan_bytes(w) : changed_bytes(w, cn);
-      if (m) *wp = (cn & m) | (w & ~m);
-      *pp = keep_residual ? residual4(p, w, cn, m, s_w) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
-  }
-}
-
-struct TopkWorkspace {
-  uint16_t* rowcount;  // [N][ncb]
-  int32_t* score;      // [N]
-  int32_t* sel_rows;   // [N]
-  int32_t* n_sel;      // [1]
-};
-
-TopkWorkspace topk_layout(void* ws, int64_t N, int64_t ncb, size_t* bytes) {
-  const size_t a = align_up(static_cast<size_t>(N) * static_cast<size_t>(ncb) * 2, 256);
-  const size_t b = align_up(static_cast<size_t>(N) * 4, 256);
-  TopkWorkspace t{};
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  if (p) {
-    t.rowcount = reinterpret_cast<uint16_t*>(p);
-    t.score = reinterpret_cast<int32_t*>(p + a);
-    t.sel_rows = reinterpret_cast<int32_t*>(p + a + b);
-    t.n_sel = reinterpret_cast<int32_t*>(p + a + 2 * b);
-  }
-  if (bytes) *bytes = a + 2 * b + 256;
-  return t;
-}
-
 }  // namespace
 
 size_t proxy_workspace_bytes(int64_t N, int64_t K) {
@@ -875,57 +561,6 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
                                                                               : static_cast<int64_t>(di->sm_count) * 8;
   return launch_pdl(proxy_clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
                     proxy, N, K, ncb, rowflag, row_mask, n_selected, keep_res ? 0 : 1);
-}
-
-size_t proxy_topk_workspace_bytes(int64_t N, int64_t K) {
-  size_t bytes = 0;
-  topk_layout(nullptr, N, (K + kTileCols - 1) / kTileCols, &bytes);
-  return bytes;
-}
-
-cudaError_t launch_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
-                                     const void* A, int64_t N, int64_t K, int64_t r, int64_t k,
-                                     uint32_t flags, uint8_t* row_mask, int32_t* n_selected,
-                                     int32_t* dev_status, void* workspace, cudaStream_t stream) {
-  const int keep_res = (flags & 4u) ? 1 : 0;  // residual-keeping clear instead of P = +0
-  const DeviceInfo* di = current_device_info();
-  if (!di) return cudaErrorInvalidDevice;
-  if (r < 1 || r > (int64_t(1) << 30) || N > (int64_t(1) << 31) - 1) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
-                  static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
-  const int rr = static_cast<int>(r);
-  const int ncb = static_cast<int>(grid.x);
-  const TopkWorkspace t = topk_layout(workspace, N, ncb, nullptr);
-  uint8_t* counts = reinterpret_cast<uint8_t*>(t.rowcount);
-  const int64_t row_groups = (N + kPipeRows - 1) / kPipeRows;
-  const int64_t units = row_groups * grid.x;
-  const bool pipe = rr <= kPipeRMax && rr % 8 == 0 && units <= (int64_t(1) << 30) &&
-                    di->max_smem_optin >= kPipeSmemBytes;
-  if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
-  cudaError_t e;
-  // 1. P' and the per-(row, column block) counts of changing codes
-  if (pipe) {
-    const int64_t resident = 2 * static_cast<int64_t>(di->sm_count);
-    const int g = static_cast<int>(units < resident ? units : resident);
-    e = launch_pipe<kModeCount>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, static_cast<int>(row_groups),
-                                static_cast<int>(units), ncb, counts, nullptr, dev_status, 0, stream);
-  } else {
-    e = launch_stream<true, kModeCount>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, counts, nullptr,
-                                        dev_status, 0, stream);
-  }
-  if (e != cudaSuccess) return e;
-  // 2. the k rows
-  e = launch_pdl(proxy_topk_select_kernel, dim3(1), dim3(kTopkThreads), 0, stream, 1u,
-                 static_cast<const uint16_t*>(t.rowcount), N, ncb, k, t.score, t.sel_rows, t.n_sel, row_mask,
-                 n_selected);
-  if (e != cudaSuccess) return e;
-  // 3. requantize and clear them
-  const int64_t cap = static_cast<int64_t>(di->sm_count) * 8;
-  const int64_t kmax = k < N ? k : N;
-  const int64_t blocks = kmax < 1 ? 1 : (kmax < cap ? kmax : cap);
-  return launch_pdl(proxy_topk_apply_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
-                    wq, s_w, proxy, K, static_cast<const int32_t*>(t.sel_rows), static_cast<const int32_t*>(t.n_sel),
-                    keep_res);
 }
 
 }  // namespace falqon

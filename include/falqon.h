@@ -83,7 +83,7 @@ typedef enum falqon_op {
 /* Flags of falqon_proxy_update. */
 #define FALQON_PROXY_ACCUMULATE 1u /* P += dB_inc . A */
 #define FALQON_PROXY_SELECT 2u     /* select rows, requantize them, clear their proxy */
-#define FALQON_PROXY_KEEP_RESIDUAL 4u /* with SELECT (or top-k): keep the unapplied residual, no clear */
+#define FALQON_PROXY_KEEP_RESIDUAL 4u /* with SELECT: keep the unapplied residual, no clear */
 #define FALQON_PROXY_STRICT 8u        /* accepted, changes nothing: the accumulation is always the
                                          strict float32 FMA chain in index order, for every r */
 
@@ -242,7 +242,8 @@ FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const floa
  * The abstract and introduction: a row-wise proxy accumulates the adapter
  * updates and selectively applies substantial ones to the FP8 backbone,
  * skipping updates that would vanish under quantization.  This library's
- * rule (the pages' own rule is a top-k over rows with k not given):
+ * rule (the pages' own rule, a top-k over the r rank components with k not
+ * given, is falqon_proxy_update_topk):
  *   ACCUMULATE: D[n,k] = float32 FMA chain over i = 0..r-1 of
  *               dB_inc[n,i] * A[i,k], starting at +0; P = fl32(P + D).
  *   SELECT:     t = fl32( dec(Wq[n,k]) + fl32(s_W * P[n,k]) ), c' = E4M3(t);
@@ -277,36 +278,51 @@ FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, floa
                                   size_t workspace_bytes, void* stream);
 
 /*
- * falqon_proxy_update_topk - row-wise proxy update with top-k row selection.
+ * falqon_proxy_update_topk - proxy update with top-k selection over the r
+ * rank components of the adapter.
  *
- * The rebuttal's own rule (OpenReview reviewer 2, W7: the update is merged
- * into the weight "using top-k row selection"; reviewer 3, Q1: it costs about
- * 0.5% of the step and reduces the update from r to k).  The pages give
- * neither the score nor k; this library's reading:
- *   ACCUMULATE as in falqon_proxy_update (the same float32 FMA chain).
- *   score[n] = number of k with dec(c'[n,k]) != dec(Wq[n,k]), c' as in
- *              falqon_proxy_update's SELECT.
- *   The selected rows are the k rows of highest positive score; ties go to
- *   the lower row index; a row of score 0 is never selected.  Selected rows
- *   are requantized and cleared exactly as in falqon_proxy_update; every
- *   other row keeps Wq bit-identical and its accumulated proxy (so with
- *   k >= N the result equals falqon_proxy_update with both flags).
+ * The OpenReview rebuttal (reviewer 3, Q1) has the top-k step run over r
+ * rows, r much smaller than the layer dimension, and shrink the inner
+ * dimension of the weight update from r to k; the rebuttal to reviewer 2
+ * (W7) has the update merged into the weight by that selection, saving
+ * memory and update cost.  Neither the score nor k is printed.  This
+ * library's reading: the proxy of this rule is Q [r, N] float32, row i
+ * holding the part of B's column i (rank component i, whose update to the
+ * weight is Q[i,:]^T A[i,:]) not yet merged into the backbone.
+ *   ACCUMULATE: Q[i,n] = fl32( Q[i,n] + dB_inc[n,i] ).
+ *   SELECT:     score_i = max_n |Q[i,n]| * max_k |A[i,k]| (exact, float64);
+ *               a component whose Q or A row holds a non-finite value
+ *               scores +infinity and sets FALQON_DEV_NONFINITE.  The chosen
+ *               set S is the k components of highest positive score, ties
+ *               to the lower index.  Merge: D[n,k] = float32 FMA chain over
+ *               i in S in increasing order from +0 of Q[i,n] * A[i,k];
+ *               t = fl32( dec(Wq[n,k]) + fl32(s_W * D[n,k]) ); every code
+ *               whose value changes becomes E4M3(t), the others keep their
+ *               bits.  Clear: Q[i,:] = +0 for i in S.
+ *   STRICT:     accepted, changes nothing.
+ * Merging every component equals falqon_proxy_update (both flags) applied
+ * to a proxy P = 0 with dB_inc = Q^T: the whole r-term update.  The cost is
+ * 2 N K |S| flops and one pass over Wq; no per-weight proxy exists.
  *
- *  wq, s_w, proxy, dB_inc, A: as in falqon_proxy_update (r >= 1).
- *  k >= 0: the largest number of rows to select (0: accumulate only).
- *  flags: 0, or FALQON_PROXY_KEEP_RESIDUAL (selected rows keep the residual
- *  instead of a cleared proxy; see falqon_proxy_update), optionally with
- *  FALQON_PROXY_STRICT.
- *  row_mask [N] uint8 (0/1) and n_selected (1 int32): nullable.
+ *  wq [N, K] E4M3, in/out (read and written when SELECT); s_w 1 float.
+ *  proxy_q [r, N] float32, in/out.
+ *  dB_inc [N, r] bfloat16 (the increment of B this step; read when
+ *  ACCUMULATE).  A [r, K] bfloat16 (read when SELECT).
+ *  k >= 0: the largest number of components to merge.
+ *  comp_mask [r] uint8 (0/1) and n_selected (1 int32): written when SELECT;
+ *  nullable.
+ *  flags: ACCUMULATE and/or SELECT, optionally STRICT; KEEP_RESIDUAL is
+ *  rejected (FALQON_ERR_INVALID_ARG): this rule keeps no per-weight proxy.
  *  workspace: falqon_workspace_size(FALQON_OP_PROXY_UPDATE_TOPK, 0, N, K, r)
- *  bytes (per-(row, 256-column block) counts, row scores, the selected list).
- *  Requirements: N >= 1 and below 2^31; K multiple of 16; r >= 1; k >= 0.
- *  Three launches (accumulate and count, select, requantize), all on
- *  `stream`; nothing is synchronised with the host.
+ *  bytes when SELECT (per-CTA maxima, the chosen list).
+ *  Requirements: N >= 1 and below 2^31; K a multiple of 16; 1 <= r <= 16384
+ *  (FALQON_ERR_UNSUPPORTED beyond); k >= 0.
+ *  Launches: one with ACCUMULATE alone; with SELECT four (maxima, choice,
+ *  merge, clear), two when k == 0; nothing is synchronised with the host.
  */
-FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy,
+FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w, float* proxy_q,
                                        const void* dB_inc, const void* A, int64_t N, int64_t K,
-                                       int64_t r, int64_t k, uint32_t flags, uint8_t* row_mask,
+                                       int64_t r, int64_t k, uint32_t flags, uint8_t* comp_mask,
                                        int32_t* n_selected, int32_t* dev_status, void* workspace,
                                        size_t workspace_bytes, void* stream);
 

@@ -109,17 +109,25 @@ def test_proxy_topk_argument_errors():
     L = F.lib()
     ws = F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, 4, 16, 2)
     assert ws >= 256 and ws % 256 == 0
+    assert F.falqon_workspace_size(F.OP_PROXY_UPDATE_TOPK, 0, 4, 16, 0) == 0
     f = L.falqon_proxy_update_topk
-    assert f(None, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 1   # no codes
-    assert f(P, P, P, None, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 1   # no increment
-    assert f(P, P, P, P, P, 4, 16, 0, 1, 0, None, None, None, P, ws, None) == 1      # r = 0
-    assert f(P, P, P, P, P, 4, 16, 2, -1, 0, None, None, None, P, ws, None) == 1     # k < 0
-    assert f(P, P, P, P, P, 4, 16, 2, 1, 1, None, None, None, P, ws, None) == 1      # unknown flag
-    assert f(P, P, P, P, P, 0, 16, 2, 1, 0, None, None, None, P, ws, None) == 1      # N = 0
-    assert f(P, P, P, P, P, 4, 20, 2, 1, 4, None, None, None, P, ws, None) == 2      # K % 16
-    assert f(P, P, P, P, P, 4, 20, 2, 1, 4 | 8, None, None, None, P, ws, None) == 2  # STRICT accepted
-    assert f(P, P, P8, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 2     # unaligned proxy
-    assert f(P, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws - 256, None) == 3  # workspace
+    AS = 1 | 2  # ACCUMULATE | SELECT
+    assert f(None, P, P, P, P, 4, 16, 2, 1, AS, None, None, None, P, ws, None) == 1  # no codes
+    assert f(P, P, P, None, P, 4, 16, 2, 1, AS, None, None, None, P, ws, None) == 1  # no increment
+    assert f(P, P, P, P, None, 4, 16, 2, 1, AS, None, None, None, P, ws, None) == 1  # no A
+    assert f(P, P, None, P, P, 4, 16, 2, 1, AS, None, None, None, P, ws, None) == 1  # no proxy
+    assert f(P, P, P, P, P, 4, 16, 0, 1, AS, None, None, None, P, ws, None) == 1     # r = 0
+    assert f(P, P, P, P, P, 4, 16, 2, -1, AS, None, None, None, P, ws, None) == 1    # k < 0
+    assert f(P, P, P, P, P, 4, 16, 2, 1, 0, None, None, None, P, ws, None) == 1      # neither step
+    assert f(P, P, P, P, P, 4, 16, 2, 1, AS | 4, None, None, None, P, ws, None) == 1  # no residual form
+    assert f(P, P, P, P, P, 4, 16, 2, 1, AS | 16, None, None, None, P, ws, None) == 1  # unknown flag
+    assert f(P, P, P, P, P, 0, 16, 2, 1, AS, None, None, None, P, ws, None) == 1     # N = 0
+    assert f(P, P, P, P, P, 4, 20, 2, 1, AS, None, None, None, P, ws, None) == 2     # K % 16
+    assert f(P, P, P, P, P, 4, 20, 2, 1, AS | 8, None, None, None, P, ws, None) == 2  # STRICT accepted
+    assert f(P, P, P, P, P, 4, 16, 16385, 1, AS, None, None, None, P, 1 << 30, None) == 2  # r too large
+    assert f(P8, P, P, P, P, 4, 16, 2, 1, AS, None, None, None, P, ws, None) == 2    # unaligned codes
+    assert f(P, P, P, P, P, 4, 16, 2, 1, AS, None, None, None, P, ws - 256, None) == 3  # workspace
+    assert f(P, P, P, P, P, 4, 16, 2, 1, AS, None, None, None, P8, ws, None) == 3   # misaligned workspace
 
 
 def test_folded_argument_errors():

@@ -62,16 +62,24 @@ def test_phase_work_matches_the_stated_algorithmic_work():
 
 
 def test_traffic_is_withheld_when_a_source_changes(tmp_path, monkeypatch):
-    """bench.py reports the captured DRAM traffic only while the kernel
-    sources hash as they did at the capture."""
+    """bench.py reports a captured DRAM traffic figure only while the kernel
+    sources hash as they did at the capture; every committed figure matches
+    the committed sources."""
+    import hashlib
+
     sys.path.insert(0, ROOT)
     import bench
 
-    assert bench._traffic("proxy") == bench.TRAFFIC["proxy"]["bytes"]  # the committed sources
+    for phase, t in bench.TRAFFIC.items():  # committed figures are current
+        assert bench._traffic(phase) == t["bytes"], phase
+        assert "ncu" in t["capture"] and "--clock-control none" in t["capture"]
+    src = tmp_path / "k.cu"
+    src.write_text("kernel")
+    entry = {"bytes": 123, "capture": "ncu --clock-control none ...",
+             "sources": {"k.cu": hashlib.sha256(b"kernel").hexdigest()}}
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    for rel in bench.TRAFFIC["proxy"]["sources"]:
-        p = tmp_path / rel
-        p.parent.mkdir(parents=True, exist_ok=True)
-        p.write_text("changed")
+    monkeypatch.setattr(bench, "TRAFFIC", {"proxy": entry})
+    assert bench._traffic("proxy") == 123
+    src.write_text("changed")
     assert bench._traffic("proxy") is None
     assert bench._traffic("fwd") is None  # no capture recorded for it
