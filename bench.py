@@ -1,25 +1,30 @@
 """Throughput of one melded-FP8 linear training step (FALQON hot path) on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl falqon|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--rank R]
+                    [--impl falqon|reference]
 
-A step is the whole hot path for one synthetic token batch of the workload:
-  quantize X -> forward GEMM -> quantize dY -> adapter grads dB, dA -> dX GEMM
-  -> caller's plain SGD on B (two tiny torch ops) -> row-wise proxy update.
-All five library phases run in libfalqon's kernels through the C ABI.
+A step is the whole hot path for one synthetic token batch of the workload,
+layer by layer: the forward pass (quantize each activation once, then the
+forward GEMM of every layer that reads it), then the backward pass in reverse
+layer order (quantize dY, adapter gradients dB and dA, dX GEMM, the caller's
+plain SGD on B as two tiny torch ops, row-wise proxy update).  Every library
+phase runs in libfalqon's kernels through the C ABI.
 
-Timing: W untimed warm-up steps, then K timed steps.  The step is captured
-once per input slot in a CUDA graph and replayed; each timed step is bracketed
-by CUDA events on the launching stream and separated from the next by an L2
-flush (a 512 MB write and a 192 MB read, outside the events).  The timed region is bracketed by
-a barrier and torch.cuda.synchronize() on both sides; with N > 1 every rank
-runs an independent replica on its own batch ("replicas only", weak scaling)
-and the reported time is the max over ranks.
+Timing: W untimed warm-up steps, then K timed steps replayed back to back
+from CUDA graphs (one graph per input slot), bracketed by one pair of CUDA
+events on the launching stream, with a barrier and torch.cuda.synchronize()
+on both sides.  No L2 flush inside the timed region: the input slots cycled
+(4 by default) hold more bytes than the 126 MB L2, and each step pays for its
+own reads and for the write-back of what it writes, as in a training loop.
+With N > 1 every rank runs an independent replica on its own batch
+("replicas only", weak scaling) and the reported time is the max over ranks.
 
-Per-phase CUDA events give each kernel group's duration; the roofline object
-reports the slowest phase against the measured peaks in MEASURED_PEAKS.json.
-`e2e` repeats the step with the inputs in pinned host memory (H2D copies of X
-and dY and D2H copies of Y and dX inside the timed region).  `cpu_baseline`
-times the CPU oracle on a bounded sample (rank 0, N = 1).
+Per-phase times (for attribution only) replay each phase of the step from
+its own graph after an L2 flush; the roofline object reports the slowest
+phase against the measured peaks in MEASURED_PEAKS.json.  `e2e` repeats the
+step with the inputs in pinned host memory (H2D copies of every X and dY and
+D2H copies of every Y and dX inside the timed region).  `cpu_baseline` times
+the CPU oracle on a bounded sample (rank 0, N = 1).
 """
 
 from __future__ import annotations
@@ -36,11 +41,12 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
-from synthetic import WORKLOADS, layer_inputs  # noqa: E402
+from synthetic import WORKLOADS  # noqa: E402
 
 DEFAULT_WORKLOAD = "llama7b_attn_proj_4096x4096x4096_r64"
 METRIC = "melded FP8 linear fwd+bwd+proxy tokens/s; % of FP8 tensor peak / HBM"
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput ratio on B200
+L2_BYTES = 126 * 10**6  # B200 L2
 
 
 def _peaks():
@@ -122,95 +128,159 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
-class Step:
-    """Device buffers and the captured step for one workload layer."""
+def _device_normal(torch, dev, seed, shape, std, dtype):
+    """Seeded N(0, std^2) draws made on the device (torch's Philox generator),
+    rounded to dtype: the bench's inputs.  The parity tests draw theirs from
+    synthetic.gen; the bench's sizes (up to tens of GB for the stack) call for
+    a device generator."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(int(seed) & 0x7FFFFFFFFFFFFFFF)
+    return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std).to(dtype)
 
-    def __init__(self, wl, layer, torch, F, dev, n_slots=2, seed_offset=0):
-        self.torch, self.F, self.dev = torch, F, dev
-        self.M, self.N, self.K, self.r = wl.M, layer.N, layer.K, wl.r
-        self.lr = wl.lr
+
+def _seed(wl, *parts):
+    from synthetic import stream_seed
+    return stream_seed(wl.seed, "/".join([wl.name] + [str(p) for p in parts]))
+
+
+class LayerState:
+    """Persistent state of one layer: backbone codes and scale, adapters,
+    proxy, gradients and the caller-owned workspaces."""
+
+    def __init__(self, wl, layer, block, r, torch, F, dev, ws_q):
         t = torch
-        d0 = layer_inputs(wl, layer, step=seed_offset, with_b=True)
-
-        def bf16(bits):
-            return t.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(t.bfloat16).to(dev)
-
-        # persistent state of the layer
-        self.W = t.from_numpy(d0["W"]).to(dev)
+        self.name, self.block, self.group = layer.name, block, layer.x_group
+        self.N, self.K, self.r = layer.N, layer.K, r
+        W = _device_normal(t, dev, _seed(wl, block, layer.name, "W"), (self.N, self.K), wl.w_std, t.float32)
         self.wq = t.empty((self.N, self.K), dtype=t.uint8, device=dev)
         self.s_w = t.empty(1, dtype=t.float32, device=dev)
-        self.A = bf16(d0["A"])
-        self.B = bf16(d0["B"])
-        self.P = t.zeros((self.N, self.K), dtype=t.float32, device=dev)
         self.status = t.zeros(1, dtype=t.int32, device=dev)
-        # fresh X / dY per step: a few distinct slots, cycled
-        self.X = [bf16(layer_inputs(wl, layer, step=seed_offset + s)["X"]) for s in range(n_slots)]
-        self.dY = [bf16(layer_inputs(wl, layer, step=seed_offset + s)["dY"]) for s in range(n_slots)]
-        # outputs and intermediates
-        self.xq = t.empty((self.M, self.K), dtype=t.uint8, device=dev)
-        self.dyq = t.empty((self.M, self.N), dtype=t.uint8, device=dev)
-        self.s_x = t.empty(1, dtype=t.float32, device=dev)
-        self.s_dy = t.empty(1, dtype=t.float32, device=dev)
-        self.amax = t.empty(1, dtype=t.float32, device=dev)
-        self.y = t.empty((self.M, self.N), dtype=t.bfloat16, device=dev)
-        self.dx = t.empty((self.M, self.K), dtype=t.bfloat16, device=dev)
-        self.dA = t.empty((self.r, self.K), dtype=t.bfloat16, device=dev)
-        self.dB = t.empty((self.N, self.r), dtype=t.bfloat16, device=dev)
-        self.dB_inc = t.empty((self.N, self.r), dtype=t.bfloat16, device=dev)
+        amax = t.empty(1, dtype=t.float32, device=dev)
+        # initial quantization of the backbone (not part of the step)
+        F.falqon_quantize(W, codes=self.wq, scale=self.s_w, amax=amax, dev_status=self.status, workspace=ws_q)
+        del W
+        self.A = _device_normal(t, dev, _seed(wl, block, layer.name, "A", r), (r, self.K), wl.a_std, t.bfloat16)
+        self.B = t.zeros((self.N, r), dtype=t.bfloat16, device=dev)
+        self.P = t.zeros((self.N, self.K), dtype=t.float32, device=dev)
+        self.dA = t.empty((r, self.K), dtype=t.bfloat16, device=dev)
+        self.dB = t.empty((self.N, r), dtype=t.bfloat16, device=dev)
+        self.dB_inc = t.empty((self.N, r), dtype=t.bfloat16, device=dev)
         self.mask = t.empty(self.N, dtype=t.uint8, device=dev)
         self.n_sel = t.zeros(1, dtype=t.int32, device=dev)
 
-        def ws(op, M, N, K, r):
-            n = F.falqon_workspace_size(op, M, N, K, r)
+        def ws(op, M, N, K, rr):
+            n = F.falqon_workspace_size(op, M, N, K, rr)
             return t.empty(max(n, 256), dtype=t.uint8, device=dev)
 
-        self.ws_q = ws(F.OP_QUANTIZE, self.M, max(self.N, self.K), 0, 0)
-        self.ws_q2 = ws(F.OP_QUANTIZE, self.N, self.K, 0, 0)
-        self.ws_bwd = ws(F.OP_LINEAR_BWD, self.M, self.N, self.K, self.r)
-        self.ws_p = ws(F.OP_PROXY_UPDATE, 0, self.N, self.K, self.r)
-        # initial quantization of the backbone (not part of the step)
-        F.falqon_quantize(self.W, codes=self.wq, scale=self.s_w, amax=self.amax,
-                          dev_status=self.status, workspace=self.ws_q2)
-        # library kernels per step: quantize X (1) + forward (1) + quantize dY (1)
-        # + adapter products (T with U, dB with dA: 2) + dX (1) + proxy update and clear (2)
-        self.launches_per_step = 1 + 1 + 1 + 2 + 1 + 2
+        self.ws_bwd = ws(F.OP_LINEAR_BWD, wl.M, self.N, self.K, r)
+        self.ws_p = ws(F.OP_PROXY_UPDATE, 0, self.N, self.K, r)
 
-    # one C-ABI call per phase (the caller's SGD: two torch ops)
+
+class Step:
+    """Device buffers and the calls of one step of a workload: every layer of
+    every block, the activations shared by the layers of an input group
+    quantized once."""
+
     PHASES = ("quantX", "fwd", "quantdY", "adapters", "dX", "sgd", "proxy")
+    # library kernels per call of each phase (the caller's SGD is two torch ops)
+    LAUNCHES = {"quantX": 1, "fwd": 1, "quantdY": 1, "adapters": 2, "dX": 1, "sgd": 0, "proxy": 2}
 
-    def phase(self, slot, k):
-        """Enqueues phase k of one step on the current stream."""
+    def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None):
+        self.torch, self.F, self.dev = torch, F, dev
+        t = torch
+        self.wl = wl
+        self.M, self.r, self.lr = wl.M, (wl.r if r is None else r), wl.lr
+        self.n_slots = n_slots
+        self.n_stack = n_stack or wl.n_stack
+        maxdim = max(max(l.N, l.K) for l in wl.layers)
+        self.ws_q = t.empty(max(F.falqon_workspace_size(F.OP_QUANTIZE, self.M, maxdim, 0, 0),
+                                F.falqon_workspace_size(F.OP_QUANTIZE, maxdim, maxdim, 0, 0), 256),
+                            dtype=t.uint8, device=dev)
+        self.layers = [LayerState(wl, l, b, self.r, t, F, dev, self.ws_q)
+                       for b in range(self.n_stack) for l in wl.layers]
+        # input groups (block, x_group) in order of first use, with their K
+        self.groups = {}
+        for L in self.layers:
+            self.groups.setdefault((L.block, L.group), L.K)
+        so = seed_offset
+        self.X = [{g: _device_normal(t, dev, _seed(wl, g[0], g[1], "X", so + s), (self.M, K), wl.x_std, t.bfloat16)
+                   for g, K in self.groups.items()} for s in range(n_slots)]
+        self.dY = [[_device_normal(t, dev, _seed(wl, L.block, L.name, "dY", so + s), (self.M, L.N), wl.dy_std,
+                                   t.bfloat16) for L in self.layers] for s in range(n_slots)]
+        # codes and scales of every activation (kept from the forward for the backward)
+        self.xq = {g: t.empty((self.M, K), dtype=t.uint8, device=dev) for g, K in self.groups.items()}
+        self.s_x = {g: t.empty(1, dtype=t.float32, device=dev) for g in self.groups}
+        # per-shape outputs, reused across layers: nothing downstream reads them
+        self.y = {n: t.empty((self.M, n), dtype=t.bfloat16, device=dev) for n in {L.N for L in self.layers}}
+        self.dx = {k: t.empty((self.M, k), dtype=t.bfloat16, device=dev) for k in {L.K for L in self.layers}}
+        self.dyq = {n: t.empty((self.M, n), dtype=t.uint8, device=dev) for n in {L.N for L in self.layers}}
+        self.s_dy = t.empty(1, dtype=t.float32, device=dev)
+        self.amax = t.empty(1, dtype=t.float32, device=dev)
+        self.status = t.zeros(1, dtype=t.int32, device=dev)
+        self.calls_per_step = {p: 0 for p in self.PHASES}
+        for _, p, _ in self.calls(0):
+            self.calls_per_step[p] += 1
+        self.launches_per_step = sum(self.LAUNCHES[p] * n for p, n in self.calls_per_step.items())
+
+    @property
+    def tokens(self):
+        return self.M
+
+    def status_words(self):
+        return [self.status] + [L.status for L in self.layers]
+
+    def device_status(self) -> int:
+        v = 0
+        for s in self.status_words():
+            v |= int(s.item())
+        return v
+
+    def calls(self, slot, outs=None):
+        """The step as (layer, phase, enqueue function) in execution order.
+        outs: optional (ys, dxs), per-layer output tensors in place of the
+        shared per-shape ones."""
         F, t = self.F, self.torch
-        name = self.PHASES[k]
-        if name == "quantX":
-            F.falqon_quantize(self.X[slot], codes=self.xq, scale=self.s_x, amax=self.amax,
-                              dev_status=self.status, workspace=self.ws_q)
-        elif name == "fwd":
-            F.falqon_linear_fwd(self.xq, self.s_x, self.wq, self.s_w, y=self.y,
-                                dev_status=self.status)
-        elif name == "quantdY":
-            F.falqon_quantize(self.dY[slot], codes=self.dyq, scale=self.s_dy, amax=self.amax,
-                              dev_status=self.status, workspace=self.ws_q)
-        elif name == "adapters":
-            F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, self.xq, self.s_x, self.A,
-                                self.B, dx=None, dA=self.dA, dB=self.dB, dev_status=self.status,
-                                workspace=self.ws_bwd)
-        elif name == "dX":
-            F.falqon_linear_bwd(self.dyq, self.s_dy, self.wq, self.s_w, None, None, None, None,
-                                dx=self.dx, dA=None, dB=None, dev_status=self.status)
-        elif name == "sgd":
-            # the caller's optimizer: plain SGD on B; the proxy receives the increment
-            t.mul(self.dB, -self.lr, out=self.dB_inc)
-            self.B.add_(self.dB_inc)
-        else:
-            F.falqon_proxy_update(self.wq, self.s_w, self.P, self.dB_inc, self.A,
-                                  row_mask=self.mask, n_selected=self.n_sel,
-                                  dev_status=self.status, workspace=self.ws_p)
+        X, dY = self.X[slot], self.dY[slot]
+        yo = (lambda j, L: outs[0][j]) if outs else (lambda j, L: self.y[L.N])
+        xo = (lambda j, L: outs[1][j]) if outs else (lambda j, L: self.dx[L.K])
+        out = []
+        seen = set()
+        for jf, L in enumerate(self.layers):  # forward pass
+            g = (L.block, L.group)
+            if g not in seen:
+                seen.add(g)
+                out.append((L, "quantX", lambda g=g: F.falqon_quantize(
+                    X[g], codes=self.xq[g], scale=self.s_x[g], amax=self.amax, dev_status=self.status,
+                    workspace=self.ws_q)))
+            out.append((L, "fwd", lambda L=L, g=g, y=yo(jf, L): F.falqon_linear_fwd(
+                self.xq[g], self.s_x[g], L.wq, L.s_w, y=y, dev_status=L.status)))
+        for j in range(len(self.layers) - 1, -1, -1):  # backward pass, last layer first
+            L = self.layers[j]
+            g = (L.block, L.group)
+            dyq = self.dyq[L.N]
+            out.append((L, "quantdY", lambda j=j, L=L, dyq=dyq: F.falqon_quantize(
+                dY[j], codes=dyq, scale=self.s_dy, amax=self.amax, dev_status=self.status, workspace=self.ws_q)))
+            out.append((L, "adapters", lambda L=L, g=g, dyq=dyq: F.falqon_linear_bwd(
+                dyq, self.s_dy, L.wq, L.s_w, self.xq[g], self.s_x[g], L.A, L.B, dx=None, dA=L.dA, dB=L.dB,
+                dev_status=L.status, workspace=L.ws_bwd)))
+            out.append((L, "dX", lambda L=L, dyq=dyq, dx=xo(j, L): F.falqon_linear_bwd(
+                dyq, self.s_dy, L.wq, L.s_w, None, None, None, None, dx=dx, dA=None, dB=None,
+                dev_status=L.status)))
 
-    def phases(self, slot):
-        """Enqueues one whole step."""
-        for k in range(len(self.PHASES)):
-            self.phase(slot, k)
+            def sgd(L=L):  # the caller's optimizer: plain SGD on B; the proxy receives the increment
+                t.mul(L.dB, -self.lr, out=L.dB_inc)
+                L.B.add_(L.dB_inc)
+            out.append((L, "sgd", sgd))
+            out.append((L, "proxy", lambda L=L: F.falqon_proxy_update(
+                L.wq, L.s_w, L.P, L.dB_inc, L.A, row_mask=L.mask, n_selected=L.n_sel, dev_status=L.status,
+                workspace=L.ws_p)))
+        return out
+
+    def run(self, slot, phase=None, outs=None):
+        """Enqueues the whole step (or only the calls of one phase) on the current stream."""
+        for _, p, f in self.calls(slot, outs):
+            if phase is None or p == phase:
+                f()
 
 
 # FP32 FMA peak of the CUDA cores (the proxy's bound at large r): 148 SMs x 128
@@ -241,8 +311,9 @@ def _traffic(phase):
 
 
 def _phase_work(st):
-    """Algorithmic work and bound of each phase: flops, bytes (each tensor
-    once at its storage width), the roofline that bounds it and its kernels."""
+    """Algorithmic work and bound of each phase of one layer (st: M, N, K, r):
+    flops, bytes (each tensor once at its storage width), the roofline that
+    bounds it and its kernels."""
     M, N, K, r = st.M, st.N, st.K, st.r
     proxy_flops, proxy_bytes = 2.0 * N * K * r, 9.0 * N * K + 2.0 * r * (N + K)
     # the proxy is bound by the FP32 FMA pipe when its FMA time exceeds its HBM time
@@ -266,6 +337,33 @@ def _phase_work(st):
     }
 
 
+def _step_work(st):
+    """_phase_work summed over the calls of one step (an activation shared by
+    several layers is quantized once)."""
+    import types
+
+    tot = {}
+    for L, p, _ in st.calls(0):
+        w = _phase_work(types.SimpleNamespace(M=st.M, N=L.N, K=L.K, r=st.r))[p]  # quantX: the group's K
+        e = tot.setdefault(p, {"flops": 0.0, "bytes": 0.0, "bound": w["bound"], "kernels": w["kernels"], "calls": 0})
+        e["flops"] += w["flops"]
+        e["bytes"] += w["bytes"]
+        e["calls"] += 1
+    return tot
+
+
+def _flusher(torch, dev):
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush_tail = flush[: 192 << 20].view(torch.int32)
+
+    def l2_flush(i):
+        """Evicts L2: a 512 MB write, then a 192 MB read, so that the lines left
+        behind are clean and no write-back of the flush lands in what follows."""
+        flush.fill_(i & 0xFF)
+        flush_tail.sum()
+    return l2_flush
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -279,68 +377,63 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     F.lib()
     wl = WORKLOADS[args.workload]
-    layer = wl.layers[0]
-    st = Step(wl, layer, torch, F, dev, n_slots=2, seed_offset=rank * 1000)
+    r = args.rank if args.rank else wl.r
+    n_stack = args.blocks or wl.n_stack
+    # bytes of one slot: every activation group's X and every layer's dY (bf16)
+    slot_bytes = n_stack * wl.M * 2 * (sum(k for _, k in {(l.x_group, l.K) for l in wl.layers}) +
+                                       sum(l.N for l in wl.layers))
+    slots = args.slots or min(8, max(2, -(-(2 * L2_BYTES) // slot_bytes)))
+    st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack)
     stream = torch.cuda.Stream(device=dev)
     if args.only:
         # one phase alone, eagerly, warm-up + steps times (for profiler captures)
-        k = Step.PHASES.index(args.only)
         with torch.cuda.stream(stream):
-            st.phases(0)  # one whole step first, so every input of the phase is real data
+            st.run(0)  # one whole step first, so every input of the phase is real data
             for i in range(args.warmup + args.steps):
-                st.phase(i % 2, k)
+                st.run(i % st.n_slots, args.only)
         torch.cuda.synchronize()
-        status = int(st.status.item())
-        return {"only": args.only, "launches": args.warmup + args.steps, "device_status": status}, rank
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    flush_tail = flush[: 192 << 20].view(torch.int32)
-
-    def l2_flush(i):
-        """Evicts L2: a 512 MB write, then a 192 MB read, so that the lines left
-        behind are clean and no write-back of the flush lands in the next step."""
-        flush.fill_(i & 0xFF)
-        flush_tail.sum()
+        return {"only": args.only, "calls": (args.warmup + args.steps) * st.calls_per_step[args.only],
+                "device_status": st.device_status()}, rank
+    l2_flush = _flusher(torch, dev)
 
     # capture the step once per input slot
-    graphs = []
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        for slot in range(2):  # warm the library (attributes, tensor-map encoder) first
-            st.phases(slot)
+        for slot in range(min(2, st.n_slots)):  # warm the library (attributes, tensor-map encoder) first
+            st.run(slot)
     torch.cuda.synchronize()
-    phase_graphs = []  # [slot][phase]: each phase alone, for launch-gap-free attribution
+    graphs, phase_graphs = [], []  # phase_graphs[slot][phase]: that phase of every layer
     if not args.no_graph:
-        for slot in range(2):
+        for slot in range(st.n_slots):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                st.phases(slot)
+                st.run(slot)
             graphs.append(g)
+        for slot in range(min(2, st.n_slots)):
             per = []
-            for k in range(len(Step.PHASES)):
+            for p in Step.PHASES:
                 gk = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gk, stream=stream):
-                    st.phase(slot, k)
+                    st.run(slot, p)
                 per.append(gk)
             phase_graphs.append(per)
     torch.cuda.synchronize()
 
     def step(i):
         if graphs:
-            graphs[i % 2].replay()
+            graphs[i % st.n_slots].replay()
         else:
-            st.phases(i % 2)
+            st.run(i % st.n_slots)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            l2_flush(i)
             step(i)
     torch.cuda.synchronize()
-    if int(st.status.item()) != 0:
-        raise RuntimeError(f"device status {int(st.status.item())} after warm-up")
+    if st.device_status() != 0:
+        raise RuntimeError(f"device status {st.device_status()} after warm-up")
 
-    # timed region: per-step events, L2 flush between steps (outside the events)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    # timed region: K steps back to back, one event pair (plus one event per step)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     clocks = ClockSampler(local)
     if ws > 1:
         dist.barrier()
@@ -348,20 +441,19 @@ def run_gpu(args):
     clocks.start()
     time.sleep(0.25)
     with torch.cuda.stream(stream):
+        evs[0].record()
         for i in range(args.steps):
-            l2_flush(i)
-            starts[i].record()
-            step(i)
-            ends[i].record()
+            step(args.warmup + i)
+            evs[i + 1].record()
     torch.cuda.synchronize()
     clock_info = clocks.stop()
     if ws > 1:
         dist.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(float(np.sum(step_ms)), dev)
+    total_ms = max_over_ranks(evs[0].elapsed_time(evs[-1]), dev)
+    per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
 
-    # per-phase timing: each phase replayed from its own graph, back to back,
-    # events between the replays; same L2 flush discipline as the timed steps
+    # per-phase attribution: each phase (of every layer) replayed from its own
+    # graph, L2 flushed before each rep, events between the phases
     names = list(Step.PHASES)
     acc = {n: 0.0 for n in names}
     reps = max(5, min(50, args.steps))
@@ -370,95 +462,40 @@ def run_gpu(args):
             l2_flush(i)
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
             ev[0].record()
-            for k in range(len(names)):
+            for k, n in enumerate(names):
                 if phase_graphs:
-                    phase_graphs[i % 2][k].replay()
+                    phase_graphs[i % len(phase_graphs)][k].replay()
                 else:
-                    st.phase(i % 2, k)
+                    st.run(i % st.n_slots, n)
                 ev[k + 1].record()
             torch.cuda.synchronize()
             for j, n in enumerate(names):
                 acc[n] += ev[j].elapsed_time(ev[j + 1])
     phase_ms = {n: acc[n] / reps for n in names}
 
-    # e2e through the C ABI with host buffers (pinned), copies inside the timed
-    # region.  Inputs are copied in on one stream, the step runs on the compute
-    # stream, outputs are copied out on a third, with two slots of every
-    # buffer: the copies of neighbouring steps overlap the step and each other
-    # (the link is full duplex).  Events order each slot's reuse.
-    hostX = [x.cpu().pin_memory() for x in st.X]
-    hostdY = [x.cpu().pin_memory() for x in st.dY]
-    ys = [st.y, torch.empty_like(st.y)]
-    dxs = [st.dx, torch.empty_like(st.dx)]
-    hostY = [torch.empty(st.y.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    hostdX = [torch.empty(st.dx.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    hostSel = [torch.empty(1, dtype=torch.int32).pin_memory() for _ in range(2)]
-    sel = [torch.empty_like(st.n_sel) for _ in range(2)]  # each step's count, kept per slot
-    e2e_steps = max(3, min(args.steps, 50))
-    s_in = torch.cuda.Stream(device=dev)
-    s_out = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(e2e_steps)]
-    ev_done = [torch.cuda.Event() for _ in range(e2e_steps)]
-    ev_out = [torch.cuda.Event() for _ in range(e2e_steps)]
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e_start.record(s_in)
-    stream.wait_event(e_start)
-    s_out.wait_event(e_start)
-    for i in range(e2e_steps):
-        k = i % 2
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_done[i - 2])  # step i-2 no longer reads slot k's inputs
-            st.X[k].copy_(hostX[k], non_blocking=True)
-            st.dY[k].copy_(hostdY[k], non_blocking=True)
-            ev_in[i].record(s_in)
-        with torch.cuda.stream(stream):
-            stream.wait_event(ev_in[i])
-            if i >= 2:
-                stream.wait_event(ev_out[i - 2])  # slot k's outputs of step i-2 copied out
-            st.y, st.dx = ys[k], dxs[k]
-            st.phases(k)
-            sel[k].copy_(st.n_sel)
-            ev_done[i].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_done[i])
-            hostY[k].copy_(ys[k], non_blocking=True)
-            hostdX[k].copy_(dxs[k], non_blocking=True)
-            hostSel[k].copy_(sel[k], non_blocking=True)
-            ev_out[i].record(s_out)
-    s_out.wait_event(ev_done[e2e_steps - 1])
-    e_end.record(s_out)
-    torch.cuda.synchronize()
-    st.y, st.dx = ys[0], dxs[0]
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
-    status = int(st.status.item())
-    n_sel = int(st.n_sel.item())
-    topk = _time_topk(st, F, torch, stream, l2_flush, args, dev) if args.topk > 0 else None
-    e5 = _time_e5m2(st, F, torch, stream, l2_flush, args, dev) if args.e5m2 else None
-    folded = _time_folded(st, F, torch, stream, l2_flush, args, dev) if args.folded else None
+    e2e = _time_e2e(st, torch, stream, ws, dev, args) if args.e2e else {"skipped": "--e2e 0"}
+    status = st.device_status()
+    n_sel = sum(int(L.n_sel.item()) for L in st.layers)
+    single = len(st.layers) == 1
+    v = _single_view(st) if single else None
+    topk = _time_topk(v, F, torch, stream, l2_flush, args, dev) if (args.topk > 0 and single) else None
+    e5 = _time_e5m2(v, F, torch, stream, l2_flush, args, dev) if (args.e5m2 and single) else None
+    folded = _time_folded(v, F, torch, stream, l2_flush, args, dev) if (args.folded and single) else None
 
-    tokens_total = wl.M * args.steps * ws
+    tokens_total = st.tokens * args.steps * ws
     value = tokens_total / (total_ms / 1e3)
-    e2e_value = wl.M * e2e_steps * ws / (e2e_ms / 1e3)
-    h2d = 2 * (st.X[0].numel() * 2 + st.dY[0].numel() * 2) // 2
-    d2h = st.y.numel() * 2 + st.dx.numel() * 2 + 4
 
     peaks = _peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
-    work = _phase_work(st)
+    work = _step_work(st)
     phases = {}
     for n in names:
         ms = phase_ms[n]
         w = work[n]
         tflops = w["flops"] / (ms * 1e-3) / 1e12 if ms > 0 else 0.0
         gbs = w["bytes"] / (ms * 1e-3) / 1e9 if ms > 0 else 0.0
-        ph = {"ms": round(ms, 5), "kernels": w["kernels"], "bound": w["bound"],
-              "tflops": round(tflops, 2), "gbs": round(gbs, 1),
-              "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        ph = {"ms": round(ms, 5), "calls": w["calls"], "kernels": w["kernels"], "bound": w["bound"],
+              "tflops": round(tflops, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
         if w["bound"] == "tensor":
             ph["frac_fp8_peak"] = round(tflops / fp8_peak, 4)
         if w["bound"] == "alu":
@@ -482,24 +519,29 @@ def run_gpu(args):
         roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "hbm",
                 "achieved": phases[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": phases[dom]["frac_hbm"], "peak_source": f"{peaks['source']} copy bandwidth"}
-    roof["traffic"] = _traffic(dom)
+    roof["timing"] = "phase replayed from its own CUDA graph after an L2 flush, events on the launching stream"
+    roof["traffic"] = _traffic(dom) if single else None
     if roof["traffic"] is not None:
         roof["traffic_capture"] = TRAFFIC[dom]["capture"]
 
+    layer0 = st.layers[0]
+    slot_bytes = sum(x.numel() * 2 for x in st.X[0].values()) + sum(d.numel() * 2 for d in st.dY[0])
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M, "N": layer.N, "K": layer.K, "r": wl.r,
-                   "global_batch_tokens": wl.M * ws, "parallelism": f"replicas{ws}",
-                   "l2": "flushed between timed steps (512 MB write + 192 MB read, outside the events)",
+        "config": {"workload": wl.name, "M": st.M, "r": st.r, "layers": len(st.layers),
+                   "blocks": st.n_stack, "shapes": sorted({f"{L.K}->{L.N}" for L in st.layers}),
+                   "N": layer0.N, "K": layer0.K,
+                   "global_batch_tokens": st.M * ws, "parallelism": f"replicas{ws}",
+                   "l2": (f"back to back: no flush; {st.n_slots} input slots cycled "
+                          f"({st.n_slots * slot_bytes / 2**20:.0f} MiB of X and dY, above the 126 MB L2)"),
                    "cuda_graph": not args.no_graph, "lr": wl.lr},
+        "step_ms_median": round(float(np.median(per_step)), 5),
         "roofline": roof,
         "phases": phases,
-        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-                "pipelining": "copy-in, step and copy-out on three streams, two buffer slots"},
+        "e2e": e2e,
         "gpu_launches": st.launches_per_step * args.steps,
         "clocks": clock_info,
         "device_status": status,
@@ -507,10 +549,99 @@ def run_gpu(args):
         "extra": {"proxy_topk": topk, "e5m2_gradients": e5, "folded_adapters": folded},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(wl, layer, budget_s=args.cpu_budget)
+        out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget, r=st.r, n_stack=st.n_stack)
     if ws > 1:
         dist.destroy_process_group()
     return out, rank
+
+
+def _single_view(st):
+    """The one layer of a single-layer step, with the step's buffers, for the
+    extra rows (top-k, E5M2, folded adapters)."""
+    import types
+
+    L = st.layers[0]
+    g = (L.block, L.group)
+    return types.SimpleNamespace(
+        M=st.M, N=L.N, K=L.K, r=st.r, wq=L.wq, s_w=L.s_w, P=L.P, A=L.A, B=L.B, dA=L.dA, dB=L.dB,
+        dB_inc=L.dB_inc, xq=st.xq[g], s_x=st.s_x[g], dyq=st.dyq[L.N], s_dy=st.s_dy, dY0=st.dY[0][0],
+        y=st.y[L.N], dx=st.dx[L.K], ws_bwd=L.ws_bwd, ws_q=st.ws_q, amax=st.amax, status=L.status)
+
+
+def _time_e2e(st, torch, stream, ws, dev, args):
+    """The step through the C ABI with host buffers: every X and dY copied in
+    from pinned host memory and every Y and dX (and the selected counts) out,
+    inside the timed region.  Copy-in, step and copy-out run on three streams
+    with two buffer slots, so the copies of neighbouring steps overlap the
+    step and each other (the link is full duplex); events order each slot's
+    reuse.  The step's calls write every layer's Y and dX straight into
+    per-slot device buffers, which are copied out."""
+    in_bytes = sum(x.numel() * 2 for x in st.X[0].values()) + sum(d.numel() * 2 for d in st.dY[0])
+    if in_bytes > (4 << 30):
+        return {"skipped": f"{in_bytes / 2**30:.1f} GiB of inputs per step: pinned host slots not allocated"}
+    nslot = min(2, st.n_slots)
+    hostX = [{g: x.cpu().pin_memory() for g, x in st.X[k].items()} for k in range(nslot)]
+    hostdY = [[d.cpu().pin_memory() for d in st.dY[k]] for k in range(nslot)]
+    # per-step outputs: each layer's Y and dX in their own device and host slots
+    ys = [[torch.empty((st.M, L.N), dtype=torch.bfloat16, device=dev) for L in st.layers] for _ in range(nslot)]
+    dxs = [[torch.empty((st.M, L.K), dtype=torch.bfloat16, device=dev) for L in st.layers] for _ in range(nslot)]
+    hostY = [[torch.empty((st.M, L.N), dtype=torch.bfloat16).pin_memory() for L in st.layers] for _ in range(nslot)]
+    hostdX = [[torch.empty((st.M, L.K), dtype=torch.bfloat16).pin_memory() for L in st.layers]
+              for _ in range(nslot)]
+    sel = [torch.empty(len(st.layers), dtype=torch.int32, device=dev) for _ in range(nslot)]
+    hostSel = [torch.empty(len(st.layers), dtype=torch.int32).pin_memory() for _ in range(nslot)]
+    steps = max(3, min(args.steps, 50))
+    s_in = torch.cuda.Stream(device=dev)
+    s_out = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(steps)]
+    ev_done = [torch.cuda.Event() for _ in range(steps)]
+    ev_out = [torch.cuda.Event() for _ in range(steps)]
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    index = {id(L): j for j, L in enumerate(st.layers)}
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start.record(s_in)
+    stream.wait_event(e_start)
+    s_out.wait_event(e_start)
+    for i in range(steps):
+        k = i % nslot
+        with torch.cuda.stream(s_in):
+            if i >= nslot:
+                s_in.wait_event(ev_done[i - nslot])  # step i-2 no longer reads slot k's inputs
+            for g, x in st.X[k].items():
+                x.copy_(hostX[k][g], non_blocking=True)
+            for j, d in enumerate(st.dY[k]):
+                d.copy_(hostdY[k][j], non_blocking=True)
+            ev_in[i].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev_in[i])
+            if i >= nslot:
+                stream.wait_event(ev_out[i - nslot])  # slot k's outputs of step i-2 copied out
+            for L, p, f in st.calls(k, (ys[k], dxs[k])):
+                f()
+                if p == "proxy":
+                    j = index[id(L)]
+                    sel[k][j:j + 1].copy_(L.n_sel)
+            ev_done[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[i])
+            for j in range(len(st.layers)):
+                hostY[k][j].copy_(ys[k][j], non_blocking=True)
+                hostdX[k][j].copy_(dxs[k][j], non_blocking=True)
+            hostSel[k].copy_(sel[k], non_blocking=True)
+            ev_out[i].record(s_out)
+    s_out.wait_event(ev_done[steps - 1])
+    e_end.record(s_out)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
+    h2d = in_bytes
+    d2h = sum(L.N * st.M * 2 + L.K * st.M * 2 for L in st.layers) + 4 * len(st.layers)
+    return {"value": round(st.M * steps * ws / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "pipelining": "copy-in, step and copy-out on three streams, two buffer slots"}
 
 
 def _graph_phase_times(torch, stream, l2_flush, fns, reps, use_graph=True):
@@ -586,7 +717,7 @@ def _time_e5m2(st, F, torch, stream, l2_flush, args, dev):
     names = ("quantdY", "adapters", "dX")
     reps = max(5, min(50, args.steps))
     fns = [
-        lambda: F.falqon_quantize(st.dY[0], codes=dyq, scale=s_dy, amax=st.amax, dev_status=st.status,
+        lambda: F.falqon_quantize(st.dY0, codes=dyq, scale=s_dy, amax=st.amax, dev_status=st.status,
                                   workspace=st.ws_q, fmt="e5m2"),
         lambda: F.falqon_linear_bwd(dyq, s_dy, st.wq, st.s_w, st.xq, st.s_x, st.A, st.B, dx=None, dA=dA,
                                     dB=dB, dev_status=st.status, workspace=st.ws_bwd, dy_fmt="e5m2"),
@@ -642,57 +773,101 @@ def _time_folded(st, F, torch, stream, l2_flush, args, dev):
 
 # ------------------------------------------------------------------ CPU oracle
 class _OracleData:
-    """Inputs of the oracle arm, generated once: two X / dY slots and the backbone."""
+    """Inputs of the oracle arm for one layer shape (K -> N), drawn once with
+    synthetic.gen: the backbone (full size, so its scale is the layer's), the
+    adapters, and X / dY rows drawn per step at the sample's size."""
 
-    def __init__(self, O, wl, layer):
-        self.slots = [layer_inputs(wl, layer, step=s, with_b=True) for s in range(2)]
-        self.wq, self.s_w, _, _ = O.quantize(self.slots[0]["W"])
+    def __init__(self, O, wl, layer, r):
+        from synthetic import gen, stream_seed
+
+        self.wl, self.layer, self.r = wl, layer, r
+        tag = f"{wl.name}/oracle/{layer.name}"
+        W = gen.normal_f32(stream_seed(wl.seed, tag + "/W"), (layer.N, layer.K), wl.w_std)
+        self.wq, self.s_w, _, _ = O.quantize(W)
+        self.A = gen.normal_bf16_bits(stream_seed(wl.seed, tag + f"/A/r{r}"), (r, layer.K), wl.a_std)
+        self.B = gen.normal_bf16_bits(stream_seed(wl.seed, tag + f"/B/r{r}"), (layer.N, r), 1e-3)
+        self._tag = tag
+
+    def rows(self, step, tokens):
+        from synthetic import gen, stream_seed
+
+        wl, layer = self.wl, self.layer
+        X = gen.normal_bf16_bits(stream_seed(wl.seed, self._tag + f"/X/{step}"), (tokens, layer.K), wl.x_std)
+        dY = gen.normal_bf16_bits(stream_seed(wl.seed, self._tag + f"/dY/{step}"), (tokens, layer.N), wl.dy_std)
+        return X, dY
 
 
-def _oracle_sample_step(O, wl, layer, data, tokens, proxy_rows, step):
-    """One oracle step on a bounded sample: `tokens` rows of X and dY through
-    quantize / forward / dX / dB / dA, and `proxy_rows` rows of the proxy update."""
-    d = data.slots[step % 2]
-    X, dY = np.ascontiguousarray(d["X"][:tokens]), np.ascontiguousarray(d["dY"][:tokens])
-    wq, s_w = data.wq, data.s_w
-    P = np.zeros((proxy_rows, layer.K), dtype=np.float32)
+def _oracle_sample_step(O, wl, data, tokens, proxy_rows, step):
+    """One oracle step of one layer shape on a bounded sample: `tokens` rows of
+    X and dY through quantize / forward / dX / dB / dA, and `proxy_rows` rows
+    of the proxy update.  Returns the two times (s)."""
+    X, dY = data.rows(step, tokens)
+    wq, s_w, K = data.wq, data.s_w, data.layer.K
+    P = np.zeros((proxy_rows, K), dtype=np.float32)
     t0 = time.perf_counter()
     xq, s_x, _, _ = O.quantize(X)
     O.linear_fwd(xq, s_x, wq, s_w)
     dyq, s_dy, _, _ = O.quantize(dY)
     O.linear_dx(dyq, s_dy, wq, s_w)
-    t64, _ = O.adapter_t(xq, s_x, d["A"])
+    t64, _ = O.adapter_t(xq, s_x, data.A)
     db = O.adapter_db(dyq, s_dy, t64=t64)
-    u64, _ = O.adapter_u(dyq, s_dy, d["B"])
+    u64, _ = O.adapter_u(dyq, s_dy, data.B)
     O.adapter_da(xq, s_x, u64=u64)
     t1 = time.perf_counter()
     dB_inc = O.bf16_round(-wl.lr * O.bf16_to_f64(O.bf16_round(db)))
-    O.proxy_update(np.ascontiguousarray(wq[:proxy_rows]), s_w, P,
-                   np.ascontiguousarray(dB_inc[:proxy_rows]), d["A"])
+    O.proxy_update(np.ascontiguousarray(wq[:proxy_rows]), s_w, P, np.ascontiguousarray(dB_inc[:proxy_rows]),
+                   data.A)
     t2 = time.perf_counter()
     return t1 - t0, t2 - t1
 
 
-def cpu_baseline(wl, layer, budget_s=20.0):
+def _oracle_shapes(O, wl, r, n_stack):
+    """(data, multiplicity) for every distinct layer shape of the workload."""
+    seen = {}
+    for layer in wl.layers:
+        key = (layer.K, layer.N)
+        if key not in seen:
+            seen[key] = [_OracleData(O, wl, layer, r), 0]
+        seen[key][1] += n_stack
+    return list(seen.values())
+
+
+def _sample_pass(O, wl, shapes, tokens, prows, step):
+    """Runs the sample of every shape once; returns (seconds spent, the
+    full-step seconds its per-token and per-row costs scale to)."""
+    spent = full = 0.0
+    for data, mult in shapes:
+        tok = min(tokens, wl.M)
+        pr = min(prows, data.layer.N)
+        tg, tp = _oracle_sample_step(O, wl, data, tok, pr, step)
+        spent += tg + tp
+        full += mult * (tg * wl.M / tok + tp * data.layer.N / pr)
+    return spent, full
+
+
+def _sample_text(wl, shapes, tokens, prows, r):
+    per = "; ".join(f"{d.layer.K}->{d.layer.N} x{m}" for d, m in shapes)
+    return (f"per layer shape ({per}), r={r}: {min(tokens, wl.M)} of {wl.M} tokens through "
+            f"quantize/fwd/dX/dB/dA and {prows} proxy rows (capped at the layer's N); the "
+            f"per-token and per-row costs are scaled to one full step of every layer")
+
+
+def cpu_baseline(wl, budget_s=20.0, r=None, n_stack=None):
     import oracle as O
 
+    r = r or wl.r
+    n_stack = n_stack or wl.n_stack
     cores = os.cpu_count() or 1
     O.set_threads(cores)
-    data = _OracleData(O, wl, layer)
+    shapes = _oracle_shapes(O, wl, r, n_stack)
     # a small probe sizes the sample to about budget_s seconds of CPU work
     tokens, prows = 64, 256
-    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 0)
-    scale = max(1.0, budget_s / max(tg + tp, 1e-6))
-    tokens = int(min(wl.M, tokens * scale))
-    prows = int(min(layer.N, prows * scale))
-    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 1)
-    # per-token and per-proxy-row costs, scaled to the full workload step
-    full_s = tg * (wl.M / tokens) + tp * (layer.N / prows)
-    return {"value": round(wl.M / full_s, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"{tokens} of {wl.M} tokens through quantize/fwd/dX/dB/dA and {prows} of "
-                       f"{layer.N} proxy rows (K={layer.K}, r={wl.r}); per-token and per-row "
-                       f"times scaled to one full step"),
-            "sample_seconds": round(tg + tp, 3)}
+    spent, _ = _sample_pass(O, wl, shapes, tokens, prows, 0)
+    scale = max(1.0, budget_s / max(spent, 1e-6))
+    tokens, prows = int(tokens * scale), int(prows * scale)
+    spent, full = _sample_pass(O, wl, shapes, tokens, prows, 1)
+    return {"value": round(wl.M / full, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": _sample_text(wl, shapes, tokens, prows, r), "sample_seconds": round(spent, 3)}
 
 
 def run_reference(args):
@@ -702,34 +877,40 @@ def run_reference(args):
     import oracle as O
 
     wl = WORKLOADS[args.workload]
-    layer = wl.layers[0]
+    r = getattr(args, "rank", 0) or wl.r
+    n_stack = getattr(args, "blocks", 0) or wl.n_stack
     cores = os.cpu_count() or 1
     O.set_threads(cores)
+    shapes = _oracle_shapes(O, wl, r, n_stack)
     tokens, prows = 16, 64
-    data = _OracleData(O, wl, layer)
     # size the per-step sample so the whole run stays within ~3 minutes
-    tg, tp = _oracle_sample_step(O, wl, layer, data, tokens, prows, 0)
+    spent, _ = _sample_pass(O, wl, shapes, tokens, prows, 0)
     budget = 150.0 / max(1, args.steps + args.warmup)
-    scale = max(0.05, min(4.0, budget / max(tg + tp, 1e-6)))
-    tokens = max(1, int(tokens * scale))
-    prows = max(1, int(prows * scale))
+    scale = max(0.05, min(4.0, budget / max(spent, 1e-6)))
+    tokens, prows = max(1, int(tokens * scale)), max(1, int(prows * scale))
     for i in range(args.warmup):
-        _oracle_sample_step(O, wl, layer, data, tokens, prows, i)
-    tot_g = tot_p = 0.0
+        _sample_pass(O, wl, shapes, tokens, prows, i)
+    tot_spent = tot_full = 0.0
     for i in range(args.steps):
-        g, p = _oracle_sample_step(O, wl, layer, data, tokens, prows, args.warmup + i)
-        tot_g += g
-        tot_p += p
-    per_step = tot_g / args.steps * (wl.M / tokens) + tot_p / args.steps * (layer.N / prows)
-    value = wl.M / per_step
-    sample = (f"{tokens} of {wl.M} tokens and {prows} of {layer.N} proxy rows per step; "
-              f"times scaled to one full step")
+        sp, fu = _sample_pass(O, wl, shapes, tokens, prows, args.warmup + i)
+        tot_spent += sp
+        tot_full += fu
+    full_step_s = tot_full / args.steps
+    value = wl.M / full_step_s
+    sample = _sample_text(wl, shapes, tokens, prows, r)
+    layer0 = wl.layers[0]
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+        "steps": args.steps, "warmup": args.warmup,
+        # what was timed: each step is the bounded sample, not a full step
+        "ms_per_step": round(tot_spent / args.steps * 1e3, 3),
+        "step": "a bounded sample of one step (see sample); value = the full step's tokens / the "
+                "sample's per-token and per-row costs scaled to the full step",
+        "full_step_ms_estimate": round(full_step_s * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": wl.name, "M": wl.M, "N": layer.N, "K": layer.K, "r": wl.r},
+        "config": {"workload": wl.name, "M": wl.M, "N": layer0.N, "K": layer0.K, "r": r,
+                   "layers": len(wl.layers) * n_stack, "blocks": n_stack},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -754,6 +935,13 @@ def main():
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--topk", type=int, default=16,
                     help="also time the top-k proxy update merging this many of the r components (0: skip)")
+    ap.add_argument("--rank", type=int, default=0, help="adapter rank (0: the workload's)")
+    ap.add_argument("--blocks", type=int, default=0,
+                    help="transformer blocks of a stacked workload (0: the workload's)")
+    ap.add_argument("--slots", type=int, default=0,
+                    help="input slots cycled by the timed steps (0: enough that their X and dY exceed "
+                         "twice the 126 MB L2, at least 2)")
+    ap.add_argument("--e2e", type=int, default=1, help="also time the step with host buffers (1) or skip it (0)")
     ap.add_argument("--only", default=None, choices=list(Step.PHASES),
                     help="run one phase alone (warm-up + steps calls) and print no bench line; "
                          "for profiler captures")
