@@ -58,6 +58,7 @@ def lib():
         L.fo_proxy_topk.restype = C.c_uint32
         L.fo_proxy_topk.argtypes = [p, C.c_float, p, p, p, i64, i64, i64, i64, C.c_int, C.c_int, p, p, p]
         L.fo_proxy_select_residual.argtypes = [p, C.c_float, p, i64, i64, p, p]
+        L.fo_matmul_f64.argtypes = [p, p, i64, i64, i64, C.c_int, p]
         L.fo_set_threads.argtypes = [C.c_int]
         L.fo_get_threads.restype = C.c_int
         _lib = L
@@ -350,6 +351,20 @@ def proxy_update(wq, s_w, P, dB_inc, A, accumulate=True, select=True, keep_resid
     if not select:
         return np.array(wq, dtype=np.uint8, copy=True), Pn, None, 0
     return proxy_select_residual(wq, s_w, Pn) if keep_residual else proxy_select(wq, s_w, Pn)
+
+
+# ------------------------------------------------------------------ C-17
+def matmul_f64(a, b, b_nk: bool) -> np.ndarray:
+    """float64 sum in index order of a[m,k] * b(k,n); b is [N, K] when b_nk,
+    else [K, N]."""
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    b = np.ascontiguousarray(b, dtype=np.float64)
+    M, K = a.shape
+    N = b.shape[0] if b_nk else b.shape[1]
+    assert (b.shape[1] if b_nk else b.shape[0]) == K
+    out = np.empty((M, N), dtype=np.float64)
+    lib().fo_matmul_f64(_ptr(a), _ptr(b), M, N, K, int(bool(b_nk)), _ptr(out))
+    return out
 
 
 from .tolerance import within_tolerance, tolerance_report  # noqa: E402,F401

@@ -149,6 +149,28 @@
 //       and U.  Y and dX are unchanged.  No new arithmetic lives here: the
 //       Python layer composes C-3, C-5, C-6, C-7 and C-8.
 //
+//  C-17 Separate LoRA paths (the comparison the pages measure, not FALQON's
+//       own path).  The introduction sets FALQON against LoRA kept as a
+//       separate path beside an FP8 backbone, whose small products pay a
+//       quantization each; the rebuttals compare FP8 and FP16 adapters
+//       across ranks (reviewer 2, W4, Table R1; reviewer 3, Q3, Table R6)
+//       and find FP8 ahead only at very large ranks.  Reading, on the same
+//       FP8 backbone (Ybb = bf16(C-5), dXbb = bf16(C-6)) with bf16 X, dY, A
+//       and B; every product is a float64 sum rounded once to bf16, and the
+//       two branches are added as bf16 tensors are (float32 add, one bf16
+//       rounding), as a separate adapter layer computes them:
+//         bf16 path:  S = bf16(X A^T), Ylora = bf16(S B^T),
+//                     G = bf16(dY B),  dXlora = bf16(G A),
+//                     dB = bf16(dY^T S), dA = bf16(G^T X),
+//                     Y = bf16(fl32(Ybb + Ylora)), dX = bf16(fl32(dXbb + dXlora)).
+//         FP8 path:   the same products with every operand quantized per
+//                     tensor (C-2, C-3) right before its product: Xq and dYq
+//                     are the backbone's, A and B are quantized each step, S
+//                     and G after they are formed; each product is the sum
+//                     of decoded codes divided by its two scales.
+//       The arithmetic is C-3, C-5 and the float64 product below; the
+//       Python layer (oracle/separate.py) composes them.
+//
 // Build: g++ -O2 -ffp-contract=off -fopenmp -shared -fPIC (see build.py).
 // -ffp-contract=off keeps every float32 multiply and add separately rounded;
 // the only fused multiply-adds are the explicit std::fmaf calls of C-9.
@@ -532,6 +554,21 @@ void fo_proxy_select_residual(uint8_t* wq, float s_w, float* P, int64_t N, int64
     count += selected ? 1 : 0;
   }
   if (n_selected) *n_selected = count;
+}
+
+// ---------------------------------------------------------------- C-17
+// out[m,n] = sum_k a[m,k] * b(k,n), float64 in index order; b is [N, K]
+// (b_nk = 1) or [K, N] (b_nk = 0).  Operands are float64 (decoded codes or
+// bfloat16 values, exact).
+void fo_matmul_f64(const double* a, const double* b, int64_t M, int64_t N, int64_t K, int b_nk, double* out) {
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < K; ++k) acc += a[m * K + k] * (b_nk ? b[n * K + k] : b[k * N + n]);
+      out[m * N + n] = acc;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- C-13
