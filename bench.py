@@ -193,9 +193,8 @@ class Step:
         self.n_slots = n_slots
         self.n_stack = n_stack or wl.n_stack
         maxdim = max(max(l.N, l.K) for l in wl.layers)
-        self.ws_q = t.empty(max(F.falqon_workspace_size(F.OP_QUANTIZE, self.M, maxdim, 0, 0),
-                                F.falqon_workspace_size(F.OP_QUANTIZE, maxdim, maxdim, 0, 0), 256),
-                            dtype=t.uint8, device=dev)
+        # one quantize workspace for every call of the step, initialised once
+        self.ws_q = F.workspace(F.OP_QUANTIZE, self.M, maxdim, device=dev)
         self.layers = [LayerState(wl, l, b, self.r, t, F, dev, self.ws_q)
                        for b in range(self.n_stack) for l in wl.layers]
         # input groups (block, x_group) in order of first use, with their K
@@ -743,8 +742,7 @@ def _time_folded(st, F, torch, stream, l2_flush, args, dev):
     bq = torch.empty((st.N, st.r), dtype=torch.uint8, device=dev)
     s_b = torch.empty(1, dtype=torch.float32, device=dev)
     amax = torch.empty(1, dtype=torch.float32, device=dev)
-    ws_b = torch.empty(max(F.falqon_workspace_size(F.OP_QUANTIZE, st.N, st.r), 256), dtype=torch.uint8,
-                       device=dev)
+    ws_b = F.workspace(F.OP_QUANTIZE, st.N, st.r, device=dev)
     t_saved = torch.empty(F.falqon_workspace_size(F.OP_FOLDED_T, st.M, 0, 0, st.r), dtype=torch.uint8,
                           device=dev)
     ws_u = torch.empty(F.falqon_workspace_size(F.OP_LINEAR_BWD_FOLDED, st.M, st.N, st.K, st.r),

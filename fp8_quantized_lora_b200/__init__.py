@@ -19,7 +19,8 @@ __all__ = [
     "FalqonError", "lib", "falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd",
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
-    "falqon_linear_bwd_folded", "folded_t_planes", "falqon_selftest_bounded_waits", "OP_QUANTIZE",
+    "falqon_linear_bwd_folded", "folded_t_planes", "falqon_selftest_bounded_waits", "falqon_workspace_init",
+    "workspace", "OP_QUANTIZE",
     "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
     "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
@@ -40,7 +41,7 @@ EXPORTED_SYMBOLS = (
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
     "falqon_linear_bwd_e5m2", "falqon_linear_fwd_folded", "falqon_linear_bwd_folded",
-    "falqon_selftest_bounded_waits",
+    "falqon_selftest_bounded_waits", "falqon_workspace_init",
 )
 
 
@@ -80,6 +81,8 @@ def lib():
     for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
               "falqon_linear_bwd_noalloc"):
         getattr(L, f).restype = C.c_int
+    L.falqon_workspace_init.argtypes = [p, sz, p]
+    L.falqon_workspace_init.restype = C.c_int
     L.falqon_workspace_size.argtypes = [C.c_int, i64, i64, i64, i64]
     L.falqon_workspace_size.restype = sz
     L.falqon_status_string.argtypes = [C.c_int]
@@ -122,14 +125,31 @@ def _check(status: int, where: str):
         raise FalqonError(status, where)
 
 
+def falqon_workspace_init(workspace, stream=None):
+    """Zero-fills a workspace (uint8 tensor, 256-byte aligned) on the stream:
+    required once for a quantize workspace before its first use."""
+    st = lib().falqon_workspace_init(_ptr(workspace), workspace.numel(), _stream(stream, workspace.device))
+    _check(st, "falqon_workspace_init")
+    return workspace
+
+
+def workspace(op, M=0, N=0, K=0, r=0, device="cuda", stream=None):
+    """A 256-byte-aligned workspace for `op` at these sizes, initialised
+    (falqon_workspace_init), or None when the op needs none."""
+    need = falqon_workspace_size(op, M, N, K, r)
+    if need == 0:
+        return None
+    raw = torch.empty(need + 256, dtype=torch.uint8, device=device)
+    off = (-raw.data_ptr()) % 256
+    return falqon_workspace_init(raw[off:off + need], stream)
+
+
 def _workspace(op, M, N, K, r, device, workspace):
     need = falqon_workspace_size(op, M, N, K, r)
     if need == 0:
         return None, 0
     if workspace is None:
-        workspace = torch.empty(need + 256, dtype=torch.uint8, device=device)
-        off = (-workspace.data_ptr()) % 256
-        workspace = workspace[off:off + need]
+        workspace = globals()["workspace"](op, M, N, K, r, device)
     return workspace, workspace.numel()
 
 

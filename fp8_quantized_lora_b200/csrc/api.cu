@@ -47,6 +47,32 @@ const DeviceInfo* current_device_info() {
   return g_info[dev].sm_count > 0 ? &g_info[dev] : nullptr;
 }
 
+falqon_status linear_bwd_validate(const uint8_t* dyq, const float* s_dy, const uint8_t* wq, const float* s_w,
+                                  const uint8_t* xq, const float* s_x, const void* A, const void* B, int64_t M,
+                                  int64_t N, int64_t K, int64_t r, const void* dx, const void* dA,
+                                  const void* dB) {
+  if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
+  if (!dyq || !s_dy) return FALQON_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256)
+    return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(dyq)) return FALQON_ERR_UNSUPPORTED;
+  if (dx) {
+    if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;
+    if (!aligned16(wq) || !aligned16(dx)) return FALQON_ERR_UNSUPPORTED;
+  }
+  if (dA || dB) {
+    if (r <= 0 || !xq || !s_x || !A) return FALQON_ERR_INVALID_ARG;
+    if (dA && !B) return FALQON_ERR_INVALID_ARG;
+    if (r % 16 != 0 || r > 65536) return FALQON_ERR_UNSUPPORTED;
+    if (!aligned16(xq) || !aligned16(A) || (B && !aligned16(B)) || (dA && !aligned16(dA)) ||
+        (dB && !aligned16(dB)))
+      return FALQON_ERR_UNSUPPORTED;
+  }
+  return FALQON_OK;
+}
+
 EncodeTiledFn encode_tiled_fn() {
   std::call_once(g_encode_once, []() {
     void* fn = nullptr;
@@ -92,6 +118,14 @@ const char* falqon_status_string(falqon_status s) {
     case FALQON_ERR_CUDA: return "CUDA error";
   }
   return "unknown status";
+}
+
+falqon_status falqon_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace || workspace_bytes == 0) return FALQON_ERR_INVALID_ARG;
+  if (!aligned256(workspace)) return FALQON_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FALQON_OK
+             : FALQON_ERR_CUDA;
 }
 
 size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r) {
@@ -180,25 +214,10 @@ falqon_status linear_bwd_call(const uint8_t* dyq, const float* s_dy, const uint8
                               const uint8_t* xq, const float* s_x, const void* A, const void* B, int64_t M,
                               int64_t N, int64_t K, int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status,
                               void* workspace, size_t workspace_bytes, void* stream, bool dy_e5m2) {
-  if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
-  if (!dyq || !s_dy) return FALQON_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
-  if (N % 16 != 0 || K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
-  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256)
-    return FALQON_ERR_UNSUPPORTED;
-  if (!aligned16(dyq)) return FALQON_ERR_UNSUPPORTED;
-  if (dx) {
-    if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;
-    if (!aligned16(wq) || !aligned16(dx)) return FALQON_ERR_UNSUPPORTED;
-  }
+  falqon_status s0 = linear_bwd_validate(dyq, s_dy, wq, s_w, xq, s_x, A, B, M, N, K, r, dx, dA, dB);
+  if (s0 != FALQON_OK) return s0;
   const bool adapters = dA || dB;
   if (adapters) {
-    if (r <= 0 || !xq || !s_x || !A) return FALQON_ERR_INVALID_ARG;
-    if (dA && !B) return FALQON_ERR_INVALID_ARG;
-    if (r % 16 != 0 || r > 65536) return FALQON_ERR_UNSUPPORTED;
-    if (!aligned16(xq) || !aligned16(A) || (B && !aligned16(B)) || (dA && !aligned16(dA)) ||
-        (dB && !aligned16(dB)))
-      return FALQON_ERR_UNSUPPORTED;
     falqon_status s =
         check_ws(adapter_workspace_bytes(M, N, K, r, dA != nullptr), workspace, workspace_bytes);
     if (s != FALQON_OK) return s;

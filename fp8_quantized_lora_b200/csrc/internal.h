@@ -7,6 +7,8 @@
 #include <cstdint>
 #include <utility>
 
+#include "../../include/falqon.h"
+
 namespace falqon {
 
 struct DeviceInfo {
@@ -82,6 +84,12 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
                                int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
 
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da);
+// Every argument check of falqon_linear_bwd except the workspace's (returns
+// the status that call would return before launching, or FALQON_OK).
+falqon_status linear_bwd_validate(const uint8_t* dyq, const float* s_dy, const uint8_t* wq, const float* s_w,
+                                  const uint8_t* xq, const float* s_x, const void* A, const void* B, int64_t M,
+                                  int64_t N, int64_t K, int64_t r, const void* dx, const void* dA,
+                                  const void* dB);
 cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const uint8_t* xq,
                                  const float* s_x, const void* A, const void* B, int64_t M,
                                  int64_t N, int64_t K, int64_t r, void* dA, void* dB,

@@ -13,10 +13,12 @@
 // The array is a file-scope __device__ object, so every GPU that loads the
 // library holds kScratchBytes of it until the process exits.  Host code may
 // not pass its name to a kernel (on the host it is a stand-in, not a device
-// address); its device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, on the first call made
-// on that device.  That first call must therefore come before any stream
-// capture on that device.
+// address); its device address is looked up with cudaGetSymbolAddress, with
+// that device current, by the first call on that device that needs scratch
+// (one asking for dA or dB) and cached.  A failed lookup is not cached: the
+// next such call tries again.  That first call must come before any stream
+// capture on that device.  A dX-only call needs no scratch and does no
+// lookup.
 //
 // Every call shares the array and it keeps whatever the last call left in
 // it; nothing in it needs to start at zero (each kernel writes every
@@ -36,11 +38,11 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_bwd_scratch[kScratchBytes];
 
-std::once_flag g_once[kMaxDevices];
-void* g_addr[kMaxDevices];
-cudaError_t g_err[kMaxDevices];
+std::mutex g_mu;
+void* g_addr[kMaxDevices];  // cached after a successful lookup only
 
-// Device address of the scratch array for the current device (set-up on first use).
+// Device address of the scratch array for the current device (looked up on
+// the first call that needs it; a failure is returned and not remembered).
 void* scratch_address(cudaError_t* err) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -48,12 +50,17 @@ void* scratch_address(cudaError_t* err) {
     *err = e != cudaSuccess ? e : cudaErrorInvalidDevice;
     return nullptr;
   }
-  std::call_once(g_once[dev], [dev]() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_addr[dev]) {
     void* p = nullptr;
-    g_err[dev] = cudaGetSymbolAddress(&p, g_bwd_scratch);
-    g_addr[dev] = g_err[dev] == cudaSuccess ? p : nullptr;
-  });
-  *err = g_err[dev];
+    e = cudaGetSymbolAddress(&p, g_bwd_scratch);
+    if (e != cudaSuccess) {
+      *err = e;
+      return nullptr;
+    }
+    g_addr[dev] = p;
+  }
+  *err = cudaSuccess;
   return g_addr[dev];
 }
 
@@ -65,12 +72,14 @@ extern "C" FALQON_API falqon_status falqon_linear_bwd_noalloc(
     const uint8_t* xq, const float* s_x, const void* A, const void* B, int64_t M, int64_t N,
     int64_t K, int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status, void* stream) {
   using namespace falqon;
-  if (dA || dB) {
-    // refuse problems whose intermediates would not fit the built-in scratch
-    if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return FALQON_ERR_INVALID_ARG;
-    if (adapter_workspace_bytes(M, N, K, r, dA != nullptr) > kScratchBytes)
-      return FALQON_ERR_WORKSPACE;
-  }
+  // the same argument checks, in the same order, as falqon_linear_bwd
+  const falqon_status s = linear_bwd_validate(dyq, s_dy, wq, s_w, xq, s_x, A, B, M, N, K, r, dx, dA, dB);
+  if (s != FALQON_OK) return s;
+  if (!dA && !dB)  // dX alone needs no scratch
+    return falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, M, N, K, r, dx, dA, dB, dev_status, nullptr, 0,
+                             stream);
+  // refuse problems whose intermediates would not fit the built-in scratch
+  if (adapter_workspace_bytes(M, N, K, r, dA != nullptr) > kScratchBytes) return FALQON_ERR_WORKSPACE;
   cudaError_t err = cudaSuccess;
   void* scratch = scratch_address(&err);
   if (!scratch) return FALQON_ERR_CUDA;

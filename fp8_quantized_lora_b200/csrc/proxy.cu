@@ -10,13 +10,14 @@
 //
 // Two launches per update (one of the first two kernels, then the clear), no
 // cross-CTA synchronisation:
-//   proxy_pipe_kernel  (accumulation with r <= 64, r % 8 == 0; persistent,
+//   proxy_ws_kernel  (accumulation with r <= 64, r % 8 == 0; persistent,
 //     two CTAs per SM) walks a contiguous range of 32 x 256 tiles of P,
-//     column block by column block, keeping the block's A columns in shared
-//     memory.  The next tile's dB_inc rows are fetched with cp.async one tile
-//     ahead; each thread's P and Wq slices of the current tile are fetched when
-//     the tile starts and land while its FMA chains run (8 rows x 8 columns per
-//     thread).  The arithmetic is the one below.
+//     column block by column block.  Four math warps run only the FMA chains
+//     (8 rows x 8 columns per thread) from A's columns and the tile's dB_inc
+//     pairs in shared memory and hand D over in shared memory; four epilogue
+//     warps stage those operands one tile ahead, hold the tile's P and Wq in
+//     registers while D is computed, and run the epilogue below.  The roles
+//     meet on mbarriers with bounded waits.  The arithmetic is the one below.
 //   proxy_stream_kernel  (grid over 32 x 256 tiles of P; two CTAs per SM;
 //     any r)
 //     Each thread owns 8 rows x 4 columns.  Its P and Wq slices stream in
@@ -209,221 +210,228 @@ __global__ void __launch_bounds__(kThreads, 2)
     atomicOr(dev_status, kDevNonfinite);
 }
 
-// ---------------------------------------------------------------- persistent pipeline
-// Tiles of 32 rows x 256 columns, four warps per CTA, two CTAs per SM: while
-// one CTA runs its epilogue (memory and integer work) the other keeps the FMA
-// pipe busy.  Warp w owns rows 8w .. 8w+7 of the tile and lane l the columns
-// 8l .. 8l+7, so every thread keeps 8 x 8 accumulators (32 packed FMAs per
-// rank against one 16-byte load of A and four broadcast loads of dB_inc pairs).
-constexpr int kPipeThreads = 128;
-constexpr int kPipeRows = 32;
-constexpr int kPipeRT = 8;                          // rows per thread
-constexpr int kPipeCT = 8;                          // columns per thread
-constexpr int kPipeRMax = 64;                       // ranks held in shared memory
-constexpr int kDbStride = kPipeRMax * 2 + 16;       // bytes per staged dB_inc row (padded)
-constexpr int kPipePBytes = kPipeRows * kTileCols * 4;            // P tile          32 KB
-constexpr int kPipeWBytes = kPipeRows * kTileCols;                // Wq tile          8 KB
-constexpr int kPipeDbBytes = kPipeRows * kDbStride;               // dB_inc rows    4.5 KB
-constexpr int kPipeAsBytes = kPipeRMax * kTileCols * 2;           // A columns       32 KB
-constexpr int kPipeBsBytes = kPipeRMax * kPipeRows * 8;           // (b, b) pairs    16 KB
-constexpr int kPipeSmemBytes =
-    kPipePBytes + kPipeWBytes + 2 * kPipeDbBytes + kPipeAsBytes + kPipeBsBytes;  // 97 KB
+// ---------------------------------------------------------------- warp-specialised pipeline
+// Persistent, two CTAs per SM, 32 x 256 tiles of P taken column block by
+// column block.  Warps 0-3 run only the float32 FMA chains: warp w owns
+// columns 64w .. 64w+63 of the tile, lane (g, c) = (l / 8, l % 8) rows
+// 8g .. 8g+7 and columns 64w + 8c .. +7, 8 x 8 accumulators per thread (32
+// packed FMAs per rank against one 16-byte load of A and two of dB_inc
+// values, whose (b, b) pairs are formed in registers).  Warps 4-7 stage the
+// operands (A's columns of the block when it changes, the (b, b) pairs of
+// the next tile's dB_inc rows), prefetch the tile's P and Wq into registers
+// and run the epilogue from D, which the math warps hand over in shared
+// memory.  The two roles meet on mbarriers whose waits are bounded.
+constexpr int kWsThreads = 256;
+constexpr int kWsRows = 32;
+constexpr int kWsRMax = 64;                                   // ranks held in shared memory
+constexpr int kWsAsBytes = kWsRMax * kTileCols * 2;           // A columns, bf16      32 KB
+constexpr int kWsBsBytes = kWsRMax * kWsRows * 4;             // dB_inc values, each   8 KB
+constexpr int kWsDBytes = kWsRows * kTileCols * 4;            // D of one tile        32 KB
+constexpr int kWsSmemBytes = kWsAsBytes + 2 * kWsBsBytes + kWsDBytes + 64;  // 80 KB + 6 mbarriers
 
 template <int kSel>
-__global__ void __launch_bounds__(kPipeThreads, 2)
-    proxy_pipe_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr,
-                      float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
-                      const uint16_t* __restrict__ A, int64_t N, int64_t K, int r, int row_groups,
-                      int units, int ncb, uint8_t* __restrict__ rowflag,
-                      int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status,
-                      int keep_residual) {
-  // No early trigger: the clear kernel that follows needs no shared memory, so
-  // its CTAs would sit beside this kernel's on the SMs while they wait.
-  pdl_wait();  // the previous kernel's results are complete and visible
-  extern __shared__ __align__(16) uint8_t sm[];
-  float4* pst = reinterpret_cast<float4*>(sm);                                 // [8][2][128]
-  uint2* wst = reinterpret_cast<uint2*>(sm + kPipePBytes);                     // [8][128]
-  uint8_t* dbraw = sm + kPipePBytes + kPipeWBytes;                             // [2][32][kDbStride]
-  uint16_t* As = reinterpret_cast<uint16_t*>(dbraw + 2 * kPipeDbBytes);       // [r][256]
-  float2* Bs = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(As) + kPipeAsBytes);  // [r][32]
+__global__ void __launch_bounds__(kWsThreads, 2)
+    proxy_ws_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr, float* __restrict__ proxy,
+                    const uint16_t* __restrict__ dB_inc, const uint16_t* __restrict__ A, int64_t N, int64_t K,
+                    int r, int row_groups, int units, int ncb, uint8_t* __restrict__ rowflag,
+                    int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status, int keep_residual) {
+  // No early trigger: the clear kernel that follows would only sit on the SMs.
+  pdl_wait();
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint16_t* As = reinterpret_cast<uint16_t*>(sm);                                     // [r][256]
+  float* Bs = reinterpret_cast<float*>(sm + kWsAsBytes);                              // [2][64][32]
+  float* Ds = reinterpret_cast<float*>(sm + kWsAsBytes + 2 * kWsBsBytes);             // [32][256]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kWsAsBytes + 2 * kWsBsBytes + kWsDBytes);
+  uint64_t* full_ops = bars;      // [2] operands of a tile staged (epilogue -> math)
+  uint64_t* empty_ops = bars + 2; // [2] a tile's operands consumed (math -> epilogue)
+  uint64_t* full_d = bars + 4;    // D of a tile written (math -> epilogue)
+  uint64_t* empty_d = bars + 5;   // D read (epilogue -> math)
+  __shared__ int abort_flag;
 
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int tr = tid >> 5;  // rows r0 + 8*tr .. +7
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int u_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * units / gridDim.x);
   const int u_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * units / gridDim.x);
   if (u_begin >= u_end) return;
-  const int chunks_per_row = r / 8;  // 16-byte chunks of one dB_inc row
+  const int ntiles = u_end - u_begin;
+  if (tid == 0) {
+    for (int b = 0; b < 6; ++b) mbar_init(bars + b, 128);
+    abort_flag = 0;
+    fence_barrier_init();
+    if (kSel == kModeSelect && n_selected && blockIdx.x == 0) *n_selected = 0;  // the clear pass counts
+  }
+  __syncthreads();
+  auto give_up = [&]() {
+    abort_flag = 1;
+    if (dev_status) atomicOr(dev_status, kDevTimeout);
+  };
 
-  auto tile_r0 = [&](int v) { return static_cast<int64_t>(v % row_groups) * kPipeRows; };
-  auto tile_col = [&](int v) {
-    return static_cast<int64_t>(v / row_groups) * kTileCols + kPipeCT * lane;
-  };
-  // this thread's P and Wq slices of tile v (read back only by this thread)
-  auto issue_pw = [&](int v) {
-    const int64_t r0 = tile_r0(v), col = tile_col(v);
-    const bool col_ok = col < K;
-#pragma unroll
-    for (int j = 0; j < kPipeRT; ++j) {
-      const int64_t n = r0 + tr * kPipeRT + j;
-      const bool ok = col_ok && n < N;
-      const float* src = ok ? proxy + n * K + col : proxy;
-      cp_async16(pst + (2 * j) * kPipeThreads + tid, src, ok ? 16u : 0u);
-      cp_async16(pst + (2 * j + 1) * kPipeThreads + tid, ok ? src + 4 : proxy, ok ? 16u : 0u);
-      if (kSel != kModeNone) {
-        const uint8_t* wsrc = ok ? wq + n * K + col : wq;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(wst + j * kPipeThreads + tid)),
-                     "l"(wsrc), "r"(ok ? 8u : 0u)
-                     : "memory");
+  if (warp < 4) {
+    // ------------------------------------------------------------ math warps
+    const int g = lane >> 3, c = lane & 7;
+    const int colw = 64 * warp + 8 * c;
+    for (int t = 0; t < ntiles; ++t) {
+      if (!mbar_wait(&full_ops[t & 1], (t >> 1) & 1, &abort_flag)) {
+        give_up();
+        break;
       }
+      float2 acc[8][4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int h = 0; h < 4; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
+      // shared-memory bytes per 32 packed FMAs are what bounds this loop: A
+      // arrives as 8 bf16 (16 bytes), the 8 rows' dB_inc values as floats (32
+      // bytes) and their (b, b) pairs are formed in registers
+      const uint16_t* arow = As + colw;
+      const float* brow = Bs + (t & 1) * (kWsRMax * kWsRows) + 8 * g;
+#pragma unroll 2
+      for (int i = 0; i < r; ++i) {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(arow + i * kTileCols);
+        const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
+        float2 av[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+          av[h] = make_float2(__uint_as_float(aw[h] << 16), __uint_as_float(aw[h] & 0xFFFF0000u));
+        const float4 q0 = *reinterpret_cast<const float4*>(brow + i * kWsRows);
+        const float4 q1 = *reinterpret_cast<const float4*>(brow + i * kWsRows + 4);
+        const float bv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 b = make_float2(bv[j], bv[j]);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) acc[j][h] = __ffma2_rn(b, av[h], acc[j][h]);
+        }
+      }
+      mbar_arrive(&empty_ops[t & 1]);
+      if (!mbar_wait(empty_d, (t & 1) ^ 1, &abort_flag)) {
+        give_up();
+        break;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4* dst = reinterpret_cast<float4*>(Ds + (8 * g + j) * kTileCols + colw);
+        dst[0] = make_float4(acc[j][0].x, acc[j][0].y, acc[j][1].x, acc[j][1].y);
+        dst[1] = make_float4(acc[j][2].x, acc[j][2].y, acc[j][3].x, acc[j][3].y);
+      }
+      mbar_arrive(full_d);
     }
-  };
-  // dB_inc rows of tile v -> dbraw[buf] (shared by the CTA)
-  auto issue_db = [&](int v, int buf) {
-    const int64_t r0 = tile_r0(v);
-    for (int e = tid; e < kPipeRows * chunks_per_row; e += kPipeThreads) {
+    return;
+  }
+
+  // -------------------------------------------------------------- epilogue warps
+  const int et = tid - 128;
+  const int ew = et >> 5;  // rows 8ew .. 8ew+7 of the tile; lane: columns 4l .. 4l+3 and 128 + 4l .. +3
+  const int chunks_per_row = r / 8;
+  auto stage = [&](int v, bool with_a) {
+    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kWsRows;
+    float* B = Bs + ((v - u_begin) & 1) * (kWsRMax * kWsRows);
+    for (int e = et; e < kWsRows * chunks_per_row; e += 128) {
       const int row = e / chunks_per_row, c8 = e % chunks_per_row;
       const int64_t n = r0 + row;
-      const bool ok = n < N;
-      cp_async16(dbraw + buf * kPipeDbBytes + row * kDbStride + 16 * c8,
-                 ok ? static_cast<const void*>(dB_inc + n * r + 8 * c8) : dB_inc, ok ? 16u : 0u);
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      if (n < N) q = *reinterpret_cast<const uint4*>(dB_inc + n * r + 8 * c8);
+      const uint32_t wds[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        B[(8 * c8 + 2 * h) * kWsRows + row] = __uint_as_float(wds[h] << 16);
+        B[(8 * c8 + 2 * h + 1) * kWsRows + row] = __uint_as_float(wds[h] & 0xFFFF0000u);
+      }
+    }
+    if (with_a) {
+      const int64_t cb = v / row_groups;
+      for (int e = et; e < r * (kTileCols / 8); e += 128) {
+        const int i = e / (kTileCols / 8), c8 = e % (kTileCols / 8);
+        const int64_t gc = cb * kTileCols + 8 * c8;
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (gc < K) q = *reinterpret_cast<const uint4*>(A + static_cast<int64_t>(i) * K + gc);
+        *reinterpret_cast<uint4*>(As + i * kTileCols + 8 * c8) = q;
+      }
     }
   };
-  // A[0:r, cb*256 : cb*256+256] -> As (zero beyond K)
-  auto issue_A = [&](int cb) {
-    for (int e = tid; e < r * (kTileCols / 8); e += kPipeThreads) {
-      const int i = e / (kTileCols / 8), c8 = e % (kTileCols / 8);
-      const int64_t gc = static_cast<int64_t>(cb) * kTileCols + 8 * c8;
-      const bool ok = gc < K;
-      cp_async16(As + i * kTileCols + 8 * c8,
-                 ok ? static_cast<const void*>(A + static_cast<int64_t>(i) * K + gc) : A,
-                 ok ? 16u : 0u);
-    }
-  };
-
-  // prologue: dB_inc rows of the first tile
-  issue_db(u_begin, 0);
-  cp_async_commit();
-
+  stage(u_begin, true);
+  mbar_arrive(&full_ops[0]);
   const float s_w = kSel != kModeNone ? *s_w_ptr : 1.0f;
-  if (kSel == kModeSelect && n_selected && blockIdx.x == 0 && threadIdx.x == 0)
-    *n_selected = 0;  // the clear pass counts
   uint32_t maxmag = 0;  // largest |P'| bit pattern: >= 0x7F800000 means inf or NaN
-  int cur_cb = -1, dbuf = 0;
-  for (int v = u_begin; v < u_end; ++v) {
-    cp_async_wait_all();  // dB_inc rows of tile v (this thread's copies)
-    __syncthreads();      // everyone's copies visible; tile v-1 finished everywhere
-    // groups, oldest first: A (empty unless the column block changes), P / Wq of
-    // tile v, dB_inc rows of tile v+1
+  for (int t = 0; t < ntiles; ++t) {
+    const int v = u_begin + t;
     const int cb = v / row_groups;
-    const bool new_block = cb != cur_cb;
-    if (new_block) issue_A(cb);
-    cp_async_commit();
-    issue_pw(v);
-    cp_async_commit();
-    if (v + 1 < u_end) issue_db(v + 1, dbuf ^ 1);
-    cp_async_commit();
-    cur_cb = cb;
-    // dB_inc rows of tile v -> (b, b) pairs, [i][row]
-    {
-      const uint8_t* raw = dbraw + dbuf * kPipeDbBytes;
-      for (int e = tid; e < kPipeRows * chunks_per_row; e += kPipeThreads) {
-        const int row = e % kPipeRows, c8 = e / kPipeRows;
-        const uint4 q = *reinterpret_cast<const uint4*>(raw + row * kDbStride + 16 * c8);
-        const uint32_t wds[4] = {q.x, q.y, q.z, q.w};
+    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kWsRows;
+    const int64_t cbase = static_cast<int64_t>(cb) * kTileCols + 4 * lane;
+    // 1. this tile's P and Wq slices, in registers while the math warps compute D
+    float4 p[8][2];
+    uint32_t w[8][2];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float f0 = __uint_as_float(wds[h] << 16);
-          const float f1 = __uint_as_float(wds[h] & 0xFFFF0000u);
-          Bs[(8 * c8 + 2 * h) * kPipeRows + row] = make_float2(f0, f0);
-          Bs[(8 * c8 + 2 * h + 1) * kPipeRows + row] = make_float2(f1, f1);
-        }
+    for (int j = 0; j < 8; ++j) {
+      const int64_t n = r0 + 8 * ew + j;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t col = cbase + 128 * h;
+        const bool ok = n < N && col < K;  // K % 16 == 0: four columns in or out together
+        p[j][h] = ok ? *reinterpret_cast<const float4*>(proxy + n * K + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+        w[j][h] = (ok && kSel != kModeNone) ? *reinterpret_cast<const uint32_t*>(wq + n * K + col) : 0u;
       }
     }
-    if (new_block) cp_async_wait_group<2>();  // this thread's share of A has landed
-    __syncthreads();                           // Bs and A complete
-
-    float2 acc[kPipeRT][4];
-#pragma unroll
-    for (int j = 0; j < kPipeRT; ++j)
-#pragma unroll
-      for (int h = 0; h < 4; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
-    const uint16_t* arow = As + kPipeCT * lane;
-    const float2* brow = Bs + tr * kPipeRT;
-#pragma unroll 4
-    for (int i = 0; i < r; ++i) {
-      const uint4 a4 = *reinterpret_cast<const uint4*>(arow + i * kTileCols);
-      const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w};
-      float2 av[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h)
-        av[h] = make_float2(__uint_as_float(aw[h] << 16), __uint_as_float(aw[h] & 0xFFFF0000u));
-#pragma unroll
-      for (int j = 0; j < kPipeRT; j += 2) {
-        const float4 q = *reinterpret_cast<const float4*>(brow + i * kPipeRows + j);
-        const float2 b0 = make_float2(q.x, q.y), b1 = make_float2(q.z, q.w);
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          acc[j][h] = __ffma2_rn(b0, av[h], acc[j][h]);
-          acc[j + 1][h] = __ffma2_rn(b1, av[h], acc[j + 1][h]);
-        }
+    // 2. operands of the next tile (its A columns only when the column block changes)
+    if (t + 1 < ntiles) {
+      const int tn = t + 1;
+      const bool new_block = (v + 1) / row_groups != cb;
+      bool ok = true;
+      if (new_block) ok = mbar_wait(&empty_ops[t & 1], (t >> 1) & 1, &abort_flag);  // As free
+      if (ok) ok = mbar_wait(&empty_ops[tn & 1], ((tn >> 1) & 1) ^ 1, &abort_flag);   // Bs[tn & 1] free
+      if (!ok) {
+        give_up();
+        break;
       }
+      stage(v + 1, new_block);
+      mbar_arrive(&full_ops[tn & 1]);
     }
-
-    // epilogue: P' = P + D; requantize; write P' and the changed codes
-    cp_async_wait_group<1>();  // P / Wq of tile v (not dB_inc of tile v+1)
-    const int64_t r0 = tile_r0(v), col = tile_col(v);
-    const bool col_ok = col < K;
+    // 3. D of this tile
+    if (!mbar_wait(full_d, t & 1, &abort_flag)) {
+      give_up();
+      break;
+    }
+    // 4. P' = P + D, requantize, write P' and the changed codes, the tile's row verdicts
+    //    (D is read row by row; the math warps need its buffer only after their next tile)
 #pragma unroll
-    for (int j = 0; j < kPipeRT; ++j) {
-      const int64_t n = r0 + tr * kPipeRT + j;  // the warp's row: uniform across the warp
+    for (int j = 0; j < 8; ++j) {
+      const int64_t n = r0 + 8 * ew + j;  // uniform across the warp
       bool changed = false;
-      if (col_ok && n < N) {
-        float4 p0 = pst[(2 * j) * kPipeThreads + tid];
-        float4 p1 = pst[(2 * j + 1) * kPipeThreads + tid];
-        p0.x = __fadd_rn(p0.x, acc[j][0].x);
-        p0.y = __fadd_rn(p0.y, acc[j][0].y);
-        p0.z = __fadd_rn(p0.z, acc[j][1].x);
-        p0.w = __fadd_rn(p0.w, acc[j][1].y);
-        p1.x = __fadd_rn(p1.x, acc[j][2].x);
-        p1.y = __fadd_rn(p1.y, acc[j][2].y);
-        p1.z = __fadd_rn(p1.z, acc[j][3].x);
-        p1.w = __fadd_rn(p1.w, acc[j][3].y);
-        float4* dst = reinterpret_cast<float4*>(proxy + n * K + col);
-        dst[0] = p0;
-        dst[1] = p1;
-        const uint32_t mg = 0x7FFFFFFFu;
-        maxmag = max(maxmag, max(max(max(__float_as_uint(p0.x) & mg, __float_as_uint(p0.y) & mg),
-                                     max(__float_as_uint(p0.z) & mg, __float_as_uint(p0.w) & mg)),
-                                 max(max(__float_as_uint(p1.x) & mg, __float_as_uint(p1.y) & mg),
-                                     max(__float_as_uint(p1.z) & mg, __float_as_uint(p1.w) & mg))));
-        if constexpr (kSel != kModeNone) {
-          const uint2 w = wst[j * kPipeThreads + tid];
-          const uint32_t c0 = requantized4(w.x, s_w, p0);
-          const uint32_t c1 = requantized4(w.y, s_w, p1);
-          // identical words change only where they hold NaN codes (the common case)
-          const uint32_t m0 = c0 == w.x ? nan_bytes(w.x) : changed_bytes(w.x, c0);
-          const uint32_t m1 = c1 == w.y ? nan_bytes(w.y) : changed_bytes(w.y, c1);
-          if (m0 | m1) {
-            *reinterpret_cast<uint2*>(wq + n * K + col) =
-                make_uint2((c0 & m0) | (w.x & ~m0), (c1 & m1) | (w.y & ~m1));
-            changed = true;
-            if (keep_residual) {
-              dst[0] = residual4(p0, w.x, c0, m0, s_w);
-              dst[1] = residual4(p1, w.y, c1, m1, s_w);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t col = cbase + 128 * h;
+        const float4 dv = *reinterpret_cast<const float4*>(Ds + (8 * ew + j) * kTileCols + 4 * lane + 128 * h);
+        if (n < N && col < K) {
+          float4 q = p[j][h];
+          q.x = __fadd_rn(q.x, dv.x);
+          q.y = __fadd_rn(q.y, dv.y);
+          q.z = __fadd_rn(q.z, dv.z);
+          q.w = __fadd_rn(q.w, dv.w);
+          const uint32_t mg = 0x7FFFFFFFu;
+          maxmag = max(maxmag, max(max(__float_as_uint(q.x) & mg, __float_as_uint(q.y) & mg),
+                                   max(__float_as_uint(q.z) & mg, __float_as_uint(q.w) & mg)));
+          float4 out = q;
+          if constexpr (kSel != kModeNone) {
+            const uint32_t wv = w[j][h];
+            const uint32_t cn = requantized4(wv, s_w, q);
+            // identical words change only where they hold NaN codes (the common case)
+            const uint32_t m = cn == wv ? nan_bytes(wv) : changed_bytes(wv, cn);
+            if (m) {
+              *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (wv & ~m);
+              changed = true;
+              if (keep_residual) out = residual4(q, wv, cn, m, s_w);
             }
           }
+          *reinterpret_cast<float4*>(proxy + n * K + col) = out;
         }
       }
       if constexpr (kSel == kModeSelect) {
         // the tile's verdict for row n, written whether or not a code changed
         const bool any = __any_sync(0xFFFFFFFFu, changed);
-        if (lane == 0 && n < N) rowflag[n * ncb + v / row_groups] = any ? 1 : 0;
+        if (lane == 0 && n < N) rowflag[n * ncb + cb] = any ? 1 : 0;
       }
     }
-    dbuf ^= 1;
+    mbar_arrive(empty_d);
   }
-  cp_async_wait_all();
   if (__any_sync(0xFFFFFFFFu, maxmag >= 0x7F800000u) && lane == 0 && dev_status)
     atomicOr(dev_status, kDevNonfinite);
 }
@@ -495,12 +503,12 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   cudaGetDevice(&dev);
   const int bit = dev < 31 ? (1 << dev) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(proxy_pipe_kernel<kSel>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPipeSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(proxy_ws_kernel<kSel>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kWsSmemBytes);
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
   }
-  return launch_pdl(proxy_pipe_kernel<kSel>, dim3(grid), dim3(kPipeThreads), kPipeSmemBytes, stream, 1u, wq,
+  return launch_pdl(proxy_ws_kernel<kSel>, dim3(grid), dim3(kWsThreads), kWsSmemBytes, stream, 1u, wq,
                     s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
                     row_groups, units, ncb, rowflag, n_selected, dev_status, keep_residual);
 }
@@ -524,12 +532,12 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
                   static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
   const int rr = acc ? static_cast<int>(r) : 0;
-  const int64_t row_groups = (N + kPipeRows - 1) / kPipeRows;
+  const int64_t row_groups = (N + kWsRows - 1) / kWsRows;
   const int64_t units = row_groups * grid.x;
   // the persistent kernel accumulates with A and dB_inc slices of up to 64
   // ranks held in 16-byte chunks; selection alone streams through the grid kernel
-  const bool pipe = acc && rr >= 1 && rr <= kPipeRMax && rr % 8 == 0 &&
-                    units <= (int64_t(1) << 30) && di->max_smem_optin >= kPipeSmemBytes;
+  const bool pipe = acc && rr >= 1 && rr <= kWsRMax && rr % 8 == 0 &&
+                    units <= (int64_t(1) << 30) && di->max_smem_optin >= kWsSmemBytes;
   if (!pipe && grid.y > 65535u) return cudaErrorInvalidValue;
   // per (row, 256-column block) verdicts, each written by the tile that owns it:
   // nothing to clear beforehand

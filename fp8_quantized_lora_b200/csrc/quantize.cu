@@ -304,6 +304,8 @@ constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
 constexpr int kBarWords = 64;                          // per-CTA words start 256 bytes in
+constexpr int kExchangeWords = 4096;                   // generation + 64-bit words of at most 2016 CTAs
+constexpr int kPartialWords = 1024;                    // two-launch path: its per-CTA partial maxima
 constexpr long long kBarrierBudget = 2000000000LL;    // cycles (about 1 s), then give up
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -348,6 +350,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   __syncthreads();
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // (no-op: this launch is cooperative and waits in order)
+  // this call's generation of the exchange words (see the exchange below)
+  const uint32_t gen = *reinterpret_cast<volatile const uint32_t*>(ws);
 
   int stage = 0;
   uint32_t phase = 0;
@@ -427,18 +431,21 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   m = block_max_u32(m, red);
 
   // Grid exchange of the per-CTA maxima (the launch is cooperative, so every
-  // CTA is resident).  A CTA's word is its max with bit 31 set as the arrival
-  // mark (a magnitude pattern never has it); the words were zeroed before the
-  // launch.  Warp 0 of every CTA polls all words (relaxed loads, one acquire
-  // fence once all are marked), bounded, and reduces them.  A poll round
-  // issues all of a lane's loads before it looks at any: one L2 round trip
-  // per round, not one per word.
-  uint32_t* partials = ws + kBarWords;
+  // CTA is resident).  The workspace holds a generation counter g (word 0)
+  // and one 64-bit word per CTA.  Every CTA read g at its start; it publishes
+  // (g + 1) << 32 | max with a release store, and warp 0 of every CTA polls
+  // all words (relaxed loads, one acquire fence once all carry the tag
+  // g + 1), bounded, and reduces them.  Words left by earlier calls carry
+  // older tags, so nothing is cleared between calls; CTA 0 advances g once
+  // its own exchange is over (or its wait ran out), after every CTA has read
+  // it.  A poll round issues all of a lane's loads before it looks at any:
+  // one L2 round trip per round, not one per word.
+  uint64_t* words = reinterpret_cast<uint64_t*>(ws + kBarWords);
+  const uint64_t tag = static_cast<uint64_t>(gen + 1u) << 32;
   __shared__ uint32_t amax_bits;
   if (warp == 0) {
     if (lane == 0)
-      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(partials + blockIdx.x), "r"(m | 0x80000000u)
-                   : "memory");
+      asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(words + blockIdx.x), "l"(tag | m) : "memory");
     __syncwarp();
     const long long t0 = clock64();
     uint32_t mx = 0;
@@ -447,22 +454,22 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       bool all = true;
       mx = 0;
       for (int b = 0; b < static_cast<int>(gridDim.x); b += 32 * kPerLane) {
-        uint32_t w[kPerLane];
+        uint64_t w[kPerLane];
 #pragma unroll
         for (int k = 0; k < kPerLane; ++k) {
           const int i = b + lane + 32 * k;
-          w[k] = 0x80000000u;  // absent CTAs count as arrived with max 0
+          w[k] = tag;  // absent CTAs count as arrived with max 0
           if (i < static_cast<int>(gridDim.x))
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(w[k]) : "l"(partials + i));
+            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w[k]) : "l"(words + i));
         }
 #pragma unroll
         for (int k = 0; k < kPerLane; ++k) {
-          all = all && (w[k] >> 31) != 0u;
-          mx = max(mx, w[k] & 0x7FFFFFFFu);
+          all = all && (w[k] & 0xFFFFFFFF00000000ull) == tag;
+          mx = max(mx, static_cast<uint32_t>(w[k]));
         }
       }
       if (__all_sync(0xFFFFFFFFu, all)) {
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the marked words
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the tagged words
         break;
       }
       if (clock64() - t0 > kBarrierBudget) {
@@ -471,7 +478,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
       }
     }
     mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) amax_bits = mx;
+    if (lane == 0) {
+      amax_bits = mx;
+      if (blockIdx.x == 0)  // every CTA has read the generation: the next call may use the next one
+        asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(ws), "r"(gen + 1u) : "memory");
+    }
   }
   __syncthreads();
   const float s = scale_from_amax(amax_bits, kFmtMax<kE5>, &s_shared, scale_out, amax_out, dev_status);
@@ -554,7 +565,8 @@ constexpr int64_t kSmallTensor = int64_t(1) << 20;  // elements
 int amax_blocks(int64_t n, int sm_count) {
   const int64_t per_block = static_cast<int64_t>(kThreads) * 64;  // >= 64 elements per thread
   int64_t b = (n + per_block - 1) / per_block;
-  const int64_t cap = static_cast<int64_t>(sm_count) * 4;
+  int64_t cap = static_cast<int64_t>(sm_count) * 4;
+  if (cap > kPartialWords) cap = kPartialWords;
   if (b > cap) b = cap;
   if (b < 1) b = 1;
   return static_cast<int>(b);
@@ -564,7 +576,10 @@ int amax_blocks(int64_t n, int sm_count) {
 
 size_t quantize_workspace_bytes(int64_t n) {
   (void)n;
-  return 4096 * sizeof(uint32_t);  // barrier words + amax partials (at most 4032 CTAs)
+  // the generation word and the 64-bit exchange words of the one-launch
+  // path, then the partial maxima of the two-launch path (a region of its
+  // own, so that a small tensor never disturbs the exchange's generation)
+  return static_cast<size_t>(kExchangeWords + kPartialWords) * sizeof(uint32_t);
 }
 
 namespace {
@@ -590,9 +605,7 @@ cudaError_t launch_quantize_t(const DeviceInfo* di, const void* x, int64_t n, ui
     const int64_t body = (n * (kBF16 ? 2 : 4)) / 16 * 16;
     int64_t chunks = (body + kChunkBytes - 1) / kChunkBytes;
     int grid = static_cast<int>(chunks < di->sm_count ? (chunks > 0 ? chunks : 1) : di->sm_count);
-    if (grid > 4096 - kBarWords) grid = 4096 - kBarWords;
-    cudaError_t e = cudaMemsetAsync(ws + kBarWords, 0, static_cast<size_t>(grid) * sizeof(uint32_t), stream);
-    if (e != cudaSuccess) return e;
+    if (grid > (kExchangeWords - kBarWords) / 2) grid = (kExchangeWords - kBarWords) / 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kStreamThreads);
@@ -606,7 +619,7 @@ cudaError_t launch_quantize_t(const DeviceInfo* di, const void* x, int64_t n, ui
     return cudaLaunchKernelEx(&cfg, quantize_stream_kernel<kBF16, kE5>, x, n, ws, codes, scale, amax, residual,
                               dev_status);
   }
-  uint32_t* partials = ws;
+  uint32_t* partials = ws + kExchangeWords;
   const int pb = amax_blocks(n, di->sm_count);
   const int64_t per_cast_block = static_cast<int64_t>(kThreads) * 16 * 4;
   int64_t cb = (n + per_cast_block - 1) / per_cast_block;

@@ -29,7 +29,8 @@
 //   topk_merge_kernel   persistent, 32 x 256 tiles of Wq taken column block
 //                       by column block, the chosen rows of A for the block
 //                       kept in shared memory, the chosen Q entries of the
-//                       tile's rows staged as duplicated float pairs; each
+//                       next tile's rows fetched one tile ahead and expanded
+//                       into duplicated float pairs; each
 //                       thread holds 8 rows x 8 columns of D (packed FMAs)
 //                       and writes the codes whose value changes.  2 N K k
 //                       flops and one pass over Wq.
@@ -58,8 +59,9 @@ constexpr int kMChunk = 64;     // components staged per pass
 constexpr int kMCtasPerSm = 3;
 constexpr int kMAsBytes = kMChunk * kMCols * 2;  // chosen rows of A, bf16    32 KB
 constexpr int kMBsBytes = kMChunk * kMRows * 8;  // (q, q) pairs              16 KB
+constexpr int kMQBytes = 2 * kMChunk * kMRows * 4;  // raw Q entries, two tiles  16 KB
 constexpr int kMWBytes = kMRT * kMThreads * 8;   // this thread's Wq slices    8 KB
-constexpr int kMSmemBytes = kMAsBytes + kMBsBytes + kMWBytes;  // 56 KB
+constexpr int kMSmemBytes = kMAsBytes + kMBsBytes + kMQBytes + kMWBytes;  // 72 KB
 
 constexpr int kClearThreads = 256;
 
@@ -93,19 +95,28 @@ __global__ void __launch_bounds__(kAccThreads)
     __syncthreads();
     const int nn = tid % kAccN;
     const int64_t n = n0 + nn;
-    // warp w covers half a row of the tile: the component index is uniform across the warp
-    for (int ii = tid / kAccN; ii < kAccI; ii += kAccThreads / kAccN) {
+    // warp w covers half a row of the tile: the component index is uniform
+    // across the warp.  All of a thread's loads are issued before any use.
+    constexpr int kPer = kAccI / (kAccThreads / kAccN);
+    float v[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int i = i0 + tid / kAccN + q * (kAccThreads / kAccN);
+      v[q] = (i < r && n < N) ? Q[static_cast<int64_t>(i) * N + n] : 0.0f;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int ii = tid / kAccN + q * (kAccThreads / kAccN);
       const int i = i0 + ii;
-      uint32_t m = 0u;
-      if (i < r && n < N) {
-        float* q = Q + static_cast<int64_t>(i) * N + n;
-        float v = *q;
-        if (accumulate) {
-          v = __fadd_rn(v, tile[ii][nn]);
-          *q = v;
-        }
-        m = __float_as_uint(v) & 0x7FFFFFFFu;  // NaN patterns lie above infinity's
+      if (accumulate && i < r && n < N) {
+        v[q] = __fadd_rn(v[q], tile[ii][nn]);
+        Q[static_cast<int64_t>(i) * N + n] = v[q];
       }
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int ii = tid / kAccN + q * (kAccThreads / kAccN);
+      uint32_t m = __float_as_uint(v[q]) & 0x7FFFFFFFu;  // NaN patterns lie above infinity's
       m = __reduce_max_sync(0xFFFFFFFFu, m);
       if ((tid & 31) == 0 && m) atomicMax(&qmax[ii], m);
     }
@@ -225,68 +236,83 @@ __global__ void __launch_bounds__(kMThreads, kMCtasPerSm)
   const int ns = *n_sel;
   if (ns <= 0) return;
   extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kMChunk][256]
-  float2* Bs = reinterpret_cast<float2*>(sm + kMAsBytes);                      // [kMChunk][32]
-  uint2* wst = reinterpret_cast<uint2*>(sm + kMAsBytes + kMBsBytes);           // [8][128]
+  uint16_t* As = reinterpret_cast<uint16_t*>(sm);                                   // [kMChunk][256]
+  float2* Bs = reinterpret_cast<float2*>(sm + kMAsBytes);                           // [kMChunk][32]
+  float* qraw = reinterpret_cast<float*>(sm + kMAsBytes + kMBsBytes);               // [2][kMChunk][32]
+  uint2* wst = reinterpret_cast<uint2*>(sm + kMAsBytes + kMBsBytes + kMQBytes);     // [8][128]
+  __shared__ int s_sel[kMChunk];  // the chosen components of the first chunk
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int tr = tid >> 5;
   const int u_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * units / gridDim.x);
   const int u_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * units / gridDim.x);
+  if (u_begin >= u_end) return;
+  const int n0c = ns < kMChunk ? ns : kMChunk;  // components of the first chunk
+  for (int j = tid; j < n0c; j += kMThreads) s_sel[j] = sel[j];
+  __syncthreads();
+  // Q entries of the first chunk for the rows of tile v -> qraw[buf] (one tile ahead)
+  auto issue_q = [&](int v, int buf) {
+    const int64_t r0 = static_cast<int64_t>(v % row_groups) * kMRows;
+    float* dst = qraw + buf * (kMChunk * kMRows);
+    for (int e = tid; e < n0c * kMRows; e += kMThreads) {
+      const int j = e / kMRows, row = e % kMRows;
+      const int64_t n = r0 + row;
+      const bool ok = n < N;
+      cp_async4(dst + e, ok ? static_cast<const void*>(Q + static_cast<int64_t>(s_sel[j]) * N + n) : Q,
+                ok ? 4u : 0u);
+    }
+  };
+  issue_q(u_begin, 0);
+  cp_async_commit();
   const float s_w = *s_w_ptr;
   int cur_cb = -1;
   for (int v = u_begin; v < u_end; ++v) {
+    const int buf = (v - u_begin) & 1;
     const int cb = v / row_groups;
     const int64_t r0 = static_cast<int64_t>(v % row_groups) * kMRows;
     const int64_t c0 = static_cast<int64_t>(cb) * kMCols;
     const int64_t col = c0 + 8 * lane;
     const bool col_ok = col < K;  // K % 16 == 0: the 8 columns are in or out together
+    cp_async_wait_all();  // this thread's copies of tile v's Q entries
+    __syncthreads();      // everyone's copies visible; the previous tile's FMA loop is done everywhere
+    // groups, oldest first: A of the first chunk (empty while it stays), Wq slices of
+    // tile v, Q entries of tile v+1
+    if (ns > kMChunk || cb != cur_cb) {
+      for (int e = tid; e < n0c * (kMCols / 8); e += kMThreads) {
+        const int j = e / (kMCols / 8), c8 = e % (kMCols / 8);
+        const int64_t gc = c0 + 8 * c8;
+        const bool ok = gc < K;
+        cp_async16(As + j * kMCols + 8 * c8,
+                   ok ? static_cast<const void*>(A + static_cast<int64_t>(s_sel[j]) * K + gc) : A, ok ? 16u : 0u);
+      }
+    }
+    cp_async_commit();
+#pragma unroll
+    for (int j = 0; j < kMRT; ++j) {
+      const int64_t n = r0 + tr * kMRT + j;
+      const bool ok = col_ok && n < N;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(wst + j * kMThreads + tid)),
+                   "l"(ok ? wq + n * K + col : wq), "r"(ok ? 8u : 0u)
+                   : "memory");
+    }
+    cp_async_commit();
+    if (v + 1 < u_end) issue_q(v + 1, buf ^ 1);
+    cp_async_commit();
+    // (q, q) pairs of the first chunk, [j][row]
+    const float* qsrc = qraw + buf * (kMChunk * kMRows);
+    for (int e = tid; e < n0c * kMRows; e += kMThreads) Bs[e] = make_float2(qsrc[e], qsrc[e]);
+    cp_async_wait_group<2>();  // A of the first chunk
+    __syncthreads();           // As and Bs complete
+    cur_cb = cb;
 
     float2 acc[kMRT][4];
 #pragma unroll
     for (int j = 0; j < kMRT; ++j)
 #pragma unroll
       for (int h = 0; h < 4; ++h) acc[j][h] = make_float2(0.0f, 0.0f);
-
-    for (int j0 = 0; j0 < ns; j0 += kMChunk) {
-      const int nj = ns - j0 < kMChunk ? ns - j0 : kMChunk;
-      __syncthreads();  // every thread is done with As and Bs
-      // the chosen rows of A for this column block (kept while the block and the chunk stay)
-      if (ns > kMChunk || cb != cur_cb) {
-        for (int e = tid; e < nj * (kMCols / 8); e += kMThreads) {
-          const int j = e / (kMCols / 8), c8 = e % (kMCols / 8);
-          const int64_t gc = c0 + 8 * c8;
-          const bool ok = gc < K;
-          const int64_t i = sel[j0 + j];
-          cp_async16(As + j * kMCols + 8 * c8, ok ? static_cast<const void*>(A + i * K + gc) : A, ok ? 16u : 0u);
-        }
-      }
-      cp_async_commit();
-      if (j0 == 0) {
-        // this thread's Wq slices of the tile land while the FMA chains run
-#pragma unroll
-        for (int j = 0; j < kMRT; ++j) {
-          const int64_t n = r0 + tr * kMRT + j;
-          const bool ok = col_ok && n < N;
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(wst + j * kMThreads + tid)),
-                       "l"(ok ? wq + n * K + col : wq), "r"(ok ? 8u : 0u)
-                       : "memory");
-        }
-        cp_async_commit();
-      }
-      // Q[sel[j0 + j], r0 + row] as (q, q) pairs, [j][row]
-      for (int e = tid; e < nj * kMRows; e += kMThreads) {
-        const int j = e / kMRows, row = e % kMRows;
-        const int64_t n = r0 + row;
-        const float q = n < N ? Q[static_cast<int64_t>(sel[j0 + j]) * N + n] : 0.0f;
-        Bs[j * kMRows + row] = make_float2(q, q);
-      }
-      if (j0 == 0)
-        cp_async_wait_group<1>();  // A (the Wq slices may still be in flight)
-      else
-        cp_async_wait_all();
-      __syncthreads();  // As and Bs complete
+    int nj = n0c;
+    for (int j0 = 0;;) {
       const uint16_t* arow = As + 8 * lane;
       const float2* brow = Bs + tr * kMRT;
 #pragma unroll 4
@@ -308,9 +334,29 @@ __global__ void __launch_bounds__(kMThreads, kMCtasPerSm)
           }
         }
       }
+      j0 += nj;
+      if (j0 >= ns) break;
+      // a further chunk of components (more than kMChunk chosen): staged in place
+      nj = ns - j0 < kMChunk ? ns - j0 : kMChunk;
+      __syncthreads();  // every thread is done with As and Bs
+      for (int e = tid; e < nj * (kMCols / 8); e += kMThreads) {
+        const int j = e / (kMCols / 8), c8 = e % (kMCols / 8);
+        const int64_t gc = c0 + 8 * c8;
+        const bool ok = gc < K;
+        const int64_t i = sel[j0 + j];
+        cp_async16(As + j * kMCols + 8 * c8, ok ? static_cast<const void*>(A + i * K + gc) : A, ok ? 16u : 0u);
+      }
+      cp_async_commit();
+      for (int e = tid; e < nj * kMRows; e += kMThreads) {
+        const int j = e / kMRows, row = e % kMRows;
+        const int64_t n = r0 + row;
+        const float q = n < N ? Q[static_cast<int64_t>(sel[j0 + j]) * N + n] : 0.0f;
+        Bs[j * kMRows + row] = make_float2(q, q);
+      }
+      cp_async_wait_all();
+      __syncthreads();
     }
-    cur_cb = cb;
-    cp_async_wait_all();  // this thread's Wq slices
+    cp_async_wait_group<1>();  // this thread's Wq slices (tile v+1's Q entries may still be in flight)
 #pragma unroll
     for (int j = 0; j < kMRT; ++j) {
       const int64_t n = r0 + tr * kMRT + j;
@@ -327,6 +373,7 @@ __global__ void __launch_bounds__(kMThreads, kMCtasPerSm)
         *reinterpret_cast<uint2*>(wq + n * K + col) = make_uint2((c0w & m0) | (w.x & ~m0), (c1w & m1) | (w.y & ~m1));
     }
   }
+  cp_async_wait_all();
 }
 
 __global__ void __launch_bounds__(kClearThreads)

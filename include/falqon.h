@@ -32,6 +32,13 @@
  *    when that size is 0.  Calls that overlap on the GPU must not share a
  *    workspace.  No other aliasing between arguments is allowed except the
  *    documented in-place operands of falqon_proxy_update.
+ *  - A workspace given to falqon_quantize or falqon_quantize_e5m2 must be
+ *    initialised once, before its first use, by falqon_workspace_init (or
+ *    filled with zero bytes by the caller).  Every quantize call leaves it
+ *    initialised for the next, whatever the size of the tensor and
+ *    whether or not a bounded wait ran out (FALQON_DEV_TIMEOUT): the calls
+ *    keep a generation counter in it instead of clearing it, so no clearing
+ *    step runs per call.  Other workspaces need no initialisation.
  *  - Every function is reentrant; the only global state is a per-device
  *    cache of device attributes and of the driver's tensor-map encoder.
  */
@@ -338,13 +345,16 @@ FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w,
  * intermediates in one scratch array compiled into the library.
  *
  *  - Limit: the scratch array is 16 MiB per device, held by every GPU that
- *    loads the library until the process exits.  A call whose
- *    falqon_workspace_size(FALQON_OP_LINEAR_BWD, M, N, K, r) exceeds it (with
- *    dA requested; slightly less without) returns FALQON_ERR_WORKSPACE before
- *    launching anything.  A dX-only call needs no scratch.
- *  - Set-up: the first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, once per device); make that first call before
- *    any stream capture on that device.
+ *    loads the library until the process exits.  A call asking for dA or dB
+ *    needs 4 * align256(round_up(M, 8) * r * 2) bytes of it (the same with or
+ *    without dA; falqon_workspace_size(FALQON_OP_LINEAR_BWD, M, N, K, r));
+ *    beyond 16 MiB it returns FALQON_ERR_WORKSPACE before launching
+ *    anything.  Every other argument error is reported first, exactly as
+ *    falqon_linear_bwd reports it.  A dX-only call needs no scratch.
+ *  - Set-up: the first call on a device that needs scratch looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture on that device.  A failed lookup
+ *    returns FALQON_ERR_CUDA and is not cached: a later call tries again.
  *  - Sharing: every call uses the same array, which keeps the last call's
  *    contents (nothing in it needs to start at zero).  Calls that overlap on
  *    the GPU race on it; serialise them.
@@ -377,6 +387,15 @@ FALQON_API falqon_status falqon_linear_bwd_noalloc(const uint8_t* dyq, const flo
  */
 FALQON_API falqon_status falqon_selftest_bounded_waits(const int32_t* flag, int32_t* dev_status,
                                                        int32_t* which, void* stream);
+
+/*
+ * falqon_workspace_init - prepares a workspace for its first use: fills
+ * `workspace_bytes` bytes with zeros on `stream` (asynchronous).  Required
+ * once for a quantize workspace (see the conventions above); harmless for
+ * any other.  Errors: NULL or 0 bytes -> FALQON_ERR_INVALID_ARG; not 256-byte
+ * aligned -> FALQON_ERR_WORKSPACE; the fill failed -> FALQON_ERR_CUDA.
+ */
+FALQON_API falqon_status falqon_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Workspace bytes `op` needs for these sizes (arguments an op ignores may be 0). */
 FALQON_API size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int64_t r);

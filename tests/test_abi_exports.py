@@ -177,3 +177,31 @@ def test_binding_refuses_cpu_tensors(name):
             F.falqon_quantize(x)
         else:
             F.falqon_linear_fwd(x.to(torch.uint8), torch.ones(1), x.to(torch.uint8), torch.ones(1))
+
+
+def test_noalloc_reports_argument_errors_like_the_workspace_call():
+    """The no-allocation backward runs falqon_linear_bwd's argument checks
+    before its own scratch-size check: the same bad arguments give the same
+    status, even on a problem too large for its scratch."""
+    L = F.lib()
+    bwd, na = L.falqon_linear_bwd, L.falqon_linear_bwd_noalloc
+    big = 1 << 40  # a workspace size that never limits falqon_linear_bwd's checks
+
+    def both(M, N, K, r, dx=P, dA=P, dB=P, A=P, dyq=P):
+        s1 = bwd(dyq, P, P, P, P, P, A, P, M, N, K, r, dx, dA, dB, None, P, big, None)
+        s2 = na(dyq, P, P, P, P, P, A, P, M, N, K, r, dx, dA, dB, None, None)
+        return s1, s2
+    M = 32768  # with r = 256 the intermediates need 64 MiB, beyond the 16 MiB scratch
+    assert both(M, 256, 256, 24) == (2, 2)            # r % 16: UNSUPPORTED first
+    assert both(M, 256, 256, 256, A=None) == (1, 1)   # no A: INVALID_ARG first
+    assert both(M, 250, 256, 256) == (2, 2)           # N % 16
+    assert both(M, 256, 256, 256, dyq=P8) == (2, 2)   # unaligned codes
+    assert both(M, 256, 256, 256, dx=None, dA=None, dB=None) == (1, 1)
+    assert na(P, P, P, P, P, P, P, P, M, 256, 256, 256, P, P, P, None, None) == 3  # then the scratch limit
+
+
+def test_workspace_init_argument_errors():
+    L = F.lib()
+    assert L.falqon_workspace_init(None, 256, None) == 1   # no workspace
+    assert L.falqon_workspace_init(P, 0, None) == 1        # no bytes
+    assert L.falqon_workspace_init(P8, 256, None) == 3     # not 256-byte aligned

@@ -129,7 +129,7 @@ def test_every_fp32_pattern_up_to_448_encodes_like_the_oracle(cuda_device):
     chunk = 1 << 27
     dev = torch.device("cuda:0")
     st = status_word()
-    ws = torch.empty(F.falqon_workspace_size(F.OP_QUANTIZE, 1, chunk + 16), dtype=torch.uint8, device=dev)
+    ws = F.workspace(F.OP_QUANTIZE, 1, chunk + 16, device=dev)  # initialised once, reused by every call
     pool = ThreadPoolExecutor(max_workers=16)
 
     def oracle_codes(f):
@@ -151,4 +151,42 @@ def test_every_fp32_pattern_up_to_448_encodes_like_the_oracle(cuda_device):
         np.testing.assert_array_equal(host(codes).reshape(-1)[: len(pats)], oracle_codes(pats.view(np.float32)),
                                       err_msg=hex(lo))
     pool.shutdown()
+    assert int(st.item()) == 0
+
+
+def test_one_workspace_reused_across_sizes_and_graph_replays(cuda_device):
+    """The workspace contract: initialised once, then reused by calls of both
+    paths (small tensors take the two-launch path, large ones the exchange
+    with its generation counter) and by replays of a captured graph; every
+    call's scale and codes equal the oracle's."""
+    dev = torch.device("cuda:0")
+    ws = F.workspace(F.OP_QUANTIZE, 1, 16, device=dev)
+    st = status_word()
+    shapes = [(4096, 1024), (64, 64), (2048, 2048), (4096, 1024), (512, 512), (8192, 512)]
+    for i, shape in enumerate(shapes):
+        x = gen.normal_bf16_bits(500 + i, shape, 10.0 ** (i % 3 - 1))
+        codes, s, _ = F.falqon_quantize(dev_bf16(x), dev_status=st, workspace=ws)
+        rc, rs, _, _ = O.quantize(x)
+        torch.cuda.synchronize()
+        assert float(s.item()) == float(rs), shape
+        np.testing.assert_array_equal(host(codes), rc)
+    # a captured quantize replayed on changing data reuses the same workspace words
+    xs = dev_bf16(gen.normal_bf16_bits(600, (4096, 1024), 1.0))
+    codes = torch.empty(xs.shape, dtype=torch.uint8, device=dev)
+    scale = torch.empty(1, dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        F.falqon_quantize(xs, codes=codes, scale=scale, dev_status=st, workspace=ws)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        F.falqon_quantize(xs, codes=codes, scale=scale, dev_status=st, workspace=ws)
+    for k in range(5):
+        x = gen.normal_bf16_bits(700 + k, (4096, 1024), 2.0 ** (k - 2))
+        xs.copy_(dev_bf16(x))
+        g.replay()
+        torch.cuda.synchronize()
+        rc, rs, _, _ = O.quantize(x)
+        assert float(scale.item()) == float(rs), k
+        np.testing.assert_array_equal(host(codes), rc)
     assert int(st.item()) == 0

@@ -52,6 +52,44 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_device, M, N, K, r):
             _same(g, rr)
 
 
+@pytest.mark.parametrize("outputs", ["dx", "dA", "dB", "dA+dB", "dx+dB"])
+def test_noalloc_output_subsets_after_a_full_call(cuda_device, outputs):
+    """A call asking for only some outputs, right after a full call on other
+    data: the half of the shared scratch it does not write still holds the
+    first call's values, and must not leak into its results."""
+    M, N, K, r = 520, 272, 336, 48
+    full = _inputs(101, M, N, K, r)
+    F.falqon_linear_bwd_noalloc(*full)
+    args = _inputs(202, M, N, K, r)
+    want = {k: (k in outputs.split("+")) for k in ("dx", "dA", "dB")}
+    st1, st2 = status_word(), status_word()
+    ref = F.falqon_linear_bwd(*args, dx=want["dx"], dA=want["dA"], dB=want["dB"], dev_status=st1)
+    got = F.falqon_linear_bwd_noalloc(*args, dx=want["dx"], dA=want["dA"], dB=want["dB"], dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st1.item()) == 0 and int(st2.item()) == 0
+    for name, g, rr in zip(("dx", "dA", "dB"), got, ref):
+        assert (g is None) == (not want[name]) and (rr is None) == (not want[name])
+        if g is not None:
+            _same(g, rr)
+
+
+def test_noalloc_shape_just_under_the_scratch_limit(cuda_device):
+    """M = 32760, r = 64: four planes of 32760 x 64 bf16 take 16 773 120 bytes
+    of the 16 777 216-byte scratch (4 KiB short of it)."""
+    M, N, K, r = 32760, 256, 256, 64
+    need = F.falqon_workspace_size(F.OP_LINEAR_BWD, M, N, K, r)
+    assert need == (16 << 20) - 4096
+    for seed in (7, 8):
+        args = _inputs(seed, M, N, K, r)
+        st1, st2 = status_word(), status_word()
+        ref = F.falqon_linear_bwd(*args, dev_status=st1)
+        got = F.falqon_linear_bwd_noalloc(*args, dev_status=st2)
+        torch.cuda.synchronize()
+        assert int(st1.item()) == 0 and int(st2.item()) == 0
+        for g, rr in zip(got, ref):
+            _same(g, rr)
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
     # M = 32768, r = 256 needs far more than the 16 MiB built-in scratch
     M, N, K, r = 32768, 256, 256, 256
