@@ -480,6 +480,7 @@ def run_gpu(args):
     topk = _time_topk(v, F, torch, stream, l2_flush, args, dev) if (args.topk > 0 and single) else None
     e5 = _time_e5m2(v, F, torch, stream, l2_flush, args, dev) if (args.e5m2 and single) else None
     folded = _time_folded(v, F, torch, stream, l2_flush, args, dev) if (args.folded and single) else None
+    separate = _time_separate(v, F, torch, stream, l2_flush, args, dev) if (args.separate and single) else None
 
     tokens_total = st.tokens * args.steps * ws
     value = tokens_total / (total_ms / 1e3)
@@ -545,7 +546,8 @@ def run_gpu(args):
         "clocks": clock_info,
         "device_status": status,
         "rows_selected_last_step": n_sel,
-        "extra": {"proxy_topk": topk, "e5m2_gradients": e5, "folded_adapters": folded},
+        "extra": {"proxy_topk": topk, "e5m2_gradients": e5, "folded_adapters": folded,
+                  "separate_lora": separate},
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget, r=st.r, n_stack=st.n_stack)
@@ -563,7 +565,7 @@ def _single_view(st):
     g = (L.block, L.group)
     return types.SimpleNamespace(
         M=st.M, N=L.N, K=L.K, r=st.r, wq=L.wq, s_w=L.s_w, P=L.P, A=L.A, B=L.B, dA=L.dA, dB=L.dB,
-        dB_inc=L.dB_inc, xq=st.xq[g], s_x=st.s_x[g], dyq=st.dyq[L.N], s_dy=st.s_dy, dY0=st.dY[0][0],
+        dB_inc=L.dB_inc, xq=st.xq[g], s_x=st.s_x[g], dyq=st.dyq[L.N], s_dy=st.s_dy, dY0=st.dY[0][0], X0=st.X[0][g],
         y=st.y[L.N], dx=st.dx[L.K], ws_bwd=L.ws_bwd, ws_q=st.ws_q, amax=st.amax, status=L.status)
 
 
@@ -769,6 +771,36 @@ def _time_folded(st, F, torch, stream, l2_flush, args, dev):
     return out
 
 
+def _time_separate(st, F, torch, stream, l2_flush, args, dev):
+    """The comparison the pages measure (not part of the step): LoRA kept as
+    a separate path beside the same FP8 backbone, in bf16 and with every
+    adapter operand quantized to E4M3 (forward and backward of one layer,
+    the backbone products included).  The melded step's forward, adapter
+    gradients and dX phases are the corresponding FALQON work."""
+    M, N, K, r = st.M, st.N, st.K, st.r
+    X = st.X0
+    out = {"unit": "ms per call", "timing": "CUDA graph replay per call, events on the launching stream"}
+    reps = max(5, min(50, args.steps))
+    for name, prec in (("bf16", F.SEPARATE_BF16), ("fp8", F.SEPARATE_FP8)):
+        sop = F.OP_SEPARATE_SAVED_FP8 if prec == F.SEPARATE_FP8 else F.OP_SEPARATE_SAVED_BF16
+        bop = F.OP_SEPARATE_BWD_FP8 if prec == F.SEPARATE_FP8 else F.OP_SEPARATE_BWD_BF16
+        saved = F.workspace(sop, M, N, K, r, device=dev)
+        wf = F.workspace(F.OP_SEPARATE_FWD_FP8, M, N, K, r, device=dev) if prec == F.SEPARATE_FP8 else None
+        wb = F.workspace(bop, M, N, K, r, device=dev)
+        y, dx = torch.empty_like(st.y), torch.empty_like(st.dx)
+        dA, dB = torch.empty_like(st.dA), torch.empty_like(st.dB)
+        fns = [
+            lambda: F.falqon_lora_separate_fwd(prec, st.xq, st.s_x, X, st.wq, st.s_w, st.A, st.B, y=y, saved=saved,
+                                               dev_status=st.status, workspace=wf),
+            lambda: F.falqon_lora_separate_bwd(prec, st.dyq, st.s_dy, st.dY0, st.wq, st.s_w, st.xq, st.s_x, X, st.A,
+                                               st.B, saved, dx=dx, dA=dA, dB=dB, dev_status=st.status, workspace=wb),
+        ]
+        ms = _graph_phase_times(torch, stream, l2_flush, fns, reps, not args.no_graph)
+        out[name] = {"fwd": round(ms[0], 5), "bwd": round(ms[1], 5), "total": round(sum(ms), 5)}
+    out["device_status"] = int(st.status.item())
+    return out
+
+
 # ------------------------------------------------------------------ CPU oracle
 class _OracleData:
     """Inputs of the oracle arm for one layer shape (K -> N), drawn once with
@@ -931,6 +963,8 @@ def main():
                     help="also time the folded quantized-adapter path (1) or skip it (0)")
     ap.add_argument("--e5m2", type=int, default=1,
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
+    ap.add_argument("--separate", type=int, default=1,
+                    help="also time the separate bf16 and FP8 LoRA paths (the pages' comparison) (1) or not (0)")
     ap.add_argument("--topk", type=int, default=16,
                     help="also time the top-k proxy update merging this many of the r components (0: skip)")
     ap.add_argument("--rank", type=int, default=0, help="adapter rank (0: the workload's)")

@@ -20,7 +20,9 @@ __all__ = [
     "falqon_proxy_update", "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
     "falqon_linear_bwd_folded", "folded_t_planes", "falqon_selftest_bounded_waits", "falqon_workspace_init",
-    "workspace", "OP_QUANTIZE",
+    "workspace", "falqon_lora_separate_fwd", "falqon_lora_separate_bwd", "separate_saved_views",
+    "separate_bwd_views",
+    "SEPARATE_BF16", "SEPARATE_FP8", "OP_QUANTIZE",
     "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
     "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
@@ -31,6 +33,9 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfalqon.s
 
 OP_QUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD, OP_PROXY_UPDATE, OP_PROXY_UPDATE_TOPK = 0, 1, 2, 3, 4
 OP_FOLDED_T, OP_LINEAR_BWD_FOLDED = 5, 6
+OP_SEPARATE_SAVED_BF16, OP_SEPARATE_SAVED_FP8, OP_SEPARATE_FWD_FP8 = 7, 8, 9
+OP_SEPARATE_BWD_BF16, OP_SEPARATE_BWD_FP8 = 10, 11
+SEPARATE_BF16, SEPARATE_FP8 = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
 PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL, PROXY_STRICT = 1, 2, 4, 8
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
@@ -41,7 +46,8 @@ EXPORTED_SYMBOLS = (
     "falqon_workspace_size", "falqon_status_string", "falqon_version",
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
     "falqon_linear_bwd_e5m2", "falqon_linear_fwd_folded", "falqon_linear_bwd_folded",
-    "falqon_selftest_bounded_waits", "falqon_workspace_init",
+    "falqon_selftest_bounded_waits", "falqon_workspace_init", "falqon_lora_separate_fwd",
+    "falqon_lora_separate_bwd",
 )
 
 
@@ -81,6 +87,9 @@ def lib():
     for f in ("falqon_quantize", "falqon_linear_fwd", "falqon_linear_bwd", "falqon_proxy_update",
               "falqon_linear_bwd_noalloc"):
         getattr(L, f).restype = C.c_int
+    L.falqon_lora_separate_fwd.argtypes = [C.c_int, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p, p, sz, p]
+    L.falqon_lora_separate_bwd.argtypes = [C.c_int, p, p, p, p, p, p, p, p, p, p, p, sz, i64, i64, i64, i64, p, p,
+                                           p, p, p, sz, p]
     L.falqon_workspace_init.argtypes = [p, sz, p]
     L.falqon_workspace_init.restype = C.c_int
     L.falqon_workspace_size.argtypes = [C.c_int, i64, i64, i64, i64]
@@ -357,3 +366,87 @@ def falqon_selftest_bounded_waits(flag, dev_status, which, stream=None):
     st = lib().falqon_selftest_bounded_waits(_ptr(flag), _ptr(dev_status), _ptr(which),
                                              _stream(stream, flag.device))
     _check(st, "falqon_selftest_bounded_waits")
+
+
+# ------------------------------------------------------------------ separate LoRA paths (the comparison)
+def _a256(v):
+    return (v + 255) // 256 * 256
+
+
+def separate_saved_views(saved, precision, M, N, K, r):
+    """Views of the forward's saved buffer: {"S": bf16 [M, r]} and, for the
+    FP8 path, "sq" [M, r], "aq" [r, K], "bq" [N, r] codes and "scales" (s_S,
+    s_A, s_B) as float32 [3]."""
+    o = 0
+    v = {"S": saved[o:o + M * r * 2].view(torch.bfloat16).view(M, r)}
+    o += _a256(M * r * 2)
+    if precision == SEPARATE_FP8:
+        v["sq"] = saved[o:o + M * r].view(M, r)
+        o += _a256(M * r)
+        v["aq"] = saved[o:o + r * K].view(r, K)
+        o += _a256(r * K)
+        v["bq"] = saved[o:o + N * r].view(N, r)
+        o += _a256(N * r)
+        v["scales"] = saved[o:o + 12].view(torch.float32)
+    return v
+
+
+def separate_bwd_views(workspace, precision, M, N, r, quantize_ws_bytes):
+    """Views of the backward's workspace: "G" bf16 [M, r] and, for the FP8
+    path, "gq" [M, r] codes and "s_g" float32 [1]."""
+    o = _a256(quantize_ws_bytes)
+    v = {"G": workspace[o:o + M * r * 2].view(torch.bfloat16).view(M, r)}
+    o += _a256(M * r * 2)
+    if precision == SEPARATE_FP8:
+        v["gq"] = workspace[o:o + M * r].view(M, r)
+        o += _a256(M * r)
+    ldt = (M + 15) // 16 * 16
+    o += 2 * _a256(ldt * r * (1 if precision == SEPARATE_FP8 else 2)) + _a256(N * r * 2)
+    v["s_g"] = workspace[o:o + 4].view(torch.float32)
+    return v
+
+
+def falqon_lora_separate_fwd(precision, xq, s_x, x, wq, s_w, A, B, y=None, saved=None, dev_status=None,
+                             workspace=None, stream=None):
+    """Separate LoRA path forward (bf16 or FP8 adapter products beside the FP8
+    backbone); returns (y, saved)."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    r = A.shape[0]
+    dev = xq.device
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev) if y is None else y
+    sop = OP_SEPARATE_SAVED_FP8 if precision == SEPARATE_FP8 else OP_SEPARATE_SAVED_BF16
+    if saved is None:
+        saved, _ = _workspace(sop, M, N, K, r, dev, None)
+    ws, wsb = (None, 0)
+    if precision == SEPARATE_FP8:
+        ws, wsb = _workspace(OP_SEPARATE_FWD_FP8, M, N, K, r, dev, workspace)
+    st = lib().falqon_lora_separate_fwd(int(precision), _ptr(_u8(xq)), _ptr(s_x), _ptr(x), _ptr(_u8(wq)), _ptr(s_w),
+                                        _ptr(A), _ptr(B), M, N, K, r, _ptr(y), _ptr(saved), saved.numel(),
+                                        _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_lora_separate_fwd")
+    return y, saved
+
+
+def falqon_lora_separate_bwd(precision, dyq, s_dy, dy, wq, s_w, xq, s_x, x, A, B, saved, dx=True, dA=True, dB=True,
+                             dev_status=None, workspace=None, stream=None):
+    """Separate LoRA path backward; each output may be True (allocate), a
+    tensor, or None.  Returns (dx, dA, dB)."""
+    M, N = dyq.shape
+    r, K = A.shape
+    dev = dyq.device
+
+    def out(v, shape):
+        if v is True:
+            return torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        return v if v is not None and v is not False else None
+
+    dx_t, dA_t, dB_t = out(dx, (M, K)), out(dA, (r, K)), out(dB, (N, r))
+    bop = OP_SEPARATE_BWD_FP8 if precision == SEPARATE_FP8 else OP_SEPARATE_BWD_BF16
+    ws, wsb = _workspace(bop, M, N, K, r, dev, workspace)
+    st = lib().falqon_lora_separate_bwd(
+        int(precision), _ptr(_u8(dyq)), _ptr(s_dy), _ptr(dy), _ptr(None if wq is None else _u8(wq)), _ptr(s_w),
+        _ptr(None if xq is None else _u8(xq)), _ptr(s_x), _ptr(x), _ptr(A), _ptr(B), _ptr(saved), saved.numel(),
+        M, N, K, r, _ptr(dx_t), _ptr(dA_t), _ptr(dB_t), _ptr(dev_status), _ptr(ws), wsb, _stream(stream, dev))
+    _check(st, "falqon_lora_separate_bwd")
+    return dx_t, dA_t, dB_t

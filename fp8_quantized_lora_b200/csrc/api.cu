@@ -145,6 +145,16 @@ size_t falqon_workspace_size(falqon_op op, int64_t M, int64_t N, int64_t K, int6
     case FALQON_OP_LINEAR_BWD_FOLDED:
       if (M <= 0 || r <= 0) return 0;
       return 2 * adapter_plane_bytes(M, r);
+    case FALQON_OP_SEPARATE_SAVED_BF16:
+    case FALQON_OP_SEPARATE_SAVED_FP8:
+      if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+      return separate_saved_bytes(op == FALQON_OP_SEPARATE_SAVED_FP8, M, N, K, r);
+    case FALQON_OP_SEPARATE_FWD_FP8:
+      return separate_fwd_workspace_bytes(true, M, N, K, r);
+    case FALQON_OP_SEPARATE_BWD_BF16:
+    case FALQON_OP_SEPARATE_BWD_FP8:
+      if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return 0;
+      return separate_bwd_workspace_bytes(op == FALQON_OP_SEPARATE_BWD_FP8, M, N, K, r);
   }
   return 0;
 }
@@ -381,6 +391,72 @@ falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const float* s_dy, co
   return from_cuda(launch_adapter_stage2(dyq, s_dy, xq, s_x, dB ? t : nullptr, dB ? t + plane : nullptr,
                                          dA ? u : nullptr, dA ? u + plane : nullptr, ld, M, N, K, r, dA, dB,
                                          dev_status, st));
+}
+
+}  // extern "C"
+
+namespace {
+
+falqon_status separate_shape(int precision, int64_t M, int64_t N, int64_t K, int64_t r) {
+  if (precision != FALQON_SEPARATE_BF16 && precision != FALQON_SEPARATE_FP8) return FALQON_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || r <= 0) return FALQON_ERR_INVALID_ARG;
+  if (N % 16 != 0 || K % 16 != 0 || r % 16 != 0 || r > 65536) return FALQON_ERR_UNSUPPORTED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256 ||
+      (M + 31) / 32 > 65535)
+    return FALQON_ERR_UNSUPPORTED;
+  return FALQON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+falqon_status falqon_lora_separate_fwd(int precision, const uint8_t* xq, const float* s_x, const void* x,
+                                       const uint8_t* wq, const float* s_w, const void* A, const void* B, int64_t M,
+                                       int64_t N, int64_t K, int64_t r, void* y, void* saved, size_t saved_bytes,
+                                       int32_t* dev_status, void* workspace, size_t workspace_bytes, void* stream) {
+  falqon_status s = separate_shape(precision, M, N, K, r);
+  if (s != FALQON_OK) return s;
+  const bool fp8 = precision == FALQON_SEPARATE_FP8;
+  if (!xq || !s_x || !wq || !s_w || !A || !B || !y || !saved) return FALQON_ERR_INVALID_ARG;
+  if (!fp8 && !x) return FALQON_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq) || !aligned16(A) || !aligned16(B) || !aligned16(y) ||
+      (x && !aligned16(x)))
+    return FALQON_ERR_UNSUPPORTED;
+  s = check_ws(separate_saved_bytes(fp8, M, N, K, r), saved, saved_bytes);
+  if (s != FALQON_OK) return s;
+  s = check_ws(separate_fwd_workspace_bytes(fp8, M, N, K, r), workspace, workspace_bytes);
+  if (s != FALQON_OK) return s;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_separate_fwd(fp8, xq, s_x, x, wq, s_w, A, B, M, N, K, r, y, saved, dev_status, workspace,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+falqon_status falqon_lora_separate_bwd(int precision, const uint8_t* dyq, const float* s_dy, const void* dy,
+                                       const uint8_t* wq, const float* s_w, const uint8_t* xq, const float* s_x,
+                                       const void* x, const void* A, const void* B, const void* saved,
+                                       size_t saved_bytes, int64_t M, int64_t N, int64_t K, int64_t r, void* dx,
+                                       void* dA, void* dB, int32_t* dev_status, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  falqon_status s = separate_shape(precision, M, N, K, r);
+  if (s != FALQON_OK) return s;
+  const bool fp8 = precision == FALQON_SEPARATE_FP8;
+  if (!dx && !dA && !dB) return FALQON_ERR_INVALID_ARG;
+  if (!dyq || !s_dy || !A || !B || !saved) return FALQON_ERR_INVALID_ARG;
+  if (dx && (!wq || !s_w)) return FALQON_ERR_INVALID_ARG;
+  if (!fp8 && !dy) return FALQON_ERR_INVALID_ARG;
+  if (dA && (fp8 ? (!xq || !s_x) : !x)) return FALQON_ERR_INVALID_ARG;
+  if (!aligned16(dyq) || !aligned16(A) || !aligned16(B) || (dy && !aligned16(dy)) || (wq && !aligned16(wq)) ||
+      (xq && !aligned16(xq)) || (x && !aligned16(x)) || (dx && !aligned16(dx)) || (dA && !aligned16(dA)) ||
+      (dB && !aligned16(dB)))
+    return FALQON_ERR_UNSUPPORTED;
+  s = check_ws(separate_saved_bytes(fp8, M, N, K, r), saved, saved_bytes);
+  if (s != FALQON_OK) return s;
+  s = check_ws(separate_bwd_workspace_bytes(fp8, M, N, K, r), workspace, workspace_bytes);
+  if (s != FALQON_OK) return s;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_separate_bwd(fp8, dyq, s_dy, dy, wq, s_w, xq, s_x, x, A, B, saved, M, N, K, r, dx, dA, dB,
+                                       dev_status, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

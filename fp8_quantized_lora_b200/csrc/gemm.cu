@@ -62,23 +62,27 @@ struct GemmArgs {
   void* out2_lo;
   int64_t ld2;
   const float* scale_b2;   // alpha2 = 1 / (scale_a * scale_b2)
+  const void* addend;      // bf16 [M][ldo] added to the rounded product (nullable)
   int32_t* dev_status;
 };
 
-template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks, int kHalves, int kAFmt = 0>
+template <bool kBMn, int kBN, int kStages, int kAcc, int kMinBlocks, int kHalves, int kAFmt = 0, bool kBf16 = false>
 struct Cfg {
   static constexpr bool BMn = kBMn;
+  static constexpr bool Bf16 = kBf16;                 // bf16 operands (kind::f16), else 8-bit codes
+  static constexpr int ElemBytes = kBf16 ? 2 : 1;
   static constexpr int BN = kBN;
   static constexpr int Stages = kStages;
   static constexpr int Acc = kAcc;              // accumulator buffers in TMEM
   static constexpr int MinBlocks = kMinBlocks;  // CTAs per SM
   static constexpr int Halves = kHalves;        // 128-row halves of a tile (one MMA each per K step)
   static constexpr int TileM = kHalves * kBM;
-  static constexpr int BK = kRowBytes;                // K per stage (128 E4M3 codes)
-  static constexpr int KSteps = BK / 32;              // UMMA K = 32 for 8-bit kinds
-  static constexpr int AHalfBytes = kBM * BK;         // 16 KB
+  static constexpr int BK = kRowBytes / ElemBytes;    // K per stage: one 128-byte row (128 codes or 64 bf16)
+  static constexpr int KSteps = kRowBytes / 32;       // UMMA K is 32 bytes of K (32 codes or 16 bf16)
+  static constexpr int BNBlock = kRowBytes / ElemBytes;  // N elements of one MN-major 128-byte column block
+  static constexpr int AHalfBytes = kBM * kRowBytes;  // 16 KB
   static constexpr int ABytes = kHalves * AHalfBytes;
-  static constexpr int BBytes = kBN * BK;
+  static constexpr int BBytes = kBN * kRowBytes;
   static constexpr int StageBytes = ABytes + BBytes;
   static constexpr int EpiWarps = 4 * kHalves;        // warps 2 .. 2 + EpiWarps - 1
   static constexpr int WaiterWarp = 2 + EpiWarps;
@@ -88,15 +92,17 @@ struct Cfg {
   static constexpr uint32_t TmemCols = AccCols <= 32 ? 32 : (AccCols <= 64 ? 64 : (AccCols <= 128 ? 128 : (AccCols <= 256 ? 256 : 512)));
   static constexpr int BarBytes = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
   static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
-  // A in E4M3 (kAFmt 0) or E5M2 (1; the dX GEMM of E5M2 gradients), B in E4M3
-  static constexpr uint32_t IDesc = idesc_f32acc(static_cast<uint32_t>(kAFmt), 0u, 0u, kBMn ? 1u : 0u, kBM, kBN);
-  // a half tile: the first 128 columns of the B tile (one 128-byte block when MN-major)
-  static constexpr int HalfN = kRowBytes;
-  static constexpr uint32_t IDescHalf =
-      idesc_f32acc(static_cast<uint32_t>(kAFmt), 0u, 0u, kBMn ? 1u : 0u, kBM, HalfN);
+  // 8-bit kinds: A in E4M3 (kAFmt 0) or E5M2 (1; the dX GEMM of E5M2 gradients), B in E4M3;
+  // kind::f16: A and B bf16 (format 1)
+  static constexpr uint32_t AFmt = kBf16 ? 1u : static_cast<uint32_t>(kAFmt);
+  static constexpr uint32_t BFmt = kBf16 ? 1u : 0u;
+  static constexpr uint32_t IDesc = idesc_f32acc(AFmt, BFmt, 0u, kBMn ? 1u : 0u, kBM, kBN);
+  // a half tile: the first 128 columns of the B tile
+  static constexpr int HalfN = 128;
+  static constexpr uint32_t IDescHalf = idesc_f32acc(AFmt, BFmt, 0u, kBMn ? 1u : 0u, kBM, HalfN);
   static constexpr int HalfStageBytes = ABytes + BBytes / 2;
   static_assert(kBN % 16 == 0 && kBN >= 16 && kBN <= 256, "UMMA N");
-  static_assert(!kBMn || kBN % kRowBytes == 0, "MN-major B needs 128-byte blocks");
+  static_assert(!kBMn || kBN % BNBlock == 0, "MN-major B needs whole 128-byte blocks");
   static_assert(SmemBytes <= 232448, "shared memory per CTA");
   static_assert(kMinBlocks * (SmemBytes + 1024) <= 233472, "shared memory per SM");
   static_assert(kMinBlocks * TmemCols <= 512, "tensor memory per SM");
@@ -196,10 +202,11 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
           for (int h = 0; h < C::Halves; ++h)  // rows m0 + 128 h .., K block kb
             tma_load_2d(sA + h * C::AHalfBytes, &tmA, &full[stage], kb * C::BK, m0 + h * kBM);
           if constexpr (C::BMn) {
-            // B is [K][N] row-major: 128-byte column blocks of BK rows each (one for a half tile)
-            const int blocks = nh >= 0 ? 1 : C::BN / kRowBytes;
+            // B is [K][N] row-major: 128-byte column blocks of BK rows each (the first
+            // 128 columns for a half tile)
+            const int blocks = (nh >= 0 ? C::HalfN : C::BN) / C::BNBlock;
             for (int c = 0; c < blocks; ++c)
-              tma_load_2d(sB + c * C::BK * kRowBytes, tb, &full[stage], n0 + c * kRowBytes, kb * C::BK);
+              tma_load_2d(sB + c * C::BK * kRowBytes, tb, &full[stage], n0 + c * C::BNBlock, kb * C::BK);
           } else {
             // a half tile loads 128 rows of B through the half-height box
             tma_load_2d(sB, nh >= 0 ? &tmBh : tb, &full[stage], kb * C::BK, n0);
@@ -234,11 +241,15 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
           const uint32_t b_base = a_base + C::ABytes;
 #pragma unroll
           for (int ks = 0; ks < C::KSteps; ++ks) {
-            const uint64_t bd = operand_desc<C::BMn, 1, C::BK>(b_base, ks);
+            const uint64_t bd = operand_desc<C::BMn, C::ElemBytes, C::BK>(b_base, ks);
 #pragma unroll
-            for (int h = 0; h < C::Halves; ++h)  // the halves share the B tile
-              umma_f8(tmem_d + h * C::BN, operand_desc<false, 1, C::BK>(a_base + h * C::AHalfBytes, ks), bd,
-                      idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            for (int h = 0; h < C::Halves; ++h) {  // the halves share the B tile
+              const uint64_t ad = operand_desc<false, C::ElemBytes, C::BK>(a_base + h * C::AHalfBytes, ks);
+              if constexpr (C::Bf16)
+                umma_bf16(tmem_d + h * C::BN, ad, bd, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+              else
+                umma_f8(tmem_d + h * C::BN, ad, bd, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&empty[stage]);
         }
@@ -343,16 +354,26 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         tmem_ld_wait();
         if (row < g.M) {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
+          const __nv_bfloat16* add = g.addend ? static_cast<const __nv_bfloat16*>(g.addend) + row * g.ldo : nullptr;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int64_t col = col_base + c * 32 + 8 * j;
             if (col < g.N) {
               uint32_t pk[4];
+              uint4 ad = make_uint4(0u, 0u, 0u, 0u);
+              if (add) ad = *reinterpret_cast<const uint4*>(add + col);
+              const uint32_t aw[4] = {ad.x, ad.y, ad.z, ad.w};
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 b = __floats2bfloat162_rn(
-                    __uint_as_float(r[8 * j + 2 * h]) * alpha,
-                    __uint_as_float(r[8 * j + 2 * h + 1]) * alpha);
+                __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * h]) * alpha,
+                                                         __uint_as_float(r[8 * j + 2 * h + 1]) * alpha);
+                if (add) {
+                  // the product rounded to bf16, then added as bf16 tensors add:
+                  // a float32 sum rounded once to bf16
+                  const float2 pf = __bfloat1622float2(b);
+                  b = __floats2bfloat162_rn(__fadd_rn(pf.x, __uint_as_float(aw[h] << 16)),
+                                            __fadd_rn(pf.y, __uint_as_float(aw[h] & 0xFFFF0000u)));
+                }
                 memcpy(&pk[h], &b, 4);
               }
               *reinterpret_cast<uint4*>(dst + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -419,7 +440,7 @@ using DxE5Cfg = Cfg<true, 256, 4, 2, 1, 1, 1>;  // dYq in E5M2
 // out2_hi / out2_lo [N2][ld2].  `out` may be null (no backbone segment: the
 // grid then covers the adapter tiles alone).
 struct Segment2 {
-  const uint8_t* b = nullptr;
+  const void* b = nullptr;
   const float* sb = nullptr;
   int64_t n = 0;
   void* hi = nullptr;
@@ -428,19 +449,27 @@ struct Segment2 {
 };
 
 template <class C>
-bool b_tmap(CUtensorMap* t, const uint8_t* b, int64_t Ncols, int64_t Kc) {
-  // B K-major [Ncols, Kc] or MN-major [Kc, Ncols]
-  return C::BMn ? make_tmap_2d(t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Ncols, Kc, 128, C::BK, true)
-                : make_tmap_2d(t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::BN, true);
+constexpr CUtensorMapDataType tmap_dtype() {
+  return C::Bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
 }
 
 template <class C>
-cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
-                     int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
-                     cudaStream_t stream, const Segment2& s2 = Segment2{}) {
+bool b_tmap(CUtensorMap* t, const void* b, int64_t Ncols, int64_t Kc) {
+  // B K-major [Ncols, Kc] or MN-major [Kc, Ncols]; boxes are one 128-byte row wide
+  return C::BMn ? make_tmap_2d(t, tmap_dtype<C>(), C::ElemBytes, b, Ncols, Kc, C::BNBlock, C::BK, true)
+                : make_tmap_2d(t, tmap_dtype<C>(), C::ElemBytes, b, Kc, Ncols, C::BK, C::BN, true);
+}
+
+// C[M, Ncols] = bf16(A . B / (sa sb)) (+ addend, rounded as bf16 tensors add);
+// A [M, Kc] K-major; B per C::BMn.  Operands are 8-bit codes, or bf16 when C::Bf16.
+template <class C>
+cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* sb,
+                    int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
+                    cudaStream_t stream, const Segment2& s2 = Segment2{}, const void* addend = nullptr,
+                    int64_t lda = 0) {
   CUtensorMap tA, tB, tB2, tBh;
-  // A [M, Kc] K-major
-  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a, Kc, M, 128, kBM, true))
+  // A [M, Kc] K-major, rows lda elements apart (0: Kc)
+  if (!make_tmap_2d(&tA, tmap_dtype<C>(), C::ElemBytes, a, Kc, M, C::BK, kBM, true, static_cast<uint64_t>(lda)))
     return cudaErrorInvalidValue;
   const bool seg1 = out != nullptr;
   if (seg1 && !b_tmap<C>(&tB, b, Ncols, Kc)) return cudaErrorInvalidValue;
@@ -449,7 +478,8 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
   if (s2.n <= 0) tB2 = tB;
   // K-major half tiles load 128 rows of B through a half-height box
   tBh = tB;
-  if (!C::BMn && seg1 && !make_tmap_2d(&tBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, b, Kc, Ncols, 128, C::HalfN, true))
+  if (!C::BMn && seg1 &&
+      !make_tmap_2d(&tBh, tmap_dtype<C>(), C::ElemBytes, b, Kc, Ncols, C::BK, C::HalfN, true))
     return cudaErrorInvalidValue;
   GemmArgs g{};
   g.m_tiles = ceil_div(M, C::TileM);
@@ -467,11 +497,22 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
   g.out2_lo = s2.lo;
   g.ld2 = s2.ld;
   g.scale_b2 = s2.sb;
+  g.addend = addend;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
   if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, tBh, g, stream);
   return launch_gemm<C, false>(tA, tB, tB2, tBh, g, stream);
 }
+
+template <class C>
+cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const float* sb,
+                     int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
+                     cudaStream_t stream, const Segment2& s2 = Segment2{}) {
+  return tc_gemm<C>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, s2);
+}
+
+using BfFwdCfg = Cfg<false, 256, 4, 2, 1, 1, 0, true>;  // bf16 operands, B K-major
+using BfDxCfg = Cfg<true, 256, 4, 2, 1, 1, 0, true>;    // bf16 operands, B MN-major
 
 }  // namespace
 
@@ -506,6 +547,20 @@ cudaError_t launch_fp8_gemm_dx_folded(const uint8_t* dyq, const float* s_dy, con
   Segment2 s2;
   s2.b = bq; s2.sb = s_b; s2.n = bq ? r : 0; s2.hi = u_hi; s2.lo = u_lo; s2.ld = ld;
   return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream, s2);
+}
+
+cudaError_t launch_gemm_nt(bool bf16, const void* a, const float* sa, const void* b, const float* sb, int64_t M,
+                           int64_t Ncols, int64_t Kc, void* out, const void* addend, int32_t* dev_status,
+                           cudaStream_t stream) {
+  return bf16 ? tc_gemm<BfFwdCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend)
+              : tc_gemm<FwdCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend);
+}
+
+cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void* b, const float* sb, int64_t M,
+                           int64_t Ncols, int64_t Kc, void* out, const void* addend, int32_t* dev_status,
+                           cudaStream_t stream, int64_t lda) {
+  return bf16 ? tc_gemm<BfDxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda)
+              : tc_gemm<DxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda);
 }
 
 }  // namespace falqon

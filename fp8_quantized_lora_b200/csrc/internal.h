@@ -83,6 +83,18 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
                                int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
 
+// Plain products on the tcgen05 GEMM: C[M, Ncols] = bf16(A . op(B) / (sa sb)),
+// then, when addend is not null, bf16(fl32(C + addend)) (bf16 tensors adding).
+// A [M, Kc] K-major.  _nt: B [Ncols, Kc] (K-major);  _nn: B [Kc, Ncols] (MN-major).
+// bf16: operands are bf16 (kind::f16) and the scales may be null; else E4M3 codes.
+cudaError_t launch_gemm_nt(bool bf16, const void* a, const float* sa, const void* b, const float* sb, int64_t M,
+                           int64_t Ncols, int64_t Kc, void* out, const void* addend, int32_t* dev_status,
+                           cudaStream_t stream);
+// lda: elements between rows of A (0: Kc); a multiple of 16 bytes.
+cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void* b, const float* sb, int64_t M,
+                           int64_t Ncols, int64_t Kc, void* out, const void* addend, int32_t* dev_status,
+                           cudaStream_t stream, int64_t lda = 0);
+
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da);
 // Every argument check of falqon_linear_bwd except the workspace's (returns
 // the status that call would return before launching, or FALQON_OK).
@@ -118,6 +130,20 @@ cudaError_t launch_fp8_gemm_dx_folded(const uint8_t* dyq, const float* s_dy, con
                                       const float* s_w, const uint8_t* bq, const float* s_b, int64_t M,
                                       int64_t N, int64_t K, int64_t r, void* dx, void* u_hi, void* u_lo,
                                       int64_t ld, int32_t* dev_status, cudaStream_t stream);
+
+// ---------------------------------------------------------------- separate LoRA paths
+size_t separate_saved_bytes(bool fp8, int64_t M, int64_t N, int64_t K, int64_t r);
+size_t separate_fwd_workspace_bytes(bool fp8, int64_t M, int64_t N, int64_t K, int64_t r);
+size_t separate_bwd_workspace_bytes(bool fp8, int64_t M, int64_t N, int64_t K, int64_t r);
+cudaError_t launch_separate_fwd(bool fp8, const uint8_t* xq, const float* s_x, const void* x, const uint8_t* wq,
+                                const float* s_w, const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                int64_t r, void* y, void* saved, int32_t* dev_status, void* workspace,
+                                cudaStream_t stream);
+cudaError_t launch_separate_bwd(bool fp8, const uint8_t* dyq, const float* s_dy, const void* dy, const uint8_t* wq,
+                                const float* s_w, const uint8_t* xq, const float* s_x, const void* x,
+                                const void* A, const void* B, const void* saved, int64_t M, int64_t N, int64_t K,
+                                int64_t r, void* dx, void* dA, void* dB, int32_t* dev_status, void* workspace,
+                                cudaStream_t stream);
 
 // ---------------------------------------------------------------- proxy
 size_t proxy_workspace_bytes(int64_t N, int64_t K);

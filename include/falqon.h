@@ -78,8 +78,19 @@ typedef enum falqon_op {
   FALQON_OP_PROXY_UPDATE = 3,
   FALQON_OP_PROXY_UPDATE_TOPK = 4,
   FALQON_OP_FOLDED_T = 5,          /* the buffer T of the folded forward keeps for the backward */
-  FALQON_OP_LINEAR_BWD_FOLDED = 6  /* workspace of falqon_linear_bwd_folded (U, when dA is wanted) */
+  FALQON_OP_LINEAR_BWD_FOLDED = 6, /* workspace of falqon_linear_bwd_folded (U, when dA is wanted) */
+  FALQON_OP_SEPARATE_SAVED_BF16 = 7, /* what falqon_lora_separate_fwd keeps for the backward, bf16 path */
+  FALQON_OP_SEPARATE_SAVED_FP8 = 8,  /* the same, FP8 path */
+  FALQON_OP_SEPARATE_FWD_FP8 = 9,    /* workspace of the FP8 separate forward (a quantize workspace) */
+  FALQON_OP_SEPARATE_BWD_BF16 = 10,  /* workspace of falqon_lora_separate_bwd, bf16 path */
+  FALQON_OP_SEPARATE_BWD_FP8 = 11    /* the same, FP8 path */
 } falqon_op;
+
+/* Precision of the separate LoRA paths (falqon_lora_separate_fwd / _bwd). */
+typedef enum falqon_separate_precision {
+  FALQON_SEPARATE_BF16 = 0, /* adapter products in bf16 */
+  FALQON_SEPARATE_FP8 = 1   /* every adapter operand quantized to E4M3 per product */
+} falqon_separate_precision;
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define FALQON_DEV_NONFINITE 1      /* amax of an input was NaN or infinite */
@@ -367,6 +378,60 @@ FALQON_API falqon_status falqon_linear_bwd_noalloc(const uint8_t* dyq, const flo
                                                    int64_t N, int64_t K, int64_t r, void* dx,
                                                    void* dA, void* dB, int32_t* dev_status,
                                                    void* stream);
+
+/*
+ * falqon_lora_separate_fwd / falqon_lora_separate_bwd - LoRA kept as a
+ * separate path beside the FP8 backbone: the comparison FALQON is measured
+ * against, not FALQON's own path (which merges the adapter into Wq).
+ *
+ * The paper's introduction sets FALQON against separate LoRA paths on an FP8
+ * backbone, whose small adapter products each pay a quantization; the
+ * OpenReview rebuttals compare FP8 and FP16 adapters across ranks (reviewer
+ * 2, W4, Table R1; reviewer 3, Q3, Table R6).  The adapter branch is a
+ * separate layer; each of its products is rounded to bf16 and the branch is
+ * added to the backbone's bf16 output as bf16 tensors add (a float32 sum
+ * rounded once to bf16):
+ *   forward   Ybb = the backbone product (falqon_linear_fwd),
+ *             S = bf16(X . A^T), Y = bf16(fl32(Ybb + bf16(S . B^T)))
+ *   backward  dXbb = the backbone product (falqon_linear_bwd's dX),
+ *             G = bf16(dY . B), dX = bf16(fl32(dXbb + bf16(G . A))),
+ *             dB = bf16(dY^T . S), dA = bf16(G^T . X)
+ * FALQON_SEPARATE_BF16: the adapter products take X, dY, A and B as bf16.
+ * FALQON_SEPARATE_FP8: every adapter operand is quantized per tensor to
+ * E4M3 right before its product (as falqon_quantize): X and dY are the
+ * backbone's codes xq and dyq, A and B are quantized each forward, S and G
+ * once formed; each product divides by its two scales.
+ *
+ * Forward arguments: xq, s_x and wq, s_w as falqon_linear_fwd; x [M, K] bf16
+ * (read by the bf16 path); A [r, K], B [N, r] bf16; y [M, N] bf16, written.
+ * saved: caller-owned, falqon_workspace_size(FALQON_OP_SEPARATE_SAVED_BF16 or
+ * _FP8, M, N, K, r) bytes, written (S, and in FP8 the codes and scales of S,
+ * A and B), read by the backward.  workspace: FP8 path only,
+ * falqon_workspace_size(FALQON_OP_SEPARATE_FWD_FP8, ...) bytes, a quantize
+ * workspace (initialise it once with falqon_workspace_init).
+ *
+ * Backward arguments: dyq, s_dy as falqon_linear_bwd; dy [M, N] bf16 (bf16
+ * path); wq, s_w (read when dx is wanted); xq, s_x (FP8 path, for dA); x
+ * (bf16 path, for dA); A, B and saved as the forward left them.  dx [M, K],
+ * dA [r, K], dB [N, r]: bf16 outputs, each nullable, not all null.
+ * workspace: falqon_workspace_size(FALQON_OP_SEPARATE_BWD_BF16 or _FP8, M, N,
+ * K, r) bytes; it holds a quantize workspace, so initialise it once with
+ * falqon_workspace_init.
+ * Requirements: M >= 1; N, K, r multiples of 16; r <= 65536.
+ */
+FALQON_API falqon_status falqon_lora_separate_fwd(int precision, const uint8_t* xq, const float* s_x,
+                                                  const void* x, const uint8_t* wq, const float* s_w,
+                                                  const void* A, const void* B, int64_t M, int64_t N, int64_t K,
+                                                  int64_t r, void* y, void* saved, size_t saved_bytes,
+                                                  int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                                                  void* stream);
+FALQON_API falqon_status falqon_lora_separate_bwd(int precision, const uint8_t* dyq, const float* s_dy,
+                                                  const void* dy, const uint8_t* wq, const float* s_w,
+                                                  const uint8_t* xq, const float* s_x, const void* x,
+                                                  const void* A, const void* B, const void* saved,
+                                                  size_t saved_bytes, int64_t M, int64_t N, int64_t K, int64_t r,
+                                                  void* dx, void* dA, void* dB, int32_t* dev_status,
+                                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * falqon_selftest_bounded_waits - exercises the failure detection on the GPU

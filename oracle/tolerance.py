@@ -68,3 +68,29 @@ def tolerance_report(G, R, Rb=None) -> dict:
 
 def within_tolerance(G, R, Rb=None) -> bool:
     return tolerance_report(G, R, Rb)["ok"]
+
+
+def branch_sum_report(G, Y, branches) -> dict:
+    """Acceptance for a sum of bf16 branches (C-17: the backbone output plus
+    the separate adapter branch, each rounded to bf16 before the bf16 add).
+    Y: the oracle's result (float64 values of bf16); branches: the oracle's
+    rounded branch values.  Each branch of the implementation may differ
+    from the oracle's by one bf16 unit (its float32 accumulation against the
+    oracle's float64), and the sum is rounded once more:
+
+        |G - Y| <= ulp(max(|Y|, tau)) + sum_b ulp(max(|b|, tau_b)),
+
+    every tau being 2^-8 of the tensor's largest magnitude."""
+    G = _bf16_to_f64(G) if np.asarray(G).dtype == np.uint16 else np.asarray(G, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+
+    def unit(v):
+        v = np.asarray(v, dtype=np.float64)
+        t = TAU_FRACTION * (np.max(np.abs(v)) if v.size else 0.0)
+        return ulp_bf16(np.maximum(np.abs(v), t)) if t > 0 else np.zeros(v.shape)
+    bound = unit(Y) + sum(unit(b) for b in branches)
+    err = np.abs(G - Y)
+    ok = err <= bound
+    return {"ok": bool(np.all(ok)), "n_bad": int(np.sum(~ok)),
+            "max_err_over_bound": float(np.max(err / np.maximum(bound, _MIN_ULP))) if G.size else 0.0,
+            "first_bad": None if np.all(ok) else int(np.flatnonzero(~ok.ravel())[0])}

@@ -205,3 +205,32 @@ def test_workspace_init_argument_errors():
     assert L.falqon_workspace_init(None, 256, None) == 1   # no workspace
     assert L.falqon_workspace_init(P, 0, None) == 1        # no bytes
     assert L.falqon_workspace_init(P8, 256, None) == 3     # not 256-byte aligned
+
+
+def test_separate_path_argument_errors():
+    L = F.lib()
+    M, N, K, r = 64, 32, 48, 16
+    sb = F.falqon_workspace_size(F.OP_SEPARATE_SAVED_FP8, M, N, K, r)
+    wf = F.falqon_workspace_size(F.OP_SEPARATE_FWD_FP8, M, N, K, r)
+    wb = F.falqon_workspace_size(F.OP_SEPARATE_BWD_FP8, M, N, K, r)
+    assert sb % 256 == 0 and wf % 256 == 0 and wb % 256 == 0
+    assert F.falqon_workspace_size(F.OP_SEPARATE_SAVED_BF16, M, N, K, r) < sb
+    fwd, bwd = L.falqon_lora_separate_fwd, L.falqon_lora_separate_bwd
+
+    def f(prec=1, x=P, A=P, y=P, r_=r, K_=K, saved=P, sbytes=sb, ws=P, wsb=wf):
+        return fwd(prec, P, P, x, P, P, A, P, M, N, K_, r_, y, saved, sbytes, None, ws, wsb, None)
+    assert f(prec=2) == 1                 # unknown precision
+    assert f(A=None) == 1                 # no A
+    assert f(prec=0, x=None) == 1         # the bf16 path reads X
+    assert f(r_=24) == 2                  # r % 16
+    assert f(K_=40) == 2                  # K % 16
+    assert f(y=P8) == 2                   # unaligned output
+    assert f(sbytes=sb - 256) == 3        # saved buffer too small
+    assert f(ws=None, wsb=0) == 3         # the FP8 forward needs its quantize workspace
+
+    def b(prec=1, dx=P, dA=P, dB=P, xq=P, x=P, dy=P, ws=P, wsb=wb):
+        return bwd(prec, P, P, dy, P, P, xq, P, x, P, P, P, sb, M, N, K, r, dx, dA, dB, None, ws, wsb, None)
+    assert b(dx=None, dA=None, dB=None) == 1  # nothing to compute
+    assert b(xq=None) == 1                    # FP8 dA reads the codes of X
+    assert b(prec=0, dy=None) == 1            # the bf16 path reads dY
+    assert b(wsb=wb - 256) == 3               # workspace too small
