@@ -185,13 +185,16 @@ class Step:
     # library kernels per call of each phase (the caller's SGD is two torch ops)
     LAUNCHES = {"quantX": 1, "fwd": 1, "quantdY": 1, "adapters": 2, "dX": 1, "sgd": 0, "proxy": 2}
 
-    def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None):
+    def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None, tensor_from=256):
         self.torch, self.F, self.dev = torch, F, dev
         t = torch
         self.wl = wl
         self.M, self.r, self.lr = wl.M, (wl.r if r is None else r), wl.lr
         self.n_slots = n_slots
         self.n_stack = n_stack or wl.n_stack
+        # the proxy's accumulation: the strict float32 chain, or the tensor cores from rank tensor_from up
+        self.proxy_tensor = tensor_from > 0 and self.r >= tensor_from
+        self.proxy_flags = F.PROXY_ACCUMULATE | F.PROXY_SELECT | (F.PROXY_TENSOR if self.proxy_tensor else 0)
         maxdim = max(max(l.N, l.K) for l in wl.layers)
         # one quantize workspace for every call of the step, initialised once
         self.ws_q = F.workspace(F.OP_QUANTIZE, self.M, maxdim, device=dev)
@@ -271,8 +274,8 @@ class Step:
                 L.B.add_(L.dB_inc)
             out.append((L, "sgd", sgd))
             out.append((L, "proxy", lambda L=L: F.falqon_proxy_update(
-                L.wq, L.s_w, L.P, L.dB_inc, L.A, row_mask=L.mask, n_selected=L.n_sel, dev_status=L.status,
-                workspace=L.ws_p)))
+                L.wq, L.s_w, L.P, L.dB_inc, L.A, flags=self.proxy_flags, row_mask=L.mask, n_selected=L.n_sel,
+                dev_status=L.status, workspace=L.ws_p)))
         return out
 
     def run(self, slot, phase=None, outs=None):
@@ -332,7 +335,7 @@ def _phase_work(st):
                "kernels": "tc_gemm_kernel (dX)"},
         "sgd": {"flops": 0.0, "bytes": 8.0 * N * r, "bound": None, "kernels": "torch (caller's SGD)"},
         "proxy": {"flops": proxy_flops, "bytes": proxy_bytes, "bound": "alu" if proxy_alu else "hbm",
-                  "kernels": "proxy_pipe_kernel + proxy_clear_kernel"},
+                  "kernels": "proxy_ws_kernel + proxy_clear_kernel"},
     }
 
 
@@ -382,7 +385,8 @@ def run_gpu(args):
     slot_bytes = n_stack * wl.M * 2 * (sum(k for _, k in {(l.x_group, l.K) for l in wl.layers}) +
                                        sum(l.N for l in wl.layers))
     slots = args.slots or min(8, max(2, -(-(2 * L2_BYTES) // slot_bytes)))
-    st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack)
+    st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack,
+              tensor_from=args.proxy_tensor_from)
     stream = torch.cuda.Stream(device=dev)
     if args.only:
         # one phase alone, eagerly, warm-up + steps times (for profiler captures)
@@ -537,7 +541,9 @@ def run_gpu(args):
                    "global_batch_tokens": st.M * ws, "parallelism": f"replicas{ws}",
                    "l2": (f"back to back: no flush; {st.n_slots} input slots cycled "
                           f"({st.n_slots * slot_bytes / 2**20:.0f} MiB of X and dY, above the 126 MB L2)"),
-                   "cuda_graph": not args.no_graph, "lr": wl.lr},
+                   "cuda_graph": not args.no_graph, "lr": wl.lr,
+                   "proxy_accumulation": ("tensor cores (bf16 products, float32 sums)" if st.proxy_tensor
+                                          else "strict float32 FMA chain")},
         "step_ms_median": round(float(np.median(per_step)), 5),
         "roofline": roof,
         "phases": phases,
@@ -963,6 +969,8 @@ def main():
                     help="also time the folded quantized-adapter path (1) or skip it (0)")
     ap.add_argument("--e5m2", type=int, default=1,
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
+    ap.add_argument("--proxy-tensor-from", type=int, default=256,
+                    help="rank from which the proxy accumulates on the tensor cores (0: never)")
     ap.add_argument("--separate", type=int, default=1,
                     help="also time the separate bf16 and FP8 LoRA paths (the pages' comparison) (1) or not (0)")
     ap.add_argument("--topk", type=int, default=16,

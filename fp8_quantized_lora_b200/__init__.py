@@ -25,7 +25,7 @@ __all__ = [
     "SEPARATE_BF16", "SEPARATE_FP8", "OP_QUANTIZE",
     "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
-    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
+    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "PROXY_TENSOR", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
@@ -37,7 +37,7 @@ OP_SEPARATE_SAVED_BF16, OP_SEPARATE_SAVED_FP8, OP_SEPARATE_FWD_FP8 = 7, 8, 9
 OP_SEPARATE_BWD_BF16, OP_SEPARATE_BWD_FP8 = 10, 11
 SEPARATE_BF16, SEPARATE_FP8 = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
-PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL, PROXY_STRICT = 1, 2, 4, 8
+PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL, PROXY_STRICT, PROXY_TENSOR = 1, 2, 4, 8, 16
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
 

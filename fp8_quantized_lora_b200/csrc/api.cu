@@ -270,15 +270,22 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   int64_t r, uint32_t flags, uint8_t* row_mask,
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream) {
-  const uint32_t known =
-      FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL | FALQON_PROXY_STRICT;
+  const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL |
+                         FALQON_PROXY_STRICT | FALQON_PROXY_TENSOR;
   if ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
   if ((flags & FALQON_PROXY_KEEP_RESIDUAL) && !(flags & FALQON_PROXY_SELECT)) return FALQON_ERR_INVALID_ARG;
+  if ((flags & FALQON_PROXY_TENSOR) &&
+      (!(flags & FALQON_PROXY_ACCUMULATE) || (flags & FALQON_PROXY_STRICT)))
+    return FALQON_ERR_INVALID_ARG;
   if (!proxy || N <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
   if (K % 16 != 0) return FALQON_ERR_UNSUPPORTED;
   if (!aligned16(proxy)) return FALQON_ERR_UNSUPPORTED;
   if (flags & FALQON_PROXY_ACCUMULATE) {
     if (!dB_inc || !A || r <= 0) return FALQON_ERR_INVALID_ARG;
+  }
+  if (flags & FALQON_PROXY_TENSOR) {
+    if (r % 8 != 0 || N > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256) return FALQON_ERR_UNSUPPORTED;
+    if (!aligned16(dB_inc) || !aligned16(A)) return FALQON_ERR_UNSUPPORTED;
   }
   if (flags & FALQON_PROXY_SELECT) {
     if (!wq || !s_w) return FALQON_ERR_INVALID_ARG;

@@ -63,6 +63,7 @@ struct GemmArgs {
   int64_t ld2;
   const float* scale_b2;   // alpha2 = 1 / (scale_a * scale_b2)
   const void* addend;      // bf16 [M][ldo] added to the rounded product (nullable)
+  int32_t f32_accumulate;  // out is float32 [M][ldo]: out = fl32(out + alpha * product), no bf16 rounding
   int32_t* dev_status;
 };
 
@@ -91,7 +92,10 @@ struct Cfg {
   static constexpr int AccCols = kAcc * kHalves * kBN;
   static constexpr uint32_t TmemCols = AccCols <= 32 ? 32 : (AccCols <= 64 ? 64 : (AccCols <= 128 ? 128 : (AccCols <= 256 ? 256 : 512)));
   static constexpr int BarBytes = 8 * (2 * kStages + 2 * kAcc + 1) + 16;
-  static constexpr int SmemBytes = kStages * StageBytes + BarBytes + 1024;
+  // float32-accumulate epilogue (bf16 configurations only): one 32 x 33 float
+  // transpose buffer per epilogue warp, so that P moves in contiguous rows
+  static constexpr int EpiStageBytes = kBf16 ? EpiWarps * 32 * 33 * 4 : 0;
+  static constexpr int SmemBytes = kStages * StageBytes + BarBytes + EpiStageBytes + 1024;
   // 8-bit kinds: A in E4M3 (kAFmt 0) or E5M2 (1; the dX GEMM of E5M2 gradients), B in E4M3;
   // kind::f16: A and B bf16 (format 1)
   static constexpr uint32_t AFmt = kBf16 ? 1u : static_cast<uint32_t>(kAFmt);
@@ -352,6 +356,38 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         tmem_ld_32cols(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + (acc * C::Halves + half) * C::BN +
                            c * 32, r);
         tmem_ld_wait();
+        if constexpr (C::EpiStageBytes > 0) {
+          if (g.f32_accumulate) {
+            // float32 output accumulated in place, out = fl32(out + alpha * D).
+            // Lane l holds row l of the warp's 32 rows; the 32 x 32 chunk goes
+            // through shared memory so that every access below covers four
+            // rows of 128 contiguous bytes.
+            float* stg = reinterpret_cast<float*>(smem + C::Stages * C::StageBytes + C::BarBytes) +
+                         (warp - 2) * (32 * 33);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[lane * 33 + j] = __fmul_rn(__uint_as_float(r[j]), alpha);
+            __syncwarp();
+            const int64_t row0 = row - lane;  // the warp's first row
+            const int64_t col = col_base + c * 32 + 4 * (lane & 7);
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int rr = 4 * it + (lane >> 3);
+              const int64_t grow = row0 + rr;
+              if (grow < g.M && col < g.N) {  // Ncols % 4 == 0: four columns in or out together
+                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + grow * g.ldo + col);
+                float4 p = *dst;
+                const float* src = stg + rr * 33 + 4 * (lane & 7);
+                p.x = __fadd_rn(p.x, src[0]);
+                p.y = __fadd_rn(p.y, src[1]);
+                p.z = __fadd_rn(p.z, src[2]);
+                p.w = __fadd_rn(p.w, src[3]);
+                *dst = p;
+              }
+            }
+            __syncwarp();  // the buffer is reused by the next chunk
+            continue;
+          }
+        }
         if (row < g.M) {
           __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
           const __nv_bfloat16* add = g.addend ? static_cast<const __nv_bfloat16*>(g.addend) + row * g.ldo : nullptr;
@@ -466,7 +502,7 @@ template <class C>
 cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* sb,
                     int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
                     cudaStream_t stream, const Segment2& s2 = Segment2{}, const void* addend = nullptr,
-                    int64_t lda = 0) {
+                    int64_t lda = 0, bool f32_accumulate = false) {
   CUtensorMap tA, tB, tB2, tBh;
   // A [M, Kc] K-major, rows lda elements apart (0: Kc)
   if (!make_tmap_2d(&tA, tmap_dtype<C>(), C::ElemBytes, a, Kc, M, C::BK, kBM, true, static_cast<uint64_t>(lda)))
@@ -498,6 +534,7 @@ cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* 
   g.ld2 = s2.ld;
   g.scale_b2 = s2.sb;
   g.addend = addend;
+  g.f32_accumulate = f32_accumulate ? 1 : 0;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
   if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, tBh, g, stream);
@@ -561,6 +598,12 @@ cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void
                            cudaStream_t stream, int64_t lda) {
   return bf16 ? tc_gemm<BfDxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda)
               : tc_gemm<DxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda);
+}
+
+cudaError_t launch_gemm_nn_f32acc(const void* a, const void* b, int64_t M, int64_t Ncols, int64_t Kc, float* out,
+                                  int32_t* dev_status, cudaStream_t stream) {
+  return tc_gemm<BfDxCfg>(a, nullptr, b, nullptr, M, Ncols, Kc, out, dev_status, stream, Segment2{}, nullptr, 0,
+                          true);
 }
 
 }  // namespace falqon

@@ -95,6 +95,11 @@ cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void
                            int64_t Ncols, int64_t Kc, void* out, const void* addend, int32_t* dev_status,
                            cudaStream_t stream, int64_t lda = 0);
 
+// out[M, Ncols] (float32) = fl32(out + A . B): A [M, Kc] and B [Kc, Ncols]
+// bf16, float32 accumulation on the tensor cores (kind::f16).
+cudaError_t launch_gemm_nn_f32acc(const void* a, const void* b, int64_t M, int64_t Ncols, int64_t Kc, float* out,
+                                  int32_t* dev_status, cudaStream_t stream);
+
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da);
 // Every argument check of falqon_linear_bwd except the workspace's (returns
 // the status that call would return before launching, or FALQON_OK).

@@ -526,9 +526,17 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
                                 void* workspace, cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
-  const bool acc = flags & 1u, sel = flags & 2u;
+  bool acc = flags & 1u;
+  const bool sel = flags & 2u;
   const int keep_res = (flags & 4u) ? 1 : 0;  // residual-keeping clear instead of P = +0
   if (r > (int64_t(1) << 30)) return cudaErrorInvalidValue;
+  if (acc && (flags & 16u)) {
+    // tensor-core accumulation: P = fl32(P + dB_inc . A), float32 accumulation
+    // in the tensor cores' order; the selection below reads the result
+    cudaError_t e = launch_gemm_nn_f32acc(dB_inc, A, N, K, r, proxy, dev_status, stream);
+    if (e != cudaSuccess || !sel) return e;
+    acc = false;
+  }
   const dim3 grid(static_cast<unsigned>((K + kTileCols - 1) / kTileCols),
                   static_cast<unsigned>((N + kTileRows - 1) / kTileRows));
   const int rr = acc ? static_cast<int>(r) : 0;

@@ -102,8 +102,9 @@ typedef enum falqon_separate_precision {
 #define FALQON_PROXY_ACCUMULATE 1u /* P += dB_inc . A */
 #define FALQON_PROXY_SELECT 2u     /* select rows, requantize them, clear their proxy */
 #define FALQON_PROXY_KEEP_RESIDUAL 4u /* with SELECT: keep the unapplied residual, no clear */
-#define FALQON_PROXY_STRICT 8u        /* accepted, changes nothing: the accumulation is always the
-                                         strict float32 FMA chain in index order, for every r */
+#define FALQON_PROXY_STRICT 8u        /* the strict float32 FMA chain in index order (the default) */
+#define FALQON_PROXY_TENSOR 16u       /* with ACCUMULATE: the accumulation on the tensor cores (see
+                                         falqon_proxy_update); not with STRICT */
 
 /*
  * falqon_quantize - per-tensor E4M3 quantization.
@@ -276,9 +277,19 @@ FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const floa
  *               sub-step residual): a code whose value changes keeps
  *               P = fl32(P - fl32(fl32(dec(c') - dec(old)) / s_W)); every
  *               other code keeps its proxy.  Row mask and count as SELECT.
- *   STRICT:     accepted with the flags above and changes nothing: the
- *               accumulation is always the strict float32 chain.
- * The float32 chain is reproduced bit-for-bit (no tensor cores).
+ *   STRICT:     the accumulation is the strict float32 chain above, which
+ *               is also the default.
+ *   TENSOR:     (with ACCUMULATE, not STRICT) P = fl32(P + D) with
+ *               D = dB_inc . A formed on the tensor cores: bf16 products
+ *               (exact) summed in float32 in the hardware's order, which no
+ *               fixed sequence reproduces.  For large r the chain's r FMAs
+ *               per element bound it by the float32 pipe (at r = 8192 and
+ *               N = K = 4096, 275 GFLOP); the tensor cores take them at bf16
+ *               tensor rate.  SELECT then runs on the resulting P as a pass
+ *               of its own (with both flags, or in a later call), and it
+ *               is that pass that reports a non-finite P.
+ *               Requirements: r a multiple of 8.
+ * The default float32 chain is reproduced bit-for-bit.
  *
  *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);
  *  proxy [N, K] float32, in/out;  dB_inc [N, r] bfloat16 (the increment of
@@ -287,7 +298,7 @@ FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const floa
  *  set; nullable.
  *  Requirements: N >= 1; K multiple of 16; r >= 1 (r unused without
  *  ACCUMULATE); flags: ACCUMULATE and/or SELECT, plus KEEP_RESIDUAL only
- *  with SELECT.
+ *  with SELECT, TENSOR only with ACCUMULATE.
  */
 FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   const void* dB_inc, const void* A, int64_t N, int64_t K,

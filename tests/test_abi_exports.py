@@ -102,7 +102,7 @@ def test_proxy_argument_errors():
         assert L.falqon_proxy_update(P, P, P, P, P, 4, 20, 2, flags, None, None, None, P, 1 << 20, None) == 2
     # ... but not alone, and unknown bits are still rejected
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 8, None, None, None, P, 1 << 20, None) == 1
-    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3 | 16, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3 | 32, None, None, None, P, 1 << 20, None) == 1
 
 
 def test_proxy_topk_argument_errors():
@@ -234,3 +234,13 @@ def test_separate_path_argument_errors():
     assert b(xq=None) == 1                    # FP8 dA reads the codes of X
     assert b(prec=0, dy=None) == 1            # the bf16 path reads dY
     assert b(wsb=wb - 256) == 3               # workspace too small
+
+
+def test_proxy_tensor_flag_errors():
+    L = F.lib()
+    f = L.falqon_proxy_update
+    ws = 1 << 20
+    assert f(P, P, P, P, P, 4, 16, 16, 2 | 16, None, None, None, P, ws, None) == 1       # TENSOR without ACCUMULATE
+    assert f(P, P, P, P, P, 4, 16, 16, 1 | 8 | 16, None, None, None, P, ws, None) == 1   # TENSOR with STRICT
+    assert f(P, P, P, P, P, 4, 16, 12, 1 | 16, None, None, None, P, ws, None) == 2       # r % 8
+    assert f(P, P, P, P8, P, 4, 16, 16, 1 | 16, None, None, None, P, ws, None) == 2      # unaligned dB_inc
