@@ -185,8 +185,10 @@ class Step:
     # library kernels per call of each phase (the caller's SGD is two torch ops)
     LAUNCHES = {"quantX": 1, "fwd": 1, "quantdY": 1, "adapters": 2, "dX": 1, "sgd": 0, "proxy": 2}
 
-    def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None, tensor_from=256):
+    def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None, tensor_from=256,
+                 grouped=True):
         self.torch, self.F, self.dev = torch, F, dev
+        self.grouped = grouped
         t = torch
         self.wl = wl
         self.M, self.r, self.lr = wl.M, (wl.r if r is None else r), wl.lr
@@ -249,13 +251,25 @@ class Step:
         seen = set()
         for jf, L in enumerate(self.layers):  # forward pass
             g = (L.block, L.group)
-            if g not in seen:
-                seen.add(g)
-                out.append((L, "quantX", lambda g=g: F.falqon_quantize(
-                    X[g], codes=self.xq[g], scale=self.s_x[g], amax=self.amax, dev_status=self.status,
-                    workspace=self.ws_q)))
-            out.append((L, "fwd", lambda L=L, g=g, y=yo(jf, L): F.falqon_linear_fwd(
-                self.xq[g], self.s_x[g], L.wq, L.s_w, y=y, dev_status=L.status)))
+            if g in seen:
+                continue
+            seen.add(g)
+            out.append((L, "quantX", lambda g=g: F.falqon_quantize(
+                X[g], codes=self.xq[g], scale=self.s_x[g], amax=self.amax, dev_status=self.status,
+                workspace=self.ws_q)))
+            # every layer of the group reads the same codes: one grouped launch (up to three)
+            members = [(j, M_) for j, M_ in enumerate(self.layers) if (M_.block, M_.group) == g]
+            for c0 in range(0, len(members), 3 if self.grouped else 1):
+                part = members[c0:c0 + (3 if self.grouped else 1)]
+                if len(part) == 1:
+                    j, M_ = part[0]
+                    out.append((M_, "fwd", lambda M_=M_, g=g, y=yo(j, M_): F.falqon_linear_fwd(
+                        self.xq[g], self.s_x[g], M_.wq, M_.s_w, y=y, dev_status=M_.status)))
+                else:
+                    out.append((part[0][1], "fwd", lambda part=part, g=g, ys=[yo(j, M_) for j, M_ in part]:
+                                F.falqon_linear_fwd_grouped(self.xq[g], self.s_x[g], [M_.wq for _, M_ in part],
+                                                            [M_.s_w for _, M_ in part], ys=ys,
+                                                            dev_status=part[0][1].status)))
         for j in range(len(self.layers) - 1, -1, -1):  # backward pass, last layer first
             L = self.layers[j]
             g = (L.block, L.group)
@@ -340,17 +354,25 @@ def _phase_work(st):
 
 
 def _step_work(st):
-    """_phase_work summed over the calls of one step (an activation shared by
-    several layers is quantized once)."""
+    """_phase_work summed over one step: every layer's products, every
+    activation group's quantization once (its layers share the codes); calls
+    as the step issues them (a grouped forward is one call)."""
     import types
 
     tot = {}
-    for L, p, _ in st.calls(0):
-        w = _phase_work(types.SimpleNamespace(M=st.M, N=L.N, K=L.K, r=st.r))[p]  # quantX: the group's K
-        e = tot.setdefault(p, {"flops": 0.0, "bytes": 0.0, "bound": w["bound"], "kernels": w["kernels"], "calls": 0})
+
+    def add(p, w):
+        e = tot.setdefault(p, {"flops": 0.0, "bytes": 0.0, "bound": w["bound"], "kernels": w["kernels"],
+                               "calls": st.calls_per_step[p]})
         e["flops"] += w["flops"]
         e["bytes"] += w["bytes"]
-        e["calls"] += 1
+    for L in st.layers:
+        w = _phase_work(types.SimpleNamespace(M=st.M, N=L.N, K=L.K, r=st.r))
+        for p in Step.PHASES:
+            if p != "quantX":
+                add(p, w[p])
+    for K in st.groups.values():
+        add("quantX", _phase_work(types.SimpleNamespace(M=st.M, N=K, K=K, r=st.r))["quantX"])
     return tot
 
 
@@ -386,7 +408,7 @@ def run_gpu(args):
                                        sum(l.N for l in wl.layers))
     slots = args.slots or min(8, max(2, -(-(2 * L2_BYTES) // slot_bytes)))
     st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack,
-              tensor_from=args.proxy_tensor_from)
+              tensor_from=args.proxy_tensor_from, grouped=bool(args.grouped))
     stream = torch.cuda.Stream(device=dev)
     if args.only:
         # one phase alone, eagerly, warm-up + steps times (for profiler captures)
@@ -543,7 +565,8 @@ def run_gpu(args):
                           f"({st.n_slots * slot_bytes / 2**20:.0f} MiB of X and dY, above the 126 MB L2)"),
                    "cuda_graph": not args.no_graph, "lr": wl.lr,
                    "proxy_accumulation": ("tensor cores (bf16 products, float32 sums)" if st.proxy_tensor
-                                          else "strict float32 FMA chain")},
+                                          else "strict float32 FMA chain"),
+                   "grouped_forward": st.grouped},
         "step_ms_median": round(float(np.median(per_step)), 5),
         "roofline": roof,
         "phases": phases,
@@ -882,10 +905,11 @@ def _sample_pass(O, wl, shapes, tokens, prows, step):
 
 
 def _sample_text(wl, shapes, tokens, prows, r):
-    per = "; ".join(f"{d.layer.K}->{d.layer.N} x{m}" for d, m in shapes)
+    per = "; ".join(f"{d.layer.K}->{d.layer.N} x{m}: {min(prows, d.layer.N)} of {d.layer.N} proxy rows"
+                    for d, m in shapes)
     return (f"per layer shape ({per}), r={r}: {min(tokens, wl.M)} of {wl.M} tokens through "
-            f"quantize/fwd/dX/dB/dA and {prows} proxy rows (capped at the layer's N); the "
-            f"per-token and per-row costs are scaled to one full step of every layer")
+            f"quantize/fwd/dX/dB/dA and the proxy rows listed; the per-token and per-row costs are "
+            f"scaled to one full step of every layer")
 
 
 def cpu_baseline(wl, budget_s=20.0, r=None, n_stack=None):
@@ -969,6 +993,8 @@ def main():
                     help="also time the folded quantized-adapter path (1) or skip it (0)")
     ap.add_argument("--e5m2", type=int, default=1,
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
+    ap.add_argument("--grouped", type=int, default=1,
+                    help="forward GEMMs of layers that read one activation in one grouped launch (1) or not (0)")
     ap.add_argument("--proxy-tensor-from", type=int, default=256,
                     help="rank from which the proxy accumulates on the tensor cores (0: never)")
     ap.add_argument("--separate", type=int, default=1,

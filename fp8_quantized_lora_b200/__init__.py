@@ -21,7 +21,7 @@ __all__ = [
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_linear_fwd_folded",
     "falqon_linear_bwd_folded", "folded_t_planes", "falqon_selftest_bounded_waits", "falqon_workspace_init",
     "workspace", "falqon_lora_separate_fwd", "falqon_lora_separate_bwd", "separate_saved_views",
-    "separate_bwd_views",
+    "separate_bwd_views", "falqon_linear_fwd_grouped",
     "SEPARATE_BF16", "SEPARATE_FP8", "OP_QUANTIZE",
     "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
@@ -47,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "falqon_linear_bwd_noalloc", "falqon_proxy_update_topk", "falqon_quantize_e5m2",
     "falqon_linear_bwd_e5m2", "falqon_linear_fwd_folded", "falqon_linear_bwd_folded",
     "falqon_selftest_bounded_waits", "falqon_workspace_init", "falqon_lora_separate_fwd",
-    "falqon_lora_separate_bwd",
+    "falqon_lora_separate_bwd", "falqon_linear_fwd_grouped",
 )
 
 
@@ -90,6 +90,8 @@ def lib():
     L.falqon_lora_separate_fwd.argtypes = [C.c_int, p, p, p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p, p, sz, p]
     L.falqon_lora_separate_bwd.argtypes = [C.c_int, p, p, p, p, p, p, p, p, p, p, p, sz, i64, i64, i64, i64, p, p,
                                            p, p, p, sz, p]
+    L.falqon_linear_fwd_grouped.argtypes = [p, p, C.c_int, p, p, p, p, i64, i64, p, p]
+    L.falqon_linear_fwd_grouped.restype = C.c_int
     L.falqon_workspace_init.argtypes = [p, sz, p]
     L.falqon_workspace_init.restype = C.c_int
     L.falqon_workspace_size.argtypes = [C.c_int, i64, i64, i64, i64]
@@ -207,6 +209,24 @@ def falqon_linear_fwd(xq, s_x, wq, s_w, y=None, dev_status=None, stream=None):
                                  _ptr(y), _ptr(dev_status), None, 0, _stream(stream, dev))
     _check(st, "falqon_linear_fwd")
     return y
+
+
+def falqon_linear_fwd_grouped(xq, s_x, wqs, s_ws, ys=None, dev_status=None, stream=None):
+    """Y_s = Xq . Wq_s^T / (s_x s_w_s) for up to three backbones that read the
+    same Xq, in one launch; returns the list of outputs."""
+    M, K = xq.shape
+    n = len(wqs)
+    dev = xq.device
+    if ys is None:
+        ys = [torch.empty((M, w.shape[0]), dtype=torch.bfloat16, device=dev) for w in wqs]
+    wp = (C.c_void_p * n)(*[_ptr(_u8(w)) for w in wqs])
+    sp = (C.c_void_p * n)(*[_ptr(sw) for sw in s_ws])
+    yp = (C.c_void_p * n)(*[_ptr(y) for y in ys])
+    Ns = (C.c_int64 * n)(*[int(w.shape[0]) for w in wqs])
+    st = lib().falqon_linear_fwd_grouped(_ptr(_u8(xq)), _ptr(s_x), n, wp, sp, Ns, yp, M, K, _ptr(dev_status),
+                                         _stream(stream, dev))
+    _check(st, "falqon_linear_fwd_grouped")
+    return ys
 
 
 def falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=True,

@@ -467,3 +467,27 @@ falqon_status falqon_lora_separate_bwd(int precision, const uint8_t* dyq, const 
 }
 
 }  // extern "C"
+
+extern "C" {
+
+falqon_status falqon_linear_fwd_grouped(const uint8_t* xq, const float* s_x, int nseg, const uint8_t* const* wq,
+                                        const float* const* s_w, const int64_t* N, void* const* y, int64_t M,
+                                        int64_t K, int32_t* dev_status, void* stream) {
+  if (!xq || !s_x || !wq || !s_w || !N || !y) return FALQON_ERR_INVALID_ARG;
+  if (nseg < 1 || nseg > 3 || M <= 0 || K <= 0) return FALQON_ERR_INVALID_ARG;
+  if (K % 16 != 0 || M > (int64_t(1) << 31) - 256 || K > (int64_t(1) << 31) - 256) return FALQON_ERR_UNSUPPORTED;
+  if (!aligned16(xq)) return FALQON_ERR_UNSUPPORTED;
+  int64_t tiles = 0;
+  for (int s = 0; s < nseg; ++s) {
+    if (!wq[s] || !s_w[s] || !y[s] || N[s] <= 0) return FALQON_ERR_INVALID_ARG;
+    if (N[s] % 16 != 0 || N[s] > (int64_t(1) << 31) - 256) return FALQON_ERR_UNSUPPORTED;
+    if (!aligned16(wq[s]) || !aligned16(y[s])) return FALQON_ERR_UNSUPPORTED;
+    tiles += (N[s] + 255) / 256;
+  }
+  if (tiles * ((M + 127) / 128) > (int64_t(1) << 30)) return FALQON_ERR_UNSUPPORTED;
+  if (!current_device_info()) return FALQON_ERR_CUDA;
+  return from_cuda(launch_fp8_gemm_fwd_grouped(xq, s_x, nseg, wq, s_w, N, y, M, K, dev_status,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -64,6 +64,14 @@ struct GemmArgs {
   const float* scale_b2;   // alpha2 = 1 / (scale_a * scale_b2)
   const void* addend;      // bf16 [M][ldo] added to the rounded product (nullable)
   int32_t f32_accumulate;  // out is float32 [M][ldo]: out = fl32(out + alpha * product), no bf16 rounding
+  // grouped launch (kMode 2): up to three B segments sharing A, each with its
+  // own scale and row-major bf16 output; segment s owns the tiles from
+  // seg_tile0[s] on (seg_tile0[nseg] = n_tiles)
+  int32_t nseg;
+  int32_t seg_tile0[4];
+  void* seg_out[3];
+  const float* seg_scale[3];
+  int64_t seg_n[3];
   int32_t* dev_status;
 };
 
@@ -115,13 +123,17 @@ struct Cfg {
   static_assert(AccCols <= 512, "tensor memory");
 };
 
-// kSeg2: the grid carries adapter tiles (a second B segment); the plain
-// backbone GEMMs are compiled without that code.
-template <class C, bool kSeg2>
+// kMode 0: a plain product.  1 (kSeg2): the grid also carries adapter tiles
+// (a second B segment written transposed).  2 (kGroup): up to three B
+// segments (tmB, tmB2, tmBh) share the A operand, each written row-major
+// with its own scale.  The plain GEMMs are compiled without the other code.
+template <class C, int kMode>
 __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmBh,
                    const GemmArgs g) {
+  constexpr bool kSeg2 = kMode == 1;
+  constexpr bool kGroup = kMode == 2;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -141,6 +153,16 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
   auto item = [&](int w, int& mt, int& nt, int& nh) {
     int t = w;
     nh = -1;
+    if constexpr (kMode == 2) {
+      // segment by segment (each segment's backbone stays in L2 while its
+      // tiles run), row band by row band within a segment
+      const int sg = w >= g.m_tiles * g.seg_tile0[2] ? 2 : (w >= g.m_tiles * g.seg_tile0[1] ? 1 : 0);
+      const int nts = g.seg_tile0[sg + 1] - g.seg_tile0[sg];
+      const int local = w - g.m_tiles * g.seg_tile0[sg];
+      mt = local / nts;
+      nt = g.seg_tile0[sg] + local % nts;
+      return;
+    }
     if (w >= g.n_full) {
       t = g.n_full + ((w - g.n_full) >> 1);
       nh = (w - g.n_full) & 1;
@@ -163,7 +185,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (kSeg2) tma_prefetch_desc(&tmB2);
+    if (kSeg2 || kGroup) tma_prefetch_desc(&tmB2);
+    if (kGroup && g.nseg > 2) tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TmemCols);
@@ -193,8 +216,14 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         item(w, mt, nt, nh);
         const bool seg2 = kSeg2 && nt >= g.n_tiles0;  // an adapter tile
         const CUtensorMap* tb = seg2 ? &tmB2 : &tmB;
+        int ntl = seg2 ? nt - g.n_tiles0 : nt;  // tile index within its segment
+        if constexpr (kGroup) {
+          const int sg = nt >= g.seg_tile0[2] ? 2 : (nt >= g.seg_tile0[1] ? 1 : 0);
+          tb = sg == 0 ? &tmB : (sg == 1 ? &tmB2 : &tmBh);
+          ntl = nt - g.seg_tile0[sg];
+        }
         const int m0 = mt * C::TileM;
-        const int n0 = (seg2 ? nt - g.n_tiles0 : nt) * C::BN + (nh > 0 ? C::HalfN : 0);
+        const int n0 = ntl * C::BN + (nh > 0 ? C::HalfN : 0);
         for (int kb = 0; kb < g.kb_total; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { fail(); ok = false; break; }
           uint8_t* sA = smem + stage * C::StageBytes;
@@ -309,6 +338,12 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         alpha2 = static_cast<float>(1.0 / den2);
       }
     }
+    float seg_alpha[3] = {alpha, alpha, alpha};
+    if constexpr (kGroup) {
+      const double sa = g.scale_a ? static_cast<double>(*g.scale_a) : 1.0;
+      for (int sg = 0; sg < g.nseg && sg < 3; ++sg)
+        seg_alpha[sg] = static_cast<float>(1.0 / (g.seg_scale[sg] ? sa * static_cast<double>(*g.seg_scale[sg]) : sa));
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int w = blockIdx.x; w < total; w += gridDim.x) {
@@ -348,7 +383,17 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         if (++acc == C::Acc) { acc = 0; acc_phase ^= 1; }
         continue;
       }
-      const int64_t col_base = static_cast<int64_t>(nt) * C::BN + (nh > 0 ? C::HalfN : 0);
+      int64_t col_base = static_cast<int64_t>(nt) * C::BN + (nh > 0 ? C::HalfN : 0);
+      void* out = g.out;
+      int64_t ldo = g.ldo, ncols = g.N;
+      float alpha_t = alpha;
+      if constexpr (kGroup) {
+        const int sg = nt >= g.seg_tile0[2] ? 2 : (nt >= g.seg_tile0[1] ? 1 : 0);
+        col_base = static_cast<int64_t>(nt - g.seg_tile0[sg]) * C::BN;
+        out = g.seg_out[sg];
+        ldo = ncols = g.seg_n[sg];
+        alpha_t = seg_alpha[sg];
+      }
       const int chunks = (nh >= 0 ? C::HalfN : C::BN) / 32;
 #pragma unroll 1
       for (int c = 0; c < chunks; ++c) {
@@ -389,20 +434,20 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
           }
         }
         if (row < g.M) {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(g.out) + row * g.ldo;
-          const __nv_bfloat16* add = g.addend ? static_cast<const __nv_bfloat16*>(g.addend) + row * g.ldo : nullptr;
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(out) + row * ldo;
+          const __nv_bfloat16* add = g.addend ? static_cast<const __nv_bfloat16*>(g.addend) + row * ldo : nullptr;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int64_t col = col_base + c * 32 + 8 * j;
-            if (col < g.N) {
+            if (col < ncols) {
               uint32_t pk[4];
               uint4 ad = make_uint4(0u, 0u, 0u, 0u);
               if (add) ad = *reinterpret_cast<const uint4*>(add + col);
               const uint32_t aw[4] = {ad.x, ad.y, ad.z, ad.w};
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
-                __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * h]) * alpha,
-                                                         __uint_as_float(r[8 * j + 2 * h + 1]) * alpha);
+                __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r[8 * j + 2 * h]) * alpha_t,
+                                                         __uint_as_float(r[8 * j + 2 * h + 1]) * alpha_t);
                 if (add) {
                   // the product rounded to bf16, then added as bf16 tensors add:
                   // a float32 sum rounded once to bf16
@@ -433,7 +478,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
 }
 
 // ---------------------------------------------------------------- host side
-template <class C, bool kSeg2>
+template <class C, int kMode>
 cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const CUtensorMap& tBh,
                         GemmArgs g, cudaStream_t stream) {
   const DeviceInfo* di = current_device_info();
@@ -441,7 +486,7 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
   static int configured_mask = 0;  // one bit per device ordinal < 31
   const int bit = di->device < 31 ? (1 << di->device) : 0;
   if (!bit || !(__atomic_load_n(&configured_mask, __ATOMIC_ACQUIRE) & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C, kSeg2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<C, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SmemBytes);
     if (e != cudaSuccess) return e;
     if (bit) __atomic_fetch_or(&configured_mask, bit, __ATOMIC_ACQ_REL);
@@ -455,11 +500,11 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
   const int tail = tiles % grid;
   g.n_full = tiles;
   g.n_half = 0;
-  if (!kSeg2 && C::BN == 2 * C::HalfN && tiles > grid && tail > 0 && 2 * tail <= grid) {
+  if (kMode == 0 && C::BN == 2 * C::HalfN && tiles > grid && tail > 0 && 2 * tail <= grid) {
     g.n_full = tiles - tail;
     g.n_half = 2 * tail;
   }
-  return launch_pdl(tc_gemm_kernel<C, kSeg2>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2,
+  return launch_pdl(tc_gemm_kernel<C, kMode>, dim3(grid), dim3(C::Threads), C::SmemBytes, stream, 1u, tA, tB, tB2,
                     tBh, g);
 }
 
@@ -537,8 +582,8 @@ cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* 
   g.f32_accumulate = f32_accumulate ? 1 : 0;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
-  if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, true>(tA, tB, tB2, tBh, g, stream);
-  return launch_gemm<C, false>(tA, tB, tB2, tBh, g, stream);
+  if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, 1>(tA, tB, tB2, tBh, g, stream);
+  return launch_gemm<C, 0>(tA, tB, tB2, tBh, g, stream);
 }
 
 template <class C>
@@ -546,6 +591,44 @@ cudaError_t fp8_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const 
                      int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
                      cudaStream_t stream, const Segment2& s2 = Segment2{}) {
   return tc_gemm<C>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, s2);
+}
+
+// Grouped forward (kMode 2): Y_s = bf16(Xq . Wq_s^T / (s_X s_W_s)) for up to
+// three backbones Wq_s [N_s, Kc] that read the same quantized activation.
+cudaError_t fp8_gemm_grouped(const uint8_t* a, const float* sa, int nseg, const uint8_t* const* b,
+                             const float* const* sb, const int64_t* n, void* const* out, int64_t M, int64_t Kc,
+                             int32_t* dev_status, cudaStream_t stream) {
+  using C = FwdCfg;
+  CUtensorMap tA, tb[3];
+  if (!make_tmap_2d(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a, Kc, M, C::BK, kBM, true)) return cudaErrorInvalidValue;
+  GemmArgs g{};
+  g.nseg = nseg;
+  int tiles = 0;
+  for (int sg = 0; sg < 3; ++sg) {
+    g.seg_tile0[sg] = tiles;
+    if (sg < nseg) {
+      if (!b_tmap<C>(&tb[sg], b[sg], n[sg], Kc)) return cudaErrorInvalidValue;
+      g.seg_out[sg] = out[sg];
+      g.seg_scale[sg] = sb[sg];
+      g.seg_n[sg] = n[sg];
+      tiles += ceil_div(n[sg], C::BN);
+    } else {
+      tb[sg] = tb[0];  // an absent segment owns no tile: its first tile is the end
+    }
+  }
+  g.seg_tile0[3] = tiles;
+  g.m_tiles = ceil_div(M, C::TileM);
+  g.n_tiles = g.n_tiles0 = tiles;
+  g.kb_total = ceil_div(Kc, C::BK);
+  g.M = M;
+  g.N = n[0];
+  g.out = out[0];
+  g.ldo = n[0];
+  g.scale_a = sa;
+  g.scale_b = sb[0];
+  g.dev_status = dev_status;
+  if (tiles == 0) return cudaSuccess;
+  return launch_gemm<C, 2>(tA, tb[0], tb[1], tb[2], g, stream);
 }
 
 using BfFwdCfg = Cfg<false, 256, 4, 2, 1, 1, 0, true>;  // bf16 operands, B K-major
@@ -598,6 +681,12 @@ cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void
                            cudaStream_t stream, int64_t lda) {
   return bf16 ? tc_gemm<BfDxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda)
               : tc_gemm<DxCfg>(a, sa, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, addend, lda);
+}
+
+cudaError_t launch_fp8_gemm_fwd_grouped(const uint8_t* xq, const float* s_x, int nseg, const uint8_t* const* wq,
+                                        const float* const* s_w, const int64_t* n, void* const* y, int64_t M,
+                                        int64_t K, int32_t* dev_status, cudaStream_t stream) {
+  return fp8_gemm_grouped(xq, s_x, nseg, wq, s_w, n, y, M, K, dev_status, stream);
 }
 
 cudaError_t launch_gemm_nn_f32acc(const void* a, const void* b, int64_t M, int64_t Ncols, int64_t Kc, float* out,

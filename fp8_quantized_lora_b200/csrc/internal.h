@@ -78,6 +78,11 @@ cudaError_t launch_quantize(const void* x, bool is_bf16, int64_t n, uint8_t* cod
 cudaError_t launch_fp8_gemm_fwd(const uint8_t* xq, const float* s_x, const uint8_t* wq,
                                 const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
                                 int32_t* dev_status, cudaStream_t stream);
+// Y_s[M, N_s] = bf16( Xq . Wq_s^T / (s_x s_w_s) ), s < nseg <= 3: one launch over
+// the concatenated output tiles of backbones that read the same Xq.
+cudaError_t launch_fp8_gemm_fwd_grouped(const uint8_t* xq, const float* s_x, int nseg, const uint8_t* const* wq,
+                                        const float* const* s_w, const int64_t* n, void* const* y, int64_t M,
+                                        int64_t K, int32_t* dev_status, cudaStream_t stream);
 // dX[M,K] = bf16( dYq . Wq / (s_dy s_w) )
 cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,

@@ -167,6 +167,27 @@ FALQON_API falqon_status falqon_linear_fwd(const uint8_t* xq, const float* s_x, 
                                 void* stream);
 
 /*
+ * falqon_linear_fwd_grouped - the forward of up to three layers that read the
+ * same activation, in one launch.
+ *
+ * In a transformer block the query, key and value projections (and the MLP's
+ * gate and up projections) read the same input; under FALQON each is the
+ * FP8 backbone alone (as falqon_linear_fwd), so one quantized X serves all of
+ * them:  Y_s = bf16( Xq . Wq_s^T / (s_X s_W_s) ),  s = 0 .. nseg-1.
+ * One tcgen05 GEMM walks the concatenated output tiles of the segments; each
+ * output equals falqon_linear_fwd's on the same operands, bit for bit.
+ *
+ *  xq [M, K], s_x as falqon_linear_fwd.  nseg: 1 to 3.  wq, s_w, N, y: HOST
+ *  arrays of nseg entries: wq[s] [N[s], K] E4M3 (device), s_w[s] 1 float
+ *  (device), y[s] [M, N[s]] bfloat16 (device), written.
+ *  Requirements: M >= 1; K and every N[s] multiples of 16.
+ */
+FALQON_API falqon_status falqon_linear_fwd_grouped(const uint8_t* xq, const float* s_x, int nseg,
+                                                   const uint8_t* const* wq, const float* const* s_w,
+                                                   const int64_t* N, void* const* y, int64_t M, int64_t K,
+                                                   int32_t* dev_status, void* stream);
+
+/*
  * falqon_linear_bwd - backward of the melded layer.
  *
  *   dX = dYq . Wq / (s_dY s_W)                      (backbone only; [M, K])

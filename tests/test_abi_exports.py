@@ -244,3 +244,16 @@ def test_proxy_tensor_flag_errors():
     assert f(P, P, P, P, P, 4, 16, 16, 1 | 8 | 16, None, None, None, P, ws, None) == 1   # TENSOR with STRICT
     assert f(P, P, P, P, P, 4, 16, 12, 1 | 16, None, None, None, P, ws, None) == 2       # r % 8
     assert f(P, P, P, P8, P, 4, 16, 16, 1 | 16, None, None, None, P, ws, None) == 2      # unaligned dB_inc
+
+
+def test_grouped_forward_argument_errors():
+    L = F.lib()
+    f = L.falqon_linear_fwd_grouped
+    arr = lambda *v: (C.c_void_p * len(v))(*v)
+    n = lambda *v: (C.c_int64 * len(v))(*v)
+    assert f(P, P, 0, arr(P), arr(P), n(16), arr(P), 64, 32, None, None) == 1        # no segment
+    assert f(P, P, 4, arr(P, P, P, P), arr(P, P, P, P), n(16, 16, 16, 16), arr(P, P, P, P), 64, 32, None, None) == 1
+    assert f(P, P, 2, arr(P, None), arr(P, P), n(16, 16), arr(P, P), 64, 32, None, None) == 1  # a missing backbone
+    assert f(P, P, 2, arr(P, P), arr(P, P), n(16, 24), arr(P, P), 64, 32, None, None) == 2     # N % 16
+    assert f(P, P, 1, arr(P), arr(P), n(16), arr(P8), 64, 32, None, None) == 2                # unaligned output
+    assert f(P, P, 1, arr(P), arr(P), n(16), arr(P), 64, 40, None, None) == 2                 # K % 16
