@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         int32_t* __restrict__ dev_status, int keep_residual) {
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
-  extern __shared__ __align__(16) uint8_t sm[];
+  extern __shared__ __align__(128) uint8_t sm[];
   __shared__ int tile_flag[kTileRows];  // a code of the row changed
   uint16_t* As = reinterpret_cast<uint16_t*>(sm);                              // [kIChunk][256]
   float2* Bs = reinterpret_cast<float2*>(sm + kAsBytes);                       // [kIChunk][32]

@@ -293,9 +293,9 @@ __global__ void __launch_bounds__(kThreads)
 // contiguous run of 16 KB chunks of x.  Warp 0 (one lane) streams the chunks
 // into a ring of shared-memory slots with bulk asynchronous copies; sixteen
 // consumer warps read each slot, then release it.  Pass 1 reduces max|x|;
-// every CTA publishes its maximum in a marked workspace word and waits
-// (bounded) until all words are marked, reduces them, and pass 2 writes the
-// codes: from the ring in place when the CTA's run fits it (up to 14 chunks:
+// every CTA publishes its maximum in a tagged workspace word, the last CTA
+// to arrive reduces them and publishes max|x| in one word that the others
+// wait for (bounded), and pass 2 writes the codes: from the ring in place when the CTA's run fits it (up to 14 chunks:
 // a 4096 x 4096 bf16 tensor on 148 SMs), else streaming the run again (it is
 // still in L2).
 constexpr int kChunkBytes = 16384;
@@ -303,7 +303,8 @@ constexpr int kStreamStages = 14;                      // 224 KB in flight per S
 constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
-constexpr int kBarWords = 64;                          // per-CTA words start 256 bytes in
+constexpr int kBarWords = 64;                          // per-CTA words start 256 bytes in (0: generation,
+                                                       // 1: arrivals, 2-3: result)
 constexpr int kExchangeWords = 4096;                   // generation + 64-bit words of at most 2016 CTAs
 constexpr int kPartialWords = 1024;                    // two-launch path: its per-CTA partial maxima
 constexpr long long kBarrierBudget = 2000000000LL;    // cycles (about 1 s), then give up
@@ -431,58 +432,71 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
   m = block_max_u32(m, red);
 
   // Grid exchange of the per-CTA maxima (the launch is cooperative, so every
-  // CTA is resident).  The workspace holds a generation counter g (word 0)
-  // and one 64-bit word per CTA.  Every CTA read g at its start; it publishes
-  // (g + 1) << 32 | max with a release store, and warp 0 of every CTA polls
-  // all words (relaxed loads, one acquire fence once all carry the tag
-  // g + 1), bounded, and reduces them.  Words left by earlier calls carry
-  // older tags, so nothing is cleared between calls; CTA 0 advances g once
-  // its own exchange is over (or its wait ran out), after every CTA has read
-  // it.  A poll round issues all of a lane's loads before it looks at any:
-  // one L2 round trip per round, not one per word.
+  // CTA is resident).  The workspace holds a generation counter g (word 0),
+  // an arrival counter (word 1), one result word (words 2-3) and one 64-bit
+  // word per CTA.  Every CTA read g at its start.  It publishes
+  // (g + 1) << 32 | max in its word, then (release) increments the arrival
+  // counter; the CTA that arrives last (acquire) reads every CTA's word,
+  // reduces them, resets the arrival counter, advances g (every CTA has read
+  // it) and publishes (g + 1) << 32 | amax in the result word, which the
+  // other CTAs poll (relaxed loads of one word, bounded, then one acquire
+  // fence).  The increment is unconditional, so the counter returns to zero
+  // after every call, and words left by earlier calls carry older tags:
+  // nothing is cleared between calls.
+  uint32_t* arrivals = ws + 1;
+  uint64_t* result = reinterpret_cast<uint64_t*>(ws + 2);
   uint64_t* words = reinterpret_cast<uint64_t*>(ws + kBarWords);
   const uint64_t tag = static_cast<uint64_t>(gen + 1u) << 32;
   __shared__ uint32_t amax_bits;
   if (warp == 0) {
-    if (lane == 0)
-      asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(words + blockIdx.x), "l"(tag | m) : "memory");
-    __syncwarp();
-    const long long t0 = clock64();
+    uint32_t last = 0;
+    if (lane == 0) {
+      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(words + blockIdx.x), "l"(tag | m) : "memory");
+      uint32_t old;
+      asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(arrivals) : "memory");
+      last = old == gridDim.x - 1 ? 1u : 0u;
+    }
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
     uint32_t mx = 0;
-    constexpr int kPerLane = 8;  // words per lane per batch of loads (256 CTAs)
-    while (true) {
-      bool all = true;
-      mx = 0;
-      for (int b = 0; b < static_cast<int>(gridDim.x); b += 32 * kPerLane) {
+    if (last) {
+      // every CTA's word is published (its increment released it): reduce them
+      constexpr int kPerLane = 8;  // words per lane per batch of loads (256 CTAs)
+      for (int b0 = 0; b0 < static_cast<int>(gridDim.x); b0 += 32 * kPerLane) {
         uint64_t w[kPerLane];
 #pragma unroll
         for (int k = 0; k < kPerLane; ++k) {
-          const int i = b + lane + 32 * k;
-          w[k] = tag;  // absent CTAs count as arrived with max 0
+          const int i = b0 + lane + 32 * k;
+          w[k] = tag;
           if (i < static_cast<int>(gridDim.x))
             asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w[k]) : "l"(words + i));
         }
 #pragma unroll
-        for (int k = 0; k < kPerLane; ++k) {
-          all = all && (w[k] & 0xFFFFFFFF00000000ull) == tag;
-          mx = max(mx, static_cast<uint32_t>(w[k]));
+        for (int k = 0; k < kPerLane; ++k) mx = max(mx, static_cast<uint32_t>(w[k]));
+      }
+      mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+      if (lane == 0) {
+        *reinterpret_cast<volatile uint32_t*>(arrivals) = 0u;  // ready for the next call
+        *reinterpret_cast<volatile uint32_t*>(ws) = gen + 1u;    // every CTA has read this generation
+        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(result), "l"(tag | mx) : "memory");
+      }
+    } else {
+      const long long t0 = clock64();
+      uint64_t w = 0;
+      while (true) {
+        if (lane == 0) asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(result));
+        w = __shfl_sync(0xFFFFFFFFu, w, 0);
+        if ((w & 0xFFFFFFFF00000000ull) == tag) {
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the result word
+          break;
+        }
+        if (clock64() - t0 > kBarrierBudget) {
+          if (lane == 0 && dev_status) atomicOr(dev_status, kDevTimeout);
+          break;
         }
       }
-      if (__all_sync(0xFFFFFFFFu, all)) {
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the tagged words
-        break;
-      }
-      if (clock64() - t0 > kBarrierBudget) {
-        if (lane == 0 && dev_status) atomicOr(dev_status, kDevTimeout);
-        break;
-      }
+      mx = static_cast<uint32_t>(w);
     }
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) {
-      amax_bits = mx;
-      if (blockIdx.x == 0)  // every CTA has read the generation: the next call may use the next one
-        asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(ws), "r"(gen + 1u) : "memory");
-    }
+    if (lane == 0) amax_bits = mx;
   }
   __syncthreads();
   const float s = scale_from_amax(amax_bits, kFmtMax<kE5>, &s_shared, scale_out, amax_out, dev_status);
