@@ -338,7 +338,7 @@ def _phase_work(st):
         "quantX": {"flops": 0.0, "bytes": 3.0 * M * K, "bound": "hbm",
                    "kernels": "quantize_stream_kernel"},
         "fwd": {"flops": 2.0 * M * N * K, "bytes": M * K + N * K + 2.0 * M * N, "bound": "tensor",
-                "kernels": "tc_gemm_kernel (forward)"},
+                "kernels": "tc_gemm_pair_kernel (forward)"},
         "quantdY": {"flops": 0.0, "bytes": 3.0 * M * N, "bound": "hbm",
                     "kernels": "quantize_stream_kernel"},
         # each code matrix is read by two products; A, B, dA, dB and the T / U hi-lo pairs
@@ -346,7 +346,7 @@ def _phase_work(st):
                      "bytes": 2.0 * (M * K + M * N) + 4.0 * r * (N + K) + 16.0 * M * r,
                      "bound": "hbm", "kernels": "skinny_kernel x2 (T^T with U^T, dB^T with dA)"},
         "dX": {"flops": 2.0 * M * N * K, "bytes": M * N + N * K + 2.0 * M * K, "bound": "tensor",
-               "kernels": "tc_gemm_kernel (dX)"},
+               "kernels": "tc_gemm_pair_kernel (dX)"},
         "sgd": {"flops": 0.0, "bytes": 8.0 * N * r, "bound": None, "kernels": "torch (caller's SGD)"},
         "proxy": {"flops": proxy_flops, "bytes": proxy_bytes, "bound": "alu" if proxy_alu else "hbm",
                   "kernels": "proxy_ws_kernel + proxy_clear_kernel"},

@@ -88,6 +88,15 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
                                int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
 
+// The same two products on pairs of SMs (tcgen05 cta_group::2, 256 x 256
+// tiles); launch_fp8_gemm_fwd / _dx route here.
+cudaError_t launch_fp8_gemm_fwd_pair(const uint8_t* xq, const float* s_x, const uint8_t* wq, const float* s_w,
+                                     int64_t M, int64_t N, int64_t K, void* y, int32_t* dev_status,
+                                     cudaStream_t stream);
+cudaError_t launch_fp8_gemm_dx_pair(const uint8_t* dyq, const float* s_dy, const uint8_t* wq, const float* s_w,
+                                    int64_t M, int64_t N, int64_t K, void* dx, int32_t* dev_status,
+                                    cudaStream_t stream, bool dy_e5m2);
+
 // Plain products on the tcgen05 GEMM: C[M, Ncols] = bf16(A . op(B) / (sa sb)),
 // then, when addend is not null, bf16(fl32(C + addend)) (bf16 tensors adding).
 // A [M, Kc] K-major.  _nt: B [Ncols, Kc] (K-major);  _nn: B [Kc, Ncols] (MN-major).

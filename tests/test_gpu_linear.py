@@ -67,9 +67,11 @@ def test_dx(cuda_device, M, N, K):
 
 
 def test_partial_last_wave_runs_as_half_tiles(cuda_device):
-    """185 output tiles of 128 x 256 on 148 SMs: the 37 tiles of the last
-    wave run as 74 half tiles (128 x 128, N = 128 MMAs, half the B bytes).
-    Every output element is compared, the forward and dX both."""
+    """A grid whose last wave is partial: 19 x 5 = 95 output tiles of
+    256 x 256 on the SM pairs (74 on a 148-SM B200), the last M band half
+    empty.  In the forward the 21 tiles of the last wave run as 42 halves
+    (256 x 128: N = 128 pair MMAs, 64 B rows per CTA); dX (MN-major B) runs
+    them whole.  Every output element is compared, the forward and dX both."""
     O.set_threads(os.cpu_count() or 8)
     M, N, K = 37 * 128, 5 * 256, 256
     xq, s_x = _codes(811, (M, K))
@@ -104,3 +106,21 @@ def test_llama_shapes_sampled_rows(cuda_device, M, N, K):
     dx = _dx(dyq, s_dy, wq, s_w)
     for r0 in rows:
         _assert_close(dx[r0], O.linear_dx(dyq, s_dy, wq, s_w, rows=(r0, r0 + 1))[0], ("dx", r0))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (2048, 3328, 256),   # 8 x 13 = 104 tiles of 256 x 256: 74 whole, 30 tiles as 60 halves
+    (512, 4096, 384),    # 2 x 16 = 32 tiles: fewer tiles than pairs, K not a multiple of 256
+    (300, 200, 144),     # one tile, both operands ragged: rows and columns past the ends
+])
+def test_pair_tiles_and_tails(cuda_device, M, N, K):
+    """The SM-pair GEMM (256 x 256 tiles, each CTA staging 128 rows of A and
+    128 columns of B) on grids with a partial last wave, fewer tiles than
+    pairs, and tiles that overhang both operands."""
+    O.set_threads(os.cpu_count() or 8)
+    xq, s_x = _codes(900 + M, (M, K))
+    wq, s_w = _codes(901 + N, (N, K), 0.02)
+    _assert_close(_fwd(xq, s_x, wq, s_w), O.linear_fwd(xq, s_x, wq, s_w), ("fwd", M, N, K))
+    dyq, s_dy = _codes(902 + M, (M, K), 1e-3)  # dX [M, N]: contraction over K here
+    wq2, s_w2 = _codes(903 + N, (K, N), 0.02)
+    _assert_close(_dx(dyq, s_dy, wq2, s_w2), O.linear_dx(dyq, s_dy, wq2, s_w2), ("dx", M, N, K))
