@@ -101,6 +101,20 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_2d_sw64(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
+                       uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc || box_inner * elem_bytes != 64) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace falqon
 
 using namespace falqon;

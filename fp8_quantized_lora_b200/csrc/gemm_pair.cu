@@ -29,9 +29,11 @@
 // bounded (FALQON_DEV_TIMEOUT).
 //
 // Scheduling: persistent, one pair per two SMs as far as the device can
-// co-schedule clusters of two; pairs take 256 x 256 tiles round robin.
-// With K-major B (the forward) a partial last wave of at most half the pairs
-// runs as 256 x 128 halves.
+// co-schedule clusters of two; pairs take 256 x 256 tiles round robin.  A
+// partial last wave of at most half the pairs runs as 256 x 128 halves
+// (N = 128 pair MMAs, 64 columns of B per CTA).  An MN-major half is 64
+// bytes wide, so it is staged with the 64-byte swizzle (8-row x 64-byte
+// atoms) and described to the MMA as such.
 #include <algorithm>
 
 #include "internal.h"
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
     fence_barrier_init();  // visible to the other CTA's copies and arrivals
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (!C::BMn) tma_prefetch_desc(&tmBh);
+    tma_prefetch_desc(&tmBh);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TmemCols);
@@ -166,8 +168,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           const uint32_t fb = full_lead + 8u * static_cast<uint32_t>(stage);
           tma_load_2d_pair(sA, &tmA, fb, kb * C::BK, m0);
-          if constexpr (C::BMn)
-            tma_load_2d_pair(sB, &tmB, fb, n0, kb * C::BK);  // [K rows][128 columns]: one 128-byte block
+          if constexpr (C::BMn)  // [K rows][128 columns]: one 128-byte block (64 for a half: 64-byte swizzle)
+            tma_load_2d_pair(sB, halfi ? &tmBh : &tmB, fb, n0, kb * C::BK);
           else
             tma_load_2d_pair(sB, halfi ? &tmBh : &tmB, fb, kb * C::BK, n0);
           if (++stage == C::Stages) { stage = 0; phase ^= 1; }
@@ -189,7 +191,8 @@ __global__ void __launch_bounds__(C::Threads, 1)
         if (bar_red_or(kPairMmaBar, 64, false)) break;
         tc_fence_after();
         const uint32_t tmem_d = tmem_base + static_cast<uint32_t>(acc * C::TileN);
-        const uint32_t idesc = w >= g.n_full ? C::IDescHalf : C::IDesc;
+        const bool halfi = w >= g.n_full;
+        const uint32_t idesc = halfi ? C::IDescHalf : C::IDesc;
         bool abort = false;
         for (int kb = 0; kb < g.kb_total; ++kb) {
           if (bar_red_or(kPairMmaBar, 64, false)) { abort = true; break; }
@@ -198,9 +201,13 @@ __global__ void __launch_bounds__(C::Threads, 1)
             const uint32_t a_base = smem_u32(smem + stage * C::StageBytes);
             const uint32_t b_base = a_base + C::ABytes;
 #pragma unroll
-            for (int ks = 0; ks < C::KSteps; ++ks)
-              umma_f8_pair(tmem_d, operand_desc<false, 1, C::BK>(a_base, ks),
-                           operand_desc<C::BMn, 1, C::BK>(b_base, ks), idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < C::KSteps; ++ks) {
+              // an MN-major half tile: [K rows][64 bytes], 64-byte swizzle, 8-row atoms 512 B apart
+              const uint64_t bd = (C::BMn && halfi) ? sdesc_sw64(b_base + ks * 32 * 64, 64 * C::BK, 512)
+                                                    : operand_desc<C::BMn, 1, C::BK>(b_base, ks);
+              umma_f8_pair(tmem_d, operand_desc<false, 1, C::BK>(a_base, ks), bd, idesc,
+                           (kb > 0 || ks > 0) ? 1u : 0u);
+            }
             umma_commit_pair_both(&empty[stage]);
           }
           __syncwarp();
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-// Six stages of 32 KB.
+// Six stages of 32 KB (seven measured the same).
 using PairFwdCfg = PairCfg<false, 0u, 6>;
 using PairDxCfg = PairCfg<true, 0u, 6>;
 using PairDxE5Cfg = PairCfg<true, 1u, 6>;  // dYq in E5M2
@@ -353,7 +360,7 @@ cudaError_t pair_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const
   if constexpr (C::BMn) {
     // B [Kc, Ncols] row-major: boxes of 128 columns (one 128-byte block) x BK rows
     if (!make_tmap_2d(&tB, U8, 1, b, Ncols, Kc, C::TileN / 2, C::BK, true)) return cudaErrorInvalidValue;
-    tBh = tB;
+    if (!make_tmap_2d_sw64(&tBh, U8, 1, b, Ncols, Kc, C::TileN / 4, C::BK)) return cudaErrorInvalidValue;
   } else {
     // B [Ncols, Kc] K-major: boxes of BK codes x 128 rows (64 for half tiles)
     if (!make_tmap_2d(&tB, U8, 1, b, Kc, Ncols, C::BK, C::TileN / 2, true)) return cudaErrorInvalidValue;
@@ -374,11 +381,11 @@ cudaError_t pair_gemm(const uint8_t* a, const float* sa, const uint8_t* b, const
   if (tiles == 0) return cudaSuccess;
   const int slots = resident_pairs<C>(di);
   const int pairs = tiles < slots ? tiles : slots;
-  // a partial last wave of at most half the pairs runs as 256 x 128 halves (K-major B only)
+  // a partial last wave of at most half the pairs runs as 256 x 128 halves
   const int tail = tiles % pairs;
   g.n_full = tiles;
   g.n_half = 0;
-  if (!C::BMn && tiles > pairs && tail > 0 && 2 * tail <= pairs) {
+  if (tiles > pairs && tail > 0 && 2 * tail <= pairs) {
     g.n_full = tiles - tail;
     g.n_half = 2 * tail;
   }

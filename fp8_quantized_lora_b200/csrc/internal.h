@@ -35,6 +35,9 @@ EncodeTiledFn encode_tiled_fn();
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes,
                   const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
                   uint32_t box_outer, bool swizzle128, uint64_t ld = 0);
+// The same with the 64-byte swizzle (box_inner * elem_bytes == 64).
+bool make_tmap_2d_sw64(CUtensorMap* map, CUtensorMapDataType dtype, size_t elem_bytes, const void* base,
+                       uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer);
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

@@ -111,7 +111,7 @@ def test_llama_shapes_sampled_rows(cuda_device, M, N, K):
 @pytest.mark.parametrize("M,N,K", [
     (2048, 3328, 256),   # 8 x 13 = 104 tiles of 256 x 256: 74 whole, 30 tiles as 60 halves
     (512, 4096, 384),    # 2 x 16 = 32 tiles: fewer tiles than pairs, K not a multiple of 256
-    (300, 200, 144),     # one tile, both operands ragged: rows and columns past the ends
+    (300, 208, 144),     # one tile, both operands ragged: rows and columns past the ends
 ])
 def test_pair_tiles_and_tails(cuda_device, M, N, K):
     """The SM-pair GEMM (256 x 256 tiles, each CTA staging 128 rows of A and
