@@ -11,7 +11,8 @@
 //   dA   = (U_hi + U_lo)^T . Xq / s_X     [r, K]  A-op U^T hi over lo, B-op Xq codes MN-major
 // T and U are kept as bf16 hi/lo pairs, stored transposed ([r, M]).  In dB
 // and dA the hi and lo operands fill the upper and lower 64 rows of one
-// M = 128 tile, and the reduction adds the two halves.
+// M = 128 tile; each CTA adds the two halves of its fp32 tile before the
+// cluster sums its split-K partners.
 //
 // The E4M3 codes are expanded exactly to bf16 in shared memory (every E4M3
 // value is a bf16 value) and fed to tcgen05 kind::f16 as the B operand.  One
@@ -29,7 +30,9 @@
 // Roles per CTA:
 //   warp 0       TMA producer for the bf16 A operand (one lane)
 //   warp 1       TMEM owner; MMA issuer for even K-block pairs (one lane)
-//   warps 2-5    epilogue: TMEM -> fp32 reduction tile in shared memory
+//   warps 2-5    idle until the drain
+// After the last MMA all 16 warps drain TMEM into an fp32 tile in shared
+// memory (warp w: lane quarter w % 4, 64-column slice w / 4).
 //   warps 6-13   converters: raw E4M3 tile -> bf16, 128-byte-swizzled
 //   warp 14      TMA producer for the raw E4M3 tiles (one lane)
 //   warp 15      MMA issuer for odd K-block pairs (one lane)
@@ -263,45 +266,7 @@ __global__ void __launch_bounds__(C::Threads, 1)
     }
     __syncwarp();
   } else if (warp < 6) {
-    // ------------------------------------------------------------ epilogue
-    // acc0 + acc1 -> fp32 reduction tile in shared memory (the ring is idle
-    // once every MMA has completed): [rank][col] for row-major outputs,
-    // [col][rank] for transposed ones, so that either reduction reads
-    // float4 along the output's contiguous dimension.
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    if (warp_wait(acc_full, 0, abort_flag)) {
-      tc_fence_after();
-      const int row = q * 32 + lane;
-      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      float* red = reinterpret_cast<float*>(smem);
-#pragma unroll 1
-      for (int c = 0; c < kSkN / 16; ++c) {
-        float v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-#pragma unroll
-        for (int a = 0; a < 2; ++a) {
-          if (npairs > a) {
-            uint32_t r[16];
-            tmem_ld_16cols(lane_base + a * kSkN + c * 16, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
-          }
-        }
-        if (g.transpose) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) red[(c * 16 + j) * C::RedStrideT + row] = v[j];
-        } else {
-          float4* dst = reinterpret_cast<float4*>(red + row * C::RedStride + c * 16);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        }
-      }
-    } else if (lane == 0) {
-      fail();
-    }
-    tc_fence_before();
+    // epilogue warps: they join the drain below with every other warp
   } else {
     // ------------------------------------------------------------ converters
     // 256 threads; each expands four 16-byte chunks (64 codes) of every tile:
@@ -341,16 +306,19 @@ __global__ void __launch_bounds__(C::Threads, 1)
         break;
       }
       uint8_t* sB = ring + s * C::StageBytes + C::ABytes + blk * kBlkBytes;
+      // MN-major tiles: the 16 lanes of a half-warp share one row and cover
+      // four column blocks; odd blocks store their two 16-byte units in the
+      // other order, so that each store instruction meets every bank pair twice
+      const int swap = C::BMn ? (blk & 1) : 0;
 #pragma unroll
       for (int j = 0; j < C::ChunksPerThread; ++j) {
         uint32_t o[8];
         if (e5) e5m2x16_to_bf16(q[j], nan, o);
         else e4m3x16_to_bf16(q[j], nan, o);
         const int row = trow + j * kRowStep;
-        *reinterpret_cast<uint4*>(sB + row * kRowBytes + ((unit0 ^ (row & 7)) << 4)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(sB + row * kRowBytes + (((unit0 + 1) ^ (row & 7)) << 4)) =
-            make_uint4(o[4], o[5], o[6], o[7]);
+        const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]), hi = make_uint4(o[4], o[5], o[6], o[7]);
+        *reinterpret_cast<uint4*>(sB + row * kRowBytes + (((unit0 + swap) ^ (row & 7)) << 4)) = swap ? hi : lo;
+        *reinterpret_cast<uint4*>(sB + row * kRowBytes + (((unit0 + 1 - swap) ^ (row & 7)) << 4)) = swap ? lo : hi;
       }
       fence_proxy_async_smem();
       // the stage's A tile must have landed too: pconv[] then covers both operands
@@ -364,10 +332,76 @@ __global__ void __launch_bounds__(C::Threads, 1)
     }
   }
 
+  // ---------------------------------------------------------------- drain
+  // acc0 + acc1 -> fp32 reduction tile in shared memory (the ring is idle once
+  // every MMA has completed), by all 16 warps: warp w reads TMEM lane quarter
+  // w % 4 and the 64 columns of slice w / 4.  [rank][col] for row-major
+  // outputs, [col][rank] for transposed ones, so that the reduction reads
+  // float4 along the output's contiguous dimension.
+  __syncwarp();
+  {
+    const int q = warp & 3, slice = warp >> 2;
+    if (warp_wait(acc_full, 0, abort_flag)) {
+      tc_fence_after();
+      const int row = q * 32 + lane;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      float* red = reinterpret_cast<float*>(smem);
+#pragma unroll 1
+      for (int c = slice * 4; c < slice * 4 + 4; ++c) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+#pragma unroll
+        for (int a = 0; a < 2; ++a) {
+          if (npairs > a) {
+            uint32_t r[16];
+            tmem_ld_16cols(lane_base + a * kSkN + c * 16, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(r[j]);
+          }
+        }
+        if (g.transpose) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(c * 16 + j) * C::RedStrideT + row] = v[j];
+        } else {
+          float4* dst = reinterpret_cast<float4*>(red + row * C::RedStride + c * 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+    } else if (lane == 0) {
+      fail();
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (hilo) {
+    // the lo operand's rows (64 .. 127) onto the hi operand's (0 .. 63), in
+    // this CTA: the cluster then sums one 64-rank tile per CTA
+    float* red = reinterpret_cast<float*>(smem);
+    const bool tr = g.transpose != 0;
+    for (int e = static_cast<int>(threadIdx.x); e < 64 * (kSkN / 4); e += blockDim.x) {
+      // 4096 float4 groups either way: [col][rank] 256 columns x 16 groups of
+      // four hi ranks; [rank][col] 64 hi ranks x 64 groups of four columns
+      float* h = tr ? red + (e / 16) * C::RedStrideT + 4 * (e % 16)
+                    : red + (e / (kSkN / 4)) * C::RedStride + 4 * (e % (kSkN / 4));
+      const float* l = h + (tr ? 64 : 64 * C::RedStride);
+      float4 x = *reinterpret_cast<float4*>(h);
+      const float4 y = *reinterpret_cast<const float4*>(l);
+      x.x += y.x;
+      x.y += y.y;
+      x.z += y.z;
+      x.w += y.w;
+      *reinterpret_cast<float4*>(h) = x;
+    }
+  }
+
   // ---------------------------------------------------------------- split-K reduction
   // The cluster's tiles are summed in rank order over a flat range of float4
   // groups (this CTA owns one slice), scaled by 1/s and written as bf16 (or
-  // hi/lo pairs).
+  // hi/lo pairs).  Each thread issues the peer loads of both its groups
+  // before it sums either.
   __syncthreads();
   cluster_sync_all();
   {
@@ -385,53 +419,53 @@ __global__ void __launch_bounds__(C::Threads, 1)
 #pragma unroll
     for (int sidx = 0; sidx < kMaxSplits; ++sidx) peer[sidx] = dsmem_addr(red, sidx < S ? sidx : 0);
     const float alpha = g.scale ? static_cast<float>(1.0 / static_cast<double>(*g.scale)) : 1.0f;
-    // offset of the lo half: 64 ranks further on
-    const uint32_t lo_off = static_cast<uint32_t>((tr ? 64 : 64 * C::RedStride) * 4);
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(g.out);
     __nv_bfloat16* out_lo = static_cast<__nv_bfloat16*>(g.out_lo);
-    for (int e = e_begin + static_cast<int>(threadIdx.x); e < e_end; e += blockDim.x) {
-      const int major = e / ng, lg = e % ng;  // tr: (col, rank group); else (rank, col group)
-      const int64_t gcol = n0 + (tr ? major : 4 * lg);
-      if (gcol >= g.cols) continue;  // row-major outputs: ldo covers the whole group
-      const uint32_t off = static_cast<uint32_t>(
-          (tr ? major * C::RedStrideT + 4 * lg : major * C::RedStride + 4 * lg) * 4);
-      float4 part[kMaxSplits], part_lo[kMaxSplits];
+    for (int e0 = e_begin + static_cast<int>(threadIdx.x); e0 < e_end; e0 += 2 * blockDim.x) {
+      float4 part[2][kMaxSplits];
+      int64_t gcol[2];
+      bool live[2];
 #pragma unroll
-      for (int sidx = 0; sidx < kMaxSplits; ++sidx) {
-        if (sidx < S) {
-          part[sidx] = dsmem_load_f32x4(peer[sidx] + off);
-          if (hilo) part_lo[sidx] = dsmem_load_f32x4(peer[sidx] + off + lo_off);
-        }
+      for (int u = 0; u < 2; ++u) {
+        const int e = e0 + u * static_cast<int>(blockDim.x);
+        const int major = e / ng, lg = e % ng;  // tr: (col, rank group); else (rank, col group)
+        gcol[u] = n0 + (tr ? major : 4 * lg);
+        live[u] = e < e_end && gcol[u] < g.cols;  // row-major outputs: ldo covers the whole group
+        const uint32_t off = static_cast<uint32_t>(
+            (tr ? major * C::RedStrideT + 4 * lg : major * C::RedStride + 4 * lg) * 4);
+#pragma unroll
+        for (int sidx = 0; sidx < kMaxSplits; ++sidx)
+          if (live[u] && sidx < S) part[u][sidx] = dsmem_load_f32x4(peer[sidx] + off);
       }
-      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-      for (int sidx = 0; sidx < kMaxSplits; ++sidx) {  // fixed order: rank 0, 1, ...
-        if (sidx < S) {
-          acc.x += part[sidx].x;
-          acc.y += part[sidx].y;
-          acc.z += part[sidx].z;
-          acc.w += part[sidx].w;
-          if (hilo) {
-            acc.x += part_lo[sidx].x;
-            acc.y += part_lo[sidx].y;
-            acc.z += part_lo[sidx].z;
-            acc.w += part_lo[sidx].w;
+      for (int u = 0; u < 2; ++u) {
+        if (!live[u]) continue;
+        const int e = e0 + u * static_cast<int>(blockDim.x);
+        const int major = e / ng, lg = e % ng;
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int sidx = 0; sidx < kMaxSplits; ++sidx) {  // fixed order: rank 0, 1, ...
+          if (sidx < S) {
+            acc.x += part[u][sidx].x;
+            acc.y += part[u][sidx].y;
+            acc.z += part[u][sidx].z;
+            acc.w += part[u][sidx].w;
           }
         }
-      }
-      const float vals[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
-      __nv_bfloat16 hi[4], lo[4];
+        const float vals[4] = {acc.x * alpha, acc.y * alpha, acc.z * alpha, acc.w * alpha};
+        __nv_bfloat16 hi[4], lo[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        hi[k] = __float2bfloat16_rn(vals[k]);
-        lo[k] = __float2bfloat16_rn(vals[k] - __bfloat162float(hi[k]));
+        for (int k = 0; k < 4; ++k) {
+          hi[k] = __float2bfloat16_rn(vals[k]);
+          lo[k] = __float2bfloat16_rn(vals[k] - __bfloat162float(hi[k]));
+        }
+        const int64_t o = tr ? gcol[u] * g.ldo + i0 + 4 * lg : static_cast<int64_t>(i0 + major) * g.ldo + gcol[u];
+        uint2 ph, pl;
+        memcpy(&ph, hi, 8);
+        memcpy(&pl, lo, 8);
+        *reinterpret_cast<uint2*>(out + o) = ph;
+        if (out_lo) *reinterpret_cast<uint2*>(out_lo + o) = pl;
       }
-      const int64_t o = tr ? gcol * g.ldo + i0 + 4 * lg : static_cast<int64_t>(i0 + major) * g.ldo + gcol;
-      uint2 ph, pl;
-      memcpy(&ph, hi, 8);
-      memcpy(&pl, lo, 8);
-      *reinterpret_cast<uint2*>(out + o) = ph;
-      if (out_lo) *reinterpret_cast<uint2*>(out_lo + o) = pl;
     }
   }
   cluster_sync_all();  // no CTA leaves while a peer still reads its tile
