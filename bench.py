@@ -165,7 +165,7 @@ class LayerState:
         self.dA = t.empty((r, self.K), dtype=t.bfloat16, device=dev)
         self.dB = t.empty((self.N, r), dtype=t.bfloat16, device=dev)
         self.dB_inc = t.empty((self.N, r), dtype=t.bfloat16, device=dev)
-        self.mask = t.empty(self.N, dtype=t.uint8, device=dev)
+        self.mask = t.zeros(self.N, dtype=t.uint8, device=dev)  # no selection before the first step
         self.n_sel = t.zeros(1, dtype=t.int32, device=dev)
 
         def ws(op, M, N, K, rr):
@@ -186,7 +186,7 @@ class Step:
     LAUNCHES = {"quantX": 1, "fwd": 1, "quantdY": 1, "adapters": 2, "dX": 1, "sgd": 0, "proxy": 2}
 
     def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None, tensor_from=256,
-                 grouped=True):
+                 grouped=True, defer_clear=True):
         self.torch, self.F, self.dev = torch, F, dev
         self.grouped = grouped
         t = torch
@@ -197,6 +197,10 @@ class Step:
         # the proxy's accumulation: the strict float32 chain, or the tensor cores from rank tensor_from up
         self.proxy_tensor = tensor_from > 0 and self.r >= tensor_from
         self.proxy_flags = F.PROXY_ACCUMULATE | F.PROXY_SELECT | (F.PROXY_TENSOR if self.proxy_tensor else 0)
+        # the clear of the selected rows carried to the next step through row_mask (not with TENSOR)
+        self.defer_clear = bool(defer_clear) and not self.proxy_tensor
+        if self.defer_clear:
+            self.proxy_flags |= F.PROXY_DEFER_CLEAR
         maxdim = max(max(l.N, l.K) for l in wl.layers)
         # one quantize workspace for every call of the step, initialised once
         self.ws_q = F.workspace(F.OP_QUANTIZE, self.M, maxdim, device=dev)
@@ -408,7 +412,7 @@ def run_gpu(args):
                                        sum(l.N for l in wl.layers))
     slots = args.slots or min(8, max(2, -(-(2 * L2_BYTES) // slot_bytes)))
     st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack,
-              tensor_from=args.proxy_tensor_from, grouped=bool(args.grouped))
+              tensor_from=args.proxy_tensor_from, grouped=bool(args.grouped), defer_clear=bool(args.proxy_defer))
     stream = torch.cuda.Stream(device=dev)
     if args.only:
         # one phase alone, eagerly, warm-up + steps times (for profiler captures)
@@ -566,6 +570,8 @@ def run_gpu(args):
                    "cuda_graph": not args.no_graph, "lr": wl.lr,
                    "proxy_accumulation": ("tensor cores (bf16 products, float32 sums)" if st.proxy_tensor
                                           else "strict float32 FMA chain"),
+                   "proxy_clear": ("deferred: row_mask carries it to the next step" if st.defer_clear
+                                   else "written every step"),
                    "grouped_forward": st.grouped},
         "step_ms_median": round(float(np.median(per_step)), 5),
         "roofline": roof,
@@ -995,6 +1001,9 @@ def main():
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--grouped", type=int, default=1,
                     help="forward GEMMs of layers that read one activation in one grouped launch (1) or not (0)")
+    ap.add_argument("--proxy-defer", type=int, default=1,
+                    help="carry the proxy clear of selected rows to the next step through row_mask (1) or "
+                         "write it every step (0)")
     ap.add_argument("--proxy-tensor-from", type=int, default=256,
                     help="rank from which the proxy accumulates on the tensor cores (0: never)")
     ap.add_argument("--separate", type=int, default=1,

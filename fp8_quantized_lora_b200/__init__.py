@@ -25,7 +25,7 @@ __all__ = [
     "SEPARATE_BF16", "SEPARATE_FP8", "OP_QUANTIZE",
     "OP_LINEAR_FWD",
     "OP_LINEAR_BWD", "OP_PROXY_UPDATE", "OP_PROXY_UPDATE_TOPK", "OP_FOLDED_T", "OP_LINEAR_BWD_FOLDED",
-    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "PROXY_TENSOR", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
+    "PROXY_ACCUMULATE", "PROXY_SELECT", "PROXY_KEEP_RESIDUAL", "PROXY_STRICT", "PROXY_TENSOR", "PROXY_DEFER_CLEAR", "DEV_NONFINITE", "DEV_SCALE_OVERFLOW", "DEV_TIMEOUT",
     "LIB_PATH", "EXPORTED_SYMBOLS",
 ]
 
@@ -38,6 +38,7 @@ OP_SEPARATE_BWD_BF16, OP_SEPARATE_BWD_FP8 = 10, 11
 SEPARATE_BF16, SEPARATE_FP8 = 0, 1
 DTYPE_BF16, DTYPE_F32 = 0, 1
 PROXY_ACCUMULATE, PROXY_SELECT, PROXY_KEEP_RESIDUAL, PROXY_STRICT, PROXY_TENSOR = 1, 2, 4, 8, 16
+PROXY_DEFER_CLEAR = 32  # with ACCUMULATE | SELECT: row_mask carries the clear to the next call
 DEV_NONFINITE, DEV_SCALE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED", 3: "WORKSPACE", 4: "CUDA"}
 
@@ -261,10 +262,14 @@ def falqon_linear_bwd(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=True, dB=Tr
 def falqon_proxy_update(wq, s_w, proxy, dB_inc, A, flags=PROXY_ACCUMULATE | PROXY_SELECT,
                         row_mask=None, n_selected=None, dev_status=None, workspace=None,
                         stream=None):
-    """Row-wise proxy update in place on (wq, proxy); returns (row_mask, n_selected)."""
+    """Row-wise proxy update in place on (wq, proxy); returns (row_mask, n_selected).
+    With PROXY_DEFER_CLEAR, row_mask is the caller's: zeros before the first
+    call, then the previous call's output (rows it marks read as +0)."""
     N, K = proxy.shape
     r = A.shape[0] if A is not None else 0
     dev = proxy.device
+    if flags & PROXY_DEFER_CLEAR and row_mask is None:
+        raise ValueError("PROXY_DEFER_CLEAR reads the previous selection: pass row_mask")
     if flags & PROXY_SELECT:
         row_mask = torch.empty(N, dtype=torch.uint8, device=dev) if row_mask is None else row_mask
         n_selected = torch.empty(1, dtype=torch.int32, device=dev) if n_selected is None else n_selected

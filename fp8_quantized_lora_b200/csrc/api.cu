@@ -285,8 +285,13 @@ falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   int32_t* n_selected, int32_t* dev_status, void* workspace,
                                   size_t workspace_bytes, void* stream) {
   const uint32_t known = FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT | FALQON_PROXY_KEEP_RESIDUAL |
-                         FALQON_PROXY_STRICT | FALQON_PROXY_TENSOR;
+                         FALQON_PROXY_STRICT | FALQON_PROXY_TENSOR | FALQON_PROXY_DEFER_CLEAR;
   if ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) == 0 || (flags & ~known)) return FALQON_ERR_INVALID_ARG;
+  // a deferred clear needs a call that rewrites every row's proxy (ACCUMULATE) and the mask (SELECT)
+  if ((flags & FALQON_PROXY_DEFER_CLEAR) &&
+      ((flags & (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT)) != (FALQON_PROXY_ACCUMULATE | FALQON_PROXY_SELECT) ||
+       (flags & (FALQON_PROXY_KEEP_RESIDUAL | FALQON_PROXY_TENSOR)) || !row_mask))
+    return FALQON_ERR_INVALID_ARG;
   if ((flags & FALQON_PROXY_KEEP_RESIDUAL) && !(flags & FALQON_PROXY_SELECT)) return FALQON_ERR_INVALID_ARG;
   if ((flags & FALQON_PROXY_TENSOR) &&
       (!(flags & FALQON_PROXY_ACCUMULATE) || (flags & FALQON_PROXY_STRICT)))

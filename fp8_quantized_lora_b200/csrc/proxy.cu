@@ -31,6 +31,8 @@
 //     selects the row -- and the row's flag is set.
 //   proxy_clear_kernel  (one warp per row)
 //     Selected rows get P = +0; writes the row mask and the selected count.
+//     With a deferred clear it writes only the mask and the count, and the
+//     next call's accumulation reads the masked rows' P as +0.
 //
 // Every step is reproduced bit-for-bit by the float32 arithmetic.
 #include <cuda_fp16.h>
@@ -81,7 +83,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         float* __restrict__ proxy, const uint16_t* __restrict__ dB_inc,
                         const uint16_t* __restrict__ A, int64_t N, int64_t K, int r,
                         uint8_t* __restrict__ rowflag, int32_t* __restrict__ n_selected,
-                        int32_t* __restrict__ dev_status, int keep_residual) {
+                        int32_t* __restrict__ dev_status, int keep_residual,
+                        const uint8_t* __restrict__ zero_rows) {
   pdl_trigger();  // the next kernel may start launching; it waits for this one
   pdl_wait();     // the previous kernel's results are complete and visible
   extern __shared__ __align__(128) uint8_t sm[];
@@ -104,8 +107,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int j = 0; j < kRT; ++j) {
     const int64_t n = r0 + tr * kRT + j;
     const bool ok = col_ok && n < N;
+    const bool pz = ok && zero_rows && zero_rows[n];  // a deferred clear: P reads as +0
     cp_async16(pbuf + j * kThreads + tid, ok ? static_cast<const void*>(proxy + n * K + col) : proxy,
-               ok ? 16u : 0u);
+               ok && !pz ? 16u : 0u);
     if (kSel != kModeNone)
       cp_async4(wbuf + j * kThreads + tid, ok ? static_cast<const void*>(wq + n * K + col) : wq,
                 ok ? 4u : 0u);
@@ -234,7 +238,8 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     proxy_ws_kernel(uint8_t* __restrict__ wq, const float* __restrict__ s_w_ptr, float* __restrict__ proxy,
                     const uint16_t* __restrict__ dB_inc, const uint16_t* __restrict__ A, int64_t N, int64_t K,
                     int r, int row_groups, int units, int ncb, uint8_t* __restrict__ rowflag,
-                    int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status, int keep_residual) {
+                    int32_t* __restrict__ n_selected, int32_t* __restrict__ dev_status, int keep_residual,
+                    const uint8_t* __restrict__ zero_rows) {
   // No early trigger: the clear kernel that follows would only sit on the SMs.
   pdl_wait();
   extern __shared__ __align__(128) uint8_t sm[];
@@ -363,11 +368,12 @@ __global__ void __launch_bounds__(kWsThreads, 2)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t n = r0 + 8 * ew + j;
+      const bool pz = zero_rows && n < N && zero_rows[n];  // a deferred clear: P reads as +0
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int64_t col = cbase + 128 * h;
         const bool ok = n < N && col < K;  // K % 16 == 0: four columns in or out together
-        p[j][h] = ok ? *reinterpret_cast<const float4*>(proxy + n * K + col) : make_float4(0.f, 0.f, 0.f, 0.f);
+        p[j][h] = ok && !pz ? *reinterpret_cast<const float4*>(proxy + n * K + col) : make_float4(0.f, 0.f, 0.f, 0.f);
         w[j][h] = (ok && kSel != kModeNone) ? *reinterpret_cast<const uint32_t*>(wq + n * K + col) : 0u;
       }
     }
@@ -477,7 +483,8 @@ __global__ void __launch_bounds__(kClearThreads)
 template <bool kAcc, int kSel>
 cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                           const void* A, int64_t N, int64_t K, int r, uint8_t* rowflag,
-                          int32_t* n_selected, int32_t* dev_status, int keep_residual, cudaStream_t stream) {
+                          int32_t* n_selected, int32_t* dev_status, int keep_residual, const uint8_t* zero_rows,
+                          cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -490,14 +497,14 @@ cudaError_t launch_stream(dim3 grid, uint8_t* wq, const float* s_w, float* proxy
   }
   return launch_pdl(proxy_stream_kernel<kAcc, kSel>, grid, dim3(kThreads), kSmemBytes, stream, 1u, wq, s_w,
                     proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
-                    rowflag, n_selected, dev_status, keep_residual);
+                    rowflag, n_selected, dev_status, keep_residual, zero_rows);
 }
 
 template <int kSel>
 cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, const void* dB_inc,
                         const void* A, int64_t N, int64_t K, int r, int row_groups, int units,
                         int ncb, uint8_t* rowflag, int32_t* n_selected, int32_t* dev_status,
-                        int keep_residual, cudaStream_t stream) {
+                        int keep_residual, const uint8_t* zero_rows, cudaStream_t stream) {
   static int configured_mask = 0;  // one bit per device ordinal < 31
   int dev = 0;
   cudaGetDevice(&dev);
@@ -510,7 +517,7 @@ cudaError_t launch_pipe(int grid, uint8_t* wq, const float* s_w, float* proxy, c
   }
   return launch_pdl(proxy_ws_kernel<kSel>, dim3(grid), dim3(kWsThreads), kWsSmemBytes, stream, 1u, wq,
                     s_w, proxy, static_cast<const uint16_t*>(dB_inc), static_cast<const uint16_t*>(A), N, K, r,
-                    row_groups, units, ncb, rowflag, n_selected, dev_status, keep_residual);
+                    row_groups, units, ncb, rowflag, n_selected, dev_status, keep_residual, zero_rows);
 }
 
 }  // namespace
@@ -529,6 +536,8 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
   bool acc = flags & 1u;
   const bool sel = flags & 2u;
   const int keep_res = (flags & 4u) ? 1 : 0;  // residual-keeping clear instead of P = +0
+  const bool defer = flags & 32u;              // the clear is carried to the next call through row_mask
+  const uint8_t* zero_rows = defer ? row_mask : nullptr;
   if (r > (int64_t(1) << 30)) return cudaErrorInvalidValue;
   if (acc && (flags & 16u)) {
     // tensor-core accumulation: P = fl32(P + dB_inc . A), float32 accumulation
@@ -558,25 +567,25 @@ cudaError_t launch_proxy_update(uint8_t* wq, const float* s_w, float* proxy, con
     const int rg = static_cast<int>(row_groups), un = static_cast<int>(units);
     if (sel)
       e = launch_pipe<kModeSelect>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                                   dev_status, keep_res, stream);
+                                   dev_status, keep_res, zero_rows, stream);
     else
       e = launch_pipe<kModeNone>(g, wq, s_w, proxy, dB_inc, A, N, K, rr, rg, un, ncb, rowflag, n_selected,
-                                 dev_status, keep_res, stream);
+                                 dev_status, keep_res, zero_rows, stream);
   } else if (acc && sel)
     e = launch_stream<true, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                         dev_status, keep_res, stream);
+                                         dev_status, keep_res, zero_rows, stream);
   else if (acc)
     e = launch_stream<true, kModeNone>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                       dev_status, keep_res, stream);
+                                       dev_status, keep_res, zero_rows, stream);
   else
     e = launch_stream<false, kModeSelect>(grid, wq, s_w, proxy, dB_inc, A, N, K, rr, rowflag, n_selected,
-                                          dev_status, keep_res, stream);
+                                          dev_status, keep_res, zero_rows, stream);
   if (e != cudaSuccess || !sel) return e;
   const int64_t row_blocks = (N + kClearWarps - 1) / kClearWarps;
   const int64_t blocks = row_blocks < static_cast<int64_t>(di->sm_count) * 8 ? row_blocks
                                                                               : static_cast<int64_t>(di->sm_count) * 8;
   return launch_pdl(proxy_clear_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kClearThreads), 0, stream, 1u,
-                    proxy, N, K, ncb, rowflag, row_mask, n_selected, keep_res ? 0 : 1);
+                    proxy, N, K, ncb, rowflag, row_mask, n_selected, keep_res || defer ? 0 : 1);
 }
 
 }  // namespace falqon

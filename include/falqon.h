@@ -105,6 +105,8 @@ typedef enum falqon_separate_precision {
 #define FALQON_PROXY_STRICT 8u        /* the strict float32 FMA chain in index order (the default) */
 #define FALQON_PROXY_TENSOR 16u       /* with ACCUMULATE: the accumulation on the tensor cores (see
                                          falqon_proxy_update); not with STRICT */
+#define FALQON_PROXY_DEFER_CLEAR 32u  /* with ACCUMULATE | SELECT: selected rows' proxy cleared by the next call
+                                         (row_mask carried between calls; see falqon_proxy_update) */
 
 /*
  * falqon_quantize - per-tensor E4M3 quantization.
@@ -310,16 +312,33 @@ FALQON_API falqon_status falqon_linear_bwd_folded(const uint8_t* dyq, const floa
  *               of its own (with both flags, or in a later call), and it
  *               is that pass that reports a non-finite P.
  *               Requirements: r a multiple of 8.
+ *   DEFER_CLEAR: (with ACCUMULATE and SELECT; not with KEEP_RESIDUAL or
+ *               TENSOR) the same
+ *               update with the clear of the selected rows carried to the
+ *               next call instead of written into P: row_mask is read on
+ *               entry, and rows n with row_mask[n] != 0 (the previous call's
+ *               selection) read P[n,:] as +0; P' is written for every row,
+ *               and row_mask (then n_selected) receives this call's
+ *               selection on exit.  The proxy the caller holds is P with the
+ *               rows marked in row_mask read as +0: it equals, bit for bit,
+ *               the P the eager clear leaves, and a chain of DEFER_CLEAR
+ *               calls updates Wq exactly as the eager calls do.  The pass
+ *               that zeroes the selected rows (about all of P when most rows
+ *               change) and the reads of those rows' proxy disappear.
+ *               row_mask is required; before the first call it holds zeros
+ *               (or the selection of a previous eager call, whose clear
+ *               already happened: zeros are then also correct).
  * The default float32 chain is reproduced bit-for-bit.
  *
  *  wq [N, K] E4M3, in/out;  s_w 1 float (the backbone's fixed scale);
  *  proxy [N, K] float32, in/out;  dB_inc [N, r] bfloat16 (the increment of
  *  B this step: the caller folds in sign and learning rate);  A [r, K] bf16.
  *  row_mask [N] uint8 (0/1) and n_selected (1 int32): written when SELECT is
- *  set; nullable.
+ *  set; nullable (row_mask is required, and also read, with DEFER_CLEAR).
  *  Requirements: N >= 1; K multiple of 16; r >= 1 (r unused without
  *  ACCUMULATE); flags: ACCUMULATE and/or SELECT, plus KEEP_RESIDUAL only
- *  with SELECT, TENSOR only with ACCUMULATE.
+ *  with SELECT, TENSOR only with ACCUMULATE, DEFER_CLEAR only with both
+ *  ACCUMULATE and SELECT and neither KEEP_RESIDUAL nor TENSOR.
  */
 FALQON_API falqon_status falqon_proxy_update(uint8_t* wq, const float* s_w, float* proxy,
                                   const void* dB_inc, const void* A, int64_t N, int64_t K,

@@ -102,7 +102,23 @@ def test_proxy_argument_errors():
         assert L.falqon_proxy_update(P, P, P, P, P, 4, 20, 2, flags, None, None, None, P, 1 << 20, None) == 2
     # ... but not alone, and unknown bits are still rejected
     assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 8, None, None, None, P, 1 << 20, None) == 1
-    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3 | 32, None, None, None, P, 1 << 20, None) == 1
+    assert L.falqon_proxy_update(P, P, P, P, P, 4, 16, 2, 3 | 64, None, None, None, P, 1 << 20, None) == 1
+
+
+def test_proxy_defer_clear_argument_errors():
+    """DEFER_CLEAR (32) goes with ACCUMULATE and SELECT both, never with
+    KEEP_RESIDUAL or TENSOR, and needs the row mask it reads and writes; a
+    valid combination gets as far as the shape check (K % 16 -> UNSUPPORTED)."""
+    L = F.lib()
+    D = 32
+    f = L.falqon_proxy_update
+    assert f(P, P, P, P, P, 4, 20, 2, 3 | D, P, None, None, P, 1 << 20, None) == 2
+    assert f(P, P, P, P, P, 4, 20, 2, 3 | 8 | D, P, None, None, P, 1 << 20, None) == 2  # with STRICT
+    assert f(P, P, P, P, P, 4, 16, 2, 3 | D, None, None, None, P, 1 << 20, None) == 1   # no row mask
+    assert f(P, P, P, P, P, 4, 16, 2, 2 | D, P, None, None, P, 1 << 20, None) == 1      # SELECT alone
+    assert f(P, P, P, P, P, 4, 16, 2, 1 | D, P, None, None, P, 1 << 20, None) == 1      # ACCUMULATE alone
+    assert f(P, P, P, P, P, 4, 16, 2, 7 | D, P, None, None, P, 1 << 20, None) == 1      # KEEP_RESIDUAL
+    assert f(P, P, P, P, P, 4, 16, 2, 3 | 16 | D, P, None, None, P, 1 << 20, None) == 1  # TENSOR
 
 
 def test_proxy_topk_argument_errors():

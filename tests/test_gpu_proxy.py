@@ -159,3 +159,41 @@ def test_keep_residual_trajectory_matches(cuda_device):
         np.testing.assert_array_equal(host(p).view(np.uint32), P.view(np.uint32))
         np.testing.assert_array_equal(host(mask), rmask)
         assert int(host(cnt)[0]) == rcnt
+
+
+@pytest.mark.parametrize("N,K,r,steps,inc", [
+    (192, 384, 16, 12, 3e-4),    # persistent kernel, nearly every row selected every step
+    (192, 384, 16, 12, 3e-5),    # about a third selected: rows leave the mask at most steps
+    (37, 48, 5, 8, 3e-3),        # grid kernel (r % 8 != 0), ragged
+    (96, 1024, 100, 6, 1e-3),    # grid kernel, r above one staging chunk
+    (130, 512, 64, 10, 3e-6),    # about a tenth selected
+])
+def test_deferred_clear_trajectory_matches(cuda_device, N, K, r, steps, inc):
+    """DEFER_CLEAR carries the clear of the selected rows to the next call
+    through row_mask.  Every step: codes, row mask and count bit-identical to
+    the oracle's eager update, and the proxy the caller holds (P with the
+    rows marked in row_mask read as +0) bit-identical to the oracle's P."""
+    O.set_threads(os.cpu_count() or 8)
+    wq, s_w, P, _, A = _state(N + K + r + 31, N, K, r, p_std=0)
+    w, p = dev_u8(wq), dev_f32(P)
+    s_dev, A_dev = dev_f32([s_w]), dev_bf16(A)
+    mask = torch.zeros(N, dtype=torch.uint8, device="cuda:0")  # no earlier selection
+    st = status_word()
+    flags = F.PROXY_ACCUMULATE | F.PROXY_SELECT | F.PROXY_DEFER_CLEAR
+    seen = 0
+    for step in range(steps):
+        dB = gen.normal_bf16_bits(5000 + 17 * N + step, (N, r), inc)
+        _, cnt = F.falqon_proxy_update(w, s_dev, p, dev_bf16(dB), A_dev, flags=flags, row_mask=mask,
+                                       dev_status=st)
+        wq, P, rmask, rcnt = O.proxy_update(wq, s_w, P, dB, A)
+        torch.cuda.synchronize()
+        hm = host(mask)
+        held = host(p).copy()
+        held[hm != 0] = 0.0  # the deferred clear: +0
+        np.testing.assert_array_equal(host(w), wq)
+        np.testing.assert_array_equal(hm, rmask)
+        assert int(host(cnt)[0]) == rcnt
+        np.testing.assert_array_equal(held.view(np.uint32), P.view(np.uint32))
+        seen += rcnt
+    assert int(host(st)[0]) == 0
+    assert seen > 0
