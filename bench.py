@@ -186,8 +186,10 @@ class Step:
     LAUNCHES = {"quantX": 1, "fwd": 1, "quantdY": 1, "adapters": 2, "dX": 1, "sgd": 0, "proxy": 2}
 
     def __init__(self, wl, torch, F, dev, n_slots=4, seed_offset=0, r=None, n_stack=None, tensor_from=256,
-                 grouped=True, defer_clear=True):
+                 grouped=True, defer_clear=True, overlap_sgd=True):
         self.torch, self.F, self.dev = torch, F, dev
+        self.overlap_sgd = bool(overlap_sgd)
+        self.side = torch.cuda.Stream(device=dev) if self.overlap_sgd else None
         self.grouped = grouped
         t = torch
         self.wl = wl
@@ -297,10 +299,31 @@ class Step:
         return out
 
     def run(self, slot, phase=None, outs=None):
-        """Enqueues the whole step (or only the calls of one phase) on the current stream."""
+        """Enqueues the whole step (or only the calls of one phase) on the current stream.
+        In a whole step the caller's SGD on B, which dX does not read, runs on a
+        second stream beside dX (forked after the adapter products, joined
+        before the proxy update that reads its increment) when overlap_sgd is set."""
+        t = self.torch
+        main = t.cuda.current_stream()
+        pending = None
         for _, p, f in self.calls(slot, outs):
-            if phase is None or p == phase:
-                f()
+            if phase is not None and p != phase:
+                continue
+            if phase is None and p == "sgd" and self.overlap_sgd:
+                fork = t.cuda.Event()
+                fork.record(main)
+                self.side.wait_event(fork)
+                with t.cuda.stream(self.side):
+                    f()
+                pending = t.cuda.Event()
+                pending.record(self.side)
+                continue
+            if p == "proxy" and pending is not None:
+                main.wait_event(pending)
+                pending = None
+            f()
+        if pending is not None:
+            main.wait_event(pending)
 
 
 # FP32 FMA peak of the CUDA cores (the proxy's bound at large r): 148 SMs x 128
@@ -412,7 +435,8 @@ def run_gpu(args):
                                        sum(l.N for l in wl.layers))
     slots = args.slots or min(8, max(2, -(-(2 * L2_BYTES) // slot_bytes)))
     st = Step(wl, torch, F, dev, n_slots=slots, seed_offset=rank * 1000, r=r, n_stack=n_stack,
-              tensor_from=args.proxy_tensor_from, grouped=bool(args.grouped), defer_clear=bool(args.proxy_defer))
+              tensor_from=args.proxy_tensor_from, grouped=bool(args.grouped), defer_clear=bool(args.proxy_defer),
+              overlap_sgd=bool(args.overlap_sgd))
     stream = torch.cuda.Stream(device=dev)
     if args.only:
         # one phase alone, eagerly, warm-up + steps times (for profiler captures)
@@ -572,6 +596,7 @@ def run_gpu(args):
                                           else "strict float32 FMA chain"),
                    "proxy_clear": ("deferred: row_mask carries it to the next step" if st.defer_clear
                                    else "written every step"),
+                   "sgd": "second stream beside dX" if st.overlap_sgd else "in line",
                    "grouped_forward": st.grouped},
         "step_ms_median": round(float(np.median(per_step)), 5),
         "roofline": roof,
@@ -1001,6 +1026,8 @@ def main():
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--grouped", type=int, default=1,
                     help="forward GEMMs of layers that read one activation in one grouped launch (1) or not (0)")
+    ap.add_argument("--overlap-sgd", type=int, default=1,
+                    help="run the caller's SGD on B on a second stream beside dX (1) or in line (0)")
     ap.add_argument("--proxy-defer", type=int, default=1,
                     help="carry the proxy clear of selected rows to the next step through row_mask (1) or "
                          "write it every step (0)")
