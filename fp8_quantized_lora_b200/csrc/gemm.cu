@@ -514,7 +514,6 @@ cudaError_t launch_gemm(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
 // 1.73 waves, no accumulator double buffer) and two CTAs per SM.
 using FwdCfg = Cfg<false, 256, 4, 2, 1, 1>;
 using DxCfg = Cfg<true, 256, 4, 2, 1, 1>;
-using DxE5Cfg = Cfg<true, 256, 4, 2, 1, 1, 1>;  // dYq in E5M2
 
 // The adapter segment, when present: B2 (A~q [N2, Kc] K-major, or B~q
 // [Kc, N2] MN-major) with scale sb2, written transposed to the hi/lo planes
@@ -648,21 +647,6 @@ cudaError_t launch_fp8_gemm_dx(const uint8_t* dyq, const float* s_dy, const uint
                                const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
                                int32_t* dev_status, cudaStream_t stream, bool dy_e5m2) {
   return launch_fp8_gemm_dx_pair(dyq, s_dy, wq, s_w, M, N, K, dx, dev_status, stream, dy_e5m2);
-}
-
-// The one-SM kernel for the same products (kept for comparison runs).
-cudaError_t launch_fp8_gemm_fwd_single(const uint8_t* xq, const float* s_x, const uint8_t* wq,
-                                       const float* s_w, int64_t M, int64_t N, int64_t K, void* y,
-                                       int32_t* dev_status, cudaStream_t stream) {
-  return fp8_gemm<FwdCfg>(xq, s_x, wq, s_w, M, N, K, y, dev_status, stream);
-}
-
-cudaError_t launch_fp8_gemm_dx_single(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
-                                      const float* s_w, int64_t M, int64_t N, int64_t K, void* dx,
-                                      int32_t* dev_status, cudaStream_t stream, bool dy_e5m2) {
-  // contraction over N: A = dYq [M, N] K-major; B = Wq [N, K] read MN-major (K contiguous)
-  if (dy_e5m2) return fp8_gemm<DxE5Cfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
-  return fp8_gemm<DxCfg>(dyq, s_dy, wq, s_w, M, K, N, dx, dev_status, stream);
 }
 
 cudaError_t launch_fp8_gemm_fwd_folded(const uint8_t* xq, const float* s_x, const uint8_t* wq,
