@@ -330,8 +330,9 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   auto stage = [&](int v, bool with_a) {
     const int64_t r0 = static_cast<int64_t>(v % row_groups) * kWsRows;
     float* B = Bs + ((v - u_begin) & 1) * (kWsRMax * kWsRows);
+    // lane = row: each store instruction of a warp writes 32 consecutive words
     for (int e = et; e < kWsRows * chunks_per_row; e += 128) {
-      const int row = e / chunks_per_row, c8 = e % chunks_per_row;
+      const int row = e % kWsRows, c8 = e / kWsRows;
       const int64_t n = r0 + row;
       uint4 q = make_uint4(0u, 0u, 0u, 0u);
       if (n < N) q = *reinterpret_cast<const uint4*>(dB_inc + n * r + 8 * c8);
@@ -398,10 +399,10 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     }
     // 4. P' = P + D, requantize, write P' and the changed codes, the tile's row verdicts
     //    (D is read row by row; the math warps need its buffer only after their next tile)
+    uint32_t changed = 0;  // bit j: a code of row 8ew + j changed in this lane's columns
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t n = r0 + 8 * ew + j;  // uniform across the warp
-      bool changed = false;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int64_t col = cbase + 128 * h;
@@ -423,18 +424,19 @@ __global__ void __launch_bounds__(kWsThreads, 2)
             const uint32_t m = cn == wv ? nan_bytes(wv) : changed_bytes(wv, cn);
             if (m) {
               *reinterpret_cast<uint32_t*>(wq + n * K + col) = (cn & m) | (wv & ~m);
-              changed = true;
+              changed |= 1u << j;
               if (keep_residual) out = residual4(q, wv, cn, m, s_w);
             }
           }
           *reinterpret_cast<float4*>(proxy + n * K + col) = out;
         }
       }
-      if constexpr (kSel == kModeSelect) {
-        // the tile's verdict for row n, written whether or not a code changed
-        const bool any = __any_sync(0xFFFFFFFFu, changed);
-        if (lane == 0 && n < N) rowflag[n * ncb + cb] = any ? 1 : 0;
-      }
+    }
+    if constexpr (kSel == kModeSelect) {
+      // the tile's verdicts for its rows 8ew .. 8ew+7, written whether or not a code changed
+      const uint32_t any = __reduce_or_sync(0xFFFFFFFFu, changed);
+      if (lane < 8 && r0 + 8 * ew + lane < N)
+        rowflag[(r0 + 8 * ew + lane) * ncb + cb] = static_cast<uint8_t>((any >> lane) & 1u);
     }
     mbar_arrive(empty_d);
   }
