@@ -63,7 +63,7 @@ struct GemmArgs {
   int64_t ld2;
   const float* scale_b2;   // alpha2 = 1 / (scale_a * scale_b2)
   const void* addend;      // bf16 [M][ldo] added to the rounded product (nullable)
-  int32_t f32_accumulate;  // out is float32 [M][ldo]: out = fl32(out + alpha * product), no bf16 rounding
+  int32_t f32_accumulate;  // out is float32 [M][ldo]: 1: out = fl32(out + alpha * product); 2: out = alpha * product
   // grouped launch (kMode 2): up to three B segments sharing A, each with its
   // own scale and row-major bf16 output; segment s owns the tiles from
   // seg_tile0[s] on (seg_tile0[nseg] = n_tiles)
@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
         tmem_ld_wait();
         if constexpr (C::EpiStageBytes > 0) {
           if (g.f32_accumulate) {
-            // float32 output accumulated in place, out = fl32(out + alpha * D).
+            // float32 output accumulated in place, out = fl32(out + alpha * D)
+            // (or written, out = fl32(alpha * D), in mode 2).
             // Lane l holds row l of the warp's 32 rows; the 32 x 32 chunk goes
             // through shared memory so that every access below covers four
             // rows of 128 contiguous bytes.
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(C::Threads, C::MinBlocks)
               const int64_t grow = row0 + rr;
               if (grow < g.M && col < g.N) {  // Ncols % 4 == 0: four columns in or out together
                 float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + grow * g.ldo + col);
-                float4 p = *dst;
+                float4 p = g.f32_accumulate == 2 ? make_float4(0.f, 0.f, 0.f, 0.f) : *dst;
                 const float* src = stg + rr * 33 + 4 * (lane & 7);
                 p.x = __fadd_rn(p.x, src[0]);
                 p.y = __fadd_rn(p.y, src[1]);
@@ -546,7 +547,7 @@ template <class C>
 cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* sb,
                     int64_t M, int64_t Ncols, int64_t Kc, void* out, int32_t* dev_status,
                     cudaStream_t stream, const Segment2& s2 = Segment2{}, const void* addend = nullptr,
-                    int64_t lda = 0, bool f32_accumulate = false) {
+                    int64_t lda = 0, int f32_accumulate = 0) {
   CUtensorMap tA, tB, tB2, tBh;
   // A [M, Kc] K-major, rows lda elements apart (0: Kc)
   if (!make_tmap_2d(&tA, tmap_dtype<C>(), C::ElemBytes, a, Kc, M, C::BK, kBM, true, static_cast<uint64_t>(lda)))
@@ -578,7 +579,7 @@ cudaError_t tc_gemm(const void* a, const float* sa, const void* b, const float* 
   g.ld2 = s2.ld;
   g.scale_b2 = s2.sb;
   g.addend = addend;
-  g.f32_accumulate = f32_accumulate ? 1 : 0;
+  g.f32_accumulate = f32_accumulate;
   g.dev_status = dev_status;
   if (g.n_tiles == 0) return cudaSuccess;
   if (g.n_tiles0 < g.n_tiles) return launch_gemm<C, 1>(tA, tB, tB2, tBh, g, stream);
@@ -690,8 +691,13 @@ cudaError_t launch_fp8_gemm_fwd_grouped(const uint8_t* xq, const float* s_x, int
 
 cudaError_t launch_gemm_nn_f32acc(const void* a, const void* b, int64_t M, int64_t Ncols, int64_t Kc, float* out,
                                   int32_t* dev_status, cudaStream_t stream) {
-  return tc_gemm<BfDxCfg>(a, nullptr, b, nullptr, M, Ncols, Kc, out, dev_status, stream, Segment2{}, nullptr, 0,
-                          true);
+  return tc_gemm<BfDxCfg>(a, nullptr, b, nullptr, M, Ncols, Kc, out, dev_status, stream, Segment2{}, nullptr, 0, 1);
+}
+
+cudaError_t launch_gemm_bf16_f32out(bool b_mn, const void* a, int64_t lda, const void* b, const float* sb, int64_t M,
+                                    int64_t Ncols, int64_t Kc, float* out, int32_t* dev_status, cudaStream_t stream) {
+  return b_mn ? tc_gemm<BfDxCfg>(a, nullptr, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, nullptr, lda, 2)
+              : tc_gemm<BfFwdCfg>(a, nullptr, b, sb, M, Ncols, Kc, out, dev_status, stream, Segment2{}, nullptr, lda, 2);
 }
 
 }  // namespace falqon

@@ -114,6 +114,11 @@ cudaError_t launch_gemm_nn(bool bf16, const void* a, const float* sa, const void
 
 // out[M, Ncols] (float32) = fl32(out + A . B): A [M, Kc] and B [Kc, Ncols]
 // bf16, float32 accumulation on the tensor cores (kind::f16).
+// out [M, Ncols] float32 = fl32(product / *sb) (sb nullable: 1), bf16 operands:
+// A [M, Kc] K-major (rows lda elements apart, 0: Kc); B [Ncols, Kc] K-major or,
+// with b_mn, [Kc, Ncols].
+cudaError_t launch_gemm_bf16_f32out(bool b_mn, const void* a, int64_t lda, const void* b, const float* sb, int64_t M,
+                                    int64_t Ncols, int64_t Kc, float* out, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_gemm_nn_f32acc(const void* a, const void* b, int64_t M, int64_t Ncols, int64_t Kc, float* out,
                                   int32_t* dev_status, cudaStream_t stream);
 
@@ -133,6 +138,14 @@ cudaError_t launch_adapter_stage2(const uint8_t* dyq, const float* s_dy, const u
                                   const void* T_hi, const void* T_lo, const void* U_hi, const void* U_lo,
                                   int64_t ld, int64_t M, int64_t N, int64_t K, int64_t r, void* dA, void* dB,
                                   int32_t* dev_status, cudaStream_t stream, bool dy_e5m2 = false);
+// Large ranks (adapter_gemm.cu): the adapter products on the bf16 GEMM, with
+// the codes expanded once; used by launch_adapter_grads when adapter_gemm_path.
+bool adapter_gemm_path(int64_t M, int64_t r);
+size_t adapter_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
+cudaError_t launch_adapter_grads_gemm(const uint8_t* dyq, const float* s_dy, const uint8_t* xq, const float* s_x,
+                                      const void* A, const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                                      void* dA, void* dB, int32_t* dev_status, void* workspace, cudaStream_t stream,
+                                      bool dy_e5m2);
 // Row stride (elements) of a transposed T / U plane: M rounded up to 8.
 inline int64_t adapter_tu_ld(int64_t M) { return (M + 7) / 8 * 8; }
 // Bytes of one [r][ld] bf16 plane, padded to 256.

@@ -577,9 +577,8 @@ int64_t tu_ld(int64_t M) { return adapter_tu_ld(M); }
 // entries by more than one bf16 ulp of the tensor's scale.  The split-K sums
 // never leave the chip (cluster reduction).
 size_t adapter_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r, bool want_da) {
-  (void)N;
-  (void)K;
   (void)want_da;
+  if (adapter_gemm_path(M, r)) return adapter_gemm_workspace_bytes(M, N, K, r);
   const size_t tu = align_up(static_cast<size_t>(tu_ld(M)) * r * 2, 256);
   return 4 * tu;
 }
@@ -590,6 +589,11 @@ cudaError_t launch_adapter_grads(const uint8_t* dyq, const float* s_dy, const ui
                                  int32_t* dev_status, void* workspace, cudaStream_t stream, bool dy_e5m2) {
   const DeviceInfo* di = current_device_info();
   if (!di) return cudaErrorInvalidDevice;
+  // past a few hundred ranks the rank-on-M kernel below would expand every
+  // code r / 128 times: the products run as plain bf16 GEMMs instead
+  if (adapter_gemm_path(M, r))
+    return launch_adapter_grads_gemm(dyq, s_dy, xq, s_x, A, B, M, N, K, r, dA, dB, dev_status, workspace, stream,
+                                     dy_e5m2);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int64_t ld = tu_ld(M);
   const size_t tu = align_up(static_cast<size_t>(ld) * r * 2, 256);

@@ -204,6 +204,13 @@ FALQON_API falqon_status falqon_linear_fwd_grouped(const uint8_t* xq, const floa
  *  A [r, K] bfloat16; B [N, r] bfloat16 (read only when dA != NULL).
  *  dx [M, K], dA [r, K], dB [N, r]: bfloat16 outputs, each nullable.
  *  Requirements: M >= 1; N, K multiples of 16; r >= 16 and a multiple of 16.
+ *  Workspace (dA or dB wanted): falqon_workspace_size(FALQON_OP_LINEAR_BWD,
+ *  M, N, K, r) bytes.  Up to r = 496 (or M not a multiple of 8) T and U are
+ *  kept as bf16 hi/lo planes, 4 * align256(round_up(M, 8) * r * 2) bytes;
+ *  from r = 512 the four products run as bf16 GEMMs on codes expanded once,
+ *  and the workspace also holds the expanded codes and the float32
+ *  intermediates (2M(K+N) + 4rM + 4r round_up(M, 8) + 8r max(N, K) bytes,
+ *  each part padded to 256).
  */
 FALQON_API falqon_status falqon_linear_bwd(const uint8_t* dyq, const float* s_dy, const uint8_t* wq,
                                 const float* s_w, const uint8_t* xq, const float* s_x,
@@ -408,8 +415,9 @@ FALQON_API falqon_status falqon_proxy_update_topk(uint8_t* wq, const float* s_w,
  *
  *  - Limit: the scratch array is 16 MiB per device, held by every GPU that
  *    loads the library until the process exits.  A call asking for dA or dB
- *    needs 4 * align256(round_up(M, 8) * r * 2) bytes of it (the same with or
- *    without dA; falqon_workspace_size(FALQON_OP_LINEAR_BWD, M, N, K, r));
+ *    needs falqon_workspace_size(FALQON_OP_LINEAR_BWD, M, N, K, r) bytes of
+ *    it (the same with or without dA; up to r = 496, 4 * align256(
+ *    round_up(M, 8) * r * 2));
  *    beyond 16 MiB it returns FALQON_ERR_WORKSPACE before launching
  *    anything.  Every other argument error is reported first, exactly as
  *    falqon_linear_bwd reports it.  A dX-only call needs no scratch.

@@ -1,5 +1,6 @@
-"""Adapter gradients dB and dA (tcgen05 kind::f16 with in-smem E4M3 expansion)
-against the oracle, within the float acceptance rule."""
+"""Adapter gradients dB and dA against the oracle, within the float acceptance
+rule: the rank-on-M kernel (tcgen05 kind::f16 with in-smem E4M3 expansion)
+and, from r = 512, the bf16-GEMM path (codes expanded once)."""
 
 import os
 
@@ -52,6 +53,12 @@ CASES = [
     (1000, 4096, 1024, 64), # many dB/dA^T tiles, few splits
     (3, 256, 512, 16),      # fewer tokens than one K block of dB / dA
     (333, 512, 768, 192),   # odd M (padded T/U rows); r over one rank tile
+    # from r = 512 (M a multiple of 8) the products run on the bf16 GEMM: codes
+    # expanded once, T and U in float32, hi + lo planes stacked in dB / dA
+    (520, 512, 768, 512),
+    (1024, 272, 1024, 576),  # N not a multiple of the 256-wide tile
+    (8, 256, 256, 512),      # one token tile
+    (333, 256, 512, 512),    # M not a multiple of 8: the rank-on-M kernel at a large rank
 ]
 
 
@@ -105,10 +112,12 @@ def _every_code(shape, offset):
     return valid[idx].reshape(shape)
 
 
-def test_every_code_expands_exactly(cuda_device):
+@pytest.mark.parametrize("r", [32, 512])
+def test_every_code_expands_exactly(cuda_device, r):
     """Each operand holds every non-NaN code (subnormals, zeros of both signs,
-    +-448), so each code's expansion to bf16 enters both products."""
-    M, N, K, r = 256, 384, 512, 32
+    +-448), so each code's expansion to bf16 enters both products (both
+    paths: the in-tile expansion and, at r = 512, the expansion pass)."""
+    M, N, K = 256, 384, 512
     xq, dyq = _every_code((M, K), 0), _every_code((M, N), 3)
     s_x, s_dy = np.float32(3.0), np.float32(0.5)
     A = gen.normal_bf16_bits(11, (r, K), 0.01)
@@ -120,10 +129,11 @@ def test_every_code_expands_exactly(cuda_device):
     assert O.tolerance_report(da, rda)["ok"]
 
 
-def test_nan_code_propagates(cuda_device):
+@pytest.mark.parametrize("r", [16, 512])
+def test_nan_code_propagates(cuda_device, r):
     """A NaN code in Xq poisons its row of T (hence all of dB) and its column
     of dA, on both sides; everything else still matches."""
-    M, N, K, r = 128, 256, 256, 16
+    M, N, K = 128, 256, 256
     xq, s_x, dyq, s_dy, A, B = _case(13, M, N, K, r)
     xq = xq.copy()
     xq[5, 77] = 0xFF

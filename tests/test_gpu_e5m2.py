@@ -84,6 +84,7 @@ def _case(seed, M, N, K, r):
     (200, 272, 336, 32),     # ragged M, N, K
     (130, 256, 128, 64),
     (512, 256, 384, 80),
+    (264, 256, 384, 512),    # large rank: the adapter products on the bf16 GEMM, E5M2 codes expanded
 ])
 def test_backward_e5m2_matches_oracle(cuda_device, M, N, K, r):
     O.set_threads(os.cpu_count() or 8)
