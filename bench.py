@@ -19,11 +19,13 @@ own reads and for the write-back of what it writes, as in a training loop.
 With N > 1 every rank runs an independent replica on its own batch
 ("replicas only", weak scaling) and the reported time is the max over ranks.
 
-Per-phase times (for attribution only) replay each phase of the step from
-its own graph after an L2 flush; the roofline object reports the slowest
-phase against the measured peaks in MEASURED_PEAKS.json.  `e2e` repeats the
-step with the inputs in pinned host memory (H2D copies of every X and dY and
-D2H copies of every Y and dX inside the timed region).  `cpu_baseline` times
+Per-phase times (for attribution only) run the phases of one step in step
+order after an L2 flush, with timing events recorded between them as event
+nodes of one CUDA graph; the roofline object reports the slowest phase
+against the measured peaks in MEASURED_PEAKS.json.  `e2e` repeats the step
+with the inputs in pinned host memory (H2D copies of every X and dY and a
+D2H read of each layer's selected-row count, or with --e2e-outputs 1 also of
+every Y and dX, inside the timed region).  `cpu_baseline` times
 the CPU oracle on a bounded sample (rank 0, N = 1).
 """
 
@@ -335,13 +337,36 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # workload (the capture command is stored beside the figure).  A figure holds
 # only for the kernel sources it was measured on: when a source's hash
 # differs, the roofline's traffic is null.
-TRAFFIC = {}
+TRAFFIC = {
+    "proxy": {
+        "workload": "llama7b_attn_proj_4096x4096x4096_r64", "r": 64, "defer_clear": True,
+        "bytes": 17920256 + 13066496,
+        "kernels": ("proxy_ws_kernel<1> (proxy_clear_kernel, which writes the row mask and the "
+                    "count, not captured)"),
+        "capture": ("ncu --set full --clock-control none -k regex:proxy_ws -s 2 -c 1 python bench.py "
+                    "--only proxy --steps 3 --warmup 3 --no-cpu-baseline: dram__bytes_read.sum "
+                    "17.92 MB + dram__bytes_write.sum 13.07 MB; with the deferred clear the rows the "
+                    "previous call selected are not read, and most of P' is still in L2 when the "
+                    "launch ends"),
+        "sources": {
+            "fp8_quantized_lora_b200/csrc/proxy.cu":
+                "b19ad80cf15cb91295e26eae64562b56318494f62ed8562a538e944101afdd0a",
+            "fp8_quantized_lora_b200/csrc/ptx.cuh":
+                "ff1913ffafac4e65526e4c62e66cb1811fd632c060b2a9c5595e488983d60665",
+            "fp8_quantized_lora_b200/csrc/codes.cuh":
+                "0daacdb7c252d2163d86f9b6ef6c40a2522e5c60497bc5d5b377385ce0f5b1b0",
+        },
+    },
+}
 
 
-def _traffic(phase):
+def _traffic(phase, st):
+    """The captured DRAM bytes of one call of ``phase``, or None when the
+    capture was of another workload, rank or clear mode, or of other kernel
+    sources."""
     import hashlib
     t = TRAFFIC.get(phase)
-    if not t:
+    if not t or t["workload"] != st.wl.name or t["r"] != st.r or t["defer_clear"] != st.defer_clear:
         return None
     for path, digest in t["sources"].items():
         try:
@@ -463,13 +488,8 @@ def run_gpu(args):
                 st.run(slot)
             graphs.append(g)
         for slot in range(min(2, st.n_slots)):
-            per = []
-            for p in Step.PHASES:
-                gk = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(gk, stream=stream):
-                    st.run(slot, p)
-                per.append(gk)
-            phase_graphs.append(per)
+            phase_graphs.append(_evented_graph(
+                torch, stream, [lambda slot=slot, p=p: st.run(slot, p) for p in Step.PHASES]))
     torch.cuda.synchronize()
 
     def step(i):
@@ -505,22 +525,25 @@ def run_gpu(args):
     total_ms = max_over_ranks(evs[0].elapsed_time(evs[-1]), dev)
     per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
 
-    # per-phase attribution: each phase (of every layer) replayed from its own
-    # graph, L2 flushed before each rep, events between the phases
+    # per-phase attribution: the phases of one step (each of every layer) in
+    # step order, one after another, L2 flushed before each rep; timing events
+    # between the phases (event nodes inside one graph: no launch gap inside
+    # a bracket, and no overlap between phases)
     names = list(Step.PHASES)
     acc = {n: 0.0 for n in names}
     reps = max(5, min(50, args.steps))
     with torch.cuda.stream(stream):
         for i in range(reps):
             l2_flush(i)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
-            ev[0].record()
-            for k, n in enumerate(names):
-                if phase_graphs:
-                    phase_graphs[i % len(phase_graphs)][k].replay()
-                else:
+            if phase_graphs:
+                g, ev = phase_graphs[i % len(phase_graphs)]
+                g.replay()
+            else:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+                ev[0].record()
+                for k, n in enumerate(names):
                     st.run(i % st.n_slots, n)
-                ev[k + 1].record()
+                    ev[k + 1].record()
             torch.cuda.synchronize()
             for j, n in enumerate(names):
                 acc[n] += ev[j].elapsed_time(ev[j + 1])
@@ -573,9 +596,11 @@ def run_gpu(args):
         roof = {"kernel": work[dom]["kernels"], "phase": dom, "bound": "hbm",
                 "achieved": phases[dom]["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": phases[dom]["frac_hbm"], "peak_source": f"{peaks['source']} copy bandwidth"}
-    roof["timing"] = "phase replayed from its own CUDA graph after an L2 flush, events on the launching stream"
-    roof["traffic"] = _traffic(dom) if single else None
+    roof["timing"] = ("phases of one step in order after an L2 flush, timing events between them as "
+                      "event nodes of one CUDA graph on the launching stream")
+    roof["traffic"] = _traffic(dom, st) if single else None
     if roof["traffic"] is not None:
+        roof["traffic_kernels"] = TRAFFIC[dom]["kernels"]
         roof["traffic_capture"] = TRAFFIC[dom]["capture"]
 
     layer0 = st.layers[0]
@@ -711,35 +736,45 @@ def _time_e2e(st, torch, stream, ws, dev, args):
             "pipelining": "copy-in, step and copy-out on three streams, two buffer slots"}
 
 
+def _evented_graph(torch, stream, fns):
+    """One CUDA graph of the enqueueing functions ``fns`` in order, with a
+    timing event recorded before the first and after each of them as event
+    nodes of the graph: a replay brackets every call on the device with no
+    graph-launch gap inside a bracket.  Returns (graph, events)."""
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(fns) + 1)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        evs[0].record()
+        for k, f in enumerate(fns):
+            f()
+            evs[k + 1].record()
+    return g, evs
+
+
 def _graph_phase_times(torch, stream, l2_flush, fns, reps, use_graph=True):
-    """Device time (ms) of each enqueueing function in ``fns``: each is
-    captured in its own CUDA graph and the graphs are replayed back to back
-    with events between them (no host launch gaps inside a phase), L2 flushed
-    before every rep outside the events; 3 untimed reps first."""
+    """Device time (ms) of each enqueueing function in ``fns``: all are
+    captured in one CUDA graph with timing events between them
+    (_evented_graph), and the graph is replayed after an L2 flush (outside
+    the events) per rep; 3 untimed reps first."""
     with torch.cuda.stream(stream):
         for f in fns:  # warm the library (attributes, tensor-map encoder)
             f()
     torch.cuda.synchronize()
-    graphs = []
-    if use_graph:
-        for f in fns:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                f()
-            graphs.append(g)
+    graph = _evented_graph(torch, stream, fns) if use_graph else None
     torch.cuda.synchronize()
     acc = [0.0] * len(fns)
     with torch.cuda.stream(stream):
         for i in range(3 + reps):
             l2_flush(i)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
-            ev[0].record()
-            for k, f in enumerate(fns):
-                if graphs:
-                    graphs[k].replay()
-                else:
+            if graph:
+                g, ev = graph
+                g.replay()
+            else:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)]
+                ev[0].record()
+                for k, f in enumerate(fns):
                     f()
-                ev[k + 1].record()
+                    ev[k + 1].record()
             torch.cuda.synchronize()
             if i >= 3:
                 for k in range(len(fns)):
@@ -771,7 +806,7 @@ def _time_topk(st, F, torch, stream, l2_flush, args, dev):
             "fp32_fma_tflops": round(flops / (ms * 1e-3) / 1e12, 2),
             "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "kernels": "topk_accum_kernel + topk_select_kernel + topk_merge_kernel + topk_clear_kernel",
-            "timing": "CUDA graph replay, events on the launching stream",
+            "timing": "one CUDA graph per rep after an L2 flush, timing events as graph nodes",
             "device_status": int(st.status.item())}
 
 
@@ -796,7 +831,7 @@ def _time_e5m2(st, F, torch, stream, l2_flush, args, dev):
     M, N, K = st.M, st.N, st.K
     out["dX_tflops"] = round(2.0 * M * N * K / (out["dX"] * 1e-3) / 1e12, 1)
     out["unit"] = "ms per call"
-    out["timing"] = "CUDA graph replay per call, events on the launching stream"
+    out["timing"] = "one CUDA graph per rep after an L2 flush, timing events as graph nodes between the calls"
     out["device_status"] = int(st.status.item())
     return out
 
@@ -830,7 +865,7 @@ def _time_folded(st, F, torch, stream, l2_flush, args, dev):
     out = {n: round(t, 5) for n, t in zip(names, ms)}
     out["total"] = round(sum(ms), 5)
     out["unit"] = "ms per call"
-    out["timing"] = "CUDA graph replay per call, events on the launching stream"
+    out["timing"] = "one CUDA graph per rep after an L2 flush, timing events as graph nodes between the calls"
     out["kernels"] = ("amax_partial_kernel + quantize_cast_kernel (B); tc_gemm_kernel with T columns; "
                       "tc_gemm_kernel (dX) with U columns + skinny_kernel (dB^T with dA)")
     out["device_status"] = int(st.status.item())
@@ -845,7 +880,7 @@ def _time_separate(st, F, torch, stream, l2_flush, args, dev):
     gradients and dX phases are the corresponding FALQON work."""
     M, N, K, r = st.M, st.N, st.K, st.r
     X = st.X0
-    out = {"unit": "ms per call", "timing": "CUDA graph replay per call, events on the launching stream"}
+    out = {"unit": "ms per call", "timing": "one CUDA graph per rep after an L2 flush, timing events as graph nodes between the calls"}
     reps = max(5, min(50, args.steps))
     for name, prec in (("bf16", F.SEPARATE_BF16), ("fp8", F.SEPARATE_FP8)):
         sop = F.OP_SEPARATE_SAVED_FP8 if prec == F.SEPARATE_FP8 else F.OP_SEPARATE_SAVED_BF16

@@ -16,8 +16,9 @@
 //     (8 rows x 8 columns per thread) from A's columns and the tile's dB_inc
 //     pairs in shared memory and hand D over in shared memory; four epilogue
 //     warps stage those operands one tile ahead, hold the tile's P and Wq in
-//     registers while D is computed, and run the epilogue below.  The roles
-//     meet on mbarriers with bounded waits.  The arithmetic is the one below.
+//     registers while D is computed, and run the epilogue below (registers
+//     are split 104 / 152 between the roles).  The roles meet on mbarriers
+//     with bounded waits.  The arithmetic is the one below.
 //   proxy_stream_kernel  (grid over 32 x 256 tiles of P; two CTAs per SM;
 //     any r)
 //     Each thread owns 8 rows x 4 columns.  Its P and Wq slices stream in
@@ -232,6 +233,13 @@ constexpr int kWsAsBytes = kWsRMax * kTileCols * 2;           // A columns, bf16
 constexpr int kWsBsBytes = kWsRMax * kWsRows * 4;             // dB_inc values, each   8 KB
 constexpr int kWsDBytes = kWsRows * kTileCols * 4;            // D of one tile        32 KB
 constexpr int kWsSmemBytes = kWsAsBytes + 2 * kWsBsBytes + kWsDBytes + 64;  // 80 KB + 6 mbarriers
+// Registers per thread of the two roles after the split (setmaxnreg): the
+// launch gives 65536 / (2 CTAs x 256 threads) = 128 per thread, and the
+// split must return exactly the CTA's pool, or the increase never completes.
+constexpr int kWsMathRegs = 104, kWsEpiRegs = 152;
+static_assert(128 * kWsMathRegs + 128 * kWsEpiRegs == kWsThreads * (65536 / (2 * kWsThreads)),
+              "the register split must balance the CTA's launch allocation");
+static_assert(kWsMathRegs % 8 == 0 && kWsEpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 
 template <int kSel>
 __global__ void __launch_bounds__(kWsThreads, 2)
@@ -270,8 +278,13 @@ __global__ void __launch_bounds__(kWsThreads, 2)
     if (dev_status) atomicOr(dev_status, kDevTimeout);
   };
 
+  // Register split between the roles: the math warps need about 90 registers
+  // (64 accumulators and the operands of one rank step) and hand the rest to
+  // the epilogue warps, which hold a tile's P and Wq slices (at 128 each,
+  // the epilogue spilled).
   if (warp < 4) {
     // ------------------------------------------------------------ math warps
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kWsMathRegs));
     const int g = lane >> 3, c = lane & 7;
     const int colw = 64 * warp + 8 * c;
     for (int t = 0; t < ntiles; ++t) {
@@ -324,6 +337,7 @@ __global__ void __launch_bounds__(kWsThreads, 2)
   }
 
   // -------------------------------------------------------------- epilogue warps
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kWsEpiRegs));
   const int et = tid - 128;
   const int ew = et >> 5;  // rows 8ew .. 8ew+7 of the tile; lane: columns 4l .. 4l+3 and 128 + 4l .. +3
   const int chunks_per_row = r / 8;

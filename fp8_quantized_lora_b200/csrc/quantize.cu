@@ -293,19 +293,19 @@ __global__ void __launch_bounds__(kThreads)
 // contiguous run of 16 KB chunks of x.  Warp 0 (one lane) streams the chunks
 // into a ring of shared-memory slots with bulk asynchronous copies; sixteen
 // consumer warps read each slot, then release it.  Pass 1 reduces max|x|;
-// every CTA publishes its maximum in a tagged workspace word, the last CTA
-// to arrive reduces them and publishes max|x| in one word that the others
-// wait for (bounded), and pass 2 writes the codes: from the ring in place when the CTA's run fits it (up to 14 chunks:
-// a 4096 x 4096 bf16 tensor on 148 SMs), else streaming the run again (it is
-// still in L2).
+// every CTA folds its maximum into one workspace word with an atomic max and
+// counts itself in; the last CTA to arrive publishes the call's generation,
+// which the others wait for (bounded) before reading the word; pass 2 writes
+// the codes: from the ring in place when the CTA's run fits it (up to 14
+// chunks: a 4096 x 4096 bf16 tensor on 148 SMs), else streaming the run
+// again (it is still in L2).
 constexpr int kChunkBytes = 16384;
 constexpr int kStreamStages = 14;                      // 224 KB in flight per SM
 constexpr int kConsumerWarps = 16;
 constexpr int kStreamThreads = 32 * (1 + kConsumerWarps);
 constexpr int kStreamSmemBytes = kStreamStages * kChunkBytes + 2 * kStreamStages * 8 + 16;
-constexpr int kBarWords = 64;                          // per-CTA words start 256 bytes in (0: generation,
-                                                       // 1: arrivals, 2-3: result)
-constexpr int kExchangeWords = 4096;                   // generation + 64-bit words of at most 2016 CTAs
+constexpr int kExchangeWords = 4096;                   // the exchange's words (0: generation, 1: arrivals,
+                                                       // 2-3: maximum slots); the rest is reserved
 constexpr int kPartialWords = 1024;                    // two-launch path: its per-CTA partial maxima
 constexpr long long kBarrierBudget = 2000000000LL;    // cycles (about 1 s), then give up
 
@@ -433,70 +433,47 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
   // Grid exchange of the per-CTA maxima (the launch is cooperative, so every
   // CTA is resident).  The workspace holds a generation counter g (word 0),
-  // an arrival counter (word 1), one result word (words 2-3) and one 64-bit
-  // word per CTA.  Every CTA read g at its start.  It publishes
-  // (g + 1) << 32 | max in its word, then (release) increments the arrival
-  // counter; the CTA that arrives last (acquire) reads every CTA's word,
-  // reduces them, resets the arrival counter, advances g (every CTA has read
-  // it) and publishes (g + 1) << 32 | amax in the result word, which the
-  // other CTAs poll (relaxed loads of one word, bounded, then one acquire
-  // fence).  The increment is unconditional, so the counter returns to zero
-  // after every call, and words left by earlier calls carry older tags:
-  // nothing is cleared between calls.
+  // an arrival counter (word 1) and two maximum slots (words 2 and 3): call g
+  // uses slot g & 1, which the call before it left at zero.  Every CTA read g
+  // at its start.  It folds its maximum into the slot (atomic max of bit
+  // patterns), then (release) increments the arrival counter; the CTA that
+  // arrives last (acquire: every maximum is in the slot) reads the slot,
+  // resets the counter, zeroes the other slot for the next call and
+  // publishes g + 1 (release).  The others poll word 0 (relaxed loads,
+  // bounded, then one acquire fence) and read the slot.  Calls on a stream
+  // run one after another, so the slot a call zeroes is the one the call
+  // before it read, and nothing else is cleared between calls.
   uint32_t* arrivals = ws + 1;
-  uint64_t* result = reinterpret_cast<uint64_t*>(ws + 2);
-  uint64_t* words = reinterpret_cast<uint64_t*>(ws + kBarWords);
-  const uint64_t tag = static_cast<uint64_t>(gen + 1u) << 32;
+  uint32_t* slot = ws + 2 + (gen & 1u);
+  uint32_t* next_slot = ws + 2 + ((gen + 1u) & 1u);
   __shared__ uint32_t amax_bits;
-  if (warp == 0) {
-    uint32_t last = 0;
-    if (lane == 0) {
-      asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(words + blockIdx.x), "l"(tag | m) : "memory");
-      uint32_t old;
-      asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(arrivals) : "memory");
-      last = old == gridDim.x - 1 ? 1u : 0u;
-    }
-    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+  if (threadIdx.x == 0) {
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(slot), "r"(m) : "memory");
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(arrivals) : "memory");
     uint32_t mx = 0;
-    if (last) {
-      // every CTA's word is published (its increment released it): reduce them
-      constexpr int kPerLane = 8;  // words per lane per batch of loads (256 CTAs)
-      for (int b0 = 0; b0 < static_cast<int>(gridDim.x); b0 += 32 * kPerLane) {
-        uint64_t w[kPerLane];
-#pragma unroll
-        for (int k = 0; k < kPerLane; ++k) {
-          const int i = b0 + lane + 32 * k;
-          w[k] = tag;
-          if (i < static_cast<int>(gridDim.x))
-            asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w[k]) : "l"(words + i));
-        }
-#pragma unroll
-        for (int k = 0; k < kPerLane; ++k) mx = max(mx, static_cast<uint32_t>(w[k]));
-      }
-      mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-      if (lane == 0) {
-        *reinterpret_cast<volatile uint32_t*>(arrivals) = 0u;  // ready for the next call
-        *reinterpret_cast<volatile uint32_t*>(ws) = gen + 1u;    // every CTA has read this generation
-        asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(result), "l"(tag | mx) : "memory");
-      }
+    if (old == gridDim.x - 1) {
+      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(mx) : "l"(slot) : "memory");
+      *reinterpret_cast<volatile uint32_t*>(arrivals) = 0u;   // ready for the next call
+      *reinterpret_cast<volatile uint32_t*>(next_slot) = 0u;  // the next call's slot
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ws), "r"(gen + 1u) : "memory");
     } else {
       const long long t0 = clock64();
-      uint64_t w = 0;
       while (true) {
-        if (lane == 0) asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(result));
-        w = __shfl_sync(0xFFFFFFFFu, w, 0);
-        if ((w & 0xFFFFFFFF00000000ull) == tag) {
-          asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of the result word
+        uint32_t g;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(ws) : "memory");
+        if (g != gen) {
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");  // acquire side of word 0
+          asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(mx) : "l"(slot) : "memory");
           break;
         }
         if (clock64() - t0 > kBarrierBudget) {
-          if (lane == 0 && dev_status) atomicOr(dev_status, kDevTimeout);
+          if (dev_status) atomicOr(dev_status, kDevTimeout);
           break;
         }
       }
-      mx = static_cast<uint32_t>(w);
     }
-    if (lane == 0) amax_bits = mx;
+    amax_bits = mx;
   }
   __syncthreads();
   const float s = scale_from_amax(amax_bits, kFmtMax<kE5>, &s_shared, scale_out, amax_out, dev_status);
@@ -590,9 +567,10 @@ int amax_blocks(int64_t n, int sm_count) {
 
 size_t quantize_workspace_bytes(int64_t n) {
   (void)n;
-  // the generation word and the 64-bit exchange words of the one-launch
-  // path, then the partial maxima of the two-launch path (a region of its
-  // own, so that a small tensor never disturbs the exchange's generation)
+  // the exchange words of the one-launch path (generation, arrivals, two
+  // maximum slots; the rest of the region is reserved), then the partial
+  // maxima of the two-launch path (a region of its own, so that a small
+  // tensor never disturbs the exchange's generation)
   return static_cast<size_t>(kExchangeWords + kPartialWords) * sizeof(uint32_t);
 }
 
@@ -619,7 +597,6 @@ cudaError_t launch_quantize_t(const DeviceInfo* di, const void* x, int64_t n, ui
     const int64_t body = (n * (kBF16 ? 2 : 4)) / 16 * 16;
     int64_t chunks = (body + kChunkBytes - 1) / kChunkBytes;
     int grid = static_cast<int>(chunks < di->sm_count ? (chunks > 0 ? chunks : 1) : di->sm_count);
-    if (grid > (kExchangeWords - kBarWords) / 2) grid = (kExchangeWords - kBarWords) / 2;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kStreamThreads);

@@ -37,8 +37,9 @@
  *    filled with zero bytes by the caller).  Every quantize call leaves it
  *    initialised for the next, whatever the size of the tensor and
  *    whether or not a bounded wait ran out (FALQON_DEV_TIMEOUT): the calls
- *    keep a generation counter in it instead of clearing it, so no clearing
- *    step runs per call.  Other workspaces need no initialisation.
+ *    keep a generation counter in it, and each call zeroes only the word
+ *    the next call folds its maximum into, so no clearing step runs per
+ *    call.  Other workspaces need no initialisation.
  *  - Every function is reentrant; the only global state is a per-device
  *    cache of device attributes and of the driver's tensor-map encoder.
  */

@@ -66,20 +66,30 @@ def test_traffic_is_withheld_when_a_source_changes(tmp_path, monkeypatch):
     sources hash as they did at the capture; every committed figure matches
     the committed sources."""
     import hashlib
+    import types
 
     sys.path.insert(0, ROOT)
     import bench
 
+    def step(t):
+        return types.SimpleNamespace(wl=types.SimpleNamespace(name=t["workload"]), r=t["r"],
+                                     defer_clear=t["defer_clear"])
+
     for phase, t in bench.TRAFFIC.items():  # committed figures are current
-        assert bench._traffic(phase) == t["bytes"], phase
+        assert t["workload"] in bench.WORKLOADS, phase
+        assert bench._traffic(phase, step(t)) == t["bytes"], phase
         assert "ncu" in t["capture"] and "--clock-control none" in t["capture"]
     src = tmp_path / "k.cu"
     src.write_text("kernel")
-    entry = {"bytes": 123, "capture": "ncu --clock-control none ...",
+    entry = {"workload": "w", "r": 64, "defer_clear": True, "bytes": 123, "capture": "ncu --clock-control none ...",
              "sources": {"k.cu": hashlib.sha256(b"kernel").hexdigest()}}
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "TRAFFIC", {"proxy": entry})
-    assert bench._traffic("proxy") == 123
+    assert bench._traffic("proxy", step(entry)) == 123
+    # another workload, rank or clear mode than the capture's: no figure
+    assert bench._traffic("proxy", step(dict(entry, workload="v"))) is None
+    assert bench._traffic("proxy", step(dict(entry, r=16))) is None
+    assert bench._traffic("proxy", step(dict(entry, defer_clear=False))) is None
     src.write_text("changed")
-    assert bench._traffic("proxy") is None
-    assert bench._traffic("fwd") is None  # no capture recorded for it
+    assert bench._traffic("proxy", step(entry)) is None
+    assert bench._traffic("fwd", step(entry)) is None  # no capture recorded for it
