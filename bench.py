@@ -340,17 +340,17 @@ FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 TRAFFIC = {
     "proxy": {
         "workload": "llama7b_attn_proj_4096x4096x4096_r64", "r": 64, "defer_clear": True,
-        "bytes": 17920256 + 13066496,
+        "bytes": 17914624 + 13597440,
         "kernels": ("proxy_ws_kernel<1> (proxy_clear_kernel, which writes the row mask and the "
                     "count, not captured)"),
         "capture": ("ncu --set full --clock-control none -k regex:proxy_ws -s 2 -c 1 python bench.py "
                     "--only proxy --steps 3 --warmup 3 --no-cpu-baseline: dram__bytes_read.sum "
-                    "17.92 MB + dram__bytes_write.sum 13.07 MB; with the deferred clear the rows the "
+                    "17.91 MB + dram__bytes_write.sum 13.60 MB; with the deferred clear the rows the "
                     "previous call selected are not read, and most of P' is still in L2 when the "
                     "launch ends"),
         "sources": {
             "fp8_quantized_lora_b200/csrc/proxy.cu":
-                "b19ad80cf15cb91295e26eae64562b56318494f62ed8562a538e944101afdd0a",
+                "bed6522e23166124fb41f662a8d32b2ea570cb2fe8aa84c89171d835e80f3c98",
             "fp8_quantized_lora_b200/csrc/ptx.cuh":
                 "ff1913ffafac4e65526e4c62e66cb1811fd632c060b2a9c5595e488983d60665",
             "fp8_quantized_lora_b200/csrc/codes.cuh":
