@@ -273,3 +273,58 @@ def test_grouped_forward_argument_errors():
     assert f(P, P, 2, arr(P, P), arr(P, P), n(16, 24), arr(P, P), 64, 32, None, None) == 2     # N % 16
     assert f(P, P, 1, arr(P), arr(P), n(16), arr(P8), 64, 32, None, None) == 2                # unaligned output
     assert f(P, P, 1, arr(P), arr(P), n(16), arr(P), 64, 40, None, None) == 2                 # K % 16
+
+
+C_CALLER = r"""
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+#include "falqon.h"
+
+/* A C99 caller of the library: host-side queries and argument checks only
+   (fake device addresses, rejected before any CUDA call). */
+int main(void) {
+  void* p = (void*)(uintptr_t)(1u << 20);
+  uint8_t* p8 = (uint8_t*)p;
+  float* pf = (float*)p;
+  size_t q = falqon_workspace_size(FALQON_OP_QUANTIZE, 4096, 4096, 0, 0);
+  size_t pu = falqon_workspace_size(FALQON_OP_PROXY_UPDATE, 0, 4096, 4096, 64);
+  printf("version %s\n", falqon_version());
+  printf("ok %s\n", falqon_status_string(FALQON_OK));
+  printf("sizes %d %d\n", q > 0 && q % 256 == 0, pu > 0 && pu % 256 == 0);
+  printf("init %d\n", (int)falqon_workspace_init(NULL, 256, NULL));
+  printf("quantize %d %d %d\n",
+         (int)falqon_quantize(NULL, FALQON_DTYPE_BF16, 4, 16, p8, pf, NULL, NULL, NULL, p, q, NULL),
+         (int)falqon_quantize(p, FALQON_DTYPE_BF16, 4, 24, p8, pf, NULL, NULL, NULL, p, q, NULL),
+         (int)falqon_quantize(p, FALQON_DTYPE_BF16, 4, 16, p8, pf, NULL, NULL, NULL, p, 8, NULL));
+  printf("proxy %d\n", (int)falqon_proxy_update(p8, pf, pf, p, p, 4, 16, 2, 3u | FALQON_PROXY_DEFER_CLEAR,
+                                                NULL, NULL, NULL, p, pu, NULL));
+  return 0;
+}
+"""
+
+
+def test_a_c99_program_builds_links_and_calls_the_library(tmp_path):
+    """The boundary is a C ABI: a plain C99 program compiles against
+    include/falqon.h (warnings are errors), links the shared library and gets
+    the documented statuses for argument errors without a GPU."""
+    import shutil
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    F.lib()  # the library is built
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(F.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                    str(src), "-o", str(exe), "-L", libdir, "-lfalqon", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines()
+    got = dict(line.split(" ", 1) for line in out)
+    assert "sm_100a" in got["version"]
+    assert got["ok"] == "ok"
+    assert got["sizes"] == "1 1"
+    assert got["init"] == "1"                  # no workspace
+    assert got["quantize"] == "1 2 3"          # null x; cols not a multiple of 16; workspace too small
+    assert got["proxy"] == "1"                 # DEFER_CLEAR without the row mask
