@@ -44,7 +44,8 @@ def _finite_table():
 
 def _brute_encode(v: np.ndarray) -> np.ndarray:
     """Nearest finite E4M3 value by exhaustive search, ties to the even code."""
-    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # signalling NaN patterns raise the invalid flag when widened
+        v = np.asarray(v, dtype=np.float32).astype(np.float64)
     tab = _finite_table()
     out = np.zeros(v.shape, dtype=np.uint8)
     nan = np.isnan(v)
