@@ -93,3 +93,30 @@ def test_traffic_is_withheld_when_a_source_changes(tmp_path, monkeypatch):
     src.write_text("changed")
     assert bench._traffic("proxy", step(entry)) is None
     assert bench._traffic("fwd", step(entry)) is None  # no capture recorded for it
+
+
+def test_step_work_counts_each_activation_group_once():
+    """Whole-step work of the MLP workload (gate and up read the same X):
+    quantize X is counted once per activation group, every other phase once
+    per layer, so that a shared input's bytes are not counted twice."""
+    import types
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from synthetic import WORKLOADS
+
+    wl = WORKLOADS["llama7b_mlp_8192tok_r64"]
+    M, r = wl.M, wl.r
+    layers = [types.SimpleNamespace(N=l.N, K=l.K) for l in wl.layers]
+    groups = {}
+    for l in wl.layers:
+        groups.setdefault((0, l.x_group), l.K)
+    st = types.SimpleNamespace(M=M, r=r, layers=layers, groups=groups,
+                               calls_per_step={p: 1 for p in bench.Step.PHASES})
+    w = bench._step_work(st)
+    assert len(groups) == 2 and len(layers) == 3
+    assert w["quantX"]["bytes"] == 3 * M * (4096 + 11008)             # x_mlp once, x_down once
+    assert w["quantdY"]["bytes"] == 3 * M * (11008 + 11008 + 4096)    # every layer's dY
+    assert w["fwd"]["flops"] == w["dX"]["flops"] == 2 * M * 3 * 4096 * 11008
+    assert w["proxy"]["flops"] == 2 * r * 3 * 4096 * 11008
+    assert w["adapters"]["flops"] == 4 * M * r * (3 * (4096 + 11008))
