@@ -327,10 +327,6 @@ def falqon_linear_bwd_noalloc(dyq, s_dy, wq, s_w, xq, s_x, A, B, dx=True, dA=Tru
     return dx_t, dA_t, dB_t
 
 
-def _folded_t_bytes(M, r):
-    return falqon_workspace_size(OP_FOLDED_T, M, 0, 0, r)
-
-
 def falqon_linear_fwd_folded(xq, s_x, wq, s_w, aq, s_a, y=None, t_saved=None, dev_status=None, stream=None):
     """[Y | T] = Xq . [Wq ; A~q]^T in one GEMM (quantized adapter folded into
     the backbone); returns (y, t_saved), t_saved being the uint8 buffer that

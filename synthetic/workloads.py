@@ -47,10 +47,6 @@ class Workload:
     description: str = ""
     ranks: tuple = field(default=())
 
-    @property
-    def tokens_per_step(self) -> int:
-        return self.M
-
 
 _ATTN = (Layer("proj", 4096, 4096, "x"),)
 _MLP = (Layer("gate", 4096, 11008, "x_mlp"), Layer("up", 4096, 11008, "x_mlp"),
