@@ -328,3 +328,20 @@ def test_a_c99_program_builds_links_and_calls_the_library(tmp_path):
     assert got["init"] == "1"                  # no workspace
     assert got["quantize"] == "1 2 3"          # null x; cols not a multiple of 16; workspace too small
     assert got["proxy"] == "1"                 # DEFER_CLEAR without the row mask
+
+
+def test_workspace_sizes_of_every_op_and_the_large_rank_path():
+    """Every op's workspace size is a multiple of 256 bytes; the backward's
+    grows with r, and from r = 512 (M % 8 == 0) it holds the codes of X and
+    dY expanded to bf16 once (2 bytes per code), which the rank-on-M path
+    never stores."""
+    M, N, K = 4096, 4096, 4096
+    for op in range(12):
+        for r in (16, 64, 512):
+            n = F.falqon_workspace_size(op, M, N, K, r)
+            assert n % 256 == 0, (op, r, n)
+    bwd = [F.falqon_workspace_size(F.OP_LINEAR_BWD, M, N, K, r) for r in (16, 64, 256, 512, 1024)]
+    assert bwd == sorted(bwd) and bwd[0] > 0
+    assert bwd[2] < 2 * M * (K + N) <= bwd[3]
+    # M not a multiple of 8 keeps the rank-on-M path (no expanded codes)
+    assert F.falqon_workspace_size(F.OP_LINEAR_BWD, M - 1, N, K, 512) < 2 * (M - 1) * (K + N)
